@@ -1,0 +1,200 @@
+"""fp64 CPU oracle for mesh gradient / block-CSR Hessian assembly.
+
+TEST INFRASTRUCTURE ONLY.  The product library never imports, links or calls
+this package; only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's
+CPU-baseline leg (``bench.py`` ``cpu_baseline`` and ``--impl reference``) use
+it.  It shares no code, header, table or helper with the CUDA path.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, closed forms, COO ->
+sort -> merge -> CSR); this module only builds it with gcc and marshals numpy
+arrays through ctypes.  It follows the page "Locality-Aware Automatic
+Differentiation on the GPU for Mesh-Based Computations", section 方法
+(method): g = sum_j S_j^T g_j, H = sum_j S_j^T H_j S_j, with the CSR pattern
+preallocated from mesh topology (key design 3) plus runtime pair blocks (key
+design 4).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+MASK_SPRING = 1
+MASK_INERTIA = 2
+MASK_SYMDIR = 4
+MASK_PAIR = 8
+
+_CFLAGS = ["-O2", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off", "-fno-fast-math"]
+
+
+def build(out: str = _LIB, mutant: int = 0) -> str:
+    """Compile oracle.c with gcc into ``out`` (a planted mistake when mutant>0)."""
+    cmd = ["gcc", *_CFLAGS, f"-DOR_MUTANT={int(mutant)}", "-o", out, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _needs_build(path: str) -> bool:
+    return (not os.path.exists(path)) or os.path.getmtime(path) < os.path.getmtime(_SRC)
+
+
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_f64p = ctypes.POINTER(ctypes.c_double)
+
+
+def _p32(a):
+    return None if a is None else a.ctypes.data_as(_i32p)
+
+
+def _pf(a):
+    return None if a is None else a.ctypes.data_as(_f64p)
+
+
+class Oracle:
+    """ctypes handle on one build of oracle.c."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        lib.or_spring_local.argtypes = [ctypes.c_int, _f64p, _f64p, ctypes.c_double,
+                                        ctypes.c_double, _f64p, _f64p, _f64p]
+        lib.or_inertia_local.argtypes = [ctypes.c_int, _f64p, _f64p, ctypes.c_double,
+                                         _f64p, _f64p, _f64p]
+        lib.or_symdir_local.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double,
+                                        _f64p, _f64p, _f64p]
+        lib.or_pattern.argtypes = [ctypes.c_int32, ctypes.c_int32, _i32p, ctypes.c_int32,
+                                   _i32p, _i32p, _i32p, ctypes.c_int64, _i64p]
+        lib.or_pattern.restype = ctypes.c_int
+        lib.or_edges.argtypes = [ctypes.c_int32, ctypes.c_int32, _i32p, _i32p,
+                                 ctypes.c_int64, _i64p]
+        lib.or_edges.restype = ctypes.c_int
+        lib.or_eval.argtypes = [ctypes.c_int32, ctypes.c_int, _f64p, ctypes.c_uint,
+                                ctypes.c_int32, _i32p, _f64p, ctypes.c_double,
+                                _f64p, ctypes.c_double,
+                                ctypes.c_int32, _i32p, _f64p, _f64p,
+                                ctypes.c_int32, _i32p, _f64p, ctypes.c_double,
+                                _i32p, _i32p, _f64p, _f64p, _f64p]
+        lib.or_eval.restype = ctypes.c_int
+        lib.or_bsr_mv.argtypes = [ctypes.c_int32, ctypes.c_int, _i32p, _i32p, _f64p,
+                                  _f64p, _f64p]
+        lib.or_bsr_mv.restype = ctypes.c_int
+        self.lib = lib
+
+    # ---- local terms ----------------------------------------------------
+    def spring_local(self, xi, xj, L0, k):
+        xi = np.ascontiguousarray(xi, np.float64)
+        xj = np.ascontiguousarray(xj, np.float64)
+        dof = xi.size
+        E = np.zeros(1)
+        g = np.zeros(2 * dof)
+        H = np.zeros((2 * dof, 2 * dof))
+        self.lib.or_spring_local(dof, _pf(xi), _pf(xj), float(L0), float(k), _pf(E),
+                                 _pf(g), _pf(H))
+        return E[0], g, H
+
+    def inertia_local(self, xi, xt, w):
+        xi = np.ascontiguousarray(xi, np.float64)
+        xt = np.ascontiguousarray(xt, np.float64)
+        dof = xi.size
+        E = np.zeros(1)
+        g = np.zeros(dof)
+        H = np.zeros((dof, dof))
+        self.lib.or_inertia_local(dof, _pf(xi), _pf(xt), float(w), _pf(E), _pf(g), _pf(H))
+        return E[0], g, H
+
+    def symdir_local(self, u0, u1, u2, Minv, area):
+        u = [np.ascontiguousarray(a, np.float64) for a in (u0, u1, u2)]
+        M = np.ascontiguousarray(Minv, np.float64).reshape(4)
+        E = np.zeros(1)
+        g = np.zeros(6)
+        H = np.zeros((6, 6))
+        self.lib.or_symdir_local(_pf(u[0]), _pf(u[1]), _pf(u[2]), _pf(M), float(area),
+                                 _pf(E), _pf(g), _pf(H))
+        return E[0], g, H
+
+    # ---- topology ---------------------------------------------------------
+    def pattern(self, V, F, pairs=None):
+        F = np.ascontiguousarray(F, np.int32).reshape(-1, 3)
+        P = None if pairs is None else np.ascontiguousarray(pairs, np.int32).reshape(-1, 2)
+        nP = 0 if P is None else P.shape[0]
+        cap = V + 6 * F.shape[0] + 2 * nP
+        rp = np.zeros(V + 1, np.int32)
+        ci = np.zeros(max(cap, 1), np.int32)
+        need = np.zeros(1, np.int64)
+        r = self.lib.or_pattern(V, F.shape[0], _p32(F), nP, _p32(P), _p32(rp), _p32(ci),
+                                cap, need.ctypes.data_as(_i64p))
+        if r < 0:
+            raise ValueError(f"or_pattern failed: {r}")
+        return rp, ci[:r].copy()
+
+    def edges(self, V, F):
+        F = np.ascontiguousarray(F, np.int32).reshape(-1, 3)
+        cap = 3 * F.shape[0]
+        ij = np.zeros((max(cap, 1), 2), np.int32)
+        need = np.zeros(1, np.int64)
+        r = self.lib.or_edges(V, F.shape[0], _p32(F), _p32(ij), cap,
+                              need.ctypes.data_as(_i64p))
+        if r < 0:
+            raise ValueError(f"or_edges failed: {r}")
+        return ij[:r].copy()
+
+    # ---- assembly -------------------------------------------------------
+    def eval(self, V, dof, x, mask, row_ptr, col_idx, *, edges=None, L0=None, k=0.0,
+             xt=None, w=0.0, F=None, Minv=None, area=None, pairs=None, prest=None,
+             kp=0.0):
+        """Assemble g [V][dof], H_vals [nnzb][dof][dof] and the energy (fp64)."""
+        f64 = lambda a: None if a is None else np.ascontiguousarray(a, np.float64)  # noqa: E731
+        i32 = lambda a: None if a is None else np.ascontiguousarray(a, np.int32)  # noqa: E731
+        x = f64(x).reshape(-1)
+        row_ptr, col_idx = i32(row_ptr), i32(col_idx)
+        edges, F, pairs = i32(edges), i32(F), i32(pairs)
+        L0, xt, Minv, area, prest = f64(L0), f64(xt), f64(Minv), f64(area), f64(prest)
+        nE = 0 if edges is None else edges.reshape(-1, 2).shape[0]
+        nF = 0 if F is None else F.reshape(-1, 3).shape[0]
+        nP = 0 if pairs is None else pairs.reshape(-1, 2).shape[0]
+        nnzb = int(row_ptr[V])
+        g = np.zeros(V * dof)
+        H = np.zeros(nnzb * dof * dof)
+        E = np.zeros(1)
+        r = self.lib.or_eval(V, dof, _pf(x), mask, nE, _p32(edges), _pf(L0), float(k),
+                             _pf(xt), float(w), nF, _p32(F), _pf(Minv), _pf(area),
+                             nP, _p32(pairs), _pf(prest), float(kp),
+                             _p32(row_ptr), _p32(col_idx), _pf(g), _pf(H), _pf(E))
+        if r != 0:
+            raise ValueError(f"or_eval failed: {r}")
+        return g.reshape(V, dof), H.reshape(nnzb, dof, dof), float(E[0])
+
+    def bsr_mv(self, V, dof, row_ptr, col_idx, H_vals, v):
+        row_ptr = np.ascontiguousarray(row_ptr, np.int32)
+        col_idx = np.ascontiguousarray(col_idx, np.int32)
+        H = np.ascontiguousarray(H_vals, np.float64).reshape(-1)
+        v = np.ascontiguousarray(v, np.float64).reshape(-1)
+        y = np.zeros(V * dof)
+        self.lib.or_bsr_mv(V, dof, _p32(row_ptr), _p32(col_idx), _pf(H), _pf(v), _pf(y))
+        return y.reshape(V, dof)
+
+
+_DEFAULT: Oracle | None = None
+
+
+def load() -> Oracle:
+    """The oracle as built from oracle.c (built on first use)."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        if _needs_build(_LIB):
+            build(_LIB)
+        _DEFAULT = Oracle(_LIB)
+    return _DEFAULT
+
+
+def load_mutant(mutant: int) -> Oracle:
+    """A build of oracle.c with planted mistake number ``mutant`` (tests only)."""
+    d = tempfile.mkdtemp(prefix="oracle_mutant_")
+    return Oracle(build(os.path.join(d, f"liboracle_m{mutant}.so"), mutant))

@@ -1,0 +1,495 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU reference for mesh gradient / block-CSR
+ * Hessian assembly.  TEST INFRASTRUCTURE ONLY: nothing in the product library
+ * links, calls or includes this file; only the test suite, the smoke check and
+ * the benchmark's CPU-baseline leg load it.
+ *
+ * What it follows
+ *   Page "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
+ *   Computations" (reading note), section 方法 (method): a scalar objective
+ *   F(x) = sum_j f_j(x_j) over local terms, each with a dense local gradient
+ *   g_j and Hessian H_j, assembled as g = sum_j S_j^T g_j and
+ *   H = sum_j S_j^T H_j S_j (S_j = selection matrix of the term's stencil);
+ *   key design 3: the block sparsity of H is fixed by mesh connectivity and
+ *   is preallocated as CSR; key design 4: runtime vertex-vertex pairs add
+ *   off-diagonal blocks.
+ *
+ * How it computes it (deliberately the plain definition, no blocking, fusion
+ * or reordering):
+ *   1. every term evaluates a hand-derived closed form of E, g_j, H_j;
+ *   2. each (row, col) block of S_j^T H_j S_j is appended to a COO list;
+ *   3. the COO list is sorted by (row, col, emission order) and equal keys
+ *      are summed in that order;
+ *   4. the merged blocks are placed into the CSR pattern; a block whose key
+ *      is absent from the pattern is an error.
+ *   g is accumulated per vertex in term order.
+ *
+ * Readings of points the pages leave open (each also listed in the design
+ * notes): the exact Hessian is assembled (no per-term PSD projection); the CSR
+ * stores both triangles, 0-based int32, columns strictly ascending, diagonal
+ * block always present, blocks contiguous and row-major inside a block;
+ * g and x are [V][dof] interleaved.
+ *
+ * Energies (the page names the applications -- mass-spring cloth,
+ * parameterization -- but prints no formulas; these are the standard forms):
+ *   spring / pair  E = 1/2 k (|xi - xj| - L0)^2
+ *   inertia        E = 1/2 w |xi - xt_i|^2          (w = m / h^2)
+ *   sym. Dirichlet E = A (|J|_F^2 + |J^-1|_F^2),  J = [u1-u0, u2-u0] Dm^-1
+ *
+ * Parity pins: every function here is pinned by tests/test_oracle.py against
+ * closed-form values, finite differences, symmetry, translation / rotation
+ * invariance and a brute-force pattern.  No function is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_OK 0
+#define OR_ERR_ARG -1
+#define OR_ERR_CAPACITY -2
+#define OR_ERR_NOT_IN_PATTERN -3
+#define OR_ERR_OOM -4
+
+/* Optional planted mistakes, compiled in only by the mutation test
+ * (-DOR_MUTANT=n) to show that the pins catch each of them. */
+#ifndef OR_MUTANT
+#define OR_MUTANT 0
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* local terms: closed forms                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Spring between xi and xj in R^dof:  E = 1/2 k (l - L0)^2, l = |xi - xj|.
+ * With n = (xi - xj)/l:
+ *   dE/dxi = k (l - L0) n = -dE/dxj
+ *   K = d2E/dxi2 = k [ n n^T + (1 - L0/l) (I - n n^T) ]
+ *   H (2dof x 2dof, row-major) = [[K, -K], [-K, K]]                        */
+void or_spring_local(int dof, const double* xi, const double* xj, double L0,
+                     double k, double* E, double* g, double* H) {
+  double d[3], l2 = 0.0;
+  for (int a = 0; a < dof; ++a) {
+    d[a] = xi[a] - xj[a];
+    l2 += d[a] * d[a];
+  }
+  double l = sqrt(l2);
+  double n[3];
+  for (int a = 0; a < dof; ++a) n[a] = d[a] / l;
+  double s = l - L0;
+  *E = 0.5 * k * s * s;
+  for (int a = 0; a < dof; ++a) {
+    g[a] = k * s * n[a];
+#if OR_MUTANT == 1 /* planted: wrong sign on the second endpoint */
+    g[dof + a] = k * s * n[a];
+#else
+    g[dof + a] = -k * s * n[a];
+#endif
+  }
+  double t = 1.0 - L0 / l;
+#if OR_MUTANT == 2 /* planted: dropped geometric-stiffness term */
+  t = 0.0;
+#endif
+  int N = 2 * dof;
+  for (int a = 0; a < dof; ++a)
+    for (int b = 0; b < dof; ++b) {
+      double K = k * (n[a] * n[b] + t * ((a == b ? 1.0 : 0.0) - n[a] * n[b]));
+      H[a * N + b] = K;
+      H[(dof + a) * N + (dof + b)] = K;
+      H[a * N + (dof + b)] = -K;
+      H[(dof + a) * N + b] = -K;
+    }
+}
+
+/* Inertia of one vertex: E = 1/2 w |xi - xt|^2, g = w (xi - xt), H = w I. */
+void or_inertia_local(int dof, const double* xi, const double* xt, double w,
+                      double* E, double* g, double* H) {
+  double e = 0.0;
+  for (int a = 0; a < dof; ++a) {
+    double r = xi[a] - xt[a];
+    e += r * r;
+    g[a] = w * r;
+    for (int b = 0; b < dof; ++b) H[a * dof + b] = (a == b) ? w : 0.0;
+  }
+  *E = 0.5 * w * e;
+}
+
+/* Symmetric Dirichlet energy of one triangle in 2D (UV):
+ *   J = [u1-u0, u2-u0] M,  M = Dm^-1 (row-major 2x2), area A
+ *   a = |J|_F^2, d = det J, |J^-1|_F^2 = a / d^2
+ *   E = A (a + a / d^2)
+ *   P = dE/dJ = A [ 2 (1 + d^-2) J - 2 a d^-3 C ],  C = cof J
+ *   with j = vec J = (J00, J01, J10, J11), c = vec C and the constant
+ *   Hessian Dd of det (Dd[0][3] = Dd[3][0] = 1, Dd[1][2] = Dd[2][1] = -1):
+ *   HJ = A [ 2 (1 + d^-2) I4 - 4 d^-3 (j c^T + c j^T) + 6 a d^-4 c c^T
+ *            - 2 a d^-3 Dd ]
+ *   dJ[al][ga]/du_k[be] = delta(al,be) w_k[ga] with w1 = M row 0,
+ *   w2 = M row 1, w0 = -(w1 + w2); so g_k[al] = sum_ga P[al][ga] w_k[ga] and
+ *   H_kl[al][be] = sum_{ga,de} HJ[(al,ga),(be,de)] w_k[ga] w_l[de].
+ * Output g[6] = (u0, u1, u2) interleaved, H 6x6 row-major.                  */
+void or_symdir_local(const double* u0, const double* u1, const double* u2,
+                     const double* M, double A, double* E, double* g,
+                     double* H) {
+  double Ds[2][2] = {{u1[0] - u0[0], u2[0] - u0[0]},
+                     {u1[1] - u0[1], u2[1] - u0[1]}};
+  double J[2][2];
+  for (int al = 0; al < 2; ++al)
+    for (int ga = 0; ga < 2; ++ga)
+      J[al][ga] = Ds[al][0] * M[0 * 2 + ga] + Ds[al][1] * M[1 * 2 + ga];
+  double a = J[0][0] * J[0][0] + J[0][1] * J[0][1] + J[1][0] * J[1][0] +
+             J[1][1] * J[1][1];
+  double d = J[0][0] * J[1][1] - J[0][1] * J[1][0];
+  double C[2][2] = {{J[1][1], -J[1][0]}, {-J[0][1], J[0][0]}};
+  double di = 1.0 / d;
+  *E = A * (a + a * di * di);
+  double P[2][2];
+  for (int al = 0; al < 2; ++al)
+    for (int ga = 0; ga < 2; ++ga)
+      P[al][ga] = A * (2.0 * (1.0 + di * di) * J[al][ga] -
+                       2.0 * a * di * di * di * C[al][ga]);
+  double j[4] = {J[0][0], J[0][1], J[1][0], J[1][1]};
+  double c[4] = {C[0][0], C[0][1], C[1][0], C[1][1]};
+  double Dd[4][4] = {{0, 0, 0, 1}, {0, 0, -1, 0}, {0, -1, 0, 0}, {1, 0, 0, 0}};
+  double HJ[4][4];
+  for (int p = 0; p < 4; ++p)
+    for (int q = 0; q < 4; ++q) {
+      double v = 2.0 * (1.0 + di * di) * (p == q ? 1.0 : 0.0);
+      v -= 4.0 * di * di * di * (j[p] * c[q] + c[p] * j[q]);
+      v += 6.0 * a * di * di * di * di * c[p] * c[q];
+      v -= 2.0 * a * di * di * di * Dd[p][q];
+      HJ[p][q] = A * v;
+    }
+  double w[3][2];
+  w[1][0] = M[0];
+  w[1][1] = M[1];
+  w[2][0] = M[2];
+  w[2][1] = M[3];
+  w[0][0] = -(w[1][0] + w[2][0]);
+  w[0][1] = -(w[1][1] + w[2][1]);
+  for (int kk = 0; kk < 3; ++kk)
+    for (int al = 0; al < 2; ++al)
+      g[2 * kk + al] = P[al][0] * w[kk][0] + P[al][1] * w[kk][1];
+  for (int kk = 0; kk < 3; ++kk)
+    for (int ll = 0; ll < 3; ++ll)
+      for (int al = 0; al < 2; ++al)
+        for (int be = 0; be < 2; ++be) {
+          double s = 0.0;
+          for (int ga = 0; ga < 2; ++ga)
+            for (int de = 0; de < 2; ++de)
+              s += HJ[2 * al + ga][2 * be + de] * w[kk][ga] * w[ll][de];
+#if OR_MUTANT == 3 /* planted: transposed off-diagonal vertex block */
+          if (kk != ll) {
+            s = 0.0;
+            for (int ga = 0; ga < 2; ++ga)
+              for (int de = 0; de < 2; ++de)
+                s += HJ[2 * be + ga][2 * al + de] * w[kk][ga] * w[ll][de];
+          }
+#endif
+          H[(2 * kk + al) * 6 + (2 * ll + be)] = s;
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* COO machinery                                                             */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  int32_t r, c;
+  int64_t seq; /* emission order, makes the sort and the merge order fixed */
+} or_key;
+
+static int or_key_cmp(const void* pa, const void* pb) {
+  const or_key* a = (const or_key*)pa;
+  const or_key* b = (const or_key*)pb;
+  if (a->r != b->r) return a->r < b->r ? -1 : 1;
+  if (a->c != b->c) return a->c < b->c ? -1 : 1;
+  if (a->seq != b->seq) return a->seq < b->seq ? -1 : 1;
+  return 0;
+}
+
+/* Block sparsity pattern from topology (key design 3: fixed by connectivity
+ * and the declared 1-ring neighbourhood; key design 4: plus runtime pairs):
+ * {(i,i)} U {(a,b) : a != b share a face} U {(i,j),(j,i) : (i,j) a pair}.
+ * Built as COO -> sort -> unique.  Returns nnzb, or OR_ERR_CAPACITY with
+ * *needed set when cap is too small.                                        */
+int or_pattern(int32_t V, int32_t nF, const int32_t* F, int32_t nP,
+               const int32_t* P, int32_t* row_ptr, int32_t* col_idx,
+               int64_t cap, int64_t* needed) {
+  if (V < 0 || nF < 0 || nP < 0) return OR_ERR_ARG;
+  int64_t n = (int64_t)V + 6 * (int64_t)nF + 2 * (int64_t)nP;
+  or_key* keys = (or_key*)malloc(sizeof(or_key) * (size_t)(n > 0 ? n : 1));
+  if (!keys) return OR_ERR_OOM;
+  int64_t m = 0;
+  for (int32_t i = 0; i < V; ++i) {
+    keys[m].r = i;
+    keys[m].c = i;
+    keys[m].seq = m;
+    ++m;
+  }
+  for (int32_t f = 0; f < nF; ++f)
+    for (int p = 0; p < 3; ++p)
+      for (int q = 0; q < 3; ++q) {
+        if (p == q) continue;
+        int32_t a = F[3 * f + p], b = F[3 * f + q];
+        if (a < 0 || a >= V || b < 0 || b >= V || a == b) {
+          free(keys);
+          return OR_ERR_ARG;
+        }
+        keys[m].r = a;
+        keys[m].c = b;
+        keys[m].seq = m;
+        ++m;
+      }
+  for (int32_t p = 0; p < nP; ++p) {
+    int32_t i = P[2 * p], j = P[2 * p + 1];
+    if (i < 0 || i >= V || j < 0 || j >= V || i == j) {
+      free(keys);
+      return OR_ERR_ARG;
+    }
+    keys[m].r = i;
+    keys[m].c = j;
+    keys[m].seq = m;
+    ++m;
+    keys[m].r = j;
+    keys[m].c = i;
+    keys[m].seq = m;
+    ++m;
+  }
+  qsort(keys, (size_t)m, sizeof(or_key), or_key_cmp);
+  int64_t u = 0;
+  for (int64_t e = 0; e < m; ++e)
+    if (e == 0 || keys[e].r != keys[e - 1].r || keys[e].c != keys[e - 1].c)
+      ++u;
+  if (needed) *needed = u;
+  if (u > cap) {
+    free(keys);
+    return OR_ERR_CAPACITY;
+  }
+  for (int32_t i = 0; i <= V; ++i) row_ptr[i] = 0;
+  u = 0;
+  for (int64_t e = 0; e < m; ++e)
+    if (e == 0 || keys[e].r != keys[e - 1].r || keys[e].c != keys[e - 1].c) {
+      col_idx[u++] = keys[e].c;
+      row_ptr[keys[e].r + 1] += 1;
+    }
+  for (int32_t i = 0; i < V; ++i) row_ptr[i + 1] += row_ptr[i];
+  free(keys);
+  return (int)u;
+}
+
+/* Unique undirected mesh edges (i < j), sorted by (i, j).  Returns E or an
+ * error; *needed is set like or_pattern.                                    */
+int or_edges(int32_t V, int32_t nF, const int32_t* F, int32_t* ij, int64_t cap,
+             int64_t* needed) {
+  int64_t n = 3 * (int64_t)nF;
+  or_key* keys = (or_key*)malloc(sizeof(or_key) * (size_t)(n > 0 ? n : 1));
+  if (!keys) return OR_ERR_OOM;
+  int64_t m = 0;
+  for (int32_t f = 0; f < nF; ++f)
+    for (int p = 0; p < 3; ++p) {
+      int32_t a = F[3 * f + p], b = F[3 * f + (p + 1) % 3];
+      if (a < 0 || a >= V || b < 0 || b >= V || a == b) {
+        free(keys);
+        return OR_ERR_ARG;
+      }
+      keys[m].r = a < b ? a : b;
+      keys[m].c = a < b ? b : a;
+      keys[m].seq = m;
+      ++m;
+    }
+  qsort(keys, (size_t)m, sizeof(or_key), or_key_cmp);
+  int64_t u = 0;
+  for (int64_t e = 0; e < m; ++e)
+    if (e == 0 || keys[e].r != keys[e - 1].r || keys[e].c != keys[e - 1].c)
+      ++u;
+  if (needed) *needed = u;
+  if (u > cap) {
+    free(keys);
+    return OR_ERR_CAPACITY;
+  }
+  u = 0;
+  for (int64_t e = 0; e < m; ++e)
+    if (e == 0 || keys[e].r != keys[e - 1].r || keys[e].c != keys[e - 1].c) {
+      ij[2 * u] = keys[e].r;
+      ij[2 * u + 1] = keys[e].c;
+      ++u;
+    }
+  free(keys);
+  return (int)u;
+}
+
+/* ------------------------------------------------------------------------ */
+/* assembly                                                                  */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  or_key* keys;
+  double* vals; /* bs doubles per entry */
+  int64_t n, cap;
+  int bs;
+} or_coo;
+
+static int coo_push(or_coo* c, int32_t r, int32_t col, const double* blk) {
+  if (c->n == c->cap) return OR_ERR_OOM;
+  c->keys[c->n].r = r;
+  c->keys[c->n].c = col;
+  c->keys[c->n].seq = c->n;
+  memcpy(c->vals + (size_t)c->n * c->bs, blk, sizeof(double) * c->bs);
+  c->n += 1;
+  return OR_OK;
+}
+
+/* Emit S^T H_j S for a term on `nv` vertices `vid` with local Hessian H of
+ * size (nv*dof)^2 row-major: block (p, q) goes to global (vid[p], vid[q]). */
+static int emit_blocks(or_coo* c, int dof, int nv, const int32_t* vid,
+                       const double* H) {
+  int N = nv * dof;
+  double blk[9];
+  for (int p = 0; p < nv; ++p)
+    for (int q = 0; q < nv; ++q) {
+      for (int a = 0; a < dof; ++a)
+        for (int b = 0; b < dof; ++b)
+          blk[a * dof + b] = H[(p * dof + a) * N + (q * dof + b)];
+      int rc = coo_push(c, vid[p], vid[q], blk);
+      if (rc) return rc;
+    }
+  return OR_OK;
+}
+
+/* Full assembly.  All float inputs are fp64 (the caller widens the stored
+ * run-dtype values).  mask bits: 1 spring, 2 inertia, 4 symmetric Dirichlet,
+ * 8 pairs.  Outputs: g [V][dof] (overwritten), H_vals [nnzb][dof][dof]
+ * (overwritten; blocks absent from every term are zero), *energy.          */
+int or_eval(int32_t V, int dof, const double* x, unsigned mask,
+            /* springs */ int32_t nE, const int32_t* edges, const double* L0,
+            double k,
+            /* inertia */ const double* xt, double w,
+            /* symmetric Dirichlet */ int32_t nF, const int32_t* F,
+            const double* Minv, const double* area,
+            /* pairs */ int32_t nP, const int32_t* pairs, const double* prest,
+            double kp,
+            /* pattern */ const int32_t* row_ptr, const int32_t* col_idx,
+            /* out */ double* g, double* H_vals, double* energy) {
+  if (dof != 2 && dof != 3) return OR_ERR_ARG;
+  if ((mask & 4) && dof != 2) return OR_ERR_ARG;
+  int bs = dof * dof;
+  int64_t n = 0;
+  if (mask & 1) n += 4 * (int64_t)nE;
+  if (mask & 2) n += V;
+  if (mask & 4) n += 9 * (int64_t)nF;
+  if (mask & 8) n += 4 * (int64_t)nP;
+  or_coo c;
+  c.bs = bs;
+  c.cap = n > 0 ? n : 1;
+  c.n = 0;
+  c.keys = (or_key*)malloc(sizeof(or_key) * (size_t)c.cap);
+  c.vals = (double*)malloc(sizeof(double) * (size_t)c.cap * bs);
+  if (!c.keys || !c.vals) {
+    free(c.keys);
+    free(c.vals);
+    return OR_ERR_OOM;
+  }
+  for (int64_t i = 0; i < (int64_t)V * dof; ++i) g[i] = 0.0;
+  double Etot = 0.0, E, gl[6], Hl[36];
+  int rc = OR_OK;
+  if (mask & 1)
+    for (int32_t e = 0; e < nE && !rc; ++e) {
+      int32_t vid[2] = {edges[2 * e], edges[2 * e + 1]};
+      or_spring_local(dof, x + (size_t)vid[0] * dof, x + (size_t)vid[1] * dof,
+                      L0[e], k, &E, gl, Hl);
+      Etot += E;
+      for (int p = 0; p < 2; ++p)
+        for (int a = 0; a < dof; ++a) g[(size_t)vid[p] * dof + a] += gl[p * dof + a];
+      rc = emit_blocks(&c, dof, 2, vid, Hl);
+    }
+  if (mask & 2)
+    for (int32_t i = 0; i < V && !rc; ++i) {
+      or_inertia_local(dof, x + (size_t)i * dof, xt + (size_t)i * dof, w, &E,
+                       gl, Hl);
+      Etot += E;
+      for (int a = 0; a < dof; ++a) g[(size_t)i * dof + a] += gl[a];
+      rc = emit_blocks(&c, dof, 1, &i, Hl);
+    }
+  if (mask & 4)
+    for (int32_t f = 0; f < nF && !rc; ++f) {
+      const int32_t* vid = F + 3 * f;
+      or_symdir_local(x + (size_t)vid[0] * 2, x + (size_t)vid[1] * 2,
+                      x + (size_t)vid[2] * 2, Minv + 4 * (size_t)f, area[f], &E,
+                      gl, Hl);
+      Etot += E;
+      for (int p = 0; p < 3; ++p)
+        for (int a = 0; a < 2; ++a) g[(size_t)vid[p] * 2 + a] += gl[p * 2 + a];
+      rc = emit_blocks(&c, 2, 3, vid, Hl);
+    }
+  if (mask & 8)
+    for (int32_t p = 0; p < nP && !rc; ++p) {
+      int32_t vid[2] = {pairs[2 * p], pairs[2 * p + 1]};
+      or_spring_local(dof, x + (size_t)vid[0] * dof, x + (size_t)vid[1] * dof,
+                      prest[p], kp, &E, gl, Hl);
+      Etot += E;
+      for (int q = 0; q < 2; ++q)
+        for (int a = 0; a < dof; ++a) g[(size_t)vid[q] * dof + a] += gl[q * dof + a];
+      rc = emit_blocks(&c, dof, 2, vid, Hl);
+    }
+  if (rc) {
+    free(c.keys);
+    free(c.vals);
+    return rc;
+  }
+  *energy = Etot;
+  /* sort an index permutation by (r, c, seq), then merge equal keys in order */
+  qsort(c.keys, (size_t)c.n, sizeof(or_key), or_key_cmp);
+  int64_t nnzb = row_ptr[V];
+  for (int64_t i = 0; i < nnzb * bs; ++i) H_vals[i] = 0.0;
+  int64_t e = 0;
+  while (e < c.n) {
+    int32_t r = c.keys[e].r, col = c.keys[e].c;
+    double acc[9] = {0};
+    while (e < c.n && c.keys[e].r == r && c.keys[e].c == col) {
+      const double* v = c.vals + (size_t)c.keys[e].seq * bs;
+      for (int t = 0; t < bs; ++t) acc[t] += v[t];
+      ++e;
+    }
+#if OR_MUTANT == 4 /* planted: merge keeps only the last contribution */
+    {
+      const double* v = c.vals + (size_t)c.keys[e - 1].seq * bs;
+      for (int t = 0; t < bs; ++t) acc[t] = v[t];
+    }
+#endif
+    /* locate (r, col) in the pattern by a linear walk of row r */
+    int64_t pos = -1;
+    for (int64_t q = row_ptr[r]; q < row_ptr[r + 1]; ++q)
+      if (col_idx[q] == col) {
+        pos = q;
+        break;
+      }
+    if (pos < 0) {
+      rc = OR_ERR_NOT_IN_PATTERN;
+      break;
+    }
+    for (int t = 0; t < bs; ++t) H_vals[pos * bs + t] = acc[t];
+  }
+  free(c.keys);
+  free(c.vals);
+  return rc;
+}
+
+/* Matrix-free product reference: y = H v with H the assembled block CSR
+ * (the parameterization workload's Hessian-vector product).               */
+int or_bsr_mv(int32_t V, int dof, const int32_t* row_ptr,
+              const int32_t* col_idx, const double* H_vals, const double* v,
+              double* y) {
+  int bs = dof * dof;
+  for (int32_t i = 0; i < V; ++i) {
+    for (int a = 0; a < dof; ++a) {
+      double s = 0.0;
+      for (int32_t q = row_ptr[i]; q < row_ptr[i + 1]; ++q) {
+        int32_t j = col_idx[q];
+        for (int b = 0; b < dof; ++b)
+          s += H_vals[(size_t)q * bs + a * dof + b] * v[(size_t)j * dof + b];
+      }
+      y[(size_t)i * dof + a] = s;
+    }
+  }
+  return OR_OK;
+}
