@@ -1,0 +1,417 @@
+#!/usr/bin/env python3
+"""Benchmark: gradient + block-CSR Hessian assembly of the 1000x1000 cloth.
+
+One step = one mad_eval (springs + inertia, fp32) on a fresh perturbation of
+the 10^6-vertex cloth: read x and the topology, write g and every Hessian
+block.  Prints ONE JSON line (rank 0).  With torchrun (N > 1) every rank runs
+its own independent replica (weak scaling, no collective on the data path);
+the time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle instead (a bounded sample of the
+same workload per step, scaled to a full step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mesh_inputs as mi  # noqa: E402
+
+N_GRID = 1000
+SEED = 1003
+# compulsory bytes of one step (read x + edge list, write g + Hessian values)
+V_FULL = N_GRID * N_GRID
+E_FULL = 2 * N_GRID * (N_GRID - 1) + (N_GRID - 1) ** 2
+NNZB_FULL = V_FULL + 2 * E_FULL
+ALGO_BYTES = 4 * (3 * V_FULL) + 8 * E_FULL + 4 * (3 * V_FULL) + 36 * NNZB_FULL
+PAGES_MS_1000 = 11.7  # the page's own 1000^2 mass-spring grad+Hessian time (RTX 4090)
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "grad+Hessian assembly ms/step (1000^2 cloth); achieved HBM GB/s vs ~8 TB/s"
+WORKLOAD = ("mass-spring cloth 1000x1000 grid (10^6 vertices, 2,996,001 springs, "
+            "6,992,002 3x3 blocks): springs + inertia, g + block-CSR H per step")
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic():
+    """DRAM bytes per launch of the assembly kernel from the committed ncu
+    summary, or None if the kernel sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    h = hashlib.sha256()
+    for f in d.get("sources", []):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != d.get("sources_sha256"):
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, dev_index=0, period=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {}
+        for attr in dir(nv):
+            if attr.startswith("nvmlClocksEventReason") or attr.startswith("nvmlClocksThrottleReason"):
+                v = getattr(nv, attr)
+                if isinstance(v, int) and v and (v & (v - 1)) == 0:
+                    key = attr.replace("nvmlClocksEventReason", "").replace("nvmlClocksThrottleReason", "")
+                    names.setdefault(v, key)
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h) if hasattr(
+                    nv, "nvmlDeviceGetCurrentClocksEventReasons") else \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for bit, nm in names.items():
+                    if r & bit and nm not in ("GpuIdle", "ApplicationsClocksSetting"):
+                        self.reasons.add(nm)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------- ours
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    import hessian_assembly_b200 as mad
+
+    dev = torch.device("cuda", env_int("LOCAL_RANK", 0))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    st = mi.cloth_static(N_GRID, np.float32)
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    terms = mad.Terms(mask=mad.MAD_TERM_SPRING | mad.MAD_TERM_INERTIA,
+                      spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
+                      inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"])
+    pool = min(args.steps + args.warmup, args.pool)
+    xs = [torch.from_numpy(mi.cloth_x(N_GRID, SEED + 7919 * rank, s, np.float32)).to(dev)
+          for s in range(pool)]
+    g = torch.empty((st["V"], 3), dtype=torch.float32, device=dev)
+    H = torch.empty((ctx.info.capacity_blocks, 3, 3), dtype=torch.float32, device=dev)
+
+    def step(k):
+        ctx.mad_eval(xs[k % pool], terms, g, H, None, stream)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        evs[k][0].record(stream)
+        step(args.warmup + k)
+        evs[k][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    if dist:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    units = world * args.steps
+    value = total_ms / units  # ms per 1000^2 step of the whole job
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        nnzb = ctx.info.nnzb_base
+        hx = [torch.from_numpy(mi.cloth_x(N_GRID, SEED + 7919 * rank, 10_000 + s, np.float32)).pin_memory()
+              for s in range(2)]
+        hg = torch.empty((st["V"], 3), dtype=torch.float32).pin_memory()
+        hH = torch.empty((nnzb, 3, 3), dtype=torch.float32).pin_memory()
+        he = torch.empty(1, dtype=torch.float64).pin_memory()
+        n_e2e = max(3, min(args.steps, 20))
+        for k in range(2):
+            ctx.mad_eval_host(hx[k % 2], terms, hg, hH, he, stream)
+        if dist:
+            dist.barrier()
+        w0 = time.perf_counter()
+        for k in range(n_e2e):
+            ctx.mad_eval_host(hx[k % 2], terms, hg, hH, he, stream)
+        w_ms = (time.perf_counter() - w0) * 1e3
+        if dist:
+            tt = torch.tensor([w_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            w_ms = float(tt.item())
+        e2e = {"value": w_ms / (n_e2e * world), "unit": "ms/step",
+               "h2d_bytes_per_step": int(hx[0].numel() * 4),
+               "d2h_bytes_per_step": int(hg.numel() * 4 + hH.numel() * 4 + 8),
+               "steps": n_e2e, "api": "mad_eval_host"}
+
+    hbm, peak_kind = peaks()
+    avg_launch_ms = statistics.mean(launch_ms)
+    achieved = ALGO_BYTES / (avg_launch_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "traffic": kernel_traffic(),
+            "kernel": "k_eval<float,3,reduced>", "algorithmic_bytes_per_launch": ALGO_BYTES,
+            "avg_launch_ms": round(avg_launch_ms, 5), "peak_kind": peak_kind}
+    out = {
+        "metric": METRIC, "value": round(value, 5), "unit": "ms/step", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": round(value / PAGES_MS_1000, 6), "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n": N_GRID, "seed": SEED, "x_pool": pool,
+                   "l2": "inputs + outputs per step 0.36 GB > 126 MB L2; x from a pool of "
+                         f"{pool} distinct perturbations", "parallelism": f"replicas x{world}",
+                   "patches": ctx.info.n_patches, "smem_bytes": ctx.info.smem_bytes},
+        "roofline": roof, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk,
+        "impl": "ours",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        out["cpu_baseline"] = cpu_baseline(st)
+    if not args.no_extra and rank == 0:
+        out["workloads"] = extra_workloads(args)
+    ctx.close()
+    return out
+
+
+def cpu_baseline(st):
+    import oracle
+    orc = oracle.load()
+    rp, ci = orc.pattern(st["V"], st["F"])
+    times = []
+    for s in range(2):
+        x = mi.cloth_x(N_GRID, SEED, 20_000 + s, np.float32)
+        t0 = time.perf_counter()
+        orc.eval(st["V"], 3, x, 3, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
+                 xt=st["xt"], w=st["w"])
+        times.append((time.perf_counter() - t0) * 1e3)
+    return {"value": round(statistics.median(times), 1), "unit": "ms/step", "cores": 1,
+            "kind": "oracle",
+            "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
+
+
+def extra_workloads(args):
+    """Secondary workloads (parameterization eval/HVP at 500^2, cloth with 10^5
+    runtime pairs at 1000^2, the small grids), CUDA-event timed, median."""
+    import torch
+
+    import hessian_assembly_b200 as mad
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    res = {}
+
+    def timeit(fn, n=50, w=5):
+        for _ in range(w):
+            fn()
+        ts = []
+        for _ in range(n):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median([a.elapsed_time(b) for a, b in ts])
+
+    # small cloths (launch-latency bound)
+    for n in (10, 100):
+        st = mi.cloth_static(n, np.float32)
+        ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+        terms = mad.Terms(mask=3, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
+                          inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"])
+        x = torch.from_numpy(mi.cloth_x(n, 1000 + n, 0, np.float32)).to(dev)
+        g = torch.empty((st["V"], 3), device=dev)
+        H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
+        res[f"cloth{n}_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+        ctx.close()
+    # parameterization 500^2: eval and HVP
+    ps = mi.param_static(500, 1004, np.float32)
+    ctx = mad.Context(ps["V"], ps["F"], 2, "float32", part_xyz=ps["X"])
+    terms = mad.Terms(mask=4, face_Minv=torch.from_numpy(ps["Minv"].reshape(-1, 4)).to(dev),
+                      face_area=torch.from_numpy(ps["area"]).to(dev))
+    x = torch.from_numpy(ps["UV"]).to(dev)
+    v = torch.from_numpy(mi.probe_vector(ps["V"], 2, 1005, np.float32)).to(dev)
+    g = torch.empty((ps["V"], 2), device=dev)
+    y = torch.empty((ps["V"], 2), device=dev)
+    H = torch.empty((ctx.info.capacity_blocks, 2, 2), device=dev)
+    res["symdir500_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+    res["symdir500_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
+    ctx.close()
+    # cloth 1000^2 + 10^5 fresh pairs per step: insertion, assembly
+    st = mi.cloth_static(N_GRID, np.float32)
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    terms = mad.Terms(mask=11, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
+                      inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"],
+                      pair_k=mi.PAIR_K)
+    nst = 8
+    xs, ps_, rs = [], [], []
+    for s in range(nst):
+        xx = mi.cloth_x(N_GRID, 1005, s, np.float32)
+        pp = mi.random_pairs(N_GRID, 100_000, 1005, s)
+        xs.append(torch.from_numpy(xx).to(dev))
+        ps_.append(torch.from_numpy(pp).to(dev))
+        rs.append(torch.from_numpy(mi.pair_rest(xx, pp, np.float32)).to(dev))
+    g = torch.empty((st["V"], 3), device=dev)
+    H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
+    ins, asm = [], []
+    for s in range(3 * nst):
+        k = s % nst
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        ctx.mad_add_pairs(ps_[k], rs[k], stream)
+        b.record(stream)
+        ctx.mad_eval(xs[k], terms, g, H, None, stream)
+        c.record(stream)
+        if s >= nst:
+            ins.append((a, b))
+            asm.append((b, c))
+    torch.cuda.synchronize()
+    res["pairs1000_insert_ms"] = round(statistics.median([a.elapsed_time(b) for a, b in ins]), 5)
+    res["pairs1000_assembly_ms"] = round(statistics.median([a.elapsed_time(b) for a, b in asm]), 5)
+    res["pairs1000_status"] = ctx.mad_status_sync(stream)
+    ctx.close()
+    return res
+
+
+# ---------------------------------------------------------------- reference
+
+
+def run_reference(args):
+    """The oracle on the host cores: each step assembles a bounded sample (the
+    250x250 grid, same energy and noise law) and is scaled to a 1000^2 step by
+    the ratio of term counts."""
+    import oracle
+    orc = oracle.load()
+    ns = args.ref_sample_n
+    st = mi.cloth_static(ns, np.float32)
+    rp, ci = orc.pattern(st["V"], st["F"])
+    terms_s = st["edges"].shape[0] + st["V"]
+    scale = (E_FULL + V_FULL) / terms_s
+    x = mi.cloth_x(ns, SEED, 0, np.float32)
+
+    def step():
+        orc.eval(st["V"], 3, x, 3, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
+                 xt=st["xt"], w=st["w"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    ms = (time.perf_counter() - t0) * 1e3 / args.steps * scale
+    sample = (f"{ns}x{ns} grid per step ({terms_s} terms), scaled by {scale:.3f} to a "
+              "1000x1000 step")
+    return {"metric": METRIC, "value": round(ms, 3), "unit": "ms/step", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": round(ms / PAGES_MS_1000, 4),
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "n": N_GRID, "sample": sample},
+            "cpu_baseline": {"value": round(ms, 3), "unit": "ms/step", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--pool", type=int, default=32)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--ref-sample-n", type=int, default=250)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(env_int("LOCAL_RANK", 0))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    out = run_ours(args, rank, world, dist)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

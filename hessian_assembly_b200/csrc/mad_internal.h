@@ -1,0 +1,162 @@
+// mad_internal.h -- structures shared by the host side of libmad and its
+// kernels.  Nothing here is part of the public C ABI (include/mad.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/mad.h"
+
+namespace mad {
+
+// One patch = a set of OWNED vertices (each vertex is owned by exactly one
+// patch) plus the ribbon: every vertex outside the set that shares a term with
+// it.  A patch evaluates every term touching one of its owned vertices and
+// writes only the rows of its owned vertices, so no two CUDA blocks ever
+// write the same Hessian block or gradient row (page "Locality-Aware
+// Automatic Differentiation on the GPU for Mesh-Based Computations", section
+// 方法, key design 2: one CUDA block per patch, ribbon elements cache the
+// cross-patch neighbours).
+struct PatchHdr {
+  int32_t vbeg, nv, no, nstage;  // local vertices [vbeg, vbeg+nv), owned first;
+                                 // nstage = base blocks of the owned rows
+  int32_t ebeg, ne, ecbeg, nce;  // edge terms; colour c spans
+                                 // ecol[ecbeg+c] .. ecol[ecbeg+c+1] (relative)
+  int32_t fbeg, nf, fcbeg, ncf;  // face terms, same layout
+};
+
+// Block-offset lookup for an edge term (built once per topology): local
+// indices of its two vertices and, for each owned endpoint, the position of
+// the other endpoint's column inside that endpoint's (mesh-pattern) row.
+// kNotOwned marks an endpoint that belongs to another patch.
+struct EdgeLut {
+  uint16_t la, lb, pab, pba;
+};
+
+// Face-term lookup: local vertex indices and pos[k][m] = position of column
+// F[m] in the row of corner k (kNotOwned when corner k is not owned).
+struct FaceLut {
+  uint16_t l[3];
+  uint16_t pos[3][3];
+  int32_t fid;
+};
+
+constexpr uint16_t kNotOwned = 0xFFFF;
+
+// Pair entry position word: low 30 bits = block position inside the row of
+// the current (dynamic) pattern; bit 30 set when this entry created that
+// block (first entry of its column and the column is not in the mesh row).
+constexpr int32_t kPairNewBlock = 1 << 30;
+constexpr int32_t kPairPosMask = (1 << 30) - 1;
+
+// Per-owned-vertex meta word: mesh-pattern row length | diagonal position << 16
+__host__ __device__ inline uint32_t pack_meta(int blen, int dpos) {
+  return (uint32_t)blen | ((uint32_t)dpos << 16);
+}
+
+// Device status bits (sticky; read by mad_status_sync).
+enum : int32_t { kStatusIndex = 1, kStatusCapacity = 2, kStatusTimeout = 4 };
+
+struct HostPatches {
+  std::vector<PatchHdr> hdr;
+  std::vector<int32_t> vgid;
+  std::vector<uint32_t> meta;   // indexed like vgid (owned entries used)
+  std::vector<EdgeLut> elut;
+  std::vector<int32_t> eid;
+  std::vector<int32_t> ecol;
+  std::vector<FaceLut> flut;
+  std::vector<int32_t> fcol;
+  int nv_max = 0, no_max = 0, stage_max = 0;
+};
+
+// Host partitioner (partition.cpp).  rp/ci: mesh pattern (host copies).
+// Returns "" on success, else an error message.
+std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
+                          const int32_t* ci, const double* xyz, int xyz_dim,
+                          int target_owned, int max_stage_blocks,
+                          HostPatches& out);
+
+// ---- dynamic pattern buffers ------------------------------------------
+struct DynBuf {
+  int32_t* rp = nullptr;      // [V+1]
+  int32_t* ci = nullptr;      // [capacity]
+  int32_t* nnzb = nullptr;    // [1]
+  int32_t* prow = nullptr;    // [V+1] pair entries per row (exclusive scan)
+  int32_t* pe_col = nullptr;  // [2*max_pairs] partner vertex, sorted per row
+  int32_t* pe_pos = nullptr;  // [2*max_pairs] position word (see above)
+  void* pe_rest = nullptr;    // [2*max_pairs] rest length (dtype)
+};
+
+// ---- launchers (defined in the .cu files) ------------------------------
+// scan.cu: exclusive scan of n int32 values in -> out[0..n], out[n] = total.
+// tmp must hold scan_tmp_elems(n) ints.
+size_t scan_tmp_elems(int64_t n);
+cudaError_t scan_exclusive(const int32_t* in, int32_t* out, int64_t n,
+                           int32_t* tmp, cudaStream_t s);
+
+// topology.cu
+struct PatternDev {
+  int32_t* rp;      // [V+1]
+  int32_t* ci;      // [nnzb]
+  int32_t* diag;    // [V]
+  int32_t* edges;   // [E][2]
+  int32_t nnzb, E;
+};
+// Builds the mesh pattern and the sorted edge list; allocates the outputs
+// with cudaMalloc.  Returns "" or an error message.
+std::string build_pattern_gpu(int V, int nF, const int32_t* F_dev,
+                              cudaStream_t s, PatternDev& out);
+
+// eval.cu
+struct EvalLaunch {
+  int dtype, dof, n_patches, nv_max, no_max, stage_cap;  // stage_cap in blocks
+  const PatchHdr* hdr;
+  const int32_t* vgid;
+  const uint32_t* meta;
+  const EdgeLut* elut;
+  const int32_t* eid;
+  const int32_t* ecol;
+  const FaceLut* flut;
+  const int32_t* fcol;
+  const int32_t* rp;  // active row_ptr
+  // pairs (active set); prow == nullptr when no pairs are active
+  const int32_t* prow;
+  const int32_t* pe_col;
+  const int32_t* pe_pos;
+  const void* pe_rest;
+  double* epart;  // [n_patches]
+};
+size_t eval_smem_bytes(const EvalLaunch& L, bool hvp);
+cudaError_t launch_eval(const EvalLaunch& L, const mad_terms& t, const void* x,
+                        void* g, void* H, double* energy, cudaStream_t s);
+cudaError_t launch_hvp(const EvalLaunch& L, const mad_terms& t, const void* x,
+                       const void* v, void* y, cudaStream_t s);
+cudaError_t eval_set_smem_limits(int dtype, int dof, size_t bytes);
+
+// pairs.cu
+struct PairLaunch {
+  int V, dtype, capacity, nnzb_base, max_pairs;
+  const int32_t* base_rp;
+  const int32_t* base_ci;
+  int32_t* cnt;     // [V+1]
+  int32_t* cur;     // [V]
+  int32_t* newcnt;  // [V+1]
+  int32_t* shift;   // [V+1]
+  int32_t* pe_pid;  // [2*max_pairs]
+  int32_t* scan_tmp;
+  int32_t* status;  // device status word
+  int32_t* flag;    // [1] overflow flag scratch
+  const int32_t* base_nnzb_dev;  // [1] block count of the mesh pattern
+};
+cudaError_t launch_add_pairs(const PairLaunch& L, int n, const int32_t* ij,
+                             const void* rest, const DynBuf& nb,
+                             const DynBuf* prev /* nullptr = mesh pattern */,
+                             cudaStream_t s);
+
+// selftest.cu
+cudaError_t selftest_dual(int n, const double* ab_dev, double* out_dev);
+
+}  // namespace mad

@@ -1,0 +1,204 @@
+// terms.cuh -- local energy terms, written once and evaluated on HyperDual
+// numbers, and the evaluators that turn one term into its local gradient and
+// Hessian blocks.
+//
+// Page "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
+// Computations", section 方法: the user writes only local energy terms on
+// vertices, edges, faces or runtime pairs; the framework evaluates,
+// differentiates (forward mode, key design 1) and assembles them.  The
+// energies below are those of the page's applications (section 实验结果):
+// mass-spring cloth with inertia, runtime contact-style pairs, and the
+// parameterization energy; the page names them but prints no formulas, so
+// the standard forms are used:
+//   spring / pair   1/2 k (|d| - L0)^2,  d = x_a - x_b
+//   inertia         1/2 w |x - xt|^2
+//   sym. Dirichlet  A (|J|_F^2 + |J^-1|_F^2) = A a (1 + 1/det(J)^2), a = |J|_F^2
+//
+// Two seeding strategies give the same derivatives:
+//  * FULL: tangents on every stencil DOF (width 2*dof for an edge or pair
+//    term, 3*dof for a face term); the energy is evaluated through the
+//    stencil-to-variable map in HyperDual arithmetic;
+//  * reduced (default): tangents on the term's natural variables (the edge
+//    vector d, width dof; the Jacobian J, width 4) and the constant linear
+//    map A from stencil DOFs to those variables is applied afterwards:
+//    g_j = A^T grad, H_j = A^T Hess A.  For an edge term A = [I, -I], so the
+//    four blocks are K, -K, -K, K.
+#pragma once
+
+#include "dual.cuh"
+
+namespace mad {
+
+// ---------------------------------------------------------------- energies
+template <typename S, int D, typename T>
+__device__ __forceinline__ S spring_energy(const S (&d)[D], T L0, T k) {
+  S s = sq(d[0]);
+#pragma unroll
+  for (int a = 1; a < D; ++a) s = s + sq(d[a]);
+  S l = sqrt(s);
+  S r = l - L0;
+  return sq(r) * (T(0.5) * k);
+}
+
+// j = (J00, J01, J10, J11)
+template <typename S, typename T>
+__device__ __forceinline__ S symdir_energy(const S (&j)[4], T A) {
+  S a = sq(j[0]) + sq(j[1]) + sq(j[2]) + sq(j[3]);
+  S det = j[0] * j[3] - j[1] * j[2];
+  S id2 = sq(inv(det));
+  return (a + a * id2) * A;
+}
+
+// ---------------------------------------------------------------- results
+// Edge / pair term: blocks are D x D row-major; the (b, a) block is the
+// transpose of Hab.
+template <typename T, int D>
+struct EdgeDerivs {
+  T E;
+  T ga[D], gb[D];
+  T Haa[D * D], Hab[D * D], Hbb[D * D];
+};
+
+template <typename T, int D, bool FULL>
+__device__ __forceinline__ void eval_edge(const T* xa, const T* xb, T L0, T k,
+                                          EdgeDerivs<T, D>& o) {
+  if constexpr (!FULL) {
+    HyperDual<T, D> d[D];
+#pragma unroll
+    for (int a = 0; a < D; ++a) d[a] = hd_var<T, D>(xa[a] - xb[a], a);
+    HyperDual<T, D> e = spring_energy(d, L0, k);
+    o.E = e.v;
+#pragma unroll
+    for (int a = 0; a < D; ++a) {
+      o.ga[a] = e.g[a];
+      o.gb[a] = -e.g[a];
+    }
+#pragma unroll
+    for (int a = 0; a < D; ++a)
+#pragma unroll
+      for (int b = 0; b < D; ++b) {
+        const T K = hess(e, a, b);
+        o.Haa[a * D + b] = K;
+        o.Hbb[a * D + b] = K;
+        o.Hab[a * D + b] = -K;
+      }
+  } else {
+    constexpr int N = 2 * D;
+    HyperDual<T, N> d[D];
+#pragma unroll
+    for (int a = 0; a < D; ++a)
+      d[a] = hd_var<T, N>(xa[a], a) - hd_var<T, N>(xb[a], D + a);
+    HyperDual<T, N> e = spring_energy(d, L0, k);
+    o.E = e.v;
+#pragma unroll
+    for (int a = 0; a < D; ++a) {
+      o.ga[a] = e.g[a];
+      o.gb[a] = e.g[D + a];
+    }
+#pragma unroll
+    for (int a = 0; a < D; ++a)
+#pragma unroll
+      for (int b = 0; b < D; ++b) {
+        o.Haa[a * D + b] = hess(e, a, b);
+        o.Hab[a * D + b] = hess(e, a, D + b);
+        o.Hbb[a * D + b] = hess(e, D + a, D + b);
+      }
+  }
+}
+
+// Inertia: reduced seeding on r = x - xt (width D)
+template <typename T, int D>
+__device__ __forceinline__ void eval_inertia(const T* x, const T* xt, T w, T& E, T* g,
+                                             T* Hd) {
+  HyperDual<T, D> s = hd_const<T, D>(T(0));
+#pragma unroll
+  for (int a = 0; a < D; ++a) s = s + sq(hd_var<T, D>(x[a] - xt[a], a));
+  HyperDual<T, D> e = s * (T(0.5) * w);
+  E = e.v;
+#pragma unroll
+  for (int a = 0; a < D; ++a) g[a] = e.g[a];
+#pragma unroll
+  for (int a = 0; a < D; ++a)
+#pragma unroll
+    for (int b = 0; b < D; ++b) Hd[a * D + b] = hess(e, a, b);
+}
+
+// Symmetric Dirichlet face term in 2D.  u0, u1, u2 are the corners' UV, M the
+// row-major Dm^-1, A the rest area.  Output g[6] (corner-major) and the 3x3
+// grid of 2x2 blocks H[k][l][4].
+template <typename T>
+struct FaceDerivs {
+  T E;
+  T g[6];
+  T H[3][3][4];
+};
+
+template <typename T, bool FULL>
+__device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u2,
+                                            const T* M, T A, FaceDerivs<T>& o) {
+  // corner weights w_k: dJ[al][ga]/du_k[be] = delta(al, be) w_k[ga]
+  const T w[3][2] = {{-(M[0] + M[2]), -(M[1] + M[3])}, {M[0], M[1]}, {M[2], M[3]}};
+  if constexpr (!FULL) {
+    T Jv[4];
+#pragma unroll
+    for (int al = 0; al < 2; ++al)
+#pragma unroll
+      for (int ga = 0; ga < 2; ++ga)
+        Jv[2 * al + ga] = (u1[al] - u0[al]) * M[ga] + (u2[al] - u0[al]) * M[2 + ga];
+    HyperDual<T, 4> j[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) j[p] = hd_var<T, 4>(Jv[p], p);
+    HyperDual<T, 4> e = symdir_energy(j, A);
+    o.E = e.v;
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int al = 0; al < 2; ++al)
+        o.g[2 * k + al] = e.g[2 * al] * w[k][0] + e.g[2 * al + 1] * w[k][1];
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int l = 0; l < 3; ++l)
+#pragma unroll
+        for (int al = 0; al < 2; ++al)
+#pragma unroll
+          for (int be = 0; be < 2; ++be) {
+            T s = T(0);
+#pragma unroll
+            for (int ga = 0; ga < 2; ++ga)
+#pragma unroll
+              for (int de = 0; de < 2; ++de)
+                s += hess(e, 2 * al + ga, 2 * be + de) * (w[k][ga] * w[l][de]);
+            o.H[k][l][2 * al + be] = s;
+          }
+  } else {
+    HyperDual<T, 6> u[3][2];
+#pragma unroll
+    for (int al = 0; al < 2; ++al) {
+      u[0][al] = hd_var<T, 6>(u0[al], 0 + al);
+      u[1][al] = hd_var<T, 6>(u1[al], 2 + al);
+      u[2][al] = hd_var<T, 6>(u2[al], 4 + al);
+    }
+    HyperDual<T, 6> j[4];
+#pragma unroll
+    for (int al = 0; al < 2; ++al)
+#pragma unroll
+      for (int ga = 0; ga < 2; ++ga)
+        j[2 * al + ga] = (u[1][al] - u[0][al]) * M[ga] + (u[2][al] - u[0][al]) * M[2 + ga];
+    HyperDual<T, 6> e = symdir_energy(j, A);
+    o.E = e.v;
+#pragma unroll
+    for (int q = 0; q < 6; ++q) o.g[q] = e.g[q];
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int l = 0; l < 3; ++l)
+#pragma unroll
+        for (int al = 0; al < 2; ++al)
+#pragma unroll
+          for (int be = 0; be < 2; ++be)
+            o.H[k][l][2 * al + be] = hess(e, 2 * k + al, 2 * l + be);
+  }
+}
+
+}  // namespace mad

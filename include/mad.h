@@ -1,0 +1,243 @@
+/*
+ * mad.h -- C ABI of the B200 mesh-autodiff assembly library (libmad.so).
+ *
+ * The library implements the data-parallel hot path described on the page
+ * "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
+ * Computations" (reading note), section 方法 (method):
+ *   * a scalar objective F(x) = sum_j f_j(x_j) of local terms on a triangle
+ *     mesh, each term depending on a small fixed stencil x_j;
+ *   * per-term forward-mode automatic differentiation giving the dense local
+ *     gradient g_j and Hessian H_j in registers (key design 1);
+ *   * assembly g = sum_j S_j^T g_j and H = sum_j S_j^T H_j S_j into a global
+ *     gradient and a block-CSR Hessian whose pattern is preallocated from
+ *     mesh topology by a parallel count + prefix sum (key design 3), with
+ *     the mesh processed patch by patch, one CUDA block per patch, and
+ *     ribbon (ghost) vertices around each patch (key design 2);
+ *   * runtime vertex-vertex interaction pairs inserted into a double-
+ *     buffered CSR with reserved slack, entirely on the GPU (key design 4);
+ *   * a matrix-free Hessian-vector product (section 实验结果 (results), the
+ *     parameterization application).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers documented "device" are CUDA device pointers in the current
+ *     device's memory; "host" pointers are ordinary CPU memory.
+ *   - Floating-point arrays use the context's dtype (MAD_F32 -> float,
+ *     MAD_F64 -> double); `energy` outputs are always double.
+ *   - Positions, gradients and vectors are [V][dof] interleaved (dof = 2 or 3).
+ *   - The Hessian is block CSR with b x b blocks, b = dof: both triangles
+ *     stored, 0-based int32 row_ptr/col_idx, columns strictly ascending in a
+ *     row, the diagonal block always present, blocks contiguous and row-major
+ *     inside a block: element (r, c) of block q is H_vals[q*b*b + r*b + c].
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call after mad_create is stream-ordered, performs no
+ *     host synchronisation and allocates no memory.
+ *   - Synchronous argument errors are returned at once and nothing is
+ *     launched.  Errors found on the device (a pair index out of range, CSR
+ *     capacity exceeded) are recorded in a sticky device status word and are
+ *     reported by mad_status_sync(); no kernel traps or asserts.
+ *   - A context is used by one host thread at a time.
+ */
+#ifndef MAD_H_
+#define MAD_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mad_ctx mad_ctx; /* opaque, owned by the library */
+
+typedef enum {
+  MAD_OK = 0,
+  MAD_ERR_INVALID_ARG = 1,   /* bad pointer, size, index, dtype or mask      */
+  MAD_ERR_CUDA = 2,          /* a CUDA runtime call failed (see last_error)  */
+  MAD_ERR_OOM = 3,           /* device or host allocation failed (create)    */
+  MAD_ERR_CAPACITY = 4,      /* pairs or CSR blocks exceed reserved capacity */
+  MAD_ERR_INDEX = 5,         /* device-detected index out of range           */
+  MAD_ERR_TIMEOUT = 6,       /* a bounded device wait gave up                */
+  MAD_ERR_UNIMPLEMENTED = 7, /* term / dof / dtype combination not built     */
+  MAD_ERR_STATE = 8          /* call not valid in the context's state        */
+} mad_status;
+
+typedef enum { MAD_F32 = 0, MAD_F64 = 1 } mad_dtype;
+
+/* Local energy terms (bit mask).  Section 方法 states the model (local
+ * terms on vertices, edges, faces and runtime pairs); the concrete energies
+ * are the applications' (section 实验结果): mass-spring cloth and the
+ * parameterization energy.                                                  */
+enum {
+  MAD_TERM_SPRING = 1u,  /* per mesh edge: 1/2 k (|xi - xj| - L0_e)^2         */
+  MAD_TERM_INERTIA = 2u, /* per vertex: 1/2 w |xi - xt_i|^2                   */
+  MAD_TERM_SYMDIR = 4u,  /* per face, dof 2: A_f (|J|_F^2 + |J^-1|_F^2),
+                            J = [u1-u0, u2-u0] Minv_f                         */
+  MAD_TERM_PAIR = 8u     /* per runtime pair: 1/2 k_p (|xi - xj| - r_p)^2     */
+};
+
+/* Evaluation flags. */
+enum {
+  /* Seed forward-mode tangents on every stencil DOF (width 2*dof per edge or
+   * pair term, 3*dof per face term) instead of the default, which seeds the
+   * term's natural variables (the edge vector; the 2x2 Jacobian J) and maps
+   * g_j, H_j back through the term's constant linear input map.  Both give
+   * the same derivatives up to rounding.                                     */
+  MAD_EVAL_FULL_STENCIL_AD = 1u
+};
+
+typedef struct {
+  int32_t patch_faces;   /* target faces per patch; default 512           */
+  float slack;           /* reserved CSR blocks beyond the mesh pattern, as a
+                            fraction of its block count; default 0.10      */
+  int32_t max_pairs;     /* largest pair set mad_add_pairs accepts; default
+                            = reserved blocks / 2, at least 1024           */
+  const double* part_xyz;/* optional host [V][part_dim] positions used only
+                            to shape patches (Morton order); NULL = shape
+                            patches by breadth-first growth on the graph   */
+  int32_t part_dim;      /* 2 or 3 when part_xyz is given                  */
+  int32_t smem_budget;   /* bytes of shared memory per CUDA block for the
+                            staged Hessian rows; 0 = library default       */
+} mad_opts;
+
+/* Term parameters for one evaluation.  All arrays are device pointers in the
+ * context's dtype, owned by the caller, read during the call only.         */
+typedef struct {
+  uint32_t mask;            /* MAD_TERM_* bits                               */
+  uint32_t flags;           /* MAD_EVAL_* bits                               */
+  const void* spring_rest;  /* [E] L0 per edge, in mad_edges() order         */
+  double spring_k;          /* stiffness k                                   */
+  const void* inertia_xt;   /* [V][dof] target positions xt                  */
+  double inertia_w;         /* w = m / h^2                                   */
+  const void* face_Minv;    /* [nF][2][2] row-major Dm^-1 per face (dof 2)   */
+  const void* face_area;    /* [nF] rest area per face                       */
+  double pair_k;            /* k_p for the current pair set                  */
+} mad_terms;
+
+typedef struct {
+  int32_t V, nF, E, dof;
+  int32_t dtype;            /* mad_dtype                                     */
+  int32_t nnzb_base;        /* blocks of the mesh pattern                    */
+  int32_t capacity_blocks;  /* blocks the dynamic CSR can hold; H_vals must
+                               hold capacity_blocks * dof * dof elements     */
+  int32_t max_pairs;
+  int32_t n_patches;
+  int32_t max_patch_vertices;   /* owned + ribbon vertices of the largest patch */
+  int32_t max_patch_owned;
+  int32_t smem_bytes;       /* dynamic shared memory of the assembly kernel  */
+  int64_t device_bytes;     /* device memory the context holds               */
+} mad_info_t;
+
+/* Fill *o with the defaults listed in mad_opts. */
+void mad_default_opts(mad_opts* o);
+
+/* Analyse the mesh and preallocate the block-CSR pattern (section 方法, key
+ * design 3: the pattern follows from connectivity and the declared 1-ring
+ * stencils; it is built on the GPU by a parallel per-row count, a prefix sum
+ * and a fill, followed by a per-row sort).  Also extracts the unique edges,
+ * partitions the vertices into patches (key design 2) and builds the
+ * per-patch term tables and CSR block-offset lookup.
+ *   V, nF   vertex and face counts (V >= 0, nF >= 0)
+ *   F       HOST [nF][3] vertex indices; each in [0, V), three distinct
+ *   dof     2 or 3;  dt  MAD_F32 or MAD_F64;  o  NULL for defaults
+ *   out     receives the new context
+ * Allocates all device memory the context will ever use and synchronises
+ * `stream` once at the end.  Errors: MAD_ERR_INVALID_ARG (bad sizes or
+ * faces), MAD_ERR_OOM, MAD_ERR_CUDA.  On error *out is NULL.               */
+mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof,
+                      mad_dtype dt, const mad_opts* o, void* stream,
+                      mad_ctx** out);
+
+/* Sizes and layout facts of a context. */
+mad_status mad_info(const mad_ctx* c, mad_info_t* info);
+
+/* Unique undirected mesh edges (i < j) sorted by (i, j): DEVICE [E][2],
+ * borrowed, valid until mad_destroy.  spring_rest is indexed in this order. */
+mad_status mad_edges(const mad_ctx* c, const int32_t** ij, int32_t* E);
+
+/* Current block-CSR pattern (the mesh pattern until the first
+ * mad_add_pairs, then the pattern holding the latest pair set):
+ * DEVICE row_ptr [V+1] and col_idx [capacity_blocks]; *nnzb_dev is a DEVICE
+ * int32 holding the block count.  Borrowed; the pointers change with each
+ * mad_add_pairs call (double buffering) and the contents are produced in
+ * stream order.                                                          */
+mad_status mad_pattern(const mad_ctx* c, const int32_t** row_ptr,
+                       const int32_t** col_idx, const int32_t** nnzb_dev);
+
+/* Fused evaluate + differentiate + assemble (section 方法: g = sum S^T g_j,
+ * H = sum S^T H_j S_j; per-term forward-mode AD in registers, patch-local
+ * pre-reduction in shared memory).  Overwrites every element of g and of
+ * the first nnzb blocks of H_vals.
+ *   x       DEVICE [V][dof] positions
+ *   t       HOST struct; its arrays are DEVICE pointers (see mad_terms)
+ *   g       DEVICE [V][dof] gradient (out)
+ *   H_vals  DEVICE [capacity_blocks][dof][dof] Hessian values (out)
+ *   energy  DEVICE double (out) or NULL to skip the energy
+ * MAD_TERM_PAIR uses the pair set of the latest mad_add_pairs on this
+ * context.  Errors: MAD_ERR_INVALID_ARG (NULL array for an active term,
+ * SYMDIR with dof 3), MAD_ERR_CUDA (launch failure).                       */
+mad_status mad_eval(mad_ctx* c, const void* x, const mad_terms* t, void* g,
+                    void* H_vals, double* energy, void* stream);
+
+/* Matrix-free Hessian-vector product y = H(x) v of the same terms, without
+ * forming H (section 实验结果, parameterization with matrix-free HVP).
+ *   x, v    DEVICE [V][dof];  y  DEVICE [V][dof] (out, overwritten)     */
+mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t,
+                   const void* v, void* y, void* stream);
+
+/* Replace the runtime pair set (section 方法, key design 4: interaction
+ * discovery is decoupled from evaluation; new off-diagonal blocks are
+ * inserted on the GPU into the inactive CSR buffer, which then becomes the
+ * active one; no host round trip).
+ *   n       number of pairs, 0 <= n <= max_pairs (n = 0 restores the mesh
+ *           pattern)
+ *   ij      DEVICE [n][2] vertex indices, i != j, any order; duplicates and
+ *           pairs on existing mesh edges are allowed and merge into one block
+ *   rest    DEVICE [n] rest length r_p of each pair (context dtype)
+ * The inputs are read in stream order during the call's kernels; the caller
+ * may reuse them once the stream has passed the call.  A pair with an index
+ * out of range or i == j is skipped and sets MAD_ERR_INDEX in the device
+ * status.  If the merged pattern would exceed capacity_blocks, the device
+ * status gets MAD_ERR_CAPACITY and the previous pattern and pair set stay in
+ * effect (the new buffer receives a copy of them).
+ * Errors returned at once: MAD_ERR_INVALID_ARG, MAD_ERR_CAPACITY
+ * (n > max_pairs).                                                         */
+mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij,
+                         const void* rest, void* stream);
+
+/* Synchronise `stream`, read and clear the sticky device status word and
+ * return it (MAD_OK when no device-side error was recorded).  Off the hot
+ * path by design.                                                          */
+mad_status mad_status_sync(mad_ctx* c, void* stream);
+
+/* mad_eval for callers whose data lives in HOST memory: copies x to the
+ * device, evaluates, copies g, H_vals and the energy back, and synchronises
+ * `stream` before returning.  x, g, H_vals, energy are HOST pointers (pinned
+ * memory gives full copy bandwidth); energy may be NULL.  The term
+ * parameter arrays in *t stay DEVICE pointers.  H_vals receives nnzb blocks
+ * where nnzb is the current pattern's block count.  The first call
+ * allocates the context's device staging buffers for x, g and H_vals.      */
+mad_status mad_eval_host(mad_ctx* c, const void* x, const mad_terms* t,
+                         void* g, void* H_vals, double* energy, void* stream);
+
+/* Human-readable description of the last error on this context (or of the
+ * last failed mad_create when c is NULL).  Never NULL.                     */
+const char* mad_last_error(const mad_ctx* c);
+
+/* Release every resource of the context (synchronises the device first).  */
+void mad_destroy(mad_ctx* c);
+
+/* Self-test of the forward-mode number types on the device, used by the test
+ * suite.  For each of n inputs (a, b) (HOST double [n][2]) it evaluates, in
+ * fp64 hyper-dual arithmetic with tangents seeded on (a, b):
+ *   f1 = a sin a,          f2 = a sin b + b cos a,
+ *   f3 = sqrt(a^2 + b^2),  f4 = a / b
+ * and writes value, gradient (2) and packed Hessian (3) of each: HOST double
+ * [n][4][6].  f1 and f2 are the worked examples (Code Examples section) of
+ * the page "How to Implement Automatic Differentiation Using the $autodiff
+ * Block for Custom Kernels", whose gradients it states in closed form.      */
+mad_status mad_selftest_dual(int32_t n, const double* ab, double* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAD_H_ */

@@ -1,0 +1,130 @@
+"""Runtime vertex-vertex pairs: GPU insertion into the double-buffered CSR
+and assembly with all terms, vs the fp64 oracle (pattern bit-exact)."""
+import numpy as np
+import pytest
+
+import mesh_inputs as mi
+from _parity import assert_close, check_cloth, cloth_context, cloth_terms, gpu_pattern, run_eval, to_dev
+
+pytestmark = pytest.mark.gpu
+FULL = 1
+
+
+def add_pairs(ctx, pairs, rest, dtype):
+    ctx.mad_add_pairs(to_dev(np.asarray(pairs, np.int32)), to_dev(np.asarray(rest), dtype))
+
+
+def pair_case(orc, n, P, dtype="float32", seed=1005, step=0, flags=0, **kw):
+    ctx, st = cloth_context(n, dtype, **kw)
+    x = mi.cloth_x(n, seed, step, np.dtype(dtype))
+    pairs = mi.random_pairs(n, P, seed, step)
+    rest = mi.pair_rest(x, pairs, np.dtype(dtype))
+    add_pairs(ctx, pairs, rest, dtype)
+    assert ctx.mad_status_sync() == 0
+    return check_cloth(orc, n, dtype, mask=11, flags=flags, step=step, seed=seed, pairs=pairs,
+                       prest=rest, ctx=ctx, st=st)
+
+
+@pytest.mark.parametrize("flags", [0, FULL])
+def test_pairs_small(orc, flags):
+    pair_case(orc, 30, 60, flags=flags)
+
+
+def test_pairs_fp64(orc):
+    pair_case(orc, 40, 150, "float64")
+
+
+def test_pairs_1000x1000_full(orc):
+    r = pair_case(orc, 1000, 100000)
+    rp, ci, nnzb = gpu_pattern(r["ctx"])
+    assert nnzb == 6992002 + 200000
+
+
+def test_replace_semantics_and_double_buffer(orc):
+    n = 25
+    ctx, st = cloth_context(n, "float64")
+    x = mi.cloth_x(n, 1, 0, np.float64)
+    for step in range(3):
+        pairs = mi.random_pairs(n, 40 + 10 * step, 7, step)
+        rest = mi.pair_rest(x, pairs, np.float64)
+        add_pairs(ctx, pairs, rest, "float64")
+        check_cloth(orc, n, "float64", mask=11, seed=1, pairs=pairs, prest=rest, ctx=ctx, st=st)
+    # n = 0 restores the mesh pattern
+    ctx.mad_add_pairs(None, None)
+    check_cloth(orc, n, "float64", mask=11, seed=1, ctx=ctx, st=st)
+
+
+def test_duplicates_edge_coincidence_and_shared_rows(orc):
+    n = 12
+    ctx, st = cloth_context(n, "float64")
+    x = mi.cloth_x(n, 3, 0, np.float64)
+    pairs = np.array([[0, 50], [50, 0], [0, 50],      # duplicates (both orders)
+                      [0, 1], [13, 12],               # on mesh edges
+                      [0, 99], [0, 143], [5, 99],     # rows 0 and 99 gain several blocks
+                      [143, 70], [70, 143]], np.int32)
+    rest = np.linspace(0.05, 0.3, len(pairs))
+    add_pairs(ctx, pairs, rest, "float64")
+    assert ctx.mad_status_sync() == 0
+    check_cloth(orc, n, "float64", mask=11, seed=3, pairs=pairs, prest=rest, ctx=ctx, st=st)
+
+
+def test_many_pairs_on_one_vertex_spill_rows(orc):
+    # vertex 0 gains 300 blocks: more than the shared-memory reserve, so its
+    # row is assembled in place in global memory
+    n = 30
+    ctx, st = cloth_context(n, "float64")
+    x = mi.cloth_x(n, 4, 0, np.float64)
+    far = np.array([v for v in range(n * n) if not mi.grid_adjacent(n, 0, v) and v != 0][:300])
+    pairs = np.stack([np.zeros_like(far), far], 1).astype(np.int32)
+    rest = mi.pair_rest(x, pairs, np.float64)
+    add_pairs(ctx, pairs, rest, "float64")
+    check_cloth(orc, n, "float64", mask=11, seed=4, pairs=pairs, prest=rest, ctx=ctx, st=st)
+
+
+def test_bad_index_sets_status_and_is_skipped(orc):
+    n = 10
+    ctx, st = cloth_context(n, "float64")
+    x = mi.cloth_x(n, 5, 0, np.float64)
+    good = np.array([[0, 55], [3, 77]], np.int32)
+    bad = np.array([[0, 100], [7, 7], [-1, 4]], np.int32)
+    pairs = np.concatenate([good[:1], bad, good[1:]])
+    rest = np.full(len(pairs), 0.2)
+    add_pairs(ctx, pairs, rest, "float64")
+    assert ctx.mad_status_sync() == 5  # MAD_ERR_INDEX
+    assert ctx.mad_status_sync() == 0  # cleared
+    check_cloth(orc, n, "float64", mask=11, seed=5, pairs=good, prest=np.full(2, 0.2), ctx=ctx, st=st)
+
+
+def test_capacity_overflow_keeps_previous_pattern(orc):
+    import hessian_assembly_b200 as mad
+    n = 10
+    ctx, st = cloth_context(n, "float64", slack=0.02, max_pairs=64)  # 12 spare blocks
+    x = mi.cloth_x(n, 6, 0, np.float64)
+    p1 = mi.random_pairs(n, 4, 6, 0)
+    r1 = mi.pair_rest(x, p1, np.float64)
+    add_pairs(ctx, p1, r1, "float64")
+    assert ctx.mad_status_sync() == 0
+    p2 = mi.random_pairs(n, 30, 6, 1)  # 60 new blocks > 12 spare
+    add_pairs(ctx, p2, mi.pair_rest(x, p2, np.float64), "float64")
+    assert ctx.mad_status_sync() == mad.MAD_ERR_CAPACITY
+    check_cloth(orc, n, "float64", mask=11, seed=6, pairs=p1, prest=r1, ctx=ctx, st=st)
+    with pytest.raises(mad.MadError) as ei:
+        add_pairs(ctx, mi.random_pairs(n, 65, 6, 2), np.ones(65), "float64")
+    assert ei.value.status == mad.MAD_ERR_CAPACITY
+
+
+def test_hvp_with_pairs(orc):
+    import torch
+    n = 30
+    ctx, st = cloth_context(n, "float64")
+    x = mi.cloth_x(n, 8, 0, np.float64)
+    pairs = mi.random_pairs(n, 80, 8, 0)
+    rest = mi.pair_rest(x, pairs, np.float64)
+    add_pairs(ctx, pairs, rest, "float64")
+    v = mi.probe_vector(st["V"], 3, 9, np.float64)
+    y = torch.zeros((st["V"], 3), dtype=torch.float64, device="cuda")
+    ctx.mad_hvp(to_dev(x), cloth_terms(st, "float64", 11), to_dev(v), y)
+    rp, ci = orc.pattern(st["V"], st["F"], pairs)
+    og, oH, oE = orc.eval(st["V"], 3, x, 11, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
+                          xt=st["xt"], w=st["w"], pairs=pairs, prest=rest, kp=mi.PAIR_K)
+    assert_close("y", y.cpu().numpy(), orc.bsr_mv(st["V"], 3, rp, ci, oH, v), "float64")
