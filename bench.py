@@ -139,8 +139,9 @@ def run_ours(args, rank, world, dist):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     st = mi.cloth_static(N_GRID, np.float32)
-    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
-    terms = mad.Terms(mask=mad.MAD_TERM_SPRING | mad.MAD_TERM_INERTIA,
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"],
+                      patch_faces=args.patch_faces)
+    terms = mad.Terms(mask=mad.MAD_TERM_SPRING | mad.MAD_TERM_INERTIA, flags=args.flags,
                       spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
                       inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"])
     pool = min(args.steps + args.warmup, args.pool)
@@ -226,7 +227,8 @@ def run_ours(args, rank, world, dist):
         "config": {"workload": WORKLOAD, "n": N_GRID, "seed": SEED, "x_pool": pool,
                    "l2": "inputs + outputs per step 0.36 GB > 126 MB L2; x from a pool of "
                          f"{pool} distinct perturbations", "parallelism": f"replicas x{world}",
-                   "patches": ctx.info.n_patches, "smem_bytes": ctx.info.smem_bytes},
+                   "patches": ctx.info.n_patches, "patch_faces": args.patch_faces,
+                   "smem_bytes": ctx.info.smem_bytes},
         "roofline": roof, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk,
         "impl": "ours",
     }
@@ -383,6 +385,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--pool", type=int, default=32)
+    ap.add_argument("--patch-faces", type=int, default=512)
+    ap.add_argument("--flags", type=int, default=0, help="MAD_EVAL_* bits for the timed step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra", action="store_true")

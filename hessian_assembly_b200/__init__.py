@@ -41,6 +41,7 @@ MAD_TERM_INERTIA = 2
 MAD_TERM_SYMDIR = 4
 MAD_TERM_PAIR = 8
 MAD_EVAL_FULL_STENCIL_AD = 1
+MAD_EVAL_EDGE_SCATTER = 2
 
 STATUS_NAMES = {0: "MAD_OK", 1: "MAD_ERR_INVALID_ARG", 2: "MAD_ERR_CUDA", 3: "MAD_ERR_OOM",
                 4: "MAD_ERR_CAPACITY", 5: "MAD_ERR_INDEX", 6: "MAD_ERR_TIMEOUT",

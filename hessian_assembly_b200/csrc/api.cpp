@@ -27,15 +27,24 @@ struct mad_ctx {
   int32_t* F_dev = nullptr;
   int32_t* base_nnzb_dev = nullptr;
   // patches
-  int n_patches = 0, nv_max = 0, no_max = 0, stage_cap = 0;
+  int n_patches = 0, nv_max = 0, no_max = 0;
+  // staging capacity in dtype elements: the largest patch's mesh-pattern rows
+  // plus 16-byte alignment room per run; stage_cap adds a reserve for pair
+  // blocks
+  int stage_base = 0;
+  int stage_cap = 0;
   PatchHdr* hdr = nullptr;
   int32_t* vgid = nullptr;
-  uint32_t* meta = nullptr;
+  uint2* meta = nullptr;
+  uint32_t* runs = nullptr;
   EdgeLut* elut = nullptr;
   int32_t* eid = nullptr;
   int32_t* ecol = nullptr;
   FaceLut* flut = nullptr;
   int32_t* fcol = nullptr;
+  uint16_t* slot_lidx = nullptr;
+  int32_t* slot_eid = nullptr;
+  int rho = 0;  // staging room per row for pair blocks (pairs active)
   double* epart = nullptr;
   size_t smem_eval = 0, smem_hvp = 0;
   // dynamic pattern
@@ -54,6 +63,7 @@ struct mad_ctx {
 
 namespace {
 
+constexpr int kMaxPatchOwned = 256;  // threads per block of the patch kernels
 std::string g_create_error;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -108,7 +118,9 @@ EvalLaunch eval_launch(const mad_ctx* c) {
   L.n_patches = c->n_patches;
   L.nv_max = c->nv_max;
   L.no_max = c->no_max;
-  L.stage_cap = c->stage_cap;
+  // without pair blocks the rows never outgrow the mesh pattern, so the
+  // kernel is launched with less shared memory (more blocks per SM)
+  L.stage_cap = c->active < 0 ? std::min(c->stage_base, c->stage_cap) : c->stage_cap;
   L.hdr = c->hdr;
   L.vgid = c->vgid;
   L.meta = c->meta;
@@ -117,6 +129,10 @@ EvalLaunch eval_launch(const mad_ctx* c) {
   L.ecol = c->ecol;
   L.flut = c->flut;
   L.fcol = c->fcol;
+  L.slot_lidx = c->slot_lidx;
+  L.slot_eid = c->slot_eid;
+  L.runs = c->runs;
+  L.rho = c->active < 0 ? 0 : c->rho;
   L.epart = c->epart;
   if (c->active < 0) {
     L.rp = c->pat.rp;
@@ -139,7 +155,7 @@ mad_status check_terms(mad_ctx* c, const mad_terms* t) {
   if (!t) return fail(c, MAD_ERR_INVALID_ARG, "terms is NULL");
   const uint32_t known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR;
   if (t->mask & ~known) return fail(c, MAD_ERR_INVALID_ARG, "unknown term bits in mask");
-  if (t->flags & ~(uint32_t)MAD_EVAL_FULL_STENCIL_AD)
+  if (t->flags & ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER))
     return fail(c, MAD_ERR_INVALID_ARG, "unknown evaluation flags");
   if ((t->mask & MAD_TERM_SPRING) && c->E > 0 && !t->spring_rest)
     return fail(c, MAD_ERR_INVALID_ARG, "spring term active but spring_rest is NULL");
@@ -259,6 +275,7 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     int target = opts.patch_faces;
     if (nF > 0)
       target = (int)std::max<long long>(1, std::llround((double)opts.patch_faces * V / nF));
+    target = std::min(target, kMaxPatchOwned);  // one owned vertex per thread
     HostPatches hp;
     msg = build_patches(V, nF, F, rp.data(), ci.data(), opts.part_xyz, opts.part_dim, target,
                         max_stage_blocks, hp);
@@ -271,7 +288,22 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     c->nv_max = std::max(1, hp.nv_max);
     c->no_max = std::max(1, hp.no_max);
     // staging room: the largest patch's rows plus a reserve for pair blocks
-    c->stage_cap = hp.stage_max + std::max(16, hp.stage_max / 4);
+    if (c->no_max > kMaxPatchOwned) {
+      g_create_error = "patch with more owned vertices than threads per block";
+      free_ctx(c);
+      return MAD_ERR_UNIMPLEMENTED;
+    }
+    // staging: rows at a fixed stride per patch; with pairs active every row
+    // gets rho spare blocks (rows that outgrow their run's window are
+    // assembled in place in H)
+    c->rho = 2;
+    size_t st0 = 1, st1 = 1;
+    for (const PatchHdr& h : hp.hdr) {
+      st0 = std::max(st0, patch_stage_elems(h, dof, c->esz, 0));
+      st1 = std::max(st1, patch_stage_elems(h, dof, c->esz, c->rho));
+    }
+    c->stage_base = (int)st0;
+    c->stage_cap = (int)st1;
     CREATE_CK(upload(c, &c->hdr, hp.hdr));
     CREATE_CK(upload(c, &c->vgid, hp.vgid));
     CREATE_CK(upload(c, &c->meta, hp.meta));
@@ -280,6 +312,9 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     CREATE_CK(upload(c, &c->ecol, hp.ecol));
     CREATE_CK(upload(c, &c->flut, hp.flut));
     CREATE_CK(upload(c, &c->fcol, hp.fcol));
+    CREATE_CK(upload(c, &c->slot_lidx, hp.slot_lidx));
+    CREATE_CK(upload(c, &c->slot_eid, hp.slot_eid));
+    CREATE_CK(upload(c, &c->runs, hp.runs));
     CREATE_CK(dev_alloc(c, &c->epart, sizeof(double) * std::max(1, c->n_patches)));
   }
   // 3. shared memory of the patch kernels
@@ -287,11 +322,13 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
                                    c->device));
   {
     EvalLaunch L = eval_launch(c);
+    L.stage_cap = c->stage_cap;
     // the static shared arrays of the kernels take a few hundred bytes
     const size_t limit = (size_t)smem_optin > 1024 ? (size_t)smem_optin - 1024 : 0;
     c->smem_eval = eval_smem_bytes(L, false);
-    while (c->smem_eval > limit && c->stage_cap > 1) {
-      c->stage_cap = std::max(1, c->stage_cap * 7 / 8);  // rows past it go in place
+    if (c->smem_eval > limit) {  // drop the pair reserve first
+      c->rho = 0;
+      c->stage_cap = c->stage_base;
       L.stage_cap = c->stage_cap;
       c->smem_eval = eval_smem_bytes(L, false);
     }

@@ -194,8 +194,9 @@ __host__ __device__ __forceinline__ double inv(double a) { return 1.0 / a; }
 template <typename T, int N>
 __host__ __device__ __forceinline__ HyperDual<T, N> sqrt(const HyperDual<T, N>& a) {
   const T f0 = ::sqrt(a.v);
-  const T f1 = T(0.5) / f0;   // d sqrt = 1 / (2 sqrt)
-  const T f2 = -f1 / (T(2) * a.v);  // d2 sqrt = -1 / (4 v^{3/2})
+  const T r0 = T(1) / f0;
+  const T f1 = T(0.5) * r0;            // d sqrt = 1 / (2 sqrt v)
+  const T f2 = T(-0.25) * r0 * r0 * r0;  // d2 sqrt = -1 / (4 v^{3/2})
   return chain(a, f0, f1, f2);
 }
 
@@ -223,6 +224,94 @@ template <typename T, int N>
 __host__ __device__ __forceinline__ HyperDual<T, N> cos(const HyperDual<T, N>& a) {
   const T s = ::sin(a.v), c = ::cos(a.v);
   return chain(a, c, -s, -c);
+}
+
+// ---- affine quantities ------------------------------------------------------
+// A value that is affine in the seeded inputs (the inputs themselves, their
+// differences, constant linear maps of them) has an identically zero
+// Hessian.  Lin<T, N> carries only value and gradient, so no arithmetic is
+// spent on those zeros; products and squares of Lin values produce the first
+// non-zero Hessians.  This is exact (no approximation): it only drops terms
+// that are zero by construction.
+template <typename T, int N>
+struct Lin {
+  T v;
+  T g[N];
+};
+
+template <typename T, int N>
+__host__ __device__ __forceinline__ Lin<T, N> lin_var(T val, int k) {
+  Lin<T, N> r;
+  r.v = val;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r.g[i] = (i == k) ? T(1) : T(0);
+  return r;
+}
+
+template <typename T, int N>
+__host__ __device__ __forceinline__ Lin<T, N> operator+(const Lin<T, N>& a, const Lin<T, N>& b) {
+  Lin<T, N> r;
+  r.v = a.v + b.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r.g[i] = a.g[i] + b.g[i];
+  return r;
+}
+template <typename T, int N>
+__host__ __device__ __forceinline__ Lin<T, N> operator-(const Lin<T, N>& a, const Lin<T, N>& b) {
+  Lin<T, N> r;
+  r.v = a.v - b.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r.g[i] = a.g[i] - b.g[i];
+  return r;
+}
+template <typename T, int N>
+__host__ __device__ __forceinline__ Lin<T, N> operator*(const Lin<T, N>& a, T c) {
+  Lin<T, N> r;
+  r.v = a.v * c;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r.g[i] = a.g[i] * c;
+  return r;
+}
+
+// promotion
+template <typename T, int N>
+__host__ __device__ __forceinline__ HyperDual<T, N> to_hd(const Lin<T, N>& a) {
+  HyperDual<T, N> r;
+  r.v = a.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r.g[i] = a.g[i];
+#pragma unroll
+  for (int i = 0; i < Tri<N>::size; ++i) r.h[i] = T(0);
+  return r;
+}
+
+// a^2 of an affine value: Hessian 2 a' a'^T
+template <typename T, int N>
+__host__ __device__ __forceinline__ HyperDual<T, N> sq(const Lin<T, N>& a) {
+  HyperDual<T, N> r;
+  r.v = a.v * a.v;
+  const T two_v = T(2) * a.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r.g[i] = two_v * a.g[i];
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+#pragma unroll
+    for (int j = i; j < N; ++j) r.h[Tri<N>::idx(i, j)] = T(2) * (a.g[i] * a.g[j]);
+  return r;
+}
+
+// product of two affine values: Hessian a' b'^T + b' a'^T
+template <typename T, int N>
+__host__ __device__ __forceinline__ HyperDual<T, N> operator*(const Lin<T, N>& a, const Lin<T, N>& b) {
+  HyperDual<T, N> r;
+  r.v = a.v * b.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i) r.g[i] = a.v * b.g[i] + b.v * a.g[i];
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+#pragma unroll
+    for (int j = i; j < N; ++j) r.h[Tri<N>::idx(i, j)] = a.g[i] * b.g[j] + a.g[j] * b.g[i];
+  return r;
 }
 
 // Hessian entry (i, j) of a packed HyperDual, any order of i and j

@@ -26,6 +26,8 @@ struct PatchHdr {
   int32_t ebeg, ne, ecbeg, nce;  // edge terms; colour c spans
                                  // ecol[ecbeg+c] .. ecol[ecbeg+c+1] (relative)
   int32_t fbeg, nf, fcbeg, ncf;  // face terms, same layout
+  int32_t sbeg, stride;  // row slots: owned row r's slot p is sbeg + r*stride + p
+  int32_t rbeg, nruns;   // runs of consecutive owned vertices: runs[rbeg .. +nruns)
 };
 
 // Block-offset lookup for an edge term (built once per topology): local
@@ -45,6 +47,7 @@ struct FaceLut {
 };
 
 constexpr uint16_t kNotOwned = 0xFFFF;
+constexpr uint16_t kNoSlot = 0xFFFF;
 
 // Pair entry position word: low 30 bits = block position inside the row of
 // the current (dynamic) pattern; bit 30 set when this entry created that
@@ -52,10 +55,18 @@ constexpr uint16_t kNotOwned = 0xFFFF;
 constexpr int32_t kPairNewBlock = 1 << 30;
 constexpr int32_t kPairPosMask = (1 << 30) - 1;
 
-// Per-owned-vertex meta word: mesh-pattern row length | diagonal position << 16
+// Per-owned-vertex meta: x = mesh-pattern row length | diagonal position << 16,
+// y = first row of the vertex's run | run index << 16.  A run is a maximal
+// sequence of owned vertices with consecutive ids; their Hessian rows are
+// consecutive in H, so a run is staged and written back as one piece.
 __host__ __device__ inline uint32_t pack_meta(int blen, int dpos) {
   return (uint32_t)blen | ((uint32_t)dpos << 16);
 }
+
+// Row slots (the gather form of the block-offset lookup): for every block of
+// an owned row of the mesh pattern, in column order, the local index of the
+// column's vertex and the id of the edge joining it to the row's vertex (-1
+// on the diagonal); rows are padded to the patch's stride with kNoSlot.
 
 // Device status bits (sticky; read by mad_status_sync).
 enum : int32_t { kStatusIndex = 1, kStatusCapacity = 2, kStatusTimeout = 4 };
@@ -63,13 +74,16 @@ enum : int32_t { kStatusIndex = 1, kStatusCapacity = 2, kStatusTimeout = 4 };
 struct HostPatches {
   std::vector<PatchHdr> hdr;
   std::vector<int32_t> vgid;
-  std::vector<uint32_t> meta;   // indexed like vgid (owned entries used)
+  std::vector<uint2> meta;      // indexed like vgid (owned entries used)
   std::vector<EdgeLut> elut;
   std::vector<int32_t> eid;
   std::vector<int32_t> ecol;
   std::vector<FaceLut> flut;
   std::vector<int32_t> fcol;
-  int nv_max = 0, no_max = 0, stage_max = 0;
+  std::vector<uint16_t> slot_lidx;
+  std::vector<int32_t> slot_eid;
+  std::vector<uint32_t> runs;  // first row | row count << 16
+  int nv_max = 0, no_max = 0;
 };
 
 // Host partitioner (partition.cpp).  rp/ci: mesh pattern (host copies).
@@ -112,15 +126,20 @@ std::string build_pattern_gpu(int V, int nF, const int32_t* F_dev,
 
 // eval.cu
 struct EvalLaunch {
-  int dtype, dof, n_patches, nv_max, no_max, stage_cap;  // stage_cap in blocks
+  int dtype, dof, n_patches, nv_max, no_max;
+  int stage_cap;  // staging capacity in elements of the dtype
   const PatchHdr* hdr;
   const int32_t* vgid;
-  const uint32_t* meta;
+  const uint2* meta;
+  const uint32_t* runs;
   const EdgeLut* elut;
   const int32_t* eid;
   const int32_t* ecol;
   const FaceLut* flut;
   const int32_t* fcol;
+  const uint16_t* slot_lidx;
+  const int32_t* slot_eid;
+  int rho;            // staging room per row for inserted pair blocks
   const int32_t* rp;  // active row_ptr
   // pairs (active set); prow == nullptr when no pairs are active
   const int32_t* prow;
@@ -130,6 +149,8 @@ struct EvalLaunch {
   double* epart;  // [n_patches]
 };
 size_t eval_smem_bytes(const EvalLaunch& L, bool hvp);
+// staging elements one patch needs with `rho` spare blocks per row
+size_t patch_stage_elems(const PatchHdr& h, int dof, int esz, int rho);
 cudaError_t launch_eval(const EvalLaunch& L, const mad_terms& t, const void* x,
                         void* g, void* H, double* energy, cudaStream_t s);
 cudaError_t launch_hvp(const EvalLaunch& L, const mad_terms& t, const void* x,

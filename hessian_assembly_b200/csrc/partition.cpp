@@ -28,21 +28,28 @@
 namespace mad {
 namespace {
 
-constexpr int kMaxColours = 256;
-
+// Greedy colouring: a term takes the smallest colour not yet used by any of
+// its owned vertices.  Colour sets grow as needed (a vertex of valence d
+// needs d colours).
 struct Colouring {
-  std::vector<uint64_t> used;  // [no][kMaxColours/64]
-  explicit Colouring(int no) : used((size_t)no * (kMaxColours / 64), 0) {}
-  // smallest colour free on every owned vertex in vs (values < 0 ignored)
+  std::vector<std::vector<uint64_t>> used;  // per owned local vertex
+  explicit Colouring(int no) : used((size_t)no) {}
   int pick(const int* vs, int n) {
-    for (int w = 0; w < kMaxColours / 64; ++w) {
+    size_t words = 1;
+    for (int i = 0; i < n; ++i)
+      if (vs[i] >= 0) words = std::max(words, used[vs[i]].size() + 1);
+    for (size_t w = 0; w < words; ++w) {
       uint64_t m = 0;
       for (int i = 0; i < n; ++i)
-        if (vs[i] >= 0) m |= used[(size_t)vs[i] * (kMaxColours / 64) + w];
+        if (vs[i] >= 0 && w < used[vs[i]].size()) m |= used[vs[i]][w];
       if (~m) {
-        int c = w * 64 + __builtin_ctzll(~m);
-        for (int i = 0; i < n; ++i)
-          if (vs[i] >= 0) used[(size_t)vs[i] * (kMaxColours / 64) + w] |= 1ull << (c & 63);
+        const int c = (int)(w * 64) + __builtin_ctzll(~m);
+        for (int i = 0; i < n; ++i) {
+          if (vs[i] < 0) continue;
+          std::vector<uint64_t>& u = used[vs[i]];
+          if (u.size() <= w) u.resize(w + 1, 0);
+          u[w] |= 1ull << (c & 63);
+        }
         return c;
       }
     }
@@ -87,16 +94,18 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
       Range r = stack.back();
       stack.pop_back();
       int size = r.e - r.b;
-      int64_t blocks = 0;
+      int64_t maxlen = 1;
       double lo[3] = {1e300, 1e300, 1e300}, hi[3] = {-1e300, -1e300, -1e300};
       for (int i = r.b; i < r.e; ++i) {
         int v = order[i];
-        blocks += len[v];
+        maxlen = std::max<int64_t>(maxlen, len[v]);
         for (int a = 0; a < xyz_dim; ++a) {
           lo[a] = std::min(lo[a], xyz[(size_t)v * xyz_dim + a]);
           hi[a] = std::max(hi[a], xyz[(size_t)v * xyz_dim + a]);
         }
       }
+      // rows are staged at a fixed stride (the longest row of the patch)
+      const int64_t blocks = (int64_t)size * maxlen;
       if (size <= target_owned && blocks <= max_stage_blocks) {
         cuts.push_back(r.b);
         continue;
@@ -140,18 +149,19 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
       queue.push_back(seed);
       taken[seed] = 1;
       size_t qh = 0;
-      int64_t blocks = 0;
+      int64_t maxlen = 1;
       int cnt = 0;
       while (qh < queue.size()) {
         int v = queue[qh++];
-        if (cnt >= target_owned || blocks + len[v] > max_stage_blocks) {
+        const int64_t ml = std::max<int64_t>(maxlen, len[v]);
+        if (cnt >= target_owned || (cnt + 1) * ml > max_stage_blocks) {
           taken[v] = 0;  // give it back; it seeds a later patch
           seeds.push_back(v);
           continue;
         }
         order[pos++] = v;
         ++cnt;
-        blocks += len[v];
+        maxlen = ml;
         for (int q = rp[v]; q < rp[v + 1]; ++q) {
           int b = ci[q];
           if (!taken[b]) {
@@ -214,17 +224,61 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
     H.vbeg = (int)out.vgid.size();
     H.nv = nv;
     H.no = no;
-    int nstage = 0;
+    int nstage = 0, stride = 1;
+    for (int r = 0; r < no; ++r) {
+      nstage += len[owned[r]];
+      stride = std::max(stride, (int)len[owned[r]]);
+    }
+    H.nstage = nstage;
+    H.stride = stride;
+    // runs of consecutive vertex ids
+    H.rbeg = (int)out.runs.size();
+    std::vector<int> run_of(no), run_start(no);
+    for (int r = 0; r < no; ++r) {
+      if (r == 0 || owned[r] != owned[r - 1] + 1) {
+        out.runs.push_back((uint32_t)r);
+        run_start[r] = r;
+      } else {
+        run_start[r] = run_start[r - 1];
+      }
+      run_of[r] = (int)out.runs.size() - 1 - H.rbeg;
+      out.runs.back() += 1u << 16;  // one more row in this run
+    }
+    H.nruns = (int)out.runs.size() - H.rbeg;
     for (int r = 0; r < no; ++r) {
       out.vgid.push_back(owned[r]);
-      out.meta.push_back(pack_meta(len[owned[r]], dpos[owned[r]]));
-      nstage += len[owned[r]];
+      uint2 m;
+      m.x = pack_meta(len[owned[r]], dpos[owned[r]]);
+      m.y = (uint32_t)run_start[r] | ((uint32_t)run_of[r] << 16);
+      out.meta.push_back(m);
     }
     for (int h : halo) {
       out.vgid.push_back(h);
-      out.meta.push_back(0);
+      out.meta.push_back(make_uint2(0, 0));
     }
-    H.nstage = nstage;
+    // row slots: column local index + edge id for every mesh-pattern block,
+    // each row padded to the stride
+    H.sbeg = (int)out.slot_lidx.size();
+    for (int r = 0; r < no; ++r) {
+      const int a = owned[r];
+      for (int q = rp[a]; q < rp[a] + stride; ++q) {
+        if (q >= rp[a + 1]) {
+          out.slot_lidx.push_back(kNoSlot);
+          out.slot_eid.push_back(-1);
+          continue;
+        }
+        const int b = ci[q];
+        out.slot_lidx.push_back((uint16_t)lidx[b]);
+        if (b == a) {
+          out.slot_eid.push_back(-1);
+        } else if (a < b) {
+          out.slot_eid.push_back((int32_t)(eptr[a] + (q - rp[a]) - dpos[a] - 1));
+        } else {
+          const int pba = find_pos(ci, rp[b], rp[b + 1], a);
+          out.slot_eid.push_back((int32_t)(eptr[b] + pba - dpos[b] - 1));
+        }
+      }
+    }
 
     // edge terms: every edge with at least one owned endpoint, once
     et.clear();
@@ -249,7 +303,6 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
           t.eid = (int32_t)(eptr[b] + pba - dpos[b] - 1);
         int vs[2] = {r, b_owned ? lidx[b] : -1};
         t.colour = ce.pick(vs, 2);
-        if (t.colour < 0) return "more than 256 term colours in a patch";
         et.push_back(t);
       }
     }
@@ -304,7 +357,6 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
           }
           t.l.fid = f;
           t.colour = cf.pick(vs, 3);
-          if (t.colour < 0) return "more than 256 term colours in a patch";
           ft.push_back(t);
         }
       }
@@ -329,7 +381,6 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
     out.hdr.push_back(H);
     out.nv_max = std::max(out.nv_max, nv);
     out.no_max = std::max(out.no_max, no);
-    out.stage_max = std::max(out.stage_max, nstage);
   }
   return "";
 }

@@ -30,22 +30,24 @@
 namespace mad {
 
 // ---------------------------------------------------------------- energies
+// S is the number type of the inputs (plain T, Lin or HyperDual); products
+// of affine inputs become HyperDual, so the results are `auto`.
 template <typename S, int D, typename T>
-__device__ __forceinline__ S spring_energy(const S (&d)[D], T L0, T k) {
-  S s = sq(d[0]);
+__device__ __forceinline__ auto spring_energy(const S (&d)[D], T L0, T k) {
+  auto s = sq(d[0]);
 #pragma unroll
   for (int a = 1; a < D; ++a) s = s + sq(d[a]);
-  S l = sqrt(s);
-  S r = l - L0;
+  auto l = sqrt(s);
+  auto r = l - L0;
   return sq(r) * (T(0.5) * k);
 }
 
 // j = (J00, J01, J10, J11)
 template <typename S, typename T>
-__device__ __forceinline__ S symdir_energy(const S (&j)[4], T A) {
-  S a = sq(j[0]) + sq(j[1]) + sq(j[2]) + sq(j[3]);
-  S det = j[0] * j[3] - j[1] * j[2];
-  S id2 = sq(inv(det));
+__device__ __forceinline__ auto symdir_energy(const S (&j)[4], T A) {
+  auto a = sq(j[0]) + sq(j[1]) + sq(j[2]) + sq(j[3]);
+  auto det = j[0] * j[3] - j[1] * j[2];
+  auto id2 = sq(inv(det));
   return (a + a * id2) * A;
 }
 
@@ -63,9 +65,9 @@ template <typename T, int D, bool FULL>
 __device__ __forceinline__ void eval_edge(const T* xa, const T* xb, T L0, T k,
                                           EdgeDerivs<T, D>& o) {
   if constexpr (!FULL) {
-    HyperDual<T, D> d[D];
+    Lin<T, D> d[D];
 #pragma unroll
-    for (int a = 0; a < D; ++a) d[a] = hd_var<T, D>(xa[a] - xb[a], a);
+    for (int a = 0; a < D; ++a) d[a] = lin_var<T, D>(xa[a] - xb[a], a);
     HyperDual<T, D> e = spring_energy(d, L0, k);
     o.E = e.v;
 #pragma unroll
@@ -84,10 +86,10 @@ __device__ __forceinline__ void eval_edge(const T* xa, const T* xb, T L0, T k,
       }
   } else {
     constexpr int N = 2 * D;
-    HyperDual<T, N> d[D];
+    Lin<T, N> d[D];
 #pragma unroll
     for (int a = 0; a < D; ++a)
-      d[a] = hd_var<T, N>(xa[a], a) - hd_var<T, N>(xb[a], D + a);
+      d[a] = lin_var<T, N>(xa[a], a) - lin_var<T, N>(xb[a], D + a);
     HyperDual<T, N> e = spring_energy(d, L0, k);
     o.E = e.v;
 #pragma unroll
@@ -106,13 +108,88 @@ __device__ __forceinline__ void eval_edge(const T* xa, const T* xb, T L0, T k,
   }
 }
 
+// Compact per-term result kept in registers between the evaluation of all of
+// a thread's edge terms and the colour phases that add them into the rows.
+// Reduced seeding: K = d2E/dd2 (packed symmetric), g = dE/dd; the blocks are
+// (a,a) = (b,b) = K, (a,b) = (b,a) = -K and g_a = g = -g_b.
+template <typename T, int D, bool FULL>
+struct EdgeRes {
+  T K[Tri<D>::size];
+  T g[D];
+  T E;
+};
+template <typename T, int D>
+struct EdgeRes<T, D, true> {
+  EdgeDerivs<T, D> d;
+};
+
+template <typename T, int D, bool FULL>
+__device__ __forceinline__ void eval_edge_res(const T* xa, const T* xb, T L0, T k,
+                                              EdgeRes<T, D, FULL>& R) {
+  if constexpr (!FULL) {
+    Lin<T, D> d[D];
+#pragma unroll
+    for (int a = 0; a < D; ++a) d[a] = lin_var<T, D>(xa[a] - xb[a], a);
+    HyperDual<T, D> e = spring_energy(d, L0, k);
+    R.E = e.v;
+#pragma unroll
+    for (int a = 0; a < D; ++a) R.g[a] = e.g[a];
+#pragma unroll
+    for (int q = 0; q < Tri<D>::size; ++q) R.K[q] = e.h[q];
+  } else {
+    eval_edge<T, D, true>(xa, xb, L0, k, R.d);
+  }
+}
+
+// Add side `side` (0 = endpoint a, 1 = endpoint b) of an edge term into an
+// owned row: the diagonal block goes to the row's packed symmetric
+// accumulator `dacc`, the off-diagonal block to `off` (stored when the term
+// is the block's only contributor, else added), the gradient to `gr`.
+template <bool STORE, typename T>
+__device__ __forceinline__ void put(T& dst, T v) {
+  if constexpr (STORE) dst = v; else dst += v;
+}
+
+template <bool STORE_OFF, typename T, int D, bool FULL>
+__device__ __forceinline__ void apply_edge_side(const EdgeRes<T, D, FULL>& R, int side, T* dacc,
+                                                T* off, T* gr) {
+  if constexpr (!FULL) {
+    const T sg = side == 0 ? T(1) : T(-1);
+#pragma unroll
+    for (int q = 0; q < Tri<D>::size; ++q) dacc[q] += R.K[q];
+#pragma unroll
+    for (int a = 0; a < D; ++a) {
+#pragma unroll
+      for (int b = 0; b < D; ++b)
+        put<STORE_OFF>(off[a * D + b], -(a <= b ? R.K[Tri<D>::idx(a, b)] : R.K[Tri<D>::idx(b, a)]));
+      gr[a] += sg * R.g[a];
+    }
+  } else {
+#pragma unroll
+    for (int a = 0; a < D; ++a) {
+#pragma unroll
+      for (int b = a; b < D; ++b)
+        dacc[Tri<D>::idx(a, b)] += side == 0 ? R.d.Haa[a * D + b] : R.d.Hbb[a * D + b];
+#pragma unroll
+      for (int b = 0; b < D; ++b)
+        put<STORE_OFF>(off[a * D + b], side == 0 ? R.d.Hab[a * D + b] : R.d.Hab[b * D + a]);
+      gr[a] += side == 0 ? R.d.ga[a] : R.d.gb[a];
+    }
+  }
+}
+
+template <typename T, int D, bool FULL>
+__device__ __forceinline__ T edge_energy(const EdgeRes<T, D, FULL>& R) {
+  if constexpr (!FULL) return R.E; else return R.d.E;
+}
+
 // Inertia: reduced seeding on r = x - xt (width D)
 template <typename T, int D>
 __device__ __forceinline__ void eval_inertia(const T* x, const T* xt, T w, T& E, T* g,
                                              T* Hd) {
-  HyperDual<T, D> s = hd_const<T, D>(T(0));
+  HyperDual<T, D> s = sq(lin_var<T, D>(x[0] - xt[0], 0));
 #pragma unroll
-  for (int a = 0; a < D; ++a) s = s + sq(hd_var<T, D>(x[a] - xt[a], a));
+  for (int a = 1; a < D; ++a) s = s + sq(lin_var<T, D>(x[a] - xt[a], a));
   HyperDual<T, D> e = s * (T(0.5) * w);
   E = e.v;
 #pragma unroll
@@ -145,9 +222,9 @@ __device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u
 #pragma unroll
       for (int ga = 0; ga < 2; ++ga)
         Jv[2 * al + ga] = (u1[al] - u0[al]) * M[ga] + (u2[al] - u0[al]) * M[2 + ga];
-    HyperDual<T, 4> j[4];
+    Lin<T, 4> j[4];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) j[p] = hd_var<T, 4>(Jv[p], p);
+    for (int p = 0; p < 4; ++p) j[p] = lin_var<T, 4>(Jv[p], p);
     HyperDual<T, 4> e = symdir_energy(j, A);
     o.E = e.v;
 #pragma unroll
@@ -172,14 +249,14 @@ __device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u
             o.H[k][l][2 * al + be] = s;
           }
   } else {
-    HyperDual<T, 6> u[3][2];
+    Lin<T, 6> u[3][2];
 #pragma unroll
     for (int al = 0; al < 2; ++al) {
-      u[0][al] = hd_var<T, 6>(u0[al], 0 + al);
-      u[1][al] = hd_var<T, 6>(u1[al], 2 + al);
-      u[2][al] = hd_var<T, 6>(u2[al], 4 + al);
+      u[0][al] = lin_var<T, 6>(u0[al], 0 + al);
+      u[1][al] = lin_var<T, 6>(u1[al], 2 + al);
+      u[2][al] = lin_var<T, 6>(u2[al], 4 + al);
     }
-    HyperDual<T, 6> j[4];
+    Lin<T, 6> j[4];
 #pragma unroll
     for (int al = 0; al < 2; ++al)
 #pragma unroll

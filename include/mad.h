@@ -81,7 +81,13 @@ enum {
    * term's natural variables (the edge vector; the 2x2 Jacobian J) and maps
    * g_j, H_j back through the term's constant linear input map.  Both give
    * the same derivatives up to rounding.                                     */
-  MAD_EVAL_FULL_STENCIL_AD = 1u
+  MAD_EVAL_FULL_STENCIL_AD = 1u,
+  /* Assemble edge terms by scattering each term once into the rows of its
+   * owned endpoints, colour by colour, instead of the default, where the
+   * thread that owns a row gathers the derivatives of the row's edge terms
+   * (each term evaluated once per owned endpoint).  Same results up to
+   * rounding; provided for comparison.                                       */
+  MAD_EVAL_EDGE_SCATTER = 2u
 };
 
 typedef struct {

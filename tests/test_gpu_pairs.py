@@ -8,6 +8,7 @@ from _parity import assert_close, check_cloth, cloth_context, cloth_terms, gpu_p
 
 pytestmark = pytest.mark.gpu
 FULL = 1
+SCAT = 2
 
 
 def add_pairs(ctx, pairs, rest, dtype):
@@ -25,7 +26,7 @@ def pair_case(orc, n, P, dtype="float32", seed=1005, step=0, flags=0, **kw):
                        prest=rest, ctx=ctx, st=st)
 
 
-@pytest.mark.parametrize("flags", [0, FULL])
+@pytest.mark.parametrize("flags", [0, FULL, SCAT])
 def test_pairs_small(orc, flags):
     pair_case(orc, 30, 60, flags=flags)
 
