@@ -23,7 +23,8 @@ from dataclasses import dataclass
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmad.so")
+# an alternative build of the same library can be selected for experiments
+LIB_PATH = os.environ.get("HESSIAN_ASSEMBLY_B200_LIB", os.path.join(_HERE, "libmad.so"))
 
 MAD_OK = 0
 MAD_ERR_INVALID_ARG = 1
@@ -42,6 +43,7 @@ MAD_TERM_SYMDIR = 4
 MAD_TERM_PAIR = 8
 MAD_EVAL_FULL_STENCIL_AD = 1
 MAD_EVAL_EDGE_SCATTER = 2
+MAD_EVAL_PATCH_STAGED = 4
 
 STATUS_NAMES = {0: "MAD_OK", 1: "MAD_ERR_INVALID_ARG", 2: "MAD_ERR_CUDA", 3: "MAD_ERR_OOM",
                 4: "MAD_ERR_CAPACITY", 5: "MAD_ERR_INDEX", 6: "MAD_ERR_TIMEOUT",

@@ -38,8 +38,8 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def _compile(src: str, extra: list[str]) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, extra: list[str], bdir: str) -> str:
+    obj = os.path.join(bdir, os.path.basename(src) + ".o")
     cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
@@ -49,21 +49,25 @@ def _compile(src: str, extra: list[str]) -> str:
     return obj
 
 
-def build(force: bool = False, extra: list[str] | None = None, jobs: int | None = None) -> str:
-    if not force and not extra and up_to_date():
+def build(force: bool = False, extra: list[str] | None = None, jobs: int | None = None,
+          out: str | None = None, build_dir: str | None = None) -> str:
+    """Compile and link; `extra` nvcc flags and `out` select a variant build."""
+    lib = out or LIB
+    if not force and not extra and out is None and up_to_date():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    bdir = build_dir or BUILD
+    os.makedirs(bdir, exist_ok=True)
     extra = list(extra or [])
     srcs = _sources()
     with cf.ThreadPoolExecutor(max_workers=jobs or min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra), srcs))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, extra, bdir), srcs))
+    tmp = lib + ".tmp"
     cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

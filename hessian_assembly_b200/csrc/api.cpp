@@ -8,6 +8,7 @@
 // runtime pairs into a double-buffered CSR on the GPU (mad_add_pairs).  After
 // mad_create nothing here allocates or synchronises (except the documented
 // host-buffer and status entry points).
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -27,7 +28,8 @@ struct mad_ctx {
   int32_t* F_dev = nullptr;
   int32_t* base_nnzb_dev = nullptr;
   // patches
-  int n_patches = 0, nv_max = 0, no_max = 0;
+  int n_patches = 0, nv_max = 0, no_max = 0, slots_max = 0;
+  int grid_base = 0, grid_pairs = 0;  // persistent grids (no pairs / pairs)
   // staging capacity in dtype elements: the largest patch's mesh-pattern rows
   // plus 16-byte alignment room per run; stage_cap adds a reserve for pair
   // blocks
@@ -45,6 +47,12 @@ struct mad_ctx {
   uint16_t* slot_lidx = nullptr;
   int32_t* slot_eid = nullptr;
   int rho = 0;  // staging room per row for pair blocks (pairs active)
+  // row-streaming kernel tables
+  int rows_s0 = 0;
+  int2* rows_slots = nullptr;
+  uint32_t* rows_meta = nullptr;
+  int32_t* rows_ofl_ptr = nullptr;
+  int2* rows_ofl = nullptr;
   double* epart = nullptr;
   size_t smem_eval = 0, smem_hvp = 0;
   // dynamic pattern
@@ -118,6 +126,8 @@ EvalLaunch eval_launch(const mad_ctx* c) {
   L.n_patches = c->n_patches;
   L.nv_max = c->nv_max;
   L.no_max = c->no_max;
+  L.slots_max = c->slots_max;
+  L.grid = c->active < 0 ? c->grid_base : c->grid_pairs;
   // without pair blocks the rows never outgrow the mesh pattern, so the
   // kernel is launched with less shared memory (more blocks per SM)
   L.stage_cap = c->active < 0 ? std::min(c->stage_base, c->stage_cap) : c->stage_cap;
@@ -151,11 +161,48 @@ EvalLaunch eval_launch(const mad_ctx* c) {
   return L;
 }
 
+RowsLaunch rows_launch(const mad_ctx* c) {
+  RowsLaunch L;
+  L.dtype = c->dtype;
+  L.dof = c->dof;
+  L.V = c->V;
+  L.s0 = c->rows_s0;
+  L.rho = c->active < 0 ? 0 : c->rho;
+  L.slots = c->rows_slots;
+  L.meta = c->rows_meta;
+  L.ofl_ptr = c->rows_ofl_ptr;
+  L.ofl = c->rows_ofl;
+  L.epart = c->epart;
+  if (c->active < 0) {
+    L.rp = c->pat.rp;
+    L.prow = nullptr;
+    L.pe_col = nullptr;
+    L.pe_pos = nullptr;
+    L.pe_rest = nullptr;
+  } else {
+    const DynBuf& b = c->buf[c->active];
+    L.rp = b.rp;
+    L.prow = b.prow;
+    L.pe_col = b.pe_col;
+    L.pe_pos = b.pe_pos;
+    L.pe_rest = b.pe_rest;
+  }
+  return L;
+}
+
+// Edge, vertex and pair terms alone go to the row-streaming kernel unless the
+// caller asks for the patch kernel or the scatter mode.
+bool use_rows(const mad_terms* t) {
+  return !(t->mask & MAD_TERM_SYMDIR) &&
+         !(t->flags & (MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED));
+}
+
 mad_status check_terms(mad_ctx* c, const mad_terms* t) {
   if (!t) return fail(c, MAD_ERR_INVALID_ARG, "terms is NULL");
   const uint32_t known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR;
   if (t->mask & ~known) return fail(c, MAD_ERR_INVALID_ARG, "unknown term bits in mask");
-  if (t->flags & ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER))
+  if (t->flags &
+      ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED))
     return fail(c, MAD_ERR_INVALID_ARG, "unknown evaluation flags");
   if ((t->mask & MAD_TERM_SPRING) && c->E > 0 && !t->spring_rest)
     return fail(c, MAD_ERR_INVALID_ARG, "spring term active but spring_rest is NULL");
@@ -287,6 +334,7 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     c->n_patches = (int)hp.hdr.size();
     c->nv_max = std::max(1, hp.nv_max);
     c->no_max = std::max(1, hp.no_max);
+    c->slots_max = std::max(1, hp.slots_max);
     // staging room: the largest patch's rows plus a reserve for pair blocks
     if (c->no_max > kMaxPatchOwned) {
       g_create_error = "patch with more owned vertices than threads per block";
@@ -315,7 +363,20 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     CREATE_CK(upload(c, &c->slot_lidx, hp.slot_lidx));
     CREATE_CK(upload(c, &c->slot_eid, hp.slot_eid));
     CREATE_CK(upload(c, &c->runs, hp.runs));
-    CREATE_CK(dev_alloc(c, &c->epart, sizeof(double) * std::max(1, c->n_patches)));
+    CREATE_CK(dev_alloc(c, &c->epart,
+                        sizeof(double) * std::max({1, c->n_patches, rows_blocks(V)})));
+    HostRowTables rt;
+    msg = build_row_tables(V, rp.data(), ci.data(), 8, rt);
+    if (!msg.empty()) {
+      g_create_error = "row tables: " + msg;
+      free_ctx(c);
+      return MAD_ERR_UNIMPLEMENTED;
+    }
+    c->rows_s0 = rt.s0;
+    CREATE_CK(upload(c, &c->rows_slots, rt.slots));
+    CREATE_CK(upload(c, &c->rows_meta, rt.meta));
+    CREATE_CK(upload(c, &c->rows_ofl_ptr, rt.ofl_ptr));
+    CREATE_CK(upload(c, &c->rows_ofl, rt.ofl));
   }
   // 3. shared memory of the patch kernels
   CREATE_CK(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
@@ -339,6 +400,17 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
       return MAD_ERR_UNIMPLEMENTED;
     }
     CREATE_CK(eval_set_smem_limits(dt, dof, std::max(c->smem_eval, c->smem_hvp)));
+    {
+      RowsLaunch R = rows_launch(c);
+      R.rho = c->rho;
+      CREATE_CK(rows_set_smem_limits(dt, dof, rows_smem_bytes(R)));
+    }
+    L.stage_cap = c->stage_base;
+    L.rho = 0;
+    c->grid_base = eval_grid(L);
+    L.stage_cap = c->stage_cap;
+    L.rho = c->rho;
+    c->grid_pairs = eval_grid(L);
   }
   // 4. dynamic CSR double buffer and insertion scratch
   {
@@ -429,8 +501,12 @@ mad_status mad_eval(mad_ctx* c, const void* x, const mad_terms* t, void* g, void
   if (st != MAD_OK) return st;
   if (c->V > 0 && (!x || !g || !H_vals))
     return fail(c, MAD_ERR_INVALID_ARG, "x, g and H_vals must be device pointers");
-  EvalLaunch L = eval_launch(c);
-  cudaError_t e = launch_eval(L, *t, x, g, H_vals, energy, as_stream(stream));
+  cudaError_t e;
+  if (use_rows(t)) {
+    e = launch_rows_eval(rows_launch(c), *t, x, g, H_vals, energy, as_stream(stream));
+  } else {
+    e = launch_eval(eval_launch(c), *t, x, g, H_vals, energy, as_stream(stream));
+  }
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval launch");
   return MAD_OK;
 }
@@ -442,8 +518,8 @@ mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t, const void* v,
   if (st != MAD_OK) return st;
   if (c->V > 0 && (!x || !v || !y))
     return fail(c, MAD_ERR_INVALID_ARG, "x, v and y must be device pointers");
-  EvalLaunch L = eval_launch(c);
-  cudaError_t e = launch_hvp(L, *t, x, v, y, as_stream(stream));
+  cudaError_t e = use_rows(t) ? launch_rows_hvp(rows_launch(c), *t, x, v, y, as_stream(stream))
+                              : launch_hvp(eval_launch(c), *t, x, v, y, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_hvp launch");
   return MAD_OK;
 }

@@ -39,6 +39,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kUnr = 8;  // row slots loaded and evaluated together
+#ifndef MAD_EVAL_MIN_BLOCKS
+#define MAD_EVAL_MIN_BLOCKS 2  // resident blocks per SM the register budget targets
+#endif
 
 template <typename T>
 struct KArgs {
@@ -289,8 +292,10 @@ __device__ __forceinline__ void gather_row_edges(const KArgs<T>& A, const PatchH
 }
 
 // ---------------------------------------------------------------------------
-template <typename T, int DOF, bool FULL>
-__global__ void __launch_bounds__(kThreads) k_eval(const KArgs<T> A) {
+// GENERAL = false: edge terms gathered per row, inertia and pairs only (no
+// colour phases); GENERAL = true adds the scatter-mode edges and face terms.
+template <typename T, int DOF, bool FULL, bool GENERAL>
+__global__ void __launch_bounds__(kThreads, MAD_EVAL_MIN_BLOCKS) k_eval(const KArgs<T> A) {
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
   constexpr int VEC = 16 / (int)sizeof(T);
@@ -305,8 +310,8 @@ __global__ void __launch_bounds__(kThreads) k_eval(const KArgs<T> A) {
   const bool pairs = (A.mask & MAD_TERM_PAIR) && pairs_layout;
   const bool springs = (A.mask & MAD_TERM_SPRING) && hd.ne > 0;
   const bool gather = springs && !(A.flags & MAD_EVAL_EDGE_SCATTER);
-  const bool scatter = springs && !gather;
-  const bool faces = DOF == 2 && (A.mask & MAD_TERM_SYMDIR) && hd.nf > 0;
+  const bool scatter = GENERAL && springs && !gather;
+  const bool faces = GENERAL && DOF == 2 && (A.mask & MAD_TERM_SYMDIR) && hd.nf > 0;
   const bool inertia = A.mask & MAD_TERM_INERTIA;
   // Every off-diagonal mesh block of a row belongs to exactly one edge, so
   // when the gathered springs write a row first they store its blocks and the
@@ -373,7 +378,7 @@ __global__ void __launch_bounds__(kThreads) k_eval(const KArgs<T> A) {
 
   // ---- 2s. colour phases (scatter-mode edges, face terms): accumulators in
   //      shared memory, one colour at a time ----------------------------------
-  if (colour_phases) {
+  if (GENERAL && colour_phases) {
     if (has_row) {
 #pragma unroll
       for (int q = 0; q < TD; ++q) S.dacc[tid * TD + q] = acc[q];
@@ -752,10 +757,16 @@ cudaError_t run_eval(const EvalLaunch& L, const mad_terms& t, const void* x, voi
                      void* H, double* energy, cudaStream_t s) {
   KArgs<T> A = make_args<T>(L, t, x, nullptr, g, H, nullptr, energy != nullptr);
   const size_t smem = eval_smem_bytes(L, false);
-  if (t.flags & MAD_EVAL_FULL_STENCIL_AD)
-    k_eval<T, DOF, true><<<L.n_patches, kThreads, smem, s>>>(A);
+  const bool general = (t.mask & MAD_TERM_SYMDIR) || (t.flags & MAD_EVAL_EDGE_SCATTER);
+  const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
+  if (full && general)
+    k_eval<T, DOF, true, true><<<L.n_patches, kThreads, smem, s>>>(A);
+  else if (full)
+    k_eval<T, DOF, true, false><<<L.n_patches, kThreads, smem, s>>>(A);
+  else if (general)
+    k_eval<T, DOF, false, true><<<L.n_patches, kThreads, smem, s>>>(A);
   else
-    k_eval<T, DOF, false><<<L.n_patches, kThreads, smem, s>>>(A);
+    k_eval<T, DOF, false, false><<<L.n_patches, kThreads, smem, s>>>(A);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum<<<1, 1024, 0, s>>>(L.epart, L.n_patches, energy);
@@ -777,11 +788,17 @@ cudaError_t run_hvp(const EvalLaunch& L, const mad_terms& t, const void* x, cons
 template <typename T, int DOF>
 cudaError_t set_limits(size_t bytes) {
   cudaError_t e;
-  e = cudaFuncSetAttribute(k_eval<T, DOF, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)bytes);
+  e = cudaFuncSetAttribute(k_eval<T, DOF, false, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_eval<T, DOF, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)bytes);
+  e = cudaFuncSetAttribute(k_eval<T, DOF, true, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_eval<T, DOF, false, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_eval<T, DOF, true, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_hvp<T, DOF, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)bytes);
@@ -791,6 +808,8 @@ cudaError_t set_limits(size_t bytes) {
 }
 
 }  // namespace
+
+int eval_grid(const EvalLaunch&) { return 0; }  // one block per patch
 
 size_t patch_stage_elems(const PatchHdr& h, int dof, int esz, int rho) {
   return (size_t)h.no * (size_t)row_stage_elems(h.stride, rho, dof, esz) +

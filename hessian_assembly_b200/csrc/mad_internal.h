@@ -84,6 +84,7 @@ struct HostPatches {
   std::vector<int32_t> slot_eid;
   std::vector<uint32_t> runs;  // first row | row count << 16
   int nv_max = 0, no_max = 0;
+  int slots_max = 0;  // most row slots (owned rows x stride) of one patch
 };
 
 // Host partitioner (partition.cpp).  rp/ci: mesh pattern (host copies).
@@ -92,6 +93,22 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
                           const int32_t* ci, const double* xyz, int xyz_dim,
                           int target_owned, int max_stage_blocks,
                           HostPatches& out);
+
+// Row tables of the row-streaming assembly kernel (rows.cu): warp w owns
+// rows 32w .. 32w+31.  For every row, its off-diagonal mesh-pattern blocks in
+// column order: the column vertex and the id of the edge joining it to the
+// row's vertex.  The first `s0` of them are stored slot-major per tile of 32
+// rows (slot k of row 32t+l at (t*s0 + k)*32 + l, so a warp's loads are
+// coalesced); further ones (rows longer than s0) in an overflow table.
+struct HostRowTables {
+  int s0 = 0;
+  std::vector<int2> slots;        // [ntiles][s0][32] {col, eid}, {-1,-1} empty
+  std::vector<uint32_t> meta;     // [V] off-diagonal count | diagonal position << 16
+  std::vector<int32_t> ofl_ptr;   // [V+1] overflow slots per row (prefix sums)
+  std::vector<int2> ofl;          // overflow slots
+};
+std::string build_row_tables(int V, const int32_t* rp, const int32_t* ci, int s0_cap,
+                             HostRowTables& out);
 
 // ---- dynamic pattern buffers ------------------------------------------
 struct DynBuf {
@@ -126,7 +143,8 @@ std::string build_pattern_gpu(int V, int nF, const int32_t* F_dev,
 
 // eval.cu
 struct EvalLaunch {
-  int dtype, dof, n_patches, nv_max, no_max;
+  int dtype, dof, n_patches, nv_max, no_max, slots_max;
+  int grid;       // persistent blocks of the assembly kernel (0 = one per patch)
   int stage_cap;  // staging capacity in elements of the dtype
   const PatchHdr* hdr;
   const int32_t* vgid;
@@ -149,6 +167,8 @@ struct EvalLaunch {
   double* epart;  // [n_patches]
 };
 size_t eval_smem_bytes(const EvalLaunch& L, bool hvp);
+// persistent grid of the assembly kernel for this launch's shared memory
+int eval_grid(const EvalLaunch& L);
 // staging elements one patch needs with `rho` spare blocks per row
 size_t patch_stage_elems(const PatchHdr& h, int dof, int esz, int rho);
 cudaError_t launch_eval(const EvalLaunch& L, const mad_terms& t, const void* x,
@@ -176,6 +196,28 @@ cudaError_t launch_add_pairs(const PairLaunch& L, int n, const int32_t* ij,
                              const void* rest, const DynBuf& nb,
                              const DynBuf* prev /* nullptr = mesh pattern */,
                              cudaStream_t s);
+
+// rows.cu
+struct RowsLaunch {
+  int dtype, dof, V, s0, rho;
+  const int2* slots;
+  const uint32_t* meta;
+  const int32_t* ofl_ptr;
+  const int2* ofl;
+  const int32_t* rp;  // active row_ptr
+  const int32_t* prow;
+  const int32_t* pe_col;
+  const int32_t* pe_pos;
+  const void* pe_rest;
+  double* epart;  // [rows_blocks(V)]
+};
+int rows_blocks(int V);
+size_t rows_smem_bytes(const RowsLaunch& L);
+cudaError_t rows_set_smem_limits(int dtype, int dof, size_t bytes);
+cudaError_t launch_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
+                             void* H, double* energy, cudaStream_t s);
+cudaError_t launch_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
+                            const void* v, void* y, cudaStream_t s);
 
 // selftest.cu
 cudaError_t selftest_dual(int n, const double* ab_dev, double* out_dev);

@@ -221,6 +221,12 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
 
     PatchHdr H;
     std::memset(&H, 0, sizeof(H));
+    // per-patch arrays start on 16-byte boundaries so the kernel can copy
+    // them to shared memory in 16-byte pieces
+    while (out.vgid.size() % 4 != 0) {
+      out.vgid.push_back(0);
+      out.meta.push_back(make_uint2(0, 0));
+    }
     H.vbeg = (int)out.vgid.size();
     H.nv = nv;
     H.no = no;
@@ -258,6 +264,10 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
     }
     // row slots: column local index + edge id for every mesh-pattern block,
     // each row padded to the stride
+    while (out.slot_lidx.size() % 8 != 0) {
+      out.slot_lidx.push_back(kNoSlot);
+      out.slot_eid.push_back(-1);
+    }
     H.sbeg = (int)out.slot_lidx.size();
     for (int r = 0; r < no; ++r) {
       const int a = owned[r];
@@ -381,6 +391,64 @@ std::string build_patches(int V, int nF, const int32_t* F, const int32_t* rp,
     out.hdr.push_back(H);
     out.nv_max = std::max(out.nv_max, nv);
     out.no_max = std::max(out.no_max, no);
+    out.slots_max = std::max(out.slots_max, no * H.stride);
+  }
+  // slack so that 16-byte copies rounded up past a patch's end stay in bounds
+  for (int i = 0; i < 8; ++i) {
+    out.vgid.push_back(0);
+    out.meta.push_back(make_uint2(0, 0));
+    out.slot_lidx.push_back(kNoSlot);
+    out.slot_eid.push_back(-1);
+  }
+  return "";
+}
+
+std::string build_row_tables(int V, const int32_t* rp, const int32_t* ci, int s0_cap,
+                             HostRowTables& out) {
+  out = HostRowTables();
+  std::vector<int32_t> dpos(V);
+  std::vector<int64_t> eptr(V + 1, 0);
+  int maxoff = 0;
+  for (int v = 0; v < V; ++v) {
+    dpos[v] = find_pos(ci, rp[v], rp[v + 1], v);
+    if (dpos[v] < 0) return "pattern row without diagonal";
+    const int len = rp[v + 1] - rp[v];
+    if (len > 0xFFFF) return "vertex valence too large";
+    maxoff = std::max(maxoff, len - 1);
+    eptr[v + 1] = eptr[v] + (len - dpos[v] - 1);
+  }
+  const int s0 = std::max(1, std::min(maxoff, s0_cap));
+  out.s0 = s0;
+  const int ntiles = (V + 31) / 32;
+  out.slots.assign((size_t)ntiles * s0 * 32, make_int2(-1, -1));
+  out.meta.resize(V);
+  out.ofl_ptr.assign(V + 1, 0);
+  for (int v = 0; v < V; ++v) {
+    const int len = rp[v + 1] - rp[v];
+    out.meta[v] = (uint32_t)(len - 1) | ((uint32_t)dpos[v] << 16);
+    out.ofl_ptr[v + 1] = out.ofl_ptr[v] + std::max(0, len - 1 - s0);
+  }
+  out.ofl.resize(std::max<int32_t>(1, out.ofl_ptr[V]));
+  for (int v = 0; v < V; ++v) {
+    int k = 0;
+    const int t = v / 32, l = v % 32;
+    for (int q = rp[v]; q < rp[v + 1]; ++q) {
+      const int b = ci[q];
+      if (b == v) continue;
+      int32_t eid;
+      if (v < b) {
+        eid = (int32_t)(eptr[v] + (q - rp[v]) - dpos[v] - 1);
+      } else {
+        const int pba = find_pos(ci, rp[b], rp[b + 1], v);
+        eid = (int32_t)(eptr[b] + pba - dpos[b] - 1);
+      }
+      const int2 e = make_int2(b, eid);
+      if (k < s0)
+        out.slots[((size_t)t * s0 + k) * 32 + l] = e;
+      else
+        out.ofl[out.ofl_ptr[v] + (k - s0)] = e;
+      ++k;
+    }
   }
   return "";
 }

@@ -1,0 +1,472 @@
+// rows.cu -- row-streaming assembly: one warp per 32 consecutive Hessian rows,
+// no block-wide barriers.
+//
+// Page "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
+// Computations", section 方法: per-term forward-mode AD in registers (key
+// design 1), assembly g = sum S^T g_j, H = sum S^T H_j S_j into the
+// preallocated CSR (key design 3), runtime pair blocks (key design 4).
+//
+// This kernel is the gather form of that assembly for terms whose stencil is
+// an edge, a vertex or a runtime pair.  Thread = row i (vertex i): it
+// evaluates the inertia term of i and every edge term (i, b) of its row with
+// HyperDual numbers, keeps the diagonal block and the gradient in registers,
+// and writes each off-diagonal block once (each edge term is evaluated once
+// per endpoint).  Rows 32w .. 32w+31 are consecutive in H, so warp w stages
+// them contiguously in its own slice of shared memory, at the same offset
+// modulo 16 bytes as in H, and writes them back with one 1-D bulk (TMA) copy.
+// Neighbour positions are read through the L1/L2 caches.  Warps never wait
+// for each other, so memory latency is hidden across the resident warps.
+// A thread writes only its own row: no zeroing pass, no atomics.
+#include <algorithm>
+
+#include "mad_internal.h"
+#include "terms.cuh"
+
+namespace mad {
+namespace {
+
+constexpr int kRowThreads = 128;  // 4 warps per block
+constexpr int kWarps = kRowThreads / 32;
+constexpr int kS0Max = 8;         // slots read in the first batch
+#ifndef MAD_ROWS_MIN_BLOCKS
+#define MAD_ROWS_MIN_BLOCKS 6  // resident blocks per SM (fp32) the register budget targets
+#endif
+template <typename T>
+constexpr int rows_min_blocks() { return sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3; }
+
+template <typename T>
+struct RArgs {
+  const int2* slots;
+  const uint32_t* meta;
+  const int32_t* ofl_ptr;
+  const int2* ofl;
+  const int32_t* rp;
+  const int32_t* prow;
+  const int32_t* pe_col;
+  const int32_t* pe_pos;
+  const T* pe_rest;
+  const T* x;
+  const T* v;
+  T* g;
+  T* H;
+  T* y;
+  const T* L0;
+  T k;
+  const T* xt;
+  T w;
+  T kp;
+  unsigned mask;
+  double* epart;
+  int V, s0, wstage;  // wstage: staging elements per warp
+};
+
+__device__ __forceinline__ int row_pos(const int32_t* __restrict__ pe_pos, int pb, int pn,
+                                       int nins, int p) {
+  if (nins == 0) return p;
+  for (int e = pb; e < pb + pn; ++e) {
+    const int32_t wv = pe_pos[e];
+    if ((wv & kPairNewBlock) && (wv & kPairPosMask) <= p) ++p;
+  }
+  return p;
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(ssrc);
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(sa), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Per-block energy partial (all threads of the block call it).
+__device__ __forceinline__ void block_energy(double e, double* out) {
+  __shared__ double red[kWarps];
+  e = warp_sum(e);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = e;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < kWarps; ++i) s += red[i];
+    *out = s;
+  }
+}
+
+// Calls on_term(R, p, col) for every edge term (i, col) of row i, where p is
+// the block position of column col in the mesh-pattern row.
+template <typename T, int DOF, bool FULL, typename OnTerm>
+__device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, int lane,
+                                          uint32_t m, const T* xi, OnTerm on_term) {
+  const int noff = (int)(m & 0xFFFFu), dpos = (int)(m >> 16);
+  int2 sl[kS0Max];
+#pragma unroll
+  for (int k = 0; k < kS0Max; ++k) {
+    sl[k] = make_int2(-1, -1);
+    if (k < A.s0) sl[k] = A.slots[((size_t)tile * A.s0 + k) * 32 + lane];
+  }
+  T xb[kS0Max][DOF];
+  T l0[kS0Max];
+#pragma unroll
+  for (int k = 0; k < kS0Max; ++k) {
+    if (sl[k].x < 0) continue;
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xb[k][a] = A.x[(int64_t)sl[k].x * DOF + a];
+    l0[k] = A.L0[sl[k].y];
+  }
+#pragma unroll
+  for (int k = 0; k < kS0Max; ++k) {
+    if (sl[k].x < 0) continue;
+    EdgeRes<T, DOF, FULL> R;
+    eval_edge_res<T, DOF, FULL>(xi, xb[k], l0[k], A.k, R);
+    on_term(R, k < dpos ? k : k + 1, sl[k].x);
+  }
+  if (noff > A.s0) {  // rows longer than the slot table: the overflow slots
+    const int o0 = A.ofl_ptr[i];
+    for (int k = A.s0; k < noff; ++k) {
+      const int2 e = A.ofl[o0 + k - A.s0];
+      T xo[DOF];
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) xo[a] = A.x[(int64_t)e.x * DOF + a];
+      EdgeRes<T, DOF, FULL> R;
+      eval_edge_res<T, DOF, FULL>(xi, xo, A.L0[e.y], A.k, R);
+      on_term(R, k < dpos ? k : k + 1, e.x);
+    }
+  }
+}
+
+template <typename T, int DOF, bool FULL>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval(const RArgs<T> A) {
+  constexpr int B = DOF * DOF;
+  constexpr int TD = Tri<DOF>::size;
+  constexpr int VEC = 16 / (int)sizeof(T);
+  extern __shared__ __align__(16) char smem_raw[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int tile = blockIdx.x * kWarps + wib;
+  const int i = tile * 32 + lane;
+  const bool tile_live = tile * 32 < A.V;
+  const bool has = i < A.V;
+  const bool pairs_layout = A.prow != nullptr;
+  const bool pairs = (A.mask & MAD_TERM_PAIR) && pairs_layout;
+  const bool springs = A.mask & MAD_TERM_SPRING;
+  const bool inertia = A.mask & MAD_TERM_INERTIA;
+  T* stage = (T*)smem_raw + (size_t)wib * A.wstage;
+  double energy = 0.0;
+
+  int d0 = 0, d1 = 0, pb = 0, pn = 0;
+  uint32_t m = 0;
+  T xi[DOF], xti[DOF];
+  if (has) {
+    d0 = A.rp[i];
+    d1 = A.rp[i + 1];
+    m = A.meta[i];
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xi[a] = A.x[(int64_t)i * DOF + a];
+    if (inertia) {
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(int64_t)i * DOF + a];
+    }
+    if (pairs_layout) {
+      pb = A.prow[i];
+      pn = A.prow[i + 1] - pb;
+    }
+  }
+  // the warp's rows are consecutive in H: stage them from the first one
+  const int dfirst = __shfl_sync(0xffffffffu, d0, 0);
+  const int mis = (int)(((uintptr_t)(A.H + (int64_t)dfirst * B) / sizeof(T)) % VEC);
+  const int off = mis + (d0 - dfirst) * B;
+  const bool staged = has && off + (d1 - d0) * B <= A.wstage;
+  T* row = staged ? stage + off : A.H + (int64_t)d0 * B;
+  const int nins = has ? (d1 - d0) - ((int)(m & 0xFFFFu) + 1) : 0;
+
+  T acc[TD], gr[DOF];
+  if (has) {
+    if (pairs_layout)  // blocks inserted by pairs are accumulated into
+      for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
+    if (inertia) {
+      T Ei, Hi[B];
+      eval_inertia<T, DOF>(xi, xti, A.w, Ei, gr, Hi);
+      energy += (double)Ei;
+#pragma unroll
+      for (int a = 0; a < DOF; ++a)
+#pragma unroll
+        for (int b = a; b < DOF; ++b) acc[Tri<DOF>::idx(a, b)] = Hi[a * DOF + b];
+    } else {
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) gr[a] = T(0);
+#pragma unroll
+      for (int q = 0; q < TD; ++q) acc[q] = T(0);
+    }
+    if (springs) {
+      row_edges<T, DOF, FULL>(A, i, tile, lane, m, xi,
+                              [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
+                                const int op = nins == 0 ? p : row_pos(A.pe_pos, pb, pn, nins, p);
+                                apply_edge_side<true>(R, 0, acc, row + op * B, gr);
+                                energy += 0.5 * (double)edge_energy(R);
+                              });
+    } else if (!pairs_layout) {
+      for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
+    }
+    if (pairs) {
+      for (int e = pb; e < pb + pn; ++e) {
+        const int j = A.pe_col[e];
+        const int pos = A.pe_pos[e] & kPairPosMask;
+        T xj[DOF];
+#pragma unroll
+        for (int a = 0; a < DOF; ++a) xj[a] = A.x[(int64_t)j * DOF + a];
+        EdgeRes<T, DOF, FULL> Rp;
+        eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
+        apply_edge_side<false>(Rp, 0, acc, row + pos * B, gr);
+        energy += 0.5 * (double)edge_energy(Rp);
+      }
+    }
+    const int dp = row_pos(A.pe_pos, pb, pn, nins, (int)(m >> 16));
+    T* d = row + dp * B;
+#pragma unroll
+    for (int a = 0; a < DOF; ++a)
+#pragma unroll
+      for (int b = 0; b < DOF; ++b)
+        d[a * DOF + b] = a <= b ? acc[Tri<DOF>::idx(a, b)] : acc[Tri<DOF>::idx(b, a)];
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) A.g[(int64_t)i * DOF + a] = gr[a];
+  }
+  // ---- write-back of the warp's staged rows (a prefix of its 32 rows) -------
+  fence_async_smem();
+  __syncwarp();
+  if (tile_live) {
+    const unsigned st = __ballot_sync(0xffffffffu, staged);
+    if (st) {
+      const int last = 31 - __clz(st);  // staged rows form a prefix
+      const int dend = __shfl_sync(0xffffffffu, d1, last);
+      const int n = (dend - dfirst) * B;
+      T* dst = A.H + (int64_t)dfirst * B;
+      const T* src = stage + mis;
+      const int head = min(n, (VEC - mis) % VEC);
+      const int body = ((n - head) / VEC) * VEC;
+      for (int e = lane; e < head; e += 32) dst[e] = src[e];
+      for (int e = head + body + lane; e < n; e += 32) dst[e] = src[e];
+      const bool aligned = ((((uintptr_t)(dst + head)) | ((uintptr_t)(src + head))) & 15u) == 0;
+      if (body > 0 && !aligned)
+        for (int e = head + lane; e < head + body; e += 32) dst[e] = src[e];
+      if (lane == 0 && body > 0 && aligned) {
+        bulk_store(dst + head, src + head, (uint32_t)(body * sizeof(T)));
+        bulk_commit_and_wait_read();
+      }
+    }
+  }
+  if (A.epart) block_energy(energy, A.epart + blockIdx.x);
+}
+
+template <typename T, int DOF, bool FULL>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(const RArgs<T> A) {
+  constexpr int TD = Tri<DOF>::size;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int tile = blockIdx.x * kWarps + wib;
+  const int i = tile * 32 + lane;
+  if (i >= A.V) return;
+  const bool pairs = (A.mask & MAD_TERM_PAIR) && A.prow != nullptr;
+  T xi[DOF], vi[DOF], yr[DOF];
+#pragma unroll
+  for (int a = 0; a < DOF; ++a) {
+    xi[a] = A.x[(int64_t)i * DOF + a];
+    vi[a] = A.v[(int64_t)i * DOF + a];
+    yr[a] = T(0);
+  }
+  const uint32_t m = A.meta[i];
+  if (A.mask & MAD_TERM_INERTIA) {
+    T xti[DOF], Ei, gi[DOF], Hi[DOF * DOF];
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(int64_t)i * DOF + a];
+    eval_inertia<T, DOF>(xi, xti, A.w, Ei, gi, Hi);
+#pragma unroll
+    for (int a = 0; a < DOF; ++a)
+#pragma unroll
+      for (int b = 0; b < DOF; ++b) yr[a] += Hi[a * DOF + b] * vi[b];
+  }
+  auto hv = [&](const EdgeRes<T, DOF, FULL>& R, const T* vj) {
+    if constexpr (!FULL) {
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) {
+        T s = T(0);
+#pragma unroll
+        for (int b = 0; b < DOF; ++b)
+          s += (a <= b ? R.K[Tri<DOF>::idx(a, b)] : R.K[Tri<DOF>::idx(b, a)]) * (vi[b] - vj[b]);
+        yr[a] += s;
+      }
+    } else {
+#pragma unroll
+      for (int a = 0; a < DOF; ++a)
+#pragma unroll
+        for (int b = 0; b < DOF; ++b)
+          yr[a] += R.d.Haa[a * DOF + b] * vi[b] + R.d.Hab[a * DOF + b] * vj[b];
+    }
+  };
+  if (A.mask & MAD_TERM_SPRING) {
+    row_edges<T, DOF, FULL>(A, i, tile, lane, m, xi,
+                            [&](const EdgeRes<T, DOF, FULL>& R, int, int col) {
+                              T vj[DOF];
+#pragma unroll
+                              for (int a = 0; a < DOF; ++a) vj[a] = A.v[(int64_t)col * DOF + a];
+                              hv(R, vj);
+                            });
+  }
+  if (pairs) {
+    const int pb = A.prow[i], pe = A.prow[i + 1];
+    for (int e = pb; e < pe; ++e) {
+      const int j = A.pe_col[e];
+      T xj[DOF], vj[DOF];
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) {
+        xj[a] = A.x[(int64_t)j * DOF + a];
+        vj[a] = A.v[(int64_t)j * DOF + a];
+      }
+      EdgeRes<T, DOF, FULL> Rp;
+      eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
+      hv(Rp, vj);
+    }
+  }
+  (void)TD;
+#pragma unroll
+  for (int a = 0; a < DOF; ++a) A.y[(int64_t)i * DOF + a] = yr[a];
+}
+
+template <typename T>
+RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
+                    void* g, void* H, void* y, bool energy) {
+  RArgs<T> A;
+  A.slots = L.slots;
+  A.meta = L.meta;
+  A.ofl_ptr = L.ofl_ptr;
+  A.ofl = L.ofl;
+  A.rp = L.rp;
+  A.prow = L.prow;
+  A.pe_col = L.pe_col;
+  A.pe_pos = L.pe_pos;
+  A.pe_rest = (const T*)L.pe_rest;
+  A.x = (const T*)x;
+  A.v = (const T*)v;
+  A.g = (T*)g;
+  A.H = (T*)H;
+  A.y = (T*)y;
+  A.L0 = (const T*)t.spring_rest;
+  A.k = (T)t.spring_k;
+  A.xt = (const T*)t.inertia_xt;
+  A.w = (T)t.inertia_w;
+  A.kp = (T)t.pair_k;
+  A.mask = t.mask;
+  A.epart = energy ? L.epart : nullptr;
+  A.V = L.V;
+  A.s0 = L.s0;
+  const int vec = 16 / (int)sizeof(T);
+  const int rows = 32 * (L.s0 + 1 + L.rho) * L.dof * L.dof;
+  A.wstage = ((rows + vec - 1) / vec) * vec + vec;
+  return A;
+}
+
+__global__ void k_energy_sum_rows(const double* __restrict__ part, int n, double* out) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += part[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    *out = t;
+  }
+}
+
+template <typename T, int DOF>
+cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
+                          void* H, double* energy, cudaStream_t s) {
+  RArgs<T> A = make_rargs<T>(L, t, x, nullptr, g, H, nullptr, energy != nullptr);
+  const int nb = rows_blocks(L.V);
+  const size_t smem = rows_smem_bytes(L);
+  if (t.flags & MAD_EVAL_FULL_STENCIL_AD)
+    k_rows_eval<T, DOF, true><<<nb, kRowThreads, smem, s>>>(A);
+  else
+    k_rows_eval<T, DOF, false><<<nb, kRowThreads, smem, s>>>(A);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !energy) return e;
+  k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
+  return cudaGetLastError();
+}
+
+template <typename T, int DOF>
+cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
+                         void* y, cudaStream_t s) {
+  RArgs<T> A = make_rargs<T>(L, t, x, v, nullptr, nullptr, y, false);
+  const int nb = rows_blocks(L.V);
+  if (t.flags & MAD_EVAL_FULL_STENCIL_AD)
+    k_rows_hvp<T, DOF, true><<<nb, kRowThreads, 0, s>>>(A);
+  else
+    k_rows_hvp<T, DOF, false><<<nb, kRowThreads, 0, s>>>(A);
+  return cudaGetLastError();
+}
+
+template <typename T, int DOF>
+cudaError_t set_rows_limits(size_t bytes) {
+  cudaError_t e = cudaFuncSetAttribute(k_rows_eval<T, DOF, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_rows_eval<T, DOF, true>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+}  // namespace
+
+int rows_blocks(int V) {
+  const int tiles = (V + 31) / 32;
+  return std::max(1, (tiles + kWarps - 1) / kWarps);
+}
+
+size_t rows_smem_bytes(const RowsLaunch& L) {
+  const int esz = L.dtype == MAD_F64 ? 8 : 4;
+  const int vec = 16 / esz;
+  const int rows = 32 * (L.s0 + 1 + L.rho) * L.dof * L.dof;
+  const int wstage = ((rows + vec - 1) / vec) * vec + vec;
+  return (size_t)kWarps * wstage * esz;
+}
+
+cudaError_t rows_set_smem_limits(int dtype, int dof, size_t bytes) {
+  if (dtype == MAD_F64)
+    return dof == 2 ? set_rows_limits<double, 2>(bytes) : set_rows_limits<double, 3>(bytes);
+  return dof == 2 ? set_rows_limits<float, 2>(bytes) : set_rows_limits<float, 3>(bytes);
+}
+
+cudaError_t launch_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
+                             void* H, double* energy, cudaStream_t s) {
+  if (L.V == 0) {
+    if (energy) return cudaMemsetAsync(energy, 0, sizeof(double), s);
+    return cudaSuccess;
+  }
+  if (L.dtype == MAD_F64)
+    return L.dof == 2 ? run_rows_eval<double, 2>(L, t, x, g, H, energy, s)
+                      : run_rows_eval<double, 3>(L, t, x, g, H, energy, s);
+  return L.dof == 2 ? run_rows_eval<float, 2>(L, t, x, g, H, energy, s)
+                    : run_rows_eval<float, 3>(L, t, x, g, H, energy, s);
+}
+
+cudaError_t launch_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
+                            const void* v, void* y, cudaStream_t s) {
+  if (L.V == 0) return cudaSuccess;
+  if (L.dtype == MAD_F64)
+    return L.dof == 2 ? run_rows_hvp<double, 2>(L, t, x, v, y, s)
+                      : run_rows_hvp<double, 3>(L, t, x, v, y, s);
+  return L.dof == 2 ? run_rows_hvp<float, 2>(L, t, x, v, y, s)
+                    : run_rows_hvp<float, 3>(L, t, x, v, y, s);
+}
+
+}  // namespace mad

@@ -87,7 +87,14 @@ enum {
    * thread that owns a row gathers the derivatives of the row's edge terms
    * (each term evaluated once per owned endpoint).  Same results up to
    * rounding; provided for comparison.                                       */
-  MAD_EVAL_EDGE_SCATTER = 2u
+  MAD_EVAL_EDGE_SCATTER = 2u,
+  /* Use the patch kernel (one CUDA block per patch, positions of the patch's
+   * owned and ribbon vertices staged in shared memory) for terms that the
+   * row-streaming kernel also handles.  Face terms always use the patch
+   * kernel; edge, vertex and pair terms alone default to the row-streaming
+   * kernel (one warp per 32 consecutive rows, no block-wide barriers).
+   * Same results up to rounding.                                            */
+  MAD_EVAL_PATCH_STAGED = 4u
 };
 
 typedef struct {

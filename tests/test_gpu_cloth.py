@@ -16,31 +16,33 @@ pytestmark = pytest.mark.gpu
 
 FULL = 1  # MAD_EVAL_FULL_STENCIL_AD
 SCAT = 2  # MAD_EVAL_EDGE_SCATTER
+PATCH = 4  # MAD_EVAL_PATCH_STAGED
 
 
-@pytest.mark.parametrize("flags", [0, FULL, SCAT, FULL | SCAT])
+@pytest.mark.parametrize("flags", [0, FULL, SCAT, FULL | SCAT, PATCH, PATCH | FULL])
 @pytest.mark.parametrize("part", ["rcb", "bfs"])
 def test_cloth_10x10(orc, flags, part):
     check_cloth(orc, 10, "float32", flags=flags, part=part, seed=1001)
 
 
 @pytest.mark.parametrize("dtype", ["float32", "float64"])
-@pytest.mark.parametrize("flags", [0, FULL, SCAT])
+@pytest.mark.parametrize("flags", [0, FULL, SCAT, PATCH])
 def test_cloth_100x100(orc, dtype, flags):
     check_cloth(orc, 100, dtype, flags=flags, seed=1002)
 
 
 @pytest.mark.parametrize("mask", [1, 2])
-@pytest.mark.parametrize("flags", [0, SCAT])
+@pytest.mark.parametrize("flags", [0, SCAT, PATCH])
 def test_single_term_types(orc, mask, flags):
     check_cloth(orc, 23, "float32", mask=mask, flags=flags)
 
 
 @pytest.mark.parametrize("patch_faces", [4, 37, 100000])
-def test_partition_granularity(orc, patch_faces):
+@pytest.mark.parametrize("flags", [0, PATCH])
+def test_partition_granularity(orc, patch_faces, flags):
     # the largest patches (100000 faces asked, capped at 256 owned vertices),
     # tiny patches (4), and an odd size
-    check_cloth(orc, 17, "float64", patch_faces=patch_faces)
+    check_cloth(orc, 17, "float64", patch_faces=patch_faces, flags=flags)
 
 
 def test_cloth_1000x1000_full(orc):
@@ -54,6 +56,10 @@ def test_cloth_1000x1000_second_step_and_full_ad(orc):
 
 def test_cloth_1000x1000_scatter(orc):
     check_cloth(orc, 1000, "float32", seed=1003, step=3, flags=SCAT)
+
+
+def test_cloth_1000x1000_patch_staged(orc):
+    check_cloth(orc, 1000, "float32", seed=1003, step=5, flags=PATCH)
 
 
 def test_permuted_vertex_numbering(orc):

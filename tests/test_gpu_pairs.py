@@ -9,6 +9,7 @@ from _parity import assert_close, check_cloth, cloth_context, cloth_terms, gpu_p
 pytestmark = pytest.mark.gpu
 FULL = 1
 SCAT = 2
+PATCH = 4
 
 
 def add_pairs(ctx, pairs, rest, dtype):
@@ -26,7 +27,7 @@ def pair_case(orc, n, P, dtype="float32", seed=1005, step=0, flags=0, **kw):
                        prest=rest, ctx=ctx, st=st)
 
 
-@pytest.mark.parametrize("flags", [0, FULL, SCAT])
+@pytest.mark.parametrize("flags", [0, FULL, SCAT, PATCH])
 def test_pairs_small(orc, flags):
     pair_case(orc, 30, 60, flags=flags)
 
@@ -35,8 +36,9 @@ def test_pairs_fp64(orc):
     pair_case(orc, 40, 150, "float64")
 
 
-def test_pairs_1000x1000_full(orc):
-    r = pair_case(orc, 1000, 100000)
+@pytest.mark.parametrize("flags", [0, PATCH])
+def test_pairs_1000x1000_full(orc, flags):
+    r = pair_case(orc, 1000, 100000, flags=flags)
     rp, ci, nnzb = gpu_pattern(r["ctx"])
     assert nnzb == 6992002 + 200000
 
@@ -69,9 +71,10 @@ def test_duplicates_edge_coincidence_and_shared_rows(orc):
     check_cloth(orc, n, "float64", mask=11, seed=3, pairs=pairs, prest=rest, ctx=ctx, st=st)
 
 
-def test_many_pairs_on_one_vertex_spill_rows(orc):
+@pytest.mark.parametrize("flags", [0, PATCH])
+def test_many_pairs_on_one_vertex_spill_rows(orc, flags):
     # vertex 0 gains 300 blocks: more than the shared-memory reserve, so its
-    # row is assembled in place in global memory
+    # row (and the rows staged after it) is assembled in place in global memory
     n = 30
     ctx, st = cloth_context(n, "float64")
     x = mi.cloth_x(n, 4, 0, np.float64)
@@ -79,7 +82,8 @@ def test_many_pairs_on_one_vertex_spill_rows(orc):
     pairs = np.stack([np.zeros_like(far), far], 1).astype(np.int32)
     rest = mi.pair_rest(x, pairs, np.float64)
     add_pairs(ctx, pairs, rest, "float64")
-    check_cloth(orc, n, "float64", mask=11, seed=4, pairs=pairs, prest=rest, ctx=ctx, st=st)
+    check_cloth(orc, n, "float64", mask=11, seed=4, pairs=pairs, prest=rest, ctx=ctx, st=st,
+                flags=flags)
 
 
 def test_bad_index_sets_status_and_is_skipped(orc):
