@@ -52,7 +52,7 @@ STATUS_NAMES = {0: "MAD_OK", 1: "MAD_ERR_INVALID_ARG", 2: "MAD_ERR_CUDA", 3: "MA
 # every symbol include/mad.h declares
 EXPORTS = ("mad_default_opts", "mad_create", "mad_info", "mad_edges", "mad_pattern",
            "mad_eval", "mad_hvp", "mad_add_pairs", "mad_status_sync", "mad_eval_host",
-           "mad_last_error", "mad_destroy", "mad_selftest_dual")
+           "mad_last_error", "mad_destroy", "mad_selftest_dual", "mad_energy_noalloc")
 
 
 class mad_opts(ctypes.Structure):
@@ -124,6 +124,9 @@ def load_library(path: str = LIB_PATH):
     lib.mad_destroy.restype = None
     lib.mad_selftest_dual.argtypes = [i32, vp, vp]
     lib.mad_selftest_dual.restype = ctypes.c_int
+    lib.mad_energy_noalloc.argtypes = [i32, i32, ctypes.c_int, vp, ctypes.POINTER(mad_terms), i32,
+                                       vp, i32, vp, i32, vp, vp, vp, vp]
+    lib.mad_energy_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -328,3 +331,23 @@ def mad_selftest_dual(ab: np.ndarray) -> np.ndarray:
     if st != MAD_OK:
         raise MadError(st, lib.mad_last_error(None).decode())
     return out
+
+
+def mad_energy_noalloc(V, dof, x, terms: Terms, energy, *, edges=None, F=None, pairs=None,
+                       pair_rest=None, stream=None) -> int:
+    """Energy of the given terms without a context and without any allocation
+    (see include/mad.h).  Tensors are CUDA tensors; `energy` is a float64 [1]
+    CUDA tensor.  Returns the mad_status code."""
+    torch = _torch()
+    lib = load_library()
+    dt = MAD_F64 if x.dtype == torch.float64 else MAD_F32
+    tc = terms.to_c(x.dtype)
+    n = lambda a: 0 if a is None else int(a.shape[0])  # noqa: E731
+    p = lambda a, d, nm: None if a is None else _dev_ptr(a, d, nm)  # noqa: E731
+    return int(lib.mad_energy_noalloc(int(V), int(dof), dt, _dev_ptr(x, x.dtype, "x"),
+                                      ctypes.byref(tc), n(edges), p(edges, torch.int32, "edges"),
+                                      n(F), p(F, torch.int32, "F"), n(pairs),
+                                      p(pairs, torch.int32, "pairs"),
+                                      p(pair_rest, x.dtype, "pair_rest"),
+                                      _dev_ptr(energy, torch.float64, "energy"),
+                                      _stream_ptr(stream)))

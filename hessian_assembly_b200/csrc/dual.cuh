@@ -190,6 +190,8 @@ __host__ __device__ __forceinline__ float sq(float a) { return a * a; }
 __host__ __device__ __forceinline__ double sq(double a) { return a * a; }
 __host__ __device__ __forceinline__ float inv(float a) { return 1.0f / a; }
 __host__ __device__ __forceinline__ double inv(double a) { return 1.0 / a; }
+__host__ __device__ __forceinline__ float sqrt(float a) { return ::sqrtf(a); }
+__host__ __device__ __forceinline__ double sqrt(double a) { return ::sqrt(a); }
 
 template <typename T, int N>
 __host__ __device__ __forceinline__ HyperDual<T, N> sqrt(const HyperDual<T, N>& a) {

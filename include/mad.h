@@ -238,6 +238,37 @@ const char* mad_last_error(const mad_ctx* c);
 /* Release every resource of the context (synchronises the device first).  */
 void mad_destroy(mad_ctx* c);
 
+/* Total energy of the given terms, for callers that cannot allocate device
+ * memory: code whose device memory is owned by another allocator (a caching
+ * allocator of a host framework that has reserved the GPU), and loops that
+ * must not allocate after their set-up.  Such callers cannot create a
+ * context either (mad_create allocates), so everything is passed in: all
+ * arrays are DEVICE pointers in dtype `dt` (index arrays int32), `t` is a
+ * HOST struct as for mad_eval, and `energy` is a DEVICE double (out).
+ *   springs  nE edges [nE][2] with t->spring_rest [nE] (e.g. mad_edges order)
+ *   inertia  the V vertices with t->inertia_xt [V][dof]
+ *   faces    nF faces F [nF][3] with t->face_Minv, t->face_area (dof 2)
+ *   pairs    nP pairs [nP][2] with pair_rest [nP] and t->pair_k
+ * Only the bits of t->mask select terms; t->flags is ignored.  No paper
+ * counterpart: it is the energy reduction of mad_eval without a context.
+ * Memory: the per-block partial sums live in a fixed device array of this
+ * library (65,536 doubles, held by every device that loads the library until
+ * the process exits); nothing is allocated or freed.  The array is shared by
+ * every call on a device and keeps the last call's values; each call writes
+ * every slot it reads, so nothing needs clearing, but calls that overlap on
+ * the GPU (different streams at once) race.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.
+ * Errors: MAD_ERR_INVALID_ARG (sizes, dtype, missing arrays),
+ * MAD_ERR_UNIMPLEMENTED (faces with dof 3), MAD_ERR_CAPACITY (more than
+ * 16,777,216 terms in total: the fixed array holds 65,536 sums of 256 terms),
+ * MAD_ERR_CUDA.                                                            */
+mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, const void* x,
+                              const mad_terms* t, int32_t nE, const int32_t* edges,
+                              int32_t nF, const int32_t* F, int32_t nP,
+                              const int32_t* pairs, const void* pair_rest,
+                              double* energy, void* stream);
+
 /* Self-test of the forward-mode number types on the device, used by the test
  * suite.  For each of n inputs (a, b) (HOST double [n][2]) it evaluates, in
  * fp64 hyper-dual arithmetic with tangents seeded on (a, b):
