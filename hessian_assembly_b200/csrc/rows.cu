@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kRowThreads = 128;  // 4 warps per block
 constexpr int kWarps = kRowThreads / 32;
-constexpr int kS0Max = 8;         // slots read in the first batch
+constexpr int kS0Max = 8;         // most slots per row in the slot table
 #ifndef MAD_ROWS_MIN_BLOCKS
 #define MAD_ROWS_MIN_BLOCKS 6  // resident blocks per SM (fp32) the register budget targets
 #endif
@@ -105,27 +105,28 @@ __device__ __forceinline__ void block_energy(double e, double* out) {
 
 // Calls on_term(R, p, col) for every edge term (i, col) of row i, where p is
 // the block position of column col in the mesh-pattern row.
-template <typename T, int DOF, bool FULL, typename OnTerm>
+// S0 (compile time) >= the slot table's row width A.s0.
+template <typename T, int DOF, bool FULL, int S0, typename OnTerm>
 __device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, int lane,
                                           uint32_t m, const T* xi, OnTerm on_term) {
   const int noff = (int)(m & 0xFFFFu), dpos = (int)(m >> 16);
-  int2 sl[kS0Max];
+  int2 sl[S0];
 #pragma unroll
-  for (int k = 0; k < kS0Max; ++k) {
+  for (int k = 0; k < S0; ++k) {
     sl[k] = make_int2(-1, -1);
-    if (k < A.s0) sl[k] = A.slots[((size_t)tile * A.s0 + k) * 32 + lane];
+    if (k < A.s0) sl[k] = A.slots[(uint32_t)((tile * A.s0 + k) * 32 + lane)];
   }
-  T xb[kS0Max][DOF];
-  T l0[kS0Max];
+  T xb[S0][DOF];
+  T l0[S0];
 #pragma unroll
-  for (int k = 0; k < kS0Max; ++k) {
+  for (int k = 0; k < S0; ++k) {
     if (sl[k].x < 0) continue;
 #pragma unroll
-    for (int a = 0; a < DOF; ++a) xb[k][a] = A.x[(int64_t)sl[k].x * DOF + a];
+    for (int a = 0; a < DOF; ++a) xb[k][a] = A.x[(uint32_t)(sl[k].x * DOF + a)];
     l0[k] = A.L0[sl[k].y];
   }
 #pragma unroll
-  for (int k = 0; k < kS0Max; ++k) {
+  for (int k = 0; k < S0; ++k) {
     if (sl[k].x < 0) continue;
     EdgeRes<T, DOF, FULL> R;
     eval_edge_res<T, DOF, FULL>(xi, xb[k], l0[k], A.k, R);
@@ -137,7 +138,7 @@ __device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, in
       const int2 e = A.ofl[o0 + k - A.s0];
       T xo[DOF];
 #pragma unroll
-      for (int a = 0; a < DOF; ++a) xo[a] = A.x[(int64_t)e.x * DOF + a];
+      for (int a = 0; a < DOF; ++a) xo[a] = A.x[(uint32_t)(e.x * DOF + a)];
       EdgeRes<T, DOF, FULL> R;
       eval_edge_res<T, DOF, FULL>(xi, xo, A.L0[e.y], A.k, R);
       on_term(R, k < dpos ? k : k + 1, e.x);
@@ -145,10 +146,70 @@ __device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, in
   }
 }
 
-template <typename T, int DOF, bool FULL>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval(const RArgs<T> A) {
+// The work of one row, writing the row's blocks through `row` (a shared-memory
+// staging slot or, for rows that do not fit, the row's place in H).
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+__device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile, int lane,
+                                              uint32_t m, int d0, int d1, int pb, int pn,
+                                              const T* xi, const T* xti, T* row, double& energy) {
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
+  const bool pairs_layout = A.prow != nullptr;
+  const bool pairs = (A.mask & MAD_TERM_PAIR) && pairs_layout;
+  const bool springs = A.mask & MAD_TERM_SPRING;
+  const int nins = (d1 - d0) - ((int)(m & 0xFFFFu) + 1);
+  T acc[TD], gr[DOF];
+  if (pairs_layout || !springs)  // blocks not stored by an edge term start at 0
+    for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
+  if (A.mask & MAD_TERM_INERTIA) {
+    T Ei, Hi[B];
+    eval_inertia<T, DOF>(xi, xti, A.w, Ei, gr, Hi);
+    if (ENERGY) energy += (double)Ei;
+#pragma unroll
+    for (int a = 0; a < DOF; ++a)
+#pragma unroll
+      for (int b = a; b < DOF; ++b) acc[Tri<DOF>::idx(a, b)] = Hi[a * DOF + b];
+  } else {
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) gr[a] = T(0);
+#pragma unroll
+    for (int q = 0; q < TD; ++q) acc[q] = T(0);
+  }
+  if (springs) {
+    row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
+                            [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
+                              const int op = nins == 0 ? p : row_pos(A.pe_pos, pb, pn, nins, p);
+                              apply_edge_side<true>(R, 0, acc, row + op * B, gr);
+                              if (ENERGY) energy += 0.5 * (double)edge_energy(R);
+                            });
+  }
+  if (pairs) {
+    for (int e = pb; e < pb + pn; ++e) {
+      const int j = A.pe_col[e];
+      const int pos = A.pe_pos[e] & kPairPosMask;
+      T xj[DOF];
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) xj[a] = A.x[(uint32_t)(j * DOF + a)];
+      EdgeRes<T, DOF, FULL> Rp;
+      eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
+      apply_edge_side<false>(Rp, 0, acc, row + pos * B, gr);
+      if (ENERGY) energy += 0.5 * (double)edge_energy(Rp);
+    }
+  }
+  const int dp = row_pos(A.pe_pos, pb, pn, nins, (int)(m >> 16));
+  T* d = row + dp * B;
+#pragma unroll
+  for (int a = 0; a < DOF; ++a)
+#pragma unroll
+    for (int b = 0; b < DOF; ++b)
+      d[a * DOF + b] = a <= b ? acc[Tri<DOF>::idx(a, b)] : acc[Tri<DOF>::idx(b, a)];
+#pragma unroll
+  for (int a = 0; a < DOF; ++a) A.g[(uint32_t)(i * DOF + a)] = gr[a];
+}
+
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval(const RArgs<T> A) {
+  constexpr int B = DOF * DOF;
   constexpr int VEC = 16 / (int)sizeof(T);
   extern __shared__ __align__(16) char smem_raw[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -156,11 +217,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval
   const int i = tile * 32 + lane;
   const bool tile_live = tile * 32 < A.V;
   const bool has = i < A.V;
-  const bool pairs_layout = A.prow != nullptr;
-  const bool pairs = (A.mask & MAD_TERM_PAIR) && pairs_layout;
-  const bool springs = A.mask & MAD_TERM_SPRING;
-  const bool inertia = A.mask & MAD_TERM_INERTIA;
-  T* stage = (T*)smem_raw + (size_t)wib * A.wstage;
+  T* stage = (T*)smem_raw + wib * A.wstage;
   double energy = 0.0;
 
   int d0 = 0, d1 = 0, pb = 0, pn = 0;
@@ -171,75 +228,25 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval
     d1 = A.rp[i + 1];
     m = A.meta[i];
 #pragma unroll
-    for (int a = 0; a < DOF; ++a) xi[a] = A.x[(int64_t)i * DOF + a];
-    if (inertia) {
+    for (int a = 0; a < DOF; ++a) xi[a] = A.x[(uint32_t)(i * DOF + a)];
+    if (A.mask & MAD_TERM_INERTIA) {
 #pragma unroll
-      for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(int64_t)i * DOF + a];
+      for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(uint32_t)(i * DOF + a)];
     }
-    if (pairs_layout) {
+    if (A.prow != nullptr) {
       pb = A.prow[i];
       pn = A.prow[i + 1] - pb;
     }
   }
   // the warp's rows are consecutive in H: stage them from the first one
   const int dfirst = __shfl_sync(0xffffffffu, d0, 0);
-  const int mis = (int)(((uintptr_t)(A.H + (int64_t)dfirst * B) / sizeof(T)) % VEC);
+  const int mis = (int)(((uintptr_t)(A.H + (uint32_t)(dfirst * B)) / sizeof(T)) % VEC);
   const int off = mis + (d0 - dfirst) * B;
   const bool staged = has && off + (d1 - d0) * B <= A.wstage;
-  T* row = staged ? stage + off : A.H + (int64_t)d0 * B;
-  const int nins = has ? (d1 - d0) - ((int)(m & 0xFFFFu) + 1) : 0;
-
-  T acc[TD], gr[DOF];
-  if (has) {
-    if (pairs_layout)  // blocks inserted by pairs are accumulated into
-      for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
-    if (inertia) {
-      T Ei, Hi[B];
-      eval_inertia<T, DOF>(xi, xti, A.w, Ei, gr, Hi);
-      energy += (double)Ei;
-#pragma unroll
-      for (int a = 0; a < DOF; ++a)
-#pragma unroll
-        for (int b = a; b < DOF; ++b) acc[Tri<DOF>::idx(a, b)] = Hi[a * DOF + b];
-    } else {
-#pragma unroll
-      for (int a = 0; a < DOF; ++a) gr[a] = T(0);
-#pragma unroll
-      for (int q = 0; q < TD; ++q) acc[q] = T(0);
-    }
-    if (springs) {
-      row_edges<T, DOF, FULL>(A, i, tile, lane, m, xi,
-                              [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
-                                const int op = nins == 0 ? p : row_pos(A.pe_pos, pb, pn, nins, p);
-                                apply_edge_side<true>(R, 0, acc, row + op * B, gr);
-                                energy += 0.5 * (double)edge_energy(R);
-                              });
-    } else if (!pairs_layout) {
-      for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
-    }
-    if (pairs) {
-      for (int e = pb; e < pb + pn; ++e) {
-        const int j = A.pe_col[e];
-        const int pos = A.pe_pos[e] & kPairPosMask;
-        T xj[DOF];
-#pragma unroll
-        for (int a = 0; a < DOF; ++a) xj[a] = A.x[(int64_t)j * DOF + a];
-        EdgeRes<T, DOF, FULL> Rp;
-        eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
-        apply_edge_side<false>(Rp, 0, acc, row + pos * B, gr);
-        energy += 0.5 * (double)edge_energy(Rp);
-      }
-    }
-    const int dp = row_pos(A.pe_pos, pb, pn, nins, (int)(m >> 16));
-    T* d = row + dp * B;
-#pragma unroll
-    for (int a = 0; a < DOF; ++a)
-#pragma unroll
-      for (int b = 0; b < DOF; ++b)
-        d[a * DOF + b] = a <= b ? acc[Tri<DOF>::idx(a, b)] : acc[Tri<DOF>::idx(b, a)];
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) A.g[(int64_t)i * DOF + a] = gr[a];
-  }
+  // rows that do not fit their warp's slice are assembled in place in H
+  if (has)
+    rows_eval_row<T, DOF, FULL, ENERGY, S0>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
+                                        staged ? stage + off : A.H + (uint32_t)(d0 * B), energy);
   // ---- write-back of the warp's staged rows (a prefix of its 32 rows) -------
   fence_async_smem();
   __syncwarp();
@@ -249,7 +256,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval
       const int last = 31 - __clz(st);  // staged rows form a prefix
       const int dend = __shfl_sync(0xffffffffu, d1, last);
       const int n = (dend - dfirst) * B;
-      T* dst = A.H + (int64_t)dfirst * B;
+      T* dst = A.H + (uint32_t)(dfirst * B);
       const T* src = stage + mis;
       const int head = min(n, (VEC - mis) % VEC);
       const int body = ((n - head) / VEC) * VEC;
@@ -264,10 +271,10 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval
       }
     }
   }
-  if (A.epart) block_energy(energy, A.epart + blockIdx.x);
+  if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
 }
 
-template <typename T, int DOF, bool FULL>
+template <typename T, int DOF, bool FULL, int S0>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(const RArgs<T> A) {
   constexpr int TD = Tri<DOF>::size;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -278,15 +285,15 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(
   T xi[DOF], vi[DOF], yr[DOF];
 #pragma unroll
   for (int a = 0; a < DOF; ++a) {
-    xi[a] = A.x[(int64_t)i * DOF + a];
-    vi[a] = A.v[(int64_t)i * DOF + a];
+    xi[a] = A.x[(uint32_t)(i * DOF + a)];
+    vi[a] = A.v[(uint32_t)(i * DOF + a)];
     yr[a] = T(0);
   }
   const uint32_t m = A.meta[i];
   if (A.mask & MAD_TERM_INERTIA) {
     T xti[DOF], Ei, gi[DOF], Hi[DOF * DOF];
 #pragma unroll
-    for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(int64_t)i * DOF + a];
+    for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(uint32_t)(i * DOF + a)];
     eval_inertia<T, DOF>(xi, xti, A.w, Ei, gi, Hi);
 #pragma unroll
     for (int a = 0; a < DOF; ++a)
@@ -312,11 +319,11 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(
     }
   };
   if (A.mask & MAD_TERM_SPRING) {
-    row_edges<T, DOF, FULL>(A, i, tile, lane, m, xi,
+    row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
                             [&](const EdgeRes<T, DOF, FULL>& R, int, int col) {
                               T vj[DOF];
 #pragma unroll
-                              for (int a = 0; a < DOF; ++a) vj[a] = A.v[(int64_t)col * DOF + a];
+                              for (int a = 0; a < DOF; ++a) vj[a] = A.v[(uint32_t)(col * DOF + a)];
                               hv(R, vj);
                             });
   }
@@ -327,8 +334,8 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(
       T xj[DOF], vj[DOF];
 #pragma unroll
       for (int a = 0; a < DOF; ++a) {
-        xj[a] = A.x[(int64_t)j * DOF + a];
-        vj[a] = A.v[(int64_t)j * DOF + a];
+        xj[a] = A.x[(uint32_t)(j * DOF + a)];
+        vj[a] = A.v[(uint32_t)(j * DOF + a)];
       }
       EdgeRes<T, DOF, FULL> Rp;
       eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(
   }
   (void)TD;
 #pragma unroll
-  for (int a = 0; a < DOF; ++a) A.y[(int64_t)i * DOF + a] = yr[a];
+  for (int a = 0; a < DOF; ++a) A.y[(uint32_t)(i * DOF + a)] = yr[a];
 }
 
 template <typename T>
@@ -394,10 +401,28 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   RArgs<T> A = make_rargs<T>(L, t, x, nullptr, g, H, nullptr, energy != nullptr);
   const int nb = rows_blocks(L.V);
   const size_t smem = rows_smem_bytes(L);
-  if (t.flags & MAD_EVAL_FULL_STENCIL_AD)
-    k_rows_eval<T, DOF, true><<<nb, kRowThreads, smem, s>>>(A);
-  else
-    k_rows_eval<T, DOF, false><<<nb, kRowThreads, smem, s>>>(A);
+  const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
+  // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
+  // narrower instantiation: fewer registers
+  if (L.s0 <= 6) {
+    if (full && energy)
+      k_rows_eval<T, DOF, true, true, 6><<<nb, kRowThreads, smem, s>>>(A);
+    else if (full)
+      k_rows_eval<T, DOF, true, false, 6><<<nb, kRowThreads, smem, s>>>(A);
+    else if (energy)
+      k_rows_eval<T, DOF, false, true, 6><<<nb, kRowThreads, smem, s>>>(A);
+    else
+      k_rows_eval<T, DOF, false, false, 6><<<nb, kRowThreads, smem, s>>>(A);
+  } else {
+    if (full && energy)
+      k_rows_eval<T, DOF, true, true, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+    else if (full)
+      k_rows_eval<T, DOF, true, false, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+    else if (energy)
+      k_rows_eval<T, DOF, false, true, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+    else
+      k_rows_eval<T, DOF, false, false, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
@@ -409,20 +434,36 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
                          void* y, cudaStream_t s) {
   RArgs<T> A = make_rargs<T>(L, t, x, v, nullptr, nullptr, y, false);
   const int nb = rows_blocks(L.V);
-  if (t.flags & MAD_EVAL_FULL_STENCIL_AD)
-    k_rows_hvp<T, DOF, true><<<nb, kRowThreads, 0, s>>>(A);
-  else
-    k_rows_hvp<T, DOF, false><<<nb, kRowThreads, 0, s>>>(A);
+  const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
+  if (L.s0 <= 6) {
+    if (full)
+      k_rows_hvp<T, DOF, true, 6><<<nb, kRowThreads, 0, s>>>(A);
+    else
+      k_rows_hvp<T, DOF, false, 6><<<nb, kRowThreads, 0, s>>>(A);
+  } else {
+    if (full)
+      k_rows_hvp<T, DOF, true, kS0Max><<<nb, kRowThreads, 0, s>>>(A);
+    else
+      k_rows_hvp<T, DOF, false, kS0Max><<<nb, kRowThreads, 0, s>>>(A);
+  }
   return cudaGetLastError();
 }
 
 template <typename T, int DOF>
 cudaError_t set_rows_limits(size_t bytes) {
-  cudaError_t e = cudaFuncSetAttribute(k_rows_eval<T, DOF, false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_rows_eval<T, DOF, true>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  const void* ks[8] = {(const void*)k_rows_eval<T, DOF, false, false, 6>,
+                       (const void*)k_rows_eval<T, DOF, false, true, 6>,
+                       (const void*)k_rows_eval<T, DOF, true, false, 6>,
+                       (const void*)k_rows_eval<T, DOF, true, true, 6>,
+                       (const void*)k_rows_eval<T, DOF, false, false, kS0Max>,
+                       (const void*)k_rows_eval<T, DOF, false, true, kS0Max>,
+                       (const void*)k_rows_eval<T, DOF, true, false, kS0Max>,
+                       (const void*)k_rows_eval<T, DOF, true, true, kS0Max>};
+  for (const void* k : ks) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
