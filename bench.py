@@ -263,15 +263,20 @@ def cpu_baseline(st):
             "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
 
 
-def extra_workloads(args):
+EXTRA = ("cloth_small", "symdir500", "pairs1000")
+
+
+def extra_workloads(args, only=None):
     """Secondary workloads (parameterization eval/HVP at 500^2, cloth with 10^5
-    runtime pairs at 1000^2, the small grids), CUDA-event timed, median."""
+    runtime pairs at 1000^2, the small grids), CUDA-event timed, median.
+    `only` names one of EXTRA to run alone."""
     import torch
 
     import hessian_assembly_b200 as mad
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     res = {}
+    run = lambda name: only is None or only == name  # noqa: E731
 
     def timeit(fn, n=50, w=5):
         for _ in range(w):
@@ -287,7 +292,7 @@ def extra_workloads(args):
         return statistics.median([a.elapsed_time(b) for a, b in ts])
 
     # small cloths (launch-latency bound)
-    for n in (10, 100):
+    for n in ((10, 100) if run("cloth_small") else ()):
         st = mi.cloth_static(n, np.float32)
         ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
         terms = mad.Terms(mask=3, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
@@ -298,6 +303,14 @@ def extra_workloads(args):
         res[f"cloth{n}_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
         ctx.close()
     # parameterization 500^2: eval and HVP
+    if run("symdir500"):
+        symdir500(res, mad, torch, dev, stream, timeit)
+    if run("pairs1000"):
+        pairs1000(res, mad, torch, dev, stream)
+    return res
+
+
+def symdir500(res, mad, torch, dev, stream, timeit):
     ps = mi.param_static(500, 1004, np.float32)
     ctx = mad.Context(ps["V"], ps["F"], 2, "float32", part_xyz=ps["X"])
     terms = mad.Terms(mask=4, face_Minv=torch.from_numpy(ps["Minv"].reshape(-1, 4)).to(dev),
@@ -309,8 +322,16 @@ def extra_workloads(args):
     H = torch.empty((ctx.info.capacity_blocks, 2, 2), device=dev)
     res["symdir500_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
     res["symdir500_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
+    # the same term set through the patch-staged kernel, for comparison
+    tp = mad.Terms(mask=4, flags=mad.MAD_EVAL_PATCH_STAGED, face_Minv=terms.face_Minv,
+                   face_area=terms.face_area)
+    res["symdir500_patch_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, tp, g, H, None, stream)), 5)
+    res["symdir500_patch_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, tp, v, y, stream)), 5)
     ctx.close()
-    # cloth 1000^2 + 10^5 fresh pairs per step: insertion, assembly
+
+
+def pairs1000(res, mad, torch, dev, stream):
+    """Cloth 1000^2 + 10^5 fresh pairs per step: insertion, assembly."""
     st = mi.cloth_static(N_GRID, np.float32)
     ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
     terms = mad.Terms(mask=11, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
@@ -343,7 +364,6 @@ def extra_workloads(args):
     res["pairs1000_assembly_ms"] = round(statistics.median([a.elapsed_time(b) for a, b in asm]), 5)
     res["pairs1000_status"] = ctx.mad_status_sync(stream)
     ctx.close()
-    return res
 
 
 # ---------------------------------------------------------------- reference
@@ -398,6 +418,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--ref-sample-n", type=int, default=250)
+    ap.add_argument("--only", choices=EXTRA, default=None,
+                    help="run one secondary workload alone and print its timings")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -406,6 +428,12 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.only:
+        if rank == 0:
+            import torch
+            torch.cuda.init()
+            print(json.dumps({"workloads": extra_workloads(args, args.only)}), flush=True)
         return
     dist = None
     if world > 1:

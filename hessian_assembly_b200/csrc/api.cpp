@@ -53,6 +53,11 @@ struct mad_ctx {
   uint32_t* rows_meta = nullptr;
   int32_t* rows_ofl_ptr = nullptr;
   int2* rows_ofl = nullptr;
+  // face rows of the same kernel (rows_sf == 0: face terms use the patch kernel)
+  int rows_sf = 0;
+  int4* rows_fslots = nullptr;
+  int32_t* rows_fofl_ptr = nullptr;
+  int4* rows_fofl = nullptr;
   double* epart = nullptr;
   size_t smem_eval = 0, smem_hvp = 0;
   // dynamic pattern
@@ -172,6 +177,10 @@ RowsLaunch rows_launch(const mad_ctx* c) {
   L.meta = c->rows_meta;
   L.ofl_ptr = c->rows_ofl_ptr;
   L.ofl = c->rows_ofl;
+  L.sf = c->rows_sf;
+  L.fslots = c->rows_fslots;
+  L.fofl_ptr = c->rows_fofl_ptr;
+  L.fofl = c->rows_fofl;
   L.epart = c->epart;
   if (c->active < 0) {
     L.rp = c->pat.rp;
@@ -190,11 +199,12 @@ RowsLaunch rows_launch(const mad_ctx* c) {
   return L;
 }
 
-// Edge, vertex and pair terms alone go to the row-streaming kernel unless the
-// caller asks for the patch kernel or the scatter mode.
-bool use_rows(const mad_terms* t) {
-  return !(t->mask & MAD_TERM_SYMDIR) &&
-         !(t->flags & (MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED));
+// Every term set goes to the row-streaming kernel unless the caller asks for
+// the patch kernel or the scatter mode, or face terms meet a mesh whose face
+// rows could not be built.
+bool use_rows(const mad_ctx* c, const mad_terms* t) {
+  if (t->flags & (MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED)) return false;
+  return !(t->mask & MAD_TERM_SYMDIR) || c->nF == 0 || c->rows_sf > 0;
 }
 
 mad_status check_terms(mad_ctx* c, const mad_terms* t) {
@@ -377,6 +387,15 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     CREATE_CK(upload(c, &c->rows_meta, rt.meta));
     CREATE_CK(upload(c, &c->rows_ofl_ptr, rt.ofl_ptr));
     CREATE_CK(upload(c, &c->rows_ofl, rt.ofl));
+    if (dof == 2 && nF > 0) {
+      HostFaceRows fr;
+      if (build_face_rows(V, nF, F, rp.data(), ci.data(), fr).empty()) {
+        c->rows_sf = fr.sf;
+        CREATE_CK(upload(c, &c->rows_fslots, fr.slots));
+        CREATE_CK(upload(c, &c->rows_fofl_ptr, fr.ofl_ptr));
+        CREATE_CK(upload(c, &c->rows_fofl, fr.ofl));
+      }
+    }
   }
   // 3. shared memory of the patch kernels
   CREATE_CK(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
@@ -502,7 +521,7 @@ mad_status mad_eval(mad_ctx* c, const void* x, const mad_terms* t, void* g, void
   if (c->V > 0 && (!x || !g || !H_vals))
     return fail(c, MAD_ERR_INVALID_ARG, "x, g and H_vals must be device pointers");
   cudaError_t e;
-  if (use_rows(t)) {
+  if (use_rows(c, t)) {
     e = launch_rows_eval(rows_launch(c), *t, x, g, H_vals, energy, as_stream(stream));
   } else {
     e = launch_eval(eval_launch(c), *t, x, g, H_vals, energy, as_stream(stream));
@@ -518,7 +537,7 @@ mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t, const void* v,
   if (st != MAD_OK) return st;
   if (c->V > 0 && (!x || !v || !y))
     return fail(c, MAD_ERR_INVALID_ARG, "x, v and y must be device pointers");
-  cudaError_t e = use_rows(t) ? launch_rows_hvp(rows_launch(c), *t, x, v, y, as_stream(stream))
+  cudaError_t e = use_rows(c, t) ? launch_rows_hvp(rows_launch(c), *t, x, v, y, as_stream(stream))
                               : launch_hvp(eval_launch(c), *t, x, v, y, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_hvp launch");
   return MAD_OK;

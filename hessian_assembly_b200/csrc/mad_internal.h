@@ -110,6 +110,26 @@ struct HostRowTables {
 std::string build_row_tables(int V, const int32_t* rp, const int32_t* ci, int s0_cap,
                              HostRowTables& out);
 
+// Face rows of the same kernel: for every row i, the faces that have vertex i
+// as a corner, in face order.  Entry {f, j, k, c | pj << 2 | pk << 17}: i is
+// corner c of face f, j and k are corners c+1 and c+2 (mod 3), pj and pk the
+// block positions of columns j and k in row i of the mesh pattern.  The first
+// `sf` entries of a row are stored slot-major per tile of 32 rows, like the
+// edge slots; the rest in an overflow table, and then the row's last slot has
+// the sign bit of k set.  Rows of 32768 blocks or more do
+// not fit the 15-bit positions: the builder then returns an error and the
+// face terms stay on the patch kernel.
+constexpr int kFaceRowSlots = 6;
+constexpr int kFacePosBits = 15;
+struct HostFaceRows {
+  int sf = 0;
+  std::vector<int4> slots;       // [ntiles][sf][32], f = -1 empty
+  std::vector<int32_t> ofl_ptr;  // [V+1]
+  std::vector<int4> ofl;
+};
+std::string build_face_rows(int V, int nF, const int32_t* F, const int32_t* rp,
+                            const int32_t* ci, HostFaceRows& out);
+
 // ---- dynamic pattern buffers ------------------------------------------
 struct DynBuf {
   int32_t* rp = nullptr;      // [V+1]
@@ -200,6 +220,10 @@ cudaError_t launch_add_pairs(const PairLaunch& L, int n, const int32_t* ij,
 // rows.cu
 struct RowsLaunch {
   int dtype, dof, V, s0, rho;
+  int sf;                  // face slots per row (0: no face rows)
+  const int4* fslots;
+  const int32_t* fofl_ptr;
+  const int4* fofl;
   const int2* slots;
   const uint32_t* meta;
   const int32_t* ofl_ptr;

@@ -453,4 +453,44 @@ std::string build_row_tables(int V, const int32_t* rp, const int32_t* ci, int s0
   return "";
 }
 
+std::string build_face_rows(int V, int nF, const int32_t* F, const int32_t* rp,
+                            const int32_t* ci, HostFaceRows& out) {
+  out = HostFaceRows();
+  for (int v = 0; v < V; ++v)
+    if (rp[v + 1] - rp[v] >= (1 << kFacePosBits)) return "row too long for face positions";
+  std::vector<int32_t> cnt(V + 1, 0);
+  for (int64_t f = 0; f < nF; ++f)
+    for (int c = 0; c < 3; ++c) ++cnt[F[3 * f + c] + 1];
+  int maxdeg = 0;
+  for (int v = 0; v < V; ++v) maxdeg = std::max(maxdeg, cnt[v + 1]);
+  const int sf = std::max(1, std::min(maxdeg, kFaceRowSlots));
+  out.sf = sf;
+  const int ntiles = (V + 31) / 32;
+  out.slots.assign((size_t)ntiles * sf * 32, make_int4(-1, -1, -1, 0));
+  out.ofl_ptr.assign(V + 1, 0);
+  for (int v = 0; v < V; ++v) out.ofl_ptr[v + 1] = out.ofl_ptr[v] + std::max(0, cnt[v + 1] - sf);
+  out.ofl.resize(std::max<int32_t>(1, out.ofl_ptr[V]));
+  std::vector<int32_t> fill(V, 0);
+  for (int64_t f = 0; f < nF; ++f) {  // face order within each row
+    for (int c = 0; c < 3; ++c) {
+      const int i = F[3 * f + c], j = F[3 * f + (c + 1) % 3], k = F[3 * f + (c + 2) % 3];
+      const int pj = find_pos(ci, rp[i], rp[i + 1], j);
+      const int pk = find_pos(ci, rp[i], rp[i + 1], k);
+      if (pj < 0 || pk < 0) return "face edge missing from the pattern";
+      const uint32_t w = (uint32_t)c | ((uint32_t)pj << 2) | ((uint32_t)pk << (2 + kFacePosBits));
+      const int s = fill[i]++;
+      // the last slot of a row that continues in the overflow table carries
+      // the sign bit of k
+      const bool more = s == sf - 1 && cnt[i + 1] > sf;
+      const int4 e = make_int4((int32_t)f, j, more ? (int32_t)((uint32_t)k | 0x80000000u) : k,
+                               (int32_t)w);
+      if (s < sf)
+        out.slots[((size_t)(i / 32) * sf + s) * 32 + i % 32] = e;
+      else
+        out.ofl[out.ofl_ptr[i] + (s - sf)] = e;
+    }
+  }
+  return "";
+}
+
 }  // namespace mad

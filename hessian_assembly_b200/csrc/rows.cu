@@ -6,12 +6,12 @@
 // design 1), assembly g = sum S^T g_j, H = sum S^T H_j S_j into the
 // preallocated CSR (key design 3), runtime pair blocks (key design 4).
 //
-// This kernel is the gather form of that assembly for terms whose stencil is
-// an edge, a vertex or a runtime pair.  Thread = row i (vertex i): it
-// evaluates the inertia term of i and every edge term (i, b) of its row with
-// HyperDual numbers, keeps the diagonal block and the gradient in registers,
-// and writes each off-diagonal block once (each edge term is evaluated once
-// per endpoint).  Rows 32w .. 32w+31 are consecutive in H, so warp w stages
+// This kernel is the gather form of that assembly.  Thread = row i (vertex
+// i): it evaluates the inertia term of i, every edge term (i, b) of its row
+// and every face term with i as a corner with HyperDual numbers, keeps the
+// diagonal block and the gradient in registers, and writes each off-diagonal
+// block once.  Each edge term is evaluated once per endpoint and each face
+// term once per corner, for that corner's row only.  Rows 32w .. 32w+31 are consecutive in H, so warp w stages
 // them contiguously in its own slice of shared memory, at the same offset
 // modulo 16 bytes as in H, and writes them back with one 1-D bulk (TMA) copy.
 // Neighbour positions are read through the L1/L2 caches.  Warps never wait
@@ -31,11 +31,18 @@ constexpr int kS0Max = 8;         // most slots per row in the slot table
 #ifndef MAD_ROWS_MIN_BLOCKS
 #define MAD_ROWS_MIN_BLOCKS 6  // resident blocks per SM (fp32) the register budget targets
 #endif
-template <typename T>
-constexpr int rows_min_blocks() { return sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3; }
+template <typename T, bool FACES>
+constexpr int rows_min_blocks() {
+  return FACES ? (sizeof(T) == 4 ? 4 : 2) : (sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3);
+}
 
 template <typename T>
 struct RArgs {
+  const int4* fslots;
+  const int32_t* fofl_ptr;
+  const int4* fofl;
+  const T* Minv;
+  const T* area;
   const int2* slots;
   const uint32_t* meta;
   const int32_t* ofl_ptr;
@@ -57,7 +64,7 @@ struct RArgs {
   T kp;
   unsigned mask;
   double* epart;
-  int V, s0, wstage;  // wstage: staging elements per warp
+  int V, s0, sf, wstage;  // wstage: staging elements per warp
 };
 
 __device__ __forceinline__ int row_pos(const int32_t* __restrict__ pe_pos, int pb, int pn,
@@ -146,9 +153,91 @@ __device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, in
   }
 }
 
+// Four consecutive values starting at p (16-byte loads when p allows them).
+template <typename T>
+__device__ __forceinline__ void load4(const T* __restrict__ p, T* o) {
+  if ((((uintptr_t)p) & 15u) == 0) {
+    if constexpr (sizeof(T) == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(p);
+      o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    } else {
+      const double2 a = reinterpret_cast<const double2*>(p)[0];
+      const double2 b = reinterpret_cast<const double2*>(p)[1];
+      o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o[q] = p[q];
+  }
+}
+
+// Calls on_face(xj, xk, j, k, c, pj, pk, M, area) for every face term with
+// vertex i as a corner (dof 2): j and k are the other two corners (corner
+// c+1 and c+2 of the face when i is corner c), pj and pk their mesh-pattern
+// block positions in row i, M the face's Dm^-1 and area its rest area.  The
+// loop is not unrolled (a small body stays in the instruction cache); the
+// next table entry is loaded while the current face is evaluated.
+template <typename T, typename OnFace>
+__device__ __forceinline__ void row_faces(const RArgs<T>& A, int i, int tile, int lane,
+                                          OnFace on_face) {
+  constexpr uint32_t kPm = (1u << kFacePosBits) - 1u;
+  auto one = [&](const int4& e) {
+    const int j = e.y, k = e.z & 0x7FFFFFFF;
+    const uint32_t w = (uint32_t)e.w;
+    T xj[2], xk[2], M[4];
+    xj[0] = A.x[(uint32_t)(j * 2)];
+    xj[1] = A.x[(uint32_t)(j * 2 + 1)];
+    xk[0] = A.x[(uint32_t)(k * 2)];
+    xk[1] = A.x[(uint32_t)(k * 2 + 1)];
+    load4<T>(A.Minv + (uint32_t)e.x * 4u, M);
+    const T ar = A.area[e.x];
+    on_face(xj, xk, j, k, (int)(w & 3u), (int)((w >> 2) & kPm), (int)(w >> (2 + kFacePosBits)),
+            M, ar);
+  };
+  const int4* p = A.fslots + (uint32_t)(tile * A.sf * 32 + lane);
+  int4 e = p[0];
+  bool more = false;
+#pragma unroll 1
+  for (int k = 0; k < A.sf; ++k) {  // a row's entries fill a prefix of its slots
+    if (e.x < 0) break;
+    const int4 en = k + 1 < A.sf ? p[(uint32_t)((k + 1) * 32)] : make_int4(-1, 0, 0, 0);
+    if (k == kFaceRowSlots - 1) more = e.z < 0;  // the overflow mark
+    one(e);
+    e = en;
+  }
+  if (more) {
+    const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
+#pragma unroll 1
+    for (int q = o0; q < o1; ++q) one(A.fofl[q]);
+  }
+}
+
+// b[0..3] += v[0..3] (16-byte accesses when b allows them)
+template <typename T>
+__device__ __forceinline__ void add4(T* b, const T* v) {
+  if constexpr (sizeof(T) == 4) {
+    if ((((uintptr_t)b) & 15u) == 0) {
+      float4 t = *reinterpret_cast<float4*>(b);
+      t.x += v[0]; t.y += v[1]; t.z += v[2]; t.w += v[3];
+      *reinterpret_cast<float4*>(b) = t;
+      return;
+    }
+  } else {
+    if ((((uintptr_t)b) & 15u) == 0) {
+      double2 t0 = reinterpret_cast<double2*>(b)[0], t1 = reinterpret_cast<double2*>(b)[1];
+      t0.x += v[0]; t0.y += v[1]; t1.x += v[2]; t1.y += v[3];
+      reinterpret_cast<double2*>(b)[0] = t0;
+      reinterpret_cast<double2*>(b)[1] = t1;
+      return;
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) b[q] += v[q];
+}
+
 // The work of one row, writing the row's blocks through `row` (a shared-memory
 // staging slot or, for rows that do not fit, the row's place in H).
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES>
 __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile, int lane,
                                               uint32_t m, int d0, int d1, int pb, int pn,
                                               const T* xi, const T* xti, T* row, double& energy) {
@@ -175,13 +264,34 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
 #pragma unroll
     for (int q = 0; q < TD; ++q) acc[q] = T(0);
   }
-  if (springs) {
-    row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
-                            [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
-                              const int op = nins == 0 ? p : row_pos(A.pe_pos, pb, pn, nins, p);
-                              apply_edge_side<true>(R, 0, acc, row + op * B, gr);
-                              if (ENERGY) energy += 0.5 * (double)edge_energy(R);
-                            });
+  if constexpr (S0 > 0) {  // S0 == 0: an instantiation without edge terms
+    if (springs) {
+      row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
+                              [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
+                                const int op = nins == 0 ? p : row_pos(A.pe_pos, pb, pn, nins, p);
+                                apply_edge_side<true>(R, 0, acc, row + op * B, gr);
+                                if (ENERGY) energy += 0.5 * (double)edge_energy(R);
+                              });
+    }
+  }
+  if constexpr (FACES && DOF == 2) {
+    // after the edge terms, which store their blocks: faces add to them
+    if (A.mask & MAD_TERM_SYMDIR) {
+      row_faces<T>(A, i, tile, lane,
+                   [&](const T* xj, const T* xk, int, int, int c, int pj, int pk, const T* M,
+                       T ar) {
+                     FaceRow<T> o;
+                     eval_symdir_row<T, FULL>(xi, xj, xk, c, M, ar, o);
+                     acc[0] += o.H[0][0];
+                     acc[1] += o.H[0][1];
+                     acc[2] += o.H[0][3];
+                     gr[0] += o.g[0];
+                     gr[1] += o.g[1];
+                     add4<T>(row + row_pos(A.pe_pos, pb, pn, nins, pj) * B, o.H[1]);
+                     add4<T>(row + row_pos(A.pe_pos, pb, pn, nins, pk) * B, o.H[2]);
+                     if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
+                   });
+    }
   }
   if (pairs) {
     for (int e = pb; e < pb + pn; ++e) {
@@ -207,8 +317,8 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   for (int a = 0; a < DOF; ++a) A.g[(uint32_t)(i * DOF + a)] = gr[a];
 }
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval(const RArgs<T> A) {
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_eval(const RArgs<T> A) {
   constexpr int B = DOF * DOF;
   constexpr int VEC = 16 / (int)sizeof(T);
   extern __shared__ __align__(16) char smem_raw[];
@@ -245,7 +355,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval
   const bool staged = has && off + (d1 - d0) * B <= A.wstage;
   // rows that do not fit their warp's slice are assembled in place in H
   if (has)
-    rows_eval_row<T, DOF, FULL, ENERGY, S0>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
+    rows_eval_row<T, DOF, FULL, ENERGY, S0, FACES>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
                                         staged ? stage + off : A.H + (uint32_t)(d0 * B), energy);
   // ---- write-back of the warp's staged rows (a prefix of its 32 rows) -------
   fence_async_smem();
@@ -274,8 +384,8 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_eval
   if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
 }
 
-template <typename T, int DOF, bool FULL, int S0>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(const RArgs<T> A) {
+template <typename T, int DOF, bool FULL, int S0, bool FACES>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_hvp(const RArgs<T> A) {
   constexpr int TD = Tri<DOF>::size;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int tile = blockIdx.x * kWarps + wib;
@@ -318,14 +428,30 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T>()) k_rows_hvp(
           yr[a] += R.d.Haa[a * DOF + b] * vi[b] + R.d.Hab[a * DOF + b] * vj[b];
     }
   };
-  if (A.mask & MAD_TERM_SPRING) {
-    row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
-                            [&](const EdgeRes<T, DOF, FULL>& R, int, int col) {
-                              T vj[DOF];
+  if constexpr (S0 > 0) {
+    if (A.mask & MAD_TERM_SPRING) {
+      row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
+                              [&](const EdgeRes<T, DOF, FULL>& R, int, int col) {
+                                T vj[DOF];
 #pragma unroll
-                              for (int a = 0; a < DOF; ++a) vj[a] = A.v[(uint32_t)(col * DOF + a)];
-                              hv(R, vj);
-                            });
+                                for (int a = 0; a < DOF; ++a) vj[a] = A.v[(uint32_t)(col * DOF + a)];
+                                hv(R, vj);
+                              });
+    }
+  }
+  if constexpr (FACES && DOF == 2) {
+    if (A.mask & MAD_TERM_SYMDIR) {
+      row_faces<T>(A, i, tile, lane,
+                   [&](const T* xj, const T* xk, int j, int k, int c, int, int, const T* M,
+                       T ar) {
+                     T vj[2], vk[2];
+                     vj[0] = A.v[(uint32_t)(j * 2)];
+                     vj[1] = A.v[(uint32_t)(j * 2 + 1)];
+                     vk[0] = A.v[(uint32_t)(k * 2)];
+                     vk[1] = A.v[(uint32_t)(k * 2 + 1)];
+                     hv_symdir_row<T, FULL>(xi, xj, xk, vi, vj, vk, c, M, ar, yr);
+                   });
+    }
   }
   if (pairs) {
     const int pb = A.prow[i], pe = A.prow[i + 1];
@@ -351,6 +477,12 @@ template <typename T>
 RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
                     void* g, void* H, void* y, bool energy) {
   RArgs<T> A;
+  A.fslots = L.fslots;
+  A.fofl_ptr = L.fofl_ptr;
+  A.fofl = L.fofl;
+  A.Minv = (const T*)t.face_Minv;
+  A.area = (const T*)t.face_area;
+  A.sf = L.sf;
   A.slots = L.slots;
   A.meta = L.meta;
   A.ofl_ptr = L.ofl_ptr;
@@ -402,26 +534,52 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   const int nb = rows_blocks(L.V);
   const size_t smem = rows_smem_bytes(L);
   const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
+  if constexpr (DOF == 2) {
+    if (t.mask & MAD_TERM_SYMDIR) {  // face terms: the face-row instantiations
+      // without edge terms the kernel carries no edge-slot code (S0 = 0)
+      const bool sp = t.mask & MAD_TERM_SPRING;
+      if (sp && full && energy)
+        k_rows_eval<T, DOF, true, true, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
+      else if (sp && full)
+        k_rows_eval<T, DOF, true, false, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
+      else if (sp && energy)
+        k_rows_eval<T, DOF, false, true, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
+      else if (sp)
+        k_rows_eval<T, DOF, false, false, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
+      else if (full && energy)
+        k_rows_eval<T, DOF, true, true, 0, true><<<nb, kRowThreads, smem, s>>>(A);
+      else if (full)
+        k_rows_eval<T, DOF, true, false, 0, true><<<nb, kRowThreads, smem, s>>>(A);
+      else if (energy)
+        k_rows_eval<T, DOF, false, true, 0, true><<<nb, kRowThreads, smem, s>>>(A);
+      else
+        k_rows_eval<T, DOF, false, false, 0, true><<<nb, kRowThreads, smem, s>>>(A);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess || !energy) return e;
+      k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
+      return cudaGetLastError();
+    }
+  }
   // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
   // narrower instantiation: fewer registers
   if (L.s0 <= 6) {
     if (full && energy)
-      k_rows_eval<T, DOF, true, true, 6><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, true, true, 6, false><<<nb, kRowThreads, smem, s>>>(A);
     else if (full)
-      k_rows_eval<T, DOF, true, false, 6><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, true, false, 6, false><<<nb, kRowThreads, smem, s>>>(A);
     else if (energy)
-      k_rows_eval<T, DOF, false, true, 6><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, false, true, 6, false><<<nb, kRowThreads, smem, s>>>(A);
     else
-      k_rows_eval<T, DOF, false, false, 6><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, false, false, 6, false><<<nb, kRowThreads, smem, s>>>(A);
   } else {
     if (full && energy)
-      k_rows_eval<T, DOF, true, true, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, true, true, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
     else if (full)
-      k_rows_eval<T, DOF, true, false, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, true, false, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
     else if (energy)
-      k_rows_eval<T, DOF, false, true, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, false, true, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
     else
-      k_rows_eval<T, DOF, false, false, kS0Max><<<nb, kRowThreads, smem, s>>>(A);
+      k_rows_eval<T, DOF, false, false, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !energy) return e;
@@ -435,33 +593,62 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
   RArgs<T> A = make_rargs<T>(L, t, x, v, nullptr, nullptr, y, false);
   const int nb = rows_blocks(L.V);
   const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
+  if constexpr (DOF == 2) {
+    if (t.mask & MAD_TERM_SYMDIR) {
+      const bool sp = t.mask & MAD_TERM_SPRING;
+      if (sp && full)
+        k_rows_hvp<T, DOF, true, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
+      else if (sp)
+        k_rows_hvp<T, DOF, false, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
+      else if (full)
+        k_rows_hvp<T, DOF, true, 0, true><<<nb, kRowThreads, 0, s>>>(A);
+      else
+        k_rows_hvp<T, DOF, false, 0, true><<<nb, kRowThreads, 0, s>>>(A);
+      return cudaGetLastError();
+    }
+  }
   if (L.s0 <= 6) {
     if (full)
-      k_rows_hvp<T, DOF, true, 6><<<nb, kRowThreads, 0, s>>>(A);
+      k_rows_hvp<T, DOF, true, 6, false><<<nb, kRowThreads, 0, s>>>(A);
     else
-      k_rows_hvp<T, DOF, false, 6><<<nb, kRowThreads, 0, s>>>(A);
+      k_rows_hvp<T, DOF, false, 6, false><<<nb, kRowThreads, 0, s>>>(A);
   } else {
     if (full)
-      k_rows_hvp<T, DOF, true, kS0Max><<<nb, kRowThreads, 0, s>>>(A);
+      k_rows_hvp<T, DOF, true, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
     else
-      k_rows_hvp<T, DOF, false, kS0Max><<<nb, kRowThreads, 0, s>>>(A);
+      k_rows_hvp<T, DOF, false, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
   }
   return cudaGetLastError();
 }
 
 template <typename T, int DOF>
 cudaError_t set_rows_limits(size_t bytes) {
-  const void* ks[8] = {(const void*)k_rows_eval<T, DOF, false, false, 6>,
-                       (const void*)k_rows_eval<T, DOF, false, true, 6>,
-                       (const void*)k_rows_eval<T, DOF, true, false, 6>,
-                       (const void*)k_rows_eval<T, DOF, true, true, 6>,
-                       (const void*)k_rows_eval<T, DOF, false, false, kS0Max>,
-                       (const void*)k_rows_eval<T, DOF, false, true, kS0Max>,
-                       (const void*)k_rows_eval<T, DOF, true, false, kS0Max>,
-                       (const void*)k_rows_eval<T, DOF, true, true, kS0Max>};
+  const void* ks[8] = {(const void*)k_rows_eval<T, DOF, false, false, 6, false>,
+                       (const void*)k_rows_eval<T, DOF, false, true, 6, false>,
+                       (const void*)k_rows_eval<T, DOF, true, false, 6, false>,
+                       (const void*)k_rows_eval<T, DOF, true, true, 6, false>,
+                       (const void*)k_rows_eval<T, DOF, false, false, kS0Max, false>,
+                       (const void*)k_rows_eval<T, DOF, false, true, kS0Max, false>,
+                       (const void*)k_rows_eval<T, DOF, true, false, kS0Max, false>,
+                       (const void*)k_rows_eval<T, DOF, true, true, kS0Max, false>};
   for (const void* k : ks) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
+  }
+  if constexpr (DOF == 2) {
+    const void* kf[8] = {(const void*)k_rows_eval<T, DOF, false, false, kS0Max, true>,
+                         (const void*)k_rows_eval<T, DOF, false, true, kS0Max, true>,
+                         (const void*)k_rows_eval<T, DOF, true, false, kS0Max, true>,
+                         (const void*)k_rows_eval<T, DOF, true, true, kS0Max, true>,
+                         (const void*)k_rows_eval<T, DOF, false, false, 0, true>,
+                         (const void*)k_rows_eval<T, DOF, false, true, 0, true>,
+                         (const void*)k_rows_eval<T, DOF, true, false, 0, true>,
+                         (const void*)k_rows_eval<T, DOF, true, true, 0, true>};
+    for (const void* k : kf) {
+      cudaError_t e =
+          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+      if (e != cudaSuccess) return e;
+    }
   }
   return cudaSuccess;
 }

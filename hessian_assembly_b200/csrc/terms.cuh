@@ -42,13 +42,28 @@ __device__ __forceinline__ auto spring_energy(const S (&d)[D], T L0, T k) {
   return sq(r) * (T(0.5) * k);
 }
 
-// j = (J00, J01, J10, J11)
+// s(det) = A (1 + det^-2), the factor that multiplies ||J||_F^2 in the
+// symmetric Dirichlet energy.  For HyperDual inputs it is one chain-rule step
+// with s' = -2 A det^-3 and s'' = 6 A det^-4.
+template <typename T>
+__device__ __forceinline__ T symdir_scale(T det, T A) {
+  const T r = inv(det);
+  return A + A * (r * r);
+}
+template <typename T, int N>
+__device__ __forceinline__ HyperDual<T, N> symdir_scale(const HyperDual<T, N>& det, T A) {
+  const T r = T(1) / det.v;
+  const T Ar2 = A * (r * r);
+  return chain(det, A + Ar2, T(-2) * Ar2 * r, T(6) * Ar2 * (r * r));
+}
+
+// j = (J00, J01, J10, J11): E = ||J||_F^2 (1 + det(J)^-2) A, which equals
+// A (||J||_F^2 + ||J^-1||_F^2) for 2x2 J
 template <typename S, typename T>
 __device__ __forceinline__ auto symdir_energy(const S (&j)[4], T A) {
   auto a = sq(j[0]) + sq(j[1]) + sq(j[2]) + sq(j[3]);
   auto det = j[0] * j[3] - j[1] * j[2];
-  auto id2 = sq(inv(det));
-  return (a + a * id2) * A;
+  return a * symdir_scale(det, A);
 }
 
 // ---------------------------------------------------------------- results
@@ -275,6 +290,156 @@ __device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u
 #pragma unroll
           for (int be = 0; be < 2; ++be)
             o.H[k][l][2 * al + be] = hess(e, 2 * k + al, 2 * l + be);
+  }
+}
+
+// One corner's share of a symmetric Dirichlet face term, for the row of that
+// corner's vertex i: the gradient g_i, the blocks H_ii, H_ij, H_ik (row-major
+// 2x2 each) and the energy.  The face's corners in order are (i, j, k) rotated
+// by c: i is corner c, j corner c+1, k corner c+2 (mod 3).  J is formed from
+// the face's own edge differences in its own corner order, as eval_symdir
+// does, so every corner row sees the same J up to rounding.
+template <typename T>
+struct FaceRow {
+  T E;
+  T g[2];
+  T H[3][4];  // (i,i), (i,j), (i,k)
+};
+
+template <typename T>
+__device__ __forceinline__ T sel3(int c, T a, T b, T d) {
+  return c == 0 ? a : (c == 1 ? b : d);
+}
+
+template <typename T, bool FULL>
+__device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const T* xk, int c,
+                                                const T* M, T A, FaceRow<T>& o) {
+  // corner weights of corners 0, 1, 2; then those of i, j, k
+  const T w[3][2] = {{-(M[0] + M[2]), -(M[1] + M[3])}, {M[0], M[1]}, {M[2], M[3]}};
+  if constexpr (!FULL) {
+    T wr[3][2];
+#pragma unroll
+    for (int ga = 0; ga < 2; ++ga) {
+      wr[0][ga] = sel3(c, w[0][ga], w[1][ga], w[2][ga]);
+      wr[1][ga] = sel3(c, w[1][ga], w[2][ga], w[0][ga]);
+      wr[2][ga] = sel3(c, w[2][ga], w[0][ga], w[1][ga]);
+    }
+    T Jv[4];
+#pragma unroll
+    for (int al = 0; al < 2; ++al) {
+      // corners 0, 1, 2 of the face: c = 0 -> (i, j, k), 1 -> (k, i, j), 2 -> (j, k, i)
+      const T u0 = sel3(c, xi[al], xk[al], xj[al]);
+      const T u1 = sel3(c, xj[al], xi[al], xk[al]);
+      const T u2 = sel3(c, xk[al], xj[al], xi[al]);
+#pragma unroll
+      for (int ga = 0; ga < 2; ++ga) Jv[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
+    }
+    Lin<T, 4> j[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) j[p] = lin_var<T, 4>(Jv[p], p);
+    HyperDual<T, 4> e = symdir_energy(j, A);
+    o.E = e.v;
+#pragma unroll
+    for (int al = 0; al < 2; ++al) o.g[al] = e.g[2 * al] * wr[0][0] + e.g[2 * al + 1] * wr[0][1];
+    // q[al][be][de] = sum_ga H_J[(al,ga),(be,de)] w_i[ga]
+    T q[2][2][2];
+#pragma unroll
+    for (int al = 0; al < 2; ++al)
+#pragma unroll
+      for (int be = 0; be < 2; ++be)
+#pragma unroll
+        for (int de = 0; de < 2; ++de)
+          q[al][be][de] = hess(e, 2 * al + 0, 2 * be + de) * wr[0][0] +
+                          hess(e, 2 * al + 1, 2 * be + de) * wr[0][1];
+#pragma unroll
+    for (int l = 0; l < 3; ++l)
+#pragma unroll
+      for (int al = 0; al < 2; ++al)
+#pragma unroll
+        for (int be = 0; be < 2; ++be)
+          o.H[l][2 * al + be] = q[al][be][0] * wr[l][0] + q[al][be][1] * wr[l][1];
+  } else {
+    // width-6 AD over (x_i, x_j, x_k)
+    Lin<T, 6> ui[2], uj[2], uk[2];
+#pragma unroll
+    for (int al = 0; al < 2; ++al) {
+      ui[al] = lin_var<T, 6>(xi[al], 0 + al);
+      uj[al] = lin_var<T, 6>(xj[al], 2 + al);
+      uk[al] = lin_var<T, 6>(xk[al], 4 + al);
+    }
+    Lin<T, 6> j[4];
+#pragma unroll
+    for (int al = 0; al < 2; ++al) {
+      const Lin<T, 6> u0 = c == 0 ? ui[al] : (c == 1 ? uk[al] : uj[al]);
+      const Lin<T, 6> u1 = c == 0 ? uj[al] : (c == 1 ? ui[al] : uk[al]);
+      const Lin<T, 6> u2 = c == 0 ? uk[al] : (c == 1 ? uj[al] : ui[al]);
+#pragma unroll
+      for (int ga = 0; ga < 2; ++ga) j[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
+    }
+    HyperDual<T, 6> e = symdir_energy(j, A);
+    o.E = e.v;
+    o.g[0] = e.g[0];
+    o.g[1] = e.g[1];
+#pragma unroll
+    for (int l = 0; l < 3; ++l)
+#pragma unroll
+      for (int al = 0; al < 2; ++al)
+#pragma unroll
+        for (int be = 0; be < 2; ++be) o.H[l][2 * al + be] = hess(e, al, 2 * l + be);
+  }
+}
+
+// One corner's share of (H v) for a symmetric Dirichlet face term: adds
+// (H_ii v_i + H_ij v_j + H_ik v_k) to y.  The reduced form contracts in J
+// space: dJ = sum over corners of v_corner w_corner^T, then
+// y += w_i-projection of H_J dJ.
+template <typename T, bool FULL>
+__device__ __forceinline__ void hv_symdir_row(const T* xi, const T* xj, const T* xk,
+                                              const T* vi, const T* vj, const T* vk, int c,
+                                              const T* M, T A, T* y) {
+  if constexpr (!FULL) {
+    T Jv[4], dJ[4];
+#pragma unroll
+    for (int al = 0; al < 2; ++al) {
+      const T u0 = sel3(c, xi[al], xk[al], xj[al]);
+      const T u1 = sel3(c, xj[al], xi[al], xk[al]);
+      const T u2 = sel3(c, xk[al], xj[al], xi[al]);
+      const T v0 = sel3(c, vi[al], vk[al], vj[al]);
+      const T v1 = sel3(c, vj[al], vi[al], vk[al]);
+      const T v2 = sel3(c, vk[al], vj[al], vi[al]);
+#pragma unroll
+      for (int ga = 0; ga < 2; ++ga) {
+        Jv[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
+        dJ[2 * al + ga] = (v1 - v0) * M[ga] + (v2 - v0) * M[2 + ga];
+      }
+    }
+    Lin<T, 4> j[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) j[p] = lin_var<T, 4>(Jv[p], p);
+    HyperDual<T, 4> e = symdir_energy(j, A);
+    T wi[2];
+#pragma unroll
+    for (int ga = 0; ga < 2; ++ga)
+      wi[ga] = sel3(c, -(M[ga] + M[2 + ga]), M[ga], M[2 + ga]);
+#pragma unroll
+    for (int al = 0; al < 2; ++al) {
+      T s = T(0);
+#pragma unroll
+      for (int ga = 0; ga < 2; ++ga) {
+        T t = T(0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) t += hess(e, 2 * al + ga, q) * dJ[q];
+        s += t * wi[ga];
+      }
+      y[al] += s;
+    }
+  } else {
+    FaceRow<T> o;
+    eval_symdir_row<T, true>(xi, xj, xk, c, M, A, o);
+#pragma unroll
+    for (int al = 0; al < 2; ++al)
+      y[al] += o.H[0][2 * al] * vi[0] + o.H[0][2 * al + 1] * vi[1] + o.H[1][2 * al] * vj[0] +
+               o.H[1][2 * al + 1] * vj[1] + o.H[2][2 * al] * vk[0] + o.H[2][2 * al + 1] * vk[1];
   }
 }
 
