@@ -64,8 +64,8 @@ struct mad_ctx {
   DynBuf buf[2];
   int active = -1;  // -1: mesh pattern, no pairs
   // insertion scratch
-  int32_t *cnt = nullptr, *cur = nullptr, *newcnt = nullptr, *shift = nullptr,
-          *pe_pid = nullptr, *scan_tmp = nullptr, *status = nullptr, *flag = nullptr;
+  int32_t *cnt = nullptr, *tsum = nullptr, *newcnt = nullptr, *pe_pid = nullptr,
+          *status = nullptr;
   // mad_eval_host staging (allocated on first use)
   void *hx = nullptr, *hg = nullptr, *hH = nullptr;
   double* he = nullptr;
@@ -456,13 +456,12 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
       b.pe_rest = rest_buf;
     }
     CREATE_CK(dev_alloc(c, &c->cnt, sizeof(int32_t) * (V + 1)));
-    CREATE_CK(dev_alloc(c, &c->cur, sizeof(int32_t) * (V + 1)));
+    CREATE_CK(cudaMemsetAsync(c->cnt, 0, sizeof(int32_t) * (V + 1), s));
+    CREATE_CK(dev_alloc(c, &c->tsum, sizeof(int32_t) * pair_scratch_elems(V)));
+    CREATE_CK(cudaMemsetAsync(c->tsum, 0, sizeof(int32_t) * pair_scratch_elems(V), s));
     CREATE_CK(dev_alloc(c, &c->newcnt, sizeof(int32_t) * (V + 1)));
-    CREATE_CK(dev_alloc(c, &c->shift, sizeof(int32_t) * (V + 1)));
     CREATE_CK(dev_alloc(c, &c->pe_pid, sizeof(int32_t) * pe));
-    CREATE_CK(dev_alloc(c, &c->scan_tmp, sizeof(int32_t) * scan_tmp_elems(V)));
     CREATE_CK(dev_alloc(c, &c->status, sizeof(int32_t)));
-    CREATE_CK(dev_alloc(c, &c->flag, sizeof(int32_t)));
     CREATE_CK(cudaMemsetAsync(c->status, 0, sizeof(int32_t), s));
   }
   c->device_bytes += (int64_t)sizeof(int32_t) *
@@ -563,13 +562,10 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij, const void* r
   L.base_rp = c->pat.rp;
   L.base_ci = c->pat.ci;
   L.cnt = c->cnt;
-  L.cur = c->cur;
+  L.tsum = c->tsum;
   L.newcnt = c->newcnt;
-  L.shift = c->shift;
   L.pe_pid = c->pe_pid;
-  L.scan_tmp = c->scan_tmp;
   L.status = c->status;
-  L.flag = c->flag;
   L.base_nnzb_dev = c->base_nnzb_dev;
   const DynBuf* prev = c->active < 0 ? nullptr : &c->buf[c->active];
   cudaError_t e = launch_add_pairs(L, n, ij, rest, c->buf[next], prev, as_stream(stream));

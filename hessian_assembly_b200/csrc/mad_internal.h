@@ -202,16 +202,16 @@ struct PairLaunch {
   int V, dtype, capacity, nnzb_base, max_pairs;
   const int32_t* base_rp;
   const int32_t* base_ci;
-  int32_t* cnt;     // [V+1]
-  int32_t* cur;     // [V]
-  int32_t* newcnt;  // [V+1]
-  int32_t* shift;   // [V+1]
+  int32_t* cnt;     // [V+1] pair entries per row; zero between calls
+  int32_t* tsum;    // [pair_scratch_elems(V)] per-block and per-tile counts;
+                    // zero at creation
+  int32_t* newcnt;  // [V+1] new blocks per row
   int32_t* pe_pid;  // [2*max_pairs]
-  int32_t* scan_tmp;
   int32_t* status;  // device status word
-  int32_t* flag;    // [1] overflow flag scratch
   const int32_t* base_nnzb_dev;  // [1] block count of the mesh pattern
 };
+// int32 scratch of the insertion kernels (block and tile counts)
+size_t pair_scratch_elems(int V);
 cudaError_t launch_add_pairs(const PairLaunch& L, int n, const int32_t* ij,
                              const void* rest, const DynBuf& nb,
                              const DynBuf* prev /* nullptr = mesh pattern */,

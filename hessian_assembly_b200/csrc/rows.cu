@@ -67,6 +67,42 @@ struct RArgs {
   int V, s0, sf, wstage;  // wstage: staging elements per warp
 };
 
+// New-block positions of a row with inserted pair blocks, in increasing
+// order: the first kRowNew in registers, the rest read from pe_pos.
+constexpr int kRowNew = 4;
+struct RowNew {
+  int np[kRowNew];  // merged-row positions, 0x7FFFFFFF past the row's count
+};
+
+__device__ __forceinline__ void load_row_new(const int32_t* __restrict__ pe_pos, int pb, int pn,
+                                             int nins, RowNew& rn) {
+#pragma unroll
+  for (int k = 0; k < kRowNew; ++k) rn.np[k] = 0x7FFFFFFF;
+  if (nins == 0) return;
+  int k = 0;
+  for (int e = pb; e < pb + pn && k < kRowNew; ++e) {
+    const int32_t wv = pe_pos[e];
+    if (wv & kPairNewBlock) {
+#pragma unroll
+      for (int q = 0; q < kRowNew; ++q)
+        if (q == k) rn.np[q] = wv & kPairPosMask;
+      ++k;
+    }
+  }
+}
+
+__device__ __forceinline__ int row_pos(const int32_t* __restrict__ pe_pos, int pb, int pn,
+                                       int nins, int p);
+
+// Merged-row position of mesh-pattern position p.
+__device__ __forceinline__ int row_pos_new(const RowNew& rn, const int32_t* __restrict__ pe_pos,
+                                           int pb, int pn, int nins, int p) {
+  if (nins > kRowNew) return row_pos(pe_pos, pb, pn, nins, p);
+#pragma unroll
+  for (int k = 0; k < kRowNew; ++k) p += rn.np[k] <= p;
+  return p;
+}
+
 __device__ __forceinline__ int row_pos(const int32_t* __restrict__ pe_pos, int pb, int pn,
                                        int nins, int p) {
   if (nins == 0) return p;
@@ -237,19 +273,53 @@ __device__ __forceinline__ void add4(T* b, const T* v) {
 
 // The work of one row, writing the row's blocks through `row` (a shared-memory
 // staging slot or, for rows that do not fit, the row's place in H).
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES>
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES, bool PAIRS>
 __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile, int lane,
                                               uint32_t m, int d0, int d1, int pb, int pn,
                                               const T* xi, const T* xti, T* row, double& energy) {
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
-  const bool pairs_layout = A.prow != nullptr;
-  const bool pairs = (A.mask & MAD_TERM_PAIR) && pairs_layout;
+  constexpr bool pairs_layout = PAIRS;  // the active pattern has pair blocks
+  const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
   const bool springs = A.mask & MAD_TERM_SPRING;
   const int nins = (d1 - d0) - ((int)(m & 0xFFFFu) + 1);
   T acc[TD], gr[DOF];
-  if (pairs_layout || !springs)  // blocks not stored by an edge term start at 0
+  RowNew rn;
+  if constexpr (PAIRS) load_row_new(A.pe_pos, pb, pn, nins, rn);
+  // The row's first pair entry is loaded before the edge terms are evaluated,
+  // so that its partner's position (a random vertex) arrives meanwhile.
+  int pc0 = 0, pw0 = 0;
+  T pr0 = T(0), xp0[DOF];
+  if (pairs && pn > 0) {
+    pc0 = A.pe_col[pb];
+    pw0 = A.pe_pos[pb];
+    pr0 = A.pe_rest[pb];
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xp0[a] = A.x[(uint32_t)(pc0 * DOF + a)];
+  }
+  // Blocks that no edge term stores start at 0: the whole row without edge
+  // terms, else only the blocks that pairs inserted.
+  if (!springs || S0 == 0) {
     for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
+  } else if (PAIRS && nins > 0) {
+#pragma unroll
+    for (int k = 0; k < kRowNew; ++k)
+      if (k < nins) {
+        T* b = row + rn.np[k] * B;
+#pragma unroll
+        for (int q = 0; q < B; ++q) b[q] = T(0);
+      }
+    if (nins > kRowNew) {
+      for (int e = pb; e < pb + pn; ++e) {
+        const int32_t wv = A.pe_pos[e];
+        if (wv & kPairNewBlock) {
+          T* b = row + (wv & kPairPosMask) * B;
+#pragma unroll
+          for (int q = 0; q < B; ++q) b[q] = T(0);
+        }
+      }
+    }
+  }
   if (A.mask & MAD_TERM_INERTIA) {
     T Ei, Hi[B];
     eval_inertia<T, DOF>(xi, xti, A.w, Ei, gr, Hi);
@@ -268,7 +338,8 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
     if (springs) {
       row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
                               [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
-                                const int op = nins == 0 ? p : row_pos(A.pe_pos, pb, pn, nins, p);
+                                const int op =
+                                    !PAIRS || nins == 0 ? p : row_pos_new(rn, A.pe_pos, pb, pn, nins, p);
                                 apply_edge_side<true>(R, 0, acc, row + op * B, gr);
                                 if (ENERGY) energy += 0.5 * (double)edge_energy(R);
                               });
@@ -287,26 +358,37 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                      acc[2] += o.H[0][3];
                      gr[0] += o.g[0];
                      gr[1] += o.g[1];
-                     add4<T>(row + row_pos(A.pe_pos, pb, pn, nins, pj) * B, o.H[1]);
-                     add4<T>(row + row_pos(A.pe_pos, pb, pn, nins, pk) * B, o.H[2]);
+                     const int oj = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pj) : pj;
+                     const int ok = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pk) : pk;
+                     add4<T>(row + oj * B, o.H[1]);
+                     add4<T>(row + ok * B, o.H[2]);
                      if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
                    });
     }
   }
   if (pairs) {
     for (int e = pb; e < pb + pn; ++e) {
-      const int j = A.pe_col[e];
-      const int pos = A.pe_pos[e] & kPairPosMask;
-      T xj[DOF];
+      int pw;
+      T xj[DOF], rest;
+      if (e == pb) {
+        pw = pw0;
+        rest = pr0;
 #pragma unroll
-      for (int a = 0; a < DOF; ++a) xj[a] = A.x[(uint32_t)(j * DOF + a)];
+        for (int a = 0; a < DOF; ++a) xj[a] = xp0[a];
+      } else {
+        const int j = A.pe_col[e];
+        pw = A.pe_pos[e];
+        rest = A.pe_rest[e];
+#pragma unroll
+        for (int a = 0; a < DOF; ++a) xj[a] = A.x[(uint32_t)(j * DOF + a)];
+      }
       EdgeRes<T, DOF, FULL> Rp;
-      eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
-      apply_edge_side<false>(Rp, 0, acc, row + pos * B, gr);
+      eval_edge_res<T, DOF, FULL>(xi, xj, rest, A.kp, Rp);
+      apply_edge_side<false>(Rp, 0, acc, row + (pw & kPairPosMask) * B, gr);
       if (ENERGY) energy += 0.5 * (double)edge_energy(Rp);
     }
   }
-  const int dp = row_pos(A.pe_pos, pb, pn, nins, (int)(m >> 16));
+  const int dp = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, (int)(m >> 16)) : (int)(m >> 16);
   T* d = row + dp * B;
 #pragma unroll
   for (int a = 0; a < DOF; ++a)
@@ -317,7 +399,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   for (int a = 0; a < DOF; ++a) A.g[(uint32_t)(i * DOF + a)] = gr[a];
 }
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES>
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES, bool PAIRS>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_eval(const RArgs<T> A) {
   constexpr int B = DOF * DOF;
   constexpr int VEC = 16 / (int)sizeof(T);
@@ -343,7 +425,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
 #pragma unroll
       for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(uint32_t)(i * DOF + a)];
     }
-    if (A.prow != nullptr) {
+    if constexpr (PAIRS) {
       pb = A.prow[i];
       pn = A.prow[i + 1] - pb;
     }
@@ -355,7 +437,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   const bool staged = has && off + (d1 - d0) * B <= A.wstage;
   // rows that do not fit their warp's slice are assembled in place in H
   if (has)
-    rows_eval_row<T, DOF, FULL, ENERGY, S0, FACES>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
+    rows_eval_row<T, DOF, FULL, ENERGY, S0, FACES, PAIRS>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
                                         staged ? stage + off : A.H + (uint32_t)(d0 * B), energy);
   // ---- write-back of the warp's staged rows (a prefix of its 32 rows) -------
   fence_async_smem();
@@ -527,6 +609,43 @@ __global__ void k_energy_sum_rows(const double* __restrict__ part, int n, double
   }
 }
 
+// One instantiation of the assembly kernel, chosen by whether the active
+// pattern holds pair blocks; also sets (or, with set, only sets) its shared
+// memory limit.
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES>
+cudaError_t eval_k(const RArgs<T>& A, bool pairs, int nb, size_t smem, cudaStream_t s,
+                   bool set = false) {
+  const void* kp = (const void*)k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, true>;
+  const void* kn = (const void*)k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, false>;
+  if (set) {
+    cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  }
+  if (pairs)
+    k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, true><<<nb, kRowThreads, smem, s>>>(A);
+  else
+    k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, false><<<nb, kRowThreads, smem, s>>>(A);
+  return cudaGetLastError();
+}
+
+// Every (FULL, ENERGY) instantiation for one S0 and FACES.
+template <typename T, int DOF, int S0, bool FACES>
+cudaError_t eval_k4(const RArgs<T>& A, bool full, bool energy, bool pairs, int nb, size_t smem,
+                    cudaStream_t s, bool set = false) {
+  if (set) {
+    cudaError_t e;
+    if ((e = eval_k<T, DOF, true, true, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
+    if ((e = eval_k<T, DOF, true, false, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
+    if ((e = eval_k<T, DOF, false, true, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
+    return eval_k<T, DOF, false, false, S0, FACES>(A, pairs, nb, smem, s, true);
+  }
+  if (full && energy) return eval_k<T, DOF, true, true, S0, FACES>(A, pairs, nb, smem, s);
+  if (full) return eval_k<T, DOF, true, false, S0, FACES>(A, pairs, nb, smem, s);
+  if (energy) return eval_k<T, DOF, false, true, S0, FACES>(A, pairs, nb, smem, s);
+  return eval_k<T, DOF, false, false, S0, FACES>(A, pairs, nb, smem, s);
+}
+
 template <typename T, int DOF>
 cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
                           void* H, double* energy, cudaStream_t s) {
@@ -534,54 +653,23 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   const int nb = rows_blocks(L.V);
   const size_t smem = rows_smem_bytes(L);
   const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
-  if constexpr (DOF == 2) {
-    if (t.mask & MAD_TERM_SYMDIR) {  // face terms: the face-row instantiations
-      // without edge terms the kernel carries no edge-slot code (S0 = 0)
-      const bool sp = t.mask & MAD_TERM_SPRING;
-      if (sp && full && energy)
-        k_rows_eval<T, DOF, true, true, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
-      else if (sp && full)
-        k_rows_eval<T, DOF, true, false, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
-      else if (sp && energy)
-        k_rows_eval<T, DOF, false, true, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
-      else if (sp)
-        k_rows_eval<T, DOF, false, false, kS0Max, true><<<nb, kRowThreads, smem, s>>>(A);
-      else if (full && energy)
-        k_rows_eval<T, DOF, true, true, 0, true><<<nb, kRowThreads, smem, s>>>(A);
-      else if (full)
-        k_rows_eval<T, DOF, true, false, 0, true><<<nb, kRowThreads, smem, s>>>(A);
-      else if (energy)
-        k_rows_eval<T, DOF, false, true, 0, true><<<nb, kRowThreads, smem, s>>>(A);
-      else
-        k_rows_eval<T, DOF, false, false, 0, true><<<nb, kRowThreads, smem, s>>>(A);
-      cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess || !energy) return e;
-      k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
-      return cudaGetLastError();
-    }
-  }
-  // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
-  // narrower instantiation: fewer registers
-  if (L.s0 <= 6) {
-    if (full && energy)
-      k_rows_eval<T, DOF, true, true, 6, false><<<nb, kRowThreads, smem, s>>>(A);
-    else if (full)
-      k_rows_eval<T, DOF, true, false, 6, false><<<nb, kRowThreads, smem, s>>>(A);
-    else if (energy)
-      k_rows_eval<T, DOF, false, true, 6, false><<<nb, kRowThreads, smem, s>>>(A);
+  const bool pairs = L.prow != nullptr;
+  const bool en = energy != nullptr;
+  cudaError_t e;
+  if (DOF == 2 && (t.mask & MAD_TERM_SYMDIR)) {
+    // face terms: the face-row instantiations; without edge terms the kernel
+    // carries no edge-slot code (S0 = 0)
+    if (t.mask & MAD_TERM_SPRING)
+      e = eval_k4<T, DOF, kS0Max, DOF == 2>(A, full, en, pairs, nb, smem, s);
     else
-      k_rows_eval<T, DOF, false, false, 6, false><<<nb, kRowThreads, smem, s>>>(A);
+      e = eval_k4<T, DOF, 0, DOF == 2>(A, full, en, pairs, nb, smem, s);
+  } else if (L.s0 <= 6) {
+    // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
+    // narrower instantiation: fewer registers
+    e = eval_k4<T, DOF, 6, false>(A, full, en, pairs, nb, smem, s);
   } else {
-    if (full && energy)
-      k_rows_eval<T, DOF, true, true, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
-    else if (full)
-      k_rows_eval<T, DOF, true, false, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
-    else if (energy)
-      k_rows_eval<T, DOF, false, true, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
-    else
-      k_rows_eval<T, DOF, false, false, kS0Max, false><<<nb, kRowThreads, smem, s>>>(A);
+    e = eval_k4<T, DOF, kS0Max, false>(A, full, en, pairs, nb, smem, s);
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
   return cudaGetLastError();
@@ -623,32 +711,19 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
 
 template <typename T, int DOF>
 cudaError_t set_rows_limits(size_t bytes) {
-  const void* ks[8] = {(const void*)k_rows_eval<T, DOF, false, false, 6, false>,
-                       (const void*)k_rows_eval<T, DOF, false, true, 6, false>,
-                       (const void*)k_rows_eval<T, DOF, true, false, 6, false>,
-                       (const void*)k_rows_eval<T, DOF, true, true, 6, false>,
-                       (const void*)k_rows_eval<T, DOF, false, false, kS0Max, false>,
-                       (const void*)k_rows_eval<T, DOF, false, true, kS0Max, false>,
-                       (const void*)k_rows_eval<T, DOF, true, false, kS0Max, false>,
-                       (const void*)k_rows_eval<T, DOF, true, true, kS0Max, false>};
-  for (const void* k : ks) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e != cudaSuccess) return e;
-  }
+  RArgs<T> A{};
+  cudaError_t e;
+  if ((e = eval_k4<T, DOF, 6, false>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+    return e;
+  if ((e = eval_k4<T, DOF, kS0Max, false>(A, false, false, false, 0, bytes, 0, true)) !=
+      cudaSuccess)
+    return e;
   if constexpr (DOF == 2) {
-    const void* kf[8] = {(const void*)k_rows_eval<T, DOF, false, false, kS0Max, true>,
-                         (const void*)k_rows_eval<T, DOF, false, true, kS0Max, true>,
-                         (const void*)k_rows_eval<T, DOF, true, false, kS0Max, true>,
-                         (const void*)k_rows_eval<T, DOF, true, true, kS0Max, true>,
-                         (const void*)k_rows_eval<T, DOF, false, false, 0, true>,
-                         (const void*)k_rows_eval<T, DOF, false, true, 0, true>,
-                         (const void*)k_rows_eval<T, DOF, true, false, 0, true>,
-                         (const void*)k_rows_eval<T, DOF, true, true, 0, true>};
-    for (const void* k : kf) {
-      cudaError_t e =
-          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-      if (e != cudaSuccess) return e;
-    }
+    if ((e = eval_k4<T, DOF, kS0Max, true>(A, false, false, false, 0, bytes, 0, true)) !=
+        cudaSuccess)
+      return e;
+    if ((e = eval_k4<T, DOF, 0, true>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+      return e;
   }
   return cudaSuccess;
 }

@@ -133,3 +133,82 @@ def test_hvp_with_pairs(orc):
     og, oH, oE = orc.eval(st["V"], 3, x, 11, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
                           xt=st["xt"], w=st["w"], pairs=pairs, prest=rest, kp=mi.PAIR_K)
     assert_close("y", y.cpu().numpy(), orc.bsr_mv(st["V"], 3, rp, ci, oH, v), "float64")
+
+
+def test_first_insertion_overflow_restores_mesh_pattern(orc):
+    import hessian_assembly_b200 as mad
+    n = 10
+    ctx, st = cloth_context(n, "float64", slack=0.02, max_pairs=64)
+    x = mi.cloth_x(n, 10, 0, np.float64)
+    p = mi.random_pairs(n, 30, 10, 0)  # 60 new blocks > 12 spare, from the mesh pattern
+    add_pairs(ctx, p, mi.pair_rest(x, p, np.float64), "float64")
+    assert ctx.mad_status_sync() == mad.MAD_ERR_CAPACITY
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(st["V"], st["F"])
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    check_cloth(orc, n, "float64", mask=3, seed=10, ctx=ctx, st=st)
+
+
+@pytest.mark.parametrize("mask", [3, 2 | 8, 1 | 8])
+@pytest.mark.parametrize("flags", [0, PATCH])
+def test_inserted_blocks_with_partial_term_sets(orc, mask, flags):
+    # inserted blocks without pair terms stay zero; without edge terms every
+    # block of a row starts at zero
+    n = 20
+    ctx, st = cloth_context(n, "float64")
+    x = mi.cloth_x(n, 11, 0, np.float64)
+    pairs = mi.random_pairs(n, 50, 11, 0)
+    rest = mi.pair_rest(x, pairs, np.float64)
+    add_pairs(ctx, pairs, rest, "float64")
+    check_cloth(orc, n, "float64", mask=mask, flags=flags, seed=11, pairs=pairs, prest=rest,
+                ctx=ctx, st=st)
+
+
+def test_rows_at_the_register_merge_limits(orc):
+    # vertex 0 gets 8 pair entries (two of them repeated), vertex 1 gets 9:
+    # one row at the limit of the in-register merge, one just past it
+    n = 16
+    ctx, st = cloth_context(n, "float64")
+    x = mi.cloth_x(n, 12, 0, np.float64)
+    far0 = [v for v in range(40, 200) if not mi.grid_adjacent(n, 0, v)][:6]
+    far1 = [v for v in range(60, 240) if not mi.grid_adjacent(n, 1, v) and v not in far0][:9]
+    pairs = [[0, v] for v in far0] + [[far0[0], 0], [0, far0[3]]] + [[1, v] for v in far1]
+    pairs = np.array(pairs, np.int32)
+    rest = np.linspace(0.1, 0.4, len(pairs))
+    add_pairs(ctx, pairs, rest, "float64")
+    assert ctx.mad_status_sync() == 0
+    check_cloth(orc, n, "float64", mask=11, seed=12, pairs=pairs, prest=rest, ctx=ctx, st=st)
+
+
+def test_pairs_on_a_long_mesh_row(orc):
+    """A fan hub whose mesh row (41 blocks) is longer than the columns the
+    register merge holds, with pairs on the hub and between rim vertices."""
+    import hessian_assembly_b200 as mad
+    m = 40
+    ang = 2 * np.pi * np.arange(m) / m
+    X = np.concatenate([[[0.0, 0.0, 0.0]], np.stack([np.cos(ang), np.sin(ang), 0 * ang], 1)])
+    F = np.array([[0, 1 + i, 1 + (i + 1) % m] for i in range(m)], np.int32)
+    V = m + 1
+    ctx = mad.Context(V, F, 3, "float64", part_xyz=X)
+    edges = ctx.mad_edges().cpu().numpy()
+    L0 = np.linalg.norm(X[edges[:, 0]] - X[edges[:, 1]], axis=1)
+    rng = np.random.default_rng(13)
+    x = X + 0.01 * rng.standard_normal(X.shape)
+    xt = X.copy()
+    # hub pairs are all on mesh edges; rim pairs are new blocks
+    pairs = np.array([[0, 5], [0, 17], [3, 9], [3, 25], [9, 3], [30, 10]], np.int32)
+    prest = 0.9 * np.linalg.norm(x[pairs[:, 0]] - x[pairs[:, 1]], axis=1)
+    ctx.mad_add_pairs(to_dev(pairs), to_dev(prest))
+    terms = mad.Terms(mask=11, spring_rest=to_dev(L0), spring_k=10.0, inertia_xt=to_dev(xt),
+                      inertia_w=3.0, pair_k=5.0)
+    g, H, E = run_eval(ctx, x, terms, "float64")
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(V, F, pairs)
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    og, oH, oE = orc.eval(V, 3, x, 11, orp, oci, edges=edges, L0=L0, k=10.0, xt=xt, w=3.0,
+                          pairs=pairs, prest=prest, kp=5.0)
+    assert_close("g", g, og, "float64")
+    assert_close("H", H[:nnzb], oH, "float64")
+    assert ctx.mad_status_sync() == 0
