@@ -159,19 +159,24 @@ __global__ void __launch_bounds__(kB) k_scan_rows(const int32_t* __restrict__ cn
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) prow[V] = off + total;
 }
 
+template <typename T>
 __global__ void __launch_bounds__(kB) k_pair_fill(const int32_t* __restrict__ ij, int n, int V,
                                                   const int32_t* __restrict__ prow,
                                                   int32_t* cnt, int32_t* pe_col,
-                                                  int32_t* pe_pid) {
+                                                  int32_t* pe_pid, T* pe_rest,
+                                                  const T* __restrict__ rest) {
   GRID_STRIDE(p, n) {
     const int32_t i = ij[2 * p], j = ij[2 * p + 1];
     if (!pair_ok(i, j, V)) continue;
+    const T r = rest[p];
     int32_t s = prow[i] + atomicSub(&cnt[i], 1) - 1;
     pe_col[s] = j;
     pe_pid[s] = (int32_t)p;
+    pe_rest[s] = r;
     s = prow[j] + atomicSub(&cnt[j], 1) - 1;
     pe_col[s] = i;
     pe_pid[s] = (int32_t)p;
+    pe_rest[s] = r;
   }
 }
 
@@ -221,9 +226,12 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V,
                                                   int32_t* nblk, int32_t* nsupc) {
   const int64_t v = (int64_t)blockIdx.x * kB + threadIdx.x;
   int kn = 0;
+  // both row pointers at once: the mesh row is loaded in the same round trip
+  // as the pair entries
   const int32_t b = v < V ? prow[v] : 0, e = v < V ? prow[v + 1] : 0;
+  const int32_t r0 = v < V ? base_rp[v] : 0, r1 = v < V ? base_rp[v + 1] : 0;
   if (e > b) {
-    const int32_t r0 = base_rp[v], blen = base_rp[v + 1] - r0;
+    const int32_t blen = r1 - r0;
     const int n = e - b;
     if (n <= kRegEntries && blen <= kRegMesh) {
       int32_t col[kRegEntries], pid[kRegEntries], bc[kRegMesh];
@@ -240,7 +248,7 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V,
 #pragma unroll
       for (int q = 0; q < kRegMesh; ++q) bc[q] = q < blen ? base_ci[r0 + q] : 0x7FFFFFFF;
 #pragma unroll
-      for (int q = 0; q < kRegEntries; ++q) rs[q] = q < n ? rest[pid[q]] : T(0);
+      for (int q = 0; q < kRegEntries; ++q) rs[q] = q < n ? pe_rest[b + q] : T(0);
       // sort by (col, pid): odd-even transposition, n passes
 #pragma unroll
       for (int pass = 0; pass < kRegEntries; ++pass) {
@@ -318,6 +326,15 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
   // the row's own loads first: they do not depend on the counts below
   const int32_t b0 = valid ? base_rp[v] : 0x7FFFFFFF;
   const int32_t nc0 = valid ? newcnt[v] : 0;
+  const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int gend = g * 32 + 32 < nrows ? g * 32 + 32 : nrows;
+  const int32_t z = g * 32 < nrows ? base_rp[R0 + gend] : 0;
+  // the row's pair entries (the new-block count is known only after the scan)
+  int32_t pr0 = 0, pr1 = 0;
+  if (valid && nc0) {
+    pr0 = prow[v];
+    pr1 = prow[v + 1];
+  }
   // total new blocks (capacity check) and the new blocks of earlier blocks
   int2 sums;
   {
@@ -367,11 +384,8 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
   if (valid) rp[v] = b0 + sh;
   if (R0 + nrows == V && r == 0) rp[V] = base_rp[V] + s_shift[kB];
   // one warp per 32 rows
-  const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
   if (g * 32 >= nrows) return;
-  const int gend = g * 32 + 32 < nrows ? g * 32 + 32 : nrows;
   const int32_t a = __shfl_sync(0xffffffffu, b0, 0);
-  const int32_t z = base_rp[R0 + gend];
   const unsigned any_new = __ballot_sync(0xffffffffu, nc != 0);
   if (!any_new) {  // one contiguous shifted run
     const int32_t s0 = __shfl_sync(0xffffffffu, sh, 0);
@@ -385,15 +399,36 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
   for (int k = 0; k < kRegNew; ++k) nw[k] = 0x7FFFFFFF;
   const int32_t o0 = b0 + sh;
   if (valid && nc) {
+    // the first kRegNew entries in one round trip, the rest one by one
+    int32_t w4[kRegNew], c4[kRegNew];
+#pragma unroll
+    for (int m = 0; m < kRegNew; ++m) {
+      w4[m] = 0;
+      c4[m] = 0;
+      if (pr0 + m < pr1) {
+        w4[m] = pe_pos[pr0 + m];
+        c4[m] = pe_col[pr0 + m];
+      }
+    }
     int k = 0;
-    for (int32_t e = prow[v]; e < prow[v + 1]; ++e) {
+#pragma unroll
+    for (int m = 0; m < kRegNew; ++m) {
+      if (w4[m] & kPairNewBlock) {
+        ci[o0 + (w4[m] & kPairPosMask)] = c4[m];
+#pragma unroll
+        for (int q = 0; q < kRegNew; ++q)
+          if (q == k) nw[q] = c4[m];
+        ++k;
+      }
+    }
+    for (int32_t e = pr0 + kRegNew; e < pr1; ++e) {
       const int32_t w = pe_pos[e];
       if (w & kPairNewBlock) {
         const int32_t c = pe_col[e];
         ci[o0 + (w & kPairPosMask)] = c;
 #pragma unroll
-        for (int m = 0; m < kRegNew; ++m)
-          if (m == k) nw[m] = c;
+        for (int q = 0; q < kRegNew; ++q)
+          if (q == k) nw[q] = c;
         ++k;
       }
     }
@@ -405,7 +440,7 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
     for (int k = 0; k < kRegNew; ++k) o += nw[k] < c;
     if (nc > kRegNew) {  // the columns past the registers
       int k = 0;
-      for (int32_t e = prow[v]; e < prow[v + 1]; ++e)
+      for (int32_t e = pr0; e < pr1; ++e)
         if (pe_pos[e] & kPairNewBlock) {
           if (k >= kRegNew && pe_col[e] < c) ++o;
           ++k;
@@ -423,11 +458,36 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
       if (nc == 0) {
         for (int32_t q = b0; q < b1; ++q) map[q - a] = q + sh;
       } else {
-        for (int32_t q = b0; q < b1; ++q) map[q - a] = new_place(q, base_ci[q], q + sh);
+        // the row's columns in one round trip (the first kRegMesh of them)
+        int32_t cr[kRegMesh];
+#pragma unroll
+        for (int k = 0; k < kRegMesh; ++k) cr[k] = b0 + k < b1 ? base_ci[b0 + k] : 0;
+#pragma unroll
+        for (int k = 0; k < kRegMesh; ++k)
+          if (b0 + k < b1) map[b0 + k - a] = new_place(b0 + k, cr[k], b0 + k + sh);
+        for (int32_t q = b0 + kRegMesh; q < b1; ++q)
+          map[q - a] = new_place(q, base_ci[q], q + sh);
       }
     }
     __syncwarp();
-    for (int32_t q = a + lane; q < z; q += 32) ci[map[q - a]] = base_ci[q];
+    // the copy, loads of a batch first
+    constexpr int kBatch = 8;
+    for (int32_t qb = a; qb < z; qb += 32 * kBatch) {
+      int32_t cv[kBatch], dv[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int32_t q = qb + 32 * k + lane;
+        if (q < z) {
+          cv[k] = base_ci[q];
+          dv[k] = map[q - a];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int32_t q = qb + 32 * k + lane;
+        if (q < z) ci[dv[k]] = cv[k];
+      }
+    }
     return;
   }
   // long rows: look up each column's row within the warp
@@ -488,7 +548,8 @@ cudaError_t add_pairs_t(const PairLaunch& L, int n, const int32_t* ij, const voi
   CK(cudaGetLastError());
   k_scan_rows<<<nblocks, kB, 0, s>>>(L.cnt, V, sup_c, blk_c, nb.prow);
   CK(cudaGetLastError());
-  k_pair_fill<<<grid_for(n), kB, 0, s>>>(ij, n, V, nb.prow, L.cnt, nb.pe_col, L.pe_pid);
+  k_pair_fill<T><<<grid_for(n), kB, 0, s>>>(ij, n, V, nb.prow, L.cnt, nb.pe_col, L.pe_pid,
+                                            (T*)nb.pe_rest, (const T*)rest);
   CK(cudaGetLastError());
   k_pair_rows<T><<<nblocks, kB, 0, s>>>(V, nb.prow, L.base_rp, L.base_ci, nb.pe_col,
                                         L.pe_pid, nb.pe_pos, (T*)nb.pe_rest, (const T*)rest,
