@@ -32,14 +32,32 @@ namespace mad {
 // ---------------------------------------------------------------- energies
 // S is the number type of the inputs (plain T, Lin or HyperDual); products
 // of affine inputs become HyperDual, so the results are `auto`.
+// Spring: E = k/2 (|d| - L0)^2 depends on d only through s = d.d, so it is
+// evaluated as the univariate function f(s) = k/2 (sqrt(s) - L0)^2 of the AD
+// number s, with f'(s) = k (l - L0) / (2 l) and f''(s) = k L0 / (4 l^3),
+// l = sqrt(s): one chain-rule step instead of sqrt, square and product steps.
+template <typename T>
+__device__ __forceinline__ T spring_of_s(T s, T L0, T k) {
+  const T r = sqrt(s) - L0;
+  return (T(0.5) * k) * (r * r);
+}
+template <typename T, int N>
+__device__ __forceinline__ HyperDual<T, N> spring_of_s(const HyperDual<T, N>& s, T L0, T k) {
+  const T l = sqrt(s.v);
+  const T il = T(1) / l;
+  const T r = l - L0;
+  const T hk = T(0.5) * k;
+  const T f1 = hk * r * il;
+  const T f2 = (T(0.5) * hk) * L0 * (il * il * il);
+  return chain(s, hk * (r * r), f1, f2);
+}
+
 template <typename S, int D, typename T>
 __device__ __forceinline__ auto spring_energy(const S (&d)[D], T L0, T k) {
   auto s = sq(d[0]);
 #pragma unroll
   for (int a = 1; a < D; ++a) s = s + sq(d[a]);
-  auto l = sqrt(s);
-  auto r = l - L0;
-  return sq(r) * (T(0.5) * k);
+  return spring_of_s(s, L0, k);
 }
 
 // s(det) = A (1 + det^-2), the factor that multiplies ||J||_F^2 in the
