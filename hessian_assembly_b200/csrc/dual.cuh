@@ -192,6 +192,9 @@ __host__ __device__ __forceinline__ float inv(float a) { return 1.0f / a; }
 __host__ __device__ __forceinline__ double inv(double a) { return 1.0 / a; }
 __host__ __device__ __forceinline__ float sqrt(float a) { return ::sqrtf(a); }
 __host__ __device__ __forceinline__ double sqrt(double a) { return ::sqrt(a); }
+// 1/sqrt(a) from the CUDA math library (a few ulp, not correctly rounded)
+__device__ __forceinline__ float rsqrt(float a) { return ::rsqrtf(a); }
+__device__ __forceinline__ double rsqrt(double a) { return ::rsqrt(a); }
 
 template <typename T, int N>
 __host__ __device__ __forceinline__ HyperDual<T, N> sqrt(const HyperDual<T, N>& a) {

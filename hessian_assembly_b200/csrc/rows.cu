@@ -279,7 +279,6 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                                               const T* xi, const T* xti, T* row, double& energy) {
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
-  constexpr bool pairs_layout = PAIRS;  // the active pattern has pair blocks
   const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
   const bool springs = A.mask & MAD_TERM_SPRING;
   const int nins = (d1 - d0) - ((int)(m & 0xFFFFu) + 1);

@@ -43,8 +43,8 @@ __device__ __forceinline__ T spring_of_s(T s, T L0, T k) {
 }
 template <typename T, int N>
 __device__ __forceinline__ HyperDual<T, N> spring_of_s(const HyperDual<T, N>& s, T L0, T k) {
-  const T l = sqrt(s.v);
-  const T il = T(1) / l;
+  const T il = rsqrt(s.v);
+  const T l = s.v * il;
   const T r = l - L0;
   const T hk = T(0.5) * k;
   const T f1 = hk * r * il;
