@@ -32,12 +32,13 @@
 namespace mad {
 namespace {
 
-constexpr int kB = 256;        // rows per block (one per thread)
-constexpr int kSuper = 8;      // blocks per super tile
+constexpr int kB = 256;        // rows per block unit (one per thread)
+constexpr int kSuper = 8;      // block units per super tile
+constexpr int kU = 4;          // block units per block of the row passes (rows per thread)
 constexpr int kRegEntries = 4; // pair entries of a row merged in registers
 constexpr int kRegMesh = 8;    // mesh columns of a row held in registers
 constexpr int kRegNew = 4;     // new columns of a row the write kernel keeps in registers
-constexpr int kMapPerWarp = 512;  // mesh columns of 32 rows the write kernel maps in smem
+constexpr int kMapPerWarp = 256;  // mesh columns of 32 rows the write kernel maps in smem
 
 inline unsigned grid_for(int64_t n) {
   int64_t b = (n + kB - 1) / kB;
@@ -88,6 +89,34 @@ __device__ __forceinline__ int2 block_sum2(int a, int b) {
   return s;
 }
 
+// Four sums over the block at once.
+__device__ __forceinline__ int4 block_sum4(int4 v) {
+  __shared__ int4 red4[kB / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+    v.z += __shfl_xor_sync(0xffffffffu, v.z, o);
+    v.w += __shfl_xor_sync(0xffffffffu, v.w, o);
+  }
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red4[threadIdx.x >> 5] = v;
+  __syncthreads();
+  int4 s = make_int4(0, 0, 0, 0);
+#pragma unroll
+  for (int w = 0; w < kB / 32; ++w) {
+    s.x += red4[w].x;
+    s.y += red4[w].y;
+    s.z += red4[w].z;
+    s.w += red4[w].w;
+  }
+  return s;
+}
+
+__device__ __forceinline__ int& lane_of(int4& v, int u) {
+  return u == 0 ? v.x : (u == 1 ? v.y : (u == 2 ? v.z : v.w));
+}
+
 // Exclusive scan of one value per thread over the block; *total = sum.
 __device__ __forceinline__ int block_excl_scan(int v, int* total) {
   __shared__ int ws[kB / 32];
@@ -135,27 +164,67 @@ __global__ void __launch_bounds__(kB) k_pair_count(const int32_t* __restrict__ i
   }
 }
 
+// Entries per block unit (and per super tile): block b covers units
+// kU*b .. kU*b + kU-1, thread t row t of each.
 __global__ void __launch_bounds__(kB) k_block_sums(const int32_t* __restrict__ cnt, int V,
-                                                   int32_t* blk, int32_t* sup) {
-  const int64_t v = (int64_t)blockIdx.x * kB + threadIdx.x;
-  const int s = block_sum(v < V ? cnt[v] : 0);
+                                                   int nunits, int32_t* blk, int32_t* sup) {
+  const int64_t base = (int64_t)blockIdx.x * kU * kB + threadIdx.x;
+  int4 x = make_int4(0, 0, 0, 0);
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int64_t v = base + (int64_t)u * kB;
+    lane_of(x, u) = v < V ? cnt[v] : 0;
+  }
+  int4 sm = block_sum4(x);
   if (threadIdx.x == 0) {
-    blk[blockIdx.x] = s;
-    if (s) atomicAdd(&sup[blockIdx.x / kSuper], s);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int unit = blockIdx.x * kU + u;
+      const int su = lane_of(sm, u);
+      if (unit < nunits) {
+        blk[unit] = su;
+        if (su) atomicAdd(&sup[unit / kSuper], su);
+      }
+    }
   }
 }
 
-// prow[v] = sum of cnt[0 .. v); prow[V] = total.
+// prow[v] = sum of cnt[0 .. v); prow[V] = total.  Block b scans rows
+// [b*kU*kB, (b+1)*kU*kB), thread t rows kU*t .. kU*t + kU-1 of them.
 __global__ void __launch_bounds__(kB) k_scan_rows(const int32_t* __restrict__ cnt, int V,
                                                   const int32_t* __restrict__ sup,
                                                   const int32_t* __restrict__ blk,
                                                   int32_t* __restrict__ prow) {
-  const int off = blocks_before(sup, blk);
-  const int64_t v = (int64_t)blockIdx.x * kB + threadIdx.x;
-  const int c = v < V ? cnt[v] : 0;
+  const int U0 = blockIdx.x * kU, S = U0 / kSuper;
+  const int64_t r0 = (int64_t)blockIdx.x * kU * kB + (int64_t)threadIdx.x * kU;
+  int4 c = make_int4(0, 0, 0, 0);
+  if (r0 + kU <= V) {
+    c = *reinterpret_cast<const int4*>(cnt + r0);  // 16-byte aligned: r0 % 4 == 0
+  } else {
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (r0 + u < V) lane_of(c, u) = cnt[r0 + u];
+  }
+  // counts of every unit before this block: whole super tiles, then the
+  // units of this block's super tile
+  int s = 0;
+  for (int q = threadIdx.x; q < S; q += kB) s += sup[q];
+  if ((int)threadIdx.x < U0 - S * kSuper) s += blk[S * kSuper + threadIdx.x];
+  const int off = block_sum(s);
   int total;
-  const int pre = off + block_excl_scan(c, &total);
-  if (v < V) prow[v] = pre;
+  int pre = off + block_excl_scan(c.x + c.y + c.z + c.w, &total);
+  int4 o;
+  o.x = pre;
+  o.y = o.x + c.x;
+  o.z = o.y + c.y;
+  o.w = o.z + c.z;
+  if (r0 + kU <= V) {
+    *reinterpret_cast<int4*>(prow + r0) = o;
+  } else {
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (r0 + u < V) prow[r0 + u] = lane_of(o, u);
+  }
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) prow[V] = off + total;
 }
 
@@ -214,9 +283,100 @@ __device__ int row_merge_global(int32_t b, int32_t e, const int32_t* __restrict_
   return kn;
 }
 
-// Per row: sort, merge, positions; new blocks per row, block and super tile.
+// Position of the j-th (from 0) set bit of m; j < popc(m).
+__device__ __forceinline__ int nth_set_bit(unsigned m, int j) {
+  int pos = 0;
+#pragma unroll
+  for (int w = 16; w > 0; w >>= 1) {
+    const unsigned low = m & ((1u << w) - 1u);
+    const int c = __popc(low);
+    if (j >= c) {
+      j -= c;
+      m >>= w;
+      pos += w;
+    } else {
+      m = low;
+    }
+  }
+  return pos;
+}
+
+// One row: sort its entries, merge them with the mesh row, positions;
+// returns the row's new blocks.
 template <typename T>
-__global__ void __launch_bounds__(kB) k_pair_rows(int V,
+__device__ __forceinline__ int merge_row(int32_t b, int32_t e, int32_t r0, int32_t r1,
+                                         const int32_t* __restrict__ base_ci, int32_t* pe_col,
+                                         int32_t* pe_pid, int32_t* pe_pos, T* pe_rest,
+                                         const T* __restrict__ rest) {
+  const int32_t blen = r1 - r0;
+  const int n = e - b;
+  if (n > kRegEntries || blen > kRegMesh)
+    return row_merge_global<T>(b, e, base_ci, r0, blen, pe_col, pe_pid, pe_pos, pe_rest, rest);
+  int kn = 0;
+  int32_t col[kRegEntries], pid[kRegEntries], bc[kRegMesh];
+  T rs[kRegEntries];
+#pragma unroll
+  for (int q = 0; q < kRegEntries; ++q) {
+    col[q] = 0x7FFFFFFF;
+    pid[q] = 0x7FFFFFFF;
+    rs[q] = T(0);
+    if (q < n) {
+      col[q] = pe_col[b + q];
+      pid[q] = pe_pid[b + q];
+      rs[q] = pe_rest[b + q];
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kRegMesh; ++q) bc[q] = q < blen ? base_ci[r0 + q] : 0x7FFFFFFF;
+  // sort by (col, pid): odd-even transposition, n passes
+#pragma unroll
+  for (int pass = 0; pass < kRegEntries; ++pass) {
+    if (pass >= n) break;
+#pragma unroll
+    for (int q = pass & 1; q + 1 < kRegEntries; q += 2) {
+      const bool sw = col[q] > col[q + 1] || (col[q] == col[q + 1] && pid[q] > pid[q + 1]);
+      if (sw) {
+        const int32_t tc = col[q], tp = pid[q];
+        const T tr = rs[q];
+        col[q] = col[q + 1]; pid[q] = pid[q + 1]; rs[q] = rs[q + 1];
+        col[q + 1] = tc; pid[q + 1] = tp; rs[q + 1] = tr;
+      }
+    }
+  }
+  // position in the merged row = mesh columns below c + new columns below
+  // c; entries with the same column (repeated pairs) share it
+  int prev_col = -1, kn_group = 0;
+#pragma unroll
+  for (int q = 0; q < kRegEntries; ++q) {
+    if (q < n) {
+      const int c = col[q];
+      int kb = 0;
+      bool in_mesh = false;
+#pragma unroll
+      for (int m = 0; m < kRegMesh; ++m) {
+        kb += bc[m] < c;
+        in_mesh |= bc[m] == c;
+      }
+      const bool first = c != prev_col;
+      const bool fresh = first && !in_mesh;
+      if (first) kn_group = kn;
+      pe_col[b + q] = c;
+      pe_pos[b + q] = (kb + kn_group) | (fresh ? kPairNewBlock : 0);
+      pe_rest[b + q] = rs[q];
+      if (fresh) ++kn;
+      prev_col = c;
+    }
+  }
+  return kn;
+}
+
+// Per row: merge; new blocks per row, block unit and super tile.  Block b
+// covers units kU*b .. kU*b + kU-1, thread t row t of each; the row
+// pointers of all kU rows are loaded together.  Few rows have pair entries,
+// so each warp deals its rows that have them out to its lanes, one per lane,
+// and runs the merge once per 32 such rows.
+template <typename T>
+__global__ void __launch_bounds__(kB) k_pair_rows(int V, int nunits,
                                                   const int32_t* __restrict__ prow,
                                                   const int32_t* __restrict__ base_rp,
                                                   const int32_t* __restrict__ base_ci,
@@ -224,84 +384,81 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V,
                                                   int32_t* pe_pos, T* pe_rest,
                                                   const T* __restrict__ rest, int32_t* newcnt,
                                                   int32_t* nblk, int32_t* nsupc) {
-  const int64_t v = (int64_t)blockIdx.x * kB + threadIdx.x;
-  int kn = 0;
-  // both row pointers at once: the mesh row is loaded in the same round trip
-  // as the pair entries
-  const int32_t b = v < V ? prow[v] : 0, e = v < V ? prow[v + 1] : 0;
-  const int32_t r0 = v < V ? base_rp[v] : 0, r1 = v < V ? base_rp[v + 1] : 0;
-  if (e > b) {
-    const int32_t blen = r1 - r0;
-    const int n = e - b;
-    if (n <= kRegEntries && blen <= kRegMesh) {
-      int32_t col[kRegEntries], pid[kRegEntries], bc[kRegMesh];
-      T rs[kRegEntries];
+  __shared__ int s_unit[kU];
+  const int lane = threadIdx.x & 31;
+  const int64_t base = (int64_t)blockIdx.x * kU * kB + threadIdx.x;
+  int32_t b[kU], e[kU], r0[kU], r1[kU];
+  unsigned has[kU];
 #pragma unroll
-      for (int q = 0; q < kRegEntries; ++q) {
-        col[q] = 0x7FFFFFFF;
-        pid[q] = 0x7FFFFFFF;
-        if (q < n) {
-          col[q] = pe_col[b + q];
-          pid[q] = pe_pid[b + q];
-        }
+  for (int u = 0; u < kU; ++u) {
+    const int64_t v = base + (int64_t)u * kB;
+    const bool ok = v < V;
+    b[u] = ok ? prow[v] : 0;
+    e[u] = ok ? prow[v + 1] : 0;
+    r0[u] = ok ? base_rp[v] : 0;
+    r1[u] = ok ? base_rp[v + 1] : 0;
+  }
+  if (threadIdx.x < kU) s_unit[threadIdx.x] = 0;
+  int total = 0;
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int64_t v = base + (int64_t)u * kB;
+    has[u] = __ballot_sync(0xffffffffu, e[u] > b[u]);
+    total += __popc(has[u]);
+    if (v < V && e[u] <= b[u]) newcnt[v] = 0;
+  }
+  __syncthreads();
+  for (int round = 0; round * 32 < total; ++round) {
+    // this lane's row: the j-th set bit over has[0], has[1], ...
+    int j = round * 32 + lane, uu = -1, src = 0;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = __popc(has[u]);
+      if (uu < 0 && j < c) {
+        uu = u;
+        src = nth_set_bit(has[u], j);
+      } else if (uu < 0) {
+        j -= c;
       }
+    }
+    int32_t rb = 0, re = 0, rr0 = 0, rr1 = 0;
 #pragma unroll
-      for (int q = 0; q < kRegMesh; ++q) bc[q] = q < blen ? base_ci[r0 + q] : 0x7FFFFFFF;
-#pragma unroll
-      for (int q = 0; q < kRegEntries; ++q) rs[q] = q < n ? pe_rest[b + q] : T(0);
-      // sort by (col, pid): odd-even transposition, n passes
-#pragma unroll
-      for (int pass = 0; pass < kRegEntries; ++pass) {
-        if (pass >= n) break;
-#pragma unroll
-        for (int q = pass & 1; q + 1 < kRegEntries; q += 2) {
-          const bool sw = col[q] > col[q + 1] || (col[q] == col[q + 1] && pid[q] > pid[q + 1]);
-          if (sw) {
-            const int32_t tc = col[q], tp = pid[q];
-            const T tr = rs[q];
-            col[q] = col[q + 1]; pid[q] = pid[q + 1]; rs[q] = rs[q + 1];
-            col[q + 1] = tc; pid[q + 1] = tp; rs[q + 1] = tr;
-          }
-        }
+    for (int u = 0; u < kU; ++u) {  // every lane takes part in every shuffle
+      const int32_t xb = __shfl_sync(0xffffffffu, b[u], src);
+      const int32_t xe = __shfl_sync(0xffffffffu, e[u], src);
+      const int32_t x0 = __shfl_sync(0xffffffffu, r0[u], src);
+      const int32_t x1 = __shfl_sync(0xffffffffu, r1[u], src);
+      if (u == uu) {
+        rb = xb;
+        re = xe;
+        rr0 = x0;
+        rr1 = x1;
       }
-      // position in the merged row = mesh columns below c + new columns
-      // below c; entries with the same column (repeated pairs) share it
-      int prev_col = -1, kn_group = 0;
-#pragma unroll
-      for (int q = 0; q < kRegEntries; ++q) {
-        if (q < n) {
-          const int c = col[q];
-          int kb = 0;
-          bool in_mesh = false;
-#pragma unroll
-          for (int m = 0; m < kRegMesh; ++m) {
-            kb += bc[m] < c;
-            in_mesh |= bc[m] == c;
-          }
-          const bool first = c != prev_col;
-          const bool fresh = first && !in_mesh;
-          if (first) kn_group = kn;
-          pe_col[b + q] = c;
-          pe_pos[b + q] = (kb + kn_group) | (fresh ? kPairNewBlock : 0);
-          pe_rest[b + q] = rs[q];
-          if (fresh) ++kn;
-          prev_col = c;
-        }
-      }
-    } else {
-      kn = row_merge_global<T>(b, e, base_ci, r0, blen, pe_col, pe_pid, pe_pos, pe_rest, rest);
+    }
+    if (uu >= 0) {
+      const int64_t v = (int64_t)blockIdx.x * kU * kB + (int64_t)uu * kB +
+                        (threadIdx.x - lane) + src;
+      const int kn = merge_row<T>(rb, re, rr0, rr1, base_ci, pe_col, pe_pid, pe_pos, pe_rest,
+                                  rest);
+      newcnt[v] = kn;
+      if (kn) atomicAdd(&s_unit[uu], kn);
     }
   }
-  if (v < V) newcnt[v] = kn;
-  const int s = block_sum(kn);
-  if (threadIdx.x == 0) {
-    nblk[blockIdx.x] = s;
-    if (s) atomicAdd(&nsupc[blockIdx.x / kSuper], s);
+  __syncthreads();
+  if (threadIdx.x < kU) {
+    const int unit = blockIdx.x * kU + threadIdx.x;
+    const int su = s_unit[threadIdx.x];
+    if (unit < nunits) {
+      nblk[unit] = su;
+      if (su) atomicAdd(&nsupc[unit / kSuper], su);
+    }
   }
 }
 
 // Block b writes rows [b*kB, (b+1)*kB) of the new pattern (one warp per 32
 // rows), or on capacity overflow its share of the copy of the previous state.
+// Every load that does not depend on the new-block prefix is issued first,
+// so that a block waits for memory about twice.
 template <typename T>
 __global__ void __launch_bounds__(kB, 4) k_write_pattern(
     int V, int nnzb_base, int capacity, const int32_t* __restrict__ base_rp,
@@ -316,6 +473,7 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
     const int32_t* __restrict__ prev_pe_col, const int32_t* __restrict__ prev_pe_pos,
     const T* __restrict__ prev_pe_rest, int32_t* out_prow, int32_t* out_pe_col,
     int32_t* out_pe_pos, T* out_pe_rest) {
+  constexpr int kBatch = kMapPerWarp / 32;  // mesh columns per lane held in registers
   __shared__ int32_t s_shift[kB + 1];
   __shared__ int32_t s_dst[kB / 32][kMapPerWarp];
   const int64_t R0 = (int64_t)blockIdx.x * kB;
@@ -323,31 +481,48 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
   const int r = threadIdx.x;
   const bool valid = r < nrows;
   const int64_t v = R0 + r;
-  // the row's own loads first: they do not depend on the counts below
-  const int32_t b0 = valid ? base_rp[v] : 0x7FFFFFFF;
-  const int32_t nc0 = valid ? newcnt[v] : 0;
   const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const bool warp_live = g * 32 < nrows;
   const int gend = g * 32 + 32 < nrows ? g * 32 + 32 : nrows;
-  const int32_t z = g * 32 < nrows ? base_rp[R0 + gend] : 0;
-  // the row's pair entries (the new-block count is known only after the scan)
-  int32_t pr0 = 0, pr1 = 0;
-  if (valid && nc0) {
-    pr0 = prow[v];
-    pr1 = prow[v + 1];
+  // ---- round 1: row pointers, counts, pair offsets, the warp's column range
+  const int32_t b0 = valid ? base_rp[v] : 0x7FFFFFFF;
+  const int32_t b1r = valid ? base_rp[v + 1] : 0x7FFFFFFF;
+  const int32_t nc0 = valid ? newcnt[v] : 0;
+  const int32_t pr0 = valid ? prow[v] : 0;
+  const int32_t pr1 = valid ? prow[v + 1] : 0;
+  const int32_t a = warp_live ? base_rp[R0 + g * 32] : 0;
+  const int32_t z = warp_live ? base_rp[R0 + gend] : 0;
+  const int S = blockIdx.x / kSuper;
+  int all = 0, bef = 0;
+  for (int q = threadIdx.x; q < nsup; q += kB) {
+    const int c = nsupc[q];
+    all += c;
+    if (q < S) bef += c;
   }
-  // total new blocks (capacity check) and the new blocks of earlier blocks
-  int2 sums;
-  {
-    const int S = blockIdx.x / kSuper;
-    int all = 0, bef = 0;
-    for (int q = threadIdx.x; q < nsup; q += kB) {
-      const int c = nsupc[q];
-      all += c;
-      if (q < S) bef += c;
+  if (r < (int)blockIdx.x - S * kSuper) bef += nblk[S * kSuper + r];
+  // ---- round 2: the warp's mesh columns, and for rows that gained blocks
+  // their pair entries and their own mesh columns
+  const bool mapped = warp_live && z - a <= kMapPerWarp;
+  int32_t cv[kBatch];
+#pragma unroll
+  for (int k = 0; k < kBatch; ++k) {
+    const int32_t q = a + 32 * k + lane;
+    cv[k] = mapped && q < z ? base_ci[q] : 0;
+  }
+  int32_t w4[kRegNew], c4[kRegNew], cr[kRegMesh];
+#pragma unroll
+  for (int m = 0; m < kRegNew; ++m) {
+    w4[m] = 0;
+    c4[m] = 0;
+    if (nc0 && pr0 + m < pr1) {
+      w4[m] = pe_pos[pr0 + m];
+      c4[m] = pe_col[pr0 + m];
     }
-    if (r < (int)blockIdx.x - S * kSuper) bef += nblk[S * kSuper + r];
-    sums = block_sum2(all, bef);
   }
+#pragma unroll
+  for (int k = 0; k < kRegMesh; ++k) cr[k] = nc0 && b0 + k < b1r ? base_ci[b0 + k] : 0;
+  // ---- prefix of the new-block counts; capacity check
+  const int2 sums = block_sum2(all, bef);
   const int64_t total = (int64_t)nnzb_base + sums.x;
   if (total > capacity) {
     // overflow: the new buffer becomes a copy of the previous state
@@ -383,33 +558,28 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
   const int32_t nc = s_shift[r + 1] - sh;
   if (valid) rp[v] = b0 + sh;
   if (R0 + nrows == V && r == 0) rp[V] = base_rp[V] + s_shift[kB];
-  // one warp per 32 rows
-  if (g * 32 >= nrows) return;
-  const int32_t a = __shfl_sync(0xffffffffu, b0, 0);
+  if (!warp_live) return;
   const unsigned any_new = __ballot_sync(0xffffffffu, nc != 0);
   if (!any_new) {  // one contiguous shifted run
     const int32_t s0 = __shfl_sync(0xffffffffu, sh, 0);
-    for (int32_t q = a + lane; q < z; q += 32) ci[q + s0] = base_ci[q];
+    if (mapped) {
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int32_t q = a + 32 * k + lane;
+        if (q < z) ci[q + s0] = cv[k];
+      }
+    } else {
+      for (int32_t q = a + lane; q < z; q += 32) ci[q + s0] = base_ci[q];
+    }
     return;
   }
   // each lane's new columns (in column order), placed at their merged
-  // positions and kept in registers
+  // positions; the first kRegNew kept in registers
   int32_t nw[kRegNew];
 #pragma unroll
   for (int k = 0; k < kRegNew; ++k) nw[k] = 0x7FFFFFFF;
   const int32_t o0 = b0 + sh;
   if (valid && nc) {
-    // the first kRegNew entries in one round trip, the rest one by one
-    int32_t w4[kRegNew], c4[kRegNew];
-#pragma unroll
-    for (int m = 0; m < kRegNew; ++m) {
-      w4[m] = 0;
-      c4[m] = 0;
-      if (pr0 + m < pr1) {
-        w4[m] = pe_pos[pr0 + m];
-        c4[m] = pe_col[pr0 + m];
-      }
-    }
     int k = 0;
 #pragma unroll
     for (int m = 0; m < kRegNew; ++m) {
@@ -433,9 +603,9 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
       }
     }
   }
-  // the new place of every mesh column of a row that gained blocks: after
-  // the new columns that sort before it
-  auto new_place = [&](int32_t q, int32_t c, int32_t o) {
+  // the new place of a mesh column of this lane's row: after the new
+  // columns that sort before it
+  auto new_place = [&](int32_t c, int32_t o) {
 #pragma unroll
     for (int k = 0; k < kRegNew; ++k) o += nw[k] < c;
     if (nc > kRegNew) {  // the columns past the registers
@@ -448,45 +618,25 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
     }
     return o;
   };
-  if (z - a <= kMapPerWarp) {
+  if (mapped) {
     // owners write the destination of each of their mesh columns into the
-    // warp's map; then the copy runs with coalesced loads
+    // warp's map; then the loaded columns are stored
     int32_t* map = s_dst[g];
-    const int32_t nxt = __shfl_down_sync(0xffffffffu, b0, 1);
-    const int32_t b1 = (lane == 31 || g * 32 + lane + 1 >= gend) ? z : nxt;
     if (valid) {
       if (nc == 0) {
-        for (int32_t q = b0; q < b1; ++q) map[q - a] = q + sh;
+        for (int32_t q = b0; q < b1r; ++q) map[q - a] = q + sh;
       } else {
-        // the row's columns in one round trip (the first kRegMesh of them)
-        int32_t cr[kRegMesh];
-#pragma unroll
-        for (int k = 0; k < kRegMesh; ++k) cr[k] = b0 + k < b1 ? base_ci[b0 + k] : 0;
 #pragma unroll
         for (int k = 0; k < kRegMesh; ++k)
-          if (b0 + k < b1) map[b0 + k - a] = new_place(b0 + k, cr[k], b0 + k + sh);
-        for (int32_t q = b0 + kRegMesh; q < b1; ++q)
-          map[q - a] = new_place(q, base_ci[q], q + sh);
+          if (b0 + k < b1r) map[b0 + k - a] = new_place(cr[k], b0 + k + sh);
+        for (int32_t q = b0 + kRegMesh; q < b1r; ++q) map[q - a] = new_place(base_ci[q], q + sh);
       }
     }
     __syncwarp();
-    // the copy, loads of a batch first
-    constexpr int kBatch = 8;
-    for (int32_t qb = a; qb < z; qb += 32 * kBatch) {
-      int32_t cv[kBatch], dv[kBatch];
 #pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        const int32_t q = qb + 32 * k + lane;
-        if (q < z) {
-          cv[k] = base_ci[q];
-          dv[k] = map[q - a];
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        const int32_t q = qb + 32 * k + lane;
-        if (q < z) ci[dv[k]] = cv[k];
-      }
+    for (int k = 0; k < kBatch; ++k) {
+      const int32_t q = a + 32 * k + lane;
+      if (q < z) ci[map[q - a]] = cv[k];
     }
     return;
   }
@@ -544,14 +694,15 @@ cudaError_t add_pairs_t(const PairLaunch& L, int n, const int32_t* ij, const voi
   CK(cudaMemsetAsync(sup_c, 0, sizeof(int32_t) * 2 * nsup, s));
   k_pair_count<<<grid_for(n), kB, 0, s>>>(ij, n, V, L.cnt, L.status);
   CK(cudaGetLastError());
-  k_block_sums<<<nblocks, kB, 0, s>>>(L.cnt, V, blk_c, sup_c);
+  const int ngroups = (nblocks + kU - 1) / kU;
+  k_block_sums<<<ngroups, kB, 0, s>>>(L.cnt, V, nblocks, blk_c, sup_c);
   CK(cudaGetLastError());
-  k_scan_rows<<<nblocks, kB, 0, s>>>(L.cnt, V, sup_c, blk_c, nb.prow);
+  k_scan_rows<<<ngroups, kB, 0, s>>>(L.cnt, V, sup_c, blk_c, nb.prow);
   CK(cudaGetLastError());
   k_pair_fill<T><<<grid_for(n), kB, 0, s>>>(ij, n, V, nb.prow, L.cnt, nb.pe_col, L.pe_pid,
                                             (T*)nb.pe_rest, (const T*)rest);
   CK(cudaGetLastError());
-  k_pair_rows<T><<<nblocks, kB, 0, s>>>(V, nb.prow, L.base_rp, L.base_ci, nb.pe_col,
+  k_pair_rows<T><<<ngroups, kB, 0, s>>>(V, nblocks, nb.prow, L.base_rp, L.base_ci, nb.pe_col,
                                         L.pe_pid, nb.pe_pos, (T*)nb.pe_rest, (const T*)rest,
                                         L.newcnt, blk_n, sup_n);
   CK(cudaGetLastError());
