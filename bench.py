@@ -291,16 +291,20 @@ def extra_workloads(args, only=None):
         torch.cuda.synchronize()
         return statistics.median([a.elapsed_time(b) for a, b in ts])
 
-    # small cloths (launch-latency bound)
-    for n in ((10, 100) if run("cloth_small") else ()):
-        st = mi.cloth_static(n, np.float32)
-        ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    # small cloths (launch-latency bound), fp32 and, at 100^2, fp64
+    for n, dt in (((10, "float32"), (100, "float32"), (100, "float64")) if run("cloth_small")
+                  else ()):
+        npdt = np.dtype(dt)
+        tdt = getattr(torch, dt)
+        st = mi.cloth_static(n, npdt)
+        ctx = mad.Context(st["V"], st["F"], 3, dt, part_xyz=st["X"])
         terms = mad.Terms(mask=3, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
                           inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"])
-        x = torch.from_numpy(mi.cloth_x(n, 1000 + n, 0, np.float32)).to(dev)
-        g = torch.empty((st["V"], 3), device=dev)
-        H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
-        res[f"cloth{n}_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+        x = torch.from_numpy(mi.cloth_x(n, 1000 + n, 0, npdt)).to(dev)
+        g = torch.empty((st["V"], 3), dtype=tdt, device=dev)
+        H = torch.empty((ctx.info.capacity_blocks, 3, 3), dtype=tdt, device=dev)
+        key = f"cloth{n}_eval_ms" if dt == "float32" else f"cloth{n}_f64_eval_ms"
+        res[key] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
         ctx.close()
     # parameterization 500^2: eval and HVP
     if run("symdir500"):
