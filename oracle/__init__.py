@@ -85,6 +85,20 @@ class Oracle:
         lib.or_bsr_mv.argtypes = [ctypes.c_int32, ctypes.c_int, _i32p, _i32p, _f64p,
                                   _f64p, _f64p]
         lib.or_bsr_mv.restype = ctypes.c_int
+        lib.or_spring_res.argtypes = [ctypes.c_int, _f64p, _f64p, ctypes.c_double,
+                                      ctypes.c_double, _f64p, _f64p]
+        lib.or_spring_res.restype = None
+        lib.or_symdir_res.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double, _f64p,
+                                      _f64p]
+        lib.or_symdir_res.restype = None
+        lib.or_jacobian_shape.argtypes = [ctypes.c_int32, ctypes.c_int, ctypes.c_uint,
+                                          ctypes.c_int32, ctypes.c_int32, _i64p, _i64p]
+        lib.or_jacobian_shape.restype = ctypes.c_int
+        lib.or_jacobian.argtypes = [ctypes.c_int32, ctypes.c_int, _f64p, ctypes.c_uint,
+                                    ctypes.c_int32, _i32p, _f64p, ctypes.c_double, _f64p,
+                                    ctypes.c_double, ctypes.c_int32, _i32p, _f64p, _f64p,
+                                    _f64p, _i64p, _i32p, _f64p]
+        lib.or_jacobian.restype = ctypes.c_int
         self.lib = lib
 
     # ---- local terms ----------------------------------------------------
@@ -179,6 +193,52 @@ class Oracle:
         y = np.zeros(V * dof)
         self.lib.or_bsr_mv(V, dof, _p32(row_ptr), _p32(col_idx), _pf(H), _pf(v), _pf(y))
         return y.reshape(V, dof)
+
+
+    def spring_res(self, dof, xi, xj, L0, k):
+        """Residual [1] and 1 x 2dof Jacobian of one spring."""
+        r = np.zeros(1)
+        J = np.zeros(2 * dof)
+        self.lib.or_spring_res(dof, _pf(np.ascontiguousarray(xi, np.float64)),
+                               _pf(np.ascontiguousarray(xj, np.float64)), float(L0), float(k),
+                               _pf(r), _pf(J))
+        return r, J.reshape(1, 2 * dof)
+
+    def symdir_res(self, u0, u1, u2, M, A):
+        """Residuals [8] and 8 x 6 Jacobian of one symmetric Dirichlet face."""
+        r = np.zeros(8)
+        J = np.zeros(48)
+        f = lambda a: np.ascontiguousarray(a, np.float64).reshape(-1)  # noqa: E731
+        self.lib.or_symdir_res(_pf(f(u0)), _pf(f(u1)), _pf(f(u2)), _pf(f(M)), float(A), _pf(r),
+                               _pf(J))
+        return r, J.reshape(8, 6)
+
+    def jacobian(self, V, dof, x, mask, *, edges=None, L0=None, k=0.0, xt=None, w=0.0,
+                 F=None, Minv=None, area=None):
+        """Residuals r and the CSR Jacobian (row_ptr int64, col_idx, vals) in fp64."""
+        f64 = lambda a: None if a is None else np.ascontiguousarray(a, np.float64)  # noqa: E731
+        i32 = lambda a: None if a is None else np.ascontiguousarray(a, np.int32)  # noqa: E731
+        x = f64(x).reshape(-1)
+        edges, F = i32(edges), i32(F)
+        L0, xt, Minv, area = f64(L0), f64(xt), f64(Minv), f64(area)
+        nE = 0 if edges is None else edges.reshape(-1, 2).shape[0]
+        nF = 0 if F is None else F.reshape(-1, 3).shape[0]
+        nr = np.zeros(1, np.int64)
+        nz = np.zeros(1, np.int64)
+        if self.lib.or_jacobian_shape(V, dof, mask, nE, nF, nr.ctypes.data_as(_i64p),
+                                      nz.ctypes.data_as(_i64p)) != 0:
+            raise ValueError("or_jacobian_shape failed")
+        rows, nnz = int(nr[0]), int(nz[0])
+        r = np.zeros(max(rows, 1))
+        rp = np.zeros(rows + 1, np.int64)
+        ci = np.zeros(max(nnz, 1), np.int32)
+        vals = np.zeros(max(nnz, 1))
+        st = self.lib.or_jacobian(V, dof, _pf(x), mask, nE, _p32(edges), _pf(L0), float(k),
+                                  _pf(xt), float(w), nF, _p32(F), _pf(Minv), _pf(area), _pf(r),
+                                  rp.ctypes.data_as(_i64p), _p32(ci), _pf(vals))
+        if st != 0:
+            raise ValueError(f"or_jacobian failed: {st}")
+        return r[:rows], rp, ci[:nnz], vals[:nnz]
 
 
 _DEFAULT: Oracle | None = None

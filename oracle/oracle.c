@@ -493,3 +493,178 @@ int or_bsr_mv(int32_t V, int dof, const int32_t* row_ptr,
   }
   return OR_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* vector-valued objective: residuals and the sparse Jacobian                */
+/* ------------------------------------------------------------------------ */
+/* Page "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
+ * Computations", section 方法: a vector-valued objective assembles the sparse
+ * Jacobian J = sum_j P_j^T J_j S_j, with S_j the term's stencil selection
+ * and P_j placing the term's residuals in the global residual vector.
+ *
+ * Residual form of each mesh term, chosen so that F = 1/2 |r|^2 equals the
+ * scalar energy above (so J^T r = g and J^T J is the Gauss-Newton part of H):
+ *   spring  r = sqrt(k) (l - L0)                       1 residual
+ *           dr/dxi = sqrt(k) n^T = -dr/dxj
+ *   inertia r = sqrt(w) (xi - xt)                      dof residuals
+ *           dr/dxi = sqrt(w) I
+ *   SymDir  r = sqrt(2A) (vec J, vec J^-1)             8 residuals
+ *           d(vec J)[2al+ga]/du_k[be] = delta(al,be) w_k[ga]
+ *           d(J^-1)[m][n]/du_k[be] = -J^-1[m][be] (w_k^T J^-1)[n]
+ *           (from d(J^-1) = -J^-1 dJ J^-1), vec J^-1 = (m, n) -> 2m+n.
+ * Rows: the active term types in the order springs (edge order), inertia
+ * (vertex order, dof rows each), faces (face order, 8 rows each).  Columns:
+ * vertex * dof + component, ascending within each row (the stencil's
+ * vertices sorted by index).                                                 */
+
+/* Residuals r[1] and the 1 x 2dof Jacobian of one spring (xi, xj order). */
+void or_spring_res(int dof, const double* xi, const double* xj, double L0, double k,
+                   double* r, double* Jl) {
+  double d[3], l2 = 0.0;
+  for (int a = 0; a < dof; ++a) {
+    d[a] = xi[a] - xj[a];
+    l2 += d[a] * d[a];
+  }
+  double l = sqrt(l2), sk = sqrt(k);
+  r[0] = sk * (l - L0);
+  for (int a = 0; a < dof; ++a) {
+    Jl[a] = sk * d[a] / l;
+    Jl[dof + a] = -sk * d[a] / l;
+  }
+}
+
+/* Residuals r[8] and the 8 x 6 Jacobian (row-major, columns u0, u1, u2
+ * interleaved) of one symmetric Dirichlet face. */
+void or_symdir_res(const double* u0, const double* u1, const double* u2, const double* M,
+                   double A, double* r, double* Jl) {
+  double J[2][2];
+  for (int al = 0; al < 2; ++al)
+    for (int ga = 0; ga < 2; ++ga)
+      J[al][ga] = (u1[al] - u0[al]) * M[0 * 2 + ga] + (u2[al] - u0[al]) * M[1 * 2 + ga];
+  double d = J[0][0] * J[1][1] - J[0][1] * J[1][0];
+  double Ji[2][2] = {{J[1][1] / d, -J[0][1] / d}, {-J[1][0] / d, J[0][0] / d}};
+  double s = sqrt(2.0 * A);
+#if OR_MUTANT == 5 /* planted: residual scale sqrt(A) (F = E / 2) */
+  s = sqrt(A);
+#endif
+  for (int p = 0; p < 4; ++p) r[p] = s * J[p / 2][p % 2];
+  for (int p = 0; p < 4; ++p) r[4 + p] = s * Ji[p / 2][p % 2];
+  double w[3][2];
+  w[1][0] = M[0];
+  w[1][1] = M[1];
+  w[2][0] = M[2];
+  w[2][1] = M[3];
+  w[0][0] = -(w[1][0] + w[2][0]);
+  w[0][1] = -(w[1][1] + w[2][1]);
+  for (int kk = 0; kk < 3; ++kk) {
+    double wJi[2];  /* w_k^T J^-1 */
+    for (int n = 0; n < 2; ++n) wJi[n] = w[kk][0] * Ji[0][n] + w[kk][1] * Ji[1][n];
+    for (int be = 0; be < 2; ++be) {
+      int col = 2 * kk + be;
+      for (int al = 0; al < 2; ++al)
+        for (int ga = 0; ga < 2; ++ga)
+          Jl[(2 * al + ga) * 6 + col] = s * (al == be ? w[kk][ga] : 0.0);
+      for (int m = 0; m < 2; ++m)
+        for (int n = 0; n < 2; ++n) {
+#if OR_MUTANT == 6 /* planted: d(J^-1) with the factors' indices swapped */
+          Jl[(4 + 2 * m + n) * 6 + col] = -s * Ji[be][m] * wJi[n];
+#else
+          Jl[(4 + 2 * m + n) * 6 + col] = -s * Ji[m][be] * wJi[n];
+#endif
+        }
+    }
+  }
+}
+
+typedef struct {
+  int32_t col;
+  double v;
+} or_cv;
+
+static int or_cv_cmp(const void* pa, const void* pb) {
+  const or_cv* a = (const or_cv*)pa;
+  const or_cv* b = (const or_cv*)pb;
+  return (a->col > b->col) - (a->col < b->col);
+}
+
+/* Writes one row: the entries (vertex vid[s], component c) -> Jrow[s*dof+c]
+ * for the nv stencil vertices, sorted by column. */
+static void put_row(int dof, int nv, const int32_t* vid, const double* Jrow, int64_t* q,
+                    int32_t* col_idx, double* vals) {
+  or_cv e[9];
+  int n = 0;
+  for (int s = 0; s < nv; ++s)
+    for (int c = 0; c < dof; ++c) {
+      e[n].col = vid[s] * dof + c;
+      e[n].v = Jrow[s * dof + c];
+      ++n;
+    }
+  qsort(e, (size_t)n, sizeof(or_cv), or_cv_cmp);
+  for (int t = 0; t < n; ++t) {
+    col_idx[*q] = e[t].col;
+    vals[*q] = e[t].v;
+    ++*q;
+  }
+}
+
+/* Residual vector r and CSR Jacobian (row_ptr[nrows+1], col_idx, vals) of
+ * the active mesh terms (mask bits 1 spring, 2 inertia, 4 SymDir).  The
+ * caller sizes the outputs with or_jacobian_shape.  Inertia rows hold their
+ * single nonzero.  Returns OR_OK or an error. */
+int or_jacobian_shape(int32_t V, int dof, unsigned mask, int32_t nE, int32_t nF,
+                      int64_t* nrows, int64_t* nnz) {
+  int64_t r = 0, z = 0;
+  if (mask & 1u) { r += nE; z += (int64_t)nE * 2 * dof; }
+  if (mask & 2u) { r += (int64_t)V * dof; z += (int64_t)V * dof; }
+  if (mask & 4u) {
+    if (dof != 2) return OR_ERR_ARG;
+    r += (int64_t)nF * 8;
+    z += (int64_t)nF * 8 * 6;
+  }
+  *nrows = r;
+  *nnz = z;
+  return OR_OK;
+}
+
+int or_jacobian(int32_t V, int dof, const double* x, unsigned mask, int32_t nE,
+                const int32_t* edges, const double* L0, double k, const double* xt, double w,
+                int32_t nF, const int32_t* F, const double* Minv, const double* area,
+                double* r, int64_t* row_ptr, int32_t* col_idx, double* vals) {
+  if (dof < 2 || dof > 3 || ((mask & 4u) && dof != 2)) return OR_ERR_ARG;
+  int64_t row = 0, q = 0;
+  row_ptr[0] = 0;
+  if (mask & 1u) {
+    for (int32_t e = 0; e < nE; ++e) {
+      int32_t vid[2] = {edges[2 * e], edges[2 * e + 1]};
+      double Jl[6];
+      or_spring_res(dof, x + (size_t)vid[0] * dof, x + (size_t)vid[1] * dof, L0[e], k,
+                    r + row, Jl);
+      put_row(dof, 2, vid, Jl, &q, col_idx, vals);
+      row_ptr[++row] = q;
+    }
+  }
+  if (mask & 2u) {
+    double sw = sqrt(w);
+    for (int32_t v = 0; v < V; ++v)
+      for (int a = 0; a < dof; ++a) {
+        r[row] = sw * (x[(size_t)v * dof + a] - xt[(size_t)v * dof + a]);
+        col_idx[q] = v * dof + a;
+        vals[q] = sw;
+        ++q;
+        row_ptr[++row] = q;
+      }
+  }
+  if (mask & 4u) {
+    for (int32_t f = 0; f < nF; ++f) {
+      const int32_t* vid = F + 3 * (size_t)f;
+      double Jl[48];
+      or_symdir_res(x + (size_t)vid[0] * 2, x + (size_t)vid[1] * 2, x + (size_t)vid[2] * 2,
+                    Minv + 4 * (size_t)f, area[f], r + row, Jl);
+      for (int p = 0; p < 8; ++p) {
+        put_row(2, 3, vid, Jl + 6 * p, &q, col_idx, vals);
+        row_ptr[++row] = q;
+      }
+    }
+  }
+  return OR_OK;
+}
