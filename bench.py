@@ -263,7 +263,7 @@ def cpu_baseline(st):
             "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
 
 
-EXTRA = ("cloth_small", "symdir500", "pairs1000")
+EXTRA = ("cloth_small", "symdir500", "pairs1000", "jac1000")
 
 
 def extra_workloads(args, only=None):
@@ -311,7 +311,33 @@ def extra_workloads(args, only=None):
         symdir500(res, mad, torch, dev, stream, timeit)
     if run("pairs1000"):
         pairs1000(res, mad, torch, dev, stream)
+    if run("jac1000"):
+        jac1000(res, mad, torch, dev, stream, timeit)
     return res
+
+
+def jac1000(res, mad, torch, dev, stream, timeit):
+    """Residuals + sparse Jacobian of springs + inertia on the 1000^2 cloth.
+    Algorithmic bytes: read x, edges, L0, xt; write r and the Jacobian values
+    (the pattern is written once, outside the timed calls)."""
+    st = mi.cloth_static(N_GRID, np.float32)
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    terms = mad.Terms(mask=3, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
+                      inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"])
+    rows, nnz = ctx.mad_jacobian_shape(3)
+    rp = torch.empty(rows + 1, dtype=torch.int64, device=dev)
+    ci = torch.empty(nnz, dtype=torch.int32, device=dev)
+    r = torch.empty(rows, dtype=torch.float32, device=dev)
+    J = torch.empty(nnz, dtype=torch.float32, device=dev)
+    ctx.mad_jacobian_pattern(3, rp, ci, stream)
+    x = torch.from_numpy(mi.cloth_x(N_GRID, 1006, 0, np.float32)).to(dev)
+    ms = timeit(lambda: ctx.mad_jacobian(x, terms, r, J, stream))
+    E, V = len(st["edges"]), st["V"]
+    nbytes = 12 * V + 8 * E + 4 * E + 12 * V + 4 * rows + 4 * nnz
+    res["jac1000_ms"] = round(ms, 5)
+    res["jac1000_bytes"] = int(nbytes)
+    res["jac1000_gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+    ctx.close()
 
 
 def symdir500(res, mad, torch, dev, stream, timeit):

@@ -52,7 +52,8 @@ STATUS_NAMES = {0: "MAD_OK", 1: "MAD_ERR_INVALID_ARG", 2: "MAD_ERR_CUDA", 3: "MA
 # every symbol include/mad.h declares
 EXPORTS = ("mad_default_opts", "mad_create", "mad_info", "mad_edges", "mad_pattern",
            "mad_eval", "mad_hvp", "mad_add_pairs", "mad_status_sync", "mad_eval_host",
-           "mad_last_error", "mad_destroy", "mad_selftest_dual", "mad_energy_noalloc")
+           "mad_last_error", "mad_destroy", "mad_selftest_dual", "mad_energy_noalloc",
+           "mad_jacobian_shape", "mad_jacobian_pattern", "mad_jacobian")
 
 
 class mad_opts(ctypes.Structure):
@@ -124,6 +125,13 @@ def load_library(path: str = LIB_PATH):
     lib.mad_destroy.restype = None
     lib.mad_selftest_dual.argtypes = [i32, vp, vp]
     lib.mad_selftest_dual.restype = ctypes.c_int
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    lib.mad_jacobian_shape.argtypes = [vp, ctypes.c_uint32, i64p, i64p]
+    lib.mad_jacobian_shape.restype = ctypes.c_int
+    lib.mad_jacobian_pattern.argtypes = [vp, ctypes.c_uint32, vp, vp, vp]
+    lib.mad_jacobian_pattern.restype = ctypes.c_int
+    lib.mad_jacobian.argtypes = [vp, vp, ctypes.POINTER(mad_terms), vp, vp, vp]
+    lib.mad_jacobian.restype = ctypes.c_int
     lib.mad_energy_noalloc.argtypes = [i32, i32, ctypes.c_int, vp, ctypes.POINTER(mad_terms), i32,
                                        vp, i32, vp, i32, vp, vp, vp, vp]
     lib.mad_energy_noalloc.restype = ctypes.c_int
@@ -283,6 +291,28 @@ class Context:
         st = self.lib.mad_hvp(self.h, _dev_ptr(x, self.torch_dtype, "x"), ctypes.byref(t),
                               _dev_ptr(v, self.torch_dtype, "v"), _dev_ptr(y, self.torch_dtype, "y"),
                               _stream_ptr(stream))
+        self._check(st)
+
+    def mad_jacobian_shape(self, mask: int):
+        """(rows, nonzeros) of the Jacobian of the terms in `mask`."""
+        nr, nz = ctypes.c_int64(0), ctypes.c_int64(0)
+        self._check(self.lib.mad_jacobian_shape(self.h, mask, ctypes.byref(nr), ctypes.byref(nz)))
+        return nr.value, nz.value
+
+    def mad_jacobian_pattern(self, mask: int, row_ptr, col_idx, stream=None):
+        torch = _torch()
+        st = self.lib.mad_jacobian_pattern(self.h, mask, _dev_ptr(row_ptr, torch.int64, "row_ptr"),
+                                           _dev_ptr(col_idx, torch.int32, "col_idx",
+                                                    allow_none=True),
+                                           _stream_ptr(stream))
+        self._check(st)
+
+    def mad_jacobian(self, x, terms: Terms, r, J_vals, stream=None):
+        t = terms.to_c(self.torch_dtype)
+        st = self.lib.mad_jacobian(self.h, _dev_ptr(x, self.torch_dtype, "x"), ctypes.byref(t),
+                                   _dev_ptr(r, self.torch_dtype, "r", allow_none=True),
+                                   _dev_ptr(J_vals, self.torch_dtype, "J_vals", allow_none=True),
+                                   _stream_ptr(stream))
         self._check(st)
 
     def mad_add_pairs(self, ij, rest, stream=None):

@@ -574,6 +574,73 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij, const void* r
   return MAD_OK;
 }
 
+namespace {
+mad_status jac_mask_ok(const mad_ctx* c, uint32_t mask, std::string* why) {
+  const uint32_t known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR;
+  if (mask & ~known) {
+    *why = "unknown term bits in mask";
+    return MAD_ERR_INVALID_ARG;
+  }
+  if (mask & MAD_TERM_PAIR) {
+    *why = "pair terms are not part of the vector-valued objective";
+    return MAD_ERR_UNIMPLEMENTED;
+  }
+  if ((mask & MAD_TERM_SYMDIR) && c->dof != 2) {
+    *why = "symmetric Dirichlet term needs dof 2";
+    return MAD_ERR_UNIMPLEMENTED;
+  }
+  return MAD_OK;
+}
+}  // namespace
+
+mad_status mad_jacobian_shape(const mad_ctx* c, uint32_t mask, int64_t* nrows, int64_t* nnz) {
+  if (!c || !nrows || !nnz) return MAD_ERR_INVALID_ARG;
+  std::string why;
+  const mad_status st = jac_mask_ok(c, mask, &why);
+  if (st != MAD_OK) return st;
+  jac_shape(c->V, c->dof, mask, c->E, c->nF, nrows, nnz);
+  return MAD_OK;
+}
+
+mad_status mad_jacobian_pattern(mad_ctx* c, uint32_t mask, int64_t* row_ptr, int32_t* col_idx,
+                                void* stream) {
+  if (!c) return MAD_ERR_INVALID_ARG;
+  std::string why;
+  const mad_status st = jac_mask_ok(c, mask, &why);
+  if (st != MAD_OK) return fail(c, st, why);
+  int64_t rows = 0, nnz = 0;
+  jac_shape(c->V, c->dof, mask, c->E, c->nF, &rows, &nnz);
+  if (!row_ptr || (nnz > 0 && !col_idx))
+    return fail(c, MAD_ERR_INVALID_ARG, "row_ptr and col_idx must be device pointers");
+  const cudaError_t e = launch_jac_pattern(c->V, c->dof, mask, c->E, c->pat.edges, c->nF,
+                                           c->F_dev, row_ptr, col_idx, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(c, e, "mad_jacobian_pattern launch");
+  return MAD_OK;
+}
+
+mad_status mad_jacobian(mad_ctx* c, const void* x, const mad_terms* t, void* r, void* J_vals,
+                        void* stream) {
+  if (!c) return MAD_ERR_INVALID_ARG;
+  if (!t) return fail(c, MAD_ERR_INVALID_ARG, "terms is NULL");
+  std::string why;
+  const mad_status st = jac_mask_ok(c, t->mask, &why);
+  if (st != MAD_OK) return fail(c, st, why);
+  if ((t->mask & MAD_TERM_SPRING) && c->E > 0 && !t->spring_rest)
+    return fail(c, MAD_ERR_INVALID_ARG, "spring term active but spring_rest is NULL");
+  if ((t->mask & MAD_TERM_INERTIA) && c->V > 0 && !t->inertia_xt)
+    return fail(c, MAD_ERR_INVALID_ARG, "inertia term active but inertia_xt is NULL");
+  if ((t->mask & MAD_TERM_SYMDIR) && c->nF > 0 && (!t->face_Minv || !t->face_area))
+    return fail(c, MAD_ERR_INVALID_ARG, "symmetric Dirichlet term needs face_Minv and face_area");
+  int64_t rows = 0, nnz = 0;
+  jac_shape(c->V, c->dof, t->mask, c->E, c->nF, &rows, &nnz);
+  if (rows > 0 && (!x || !r || !J_vals))
+    return fail(c, MAD_ERR_INVALID_ARG, "x, r and J_vals must be device pointers");
+  const cudaError_t e = launch_jacobian(c->dtype, c->V, c->dof, t->mask, c->E, c->pat.edges,
+                                        c->nF, c->F_dev, *t, x, r, J_vals, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(c, e, "mad_jacobian launch");
+  return MAD_OK;
+}
+
 mad_status mad_status_sync(mad_ctx* c, void* stream) {
   if (!c) return MAD_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);

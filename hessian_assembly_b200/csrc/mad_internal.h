@@ -243,6 +243,15 @@ cudaError_t launch_rows_eval(const RowsLaunch& L, const mad_terms& t, const void
 cudaError_t launch_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
                             const void* v, void* y, cudaStream_t s);
 
+// jacobian.cu
+void jac_shape(int V, int dof, unsigned mask, int nE, int nF, int64_t* rows, int64_t* nnz);
+cudaError_t launch_jac_pattern(int V, int dof, unsigned mask, int nE, const int32_t* edges,
+                               int nF, const int32_t* F, int64_t* rp, int32_t* ci,
+                               cudaStream_t s);
+cudaError_t launch_jacobian(int dtype, int V, int dof, unsigned mask, int nE,
+                            const int32_t* edges, int nF, const int32_t* F, const mad_terms& t,
+                            const void* x, void* r, void* J, cudaStream_t s);
+
 // selftest.cu
 cudaError_t selftest_dual(int n, const double* ab_dev, double* out_dev);
 

@@ -216,6 +216,47 @@ mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t,
 mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij,
                          const void* rest, void* stream);
 
+/* ---- vector-valued objective: residuals and sparse Jacobian -------------
+ * Section 方法: a vector-valued objective assembles the sparse Jacobian
+ * J = sum_j P_j^T J_j S_j (S_j selects a term's stencil, P_j places its
+ * residuals in the global residual vector); the highlights note that
+ * materialising J explicitly pays off for large geometry problems.
+ * Each mesh term contributes a residual vector whose half squared norm is
+ * the term's scalar energy, so 1/2 |r|^2 = E, J^T r = g, and J^T J is the
+ * Gauss-Newton part of H:
+ *   MAD_TERM_SPRING   r = sqrt(k) (|x_a - x_b| - L0)         1 row per edge
+ *   MAD_TERM_INERTIA  r = sqrt(w) (x_v - xt_v)              dof rows per vertex
+ *   MAD_TERM_SYMDIR   r = sqrt(2A) (vec J, vec J^-1)         8 rows per face
+ *                     (vec of a 2x2 matrix: row-major; dof 2 only)
+ * Rows are term-major: springs in mad_edges order, then inertia (vertex v,
+ * component c at row v*dof + c of that segment), then faces in face order.
+ * J is scalar CSR with int64 row pointers and int32 columns; a column is
+ * vertex*dof + component, ascending within each row (the stencil's vertices
+ * sorted by index).  Nonzeros per row: 2*dof (spring), 1 (inertia), 6 (face).
+ * MAD_TERM_PAIR is not part of the vector objective
+ * (MAD_ERR_UNIMPLEMENTED).                                                  */
+
+/* Rows and nonzeros of the Jacobian of the terms in `mask`.  Errors:
+ * MAD_ERR_INVALID_ARG (NULL outputs, unknown bits), MAD_ERR_UNIMPLEMENTED
+ * (MAD_TERM_PAIR, or MAD_TERM_SYMDIR with dof 3).                           */
+mad_status mad_jacobian_shape(const mad_ctx* c, uint32_t mask, int64_t* nrows, int64_t* nnz);
+
+/* Writes the Jacobian's pattern for `mask`: row_ptr DEVICE int64 [nrows+1],
+ * col_idx DEVICE int32 [nnz] (caller-owned, sized by mad_jacobian_shape).
+ * The pattern depends only on the mesh and the mask.  Stream-ordered.       */
+mad_status mad_jacobian_pattern(mad_ctx* c, uint32_t mask, int64_t* row_ptr, int32_t* col_idx,
+                                void* stream);
+
+/* Residuals and Jacobian values at x for the terms in t->mask (t->flags is
+ * ignored): r DEVICE [nrows] and J_vals DEVICE [nnz] in the context dtype,
+ * in the order of mad_jacobian_pattern; both are overwritten.  The local
+ * Jacobians come from first-order forward AD on each term's natural
+ * variables.  Stream-ordered, no allocation, no host synchronisation.
+ * Errors: as mad_jacobian_shape, plus MAD_ERR_INVALID_ARG for a NULL array
+ * of an active term.                                                        */
+mad_status mad_jacobian(mad_ctx* c, const void* x, const mad_terms* t, void* r, void* J_vals,
+                        void* stream);
+
 /* Synchronise `stream`, read and clear the sticky device status word and
  * return it (MAD_OK when no device-side error was recorded).  Off the hot
  * path by design.                                                          */
