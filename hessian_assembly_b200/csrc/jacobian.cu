@@ -110,41 +110,64 @@ __global__ void __launch_bounds__(kJT) k_jac_pattern(Segs S, int dof, int V,
   (void)V;
 }
 
-template <typename T, int DOF>
-__global__ void __launch_bounds__(kJT) k_jac_springs(Segs S, int nE, const int32_t* __restrict__ edges,
-                                                     const T* __restrict__ x,
-                                                     const T* __restrict__ L0, T sk,
-                                                     T* __restrict__ r, T* __restrict__ J) {
-  for (int64_t e = blockIdx.x * (int64_t)kJT + threadIdx.x; e < nE;
-       e += (int64_t)gridDim.x * kJT) {
-    const int32_t a = edges[2 * e], b = edges[2 * e + 1];
-    Dual<T, DOF> s = d_const<T, DOF>(T(0));
-#pragma unroll
-    for (int c = 0; c < DOF; ++c) {
-      const Dual<T, DOF> d = d_var<T, DOF>(x[(int64_t)a * DOF + c] - x[(int64_t)b * DOF + c], c);
-      s = s + d * d;
-    }
-    const Dual<T, DOF> res = (sqrt(s) - L0[e]) * sk;
-    r[S.r_sp + e] = res.v;
-    T* row = J + S.z_sp + e * (2 * DOF);
-    // dr/dx_a = dr/dd, dr/dx_b = -dr/dd
-#pragma unroll
-    for (int c = 0; c < DOF; ++c) {
-      row[c] = res.g[c];
-      row[DOF + c] = -res.g[c];
-    }
-  }
+__device__ __forceinline__ void jbulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(ssrc);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(sa), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kJT) k_jac_inertia(Segs S, int64_t n, const T* __restrict__ x,
-                                                     const T* __restrict__ xt, T sw,
-                                                     T* __restrict__ r, T* __restrict__ J) {
-  for (int64_t q = blockIdx.x * (int64_t)kJT + threadIdx.x; q < n;
-       q += (int64_t)gridDim.x * kJT) {
-    const Dual<T, 1> res = (d_var<T, 1>(x[q], 0) - xt[q]) * sw;
-    r[S.r_in + q] = res.v;
-    J[S.z_in + q] = res.g[0];
+// Springs and inertia in one launch: blocks [0, nbs) take kJT edges each,
+// the rest kJT inertia rows each.  A block's spring rows (kJT * 2*DOF values,
+// contiguous in J) are staged in shared memory and leave with one 1-D bulk
+// copy when its first value and its size are 16-byte aligned; otherwise
+// every thread stores its own row.
+template <typename T, int DOF>
+__global__ void __launch_bounds__(kJT) k_jac_edges_vertices(
+    Segs S, int nE, int nbs, int64_t nin, const int32_t* __restrict__ edges,
+    const T* __restrict__ x, const T* __restrict__ L0, T sk, const T* __restrict__ xt, T sw,
+    T* __restrict__ r, T* __restrict__ J) {
+  __shared__ __align__(16) T stage[kJT * 2 * DOF];
+  if ((int)blockIdx.x < nbs) {
+    const int64_t e0 = (int64_t)blockIdx.x * kJT;
+    const int64_t e = e0 + threadIdx.x;
+    const int cnt = (int)((nE - e0) < kJT ? (nE - e0) : kJT);
+    if (e < nE) {
+      const int2 ab = reinterpret_cast<const int2*>(edges)[e];
+      Dual<T, DOF> s = d_const<T, DOF>(T(0));
+#pragma unroll
+      for (int c = 0; c < DOF; ++c) {
+        const Dual<T, DOF> d =
+            d_var<T, DOF>(x[(int64_t)ab.x * DOF + c] - x[(int64_t)ab.y * DOF + c], c);
+        s = s + d * d;
+      }
+      const Dual<T, DOF> res = (sqrt(s) - L0[e]) * sk;
+      r[S.r_sp + e] = res.v;
+      // dr/dx_a = dr/dd, dr/dx_b = -dr/dd
+#pragma unroll
+      for (int c = 0; c < DOF; ++c) {
+        stage[threadIdx.x * 2 * DOF + c] = res.g[c];
+        stage[threadIdx.x * 2 * DOF + DOF + c] = -res.g[c];
+      }
+    }
+    __syncthreads();
+    T* dst = J + S.z_sp + e0 * (2 * DOF);
+    const uint32_t bytes = (uint32_t)(cnt * 2 * DOF * sizeof(T));
+    if (((((uintptr_t)dst) | bytes) & 15u) == 0) {
+      if (threadIdx.x == 0) jbulk_store(dst, stage, bytes);
+    } else {
+      for (int q = threadIdx.x; q < cnt * 2 * DOF; q += kJT) dst[q] = stage[q];
+    }
+  } else {
+    const int64_t q = (int64_t)(blockIdx.x - nbs) * kJT + threadIdx.x;
+    if (q < nin) {
+      const Dual<T, 1> res = (d_var<T, 1>(x[q], 0) - xt[q]) * sw;
+      r[S.r_in + q] = res.v;
+      J[S.z_in + q] = res.g[0];
+    }
   }
 }
 
@@ -221,21 +244,20 @@ static cudaError_t jac_values(int V, int dof, unsigned mask, int nE, const int32
                               int nF, const int32_t* F, const mad_terms& t, const void* x,
                               void* r, void* J, cudaStream_t s) {
   const Segs S = make_segs(V, dof, mask, nE, nF);
-  if ((mask & MAD_TERM_SPRING) && nE > 0) {
-    const T sk = (T)std::sqrt(t.spring_k);
+  const int64_t ne = (mask & MAD_TERM_SPRING) ? nE : 0;
+  const int64_t nin = (mask & MAD_TERM_INERTIA) ? (int64_t)V * dof : 0;
+  if (ne + nin > 0) {
+    const int nbs = (int)((ne + kJT - 1) / kJT);
+    const int nbi = (int)((nin + kJT - 1) / kJT);
+    const T sk = (T)std::sqrt(t.spring_k), sw = (T)std::sqrt(t.inertia_w);
     if (dof == 3)
-      k_jac_springs<T, 3><<<jgrid(nE), kJT, 0, s>>>(S, nE, edges, (const T*)x,
-                                                   (const T*)t.spring_rest, sk, (T*)r, (T*)J);
+      k_jac_edges_vertices<T, 3><<<nbs + nbi, kJT, 0, s>>>(
+          S, (int)ne, nbs, nin, edges, (const T*)x, (const T*)t.spring_rest, sk,
+          (const T*)t.inertia_xt, sw, (T*)r, (T*)J);
     else
-      k_jac_springs<T, 2><<<jgrid(nE), kJT, 0, s>>>(S, nE, edges, (const T*)x,
-                                                   (const T*)t.spring_rest, sk, (T*)r, (T*)J);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  if ((mask & MAD_TERM_INERTIA) && V > 0) {
-    const int64_t n = (int64_t)V * dof;
-    k_jac_inertia<T><<<jgrid(n), kJT, 0, s>>>(S, n, (const T*)x, (const T*)t.inertia_xt,
-                                             (T)std::sqrt(t.inertia_w), (T*)r, (T*)J);
+      k_jac_edges_vertices<T, 2><<<nbs + nbi, kJT, 0, s>>>(
+          S, (int)ne, nbs, nin, edges, (const T*)x, (const T*)t.spring_rest, sk,
+          (const T*)t.inertia_xt, sw, (T*)r, (T*)J);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
