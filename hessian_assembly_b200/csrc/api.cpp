@@ -58,6 +58,9 @@ struct mad_ctx {
   int4* rows_fslots = nullptr;
   int32_t* rows_fofl_ptr = nullptr;
   int4* rows_fofl = nullptr;
+  int32_t* rows_fcslots = nullptr;
+  int32_t* rows_fcofl = nullptr;
+  void* face_hv = nullptr;  // [nF][3][2] scratch of the face Hessian-vector product
   double* epart = nullptr;
   size_t smem_eval = 0, smem_hvp = 0;
   // dynamic pattern
@@ -181,6 +184,11 @@ RowsLaunch rows_launch(const mad_ctx* c) {
   L.fslots = c->rows_fslots;
   L.fofl_ptr = c->rows_fofl_ptr;
   L.fofl = c->rows_fofl;
+  L.fcslots = c->rows_fcslots;
+  L.fcofl = c->rows_fcofl;
+  L.nF = c->nF;
+  L.F = c->F_dev;
+  L.fhv = c->face_hv;
   L.epart = c->epart;
   if (c->active < 0) {
     L.rp = c->pat.rp;
@@ -394,6 +402,11 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
         CREATE_CK(upload(c, &c->rows_fslots, fr.slots));
         CREATE_CK(upload(c, &c->rows_fofl_ptr, fr.ofl_ptr));
         CREATE_CK(upload(c, &c->rows_fofl, fr.ofl));
+        CREATE_CK(upload(c, &c->rows_fcslots, fr.cslots));
+        CREATE_CK(upload(c, &c->rows_fcofl, fr.cofl));
+        char* hv = nullptr;
+        CREATE_CK(dev_alloc(c, &hv, (size_t)c->esz * 6 * (size_t)nF));
+        c->face_hv = hv;
       }
     }
   }

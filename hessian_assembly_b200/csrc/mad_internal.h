@@ -126,6 +126,11 @@ struct HostFaceRows {
   std::vector<int4> slots;       // [ntiles][sf][32], f = -1 empty
   std::vector<int32_t> ofl_ptr;  // [V+1]
   std::vector<int4> ofl;
+  // the same incidences as 3f + c only (the Hessian-vector product reads
+  // per-face corner results): -1 empty; bit 31 set on the last slot of a row
+  // that continues in the overflow table
+  std::vector<int32_t> cslots;   // [ntiles][sf][32]
+  std::vector<int32_t> cofl;     // overflow, same order as ofl
 };
 std::string build_face_rows(int V, int nF, const int32_t* F, const int32_t* rp,
                             const int32_t* ci, HostFaceRows& out);
@@ -224,6 +229,11 @@ struct RowsLaunch {
   const int4* fslots;
   const int32_t* fofl_ptr;
   const int4* fofl;
+  const int32_t* fcslots;  // incidences as 3f + c (see HostFaceRows)
+  const int32_t* fcofl;
+  int nF;
+  const int32_t* F;        // [nF][3]
+  void* fhv;               // [nF][3][2] per-face corner results of H v (scratch)
   const int2* slots;
   const uint32_t* meta;
   const int32_t* ofl_ptr;

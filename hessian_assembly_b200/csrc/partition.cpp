@@ -456,6 +456,7 @@ std::string build_row_tables(int V, const int32_t* rp, const int32_t* ci, int s0
 std::string build_face_rows(int V, int nF, const int32_t* F, const int32_t* rp,
                             const int32_t* ci, HostFaceRows& out) {
   out = HostFaceRows();
+  if ((int64_t)nF * 3 >= (int64_t)0x7FFFFFFF) return "too many faces for 3f + c";
   for (int v = 0; v < V; ++v)
     if (rp[v + 1] - rp[v] >= (1 << kFacePosBits)) return "row too long for face positions";
   std::vector<int32_t> cnt(V + 1, 0);
@@ -470,6 +471,8 @@ std::string build_face_rows(int V, int nF, const int32_t* F, const int32_t* rp,
   out.ofl_ptr.assign(V + 1, 0);
   for (int v = 0; v < V; ++v) out.ofl_ptr[v + 1] = out.ofl_ptr[v] + std::max(0, cnt[v + 1] - sf);
   out.ofl.resize(std::max<int32_t>(1, out.ofl_ptr[V]));
+  out.cslots.assign((size_t)ntiles * sf * 32, -1);
+  out.cofl.resize(out.ofl.size());
   std::vector<int32_t> fill(V, 0);
   for (int64_t f = 0; f < nF; ++f) {  // face order within each row
     for (int c = 0; c < 3; ++c) {
@@ -484,10 +487,15 @@ std::string build_face_rows(int V, int nF, const int32_t* F, const int32_t* rp,
       const bool more = s == sf - 1 && cnt[i + 1] > sf;
       const int4 e = make_int4((int32_t)f, j, more ? (int32_t)((uint32_t)k | 0x80000000u) : k,
                                (int32_t)w);
-      if (s < sf)
+      const int32_t fc = (int32_t)(3 * f + c);
+      if (s < sf) {
         out.slots[((size_t)(i / 32) * sf + s) * 32 + i % 32] = e;
-      else
+        out.cslots[((size_t)(i / 32) * sf + s) * 32 + i % 32] =
+            more ? (int32_t)((uint32_t)fc | 0x80000000u) : fc;
+      } else {
         out.ofl[out.ofl_ptr[i] + (s - sf)] = e;
+        out.cofl[out.ofl_ptr[i] + (s - sf)] = fc;
+      }
     }
   }
   return "";

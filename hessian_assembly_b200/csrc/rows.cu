@@ -18,6 +18,7 @@
 // for each other, so memory latency is hidden across the resident warps.
 // A thread writes only its own row: no zeroing pass, no atomics.
 #include <algorithm>
+#include <type_traits>
 
 #include "mad_internal.h"
 #include "terms.cuh"
@@ -38,6 +39,9 @@ constexpr int rows_min_blocks() {
 
 template <typename T>
 struct RArgs {
+  const int32_t* fcslots;
+  const int32_t* fcofl;
+  const T* fhv;
   const int4* fslots;
   const int32_t* fofl_ptr;
   const int4* fofl;
@@ -473,14 +477,25 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   const int i = tile * 32 + lane;
   if (i >= A.V) return;
   const bool pairs = (A.mask & MAD_TERM_PAIR) && A.prow != nullptr;
+  // the row's own position, direction and slot meta are needed only by the
+  // vertex, edge and pair terms (face terms come from the per-face pass)
+  const bool own = A.mask & (MAD_TERM_INERTIA | MAD_TERM_SPRING | MAD_TERM_PAIR);
   T xi[DOF], vi[DOF], yr[DOF];
+  uint32_t m = 0;
 #pragma unroll
   for (int a = 0; a < DOF; ++a) {
-    xi[a] = A.x[(uint32_t)(i * DOF + a)];
-    vi[a] = A.v[(uint32_t)(i * DOF + a)];
+    xi[a] = T(0);
+    vi[a] = T(0);
     yr[a] = T(0);
   }
-  const uint32_t m = A.meta[i];
+  if (own) {
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) {
+      xi[a] = A.x[(uint32_t)(i * DOF + a)];
+      vi[a] = A.v[(uint32_t)(i * DOF + a)];
+    }
+    m = A.meta[i];
+  }
   if (A.mask & MAD_TERM_INERTIA) {
     T xti[DOF], Ei, gi[DOF], Hi[DOF * DOF];
 #pragma unroll
@@ -522,16 +537,27 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   }
   if constexpr (FACES && DOF == 2) {
     if (A.mask & MAD_TERM_SYMDIR) {
-      row_faces<T>(A, i, tile, lane,
-                   [&](const T* xj, const T* xk, int j, int k, int c, int, int, const T* M,
-                       T ar) {
-                     T vj[2], vk[2];
-                     vj[0] = A.v[(uint32_t)(j * 2)];
-                     vj[1] = A.v[(uint32_t)(j * 2 + 1)];
-                     vk[0] = A.v[(uint32_t)(k * 2)];
-                     vk[1] = A.v[(uint32_t)(k * 2 + 1)];
-                     hv_symdir_row<T, FULL>(xi, xj, xk, vi, vj, vk, c, M, ar, yr);
-                   });
+      // the row's corners' results of the per-face pass (k_face_hv)
+      constexpr int SF = kFaceRowSlots;
+      int32_t e[SF];
+#pragma unroll
+      for (int k = 0; k < SF; ++k)
+        e[k] = k < A.sf ? A.fcslots[(uint32_t)((tile * A.sf + k) * 32 + lane)] : -1;
+#pragma unroll
+      for (int k = 0; k < SF; ++k) {
+        if (e[k] == -1) continue;
+        const uint32_t q = (uint32_t)e[k] & 0x7FFFFFFFu;
+        yr[0] += A.fhv[2 * q];
+        yr[1] += A.fhv[2 * q + 1];
+      }
+      if (e[SF - 1] != -1 && e[SF - 1] < 0) {  // the row continues in the overflow table
+        const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
+        for (int q = o0; q < o1; ++q) {
+          const uint32_t fc = (uint32_t)A.fcofl[q];
+          yr[0] += A.fhv[2 * fc];
+          yr[1] += A.fhv[2 * fc + 1];
+        }
+      }
     }
   }
   if (pairs) {
@@ -554,10 +580,56 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   for (int a = 0; a < DOF; ++a) A.y[(uint32_t)(i * DOF + a)] = yr[a];
 }
 
+// Per-face pass of the Hessian-vector product: one thread per face computes
+// (H_f v_f) for its three corners once; the row kernel then adds, for each
+// row, its corners' results.  Each face is differentiated once instead of
+// once per corner, and no atomics are needed.
+template <typename T, bool FULL>
+__global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_t* __restrict__ F,
+                                                 const T* __restrict__ x, const T* __restrict__ v,
+                                                 const T* __restrict__ Minv,
+                                                 const T* __restrict__ area, T* __restrict__ out) {
+  const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (f >= nF) return;
+  const int32_t a = F[3 * f], b = F[3 * f + 1], c = F[3 * f + 2];
+  T u[3][2], w[3][2], M[4];
+  const int32_t vid[3] = {a, b, c};
+  // [V][2] arrays: a vertex's pair is one 2-element load when both arrays
+  // are aligned to it (the caller's pointers need not be)
+  using T2 = typename std::conditional<sizeof(T) == 4, float2, double2>::type;
+  if (vec2) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const T2 xu = reinterpret_cast<const T2*>(x)[vid[k]];
+      const T2 xv = reinterpret_cast<const T2*>(v)[vid[k]];
+      u[k][0] = xu.x;
+      u[k][1] = xu.y;
+      w[k][0] = xv.x;
+      w[k][1] = xv.y;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int al = 0; al < 2; ++al) {
+        u[k][al] = x[(int64_t)vid[k] * 2 + al];
+        w[k][al] = v[(int64_t)vid[k] * 2 + al];
+      }
+  }
+  load4<T>(Minv + 4 * f, M);
+  T o[6];
+  hv_symdir_face<T, FULL>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f], o);
+#pragma unroll
+  for (int q = 0; q < 6; ++q) out[6 * f + q] = o[q];
+}
+
 template <typename T>
 RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
                     void* g, void* H, void* y, bool energy) {
   RArgs<T> A;
+  A.fcslots = L.fcslots;
+  A.fcofl = L.fcofl;
+  A.fhv = (const T*)L.fhv;
   A.fslots = L.fslots;
   A.fofl_ptr = L.fofl_ptr;
   A.fofl = L.fofl;
@@ -682,6 +754,20 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
   const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
   if constexpr (DOF == 2) {
     if (t.mask & MAD_TERM_SYMDIR) {
+      if (L.nF > 0) {
+        const unsigned nbf = (unsigned)((L.nF + 255) / 256);
+        const bool vec2 = ((((uintptr_t)x) | ((uintptr_t)v)) % (2 * sizeof(T))) == 0;
+        if (full)
+          k_face_hv<T, true><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
+                                                 (const T*)t.face_Minv, (const T*)t.face_area,
+                                                 (T*)L.fhv);
+        else
+          k_face_hv<T, false><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
+                                                  (const T*)t.face_Minv, (const T*)t.face_area,
+                                                  (T*)L.fhv);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+      }
       const bool sp = t.mask & MAD_TERM_SPRING;
       if (sp && full)
         k_rows_hvp<T, DOF, true, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);

@@ -407,57 +407,54 @@ __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const 
   }
 }
 
-// One corner's share of (H v) for a symmetric Dirichlet face term: adds
-// (H_ii v_i + H_ij v_j + H_ik v_k) to y.  The reduced form contracts in J
-// space: dJ = sum over corners of v_corner w_corner^T, then
-// y += w_i-projection of H_J dJ.
+// (H v) of one symmetric Dirichlet face for all three corners: out[2k + al]
+// = sum_l (H_kl v_l)[al], with u and v the corners' positions and direction
+// in face order.  The reduced form contracts in J space: dJ = sum_k v_k w_k^T,
+// t = H_J dJ, out_k = t projected on w_k.
 template <typename T, bool FULL>
-__device__ __forceinline__ void hv_symdir_row(const T* xi, const T* xj, const T* xk,
-                                              const T* vi, const T* vj, const T* vk, int c,
-                                              const T* M, T A, T* y) {
+__device__ __forceinline__ void hv_symdir_face(const T* u0, const T* u1, const T* u2,
+                                               const T* v0, const T* v1, const T* v2,
+                                               const T* M, T A, T* out) {
   if constexpr (!FULL) {
+    const T w[3][2] = {{-(M[0] + M[2]), -(M[1] + M[3])}, {M[0], M[1]}, {M[2], M[3]}};
     T Jv[4], dJ[4];
 #pragma unroll
-    for (int al = 0; al < 2; ++al) {
-      const T u0 = sel3(c, xi[al], xk[al], xj[al]);
-      const T u1 = sel3(c, xj[al], xi[al], xk[al]);
-      const T u2 = sel3(c, xk[al], xj[al], xi[al]);
-      const T v0 = sel3(c, vi[al], vk[al], vj[al]);
-      const T v1 = sel3(c, vj[al], vi[al], vk[al]);
-      const T v2 = sel3(c, vk[al], vj[al], vi[al]);
+    for (int al = 0; al < 2; ++al)
 #pragma unroll
       for (int ga = 0; ga < 2; ++ga) {
-        Jv[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
-        dJ[2 * al + ga] = (v1 - v0) * M[ga] + (v2 - v0) * M[2 + ga];
+        Jv[2 * al + ga] = (u1[al] - u0[al]) * M[ga] + (u2[al] - u0[al]) * M[2 + ga];
+        dJ[2 * al + ga] = (v1[al] - v0[al]) * M[ga] + (v2[al] - v0[al]) * M[2 + ga];
       }
-    }
     Lin<T, 4> j[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) j[p] = lin_var<T, 4>(Jv[p], p);
     HyperDual<T, 4> e = symdir_energy(j, A);
-    T wi[2];
+    T t[4];
 #pragma unroll
-    for (int ga = 0; ga < 2; ++ga)
-      wi[ga] = sel3(c, -(M[ga] + M[2 + ga]), M[ga], M[2 + ga]);
-#pragma unroll
-    for (int al = 0; al < 2; ++al) {
+    for (int p = 0; p < 4; ++p) {
       T s = T(0);
 #pragma unroll
-      for (int ga = 0; ga < 2; ++ga) {
-        T t = T(0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) t += hess(e, 2 * al + ga, q) * dJ[q];
-        s += t * wi[ga];
-      }
-      y[al] += s;
+      for (int q = 0; q < 4; ++q) s += hess(e, p, q) * dJ[q];
+      t[p] = s;
     }
-  } else {
-    FaceRow<T> o;
-    eval_symdir_row<T, true>(xi, xj, xk, c, M, A, o);
 #pragma unroll
-    for (int al = 0; al < 2; ++al)
-      y[al] += o.H[0][2 * al] * vi[0] + o.H[0][2 * al + 1] * vi[1] + o.H[1][2 * al] * vj[0] +
-               o.H[1][2 * al + 1] * vj[1] + o.H[2][2 * al] * vk[0] + o.H[2][2 * al + 1] * vk[1];
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int al = 0; al < 2; ++al) out[2 * k + al] = t[2 * al] * w[k][0] + t[2 * al + 1] * w[k][1];
+  } else {
+    FaceDerivs<T> o;
+    eval_symdir<T, true>(u0, u1, u2, M, A, o);
+    const T* vv[3] = {v0, v1, v2};
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+#pragma unroll
+      for (int al = 0; al < 2; ++al) {
+        T s = T(0);
+#pragma unroll
+        for (int l = 0; l < 3; ++l)
+          s += o.H[k][l][2 * al] * vv[l][0] + o.H[k][l][2 * al + 1] * vv[l][1];
+        out[2 * k + al] = s;
+      }
   }
 }
 

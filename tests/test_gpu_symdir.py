@@ -194,3 +194,38 @@ def test_symdir_with_springs_inertia_and_pairs(orc, flags):
     assert_close("H", H[:nnzb].cpu().numpy(), oH, dtype)
     assert abs(e.item() - oE) <= ETOL[dtype] * abs(oE)
     assert_close("y", y.cpu().numpy(), orc.bsr_mv(V, 2, orp, oci, oH, v), dtype)
+
+
+@pytest.mark.parametrize("dtype", ["float32", "float64"])
+def test_symdir_unaligned_caller_arrays(orc, dtype):
+    """x and v handed in at an odd element offset (not aligned to a vertex's
+    pair of values): the per-face passes fall back to element loads and the
+    results match the aligned call."""
+    import hessian_assembly_b200 as mad
+    import torch
+    n = 12
+    ps = mi.param_static(n, 2400, np.dtype(dtype))
+    V = ps["V"]
+    ctx = mad.Context(V, ps["F"], 2, dtype, part_xyz=ps["X"])
+    terms = terms_for(ps, dtype)
+    tt = getattr(torch, dtype)
+    v = mi.probe_vector(V, 2, 2401, np.dtype(dtype))
+    xa = to_dev(ps["UV"], dtype)
+    va = to_dev(v, dtype)
+    xb_buf = torch.zeros(2 * V + 1, dtype=tt, device="cuda")
+    vb_buf = torch.zeros(2 * V + 1, dtype=tt, device="cuda")
+    xb_buf[1:] = xa.reshape(-1)
+    vb_buf[1:] = va.reshape(-1)
+    xb, vb = xb_buf[1:], vb_buf[1:]
+    assert xb.data_ptr() % (2 * xb.element_size()) != 0
+    out = []
+    for x_, v_ in ((xa, va), (xb, vb)):
+        g = torch.zeros((V, 2), dtype=tt, device="cuda")
+        H = torch.zeros((ctx.info.capacity_blocks, 2, 2), dtype=tt, device="cuda")
+        y = torch.zeros((V, 2), dtype=tt, device="cuda")
+        ctx.mad_eval(x_, terms, g, H)
+        ctx.mad_hvp(x_, terms, v_, y)
+        torch.cuda.synchronize()
+        out.append((g.cpu().numpy(), H.cpu().numpy(), y.cpu().numpy()))
+    for a, b in zip(out[0], out[1]):
+        np.testing.assert_array_equal(a, b)
