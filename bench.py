@@ -305,6 +305,19 @@ def extra_workloads(args, only=None):
         H = torch.empty((ctx.info.capacity_blocks, 3, 3), dtype=tdt, device=dev)
         key = f"cloth{n}_eval_ms" if dt == "float32" else f"cloth{n}_f64_eval_ms"
         res[key] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+        if dt == "float32":  # the same step as a CUDA-graph replay of 20 steps
+            reps = 20
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                ctx.mad_eval(x, terms, g, H, None, side)
+            stream.wait_stream(side)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(reps):
+                    ctx.mad_eval(x, terms, g, H)
+            res[f"cloth{n}_graph_eval_ms"] = round(timeit(graph.replay) / reps, 5)
+            del graph
         ctx.close()
     # parameterization 500^2: eval and HVP
     if run("symdir500"):

@@ -257,6 +257,15 @@ mad_status mad_jacobian_pattern(mad_ctx* c, uint32_t mask, int64_t* row_ptr, int
 mad_status mad_jacobian(mad_ctx* c, const void* x, const mad_terms* t, void* r, void* J_vals,
                         void* stream);
 
+/* Stream capture.  mad_eval, mad_hvp, mad_add_pairs, mad_jacobian_pattern
+ * and mad_jacobian only enqueue kernels and memsets on `stream`: they
+ * neither allocate nor synchronise, so they can be recorded in a CUDA graph
+ * and replayed with new data in the captured buffers.  Host-side choices
+ * are fixed at capture: the number of pairs passed to mad_add_pairs, the
+ * term mask and flags, and which of the two CSR buffers each captured call
+ * reads or writes.  mad_status_sync, mad_eval_host, mad_create and
+ * mad_destroy synchronise or allocate and cannot be captured.               */
+
 /* Synchronise `stream`, read and clear the sticky device status word and
  * return it (MAD_OK when no device-side error was recorded).  Off the hot
  * path by design.                                                          */
