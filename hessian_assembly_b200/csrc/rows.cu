@@ -623,6 +623,18 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
   for (int q = 0; q < 6; ++q) out[6 * f + q] = o[q];
 }
 
+// Staging elements per warp: 32 mesh rows of s0 + 1 blocks, plus, when the
+// active pattern has inserted pair blocks, kWarpSpare blocks for them
+// (shared by the warp's rows; rows past the reserve are assembled in place),
+// rounded to 16 bytes, plus 16 bytes of alignment room.
+constexpr int kWarpSpare = 16;
+size_t wstage_elems(const RowsLaunch& L) {
+  const int vec = L.dtype == MAD_F64 ? 2 : 4;
+  const int blocks = 32 * (L.s0 + 1) + (L.rho > 0 ? kWarpSpare : 0);
+  const int elems = blocks * L.dof * L.dof;
+  return (size_t)(((elems + vec - 1) / vec) * vec + vec);
+}
+
 template <typename T>
 RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
                     void* g, void* H, void* y, bool energy) {
@@ -659,9 +671,7 @@ RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, cons
   A.epart = energy ? L.epart : nullptr;
   A.V = L.V;
   A.s0 = L.s0;
-  const int vec = 16 / (int)sizeof(T);
-  const int rows = 32 * (L.s0 + 1 + L.rho) * L.dof * L.dof;
-  A.wstage = ((rows + vec - 1) / vec) * vec + vec;
+  A.wstage = (int)wstage_elems(L);
   return A;
 }
 
@@ -821,11 +831,7 @@ int rows_blocks(int V) {
 }
 
 size_t rows_smem_bytes(const RowsLaunch& L) {
-  const int esz = L.dtype == MAD_F64 ? 8 : 4;
-  const int vec = 16 / esz;
-  const int rows = 32 * (L.s0 + 1 + L.rho) * L.dof * L.dof;
-  const int wstage = ((rows + vec - 1) / vec) * vec + vec;
-  return (size_t)kWarps * wstage * esz;
+  return (size_t)kWarps * wstage_elems(L) * (L.dtype == MAD_F64 ? 8 : 4);
 }
 
 cudaError_t rows_set_smem_limits(int dtype, int dof, size_t bytes) {
