@@ -241,10 +241,50 @@ def run_ours(args, rank, world, dist):
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(st)
+        if not args.no_extra:
+            out["cpu_baseline"]["rows"] = cpu_baseline_rows(st)
     if not args.no_extra and rank == 0:
         out["workloads"] = extra_workloads(args)
     ctx.close()
     return out
+
+
+def cpu_baseline_rows(st):
+    """The oracle beside each secondary workload: one run on one host core,
+    on the same seeded inputs as the GPU timings of extra_workloads."""
+    import oracle
+    orc = oracle.load()
+    res = {}
+    # SymDir 500^2: pattern + assembly, then the product with the assembled H
+    ps = mi.param_static(500, 1004, np.float32)
+    t0 = time.perf_counter()
+    rp, ci = orc.pattern(ps["V"], ps["F"])
+    og, oH, _ = orc.eval(ps["V"], 2, ps["UV"], 4, rp, ci, F=ps["F"], Minv=ps["Minv"],
+                         area=ps["area"])
+    t1 = time.perf_counter()
+    orc.bsr_mv(ps["V"], 2, rp, ci, oH, mi.probe_vector(ps["V"], 2, 1005, np.float32))
+    t2 = time.perf_counter()
+    res["symdir500_eval_ms"] = round((t1 - t0) * 1e3, 1)
+    res["symdir500_hvp_ms"] = round((t2 - t1) * 1e3, 1)
+    # cloth 1000^2 + 10^5 pairs (step 0): the pattern with the pairs, then assembly
+    xx = mi.cloth_x(N_GRID, 1005, 0, np.float32)
+    pp = mi.random_pairs(N_GRID, 100_000, 1005, 0)
+    t0 = time.perf_counter()
+    rp, ci = orc.pattern(st["V"], st["F"], pp)
+    t1 = time.perf_counter()
+    orc.eval(st["V"], 3, xx, 11, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"], xt=st["xt"],
+             w=st["w"], pairs=pp, prest=mi.pair_rest(xx, pp, np.float32), kp=mi.PAIR_K)
+    t2 = time.perf_counter()
+    res["pairs1000_insert_ms"] = round((t1 - t0) * 1e3, 1)
+    res["pairs1000_assembly_ms"] = round((t2 - t1) * 1e3, 1)
+    # residuals + Jacobian of springs + inertia at 1000^2
+    xx = mi.cloth_x(N_GRID, 1006, 0, np.float32)
+    t0 = time.perf_counter()
+    orc.jacobian(st["V"], 3, xx, 3, edges=st["edges"], L0=st["L0"], k=st["k"], xt=st["xt"],
+                 w=st["w"])
+    res["jac1000_ms"] = round((time.perf_counter() - t0) * 1e3, 1)
+    res["unit"] = "ms per call, 1 core, one run"
+    return res
 
 
 def cpu_baseline(st):
