@@ -82,6 +82,15 @@ class Oracle:
                                 ctypes.c_int32, _i32p, _f64p, ctypes.c_double,
                                 _i32p, _i32p, _f64p, _f64p, _f64p]
         lib.or_eval.restype = ctypes.c_int
+        lib.or_eval2.argtypes = [ctypes.c_int32, ctypes.c_int, _f64p, ctypes.c_uint,
+                                 ctypes.c_int32, _i32p, _f64p, ctypes.c_double, _f64p,
+                                 ctypes.c_double, ctypes.c_int32, _i32p, _f64p, _f64p,
+                                 ctypes.c_int32, _i32p, _f64p, ctypes.c_double, ctypes.c_double,
+                                 _i32p, _i32p, _f64p, _f64p, _f64p]
+        lib.or_eval2.restype = ctypes.c_int
+        lib.or_area_local.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_double,
+                                      _f64p, _f64p, _f64p]
+        lib.or_area_local.restype = None
         lib.or_bsr_mv.argtypes = [ctypes.c_int32, ctypes.c_int, _i32p, _i32p, _f64p,
                                   _f64p, _f64p]
         lib.or_bsr_mv.restype = ctypes.c_int
@@ -162,7 +171,7 @@ class Oracle:
     # ---- assembly -------------------------------------------------------
     def eval(self, V, dof, x, mask, row_ptr, col_idx, *, edges=None, L0=None, k=0.0,
              xt=None, w=0.0, F=None, Minv=None, area=None, pairs=None, prest=None,
-             kp=0.0):
+             kp=0.0, ka=0.0):
         """Assemble g [V][dof], H_vals [nnzb][dof][dof] and the energy (fp64)."""
         f64 = lambda a: None if a is None else np.ascontiguousarray(a, np.float64)  # noqa: E731
         i32 = lambda a: None if a is None else np.ascontiguousarray(a, np.int32)  # noqa: E731
@@ -177,10 +186,10 @@ class Oracle:
         g = np.zeros(V * dof)
         H = np.zeros(nnzb * dof * dof)
         E = np.zeros(1)
-        r = self.lib.or_eval(V, dof, _pf(x), mask, nE, _p32(edges), _pf(L0), float(k),
-                             _pf(xt), float(w), nF, _p32(F), _pf(Minv), _pf(area),
-                             nP, _p32(pairs), _pf(prest), float(kp),
-                             _p32(row_ptr), _p32(col_idx), _pf(g), _pf(H), _pf(E))
+        r = self.lib.or_eval2(V, dof, _pf(x), mask, nE, _p32(edges), _pf(L0), float(k),
+                              _pf(xt), float(w), nF, _p32(F), _pf(Minv), _pf(area),
+                              nP, _p32(pairs), _pf(prest), float(kp), float(ka),
+                              _p32(row_ptr), _p32(col_idx), _pf(g), _pf(H), _pf(E))
         if r != 0:
             raise ValueError(f"or_eval failed: {r}")
         return g.reshape(V, dof), H.reshape(nnzb, dof, dof), float(E[0])
@@ -194,6 +203,16 @@ class Oracle:
         self.lib.or_bsr_mv(V, dof, _p32(row_ptr), _p32(col_idx), _pf(H), _pf(v), _pf(y))
         return y.reshape(V, dof)
 
+
+    def area_local(self, x0, x1, x2, A0, k):
+        """Energy, gradient [9] and Hessian [9][9] of one area-preservation face."""
+        E = np.zeros(1)
+        g = np.zeros(9)
+        H = np.zeros(81)
+        f = lambda a: np.ascontiguousarray(a, np.float64)  # noqa: E731
+        self.lib.or_area_local(_pf(f(x0)), _pf(f(x1)), _pf(f(x2)), float(A0), float(k), _pf(E),
+                               _pf(g), _pf(H))
+        return float(E[0]), g, H.reshape(9, 9)
 
     def spring_res(self, dof, xi, xj, L0, k):
         """Residual [1] and 1 x 2dof Jacobian of one spring."""

@@ -189,6 +189,103 @@ void or_symdir_local(const double* u0, const double* u1, const double* u2,
         }
 }
 
+/* Area preservation of one triangle in 3D (a face term with a 9-variable
+ * stencil): A = 1/2 |n|, n = e1 x e2, e1 = x1 - x0, e2 = x2 - x0,
+ *   E = 1/2 k (A - A0)^2 / A0.
+ * With [a] the cross-product matrix ([a] b = a x b), nh = n / |n|:
+ *   dn/dx0 = [e2 - e1], dn/dx1 = -[e2], dn/dx2 = [e1]   (Jn, 3 x 9)
+ *   dA = 1/2 Jn^T nh
+ *   d2A = 1/2 ( Jn^T (I - nh nh^T) Jn / |n|  +  B ),
+ *   B: n is bilinear in (e1, e2) with d2 n_c / de1_a de2_b = eps_cab, so
+ *   sum_c nh_c d2 n_c is the form de1^T Q de2' + de1'^T Q de2 with
+ *   Q[a][b] = sum_c eps_cab nh_c; e1 and e2 take x with coefficients
+ *   p1 = (-1, 1, 0) and p2 = (-1, 0, 1), so block (i, j) of B is
+ *   p1_i p2_j Q + p2_i p1_j Q^T.
+ *   g = k (A - A0) / A0 dA,   H = k / A0 (dA dA^T + (A - A0) d2A).
+ * Output g[9] = (x0, x1, x2), H 9x9 row-major.                             */
+static void cross_mat(const double* a, double C[3][3]) {
+  C[0][0] = 0.0;   C[0][1] = -a[2]; C[0][2] = a[1];
+  C[1][0] = a[2];  C[1][1] = 0.0;   C[1][2] = -a[0];
+  C[2][0] = -a[1]; C[2][1] = a[0];  C[2][2] = 0.0;
+}
+
+void or_area_local(const double* x0, const double* x1, const double* x2, double A0, double k,
+                   double* E, double* g, double* H) {
+  double e1[3], e2[3], d21[3], n[3];
+  for (int a = 0; a < 3; ++a) {
+    e1[a] = x1[a] - x0[a];
+    e2[a] = x2[a] - x0[a];
+    d21[a] = e2[a] - e1[a];
+  }
+  n[0] = e1[1] * e2[2] - e1[2] * e2[1];
+  n[1] = e1[2] * e2[0] - e1[0] * e2[2];
+  n[2] = e1[0] * e2[1] - e1[1] * e2[0];
+  double l = sqrt(n[0] * n[0] + n[1] * n[1] + n[2] * n[2]);
+  double nh[3] = {n[0] / l, n[1] / l, n[2] / l};
+  double A = 0.5 * l;
+  double C0[3][3], C1[3][3], C2[3][3];
+  cross_mat(d21, C0);
+  cross_mat(e2, C1);
+  cross_mat(e1, C2);
+  double Jn[3][9];
+  for (int r = 0; r < 3; ++r)
+    for (int c = 0; c < 3; ++c) {
+      Jn[r][c] = C0[r][c];
+      Jn[r][3 + c] = -C1[r][c];
+      Jn[r][6 + c] = C2[r][c];
+    }
+  double dA[9];
+  for (int q = 0; q < 9; ++q) {
+    double s = 0.0;
+    for (int r = 0; r < 3; ++r) s += Jn[r][q] * nh[r];
+    dA[q] = 0.5 * s;
+  }
+  double P[3][3];  /* I - nh nh^T */
+  for (int r = 0; r < 3; ++r)
+    for (int c = 0; c < 3; ++c) P[r][c] = (r == c ? 1.0 : 0.0) - nh[r] * nh[c];
+  double Q[3][3];
+  for (int a = 0; a < 3; ++a)
+    for (int b = 0; b < 3; ++b) {
+      double s = 0.0;
+      for (int c = 0; c < 3; ++c) {
+        int eps = 0;
+        if ((c == 0 && a == 1 && b == 2) || (c == 1 && a == 2 && b == 0) ||
+            (c == 2 && a == 0 && b == 1))
+          eps = 1;
+        if ((c == 0 && a == 2 && b == 1) || (c == 1 && a == 0 && b == 2) ||
+            (c == 2 && a == 1 && b == 0))
+          eps = -1;
+        s += eps * nh[c];
+      }
+      Q[a][b] = s;
+    }
+  const double p1[3] = {-1.0, 1.0, 0.0}, p2[3] = {-1.0, 0.0, 1.0};
+  double d2A[9][9];
+  for (int i = 0; i < 9; ++i)
+    for (int j = 0; j < 9; ++j) {
+      double s = 0.0;
+      for (int r = 0; r < 3; ++r)
+        for (int c = 0; c < 3; ++c) s += Jn[r][i] * P[r][c] * Jn[c][j];
+      s /= l;
+      int vi = i / 3, ai = i % 3, vj = j / 3, aj = j % 3;
+      s += p1[vi] * p2[vj] * Q[ai][aj] + p2[vi] * p1[vj] * Q[aj][ai];
+      d2A[i][j] = 0.5 * s;
+    }
+  double dev = A - A0;
+  *E = 0.5 * k * dev * dev / A0;
+  for (int q = 0; q < 9; ++q) g[q] = k * dev / A0 * dA[q];
+  for (int i = 0; i < 9; ++i)
+    for (int j = 0; j < 9; ++j) {
+#if OR_MUTANT == 7 /* planted: bilinear part of d2A dropped */
+      int vi = i / 3, ai = i % 3, vj = j / 3, aj = j % 3;
+      double Bij = 0.5 * (p1[vi] * p2[vj] * Q[ai][aj] + p2[vi] * p1[vj] * Q[aj][ai]);
+      H[i * 9 + j] = k / A0 * (dA[i] * dA[j] + dev * (d2A[i][j] - Bij));
+#else
+      H[i * 9 + j] = k / A0 * (dA[i] * dA[j] + dev * d2A[i][j]);
+#endif
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* COO machinery                                                             */
 /* ------------------------------------------------------------------------ */
@@ -360,24 +457,30 @@ static int emit_blocks(or_coo* c, int dof, int nv, const int32_t* vid,
  * run-dtype values).  mask bits: 1 spring, 2 inertia, 4 symmetric Dirichlet,
  * 8 pairs.  Outputs: g [V][dof] (overwritten), H_vals [nnzb][dof][dof]
  * (overwritten; blocks absent from every term are zero), *energy.          */
-int or_eval(int32_t V, int dof, const double* x, unsigned mask,
-            /* springs */ int32_t nE, const int32_t* edges, const double* L0,
-            double k,
-            /* inertia */ const double* xt, double w,
-            /* symmetric Dirichlet */ int32_t nF, const int32_t* F,
-            const double* Minv, const double* area,
-            /* pairs */ int32_t nP, const int32_t* pairs, const double* prest,
-            double kp,
-            /* pattern */ const int32_t* row_ptr, const int32_t* col_idx,
-            /* out */ double* g, double* H_vals, double* energy) {
+/* mask bits: 1 spring, 2 inertia, 4 symmetric Dirichlet (dof 2, with Minv
+ * and area = rest area), 8 pairs, 16 area preservation (dof 3, with area =
+ * rest area A0 and stiffness ka). */
+int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
+             /* springs */ int32_t nE, const int32_t* edges, const double* L0,
+             double k,
+             /* inertia */ const double* xt, double w,
+             /* faces */ int32_t nF, const int32_t* F,
+             const double* Minv, const double* area,
+             /* pairs */ int32_t nP, const int32_t* pairs, const double* prest,
+             double kp,
+             /* area preservation */ double ka,
+             /* pattern */ const int32_t* row_ptr, const int32_t* col_idx,
+             /* out */ double* g, double* H_vals, double* energy) {
   if (dof != 2 && dof != 3) return OR_ERR_ARG;
   if ((mask & 4) && dof != 2) return OR_ERR_ARG;
+  if ((mask & 16) && dof != 3) return OR_ERR_ARG;
   int bs = dof * dof;
   int64_t n = 0;
   if (mask & 1) n += 4 * (int64_t)nE;
   if (mask & 2) n += V;
   if (mask & 4) n += 9 * (int64_t)nF;
   if (mask & 8) n += 4 * (int64_t)nP;
+  if (mask & 16) n += 9 * (int64_t)nF;
   or_coo c;
   c.bs = bs;
   c.cap = n > 0 ? n : 1;
@@ -390,7 +493,7 @@ int or_eval(int32_t V, int dof, const double* x, unsigned mask,
     return OR_ERR_OOM;
   }
   for (int64_t i = 0; i < (int64_t)V * dof; ++i) g[i] = 0.0;
-  double Etot = 0.0, E, gl[6], Hl[36];
+  double Etot = 0.0, E, gl[9], Hl[81];
   int rc = OR_OK;
   if (mask & 1)
     for (int32_t e = 0; e < nE && !rc; ++e) {
@@ -420,6 +523,16 @@ int or_eval(int32_t V, int dof, const double* x, unsigned mask,
       for (int p = 0; p < 3; ++p)
         for (int a = 0; a < 2; ++a) g[(size_t)vid[p] * 2 + a] += gl[p * 2 + a];
       rc = emit_blocks(&c, 2, 3, vid, Hl);
+    }
+  if (mask & 16)
+    for (int32_t f = 0; f < nF && !rc; ++f) {
+      const int32_t* vid = F + 3 * f;
+      or_area_local(x + (size_t)vid[0] * 3, x + (size_t)vid[1] * 3, x + (size_t)vid[2] * 3,
+                    area[f], ka, &E, gl, Hl);
+      Etot += E;
+      for (int p = 0; p < 3; ++p)
+        for (int a = 0; a < 3; ++a) g[(size_t)vid[p] * 3 + a] += gl[p * 3 + a];
+      rc = emit_blocks(&c, 3, 3, vid, Hl);
     }
   if (mask & 8)
     for (int32_t p = 0; p < nP && !rc; ++p) {
@@ -476,6 +589,15 @@ int or_eval(int32_t V, int dof, const double* x, unsigned mask,
 
 /* Matrix-free product reference: y = H v with H the assembled block CSR
  * (the parameterization workload's Hessian-vector product).               */
+int or_eval(int32_t V, int dof, const double* x, unsigned mask, int32_t nE,
+            const int32_t* edges, const double* L0, double k, const double* xt, double w,
+            int32_t nF, const int32_t* F, const double* Minv, const double* area, int32_t nP,
+            const int32_t* pairs, const double* prest, double kp, const int32_t* row_ptr,
+            const int32_t* col_idx, double* g, double* H_vals, double* energy) {
+  return or_eval2(V, dof, x, mask & ~16u, nE, edges, L0, k, xt, w, nF, F, Minv, area, nP, pairs,
+                  prest, kp, 0.0, row_ptr, col_idx, g, H_vals, energy);
+}
+
 int or_bsr_mv(int32_t V, int dof, const int32_t* row_ptr,
               const int32_t* col_idx, const double* H_vals, const double* v,
               double* y) {
