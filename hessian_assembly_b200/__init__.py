@@ -41,6 +41,7 @@ MAD_TERM_SPRING = 1
 MAD_TERM_INERTIA = 2
 MAD_TERM_SYMDIR = 4
 MAD_TERM_PAIR = 8
+MAD_TERM_AREA = 16
 MAD_EVAL_FULL_STENCIL_AD = 1
 MAD_EVAL_EDGE_SCATTER = 2
 MAD_EVAL_PATCH_STAGED = 4
@@ -67,7 +68,7 @@ class mad_terms(ctypes.Structure):
                 ("spring_rest", ctypes.c_void_p), ("spring_k", ctypes.c_double),
                 ("inertia_xt", ctypes.c_void_p), ("inertia_w", ctypes.c_double),
                 ("face_Minv", ctypes.c_void_p), ("face_area", ctypes.c_void_p),
-                ("pair_k", ctypes.c_double)]
+                ("pair_k", ctypes.c_double), ("area_k", ctypes.c_double)]
 
 
 class mad_info_t(ctypes.Structure):
@@ -189,13 +190,15 @@ class Terms:
     face_Minv: object = None
     face_area: object = None
     pair_k: float = 0.0
+    area_k: float = 0.0
 
     def to_c(self, dtype) -> mad_terms:
         p = lambda t, n: None if t is None else _dev_ptr(t, dtype, n)  # noqa: E731
         return mad_terms(self.mask, self.flags, p(self.spring_rest, "spring_rest"),
                          float(self.spring_k), p(self.inertia_xt, "inertia_xt"),
                          float(self.inertia_w), p(self.face_Minv, "face_Minv"),
-                         p(self.face_area, "face_area"), float(self.pair_k))
+                         p(self.face_area, "face_area"), float(self.pair_k),
+                         float(self.area_k))
 
 
 class Context:

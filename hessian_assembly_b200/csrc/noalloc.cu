@@ -61,6 +61,7 @@ struct NaArgs {
   const int32_t* pairs;
   const T* prest;
   T kp;
+  T ka;
   unsigned mask;
   double* partials;
 };
@@ -72,7 +73,10 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
   const int64_t t = (int64_t)blockIdx.x * kNaThreads + threadIdx.x;
   const int64_t nS = (A.mask & MAD_TERM_SPRING) ? A.nE : 0;
   const int64_t nI = (A.mask & MAD_TERM_INERTIA) ? A.V : 0;
-  const int64_t nFc = (DOF == 2 && (A.mask & MAD_TERM_SYMDIR)) ? A.nF : 0;
+  const int64_t nFc = ((DOF == 2 && (A.mask & MAD_TERM_SYMDIR)) ||
+                       (DOF == 3 && (A.mask & MAD_TERM_AREA)))
+                          ? A.nF
+                          : 0;
   const int64_t nPr = (A.mask & MAD_TERM_PAIR) ? A.nP : 0;
   double e = 0.0;
   if (t < nS) {
@@ -101,6 +105,18 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
         for (int ga = 0; ga < 2; ++ga)
           j[2 * al + ga] = (u1[al] - u0[al]) * M[ga] + (u2[al] - u0[al]) * M[2 + ga];
       e = (double)symdir_energy(j, A.area[f]);
+    } else {
+      const int64_t f = t - nS - nI;
+      const T* u0 = A.x + (int64_t)A.F[3 * f] * 3;
+      const T* u1 = A.x + (int64_t)A.F[3 * f + 1] * 3;
+      const T* u2 = A.x + (int64_t)A.F[3 * f + 2] * 3;
+      T e1[3], e2[3];
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        e1[a] = u1[a] - u0[a];
+        e2[a] = u2[a] - u0[a];
+      }
+      e = (double)area_energy(e1, e2, A.area[f], A.ka);
     }
   } else if (t < nS + nI + nFc + nPr) {
     const int64_t p = t - nS - nI - nFc;
@@ -163,19 +179,23 @@ extern "C" mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, c
       (dt != MAD_F32 && dt != MAD_F64) || !t || !energy) {
     return MAD_ERR_INVALID_ARG;
   }
-  const unsigned known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR;
+  const unsigned known =
+      MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR | MAD_TERM_AREA;
   if (t->mask & ~known) {
     return MAD_ERR_INVALID_ARG;
   }
   const bool sp = (t->mask & MAD_TERM_SPRING) && nE > 0;
   const bool in = (t->mask & MAD_TERM_INERTIA) && V > 0;
-  const bool fa = (t->mask & MAD_TERM_SYMDIR) && nF > 0;
+  const bool sd = (t->mask & MAD_TERM_SYMDIR) && nF > 0;
+  const bool ar = (t->mask & MAD_TERM_AREA) && nF > 0;
+  const bool fa = sd || ar;
   const bool pa = (t->mask & MAD_TERM_PAIR) && nP > 0;
-  if ((t->mask & MAD_TERM_SYMDIR) && dof != 2) {
+  if (((t->mask & MAD_TERM_SYMDIR) && dof != 2) || ((t->mask & MAD_TERM_AREA) && dof != 3)) {
     return MAD_ERR_UNIMPLEMENTED;
   }
   if ((V > 0 && !x) || (sp && (!edges || !t->spring_rest)) || (in && !t->inertia_xt) ||
-      (fa && (!F || !t->face_Minv || !t->face_area)) || (pa && (!pairs || !pair_rest))) {
+      (sd && (!F || !t->face_Minv || !t->face_area)) || (ar && (!F || !t->face_area)) ||
+      (pa && (!pairs || !pair_rest))) {
     return MAD_ERR_INVALID_ARG;
   }
   const int64_t terms = (sp ? (int64_t)nE : 0) + (in ? (int64_t)V : 0) + (fa ? (int64_t)nF : 0) +
@@ -191,18 +211,20 @@ extern "C" mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, c
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const unsigned mask = (sp ? MAD_TERM_SPRING : 0u) | (in ? MAD_TERM_INERTIA : 0u) |
-                        (fa ? MAD_TERM_SYMDIR : 0u) | (pa ? MAD_TERM_PAIR : 0u);
+                        (sd ? MAD_TERM_SYMDIR : 0u) | (ar ? MAD_TERM_AREA : 0u) |
+                        (pa ? MAD_TERM_PAIR : 0u);
   if (dt == MAD_F64) {
     mad::NaArgs<double> A{V, nE, nF, nP, (const double*)x, edges, (const double*)t->spring_rest,
                      t->spring_k, (const double*)t->inertia_xt, t->inertia_w, F,
                      (const double*)t->face_Minv, (const double*)t->face_area, pairs,
-                     (const double*)pair_rest, t->pair_k, mask, partials};
+                     (const double*)pair_rest, t->pair_k, t->area_k, mask, partials};
     e = mad::run(A, dof, (int)blocks, energy, s);
   } else {
     mad::NaArgs<float> A{V, nE, nF, nP, (const float*)x, edges, (const float*)t->spring_rest,
                     (float)t->spring_k, (const float*)t->inertia_xt, (float)t->inertia_w, F,
                     (const float*)t->face_Minv, (const float*)t->face_area, pairs,
-                    (const float*)pair_rest, (float)t->pair_k, mask, partials};
+                    (const float*)pair_rest, (float)t->pair_k, (float)t->area_k, mask,
+                    partials};
     e = mad::run(A, dof, (int)blocks, energy, s);
   }
   if (e != cudaSuccess) {

@@ -66,6 +66,7 @@ struct RArgs {
   const T* xt;
   T w;
   T kp;
+  T ka;  // area-preservation stiffness
   unsigned mask;
   double* epart;
   int V, s0, sf, wstage;  // wstage: staging elements per warp
@@ -252,6 +253,49 @@ __device__ __forceinline__ void row_faces(const RArgs<T>& A, int i, int tile, in
   }
 }
 
+// The dof-3 face terms of row i: calls on_face(xj, xk, c, pj, pk, A0) for
+// every face with vertex i as a corner (same table as row_faces).
+template <typename T, typename OnFace>
+__device__ __forceinline__ void row_faces3(const RArgs<T>& A, int i, int tile, int lane,
+                                           OnFace on_face) {
+  constexpr uint32_t kPm = (1u << kFacePosBits) - 1u;
+  auto one = [&](const int4& e) {
+    const int j = e.y, k = e.z & 0x7FFFFFFF;
+    const uint32_t w = (uint32_t)e.w;
+    T xj[3], xk[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      xj[a] = A.x[(uint32_t)(j * 3 + a)];
+      xk[a] = A.x[(uint32_t)(k * 3 + a)];
+    }
+    on_face(xj, xk, (int)(w & 3u), (int)((w >> 2) & kPm), (int)(w >> (2 + kFacePosBits)),
+            A.area[e.x]);
+  };
+  const int4* p = A.fslots + (uint32_t)(tile * A.sf * 32 + lane);
+  int4 e = p[0];
+  bool more = false;
+#pragma unroll 1
+  for (int k = 0; k < A.sf; ++k) {  // a row's entries fill a prefix of its slots
+    if (e.x < 0) break;
+    const int4 en = k + 1 < A.sf ? p[(uint32_t)((k + 1) * 32)] : make_int4(-1, 0, 0, 0);
+    if (k == kFaceRowSlots - 1) more = e.z < 0;  // the overflow mark
+    one(e);
+    e = en;
+  }
+  if (more) {
+    const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
+#pragma unroll 1
+    for (int q = o0; q < o1; ++q) one(A.fofl[q]);
+  }
+}
+
+// b[0..8] += v[0..8]
+template <typename T>
+__device__ __forceinline__ void add9(T* b, const T* v) {
+#pragma unroll
+  for (int q = 0; q < 9; ++q) b[q] += v[q];
+}
+
 // b[0..3] += v[0..3] (16-byte accesses when b allows them)
 template <typename T>
 __device__ __forceinline__ void add4(T* b, const T* v) {
@@ -346,6 +390,27 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                                 apply_edge_side<true>(R, 0, acc, row + op * B, gr);
                                 if (ENERGY) energy += 0.5 * (double)edge_energy(R);
                               });
+    }
+  }
+  if constexpr (FACES && DOF == 3) {
+    // area preservation after the edge terms, which store their blocks
+    if (A.mask & MAD_TERM_AREA) {
+      row_faces3<T>(A, i, tile, lane,
+                    [&](const T* xj, const T* xk, int c, int pj, int pk, T A0) {
+                      FaceRow3<T> o;
+                      eval_area_row<T, FULL>(xi, xj, xk, c, A0, A.ka, o);
+#pragma unroll
+                      for (int a = 0; a < 3; ++a)
+#pragma unroll
+                        for (int b = a; b < 3; ++b) acc[Tri<3>::idx(a, b)] += o.H[0][3 * a + b];
+#pragma unroll
+                      for (int a = 0; a < 3; ++a) gr[a] += o.g[a];
+                      const int oj = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pj) : pj;
+                      const int ok = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pk) : pk;
+                      add9<T>(row + oj * B, o.H[1]);
+                      add9<T>(row + ok * B, o.H[2]);
+                      if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
+                    });
     }
   }
   if constexpr (FACES && DOF == 2) {
@@ -535,8 +600,8 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
                               });
     }
   }
-  if constexpr (FACES && DOF == 2) {
-    if (A.mask & MAD_TERM_SYMDIR) {
+  if constexpr (FACES) {
+    if (A.mask & (DOF == 2 ? MAD_TERM_SYMDIR : MAD_TERM_AREA)) {
       // the row's corners' results of the per-face pass (k_face_hv)
       constexpr int SF = kFaceRowSlots;
       int32_t e[SF];
@@ -547,15 +612,15 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
       for (int k = 0; k < SF; ++k) {
         if (e[k] == -1) continue;
         const uint32_t q = (uint32_t)e[k] & 0x7FFFFFFFu;
-        yr[0] += A.fhv[2 * q];
-        yr[1] += A.fhv[2 * q + 1];
+#pragma unroll
+        for (int a = 0; a < DOF; ++a) yr[a] += A.fhv[DOF * q + a];
       }
       if (e[SF - 1] != -1 && e[SF - 1] < 0) {  // the row continues in the overflow table
         const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
         for (int q = o0; q < o1; ++q) {
           const uint32_t fc = (uint32_t)A.fcofl[q];
-          yr[0] += A.fhv[2 * fc];
-          yr[1] += A.fhv[2 * fc + 1];
+#pragma unroll
+          for (int a = 0; a < DOF; ++a) yr[a] += A.fhv[DOF * fc + a];
         }
       }
     }
@@ -578,6 +643,32 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   (void)TD;
 #pragma unroll
   for (int a = 0; a < DOF; ++a) A.y[(uint32_t)(i * DOF + a)] = yr[a];
+}
+
+// Per-face pass of the Hessian-vector product for area-preservation faces
+// (dof 3): one thread per face writes (H_f v_f) for its three corners.
+template <typename T, bool FULL>
+__global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __restrict__ F,
+                                                      const T* __restrict__ x,
+                                                      const T* __restrict__ v,
+                                                      const T* __restrict__ area, T ka,
+                                                      T* __restrict__ out) {
+  const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (f >= nF) return;
+  T u[3][3], w[3][3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    const int32_t vid = F[3 * f + c];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      u[c][a] = x[(int64_t)vid * 3 + a];
+      w[c][a] = v[(int64_t)vid * 3 + a];
+    }
+  }
+  T o[9];
+  hv_area_face<T, FULL>(u[0], u[1], u[2], w[0], w[1], w[2], area[f], ka, o);
+#pragma unroll
+  for (int q = 0; q < 9; ++q) out[9 * f + q] = o[q];
 }
 
 // Per-face pass of the Hessian-vector product: one thread per face computes
@@ -667,6 +758,7 @@ RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, cons
   A.xt = (const T*)t.inertia_xt;
   A.w = (T)t.inertia_w;
   A.kp = (T)t.pair_k;
+  A.ka = (T)t.area_k;
   A.mask = t.mask;
   A.epart = energy ? L.epart : nullptr;
   A.V = L.V;
@@ -737,13 +829,13 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   const bool pairs = L.prow != nullptr;
   const bool en = energy != nullptr;
   cudaError_t e;
-  if (DOF == 2 && (t.mask & MAD_TERM_SYMDIR)) {
+  if ((DOF == 2 && (t.mask & MAD_TERM_SYMDIR)) || (DOF == 3 && (t.mask & MAD_TERM_AREA))) {
     // face terms: the face-row instantiations; without edge terms the kernel
     // carries no edge-slot code (S0 = 0)
     if (t.mask & MAD_TERM_SPRING)
-      e = eval_k4<T, DOF, kS0Max, DOF == 2>(A, full, en, pairs, nb, smem, s);
+      e = eval_k4<T, DOF, kS0Max, true>(A, full, en, pairs, nb, smem, s);
     else
-      e = eval_k4<T, DOF, 0, DOF == 2>(A, full, en, pairs, nb, smem, s);
+      e = eval_k4<T, DOF, 0, true>(A, full, en, pairs, nb, smem, s);
   } else if (L.s0 <= 6) {
     // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
     // narrower instantiation: fewer registers
@@ -790,6 +882,33 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
       return cudaGetLastError();
     }
   }
+  if constexpr (DOF == 3) {
+    if (t.mask & MAD_TERM_AREA) {
+      if (L.nF > 0) {
+        const unsigned nbf = (unsigned)((L.nF + 255) / 256);
+        if (full)
+          k_face_hv_area<T, true><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
+                                                      (const T*)t.face_area, (T)t.area_k,
+                                                      (T*)L.fhv);
+        else
+          k_face_hv_area<T, false><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
+                                                       (const T*)t.face_area, (T)t.area_k,
+                                                       (T*)L.fhv);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+      }
+      const bool sp = t.mask & MAD_TERM_SPRING;
+      if (sp && full)
+        k_rows_hvp<T, DOF, true, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
+      else if (sp)
+        k_rows_hvp<T, DOF, false, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
+      else if (full)
+        k_rows_hvp<T, DOF, true, 0, true><<<nb, kRowThreads, 0, s>>>(A);
+      else
+        k_rows_hvp<T, DOF, false, 0, true><<<nb, kRowThreads, 0, s>>>(A);
+      return cudaGetLastError();
+    }
+  }
   if (L.s0 <= 6) {
     if (full)
       k_rows_hvp<T, DOF, true, 6, false><<<nb, kRowThreads, 0, s>>>(A);
@@ -813,13 +932,11 @@ cudaError_t set_rows_limits(size_t bytes) {
   if ((e = eval_k4<T, DOF, kS0Max, false>(A, false, false, false, 0, bytes, 0, true)) !=
       cudaSuccess)
     return e;
-  if constexpr (DOF == 2) {
-    if ((e = eval_k4<T, DOF, kS0Max, true>(A, false, false, false, 0, bytes, 0, true)) !=
-        cudaSuccess)
-      return e;
-    if ((e = eval_k4<T, DOF, 0, true>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
-      return e;
-  }
+  if ((e = eval_k4<T, DOF, kS0Max, true>(A, false, false, false, 0, bytes, 0, true)) !=
+      cudaSuccess)
+    return e;
+  if ((e = eval_k4<T, DOF, 0, true>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+    return e;
   return cudaSuccess;
 }
 

@@ -84,6 +84,34 @@ __device__ __forceinline__ auto symdir_energy(const S (&j)[4], T A) {
   return a * symdir_scale(det, A);
 }
 
+// Area preservation of a 3D triangle: with n = e1 x e2 (e1 = x1 - x0,
+// e2 = x2 - x0) and s = n.n, A = sqrt(s) / 2 and E = k/2 (A - A0)^2 / A0 is a
+// univariate function of s: f'(s) = (k/A0)(A - A0) / (8A), f''(s) =
+// k / (64 A^3) (from dA/ds = 1/(8A), d2A/ds2 = -1/(64 A^3)), applied as one
+// chain step on the AD number s.
+template <typename T>
+__device__ __forceinline__ T area_of_s(T s, T A0, T k) {
+  const T A = T(0.5) * sqrt(s);
+  return (T(0.5) * k / A0) * (A - A0) * (A - A0);
+}
+template <typename T, int N>
+__device__ __forceinline__ HyperDual<T, N> area_of_s(const HyperDual<T, N>& s, T A0, T k) {
+  const T A = T(0.5) * ::sqrt(s.v);
+  const T iA = T(1) / A;
+  const T f1 = (k / A0) * (A - A0) * (T(0.125) * iA);
+  const T f2 = k * (T(1) / T(64)) * (iA * iA * iA);
+  return chain(s, (T(0.5) * k / A0) * (A - A0) * (A - A0), f1, f2);
+}
+
+template <typename S, typename T>
+__device__ __forceinline__ auto area_energy(const S (&e1)[3], const S (&e2)[3], T A0, T k) {
+  auto n0 = e1[1] * e2[2] - e1[2] * e2[1];
+  auto n1 = e1[2] * e2[0] - e1[0] * e2[2];
+  auto n2 = e1[0] * e2[1] - e1[1] * e2[0];
+  auto s = sq(n0) + sq(n1) + sq(n2);
+  return area_of_s(s, A0, k);
+}
+
 // ---------------------------------------------------------------- results
 // Edge / pair term: blocks are D x D row-major; the (b, a) block is the
 // transpose of Hab.
@@ -404,6 +432,142 @@ __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const 
       for (int al = 0; al < 2; ++al)
 #pragma unroll
         for (int be = 0; be < 2; ++be) o.H[l][2 * al + be] = hess(e, al, 2 * l + be);
+  }
+}
+
+// One corner's share of an area-preservation face (dof 3): gradient g_i and
+// the blocks (i,i), (i,j), (i,k) (row-major 3x3) for the row of vertex i,
+// the face's corners being (i, j, k) rotated by c as for FaceRow.  Reduced
+// seeding on (e1, e2) (width 6) in the face's own corner order; a corner's
+// coefficients on e1 and e2 are p1 = (-1, 1, 0), p2 = (-1, 0, 1), so block
+// (a, b) = sum_{s,t} p_s[a] p_t[b] H_(s,t).
+template <typename T>
+struct FaceRow3 {
+  T E;
+  T g[3];
+  T H[3][9];  // (i,i), (i,j), (i,k)
+};
+
+template <typename T, bool FULL>
+__device__ __forceinline__ void eval_area_row(const T* xi, const T* xj, const T* xk, int c, T A0,
+                                              T k, FaceRow3<T>& o) {
+  if constexpr (!FULL) {
+    Lin<T, 6> e1[3], e2[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      const T u0 = sel3(c, xi[a], xk[a], xj[a]);
+      const T u1 = sel3(c, xj[a], xi[a], xk[a]);
+      const T u2 = sel3(c, xk[a], xj[a], xi[a]);
+      e1[a] = lin_var<T, 6>(u1 - u0, a);
+      e2[a] = lin_var<T, 6>(u2 - u0, 3 + a);
+    }
+    const HyperDual<T, 6> e = area_energy(e1, e2, A0, k);
+    o.E = e.v;
+    // coefficients of corners c, c+1, c+2 (face order) on e1 and e2
+    T p1[3], p2[3];
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      const int a = m == 0 ? c : (m == 1 ? (c == 2 ? 0 : c + 1) : (c == 0 ? 2 : c - 1));
+      p1[m] = a == 0 ? T(-1) : (a == 1 ? T(1) : T(0));
+      p2[m] = a == 0 ? T(-1) : (a == 2 ? T(1) : T(0));
+    }
+#pragma unroll
+    for (int al = 0; al < 3; ++al) o.g[al] = p1[0] * e.g[al] + p2[0] * e.g[3 + al];
+#pragma unroll
+    for (int m = 0; m < 3; ++m)
+#pragma unroll
+      for (int al = 0; al < 3; ++al)
+#pragma unroll
+        for (int be = 0; be < 3; ++be)
+          o.H[m][3 * al + be] = p1[0] * (p1[m] * hess(e, al, be) + p2[m] * hess(e, al, 3 + be)) +
+                                p2[0] * (p1[m] * hess(e, 3 + al, be) +
+                                         p2[m] * hess(e, 3 + al, 3 + be));
+  } else {
+    // width-9 AD over (x_i, x_j, x_k)
+    Lin<T, 9> ui[3], uj[3], uk[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      ui[a] = lin_var<T, 9>(xi[a], a);
+      uj[a] = lin_var<T, 9>(xj[a], 3 + a);
+      uk[a] = lin_var<T, 9>(xk[a], 6 + a);
+    }
+    Lin<T, 9> e1[3], e2[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      const Lin<T, 9> u0 = c == 0 ? ui[a] : (c == 1 ? uk[a] : uj[a]);
+      const Lin<T, 9> u1 = c == 0 ? uj[a] : (c == 1 ? ui[a] : uk[a]);
+      const Lin<T, 9> u2 = c == 0 ? uk[a] : (c == 1 ? uj[a] : ui[a]);
+      e1[a] = u1 - u0;
+      e2[a] = u2 - u0;
+    }
+    const HyperDual<T, 9> e = area_energy(e1, e2, A0, k);
+    o.E = e.v;
+#pragma unroll
+    for (int al = 0; al < 3; ++al) o.g[al] = e.g[al];
+#pragma unroll
+    for (int m = 0; m < 3; ++m)
+#pragma unroll
+      for (int al = 0; al < 3; ++al)
+#pragma unroll
+        for (int be = 0; be < 3; ++be) o.H[m][3 * al + be] = hess(e, al, 3 * m + be);
+  }
+}
+
+// (H v) of one area-preservation face for its three corners (face order):
+// out[3a + al].  Reduced form: t = H_e dE with dE = (v1 - v0, v2 - v0), then
+// corner a takes p1[a] t_e1 + p2[a] t_e2.
+template <typename T, bool FULL>
+__device__ __forceinline__ void hv_area_face(const T* u0, const T* u1, const T* u2,
+                                             const T* v0, const T* v1, const T* v2, T A0, T k,
+                                             T* out) {
+  if constexpr (!FULL) {
+    Lin<T, 6> e1[3], e2[3];
+    T d[6];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      e1[a] = lin_var<T, 6>(u1[a] - u0[a], a);
+      e2[a] = lin_var<T, 6>(u2[a] - u0[a], 3 + a);
+      d[a] = v1[a] - v0[a];
+      d[3 + a] = v2[a] - v0[a];
+    }
+    const HyperDual<T, 6> e = area_energy(e1, e2, A0, k);
+    T t[6];
+#pragma unroll
+    for (int p = 0; p < 6; ++p) {
+      T s = T(0);
+#pragma unroll
+      for (int q = 0; q < 6; ++q) s += hess(e, p, q) * d[q];
+      t[p] = s;
+    }
+#pragma unroll
+    for (int al = 0; al < 3; ++al) {
+      out[al] = -(t[al] + t[3 + al]);
+      out[3 + al] = t[al];
+      out[6 + al] = t[3 + al];
+    }
+  } else {
+    Lin<T, 9> x[3][3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      x[0][a] = lin_var<T, 9>(u0[a], a);
+      x[1][a] = lin_var<T, 9>(u1[a], 3 + a);
+      x[2][a] = lin_var<T, 9>(u2[a], 6 + a);
+    }
+    Lin<T, 9> e1[3], e2[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      e1[a] = x[1][a] - x[0][a];
+      e2[a] = x[2][a] - x[0][a];
+    }
+    const HyperDual<T, 9> e = area_energy(e1, e2, A0, k);
+    const T* vv[3] = {v0, v1, v2};
+#pragma unroll
+    for (int p = 0; p < 9; ++p) {
+      T s = T(0);
+#pragma unroll
+      for (int q = 0; q < 9; ++q) s += hess(e, p, q) * vv[q / 3][q % 3];
+      out[p] = s;
+    }
   }
 }
 
