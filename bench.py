@@ -283,6 +283,18 @@ def cpu_baseline_rows(st):
     orc.jacobian(st["V"], 3, xx, 3, edges=st["edges"], L0=st["L0"], k=st["k"], xt=st["xt"],
                  w=st["w"])
     res["jac1000_ms"] = round((time.perf_counter() - t0) * 1e3, 1)
+    # springs + inertia + area at 1000^2: assembly on the base pattern, then the product
+    xx = mi.cloth_x(N_GRID, 1007, 0, np.float32)
+    rp, ci = orc.pattern(st["V"], st["F"])
+    t0 = time.perf_counter()
+    _, oH, _ = orc.eval(st["V"], 3, xx, 19, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
+                        xt=st["xt"], w=st["w"], F=st["F"],
+                        area=cloth_rest_area(st).astype(np.float32), ka=AREA_K)
+    t1 = time.perf_counter()
+    orc.bsr_mv(st["V"], 3, rp, ci, oH, mi.probe_vector(st["V"], 3, 1008, np.float32))
+    t2 = time.perf_counter()
+    res["area1000_eval_ms"] = round((t1 - t0) * 1e3, 1)
+    res["area1000_hvp_ms"] = round((t2 - t1) * 1e3, 1)
     res["unit"] = "ms per call, 1 core, one run"
     return res
 
@@ -303,7 +315,7 @@ def cpu_baseline(st):
             "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
 
 
-EXTRA = ("cloth_small", "symdir500", "pairs1000", "jac1000")
+EXTRA = ("cloth_small", "symdir500", "pairs1000", "jac1000", "area1000")
 
 
 def extra_workloads(args, only=None):
@@ -366,7 +378,45 @@ def extra_workloads(args, only=None):
         pairs1000(res, mad, torch, dev, stream)
     if run("jac1000"):
         jac1000(res, mad, torch, dev, stream, timeit)
+    if run("area1000"):
+        area1000(res, mad, torch, dev, stream, timeit)
     return res
+
+
+def cloth_rest_area(st):
+    X, F = st["X"], st["F"]
+    return 0.5 * np.linalg.norm(np.cross(X[F[:, 1]] - X[F[:, 0]], X[F[:, 2]] - X[F[:, 0]]), axis=1)
+
+
+AREA_K = 2.0e3
+
+
+def area1000(res, mad, torch, dev, stream, timeit):
+    """Springs + inertia + area preservation (3-DOF face term) on the 1000^2
+    cloth: assembly of g and H, and the matrix-free product.  Compulsory bytes:
+    the headline step plus the faces and their rest areas (assembly); x, v,
+    edges, L0, faces, rest areas in and y out (product)."""
+    st = mi.cloth_static(N_GRID, np.float32)
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    terms = mad.Terms(mask=19, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
+                      inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"],
+                      face_area=torch.from_numpy(cloth_rest_area(st).astype(np.float32)).to(dev),
+                      area_k=AREA_K)
+    x = torch.from_numpy(mi.cloth_x(N_GRID, 1007, 0, np.float32)).to(dev)
+    v = torch.from_numpy(mi.probe_vector(st["V"], 3, 1008, np.float32)).to(dev)
+    g = torch.empty((st["V"], 3), device=dev)
+    y = torch.empty((st["V"], 3), device=dev)
+    H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
+    nF = len(st["F"])
+    eb = ALGO_BYTES + 16 * nF
+    hb = 12 * V_FULL * 3 + 12 * E_FULL + 16 * nF
+    ms = timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream))
+    res["area1000_eval_ms"] = round(ms, 5)
+    res["area1000_eval_gbs"] = round(eb / (ms * 1e-3) / 1e9, 1)
+    ms = timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream))
+    res["area1000_hvp_ms"] = round(ms, 5)
+    res["area1000_hvp_gbs"] = round(hb / (ms * 1e-3) / 1e9, 1)
+    ctx.close()
 
 
 def jac1000(res, mad, torch, dev, stream, timeit):
