@@ -140,17 +140,6 @@ __device__ __forceinline__ int block_excl_scan(int v, int* total) {
   return before + incl - v;
 }
 
-// Sum of the counts of every block before this one: whole super tiles, then
-// the blocks of this block's super tile.
-__device__ __forceinline__ int blocks_before(const int32_t* __restrict__ sup,
-                                             const int32_t* __restrict__ blk) {
-  const int b = blockIdx.x, S = b / kSuper;
-  int s = 0;
-  for (int q = threadIdx.x; q < S; q += kB) s += sup[q];
-  if ((int)threadIdx.x < b - S * kSuper) s += blk[S * kSuper + threadIdx.x];
-  return block_sum(s);
-}
-
 __global__ void __launch_bounds__(kB) k_pair_count(const int32_t* __restrict__ ij, int n, int V,
                                                    int32_t* cnt, int32_t* status) {
   GRID_STRIDE(p, n) {

@@ -396,9 +396,9 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
     // area preservation after the edge terms, which store their blocks
     if (A.mask & MAD_TERM_AREA) {
       row_faces3<T>(A, i, tile, lane,
-                    [&](const T* xj, const T* xk, int c, int pj, int pk, T A0) {
+                    [&](const T* xj, const T* xk, int, int pj, int pk, T A0) {
                       FaceRow3<T> o;
-                      eval_area_row<T, FULL>(xi, xj, xk, c, A0, A.ka, o);
+                      eval_area_row<T, FULL>(xi, xj, xk, A0, A.ka, o);
 #pragma unroll
                       for (int a = 0; a < 3; ++a)
 #pragma unroll

@@ -26,6 +26,7 @@
 #pragma once
 
 #include "dual.cuh"
+#include "sparse_ad.cuh"
 
 namespace mad {
 
@@ -41,8 +42,8 @@ __device__ __forceinline__ T spring_of_s(T s, T L0, T k) {
   const T r = sqrt(s) - L0;
   return (T(0.5) * k) * (r * r);
 }
-template <typename T, int N>
-__device__ __forceinline__ HyperDual<T, N> spring_of_s(const HyperDual<T, N>& s, T L0, T k) {
+template <typename S, typename T>
+__device__ __forceinline__ auto spring_chain(const S& s, T L0, T k) {
   const T il = rsqrt(s.v);
   const T l = s.v * il;
   const T r = l - L0;
@@ -50,6 +51,14 @@ __device__ __forceinline__ HyperDual<T, N> spring_of_s(const HyperDual<T, N>& s,
   const T f1 = hk * r * il;
   const T f2 = (T(0.5) * hk) * L0 * (il * il * il);
   return chain(s, hk * (r * r), f1, f2);
+}
+template <typename T, int N>
+__device__ __forceinline__ HyperDual<T, N> spring_of_s(const HyperDual<T, N>& s, T L0, T k) {
+  return spring_chain(s, L0, k);
+}
+template <typename T, int N, uint32_t G, uint64_t H>
+__device__ __forceinline__ auto spring_of_s(const SHD<T, N, G, H>& s, T L0, T k) {
+  return spring_chain(s, L0, k);
 }
 
 template <typename S, int D, typename T>
@@ -94,13 +103,21 @@ __device__ __forceinline__ T area_of_s(T s, T A0, T k) {
   const T A = T(0.5) * sqrt(s);
   return (T(0.5) * k / A0) * (A - A0) * (A - A0);
 }
-template <typename T, int N>
-__device__ __forceinline__ HyperDual<T, N> area_of_s(const HyperDual<T, N>& s, T A0, T k) {
+template <typename S, typename T>
+__device__ __forceinline__ auto area_chain(const S& s, T A0, T k) {
   const T A = T(0.5) * ::sqrt(s.v);
   const T iA = T(1) / A;
   const T f1 = (k / A0) * (A - A0) * (T(0.125) * iA);
   const T f2 = k * (T(1) / T(64)) * (iA * iA * iA);
   return chain(s, (T(0.5) * k / A0) * (A - A0) * (A - A0), f1, f2);
+}
+template <typename T, int N>
+__device__ __forceinline__ HyperDual<T, N> area_of_s(const HyperDual<T, N>& s, T A0, T k) {
+  return area_chain(s, A0, k);
+}
+template <typename T, int N, uint32_t G, uint64_t H>
+__device__ __forceinline__ auto area_of_s(const SHD<T, N, G, H>& s, T A0, T k) {
+  return area_chain(s, A0, k);
 }
 
 template <typename S, typename T>
@@ -110,6 +127,18 @@ __device__ __forceinline__ auto area_energy(const S (&e1)[3], const S (&e2)[3], 
   auto n2 = e1[0] * e2[1] - e1[1] * e2[0];
   auto s = sq(n0) + sq(n1) + sq(n2);
   return area_of_s(s, A0, k);
+}
+// The same energy on masked AD numbers (sparse_ad.cuh), where each component
+// of e1 and e2 has its own type.
+template <typename A0_, typename A1_, typename A2_, typename B0_, typename B1_, typename B2_,
+          typename T>
+__device__ __forceinline__ auto area_energy_m(const A0_& a0, const A1_& a1, const A2_& a2,
+                                              const B0_& b0, const B1_& b1, const B2_& b2, T A0,
+                                              T k) {
+  const auto n0 = a1 * b2 - a2 * b1;
+  const auto n1 = a2 * b0 - a0 * b2;
+  const auto n2 = a0 * b1 - a1 * b0;
+  return area_of_s(sq(n0) + sq(n1) + sq(n2), A0, k);
 }
 
 // ---------------------------------------------------------------- results
@@ -126,45 +155,40 @@ template <typename T, int D, bool FULL>
 __device__ __forceinline__ void eval_edge(const T* xa, const T* xb, T L0, T k,
                                           EdgeDerivs<T, D>& o) {
   if constexpr (!FULL) {
-    Lin<T, D> d[D];
+    T d[D];
 #pragma unroll
-    for (int a = 0; a < D; ++a) d[a] = lin_var<T, D>(xa[a] - xb[a], a);
-    HyperDual<T, D> e = spring_energy(d, L0, k);
+    for (int a = 0; a < D; ++a) d[a] = xa[a] - xb[a];
+    const auto e = spring_of_s(sqnorm_m<T, D>(d), L0, k);
     o.E = e.v;
 #pragma unroll
     for (int a = 0; a < D; ++a) {
-      o.ga[a] = e.g[a];
-      o.gb[a] = -e.g[a];
+      o.ga[a] = sgrad(e, a);
+      o.gb[a] = -sgrad(e, a);
     }
 #pragma unroll
     for (int a = 0; a < D; ++a)
 #pragma unroll
       for (int b = 0; b < D; ++b) {
-        const T K = hess(e, a, b);
+        const T K = shess(e, a, b);
         o.Haa[a * D + b] = K;
         o.Hbb[a * D + b] = K;
         o.Hab[a * D + b] = -K;
       }
   } else {
-    constexpr int N = 2 * D;
-    Lin<T, N> d[D];
-#pragma unroll
-    for (int a = 0; a < D; ++a)
-      d[a] = lin_var<T, N>(xa[a], a) - lin_var<T, N>(xb[a], D + a);
-    HyperDual<T, N> e = spring_energy(d, L0, k);
+    const auto e = spring_of_s(sqdist_m<T, D>(xa, xb), L0, k);
     o.E = e.v;
 #pragma unroll
     for (int a = 0; a < D; ++a) {
-      o.ga[a] = e.g[a];
-      o.gb[a] = e.g[D + a];
+      o.ga[a] = sgrad(e, a);
+      o.gb[a] = sgrad(e, D + a);
     }
 #pragma unroll
     for (int a = 0; a < D; ++a)
 #pragma unroll
       for (int b = 0; b < D; ++b) {
-        o.Haa[a * D + b] = hess(e, a, b);
-        o.Hab[a * D + b] = hess(e, a, D + b);
-        o.Hbb[a * D + b] = hess(e, D + a, D + b);
+        o.Haa[a * D + b] = shess(e, a, b);
+        o.Hab[a * D + b] = shess(e, a, D + b);
+        o.Hbb[a * D + b] = shess(e, D + a, D + b);
       }
   }
 }
@@ -188,15 +212,17 @@ template <typename T, int D, bool FULL>
 __device__ __forceinline__ void eval_edge_res(const T* xa, const T* xb, T L0, T k,
                                               EdgeRes<T, D, FULL>& R) {
   if constexpr (!FULL) {
-    Lin<T, D> d[D];
+    T d[D];
 #pragma unroll
-    for (int a = 0; a < D; ++a) d[a] = lin_var<T, D>(xa[a] - xb[a], a);
-    HyperDual<T, D> e = spring_energy(d, L0, k);
+    for (int a = 0; a < D; ++a) d[a] = xa[a] - xb[a];
+    const auto e = spring_of_s(sqnorm_m<T, D>(d), L0, k);
     R.E = e.v;
 #pragma unroll
-    for (int a = 0; a < D; ++a) R.g[a] = e.g[a];
+    for (int a = 0; a < D; ++a) R.g[a] = sgrad(e, a);
 #pragma unroll
-    for (int q = 0; q < Tri<D>::size; ++q) R.K[q] = e.h[q];
+    for (int a = 0; a < D; ++a)
+#pragma unroll
+      for (int b = a; b < D; ++b) R.K[Tri<D>::idx(a, b)] = shess(e, a, b);
   } else {
     eval_edge<T, D, true>(xa, xb, L0, k, R.d);
   }
@@ -248,17 +274,17 @@ __device__ __forceinline__ T edge_energy(const EdgeRes<T, D, FULL>& R) {
 template <typename T, int D>
 __device__ __forceinline__ void eval_inertia(const T* x, const T* xt, T w, T& E, T* g,
                                              T* Hd) {
-  HyperDual<T, D> s = sq(lin_var<T, D>(x[0] - xt[0], 0));
+  T r[D];
 #pragma unroll
-  for (int a = 1; a < D; ++a) s = s + sq(lin_var<T, D>(x[a] - xt[a], a));
-  HyperDual<T, D> e = s * (T(0.5) * w);
+  for (int a = 0; a < D; ++a) r[a] = x[a] - xt[a];
+  const auto e = sqnorm_m<T, D>(r) * (T(0.5) * w);
   E = e.v;
 #pragma unroll
-  for (int a = 0; a < D; ++a) g[a] = e.g[a];
+  for (int a = 0; a < D; ++a) g[a] = sgrad(e, a);
 #pragma unroll
   for (int a = 0; a < D; ++a)
 #pragma unroll
-    for (int b = 0; b < D; ++b) Hd[a * D + b] = hess(e, a, b);
+    for (int b = 0; b < D; ++b) Hd[a * D + b] = shess(e, a, b);
 }
 
 // Symmetric Dirichlet face term in 2D.  u0, u1, u2 are the corners' UV, M the
@@ -437,10 +463,14 @@ __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const 
 
 // One corner's share of an area-preservation face (dof 3): gradient g_i and
 // the blocks (i,i), (i,j), (i,k) (row-major 3x3) for the row of vertex i,
-// the face's corners being (i, j, k) rotated by c as for FaceRow.  Reduced
-// seeding on (e1, e2) (width 6) in the face's own corner order; a corner's
-// coefficients on e1 and e2 are p1 = (-1, 1, 0), p2 = (-1, 0, 1), so block
-// (a, b) = sum_{s,t} p_s[a] p_t[b] H_(s,t).
+// with (i, j, k) the face's corners rotated so that i comes first.  A cyclic
+// rotation leaves n = e1 x e2 unchanged, so the row evaluates the face with
+// e1 = x_j - x_i and e2 = x_k - x_i.  Reduced seeding on (e1, e2) (width 6):
+// corner i's coefficients on (e1, e2) are (-1, -1), j's (1, 0) and k's
+// (0, 1), so block (a, b) = sum_{s,t} p_s[a] p_t[b] H_(s,t) becomes
+//   (i,i) = H11 + H12 + H21 + H22,  (i,j) = -(H11 + H21),  (i,k) = -(H12 + H22).
+// Both seedings run on the masked AD numbers: the e components are single
+// variables (reduced) or differences of two (full).
 template <typename T>
 struct FaceRow3 {
   T E;
@@ -449,94 +479,71 @@ struct FaceRow3 {
 };
 
 template <typename T, bool FULL>
-__device__ __forceinline__ void eval_area_row(const T* xi, const T* xj, const T* xk, int c, T A0,
-                                              T k, FaceRow3<T>& o) {
+__device__ __forceinline__ void eval_area_row(const T* xi, const T* xj, const T* xk, T A0, T k,
+                                              FaceRow3<T>& o) {
   if constexpr (!FULL) {
-    Lin<T, 6> e1[3], e2[3];
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      const T u0 = sel3(c, xi[a], xk[a], xj[a]);
-      const T u1 = sel3(c, xj[a], xi[a], xk[a]);
-      const T u2 = sel3(c, xk[a], xj[a], xi[a]);
-      e1[a] = lin_var<T, 6>(u1 - u0, a);
-      e2[a] = lin_var<T, 6>(u2 - u0, 3 + a);
-    }
-    const HyperDual<T, 6> e = area_energy(e1, e2, A0, k);
+    const auto e = area_energy_m(
+        slin_var<T, 6, 0>(xj[0] - xi[0]), slin_var<T, 6, 1>(xj[1] - xi[1]),
+        slin_var<T, 6, 2>(xj[2] - xi[2]), slin_var<T, 6, 3>(xk[0] - xi[0]),
+        slin_var<T, 6, 4>(xk[1] - xi[1]), slin_var<T, 6, 5>(xk[2] - xi[2]), A0, k);
     o.E = e.v;
-    // coefficients of corners c, c+1, c+2 (face order) on e1 and e2
-    T p1[3], p2[3];
 #pragma unroll
-    for (int m = 0; m < 3; ++m) {
-      const int a = m == 0 ? c : (m == 1 ? (c == 2 ? 0 : c + 1) : (c == 0 ? 2 : c - 1));
-      p1[m] = a == 0 ? T(-1) : (a == 1 ? T(1) : T(0));
-      p2[m] = a == 0 ? T(-1) : (a == 2 ? T(1) : T(0));
-    }
+    for (int al = 0; al < 3; ++al) o.g[al] = -(sgrad(e, al) + sgrad(e, 3 + al));
 #pragma unroll
-    for (int al = 0; al < 3; ++al) o.g[al] = p1[0] * e.g[al] + p2[0] * e.g[3 + al];
+    for (int al = 0; al < 3; ++al)
 #pragma unroll
-    for (int m = 0; m < 3; ++m)
-#pragma unroll
-      for (int al = 0; al < 3; ++al)
-#pragma unroll
-        for (int be = 0; be < 3; ++be)
-          o.H[m][3 * al + be] = p1[0] * (p1[m] * hess(e, al, be) + p2[m] * hess(e, al, 3 + be)) +
-                                p2[0] * (p1[m] * hess(e, 3 + al, be) +
-                                         p2[m] * hess(e, 3 + al, 3 + be));
+      for (int be = 0; be < 3; ++be) {
+        const T h11 = shess(e, al, be), h12 = shess(e, al, 3 + be);
+        const T h21 = shess(e, 3 + al, be), h22 = shess(e, 3 + al, 3 + be);
+        o.H[0][3 * al + be] = (h11 + h12) + (h21 + h22);
+        o.H[1][3 * al + be] = -(h11 + h21);
+        o.H[2][3 * al + be] = -(h12 + h22);
+      }
   } else {
     // width-9 AD over (x_i, x_j, x_k)
-    Lin<T, 9> ui[3], uj[3], uk[3];
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      ui[a] = lin_var<T, 9>(xi[a], a);
-      uj[a] = lin_var<T, 9>(xj[a], 3 + a);
-      uk[a] = lin_var<T, 9>(xk[a], 6 + a);
-    }
-    Lin<T, 9> e1[3], e2[3];
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      const Lin<T, 9> u0 = c == 0 ? ui[a] : (c == 1 ? uk[a] : uj[a]);
-      const Lin<T, 9> u1 = c == 0 ? uj[a] : (c == 1 ? ui[a] : uk[a]);
-      const Lin<T, 9> u2 = c == 0 ? uk[a] : (c == 1 ? uj[a] : ui[a]);
-      e1[a] = u1 - u0;
-      e2[a] = u2 - u0;
-    }
-    const HyperDual<T, 9> e = area_energy(e1, e2, A0, k);
+    const auto i0 = slin_var<T, 9, 0>(xi[0]);
+    const auto i1 = slin_var<T, 9, 1>(xi[1]);
+    const auto i2 = slin_var<T, 9, 2>(xi[2]);
+    const auto e = area_energy_m(slin_var<T, 9, 3>(xj[0]) - i0, slin_var<T, 9, 4>(xj[1]) - i1,
+                                 slin_var<T, 9, 5>(xj[2]) - i2, slin_var<T, 9, 6>(xk[0]) - i0,
+                                 slin_var<T, 9, 7>(xk[1]) - i1, slin_var<T, 9, 8>(xk[2]) - i2,
+                                 A0, k);
     o.E = e.v;
 #pragma unroll
-    for (int al = 0; al < 3; ++al) o.g[al] = e.g[al];
+    for (int al = 0; al < 3; ++al) o.g[al] = sgrad(e, al);
 #pragma unroll
     for (int m = 0; m < 3; ++m)
 #pragma unroll
       for (int al = 0; al < 3; ++al)
 #pragma unroll
-        for (int be = 0; be < 3; ++be) o.H[m][3 * al + be] = hess(e, al, 3 * m + be);
+        for (int be = 0; be < 3; ++be) o.H[m][3 * al + be] = shess(e, al, 3 * m + be);
   }
 }
 
 // (H v) of one area-preservation face for its three corners (face order):
 // out[3a + al].  Reduced form: t = H_e dE with dE = (v1 - v0, v2 - v0), then
-// corner a takes p1[a] t_e1 + p2[a] t_e2.
+// corner a takes p1[a] t_e1 + p2[a] t_e2 with p1 = (-1, 1, 0), p2 = (-1, 0, 1).
 template <typename T, bool FULL>
 __device__ __forceinline__ void hv_area_face(const T* u0, const T* u1, const T* u2,
                                              const T* v0, const T* v1, const T* v2, T A0, T k,
                                              T* out) {
   if constexpr (!FULL) {
-    Lin<T, 6> e1[3], e2[3];
+    const auto e = area_energy_m(
+        slin_var<T, 6, 0>(u1[0] - u0[0]), slin_var<T, 6, 1>(u1[1] - u0[1]),
+        slin_var<T, 6, 2>(u1[2] - u0[2]), slin_var<T, 6, 3>(u2[0] - u0[0]),
+        slin_var<T, 6, 4>(u2[1] - u0[1]), slin_var<T, 6, 5>(u2[2] - u0[2]), A0, k);
     T d[6];
 #pragma unroll
     for (int a = 0; a < 3; ++a) {
-      e1[a] = lin_var<T, 6>(u1[a] - u0[a], a);
-      e2[a] = lin_var<T, 6>(u2[a] - u0[a], 3 + a);
       d[a] = v1[a] - v0[a];
       d[3 + a] = v2[a] - v0[a];
     }
-    const HyperDual<T, 6> e = area_energy(e1, e2, A0, k);
     T t[6];
 #pragma unroll
     for (int p = 0; p < 6; ++p) {
-      T s = T(0);
+      T s = shess(e, p, 0) * d[0];
 #pragma unroll
-      for (int q = 0; q < 6; ++q) s += hess(e, p, q) * d[q];
+      for (int q = 1; q < 6; ++q) s += shess(e, p, q) * d[q];
       t[p] = s;
     }
 #pragma unroll
@@ -546,26 +553,19 @@ __device__ __forceinline__ void hv_area_face(const T* u0, const T* u1, const T* 
       out[6 + al] = t[3 + al];
     }
   } else {
-    Lin<T, 9> x[3][3];
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      x[0][a] = lin_var<T, 9>(u0[a], a);
-      x[1][a] = lin_var<T, 9>(u1[a], 3 + a);
-      x[2][a] = lin_var<T, 9>(u2[a], 6 + a);
-    }
-    Lin<T, 9> e1[3], e2[3];
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      e1[a] = x[1][a] - x[0][a];
-      e2[a] = x[2][a] - x[0][a];
-    }
-    const HyperDual<T, 9> e = area_energy(e1, e2, A0, k);
+    const auto a0 = slin_var<T, 9, 0>(u0[0]);
+    const auto a1 = slin_var<T, 9, 1>(u0[1]);
+    const auto a2 = slin_var<T, 9, 2>(u0[2]);
+    const auto e = area_energy_m(slin_var<T, 9, 3>(u1[0]) - a0, slin_var<T, 9, 4>(u1[1]) - a1,
+                                 slin_var<T, 9, 5>(u1[2]) - a2, slin_var<T, 9, 6>(u2[0]) - a0,
+                                 slin_var<T, 9, 7>(u2[1]) - a1, slin_var<T, 9, 8>(u2[2]) - a2,
+                                 A0, k);
     const T* vv[3] = {v0, v1, v2};
 #pragma unroll
     for (int p = 0; p < 9; ++p) {
-      T s = T(0);
+      T s = shess(e, p, 0) * vv[0][0];
 #pragma unroll
-      for (int q = 0; q < 9; ++q) s += hess(e, p, q) * vv[q / 3][q % 3];
+      for (int q = 1; q < 9; ++q) s += shess(e, p, q) * vv[q / 3][q % 3];
       out[p] = s;
     }
   }
