@@ -91,6 +91,9 @@ class Oracle:
         lib.or_area_local.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_double,
                                       _f64p, _f64p, _f64p]
         lib.or_area_local.restype = None
+        lib.or_arap_local.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double, _f64p,
+                                      _f64p, _f64p]
+        lib.or_arap_local.restype = None
         lib.or_bsr_mv.argtypes = [ctypes.c_int32, ctypes.c_int, _i32p, _i32p, _f64p,
                                   _f64p, _f64p]
         lib.or_bsr_mv.restype = ctypes.c_int
@@ -203,6 +206,16 @@ class Oracle:
         self.lib.or_bsr_mv(V, dof, _p32(row_ptr), _p32(col_idx), _pf(H), _pf(v), _pf(y))
         return y.reshape(V, dof)
 
+
+    def arap_local(self, u0, u1, u2, M, A):
+        """Energy, gradient [6] and Hessian [6][6] of one ARAP face (UV)."""
+        E = np.zeros(1)
+        g = np.zeros(6)
+        H = np.zeros(36)
+        f = lambda a: np.ascontiguousarray(a, np.float64).reshape(-1)  # noqa: E731
+        self.lib.or_arap_local(_pf(f(u0)), _pf(f(u1)), _pf(f(u2)), _pf(f(M)), float(A), _pf(E),
+                               _pf(g), _pf(H))
+        return float(E[0]), g, H.reshape(6, 6)
 
     def area_local(self, x0, x1, x2, A0, k):
         """Energy, gradient [9] and Hessian [9][9] of one area-preservation face."""

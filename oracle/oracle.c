@@ -35,6 +35,8 @@
  *   spring / pair  E = 1/2 k (|xi - xj| - L0)^2
  *   inertia        E = 1/2 w |xi - xt_i|^2          (w = m / h^2)
  *   sym. Dirichlet E = A (|J|_F^2 + |J^-1|_F^2),  J = [u1-u0, u2-u0] Dm^-1
+ *   ARAP           E = A |J - R(J)|_F^2, R(J) the closest rotation
+ *   area           E = 1/2 k (A - A0)^2 / A0  (3D triangle area A)
  *
  * Parity pins: every function here is pinned by tests/test_oracle.py against
  * closed-form values, finite differences, symmetry, translation / rotation
@@ -186,6 +188,74 @@ void or_symdir_local(const double* u0, const double* u1, const double* u2,
           }
 #endif
           H[(2 * kk + al) * 6 + (2 * ll + be)] = s;
+        }
+}
+
+/* As-rigid-as-possible (ARAP) parameterization energy of one triangle:
+ *   E = A |J - R(J)|_F^2,   J = [u1-u0, u2-u0] Dm^-1 (as for SymDir),
+ * R(J) the rotation closest to J.  With j = (J00, J01, J10, J11),
+ * p = J00 + J11 and q = J10 - J01, the closest rotation is
+ * R = [[p, -q], [q, p]] / s with s = sqrt(p^2 + q^2) (the maximiser of
+ * tr(R^T J) over rotations, whose maximum is s), so
+ *   E = A (|J|^2 - 2 s + 2).
+ * For det J > 0, s = sigma_1 + sigma_2 and E = A sum_i (sigma_i - 1)^2.
+ *   dE/dj  = A (2 j - 2 ds/dj),   ds/dj = (p dp + q dq) / s,
+ *   dp = (1, 0, 0, 1),  dq = (0, -1, 1, 0),
+ *   d2E/dj2 = A (2 I - 2 d2s),
+ *   d2s = (q^2 dp dp^T - p q (dp dq^T + dq dp^T) + p^2 dq dq^T) / s^3.
+ * The map to the corners is SymDir's: g_k = P w_k, H_kl as there.
+ * s > 0 whenever det J > 0 (s^2 = |J|^2 + 2 det J).
+ * Output g[6] = (u0, u1, u2) interleaved, H 6x6 row-major.                  */
+void or_arap_local(const double* u0, const double* u1, const double* u2,
+                   const double* M, double A, double* E, double* g, double* H) {
+  double Ds[2][2] = {{u1[0] - u0[0], u2[0] - u0[0]},
+                     {u1[1] - u0[1], u2[1] - u0[1]}};
+  double J[2][2];
+  for (int al = 0; al < 2; ++al)
+    for (int ga = 0; ga < 2; ++ga)
+      J[al][ga] = Ds[al][0] * M[0 * 2 + ga] + Ds[al][1] * M[1 * 2 + ga];
+  double j[4] = {J[0][0], J[0][1], J[1][0], J[1][1]};
+  double p = j[0] + j[3];
+  double q = j[2] - j[1];
+  double s = sqrt(p * p + q * q);
+  double a = j[0] * j[0] + j[1] * j[1] + j[2] * j[2] + j[3] * j[3];
+  *E = A * (a - 2.0 * s + 2.0);
+  const double dp[4] = {1.0, 0.0, 0.0, 1.0};
+  const double dq[4] = {0.0, -1.0, 1.0, 0.0};
+  double Pj[4];
+  for (int r = 0; r < 4; ++r) Pj[r] = A * (2.0 * j[r] - 2.0 * (p * dp[r] + q * dq[r]) / s);
+  double s3 = s * s * s;
+  double HJ[4][4];
+  for (int r = 0; r < 4; ++r)
+    for (int c = 0; c < 4; ++c) {
+#if OR_MUTANT == 8 /* planted: sign of the mixed p-q term of d2s flipped */
+      double d2s = (q * q * dp[r] * dp[c] + p * q * (dp[r] * dq[c] + dq[r] * dp[c]) +
+                    p * p * dq[r] * dq[c]) / s3;
+#else
+      double d2s = (q * q * dp[r] * dp[c] - p * q * (dp[r] * dq[c] + dq[r] * dp[c]) +
+                    p * p * dq[r] * dq[c]) / s3;
+#endif
+      HJ[r][c] = A * (2.0 * (r == c ? 1.0 : 0.0) - 2.0 * d2s);
+    }
+  double w[3][2];
+  w[1][0] = M[0];
+  w[1][1] = M[1];
+  w[2][0] = M[2];
+  w[2][1] = M[3];
+  w[0][0] = -(w[1][0] + w[2][0]);
+  w[0][1] = -(w[1][1] + w[2][1]);
+  for (int kk = 0; kk < 3; ++kk)
+    for (int al = 0; al < 2; ++al)
+      g[2 * kk + al] = Pj[2 * al] * w[kk][0] + Pj[2 * al + 1] * w[kk][1];
+  for (int kk = 0; kk < 3; ++kk)
+    for (int ll = 0; ll < 3; ++ll)
+      for (int al = 0; al < 2; ++al)
+        for (int be = 0; be < 2; ++be) {
+          double t = 0.0;
+          for (int ga = 0; ga < 2; ++ga)
+            for (int de = 0; de < 2; ++de)
+              t += HJ[2 * al + ga][2 * be + de] * w[kk][ga] * w[ll][de];
+          H[(2 * kk + al) * 6 + (2 * ll + be)] = t;
         }
 }
 
@@ -459,7 +529,8 @@ static int emit_blocks(or_coo* c, int dof, int nv, const int32_t* vid,
  * (overwritten; blocks absent from every term are zero), *energy.          */
 /* mask bits: 1 spring, 2 inertia, 4 symmetric Dirichlet (dof 2, with Minv
  * and area = rest area), 8 pairs, 16 area preservation (dof 3, with area =
- * rest area A0 and stiffness ka). */
+ * rest area A0 and stiffness ka), 32 ARAP (dof 2, with Minv and area, like
+ * symmetric Dirichlet). */
 int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
              /* springs */ int32_t nE, const int32_t* edges, const double* L0,
              double k,
@@ -474,6 +545,7 @@ int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
   if (dof != 2 && dof != 3) return OR_ERR_ARG;
   if ((mask & 4) && dof != 2) return OR_ERR_ARG;
   if ((mask & 16) && dof != 3) return OR_ERR_ARG;
+  if ((mask & 32) && dof != 2) return OR_ERR_ARG;
   int bs = dof * dof;
   int64_t n = 0;
   if (mask & 1) n += 4 * (int64_t)nE;
@@ -481,6 +553,7 @@ int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
   if (mask & 4) n += 9 * (int64_t)nF;
   if (mask & 8) n += 4 * (int64_t)nP;
   if (mask & 16) n += 9 * (int64_t)nF;
+  if (mask & 32) n += 9 * (int64_t)nF;
   or_coo c;
   c.bs = bs;
   c.cap = n > 0 ? n : 1;
@@ -519,6 +592,16 @@ int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
       or_symdir_local(x + (size_t)vid[0] * 2, x + (size_t)vid[1] * 2,
                       x + (size_t)vid[2] * 2, Minv + 4 * (size_t)f, area[f], &E,
                       gl, Hl);
+      Etot += E;
+      for (int p = 0; p < 3; ++p)
+        for (int a = 0; a < 2; ++a) g[(size_t)vid[p] * 2 + a] += gl[p * 2 + a];
+      rc = emit_blocks(&c, 2, 3, vid, Hl);
+    }
+  if (mask & 32)
+    for (int32_t f = 0; f < nF && !rc; ++f) {
+      const int32_t* vid = F + 3 * f;
+      or_arap_local(x + (size_t)vid[0] * 2, x + (size_t)vid[1] * 2, x + (size_t)vid[2] * 2,
+                    Minv + 4 * (size_t)f, area[f], &E, gl, Hl);
       Etot += E;
       for (int p = 0; p < 3; ++p)
         for (int a = 0; a < 2; ++a) g[(size_t)vid[p] * 2 + a] += gl[p * 2 + a];
