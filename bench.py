@@ -266,6 +266,14 @@ def cpu_baseline_rows(st):
     t2 = time.perf_counter()
     res["symdir500_eval_ms"] = round((t1 - t0) * 1e3, 1)
     res["symdir500_hvp_ms"] = round((t2 - t1) * 1e3, 1)
+    t0 = time.perf_counter()
+    _, oH, _ = orc.eval(ps["V"], 2, ps["UV"], 32, rp, ci, F=ps["F"], Minv=ps["Minv"],
+                        area=ps["area"])
+    t1 = time.perf_counter()
+    orc.bsr_mv(ps["V"], 2, rp, ci, oH, mi.probe_vector(ps["V"], 2, 1005, np.float32))
+    t2 = time.perf_counter()
+    res["arap500_eval_ms"] = round((t1 - t0) * 1e3, 1)
+    res["arap500_hvp_ms"] = round((t2 - t1) * 1e3, 1)
     # cloth 1000^2 + 10^5 pairs (step 0): the pattern with the pairs, then assembly
     xx = mi.cloth_x(N_GRID, 1005, 0, np.float32)
     pp = mi.random_pairs(N_GRID, 100_000, 1005, 0)
@@ -460,6 +468,10 @@ def symdir500(res, mad, torch, dev, stream, timeit):
                    face_area=terms.face_area)
     res["symdir500_patch_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, tp, g, H, None, stream)), 5)
     res["symdir500_patch_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, tp, v, y, stream)), 5)
+    # ARAP on the same faces and inputs
+    ta = mad.Terms(mask=32, face_Minv=terms.face_Minv, face_area=terms.face_area)
+    res["arap500_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, ta, g, H, None, stream)), 5)
+    res["arap500_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, ta, v, y, stream)), 5)
     ctx.close()
 
 

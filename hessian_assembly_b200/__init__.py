@@ -42,6 +42,7 @@ MAD_TERM_INERTIA = 2
 MAD_TERM_SYMDIR = 4
 MAD_TERM_PAIR = 8
 MAD_TERM_AREA = 16
+MAD_TERM_ARAP = 32
 MAD_EVAL_FULL_STENCIL_AD = 1
 MAD_EVAL_EDGE_SCATTER = 2
 MAD_EVAL_PATCH_STAGED = 4

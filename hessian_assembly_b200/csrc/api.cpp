@@ -212,13 +212,14 @@ RowsLaunch rows_launch(const mad_ctx* c) {
 // rows could not be built.
 bool use_rows(const mad_ctx* c, const mad_terms* t) {
   if (t->flags & (MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED)) return false;
-  return !(t->mask & (MAD_TERM_SYMDIR | MAD_TERM_AREA)) || c->nF == 0 || c->rows_sf > 0;
+  return !(t->mask & (MAD_TERM_SYMDIR | MAD_TERM_AREA | MAD_TERM_ARAP)) || c->nF == 0 ||
+         c->rows_sf > 0;
 }
 
 mad_status check_terms(mad_ctx* c, const mad_terms* t) {
   if (!t) return fail(c, MAD_ERR_INVALID_ARG, "terms is NULL");
-  const uint32_t known =
-      MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR | MAD_TERM_AREA;
+  const uint32_t known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR |
+                         MAD_TERM_AREA | MAD_TERM_ARAP;
   if (t->mask & ~known) return fail(c, MAD_ERR_INVALID_ARG, "unknown term bits in mask");
   if (t->flags &
       ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED))
@@ -232,6 +233,16 @@ mad_status check_terms(mad_ctx* c, const mad_terms* t) {
       return fail(c, MAD_ERR_UNIMPLEMENTED, "symmetric Dirichlet term needs dof 2");
     if (c->nF > 0 && (!t->face_Minv || !t->face_area))
       return fail(c, MAD_ERR_INVALID_ARG, "symmetric Dirichlet term needs face_Minv and face_area");
+  }
+  if (t->mask & MAD_TERM_ARAP) {
+    if (c->dof != 2) return fail(c, MAD_ERR_UNIMPLEMENTED, "ARAP term needs dof 2");
+    if (c->nF > 0 && (!t->face_Minv || !t->face_area))
+      return fail(c, MAD_ERR_INVALID_ARG, "ARAP term needs face_Minv and face_area");
+    // only the row-streaming kernel evaluates it
+    if (t->flags & (MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED))
+      return fail(c, MAD_ERR_UNIMPLEMENTED, "ARAP term needs the row kernel");
+    if (c->nF > 0 && c->rows_sf == 0)
+      return fail(c, MAD_ERR_UNIMPLEMENTED, "ARAP term: a mesh row too long for the face rows");
   }
   if (t->mask & MAD_TERM_AREA) {
     if (c->dof != 3)
@@ -602,14 +613,14 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij, const void* r
 
 namespace {
 mad_status jac_mask_ok(const mad_ctx* c, uint32_t mask, std::string* why) {
-  const uint32_t known =
-      MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR | MAD_TERM_AREA;
+  const uint32_t known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR |
+                         MAD_TERM_AREA | MAD_TERM_ARAP;
   if (mask & ~known) {
     *why = "unknown term bits in mask";
     return MAD_ERR_INVALID_ARG;
   }
-  if (mask & (MAD_TERM_PAIR | MAD_TERM_AREA)) {
-    *why = "pair and area terms are not part of the vector-valued objective";
+  if (mask & (MAD_TERM_PAIR | MAD_TERM_AREA | MAD_TERM_ARAP)) {
+    *why = "pair, area and ARAP terms are not part of the vector-valued objective";
     return MAD_ERR_UNIMPLEMENTED;
   }
   if ((mask & MAD_TERM_SYMDIR) && c->dof != 2) {

@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
   const int64_t t = (int64_t)blockIdx.x * kNaThreads + threadIdx.x;
   const int64_t nS = (A.mask & MAD_TERM_SPRING) ? A.nE : 0;
   const int64_t nI = (A.mask & MAD_TERM_INERTIA) ? A.V : 0;
-  const int64_t nFc = ((DOF == 2 && (A.mask & MAD_TERM_SYMDIR)) ||
+  const int64_t nFc = ((DOF == 2 && (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP))) ||
                        (DOF == 3 && (A.mask & MAD_TERM_AREA)))
                           ? A.nF
                           : 0;
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
 #pragma unroll
         for (int ga = 0; ga < 2; ++ga)
           j[2 * al + ga] = (u1[al] - u0[al]) * M[ga] + (u2[al] - u0[al]) * M[2 + ga];
-      e = (double)symdir_energy(j, A.area[f]);
+      e = (double)face2_energy(j, A.area[f], face2_kind(A.mask));
     } else {
       const int64_t f = t - nS - nI;
       const T* u0 = A.x + (int64_t)A.F[3 * f] * 3;
@@ -179,22 +179,24 @@ extern "C" mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, c
       (dt != MAD_F32 && dt != MAD_F64) || !t || !energy) {
     return MAD_ERR_INVALID_ARG;
   }
-  const unsigned known =
-      MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR | MAD_TERM_AREA;
+  const unsigned known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR |
+                         MAD_TERM_AREA | MAD_TERM_ARAP;
   if (t->mask & ~known) {
     return MAD_ERR_INVALID_ARG;
   }
   const bool sp = (t->mask & MAD_TERM_SPRING) && nE > 0;
   const bool in = (t->mask & MAD_TERM_INERTIA) && V > 0;
   const bool sd = (t->mask & MAD_TERM_SYMDIR) && nF > 0;
+  const bool rp = (t->mask & MAD_TERM_ARAP) && nF > 0;
   const bool ar = (t->mask & MAD_TERM_AREA) && nF > 0;
-  const bool fa = sd || ar;
+  const bool fa = sd || rp || ar;
   const bool pa = (t->mask & MAD_TERM_PAIR) && nP > 0;
-  if (((t->mask & MAD_TERM_SYMDIR) && dof != 2) || ((t->mask & MAD_TERM_AREA) && dof != 3)) {
+  if (((t->mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) && dof != 2) ||
+      ((t->mask & MAD_TERM_AREA) && dof != 3)) {
     return MAD_ERR_UNIMPLEMENTED;
   }
   if ((V > 0 && !x) || (sp && (!edges || !t->spring_rest)) || (in && !t->inertia_xt) ||
-      (sd && (!F || !t->face_Minv || !t->face_area)) || (ar && (!F || !t->face_area)) ||
+      ((sd || rp) && (!F || !t->face_Minv || !t->face_area)) || (ar && (!F || !t->face_area)) ||
       (pa && (!pairs || !pair_rest))) {
     return MAD_ERR_INVALID_ARG;
   }
@@ -211,7 +213,8 @@ extern "C" mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, c
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const unsigned mask = (sp ? MAD_TERM_SPRING : 0u) | (in ? MAD_TERM_INERTIA : 0u) |
-                        (sd ? MAD_TERM_SYMDIR : 0u) | (ar ? MAD_TERM_AREA : 0u) |
+                        (sd ? MAD_TERM_SYMDIR : 0u) | (rp ? MAD_TERM_ARAP : 0u) |
+                        (ar ? MAD_TERM_AREA : 0u) |
                         (pa ? MAD_TERM_PAIR : 0u);
   if (dt == MAD_F64) {
     mad::NaArgs<double> A{V, nE, nF, nP, (const double*)x, edges, (const double*)t->spring_rest,

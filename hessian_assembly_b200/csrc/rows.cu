@@ -321,7 +321,7 @@ __device__ __forceinline__ void add4(T* b, const T* v) {
 
 // The work of one row, writing the row's blocks through `row` (a shared-memory
 // staging slot or, for rows that do not fit, the row's place in H).
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES, bool PAIRS>
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES, bool PAIRS>
 __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile, int lane,
                                               uint32_t m, int d0, int d1, int pb, int pn,
                                               const T* xi, const T* xti, T* row, double& energy) {
@@ -415,23 +415,32 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   }
   if constexpr (FACES && DOF == 2) {
     // after the edge terms, which store their blocks: faces add to them
-    if (A.mask & MAD_TERM_SYMDIR) {
-      row_faces<T>(A, i, tile, lane,
-                   [&](const T* xj, const T* xk, int, int, int c, int pj, int pk, const T* M,
-                       T ar) {
-                     FaceRow<T> o;
-                     eval_symdir_row<T, FULL>(xi, xj, xk, c, M, ar, o);
-                     acc[0] += o.H[0][0];
-                     acc[1] += o.H[0][1];
-                     acc[2] += o.H[0][3];
-                     gr[0] += o.g[0];
-                     gr[1] += o.g[1];
-                     const int oj = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pj) : pj;
-                     const int ok = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pk) : pk;
-                     add4<T>(row + oj * B, o.H[1]);
-                     add4<T>(row + ok * B, o.H[2]);
-                     if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
-                   });
+    if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
+      auto faces = [&](auto kc) {
+        constexpr int KIND = decltype(kc)::value;
+        row_faces<T>(A, i, tile, lane,
+                     [&](const T* xj, const T* xk, int, int, int c, int pj, int pk, const T* M,
+                         T ar) {
+                       FaceRow<T> o;
+                       eval_symdir_row<T, FULL, KIND>(xi, xj, xk, c, M, ar, o);
+                       acc[0] += o.H[0][0];
+                       acc[1] += o.H[0][1];
+                       acc[2] += o.H[0][3];
+                       gr[0] += o.g[0];
+                       gr[1] += o.g[1];
+                       const int oj = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pj) : pj;
+                       const int ok = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pk) : pk;
+                       add4<T>(row + oj * B, o.H[1]);
+                       add4<T>(row + ok * B, o.H[2]);
+                       if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
+                     });
+      };
+      if constexpr (FACES == 1) {
+        faces(std::integral_constant<int, kFaceSymDir>{});
+      } else {
+        if (!(A.mask & MAD_TERM_SYMDIR)) faces(std::integral_constant<int, kFaceArap>{});
+        else faces(std::integral_constant<int, kFaceSymDir | kFaceArap>{});
+      }
     }
   }
   if (pairs) {
@@ -467,8 +476,8 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   for (int a = 0; a < DOF; ++a) A.g[(uint32_t)(i * DOF + a)] = gr[a];
 }
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES, bool PAIRS>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_eval(const RArgs<T> A) {
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES, bool PAIRS>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, (FACES != 0)>()) k_rows_eval(const RArgs<T> A) {
   constexpr int B = DOF * DOF;
   constexpr int VEC = 16 / (int)sizeof(T);
   extern __shared__ __align__(16) char smem_raw[];
@@ -601,7 +610,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
     }
   }
   if constexpr (FACES) {
-    if (A.mask & (DOF == 2 ? MAD_TERM_SYMDIR : MAD_TERM_AREA)) {
+    if (A.mask & (DOF == 2 ? (MAD_TERM_SYMDIR | MAD_TERM_ARAP) : MAD_TERM_AREA)) {
       // the row's corners' results of the per-face pass (k_face_hv)
       constexpr int SF = kFaceRowSlots;
       int32_t e[SF];
@@ -679,7 +688,8 @@ template <typename T, bool FULL>
 __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_t* __restrict__ F,
                                                  const T* __restrict__ x, const T* __restrict__ v,
                                                  const T* __restrict__ Minv,
-                                                 const T* __restrict__ area, T* __restrict__ out) {
+                                                 const T* __restrict__ area, T* __restrict__ out,
+                                                 int kind) {
   const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (f >= nF) return;
   const int32_t a = F[3 * f], b = F[3 * f + 1], c = F[3 * f + 2];
@@ -709,7 +719,10 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
   }
   load4<T>(Minv + 4 * f, M);
   T o[6];
-  hv_symdir_face<T, FULL>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f], o);
+  with_face2_kind(kind, [&](auto kc) {
+    hv_symdir_face<T, FULL, decltype(kc)::value>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f],
+                                                 o);
+  });
 #pragma unroll
   for (int q = 0; q < 6; ++q) out[6 * f + q] = o[q];
 }
@@ -785,7 +798,7 @@ __global__ void k_energy_sum_rows(const double* __restrict__ part, int n, double
 // One instantiation of the assembly kernel, chosen by whether the active
 // pattern holds pair blocks; also sets (or, with set, only sets) its shared
 // memory limit.
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool FACES>
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES>
 cudaError_t eval_k(const RArgs<T>& A, bool pairs, int nb, size_t smem, cudaStream_t s,
                    bool set = false) {
   const void* kp = (const void*)k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, true>;
@@ -802,8 +815,12 @@ cudaError_t eval_k(const RArgs<T>& A, bool pairs, int nb, size_t smem, cudaStrea
   return cudaGetLastError();
 }
 
-// Every (FULL, ENERGY) instantiation for one S0 and FACES.
-template <typename T, int DOF, int S0, bool FACES>
+// Every (FULL, ENERGY) instantiation for one S0 and FACES.  FACES: 0 no face
+// terms; 1 the face term of the dof (symmetric Dirichlet for dof 2, area
+// preservation for dof 3); 2 (dof 2) ARAP alone or with symmetric Dirichlet,
+// an instantiation of its own so that the symmetric Dirichlet kernel keeps
+// its register budget.
+template <typename T, int DOF, int S0, int FACES>
 cudaError_t eval_k4(const RArgs<T>& A, bool full, bool energy, bool pairs, int nb, size_t smem,
                     cudaStream_t s, bool set = false) {
   if (set) {
@@ -829,19 +846,27 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   const bool pairs = L.prow != nullptr;
   const bool en = energy != nullptr;
   cudaError_t e;
-  if ((DOF == 2 && (t.mask & MAD_TERM_SYMDIR)) || (DOF == 3 && (t.mask & MAD_TERM_AREA))) {
+  if ((DOF == 2 && (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP))) ||
+      (DOF == 3 && (t.mask & MAD_TERM_AREA))) {
     // face terms: the face-row instantiations; without edge terms the kernel
     // carries no edge-slot code (S0 = 0)
+    auto faces_k = [&](auto s0c) {
+      constexpr int S0F = decltype(s0c)::value;
+      if constexpr (DOF == 2) {
+        if (t.mask & MAD_TERM_ARAP) return eval_k4<T, DOF, S0F, 2>(A, full, en, pairs, nb, smem, s);
+      }
+      return eval_k4<T, DOF, S0F, 1>(A, full, en, pairs, nb, smem, s);
+    };
     if (t.mask & MAD_TERM_SPRING)
-      e = eval_k4<T, DOF, kS0Max, true>(A, full, en, pairs, nb, smem, s);
+      e = faces_k(std::integral_constant<int, kS0Max>{});
     else
-      e = eval_k4<T, DOF, 0, true>(A, full, en, pairs, nb, smem, s);
+      e = faces_k(std::integral_constant<int, 0>{});
   } else if (L.s0 <= 6) {
     // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
     // narrower instantiation: fewer registers
-    e = eval_k4<T, DOF, 6, false>(A, full, en, pairs, nb, smem, s);
+    e = eval_k4<T, DOF, 6, 0>(A, full, en, pairs, nb, smem, s);
   } else {
-    e = eval_k4<T, DOF, kS0Max, false>(A, full, en, pairs, nb, smem, s);
+    e = eval_k4<T, DOF, kS0Max, 0>(A, full, en, pairs, nb, smem, s);
   }
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
@@ -855,18 +880,19 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
   const int nb = rows_blocks(L.V);
   const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
   if constexpr (DOF == 2) {
-    if (t.mask & MAD_TERM_SYMDIR) {
+    if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
+      const int kind = face2_kind(t.mask);
       if (L.nF > 0) {
         const unsigned nbf = (unsigned)((L.nF + 255) / 256);
         const bool vec2 = ((((uintptr_t)x) | ((uintptr_t)v)) % (2 * sizeof(T))) == 0;
         if (full)
           k_face_hv<T, true><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
                                                  (const T*)t.face_Minv, (const T*)t.face_area,
-                                                 (T*)L.fhv);
+                                                 (T*)L.fhv, kind);
         else
           k_face_hv<T, false><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
                                                   (const T*)t.face_Minv, (const T*)t.face_area,
-                                                  (T*)L.fhv);
+                                                  (T*)L.fhv, kind);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
       }
@@ -927,16 +953,21 @@ template <typename T, int DOF>
 cudaError_t set_rows_limits(size_t bytes) {
   RArgs<T> A{};
   cudaError_t e;
-  if ((e = eval_k4<T, DOF, 6, false>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+  if ((e = eval_k4<T, DOF, 6, 0>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
     return e;
-  if ((e = eval_k4<T, DOF, kS0Max, false>(A, false, false, false, 0, bytes, 0, true)) !=
-      cudaSuccess)
+  if ((e = eval_k4<T, DOF, kS0Max, 0>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
     return e;
-  if ((e = eval_k4<T, DOF, kS0Max, true>(A, false, false, false, 0, bytes, 0, true)) !=
-      cudaSuccess)
+  if ((e = eval_k4<T, DOF, kS0Max, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
     return e;
-  if ((e = eval_k4<T, DOF, 0, true>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+  if ((e = eval_k4<T, DOF, 0, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
     return e;
+  if constexpr (DOF == 2) {
+    if ((e = eval_k4<T, DOF, kS0Max, 2>(A, false, false, false, 0, bytes, 0, true)) !=
+        cudaSuccess)
+      return e;
+    if ((e = eval_k4<T, DOF, 0, 2>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+      return e;
+  }
   return cudaSuccess;
 }
 

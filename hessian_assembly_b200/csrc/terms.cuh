@@ -25,6 +25,9 @@
 //    four blocks are K, -K, -K, K.
 #pragma once
 
+#include <type_traits>
+
+#include "../../include/mad.h"
 #include "dual.cuh"
 #include "sparse_ad.cuh"
 
@@ -91,6 +94,50 @@ __device__ __forceinline__ auto symdir_energy(const S (&j)[4], T A) {
   auto a = sq(j[0]) + sq(j[1]) + sq(j[2]) + sq(j[3]);
   auto det = j[0] * j[3] - j[1] * j[2];
   return a * symdir_scale(det, A);
+}
+
+// As-rigid-as-possible parameterization energy, E = A |J - R(J)|_F^2 with
+// R(J) the rotation closest to J.  That rotation maximises tr(R^T J), whose
+// maximum over 2D rotations is s = sqrt((J00 + J11)^2 + (J10 - J01)^2), so
+// E = A (|J|_F^2 - 2 s + 2); s > 0 whenever det J > 0 (s^2 = |J|^2 + 2 det J).
+template <typename S, typename T>
+__device__ __forceinline__ auto arap_energy(const S (&j)[4], T A) {
+  auto a = sq(j[0]) + sq(j[1]) + sq(j[2]) + sq(j[3]);
+  auto s = sq(j[0] + j[3]) + sq(j[2] - j[1]);
+  return (a - sqrt(s) * T(2) + T(2)) * A;
+}
+
+// The dof-2 face energies on the same inputs (J, rest area), summed as
+// selected by kind: bit 0 symmetric Dirichlet, bit 1 ARAP.  kind is the same
+// for every thread of a launch.
+constexpr int kFaceSymDir = 1;
+constexpr int kFaceArap = 2;
+__host__ __device__ constexpr int face2_kind(uint32_t mask) {
+  return ((mask & MAD_TERM_SYMDIR) ? kFaceSymDir : 0) | ((mask & MAD_TERM_ARAP) ? kFaceArap : 0);
+}
+template <int KIND, typename S, typename T>
+__device__ __forceinline__ auto face2_energy(const S (&j)[4], T A) {
+  static_assert(KIND >= 1 && KIND <= 3, "face energy selector");
+  if constexpr (KIND == kFaceSymDir) return symdir_energy(j, A);
+  else if constexpr (KIND == kFaceArap) return arap_energy(j, A);
+  else return symdir_energy(j, A) + arap_energy(j, A);
+}
+// the same with the selector known only at run time (plain-value energies)
+template <typename S, typename T>
+__device__ __forceinline__ auto face2_energy(const S (&j)[4], T A, int kind) {
+  decltype(symdir_energy(j, A)) e;
+  if (kind == kFaceSymDir) e = face2_energy<kFaceSymDir>(j, A);
+  else if (kind == kFaceArap) e = face2_energy<kFaceArap>(j, A);
+  else e = face2_energy<kFaceSymDir | kFaceArap>(j, A);
+  return e;
+}
+// calls f(std::integral_constant<int, KIND>) for a run-time selector, so that
+// the face loop is compiled once per energy set
+template <typename F>
+__device__ __forceinline__ void with_face2_kind(int kind, F&& f) {
+  if (kind == kFaceSymDir) f(std::integral_constant<int, kFaceSymDir>{});
+  else if (kind == kFaceArap) f(std::integral_constant<int, kFaceArap>{});
+  else f(std::integral_constant<int, kFaceSymDir | kFaceArap>{});
 }
 
 // Area preservation of a 3D triangle: with n = e1 x e2 (e1 = x1 - x0,
@@ -297,7 +344,7 @@ struct FaceDerivs {
   T H[3][3][4];
 };
 
-template <typename T, bool FULL>
+template <typename T, bool FULL, int KIND = kFaceSymDir>
 __device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u2,
                                             const T* M, T A, FaceDerivs<T>& o) {
   // corner weights w_k: dJ[al][ga]/du_k[be] = delta(al, be) w_k[ga]
@@ -312,7 +359,7 @@ __device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u
     Lin<T, 4> j[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) j[p] = lin_var<T, 4>(Jv[p], p);
-    HyperDual<T, 4> e = symdir_energy(j, A);
+    HyperDual<T, 4> e = face2_energy<KIND>(j, A);
     o.E = e.v;
 #pragma unroll
     for (int k = 0; k < 3; ++k)
@@ -349,7 +396,7 @@ __device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u
 #pragma unroll
       for (int ga = 0; ga < 2; ++ga)
         j[2 * al + ga] = (u[1][al] - u[0][al]) * M[ga] + (u[2][al] - u[0][al]) * M[2 + ga];
-    HyperDual<T, 6> e = symdir_energy(j, A);
+    HyperDual<T, 6> e = face2_energy<KIND>(j, A);
     o.E = e.v;
 #pragma unroll
     for (int q = 0; q < 6; ++q) o.g[q] = e.g[q];
@@ -383,7 +430,7 @@ __device__ __forceinline__ T sel3(int c, T a, T b, T d) {
   return c == 0 ? a : (c == 1 ? b : d);
 }
 
-template <typename T, bool FULL>
+template <typename T, bool FULL, int KIND>
 __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const T* xk, int c,
                                                 const T* M, T A, FaceRow<T>& o) {
   // corner weights of corners 0, 1, 2; then those of i, j, k
@@ -409,7 +456,7 @@ __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const 
     Lin<T, 4> j[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) j[p] = lin_var<T, 4>(Jv[p], p);
-    HyperDual<T, 4> e = symdir_energy(j, A);
+    HyperDual<T, 4> e = face2_energy<KIND>(j, A);
     o.E = e.v;
 #pragma unroll
     for (int al = 0; al < 2; ++al) o.g[al] = e.g[2 * al] * wr[0][0] + e.g[2 * al + 1] * wr[0][1];
@@ -448,7 +495,7 @@ __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const 
 #pragma unroll
       for (int ga = 0; ga < 2; ++ga) j[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
     }
-    HyperDual<T, 6> e = symdir_energy(j, A);
+    HyperDual<T, 6> e = face2_energy<KIND>(j, A);
     o.E = e.v;
     o.g[0] = e.g[0];
     o.g[1] = e.g[1];
@@ -575,7 +622,7 @@ __device__ __forceinline__ void hv_area_face(const T* u0, const T* u1, const T* 
 // = sum_l (H_kl v_l)[al], with u and v the corners' positions and direction
 // in face order.  The reduced form contracts in J space: dJ = sum_k v_k w_k^T,
 // t = H_J dJ, out_k = t projected on w_k.
-template <typename T, bool FULL>
+template <typename T, bool FULL, int KIND>
 __device__ __forceinline__ void hv_symdir_face(const T* u0, const T* u1, const T* u2,
                                                const T* v0, const T* v1, const T* v2,
                                                const T* M, T A, T* out) {
@@ -592,7 +639,7 @@ __device__ __forceinline__ void hv_symdir_face(const T* u0, const T* u1, const T
     Lin<T, 4> j[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) j[p] = lin_var<T, 4>(Jv[p], p);
-    HyperDual<T, 4> e = symdir_energy(j, A);
+    HyperDual<T, 4> e = face2_energy<KIND>(j, A);
     T t[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
@@ -607,7 +654,7 @@ __device__ __forceinline__ void hv_symdir_face(const T* u0, const T* u1, const T
       for (int al = 0; al < 2; ++al) out[2 * k + al] = t[2 * al] * w[k][0] + t[2 * al + 1] * w[k][1];
   } else {
     FaceDerivs<T> o;
-    eval_symdir<T, true>(u0, u1, u2, M, A, o);
+    eval_symdir<T, true, KIND>(u0, u1, u2, M, A, o);
     const T* vv[3] = {v0, v1, v2};
 #pragma unroll
     for (int k = 0; k < 3; ++k)

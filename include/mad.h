@@ -72,9 +72,15 @@ enum {
   MAD_TERM_SYMDIR = 4u,  /* per face, dof 2: A_f (|J|_F^2 + |J^-1|_F^2),
                             J = [u1-u0, u2-u0] Minv_f                         */
   MAD_TERM_PAIR = 8u,    /* per runtime pair: 1/2 k_p (|xi - xj| - r_p)^2     */
-  MAD_TERM_AREA = 16u    /* per face, dof 3 (a 9-variable stencil): area
+  MAD_TERM_AREA = 16u,   /* per face, dof 3 (a 9-variable stencil): area
                             preservation 1/2 k_a (A_f - A0_f)^2 / A0_f with
                             A_f = |(x1-x0) x (x2-x0)| / 2, A0_f = face_area */
+  MAD_TERM_ARAP = 32u    /* per face, dof 2: as-rigid-as-possible
+                            A_f |J - R(J)|_F^2, J as for MAD_TERM_SYMDIR
+                            (same face_Minv and face_area), R(J) the closest
+                            rotation.  With MAD_TERM_SYMDIR both energies
+                            are summed per face.  Needs det J > 0 (the
+                            closest rotation is unique there).              */
 };
 
 /* Evaluation flags. */
@@ -90,12 +96,12 @@ enum {
    * thread that owns a row gathers the derivatives of the row's edge terms
    * (each term evaluated once per owned endpoint).  Same results up to
    * rounding; provided for comparison.                                       */
-  MAD_EVAL_EDGE_SCATTER = 2u,  /* (not with MAD_TERM_AREA) */
+  MAD_EVAL_EDGE_SCATTER = 2u,  /* (not with MAD_TERM_AREA or MAD_TERM_ARAP) */
   /* Use the patch kernel (one CUDA block per patch, positions of the patch's
    * owned and ribbon vertices staged in shared memory) instead of the
    * default row-streaming kernel (one warp per 32 consecutive rows, no
    * block-wide barriers).  Same results up to rounding.  The patch kernel
-   * does not evaluate MAD_TERM_AREA (MAD_ERR_UNIMPLEMENTED).                 */
+   * does not evaluate MAD_TERM_AREA or MAD_TERM_ARAP (MAD_ERR_UNIMPLEMENTED). */
   MAD_EVAL_PATCH_STAGED = 4u
 };
 
@@ -236,12 +242,13 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij,
  * J is scalar CSR with int64 row pointers and int32 columns; a column is
  * vertex*dof + component, ascending within each row (the stencil's vertices
  * sorted by index).  Nonzeros per row: 2*dof (spring), 1 (inertia), 6 (face).
- * MAD_TERM_PAIR and MAD_TERM_AREA are not part of the vector objective
- * (MAD_ERR_UNIMPLEMENTED).                                                  */
+ * MAD_TERM_PAIR, MAD_TERM_AREA and MAD_TERM_ARAP are not part of the vector
+ * objective (MAD_ERR_UNIMPLEMENTED).                                        */
 
 /* Rows and nonzeros of the Jacobian of the terms in `mask`.  Errors:
  * MAD_ERR_INVALID_ARG (NULL outputs, unknown bits), MAD_ERR_UNIMPLEMENTED
- * (MAD_TERM_PAIR, MAD_TERM_AREA, or MAD_TERM_SYMDIR with dof 3).            */
+ * (MAD_TERM_PAIR, MAD_TERM_AREA, MAD_TERM_ARAP, or MAD_TERM_SYMDIR with
+ * dof 3).                                                                   */
 mad_status mad_jacobian_shape(const mad_ctx* c, uint32_t mask, int64_t* nrows, int64_t* nnz);
 
 /* Writes the Jacobian's pattern for `mask`: row_ptr DEVICE int64 [nrows+1],
