@@ -160,6 +160,36 @@ __device__ __forceinline__ SHD<T, N, (GA | GB), (HA | HB)> operator-(const SHD<T
   return r;
 }
 
+// (ab)'' = a b'' + b a'' + a' b'^T + b' a'^T
+template <typename T, int N, uint32_t GA, uint64_t HA, uint32_t GB, uint64_t HB>
+__device__ __forceinline__ SHD<T, N, (GA | GB), (HA | HB | outer_mask<N>(GA, GB))> operator*(
+    const SHD<T, N, GA, HA>& a, const SHD<T, N, GB, HB>& b) {
+  SHD<T, N, (GA | GB), (HA | HB | outer_mask<N>(GA, GB))> r;
+  r.v = a.v * b.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    if (mbit(GA, i) && mbit(GB, i)) r.g[i] = a.v * b.g[i] + b.v * a.g[i];
+    else if (mbit(GB, i)) r.g[i] = a.v * b.g[i];
+    else if (mbit(GA, i)) r.g[i] = b.v * a.g[i];
+  }
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+#pragma unroll
+    for (int j = i; j < N; ++j) {
+      const int q = Tri<N>::idx(i, j);
+      // the four terms in the dense product's order, each only where it can be non-zero
+      const bool t0 = mbit(HB, q), t1 = mbit(HA, q);
+      const bool t2 = mbit(GA, i) && mbit(GB, j), t3 = mbit(GA, j) && mbit(GB, i);
+      T acc = T(-0.0);
+      if (t0) acc = a.v * b.h[q];
+      if (t1) acc = t0 ? acc + b.v * a.h[q] : b.v * a.h[q];
+      if (t2) acc = (t0 || t1) ? acc + a.g[i] * b.g[j] : a.g[i] * b.g[j];
+      if (t3) acc = (t0 || t1 || t2) ? acc + a.g[j] * b.g[i] : a.g[j] * b.g[i];
+      if (t0 || t1 || t2 || t3) r.h[q] = acc;
+    }
+  return r;
+}
+
 // a^2: (a^2)'' = 2 a a'' + 2 a' a'^T
 template <typename T, int N, uint32_t G, uint64_t H>
 __device__ __forceinline__ SHD<T, N, G, (H | outer_mask<N>(G, G))> sq(const SHD<T, N, G, H>& a) {
