@@ -94,6 +94,9 @@ class Oracle:
         lib.or_arap_local.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double, _f64p,
                                       _f64p, _f64p]
         lib.or_arap_local.restype = None
+        lib.or_vf_local.argtypes = [_f64p, _f64p, _f64p, _f64p, ctypes.c_double, ctypes.c_double,
+                                    _f64p, _f64p, _f64p]
+        lib.or_vf_local.restype = None
         lib.or_bsr_mv.argtypes = [ctypes.c_int32, ctypes.c_int, _i32p, _i32p, _f64p,
                                   _f64p, _f64p]
         lib.or_bsr_mv.restype = ctypes.c_int
@@ -216,6 +219,16 @@ class Oracle:
         self.lib.or_arap_local(_pf(f(u0)), _pf(f(u1)), _pf(f(u2)), _pf(f(M)), float(A), _pf(E),
                                _pf(g), _pf(H))
         return float(E[0]), g, H.reshape(6, 6)
+
+    def vf_local(self, p, a, b, c, r, k):
+        """Energy, gradient [12] and Hessian [12][12] of one vertex-face term."""
+        E = np.zeros(1)
+        g = np.zeros(12)
+        H = np.zeros(144)
+        f = lambda v: np.ascontiguousarray(v, np.float64).reshape(-1)  # noqa: E731
+        self.lib.or_vf_local(_pf(f(p)), _pf(f(a)), _pf(f(b)), _pf(f(c)), float(r), float(k),
+                             _pf(E), _pf(g), _pf(H))
+        return float(E[0]), g, H.reshape(12, 12)
 
     def area_local(self, x0, x1, x2, A0, k):
         """Energy, gradient [9] and Hessian [9][9] of one area-preservation face."""

@@ -37,6 +37,8 @@
  *   sym. Dirichlet E = A (|J|_F^2 + |J^-1|_F^2),  J = [u1-u0, u2-u0] Dm^-1
  *   ARAP           E = A |J - R(J)|_F^2, R(J) the closest rotation
  *   area           E = 1/2 k (A - A0)^2 / A0  (3D triangle area A)
+ *   vertex-face    E = 1/2 k (d - r)^2, d the signed distance of a vertex
+ *                  to a triangle's plane (local term only, so far)
  *
  * Parity pins: every function here is pinned by tests/test_oracle.py against
  * closed-form values, finite differences, symmetry, translation / rotation
@@ -353,6 +355,106 @@ void or_area_local(const double* x0, const double* x1, const double* x2, double 
 #else
       H[i * 9 + j] = k / A0 * (dA[i] * dA[j] + dev * d2A[i][j]);
 #endif
+    }
+}
+
+/* Vertex-face term (a 4-vertex stencil p, a, b, c; 12 variables): the
+ * signed distance from p to the plane of the triangle (a, b, c),
+ *   d = u . nh,  u = p - a,  n = e1 x e2,  e1 = b - a,  e2 = c - a,  nh = n/|n|,
+ * penalised as E = 1/2 k (d - r)^2.
+ * With m = |n|:
+ *   dd/du = nh,   dd/dn = w = (I - nh nh^T) u / m,
+ *   d2d/du dn = (I - nh nh^T) / m,   d2d/du2 = 0,
+ *   d2d/dn2 = (-(u nh^T + nh u^T) - d I + 3 d nh nh^T) / m^2.
+ * u takes (p, a, b, c) with Ju = [I, -I, 0, 0]; n takes them with
+ * Jn = [0, [e2 - e1], -[e2], [e1]] ([a] the cross-product matrix), and n is
+ * bilinear in (e1, e2), which adds sum_c w_c d2 n_c: the form with
+ * Q[a][b] = sum_c eps_cab w_c and corner coefficients p1 = (0, -1, 1, 0) on
+ * e1 and p2 = (0, -1, 0, 1) on e2, block (i, j) = p1_i p2_j Q + p2_i p1_j Q^T.
+ *   g = k (d - r) grad d,   H = k (grad d grad d^T + (d - r) hess d).
+ * Output g[12] = (p, a, b, c), H 12x12 row-major.                          */
+void or_vf_local(const double* p, const double* a, const double* b, const double* c, double r,
+                 double k, double* E, double* g, double* H) {
+  double u[3], e1[3], e2[3], d21[3], n[3];
+  for (int q = 0; q < 3; ++q) {
+    u[q] = p[q] - a[q];
+    e1[q] = b[q] - a[q];
+    e2[q] = c[q] - a[q];
+    d21[q] = e2[q] - e1[q];
+  }
+  n[0] = e1[1] * e2[2] - e1[2] * e2[1];
+  n[1] = e1[2] * e2[0] - e1[0] * e2[2];
+  n[2] = e1[0] * e2[1] - e1[1] * e2[0];
+  double m = sqrt(n[0] * n[0] + n[1] * n[1] + n[2] * n[2]);
+  double nh[3] = {n[0] / m, n[1] / m, n[2] / m};
+  double d = u[0] * nh[0] + u[1] * nh[1] + u[2] * nh[2];
+  double P[3][3]; /* I - nh nh^T */
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 3; ++j) P[i][j] = (i == j ? 1.0 : 0.0) - nh[i] * nh[j];
+  double w[3];
+  for (int i = 0; i < 3; ++i) w[i] = (P[i][0] * u[0] + P[i][1] * u[1] + P[i][2] * u[2]) / m;
+  /* Jz = [Ju; Jn], 6 x 12 */
+  double C0[3][3], C1[3][3], C2[3][3];
+  cross_mat(d21, C0);
+  cross_mat(e2, C1);
+  cross_mat(e1, C2);
+  double Jz[6][12];
+  memset(Jz, 0, sizeof(Jz));
+  for (int i = 0; i < 3; ++i) {
+    Jz[i][i] = 1.0;
+    Jz[i][3 + i] = -1.0;
+    for (int j = 0; j < 3; ++j) {
+      Jz[3 + i][3 + j] = C0[i][j];
+      Jz[3 + i][6 + j] = -C1[i][j];
+      Jz[3 + i][9 + j] = C2[i][j];
+    }
+  }
+  double dz[6] = {nh[0], nh[1], nh[2], w[0], w[1], w[2]};
+  double Dz[6][6];
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 3; ++j) {
+      Dz[i][j] = 0.0;
+      Dz[i][3 + j] = P[i][j] / m;
+      Dz[3 + i][j] = P[j][i] / m;
+      Dz[3 + i][3 + j] = (-(u[i] * nh[j] + nh[i] * u[j]) - d * (i == j ? 1.0 : 0.0) +
+                          3.0 * d * nh[i] * nh[j]) / (m * m);
+    }
+  double gd[12];
+  for (int q = 0; q < 12; ++q) {
+    double t = 0.0;
+    for (int z = 0; z < 6; ++z) t += Jz[z][q] * dz[z];
+    gd[q] = t;
+  }
+  double Q[3][3];
+  for (int i = 0; i < 3; ++i)
+    for (int j = 0; j < 3; ++j) {
+      double t = 0.0;
+      for (int cc = 0; cc < 3; ++cc) {
+        int eps = 0;
+        if ((cc == 0 && i == 1 && j == 2) || (cc == 1 && i == 2 && j == 0) ||
+            (cc == 2 && i == 0 && j == 1))
+          eps = 1;
+        if ((cc == 0 && i == 2 && j == 1) || (cc == 1 && i == 0 && j == 2) ||
+            (cc == 2 && i == 1 && j == 0))
+          eps = -1;
+        t += eps * w[cc];
+      }
+      Q[i][j] = t;
+    }
+  const double p1[4] = {0.0, -1.0, 1.0, 0.0}, p2[4] = {0.0, -1.0, 0.0, 1.0};
+  double dev = d - r;
+  *E = 0.5 * k * dev * dev;
+  for (int q = 0; q < 12; ++q) g[q] = k * dev * gd[q];
+  for (int i = 0; i < 12; ++i)
+    for (int j = 0; j < 12; ++j) {
+      double t = 0.0;
+      for (int y = 0; y < 6; ++y)
+        for (int z = 0; z < 6; ++z) t += Jz[y][i] * Dz[y][z] * Jz[z][j];
+      int vi = i / 3, ai = i % 3, vj = j / 3, aj = j % 3;
+#if OR_MUTANT != 9 /* planted (9): bilinear part of n dropped */
+      t += p1[vi] * p2[vj] * Q[ai][aj] + p2[vi] * p1[vj] * Q[aj][ai];
+#endif
+      H[i * 12 + j] = k * (gd[i] * gd[j] + dev * t);
     }
 }
 
