@@ -82,6 +82,13 @@ class Oracle:
                                 ctypes.c_int32, _i32p, _f64p, ctypes.c_double,
                                 _i32p, _i32p, _f64p, _f64p, _f64p]
         lib.or_eval.restype = ctypes.c_int
+        lib.or_eval3.argtypes = [ctypes.c_int32, ctypes.c_int, _f64p, ctypes.c_uint,
+                                 ctypes.c_int32, _i32p, _f64p, ctypes.c_double, _f64p,
+                                 ctypes.c_double, ctypes.c_int32, _i32p, _f64p, _f64p,
+                                 ctypes.c_int32, _i32p, _f64p, ctypes.c_double, ctypes.c_double,
+                                 ctypes.c_int32, _i32p, _f64p, ctypes.c_double,
+                                 _i32p, _i32p, _f64p, _f64p, _f64p]
+        lib.or_eval3.restype = ctypes.c_int
         lib.or_eval2.argtypes = [ctypes.c_int32, ctypes.c_int, _f64p, ctypes.c_uint,
                                  ctypes.c_int32, _i32p, _f64p, ctypes.c_double, _f64p,
                                  ctypes.c_double, ctypes.c_int32, _i32p, _f64p, _f64p,
@@ -177,14 +184,17 @@ class Oracle:
     # ---- assembly -------------------------------------------------------
     def eval(self, V, dof, x, mask, row_ptr, col_idx, *, edges=None, L0=None, k=0.0,
              xt=None, w=0.0, F=None, Minv=None, area=None, pairs=None, prest=None,
-             kp=0.0, ka=0.0):
-        """Assemble g [V][dof], H_vals [nnzb][dof][dof] and the energy (fp64)."""
+             kp=0.0, ka=0.0, vf=None, vf_rest=None, kc=0.0):
+        """Assemble g [V][dof], H_vals [nnzb][dof][dof] and the energy (fp64).
+        vf: int [nVF][2] (vertex, face) vertex-face terms (mask bit 64)."""
         f64 = lambda a: None if a is None else np.ascontiguousarray(a, np.float64)  # noqa: E731
         i32 = lambda a: None if a is None else np.ascontiguousarray(a, np.int32)  # noqa: E731
         x = f64(x).reshape(-1)
         row_ptr, col_idx = i32(row_ptr), i32(col_idx)
-        edges, F, pairs = i32(edges), i32(F), i32(pairs)
+        edges, F, pairs, vf = i32(edges), i32(F), i32(pairs), i32(vf)
         L0, xt, Minv, area, prest = f64(L0), f64(xt), f64(Minv), f64(area), f64(prest)
+        vf_rest = f64(vf_rest)
+        nVF = 0 if vf is None else vf.reshape(-1, 2).shape[0]
         nE = 0 if edges is None else edges.reshape(-1, 2).shape[0]
         nF = 0 if F is None else F.reshape(-1, 3).shape[0]
         nP = 0 if pairs is None else pairs.reshape(-1, 2).shape[0]
@@ -192,9 +202,10 @@ class Oracle:
         g = np.zeros(V * dof)
         H = np.zeros(nnzb * dof * dof)
         E = np.zeros(1)
-        r = self.lib.or_eval2(V, dof, _pf(x), mask, nE, _p32(edges), _pf(L0), float(k),
+        r = self.lib.or_eval3(V, dof, _pf(x), mask, nE, _p32(edges), _pf(L0), float(k),
                               _pf(xt), float(w), nF, _p32(F), _pf(Minv), _pf(area),
                               nP, _p32(pairs), _pf(prest), float(kp), float(ka),
+                              nVF, _p32(vf), _pf(vf_rest), float(kc),
                               _p32(row_ptr), _p32(col_idx), _pf(g), _pf(H), _pf(E))
         if r != 0:
             raise ValueError(f"or_eval failed: {r}")

@@ -38,7 +38,7 @@
  *   ARAP           E = A |J - R(J)|_F^2, R(J) the closest rotation
  *   area           E = 1/2 k (A - A0)^2 / A0  (3D triangle area A)
  *   vertex-face    E = 1/2 k (d - r)^2, d the signed distance of a vertex
- *                  to a triangle's plane (local term only, so far)
+ *                  to a triangle's plane
  *
  * Parity pins: every function here is pinned by tests/test_oracle.py against
  * closed-form values, finite differences, symmetry, translation / rotation
@@ -632,8 +632,11 @@ static int emit_blocks(or_coo* c, int dof, int nv, const int32_t* vid,
 /* mask bits: 1 spring, 2 inertia, 4 symmetric Dirichlet (dof 2, with Minv
  * and area = rest area), 8 pairs, 16 area preservation (dof 3, with area =
  * rest area A0 and stiffness ka), 32 ARAP (dof 2, with Minv and area, like
- * symmetric Dirichlet). */
-int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
+ * symmetric Dirichlet), 64 vertex-face terms (dof 3: term t couples vertex
+ * vf[2t] with the corners of face vf[2t+1], rest offset vf_rest[t],
+ * stiffness kc; the pattern must hold the blocks between the vertex and the
+ * corners). */
+int or_eval3(int32_t V, int dof, const double* x, unsigned mask,
              /* springs */ int32_t nE, const int32_t* edges, const double* L0,
              double k,
              /* inertia */ const double* xt, double w,
@@ -642,9 +645,36 @@ int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
              /* pairs */ int32_t nP, const int32_t* pairs, const double* prest,
              double kp,
              /* area preservation */ double ka,
+             /* vertex-face */ int32_t nVF, const int32_t* vf, const double* vf_rest,
+             double kc,
+             /* pattern */ const int32_t* row_ptr, const int32_t* col_idx,
+             /* out */ double* g, double* H_vals, double* energy);
+
+int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
+             int32_t nE, const int32_t* edges, const double* L0, double k,
+             const double* xt, double w, int32_t nF, const int32_t* F,
+             const double* Minv, const double* area, int32_t nP, const int32_t* pairs,
+             const double* prest, double kp, double ka, const int32_t* row_ptr,
+             const int32_t* col_idx, double* g, double* H_vals, double* energy) {
+  return or_eval3(V, dof, x, mask & ~64u, nE, edges, L0, k, xt, w, nF, F, Minv, area, nP, pairs,
+                  prest, kp, ka, 0, NULL, NULL, 0.0, row_ptr, col_idx, g, H_vals, energy);
+}
+
+int or_eval3(int32_t V, int dof, const double* x, unsigned mask,
+             /* springs */ int32_t nE, const int32_t* edges, const double* L0,
+             double k,
+             /* inertia */ const double* xt, double w,
+             /* faces */ int32_t nF, const int32_t* F,
+             const double* Minv, const double* area,
+             /* pairs */ int32_t nP, const int32_t* pairs, const double* prest,
+             double kp,
+             /* area preservation */ double ka,
+             /* vertex-face */ int32_t nVF, const int32_t* vf, const double* vf_rest,
+             double kc,
              /* pattern */ const int32_t* row_ptr, const int32_t* col_idx,
              /* out */ double* g, double* H_vals, double* energy) {
   if (dof != 2 && dof != 3) return OR_ERR_ARG;
+  if ((mask & 64) && dof != 3) return OR_ERR_ARG;
   if ((mask & 4) && dof != 2) return OR_ERR_ARG;
   if ((mask & 16) && dof != 3) return OR_ERR_ARG;
   if ((mask & 32) && dof != 2) return OR_ERR_ARG;
@@ -656,6 +686,7 @@ int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
   if (mask & 8) n += 4 * (int64_t)nP;
   if (mask & 16) n += 9 * (int64_t)nF;
   if (mask & 32) n += 9 * (int64_t)nF;
+  if (mask & 64) n += 16 * (int64_t)nVF;
   or_coo c;
   c.bs = bs;
   c.cap = n > 0 ? n : 1;
@@ -668,7 +699,7 @@ int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
     return OR_ERR_OOM;
   }
   for (int64_t i = 0; i < (int64_t)V * dof; ++i) g[i] = 0.0;
-  double Etot = 0.0, E, gl[9], Hl[81];
+  double Etot = 0.0, E, gl[12], Hl[144];
   int rc = OR_OK;
   if (mask & 1)
     for (int32_t e = 0; e < nE && !rc; ++e) {
@@ -718,6 +749,21 @@ int or_eval2(int32_t V, int dof, const double* x, unsigned mask,
       for (int p = 0; p < 3; ++p)
         for (int a = 0; a < 3; ++a) g[(size_t)vid[p] * 3 + a] += gl[p * 3 + a];
       rc = emit_blocks(&c, 3, 3, vid, Hl);
+    }
+  if (mask & 64)
+    for (int32_t t = 0; t < nVF && !rc; ++t) {
+      const int32_t f = vf[2 * t + 1];
+      if (f < 0 || f >= nF) {
+        rc = OR_ERR_ARG;
+        break;
+      }
+      int32_t vid[4] = {vf[2 * t], F[3 * f], F[3 * f + 1], F[3 * f + 2]};
+      or_vf_local(x + (size_t)vid[0] * 3, x + (size_t)vid[1] * 3, x + (size_t)vid[2] * 3,
+                  x + (size_t)vid[3] * 3, vf_rest[t], kc, &E, gl, Hl);
+      Etot += E;
+      for (int q = 0; q < 4; ++q)
+        for (int a = 0; a < 3; ++a) g[(size_t)vid[q] * 3 + a] += gl[q * 3 + a];
+      rc = emit_blocks(&c, 3, 4, vid, Hl);
     }
   if (mask & 8)
     for (int32_t p = 0; p < nP && !rc; ++p) {

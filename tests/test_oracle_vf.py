@@ -96,3 +96,52 @@ def test_vf_pins_pass_on_oracle(orc):
 
 def test_vf_pins_catch_planted_mistake():
     assert not _vf_pins_pass(oracle.load_mutant(9))
+
+
+def vf_pairs(vf, F):
+    """The three vertex pairs that a vertex-face term adds to the pattern."""
+    return np.array([(p, F[f][c]) for p, f in vf for c in range(3)], np.int32)
+
+
+def test_vf_assembled_on_cloth_fd(orc):
+    import mesh_inputs as mi
+    n = 5
+    st = mi.cloth_static(n, np.float64)
+    V, F = st["V"], st["F"]
+    rng = np.random.default_rng(9)
+    x = mi.cloth_x(n, 22, 0, np.float64) + 0.05 * rng.standard_normal((V, 3))
+    vf = []
+    while len(vf) < 6:
+        p, f = int(rng.integers(0, V)), int(rng.integers(0, len(F)))
+        if p not in F[f]:
+            vf.append((p, f))
+    vf = np.array(vf, np.int32)
+    rest = 0.01 * rng.standard_normal(len(vf))
+    rp, ci = orc.pattern(V, F, vf_pairs(vf, F))
+    kc = 40.0
+
+    def ev(xx):
+        return orc.eval(V, 3, xx, 2 | 64, rp, ci, xt=st["xt"], w=st["w"], F=F, vf=vf,
+                        vf_rest=rest, kc=kc)
+
+    g, H, E = ev(x)
+    Eloc = sum(orc.vf_local(x[p], *x[F[f]], r, kc)[0] for (p, f), r in zip(vf, rest))
+    Ein = 0.5 * st["w"] * np.sum((x - st["xt"]) ** 2)
+    assert E == pytest.approx(Eloc + Ein, rel=1e-12)
+    D = np.zeros((3 * V, 3 * V))
+    for i in range(V):
+        for q in range(rp[i], rp[i + 1]):
+            D[3 * i:3 * i + 3, 3 * ci[q]:3 * ci[q] + 3] = H[q]
+    np.testing.assert_allclose(D, D.T, atol=1e-12 * np.abs(D).max())
+    h = 1e-6
+    xf = x.reshape(-1)
+    touched = sorted({int(vf[0, 0]), *map(int, F[vf[0, 1]])})
+    for c in [3 * touched[0], 3 * touched[1] + 2, 3 * touched[-1] + 1, 0]:
+        xp = xf.copy()
+        xm = xf.copy()
+        xp[c] += h
+        xm[c] -= h
+        gp, _, Ep = ev(xp.reshape(-1, 3))
+        gm, _, Em = ev(xm.reshape(-1, 3))
+        assert g.reshape(-1)[c] == pytest.approx((Ep - Em) / (2 * h), abs=1e-6)
+        np.testing.assert_allclose(D[:, c], (gp - gm).reshape(-1) / (2 * h), atol=1e-5)
