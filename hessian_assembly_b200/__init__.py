@@ -43,6 +43,7 @@ MAD_TERM_SYMDIR = 4
 MAD_TERM_PAIR = 8
 MAD_TERM_AREA = 16
 MAD_TERM_ARAP = 32
+MAD_TERM_VF = 64
 MAD_EVAL_FULL_STENCIL_AD = 1
 MAD_EVAL_EDGE_SCATTER = 2
 MAD_EVAL_PATCH_STAGED = 4
@@ -69,7 +70,9 @@ class mad_terms(ctypes.Structure):
                 ("spring_rest", ctypes.c_void_p), ("spring_k", ctypes.c_double),
                 ("inertia_xt", ctypes.c_void_p), ("inertia_w", ctypes.c_double),
                 ("face_Minv", ctypes.c_void_p), ("face_area", ctypes.c_void_p),
-                ("pair_k", ctypes.c_double), ("area_k", ctypes.c_double)]
+                ("pair_k", ctypes.c_double), ("area_k", ctypes.c_double),
+                ("vf_n", ctypes.c_int32), ("vf", ctypes.c_void_p), ("vf_rest", ctypes.c_void_p),
+                ("vf_k", ctypes.c_double)]
 
 
 class mad_info_t(ctypes.Structure):
@@ -192,14 +195,21 @@ class Terms:
     face_area: object = None
     pair_k: float = 0.0
     area_k: float = 0.0
+    vf: object = None        # int32 [n][2] (vertex, face)
+    vf_rest: object = None
+    vf_k: float = 0.0
 
     def to_c(self, dtype) -> mad_terms:
+        torch = _torch()
         p = lambda t, n: None if t is None else _dev_ptr(t, dtype, n)  # noqa: E731
+        nvf = 0 if self.vf is None else int(self.vf.shape[0])
         return mad_terms(self.mask, self.flags, p(self.spring_rest, "spring_rest"),
                          float(self.spring_k), p(self.inertia_xt, "inertia_xt"),
                          float(self.inertia_w), p(self.face_Minv, "face_Minv"),
                          p(self.face_area, "face_area"), float(self.pair_k),
-                         float(self.area_k))
+                         float(self.area_k), nvf,
+                         None if self.vf is None else _dev_ptr(self.vf, torch.int32, "vf"),
+                         p(self.vf_rest, "vf_rest"), float(self.vf_k))
 
 
 class Context:

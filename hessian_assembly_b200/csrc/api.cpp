@@ -207,6 +207,24 @@ RowsLaunch rows_launch(const mad_ctx* c) {
   return L;
 }
 
+// The vertex-face pass reads the active pattern: the mesh pattern, or the
+// buffer that the last mad_add_pairs filled.
+VfLaunch vf_launch(const mad_ctx* c, const mad_terms* t, const void* x) {
+  VfLaunch L;
+  L.n = t->vf_n;
+  L.V = c->V;
+  L.nF = c->nF;
+  L.vf = t->vf;
+  L.rest = t->vf_rest;
+  L.k = t->vf_k;
+  L.F = c->F_dev;
+  L.x = x;
+  L.rp = c->active < 0 ? c->pat.rp : c->buf[c->active].rp;
+  L.ci = c->active < 0 ? c->pat.ci : c->buf[c->active].ci;
+  L.status = c->status;
+  return L;
+}
+
 // Every term set goes to the row-streaming kernel unless the caller asks for
 // the patch kernel or the scatter mode, or face terms meet a mesh whose face
 // rows could not be built.
@@ -219,8 +237,16 @@ bool use_rows(const mad_ctx* c, const mad_terms* t) {
 mad_status check_terms(mad_ctx* c, const mad_terms* t) {
   if (!t) return fail(c, MAD_ERR_INVALID_ARG, "terms is NULL");
   const uint32_t known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR |
-                         MAD_TERM_AREA | MAD_TERM_ARAP;
+                         MAD_TERM_AREA | MAD_TERM_ARAP | MAD_TERM_VF;
   if (t->mask & ~known) return fail(c, MAD_ERR_INVALID_ARG, "unknown term bits in mask");
+  if (t->mask & MAD_TERM_VF) {
+    if (c->dof != 3) return fail(c, MAD_ERR_UNIMPLEMENTED, "vertex-face terms need dof 3");
+    if (t->mask & MAD_TERM_PAIR)
+      return fail(c, MAD_ERR_UNIMPLEMENTED, "vertex-face terms with pair terms in one mask");
+    if (t->vf_n < 0) return fail(c, MAD_ERR_INVALID_ARG, "vf_n < 0");
+    if (t->vf_n > 0 && (!t->vf || !t->vf_rest))
+      return fail(c, MAD_ERR_INVALID_ARG, "vertex-face terms need vf and vf_rest");
+  }
   if (t->flags &
       ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED))
     return fail(c, MAD_ERR_INVALID_ARG, "unknown evaluation flags");
@@ -563,6 +589,10 @@ mad_status mad_eval(mad_ctx* c, const void* x, const mad_terms* t, void* g, void
     e = launch_eval(eval_launch(c), *t, x, g, H_vals, energy, as_stream(stream));
   }
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval launch");
+  if ((t->mask & MAD_TERM_VF) && t->vf_n > 0) {
+    e = launch_vf_eval(c->dtype, vf_launch(c, t, x), g, H_vals, energy, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval vertex-face launch");
+  }
   return MAD_OK;
 }
 
@@ -576,6 +606,10 @@ mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t, const void* v,
   cudaError_t e = use_rows(c, t) ? launch_rows_hvp(rows_launch(c), *t, x, v, y, as_stream(stream))
                               : launch_hvp(eval_launch(c), *t, x, v, y, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_hvp launch");
+  if ((t->mask & MAD_TERM_VF) && t->vf_n > 0) {
+    e = launch_vf_hvp(c->dtype, vf_launch(c, t, x), v, y, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(c, e, "mad_hvp vertex-face launch");
+  }
   return MAD_OK;
 }
 
@@ -614,13 +648,13 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij, const void* r
 namespace {
 mad_status jac_mask_ok(const mad_ctx* c, uint32_t mask, std::string* why) {
   const uint32_t known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR |
-                         MAD_TERM_AREA | MAD_TERM_ARAP;
+                         MAD_TERM_AREA | MAD_TERM_ARAP | MAD_TERM_VF;
   if (mask & ~known) {
     *why = "unknown term bits in mask";
     return MAD_ERR_INVALID_ARG;
   }
-  if (mask & (MAD_TERM_PAIR | MAD_TERM_AREA | MAD_TERM_ARAP)) {
-    *why = "pair, area and ARAP terms are not part of the vector-valued objective";
+  if (mask & (MAD_TERM_PAIR | MAD_TERM_AREA | MAD_TERM_ARAP | MAD_TERM_VF)) {
+    *why = "pair, area, ARAP and vertex-face terms are not part of the vector-valued objective";
     return MAD_ERR_UNIMPLEMENTED;
   }
   if ((mask & MAD_TERM_SYMDIR) && c->dof != 2) {

@@ -146,6 +146,22 @@ struct DynBuf {
   void* pe_rest = nullptr;    // [2*max_pairs] rest length (dtype)
 };
 
+// vertex-face terms (vf.cu): the active pattern, the terms and positions
+struct VfLaunch {
+  int n = 0, V = 0, nF = 0;
+  const int32_t* vf = nullptr;
+  const void* rest = nullptr;
+  double k = 0.0;
+  const int32_t* F = nullptr;
+  const void* x = nullptr;
+  const int32_t* rp = nullptr;
+  const int32_t* ci = nullptr;
+  int32_t* status = nullptr;
+};
+cudaError_t launch_vf_eval(int dtype, const VfLaunch& L, void* g, void* H, double* energy,
+                           cudaStream_t s);
+cudaError_t launch_vf_hvp(int dtype, const VfLaunch& L, const void* v, void* y, cudaStream_t s);
+
 // ---- launchers (defined in the .cu files) ------------------------------
 // scan.cu: exclusive scan of n int32 values in -> out[0..n], out[n] = total.
 // tmp must hold scan_tmp_elems(n) ints.

@@ -180,9 +180,12 @@ extern "C" mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, c
     return MAD_ERR_INVALID_ARG;
   }
   const unsigned known = MAD_TERM_SPRING | MAD_TERM_INERTIA | MAD_TERM_SYMDIR | MAD_TERM_PAIR |
-                         MAD_TERM_AREA | MAD_TERM_ARAP;
+                         MAD_TERM_AREA | MAD_TERM_ARAP | MAD_TERM_VF;
   if (t->mask & ~known) {
     return MAD_ERR_INVALID_ARG;
+  }
+  if (t->mask & MAD_TERM_VF) {
+    return MAD_ERR_UNIMPLEMENTED;
   }
   const bool sp = (t->mask & MAD_TERM_SPRING) && nE > 0;
   const bool in = (t->mask & MAD_TERM_INERTIA) && V > 0;

@@ -1,0 +1,239 @@
+// vf.cu -- vertex-face terms: a vertex p and the three corners (a, b, c) of a
+// mesh face, a 4-vertex stencil with 12 variables and sixteen 3x3 blocks.
+//
+// Page "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
+// Computations", section 方法 (key design 4: runtime terms whose blocks are
+// inserted into the CSR on the GPU) and section 实验结果 (the contact shell,
+// whose vertex-face terms change every step).  The energy is
+//   E = 1/2 k (d - r)^2,  d = (p - a) . n / |n|,  n = (b - a) x (c - a),
+// the signed distance of p to the face's plane against a rest offset r.
+//
+// The blocks between p and the corners are the three vertex pairs of each
+// term, inserted by mad_add_pairs; the blocks among the corners are mesh
+// blocks.  One thread evaluates one term, after the row kernel has written
+// every row, and adds its gradient, blocks and energy with atomics: the
+// scatter form of the pages' key design 4.  Contributions of several terms to
+// one block therefore add in no fixed order.
+//
+// Forward-mode AD on masked numbers (sparse_ad.cuh) seeded on the natural
+// variables z = (u, e1, e2) = (p - a, b - a, c - a), width 9; the stencil's
+// coefficients on z are p: (1, 0, 0), a: (-1, -1, -1), b: (0, 1, 0),
+// c: (0, 0, 1), so block (i, j) = sum_{s,t} c_i[s] c_j[t] H_z(s, t).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mad_internal.h"
+#include "sparse_ad.cuh"
+
+namespace mad {
+namespace {
+
+constexpr int kVfThreads = 256;
+
+// coefficient of stencil vertex v (p, a, b, c) on natural variable s (u, e1, e2)
+__host__ __device__ constexpr int vf_coef(int v, int s) {
+  return v == 0 ? (s == 0 ? 1 : 0) : v == 1 ? -1 : (v - 1 == s ? 1 : 0);
+}
+
+template <typename T, int N, uint32_t G>
+__device__ __forceinline__ SHD<T, N, G, 0> to_shd(const SLin<T, N, G>& a) {
+  SHD<T, N, G, 0> r;
+  r.v = a.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (mbit(G, i)) r.g[i] = a.g[i];
+  return r;
+}
+
+// E and its derivatives in z of one term: value, gradient [9], Hessian (packed)
+template <typename T>
+__device__ __forceinline__ auto vf_energy(const T* p, const T* a, const T* b, const T* c, T r,
+                                          T k) {
+  const auto u0 = to_shd(slin_var<T, 9, 0>(p[0] - a[0]));
+  const auto u1 = to_shd(slin_var<T, 9, 1>(p[1] - a[1]));
+  const auto u2 = to_shd(slin_var<T, 9, 2>(p[2] - a[2]));
+  const auto e10 = slin_var<T, 9, 3>(b[0] - a[0]);
+  const auto e11 = slin_var<T, 9, 4>(b[1] - a[1]);
+  const auto e12 = slin_var<T, 9, 5>(b[2] - a[2]);
+  const auto e20 = slin_var<T, 9, 6>(c[0] - a[0]);
+  const auto e21 = slin_var<T, 9, 7>(c[1] - a[1]);
+  const auto e22 = slin_var<T, 9, 8>(c[2] - a[2]);
+  const auto n0 = e11 * e22 - e12 * e21;
+  const auto n1 = e12 * e20 - e10 * e22;
+  const auto n2 = e10 * e21 - e11 * e20;
+  const auto un = u0 * n0 + u1 * n1 + u2 * n2;
+  const auto nn = sq(n0) + sq(n1) + sq(n2);
+  // 1/|n| as one chain step: s^(-1/2), -1/2 s^(-3/2), 3/4 s^(-5/2)
+  const T is = T(1) / ::sqrt(nn.v);
+  const T is2 = is * is;
+  const auto inv_m = chain(nn, is, T(-0.5) * is * is2, T(0.75) * is * is2 * is2);
+  const auto d = un * inv_m;
+  const T dev = d.v - r;
+  return chain(d, T(0.5) * k * dev * dev, k * dev, k);
+}
+
+__device__ __forceinline__ int find_col(const int32_t* __restrict__ rp,
+                                        const int32_t* __restrict__ ci, int row, int col) {
+  int lo = rp[row], hi = rp[row + 1];
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (ci[mid] < col) lo = mid + 1;
+    else hi = mid;
+  }
+  return (lo < rp[row + 1] && ci[lo] == col) ? lo : -1;
+}
+
+template <typename T>
+__device__ __forceinline__ bool load_term(int t, const int32_t* __restrict__ vf,
+                                          const int32_t* __restrict__ F, int nF, int V,
+                                          const T* __restrict__ x, int vid[4], T X[4][3]) {
+  const int p = vf[2 * t], f = vf[2 * t + 1];
+  if (p < 0 || p >= V || f < 0 || f >= nF) return false;
+  vid[0] = p;
+  vid[1] = F[3 * f];
+  vid[2] = F[3 * f + 1];
+  vid[3] = F[3 * f + 2];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int al = 0; al < 3; ++al) X[q][al] = x[(int64_t)vid[q] * 3 + al];
+  return true;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kVfThreads) k_vf_eval(
+    int n, const int32_t* __restrict__ vf, const T* __restrict__ rest, T k,
+    const int32_t* __restrict__ F, int nF, int V, const T* __restrict__ x,
+    const int32_t* __restrict__ rp, const int32_t* __restrict__ ci, T* __restrict__ g,
+    T* __restrict__ H, double* energy, int32_t* status) {
+  const int t = blockIdx.x * kVfThreads + threadIdx.x;
+  double e = 0.0;
+  int vid[4];
+  T X[4][3];
+  if (t < n) {
+    if (!load_term<T>(t, vf, F, nF, V, x, vid, X)) {
+      atomicOr(status, kStatusIndex);
+    } else {
+      const auto z = vf_energy<T>(X[0], X[1], X[2], X[3], rest[t], k);
+      e = (double)z.v;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int al = 0; al < 3; ++al) {
+          T s = T(-0.0);
+#pragma unroll
+          for (int sv = 0; sv < 3; ++sv)
+            if (vf_coef(i, sv) != 0) s += T(vf_coef(i, sv)) * sgrad(z, 3 * sv + al);
+          atomicAdd(&g[(int64_t)vid[i] * 3 + al], s);
+        }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int pos = find_col(rp, ci, vid[i], vid[j]);
+          if (pos < 0) {
+            atomicOr(status, kStatusIndex);
+            continue;
+          }
+          T* blk = H + (int64_t)pos * 9;
+#pragma unroll
+          for (int al = 0; al < 3; ++al)
+#pragma unroll
+            for (int be = 0; be < 3; ++be) {
+              T s = T(-0.0);
+#pragma unroll
+              for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+                for (int tv = 0; tv < 3; ++tv)
+                  if (vf_coef(i, sv) * vf_coef(j, tv) != 0)
+                    s += T(vf_coef(i, sv) * vf_coef(j, tv)) * shess(z, 3 * sv + al, 3 * tv + be);
+              atomicAdd(&blk[3 * al + be], s);
+            }
+        }
+    }
+  }
+  if (energy) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e += __shfl_down_sync(0xFFFFFFFFu, e, o);
+    if ((threadIdx.x & 31) == 0 && e != 0.0) atomicAdd(energy, e);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kVfThreads) k_vf_hvp(
+    int n, const int32_t* __restrict__ vf, const T* __restrict__ rest, T k,
+    const int32_t* __restrict__ F, int nF, int V, const T* __restrict__ x,
+    const T* __restrict__ v, T* __restrict__ y, int32_t* status) {
+  const int t = blockIdx.x * kVfThreads + threadIdx.x;
+  if (t >= n) return;
+  int vid[4];
+  T X[4][3];
+  if (!load_term<T>(t, vf, F, nF, V, x, vid, X)) {
+    atomicOr(status, kStatusIndex);
+    return;
+  }
+  const auto z = vf_energy<T>(X[0], X[1], X[2], X[3], rest[t], k);
+  // dz_s = sum_j c_j[s] v_j, t = H_z dz, y_i = sum_s c_i[s] t_s
+  T dz[9];
+#pragma unroll
+  for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+    for (int al = 0; al < 3; ++al) {
+      T s = T(-0.0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (vf_coef(j, sv) != 0) s += T(vf_coef(j, sv)) * v[(int64_t)vid[j] * 3 + al];
+      dz[3 * sv + al] = s;
+    }
+  T tz[9];
+#pragma unroll
+  for (int q = 0; q < 9; ++q) {
+    T s = shess(z, q, 0) * dz[0];
+#pragma unroll
+    for (int w = 1; w < 9; ++w) s += shess(z, q, w) * dz[w];
+    tz[q] = s;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int al = 0; al < 3; ++al) {
+      T s = T(-0.0);
+#pragma unroll
+      for (int sv = 0; sv < 3; ++sv)
+        if (vf_coef(i, sv) != 0) s += T(vf_coef(i, sv)) * tz[3 * sv + al];
+      atomicAdd(&y[(int64_t)vid[i] * 3 + al], s);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_vf_eval(int dtype, const VfLaunch& L, void* g, void* H, double* energy,
+                           cudaStream_t s) {
+  if (L.n <= 0) return cudaSuccess;
+  const unsigned nb = (unsigned)((L.n + kVfThreads - 1) / kVfThreads);
+  if (dtype == MAD_F64)
+    k_vf_eval<double><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const double*)L.rest, L.k, L.F,
+                                               L.nF, L.V, (const double*)L.x, L.rp, L.ci,
+                                               (double*)g, (double*)H, energy, L.status);
+  else
+    k_vf_eval<float><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const float*)L.rest, (float)L.k, L.F,
+                                              L.nF, L.V, (const float*)L.x, L.rp, L.ci,
+                                              (float*)g, (float*)H, energy, L.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vf_hvp(int dtype, const VfLaunch& L, const void* v, void* y, cudaStream_t s) {
+  if (L.n <= 0) return cudaSuccess;
+  const unsigned nb = (unsigned)((L.n + kVfThreads - 1) / kVfThreads);
+  if (dtype == MAD_F64)
+    k_vf_hvp<double><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const double*)L.rest, L.k, L.F, L.nF,
+                                              L.V, (const double*)L.x, (const double*)v,
+                                              (double*)y, L.status);
+  else
+    k_vf_hvp<float><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const float*)L.rest, (float)L.k, L.F,
+                                             L.nF, L.V, (const float*)L.x, (const float*)v,
+                                             (float*)y, L.status);
+  return cudaGetLastError();
+}
+
+}  // namespace mad

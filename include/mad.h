@@ -75,12 +75,21 @@ enum {
   MAD_TERM_AREA = 16u,   /* per face, dof 3 (a 9-variable stencil): area
                             preservation 1/2 k_a (A_f - A0_f)^2 / A0_f with
                             A_f = |(x1-x0) x (x2-x0)| / 2, A0_f = face_area */
-  MAD_TERM_ARAP = 32u    /* per face, dof 2: as-rigid-as-possible
+  MAD_TERM_ARAP = 32u,   /* per face, dof 2: as-rigid-as-possible
                             A_f |J - R(J)|_F^2, J as for MAD_TERM_SYMDIR
                             (same face_Minv and face_area), R(J) the closest
                             rotation.  With MAD_TERM_SYMDIR both energies
                             are summed per face.  Needs det J > 0 (the
                             closest rotation is unique there).              */
+  MAD_TERM_VF = 64u      /* per vertex-face term (dof 3): 1/2 k_c (d - r)^2,
+                            d the signed distance of vertex p to the plane of
+                            face f (n = (x1-x0) x (x2-x0)).  The blocks
+                            between p and the face's corners must be in the
+                            pattern: insert the pairs (p, corner) of every
+                            term with mad_add_pairs.  Not with MAD_TERM_PAIR
+                            (its pair list would hold those pairs too).
+                            Terms are added with atomics, so their blocks
+                            are not bit-reproducible across runs.           */
 };
 
 /* Evaluation flags. */
@@ -132,6 +141,10 @@ typedef struct {
   const void* face_area;    /* [nF] rest area per face                       */
   double pair_k;            /* k_p for the current pair set                  */
   double area_k;            /* k_a of MAD_TERM_AREA                          */
+  int32_t vf_n;             /* number of vertex-face terms (MAD_TERM_VF)     */
+  const int32_t* vf;        /* [vf_n][2] (vertex p, face f) per term         */
+  const void* vf_rest;      /* [vf_n] rest offset r per term                 */
+  double vf_k;              /* k_c of MAD_TERM_VF                            */
 } mad_terms;
 
 typedef struct {
@@ -242,8 +255,8 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij,
  * J is scalar CSR with int64 row pointers and int32 columns; a column is
  * vertex*dof + component, ascending within each row (the stencil's vertices
  * sorted by index).  Nonzeros per row: 2*dof (spring), 1 (inertia), 6 (face).
- * MAD_TERM_PAIR, MAD_TERM_AREA and MAD_TERM_ARAP are not part of the vector
- * objective (MAD_ERR_UNIMPLEMENTED).                                        */
+ * MAD_TERM_PAIR, MAD_TERM_AREA, MAD_TERM_ARAP and MAD_TERM_VF are not part
+ * of the vector objective (MAD_ERR_UNIMPLEMENTED).                          */
 
 /* Rows and nonzeros of the Jacobian of the terms in `mask`.  Errors:
  * MAD_ERR_INVALID_ARG (NULL outputs, unknown bits), MAD_ERR_UNIMPLEMENTED

@@ -1,0 +1,96 @@
+"""Vertex-face terms (dof 3, a 4-vertex stencil with 12 variables) on the
+cloth: the pattern holds the three (vertex, corner) pairs of each term,
+inserted with mad_add_pairs; the terms are evaluated by their own pass after
+the row kernel.  Parity of g, H, the energy and the Hessian-vector product
+against the fp64 oracle, plus the refusals."""
+import numpy as np
+import pytest
+
+import mesh_inputs as mi
+from _parity import ETOL, assert_close, cloth_context, gpu_pattern, run_eval, to_dev
+
+pytestmark = pytest.mark.gpu
+VF = 64
+KC = 50.0
+
+
+def vf_terms_for(n, nvf, seed):
+    st = mi.cloth_static(n, np.float64)
+    F = st["F"]
+    rng = np.random.default_rng(seed)
+    vf = []
+    while len(vf) < nvf:
+        p, f = int(rng.integers(0, st["V"])), int(rng.integers(0, len(F)))
+        if p not in F[f]:
+            vf.append((p, f))
+    vf = np.array(vf, np.int32)
+    rest = 0.01 * rng.standard_normal(len(vf))
+    pairs = np.array([(p, F[f][c]) for p, f in vf for c in range(3)], np.int32)
+    return vf, rest, pairs
+
+
+def check(orc, n, dtype, nvf, seed, mask=1 | 2 | VF):
+    import hessian_assembly_b200 as mad
+    import torch
+    vf, rest, pairs = vf_terms_for(n, nvf, seed)
+    ctx, st = cloth_context(n, dtype, max_pairs=len(pairs) + 8, slack=0.6)
+    ctx.mad_add_pairs(to_dev(pairs), to_dev(np.zeros(len(pairs)), dtype))
+    x = mi.cloth_x(n, seed, 0, np.dtype(dtype))
+    x = (x + 0.02 * mi.grid_spacing(n) * np.random.default_rng(seed + 1).standard_normal(x.shape)
+         ).astype(dtype)
+    terms = mad.Terms(mask=mask, spring_rest=to_dev(st["L0"], dtype), spring_k=st["k"],
+                      inertia_xt=to_dev(st["xt"], dtype), inertia_w=st["w"],
+                      vf=to_dev(vf), vf_rest=to_dev(rest, dtype), vf_k=KC)
+    g, H, E = run_eval(ctx, x, terms, dtype)
+    assert ctx.mad_status_sync() == mad.MAD_OK
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(st["V"], st["F"], pairs)
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    og, oH, oE = orc.eval(st["V"], 3, x, mask, orp, oci, edges=st["edges"], L0=st["L0"],
+                          k=st["k"], xt=st["xt"], w=st["w"], F=st["F"], vf=vf,
+                          vf_rest=rest.astype(dtype), kc=KC)
+    assert_close("g", g, og, dtype)
+    assert_close("H", H[:nnzb], oH, dtype)
+    assert abs(E - oE) <= ETOL[dtype] * abs(oE)
+    v = mi.probe_vector(st["V"], 3, seed + 2, np.dtype(dtype))
+    y = torch.full((st["V"], 3), float("nan"), dtype=getattr(torch, dtype), device="cuda")
+    ctx.mad_hvp(to_dev(x, dtype), terms, to_dev(v, dtype), y)
+    torch.cuda.synchronize()
+    assert_close("y", y.cpu().numpy(), orc.bsr_mv(st["V"], 3, orp, oci, oH, v), dtype)
+    return ctx
+
+
+@pytest.mark.parametrize("dtype", ["float32", "float64"])
+def test_vf_cloth(orc, dtype):
+    check(orc, 30, dtype, 200, 6001)
+
+
+def test_vf_only_terms(orc):
+    # no row-kernel terms: rows are zeroed, the vertex-face pass alone adds
+    check(orc, 20, "float64", 120, 6002, mask=VF)
+
+
+def test_vf_many_terms_fp32(orc):
+    check(orc, 200, "float32", 20000, 6003)
+
+
+def test_vf_refusals():
+    import hessian_assembly_b200 as mad
+    import torch
+    ctx, st = cloth_context(8, "float32", max_pairs=64)
+    vf, rest, pairs = vf_terms_for(8, 4, 6004)
+    x = to_dev(mi.cloth_x(8, 1, 0, np.float32))
+    g = torch.zeros((st["V"], 3), device="cuda")
+    H = torch.zeros((ctx.info.capacity_blocks, 3, 3), device="cuda")
+    t = mad.Terms(mask=VF | 8, vf=to_dev(vf), vf_rest=to_dev(rest, "float32"), vf_k=1.0)
+    with pytest.raises(mad.MadError) as ei:
+        ctx.mad_eval(x, t, g, H)
+    assert ei.value.status == mad.MAD_ERR_UNIMPLEMENTED
+    with pytest.raises(mad.MadError) as ei:
+        ctx.mad_jacobian_shape(VF)
+    assert ei.value.status == mad.MAD_ERR_UNIMPLEMENTED
+    # blocks missing from the pattern (the pairs were not inserted): status error
+    t = mad.Terms(mask=VF, vf=to_dev(vf), vf_rest=to_dev(rest, "float32"), vf_k=1.0)
+    ctx.mad_eval(x, t, g, H)
+    assert ctx.mad_status_sync() == mad.MAD_ERR_INDEX
