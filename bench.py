@@ -310,6 +310,18 @@ def cpu_baseline_rows(st):
     t2 = time.perf_counter()
     res["area1000_eval_ms"] = round((t1 - t0) * 1e3, 1)
     res["area1000_hvp_ms"] = round((t2 - t1) * 1e3, 1)
+    # springs + inertia + 10^5 vertex-face terms at 1000^2: pattern with their pairs, assembly
+    vf = mi.random_vf(N_GRID, N_VF, 1009, 0)
+    xx = mi.cloth_x(N_GRID, 1011, 0, np.float32)
+    rest = (0.001 * np.random.default_rng(1010).standard_normal(N_VF)).astype(np.float32)
+    t0 = time.perf_counter()
+    rp, ci = orc.pattern(st["V"], st["F"], mi.vf_pairs(vf, st["F"]))
+    t1 = time.perf_counter()
+    orc.eval(st["V"], 3, xx, 1 | 2 | 64, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
+             xt=st["xt"], w=st["w"], F=st["F"], vf=vf, vf_rest=rest, kc=KC)
+    t2 = time.perf_counter()
+    res["vf1000_insert_ms"] = round((t1 - t0) * 1e3, 1)
+    res["vf1000_eval_ms"] = round((t2 - t1) * 1e3, 1)
     res["unit"] = "ms per call, 1 core, one run"
     return res
 
@@ -330,7 +342,7 @@ def cpu_baseline(st):
             "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
 
 
-EXTRA = ("cloth_small", "symdir500", "pairs1000", "jac1000", "area1000")
+EXTRA = ("cloth_small", "symdir500", "pairs1000", "jac1000", "area1000", "vf1000")
 
 
 def extra_workloads(args, only=None):
@@ -395,7 +407,41 @@ def extra_workloads(args, only=None):
         jac1000(res, mad, torch, dev, stream, timeit)
     if run("area1000"):
         area1000(res, mad, torch, dev, stream, timeit)
+    if run("vf1000"):
+        vf1000(res, mad, torch, dev, stream, timeit)
     return res
+
+
+N_VF = 100_000
+KC = 50.0
+
+
+def vf1000(res, mad, torch, dev, stream, timeit):
+    """Springs + inertia + 10^5 vertex-face terms on the 1000^2 cloth: the
+    insertion of their 3 x 10^5 (vertex, corner) pairs, then eval and the
+    product; the row kernel runs first, the vertex-face pass after it."""
+    st = mi.cloth_static(N_GRID, np.float32)
+    vf = mi.random_vf(N_GRID, N_VF, 1009, 0)
+    pairs = mi.vf_pairs(vf, st["F"])
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"], max_pairs=len(pairs),
+                      slack=0.2)
+    dp = torch.from_numpy(pairs).to(dev)
+    dr = torch.zeros(len(pairs), dtype=torch.float32, device=dev)
+    res["vf1000_insert_ms"] = round(timeit(lambda: ctx.mad_add_pairs(dp, dr, stream), n=16), 5)
+    rest = (0.001 * np.random.default_rng(1010).standard_normal(N_VF)).astype(np.float32)
+    terms = mad.Terms(mask=1 | 2 | 64, spring_rest=torch.from_numpy(st["L0"]).to(dev),
+                      spring_k=st["k"], inertia_xt=torch.from_numpy(st["xt"]).to(dev),
+                      inertia_w=st["w"], vf=torch.from_numpy(vf).to(dev),
+                      vf_rest=torch.from_numpy(rest).to(dev), vf_k=KC)
+    x = torch.from_numpy(mi.cloth_x(N_GRID, 1011, 0, np.float32)).to(dev)
+    v = torch.from_numpy(mi.probe_vector(st["V"], 3, 1012, np.float32)).to(dev)
+    g = torch.empty((st["V"], 3), device=dev)
+    y = torch.empty((st["V"], 3), device=dev)
+    H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
+    res["vf1000_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+    res["vf1000_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
+    res["vf1000_status"] = ctx.mad_status_sync()
+    ctx.close()
 
 
 def cloth_rest_area(st):

@@ -145,6 +145,36 @@ def pair_rest(x, pairs, dtype=np.float32):
     return (0.9 * d).astype(dtype)
 
 
+def random_vf(n: int, nvf: int, seed: int, step: int):
+    """nvf vertex-face terms (vertex, face) of the n x n grid, int32 [nvf][2]:
+    a uniform face, and a vertex within two grid steps of the face's first
+    corner that is not one of its corners (a contact-like neighbourhood)."""
+    _, F = grid_mesh(n, 3)
+    rng = _rng(seed, step, 5)
+    out = []
+    while len(out) < nvf:
+        m = 2 * (nvf - len(out)) + 64
+        f = rng.integers(0, F.shape[0], size=m)
+        a = F[f, 0]
+        di = rng.integers(-2, 3, size=m)
+        dj = rng.integers(-2, 3, size=m)
+        i, j = a % n + di, a // n + dj
+        ok = (i >= 0) & (i < n) & (j >= 0) & (j < n)
+        p = j * n + i
+        ok &= (p != F[f, 0]) & (p != F[f, 1]) & (p != F[f, 2])
+        for pp, ff in zip(p[ok], f[ok]):
+            out.append((pp, ff))
+            if len(out) == nvf:
+                break
+    return np.array(out, np.int32)
+
+
+def vf_pairs(vf, F):
+    """The (vertex, corner) pairs whose blocks vertex-face terms need."""
+    F = np.asarray(F)
+    return np.stack([np.repeat(vf[:, 0], 3), F[vf[:, 1]].reshape(-1)], axis=1).astype(np.int32)
+
+
 def param_static(n: int, seed: int, dtype=np.float32):
     """The n x n parameterization problem: 2D rest grid, faces, per-face
     Dm^-1 [F][2][2] and area [F], and non-inverted noisy UV [V][2]."""

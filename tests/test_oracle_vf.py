@@ -145,3 +145,19 @@ def test_vf_assembled_on_cloth_fd(orc):
         gm, _, Em = ev(xm.reshape(-1, 3))
         assert g.reshape(-1)[c] == pytest.approx((Ep - Em) / (2 * h), abs=1e-6)
         np.testing.assert_allclose(D[:, c], (gp - gm).reshape(-1) / (2 * h), atol=1e-5)
+
+
+def test_random_vf_inputs():
+    import mesh_inputs as mi
+    n = 12
+    _, F = mi.grid_mesh(n, 3)
+    vf = mi.random_vf(n, 500, 3, 0)
+    assert vf.shape == (500, 2) and vf.dtype == np.int32
+    p, f = vf[:, 0], vf[:, 1]
+    assert not (p[:, None] == F[f]).any()
+    a = F[f, 0]
+    assert (np.abs(p % n - a % n) <= 2).all() and (np.abs(p // n - a // n) <= 2).all()
+    pairs = mi.vf_pairs(vf, F)
+    np.testing.assert_array_equal(pairs[:, 0], np.repeat(p, 3))
+    np.testing.assert_array_equal(pairs[:, 1], F[f].reshape(-1))
+    np.testing.assert_array_equal(mi.random_vf(n, 500, 3, 0), vf)
