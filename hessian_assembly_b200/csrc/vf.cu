@@ -83,6 +83,33 @@ __device__ __forceinline__ int find_col(const int32_t* __restrict__ rp,
   return (lo < rp[row + 1] && ci[lo] == col) ? lo : -1;
 }
 
+// dst[0..n-1] += v[0..n-1] for n = 3 (a vertex's gradient) or 9 (a block).
+// fp32: pairs of adds as one 8-byte vector reduction
+// (red.global.add.v2.f32), starting at element 0 when dst is 8-byte aligned
+// and at element 1 otherwise, so that every pair is 8-byte aligned; the one
+// element left over takes a scalar add.  fp64: scalar adds.
+__device__ __forceinline__ void red_add2(float* a, float x, float y) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(a), "f"(x), "f"(y) : "memory");
+}
+template <int NV, typename T>
+__device__ __forceinline__ void add_vec(T* dst, const T (&v)[NV]) {
+  static_assert(NV % 2 == 1, "odd length: one scalar add");
+  if constexpr (sizeof(T) == 4) {
+    if ((reinterpret_cast<uintptr_t>(dst) & 7u) == 0) {
+#pragma unroll
+      for (int q = 0; q + 1 < NV; q += 2) red_add2(dst + q, v[q], v[q + 1]);
+      atomicAdd(dst + NV - 1, v[NV - 1]);
+    } else {
+      atomicAdd(dst, v[0]);
+#pragma unroll
+      for (int q = 1; q + 1 < NV + 1; q += 2) red_add2(dst + q, v[q], v[q + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < NV; ++q) atomicAdd(dst + q, v[q]);
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ bool load_term(int t, const int32_t* __restrict__ vf,
                                           const int32_t* __restrict__ F, int nF, int V,
@@ -117,15 +144,18 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_eval(
       const auto z = vf_energy<T>(X[0], X[1], X[2], X[3], rest[t], k);
       e = (double)z.v;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) {
+        T gi[3];
 #pragma unroll
         for (int al = 0; al < 3; ++al) {
           T s = T(-0.0);
 #pragma unroll
           for (int sv = 0; sv < 3; ++sv)
             if (vf_coef(i, sv) != 0) s += T(vf_coef(i, sv)) * sgrad(z, 3 * sv + al);
-          atomicAdd(&g[(int64_t)vid[i] * 3 + al], s);
+          gi[al] = s;
         }
+        add_vec<3>(g + (int64_t)vid[i] * 3, gi);
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -135,7 +165,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_eval(
             atomicOr(status, kStatusIndex);
             continue;
           }
-          T* blk = H + (int64_t)pos * 9;
+          T bv[9];
 #pragma unroll
           for (int al = 0; al < 3; ++al)
 #pragma unroll
@@ -147,8 +177,9 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_eval(
                 for (int tv = 0; tv < 3; ++tv)
                   if (vf_coef(i, sv) * vf_coef(j, tv) != 0)
                     s += T(vf_coef(i, sv) * vf_coef(j, tv)) * shess(z, 3 * sv + al, 3 * tv + be);
-              atomicAdd(&blk[3 * al + be], s);
+              bv[3 * al + be] = s;
             }
+          add_vec<9>(H + (int64_t)pos * 9, bv);
         }
     }
   }
@@ -194,15 +225,18 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_hvp(
     tz[q] = s;
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 4; ++i) {
+    T yi[3];
 #pragma unroll
     for (int al = 0; al < 3; ++al) {
       T s = T(-0.0);
 #pragma unroll
       for (int sv = 0; sv < 3; ++sv)
         if (vf_coef(i, sv) != 0) s += T(vf_coef(i, sv)) * tz[3 * sv + al];
-      atomicAdd(&y[(int64_t)vid[i] * 3 + al], s);
+      yi[al] = s;
     }
+    add_vec<3>(y + (int64_t)vid[i] * 3, yi);
+  }
 }
 
 }  // namespace
