@@ -27,8 +27,7 @@ def _sources():
 
 
 def _deps():
-    return _sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
-        [os.path.join(HERE, "..", "include", "mad.h")]
+    return _sources() + _headers()
 
 
 def up_to_date() -> bool:
@@ -38,8 +37,19 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def _compile(src: str, extra: list[str], bdir: str) -> str:
+def _headers():
+    return glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+        [os.path.join(HERE, "..", "include", "mad.h")]
+
+
+def _compile(src: str, extra: list[str], bdir: str, force: bool) -> str:
     obj = os.path.join(bdir, os.path.basename(src) + ".o")
+    # an object newer than its source and every header is reused (every unit
+    # is treated as depending on every header)
+    if not force and os.path.exists(obj):
+        t = os.path.getmtime(obj)
+        if all(os.path.getmtime(d) <= t for d in [src, *_headers()]):
+            return obj
     cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
@@ -58,9 +68,13 @@ def build(force: bool = False, extra: list[str] | None = None, jobs: int | None 
     bdir = build_dir or BUILD
     os.makedirs(bdir, exist_ok=True)
     extra = list(extra or [])
+    # variant builds (extra flags) compile everything into their own folder
+    fresh = force or bool(extra)
     srcs = _sources()
+    # the longest units first, so that they do not finish last
+    srcs.sort(key=lambda s: -os.path.getsize(s) - (1 << 20) * s.endswith("_d3.cu"))
     with cf.ThreadPoolExecutor(max_workers=jobs or min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra, bdir), srcs))
+        objs = list(ex.map(lambda s: _compile(s, extra, bdir, fresh), srcs))
     tmp = lib + ".tmp"
     cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)

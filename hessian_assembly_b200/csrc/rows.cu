@@ -1,977 +1,10 @@
-// rows.cu -- row-streaming assembly: one warp per 32 consecutive Hessian rows,
-// no block-wide barriers.
-//
-// Page "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
-// Computations", section 方法: per-term forward-mode AD in registers (key
-// design 1), assembly g = sum S^T g_j, H = sum S^T H_j S_j into the
-// preallocated CSR (key design 3), runtime pair blocks (key design 4).
-//
-// This kernel is the gather form of that assembly.  Thread = row i (vertex
-// i): it evaluates the inertia term of i, every edge term (i, b) of its row
-// and every face term with i as a corner with HyperDual numbers, keeps the
-// diagonal block and the gradient in registers, and writes each off-diagonal
-// block once.  Each edge term is evaluated once per endpoint and each face
-// term once per corner, for that corner's row only.  Rows 32w .. 32w+31 are consecutive in H, so warp w stages
-// them contiguously in its own slice of shared memory, at the same offset
-// modulo 16 bytes as in H, and writes them back with one 1-D bulk (TMA) copy.
-// Neighbour positions are read through the L1/L2 caches.  Warps never wait
-// for each other, so memory latency is hidden across the resident warps.
-// A thread writes only its own row: no zeroing pass, no atomics.
+// rows.cu -- host-side dispatch of the row-streaming assembly kernels
+// (rows_impl.cuh) by dtype and dof.
 #include <algorithm>
-#include <type_traits>
 
-#include "mad_internal.h"
-#include "terms.cuh"
+#include "rows_common.h"
 
 namespace mad {
-namespace {
-
-constexpr int kRowThreads = 128;  // 4 warps per block
-constexpr int kWarps = kRowThreads / 32;
-constexpr int kS0Max = 8;         // most slots per row in the slot table
-#ifndef MAD_ROWS_MIN_BLOCKS
-#define MAD_ROWS_MIN_BLOCKS 6  // resident blocks per SM (fp32) the register budget targets
-#endif
-template <typename T, bool FACES>
-constexpr int rows_min_blocks() {
-  return FACES ? (sizeof(T) == 4 ? 4 : 2) : (sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3);
-}
-
-template <typename T>
-struct RArgs {
-  const int32_t* fcslots;
-  const int32_t* fcofl;
-  const T* fhv;
-  const int4* fslots;
-  const int32_t* fofl_ptr;
-  const int4* fofl;
-  const T* Minv;
-  const T* area;
-  const int2* slots;
-  const uint32_t* meta;
-  const int32_t* ofl_ptr;
-  const int2* ofl;
-  const int32_t* rp;
-  const int32_t* prow;
-  const int32_t* pe_col;
-  const int32_t* pe_pos;
-  const T* pe_rest;
-  const T* x;
-  const T* v;
-  T* g;
-  T* H;
-  T* y;
-  const T* L0;
-  T k;
-  const T* xt;
-  T w;
-  T kp;
-  T ka;  // area-preservation stiffness
-  unsigned mask;
-  double* epart;
-  int V, s0, sf, wstage;  // wstage: staging elements per warp
-};
-
-// New-block positions of a row with inserted pair blocks, in increasing
-// order: the first kRowNew in registers, the rest read from pe_pos.
-constexpr int kRowNew = 4;
-struct RowNew {
-  int np[kRowNew];  // merged-row positions, 0x7FFFFFFF past the row's count
-};
-
-__device__ __forceinline__ void load_row_new(const int32_t* __restrict__ pe_pos, int pb, int pn,
-                                             int nins, RowNew& rn) {
-#pragma unroll
-  for (int k = 0; k < kRowNew; ++k) rn.np[k] = 0x7FFFFFFF;
-  if (nins == 0) return;
-  int k = 0;
-  for (int e = pb; e < pb + pn && k < kRowNew; ++e) {
-    const int32_t wv = pe_pos[e];
-    if (wv & kPairNewBlock) {
-#pragma unroll
-      for (int q = 0; q < kRowNew; ++q)
-        if (q == k) rn.np[q] = wv & kPairPosMask;
-      ++k;
-    }
-  }
-}
-
-__device__ __forceinline__ int row_pos(const int32_t* __restrict__ pe_pos, int pb, int pn,
-                                       int nins, int p);
-
-// Merged-row position of mesh-pattern position p.
-__device__ __forceinline__ int row_pos_new(const RowNew& rn, const int32_t* __restrict__ pe_pos,
-                                           int pb, int pn, int nins, int p) {
-  if (nins > kRowNew) return row_pos(pe_pos, pb, pn, nins, p);
-#pragma unroll
-  for (int k = 0; k < kRowNew; ++k) p += rn.np[k] <= p;
-  return p;
-}
-
-__device__ __forceinline__ int row_pos(const int32_t* __restrict__ pe_pos, int pb, int pn,
-                                       int nins, int p) {
-  if (nins == 0) return p;
-  for (int e = pb; e < pb + pn; ++e) {
-    const int32_t wv = pe_pos[e];
-    if ((wv & kPairNewBlock) && (wv & kPairPosMask) <= p) ++p;
-  }
-  return p;
-}
-
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
-  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(ssrc);
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-               "r"(sa), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_and_wait_read() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-__device__ __forceinline__ double warp_sum(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// Per-block energy partial (all threads of the block call it).
-__device__ __forceinline__ void block_energy(double e, double* out) {
-  __shared__ double red[kWarps];
-  e = warp_sum(e);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = e;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double s = 0.0;
-    for (int i = 0; i < kWarps; ++i) s += red[i];
-    *out = s;
-  }
-}
-
-// Calls on_term(R, p, col) for every edge term (i, col) of row i, where p is
-// the block position of column col in the mesh-pattern row.
-// S0 (compile time) >= the slot table's row width A.s0.
-template <typename T, int DOF, bool FULL, int S0, typename OnTerm>
-__device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, int lane,
-                                          uint32_t m, const T* xi, OnTerm on_term) {
-  const int noff = (int)(m & 0xFFFFu), dpos = (int)(m >> 16);
-  int2 sl[S0];
-#pragma unroll
-  for (int k = 0; k < S0; ++k) {
-    sl[k] = make_int2(-1, -1);
-    if (k < A.s0) sl[k] = A.slots[(uint32_t)((tile * A.s0 + k) * 32 + lane)];
-  }
-  T xb[S0][DOF];
-  T l0[S0];
-#pragma unroll
-  for (int k = 0; k < S0; ++k) {
-    if (sl[k].x < 0) continue;
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) xb[k][a] = A.x[(uint32_t)(sl[k].x * DOF + a)];
-    l0[k] = A.L0[sl[k].y];
-  }
-#pragma unroll
-  for (int k = 0; k < S0; ++k) {
-    if (sl[k].x < 0) continue;
-    EdgeRes<T, DOF, FULL> R;
-    eval_edge_res<T, DOF, FULL>(xi, xb[k], l0[k], A.k, R);
-    on_term(R, k < dpos ? k : k + 1, sl[k].x);
-  }
-  if (noff > A.s0) {  // rows longer than the slot table: the overflow slots
-    const int o0 = A.ofl_ptr[i];
-    for (int k = A.s0; k < noff; ++k) {
-      const int2 e = A.ofl[o0 + k - A.s0];
-      T xo[DOF];
-#pragma unroll
-      for (int a = 0; a < DOF; ++a) xo[a] = A.x[(uint32_t)(e.x * DOF + a)];
-      EdgeRes<T, DOF, FULL> R;
-      eval_edge_res<T, DOF, FULL>(xi, xo, A.L0[e.y], A.k, R);
-      on_term(R, k < dpos ? k : k + 1, e.x);
-    }
-  }
-}
-
-// Four consecutive values starting at p (16-byte loads when p allows them).
-template <typename T>
-__device__ __forceinline__ void load4(const T* __restrict__ p, T* o) {
-  if ((((uintptr_t)p) & 15u) == 0) {
-    if constexpr (sizeof(T) == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(p);
-      o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-    } else {
-      const double2 a = reinterpret_cast<const double2*>(p)[0];
-      const double2 b = reinterpret_cast<const double2*>(p)[1];
-      o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) o[q] = p[q];
-  }
-}
-
-// Calls on_face(xj, xk, j, k, c, pj, pk, M, area) for every face term with
-// vertex i as a corner (dof 2): j and k are the other two corners (corner
-// c+1 and c+2 of the face when i is corner c), pj and pk their mesh-pattern
-// block positions in row i, M the face's Dm^-1 and area its rest area.  The
-// loop is not unrolled (a small body stays in the instruction cache); the
-// next table entry is loaded while the current face is evaluated.
-template <typename T, typename OnFace>
-__device__ __forceinline__ void row_faces(const RArgs<T>& A, int i, int tile, int lane,
-                                          OnFace on_face) {
-  constexpr uint32_t kPm = (1u << kFacePosBits) - 1u;
-  auto one = [&](const int4& e) {
-    const int j = e.y, k = e.z & 0x7FFFFFFF;
-    const uint32_t w = (uint32_t)e.w;
-    T xj[2], xk[2], M[4];
-    xj[0] = A.x[(uint32_t)(j * 2)];
-    xj[1] = A.x[(uint32_t)(j * 2 + 1)];
-    xk[0] = A.x[(uint32_t)(k * 2)];
-    xk[1] = A.x[(uint32_t)(k * 2 + 1)];
-    load4<T>(A.Minv + (uint32_t)e.x * 4u, M);
-    const T ar = A.area[e.x];
-    on_face(xj, xk, j, k, (int)(w & 3u), (int)((w >> 2) & kPm), (int)(w >> (2 + kFacePosBits)),
-            M, ar);
-  };
-  const int4* p = A.fslots + (uint32_t)(tile * A.sf * 32 + lane);
-  int4 e = p[0];
-  bool more = false;
-#pragma unroll 1
-  for (int k = 0; k < A.sf; ++k) {  // a row's entries fill a prefix of its slots
-    if (e.x < 0) break;
-    const int4 en = k + 1 < A.sf ? p[(uint32_t)((k + 1) * 32)] : make_int4(-1, 0, 0, 0);
-    if (k == kFaceRowSlots - 1) more = e.z < 0;  // the overflow mark
-    one(e);
-    e = en;
-  }
-  if (more) {
-    const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
-#pragma unroll 1
-    for (int q = o0; q < o1; ++q) one(A.fofl[q]);
-  }
-}
-
-// The dof-3 face terms of row i: calls on_face(xj, xk, c, pj, pk, A0) for
-// every face with vertex i as a corner (same table as row_faces).
-template <typename T, typename OnFace>
-__device__ __forceinline__ void row_faces3(const RArgs<T>& A, int i, int tile, int lane,
-                                           OnFace on_face) {
-  constexpr uint32_t kPm = (1u << kFacePosBits) - 1u;
-  auto one = [&](const int4& e) {
-    const int j = e.y, k = e.z & 0x7FFFFFFF;
-    const uint32_t w = (uint32_t)e.w;
-    T xj[3], xk[3];
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      xj[a] = A.x[(uint32_t)(j * 3 + a)];
-      xk[a] = A.x[(uint32_t)(k * 3 + a)];
-    }
-    on_face(xj, xk, (int)(w & 3u), (int)((w >> 2) & kPm), (int)(w >> (2 + kFacePosBits)),
-            A.area[e.x]);
-  };
-  const int4* p = A.fslots + (uint32_t)(tile * A.sf * 32 + lane);
-  int4 e = p[0];
-  bool more = false;
-#pragma unroll 1
-  for (int k = 0; k < A.sf; ++k) {  // a row's entries fill a prefix of its slots
-    if (e.x < 0) break;
-    const int4 en = k + 1 < A.sf ? p[(uint32_t)((k + 1) * 32)] : make_int4(-1, 0, 0, 0);
-    if (k == kFaceRowSlots - 1) more = e.z < 0;  // the overflow mark
-    one(e);
-    e = en;
-  }
-  if (more) {
-    const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
-#pragma unroll 1
-    for (int q = o0; q < o1; ++q) one(A.fofl[q]);
-  }
-}
-
-// b[0..8] += v[0..8]
-template <typename T>
-__device__ __forceinline__ void add9(T* b, const T* v) {
-#pragma unroll
-  for (int q = 0; q < 9; ++q) b[q] += v[q];
-}
-
-// b[0..3] += v[0..3] (16-byte accesses when b allows them)
-template <typename T>
-__device__ __forceinline__ void add4(T* b, const T* v) {
-  if constexpr (sizeof(T) == 4) {
-    if ((((uintptr_t)b) & 15u) == 0) {
-      float4 t = *reinterpret_cast<float4*>(b);
-      t.x += v[0]; t.y += v[1]; t.z += v[2]; t.w += v[3];
-      *reinterpret_cast<float4*>(b) = t;
-      return;
-    }
-  } else {
-    if ((((uintptr_t)b) & 15u) == 0) {
-      double2 t0 = reinterpret_cast<double2*>(b)[0], t1 = reinterpret_cast<double2*>(b)[1];
-      t0.x += v[0]; t0.y += v[1]; t1.x += v[2]; t1.y += v[3];
-      reinterpret_cast<double2*>(b)[0] = t0;
-      reinterpret_cast<double2*>(b)[1] = t1;
-      return;
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) b[q] += v[q];
-}
-
-// The work of one row, writing the row's blocks through `row` (a shared-memory
-// staging slot or, for rows that do not fit, the row's place in H).
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES, bool PAIRS>
-__device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile, int lane,
-                                              uint32_t m, int d0, int d1, int pb, int pn,
-                                              const T* xi, const T* xti, T* row, double& energy) {
-  constexpr int B = DOF * DOF;
-  constexpr int TD = Tri<DOF>::size;
-  const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
-  const bool springs = A.mask & MAD_TERM_SPRING;
-  const int nins = (d1 - d0) - ((int)(m & 0xFFFFu) + 1);
-  T acc[TD], gr[DOF];
-  RowNew rn;
-  if constexpr (PAIRS) load_row_new(A.pe_pos, pb, pn, nins, rn);
-  // The row's first pair entry is loaded before the edge terms are evaluated,
-  // so that its partner's position (a random vertex) arrives meanwhile.
-  int pc0 = 0, pw0 = 0;
-  T pr0 = T(0), xp0[DOF];
-  if (pairs && pn > 0) {
-    pc0 = A.pe_col[pb];
-    pw0 = A.pe_pos[pb];
-    pr0 = A.pe_rest[pb];
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) xp0[a] = A.x[(uint32_t)(pc0 * DOF + a)];
-  }
-  // Blocks that no edge term stores start at 0: the whole row without edge
-  // terms, else only the blocks that pairs inserted.
-  if (!springs || S0 == 0) {
-    for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
-  } else if (PAIRS && nins > 0) {
-#pragma unroll
-    for (int k = 0; k < kRowNew; ++k)
-      if (k < nins) {
-        T* b = row + rn.np[k] * B;
-#pragma unroll
-        for (int q = 0; q < B; ++q) b[q] = T(0);
-      }
-    if (nins > kRowNew) {
-      for (int e = pb; e < pb + pn; ++e) {
-        const int32_t wv = A.pe_pos[e];
-        if (wv & kPairNewBlock) {
-          T* b = row + (wv & kPairPosMask) * B;
-#pragma unroll
-          for (int q = 0; q < B; ++q) b[q] = T(0);
-        }
-      }
-    }
-  }
-  if (A.mask & MAD_TERM_INERTIA) {
-    T Ei, Hi[B];
-    eval_inertia<T, DOF>(xi, xti, A.w, Ei, gr, Hi);
-    if (ENERGY) energy += (double)Ei;
-#pragma unroll
-    for (int a = 0; a < DOF; ++a)
-#pragma unroll
-      for (int b = a; b < DOF; ++b) acc[Tri<DOF>::idx(a, b)] = Hi[a * DOF + b];
-  } else {
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) gr[a] = T(0);
-#pragma unroll
-    for (int q = 0; q < TD; ++q) acc[q] = T(0);
-  }
-  if constexpr (S0 > 0) {  // S0 == 0: an instantiation without edge terms
-    if (springs) {
-      row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
-                              [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
-                                const int op =
-                                    !PAIRS || nins == 0 ? p : row_pos_new(rn, A.pe_pos, pb, pn, nins, p);
-                                apply_edge_side<true>(R, 0, acc, row + op * B, gr);
-                                if (ENERGY) energy += 0.5 * (double)edge_energy(R);
-                              });
-    }
-  }
-  if constexpr (FACES && DOF == 3) {
-    // area preservation after the edge terms, which store their blocks
-    if (A.mask & MAD_TERM_AREA) {
-      row_faces3<T>(A, i, tile, lane,
-                    [&](const T* xj, const T* xk, int, int pj, int pk, T A0) {
-                      FaceRow3<T> o;
-                      eval_area_row<T, FULL>(xi, xj, xk, A0, A.ka, o);
-#pragma unroll
-                      for (int a = 0; a < 3; ++a)
-#pragma unroll
-                        for (int b = a; b < 3; ++b) acc[Tri<3>::idx(a, b)] += o.H[0][3 * a + b];
-#pragma unroll
-                      for (int a = 0; a < 3; ++a) gr[a] += o.g[a];
-                      const int oj = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pj) : pj;
-                      const int ok = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pk) : pk;
-                      add9<T>(row + oj * B, o.H[1]);
-                      add9<T>(row + ok * B, o.H[2]);
-                      if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
-                    });
-    }
-  }
-  if constexpr (FACES && DOF == 2) {
-    // after the edge terms, which store their blocks: faces add to them
-    if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
-      auto faces = [&](auto kc) {
-        constexpr int KIND = decltype(kc)::value;
-        row_faces<T>(A, i, tile, lane,
-                     [&](const T* xj, const T* xk, int, int, int c, int pj, int pk, const T* M,
-                         T ar) {
-                       FaceRow<T> o;
-                       eval_symdir_row<T, FULL, KIND>(xi, xj, xk, c, M, ar, o);
-                       acc[0] += o.H[0][0];
-                       acc[1] += o.H[0][1];
-                       acc[2] += o.H[0][3];
-                       gr[0] += o.g[0];
-                       gr[1] += o.g[1];
-                       const int oj = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pj) : pj;
-                       const int ok = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pk) : pk;
-                       add4<T>(row + oj * B, o.H[1]);
-                       add4<T>(row + ok * B, o.H[2]);
-                       if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
-                     });
-      };
-      if constexpr (FACES == 1) {
-        faces(std::integral_constant<int, kFaceSymDir>{});
-      } else {
-        if (!(A.mask & MAD_TERM_SYMDIR)) faces(std::integral_constant<int, kFaceArap>{});
-        else faces(std::integral_constant<int, kFaceSymDir | kFaceArap>{});
-      }
-    }
-  }
-  if (pairs) {
-    for (int e = pb; e < pb + pn; ++e) {
-      int pw;
-      T xj[DOF], rest;
-      if (e == pb) {
-        pw = pw0;
-        rest = pr0;
-#pragma unroll
-        for (int a = 0; a < DOF; ++a) xj[a] = xp0[a];
-      } else {
-        const int j = A.pe_col[e];
-        pw = A.pe_pos[e];
-        rest = A.pe_rest[e];
-#pragma unroll
-        for (int a = 0; a < DOF; ++a) xj[a] = A.x[(uint32_t)(j * DOF + a)];
-      }
-      EdgeRes<T, DOF, FULL> Rp;
-      eval_edge_res<T, DOF, FULL>(xi, xj, rest, A.kp, Rp);
-      apply_edge_side<false>(Rp, 0, acc, row + (pw & kPairPosMask) * B, gr);
-      if (ENERGY) energy += 0.5 * (double)edge_energy(Rp);
-    }
-  }
-  const int dp = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, (int)(m >> 16)) : (int)(m >> 16);
-  T* d = row + dp * B;
-#pragma unroll
-  for (int a = 0; a < DOF; ++a)
-#pragma unroll
-    for (int b = 0; b < DOF; ++b)
-      d[a * DOF + b] = a <= b ? acc[Tri<DOF>::idx(a, b)] : acc[Tri<DOF>::idx(b, a)];
-#pragma unroll
-  for (int a = 0; a < DOF; ++a) A.g[(uint32_t)(i * DOF + a)] = gr[a];
-}
-
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES, bool PAIRS>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, (FACES != 0)>()) k_rows_eval(const RArgs<T> A) {
-  constexpr int B = DOF * DOF;
-  constexpr int VEC = 16 / (int)sizeof(T);
-  extern __shared__ __align__(16) char smem_raw[];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int tile = blockIdx.x * kWarps + wib;
-  const int i = tile * 32 + lane;
-  const bool tile_live = tile * 32 < A.V;
-  const bool has = i < A.V;
-  T* stage = (T*)smem_raw + wib * A.wstage;
-  double energy = 0.0;
-
-  int d0 = 0, d1 = 0, pb = 0, pn = 0;
-  uint32_t m = 0;
-  T xi[DOF], xti[DOF];
-  if (has) {
-    d0 = A.rp[i];
-    d1 = A.rp[i + 1];
-    m = A.meta[i];
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) xi[a] = A.x[(uint32_t)(i * DOF + a)];
-    if (A.mask & MAD_TERM_INERTIA) {
-#pragma unroll
-      for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(uint32_t)(i * DOF + a)];
-    }
-    if constexpr (PAIRS) {
-      pb = A.prow[i];
-      pn = A.prow[i + 1] - pb;
-    }
-  }
-  // the warp's rows are consecutive in H: stage them from the first one
-  const int dfirst = __shfl_sync(0xffffffffu, d0, 0);
-  const int mis = (int)(((uintptr_t)(A.H + (uint32_t)(dfirst * B)) / sizeof(T)) % VEC);
-  const int off = mis + (d0 - dfirst) * B;
-  const bool staged = has && off + (d1 - d0) * B <= A.wstage;
-  // rows that do not fit their warp's slice are assembled in place in H
-  if (has)
-    rows_eval_row<T, DOF, FULL, ENERGY, S0, FACES, PAIRS>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
-                                        staged ? stage + off : A.H + (uint32_t)(d0 * B), energy);
-  // ---- write-back of the warp's staged rows (a prefix of its 32 rows) -------
-  fence_async_smem();
-  __syncwarp();
-  if (tile_live) {
-    const unsigned st = __ballot_sync(0xffffffffu, staged);
-    if (st) {
-      const int last = 31 - __clz(st);  // staged rows form a prefix
-      const int dend = __shfl_sync(0xffffffffu, d1, last);
-      const int n = (dend - dfirst) * B;
-      T* dst = A.H + (uint32_t)(dfirst * B);
-      const T* src = stage + mis;
-      const int head = min(n, (VEC - mis) % VEC);
-      const int body = ((n - head) / VEC) * VEC;
-      for (int e = lane; e < head; e += 32) dst[e] = src[e];
-      for (int e = head + body + lane; e < n; e += 32) dst[e] = src[e];
-      const bool aligned = ((((uintptr_t)(dst + head)) | ((uintptr_t)(src + head))) & 15u) == 0;
-      if (body > 0 && !aligned)
-        for (int e = head + lane; e < head + body; e += 32) dst[e] = src[e];
-      if (lane == 0 && body > 0 && aligned) {
-        bulk_store(dst + head, src + head, (uint32_t)(body * sizeof(T)));
-        bulk_commit_and_wait_read();
-      }
-    }
-  }
-  if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
-}
-
-template <typename T, int DOF, bool FULL, int S0, bool FACES>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_hvp(const RArgs<T> A) {
-  constexpr int TD = Tri<DOF>::size;
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int tile = blockIdx.x * kWarps + wib;
-  const int i = tile * 32 + lane;
-  if (i >= A.V) return;
-  const bool pairs = (A.mask & MAD_TERM_PAIR) && A.prow != nullptr;
-  // the row's own position, direction and slot meta are needed only by the
-  // vertex, edge and pair terms (face terms come from the per-face pass)
-  const bool own = A.mask & (MAD_TERM_INERTIA | MAD_TERM_SPRING | MAD_TERM_PAIR);
-  T xi[DOF], vi[DOF], yr[DOF];
-  uint32_t m = 0;
-#pragma unroll
-  for (int a = 0; a < DOF; ++a) {
-    xi[a] = T(0);
-    vi[a] = T(0);
-    yr[a] = T(0);
-  }
-  if (own) {
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) {
-      xi[a] = A.x[(uint32_t)(i * DOF + a)];
-      vi[a] = A.v[(uint32_t)(i * DOF + a)];
-    }
-    m = A.meta[i];
-  }
-  if (A.mask & MAD_TERM_INERTIA) {
-    T xti[DOF], Ei, gi[DOF], Hi[DOF * DOF];
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(uint32_t)(i * DOF + a)];
-    eval_inertia<T, DOF>(xi, xti, A.w, Ei, gi, Hi);
-#pragma unroll
-    for (int a = 0; a < DOF; ++a)
-#pragma unroll
-      for (int b = 0; b < DOF; ++b) yr[a] += Hi[a * DOF + b] * vi[b];
-  }
-  auto hv = [&](const EdgeRes<T, DOF, FULL>& R, const T* vj) {
-    if constexpr (!FULL) {
-#pragma unroll
-      for (int a = 0; a < DOF; ++a) {
-        T s = T(0);
-#pragma unroll
-        for (int b = 0; b < DOF; ++b)
-          s += (a <= b ? R.K[Tri<DOF>::idx(a, b)] : R.K[Tri<DOF>::idx(b, a)]) * (vi[b] - vj[b]);
-        yr[a] += s;
-      }
-    } else {
-#pragma unroll
-      for (int a = 0; a < DOF; ++a)
-#pragma unroll
-        for (int b = 0; b < DOF; ++b)
-          yr[a] += R.d.Haa[a * DOF + b] * vi[b] + R.d.Hab[a * DOF + b] * vj[b];
-    }
-  };
-  if constexpr (S0 > 0) {
-    if (A.mask & MAD_TERM_SPRING) {
-      row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
-                              [&](const EdgeRes<T, DOF, FULL>& R, int, int col) {
-                                T vj[DOF];
-#pragma unroll
-                                for (int a = 0; a < DOF; ++a) vj[a] = A.v[(uint32_t)(col * DOF + a)];
-                                hv(R, vj);
-                              });
-    }
-  }
-  if constexpr (FACES) {
-    if (A.mask & (DOF == 2 ? (MAD_TERM_SYMDIR | MAD_TERM_ARAP) : MAD_TERM_AREA)) {
-      // the row's corners' results of the per-face pass (k_face_hv)
-      constexpr int SF = kFaceRowSlots;
-      int32_t e[SF];
-#pragma unroll
-      for (int k = 0; k < SF; ++k)
-        e[k] = k < A.sf ? A.fcslots[(uint32_t)((tile * A.sf + k) * 32 + lane)] : -1;
-#pragma unroll
-      for (int k = 0; k < SF; ++k) {
-        if (e[k] == -1) continue;
-        const uint32_t q = (uint32_t)e[k] & 0x7FFFFFFFu;
-#pragma unroll
-        for (int a = 0; a < DOF; ++a) yr[a] += A.fhv[DOF * q + a];
-      }
-      if (e[SF - 1] != -1 && e[SF - 1] < 0) {  // the row continues in the overflow table
-        const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
-        for (int q = o0; q < o1; ++q) {
-          const uint32_t fc = (uint32_t)A.fcofl[q];
-#pragma unroll
-          for (int a = 0; a < DOF; ++a) yr[a] += A.fhv[DOF * fc + a];
-        }
-      }
-    }
-  }
-  if (pairs) {
-    const int pb = A.prow[i], pe = A.prow[i + 1];
-    for (int e = pb; e < pe; ++e) {
-      const int j = A.pe_col[e];
-      T xj[DOF], vj[DOF];
-#pragma unroll
-      for (int a = 0; a < DOF; ++a) {
-        xj[a] = A.x[(uint32_t)(j * DOF + a)];
-        vj[a] = A.v[(uint32_t)(j * DOF + a)];
-      }
-      EdgeRes<T, DOF, FULL> Rp;
-      eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
-      hv(Rp, vj);
-    }
-  }
-  (void)TD;
-#pragma unroll
-  for (int a = 0; a < DOF; ++a) A.y[(uint32_t)(i * DOF + a)] = yr[a];
-}
-
-// Per-face pass of the Hessian-vector product for area-preservation faces
-// (dof 3): one thread per face writes (H_f v_f) for its three corners.
-template <typename T, bool FULL>
-__global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __restrict__ F,
-                                                      const T* __restrict__ x,
-                                                      const T* __restrict__ v,
-                                                      const T* __restrict__ area, T ka,
-                                                      T* __restrict__ out) {
-  const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (f >= nF) return;
-  T u[3][3], w[3][3];
-#pragma unroll
-  for (int c = 0; c < 3; ++c) {
-    const int32_t vid = F[3 * f + c];
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      u[c][a] = x[(int64_t)vid * 3 + a];
-      w[c][a] = v[(int64_t)vid * 3 + a];
-    }
-  }
-  T o[9];
-  hv_area_face<T, FULL>(u[0], u[1], u[2], w[0], w[1], w[2], area[f], ka, o);
-#pragma unroll
-  for (int q = 0; q < 9; ++q) out[9 * f + q] = o[q];
-}
-
-// Per-face pass of the Hessian-vector product: one thread per face computes
-// (H_f v_f) for its three corners once; the row kernel then adds, for each
-// row, its corners' results.  Each face is differentiated once instead of
-// once per corner, and no atomics are needed.
-template <typename T, bool FULL>
-__global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_t* __restrict__ F,
-                                                 const T* __restrict__ x, const T* __restrict__ v,
-                                                 const T* __restrict__ Minv,
-                                                 const T* __restrict__ area, T* __restrict__ out,
-                                                 int kind) {
-  const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (f >= nF) return;
-  const int32_t a = F[3 * f], b = F[3 * f + 1], c = F[3 * f + 2];
-  T u[3][2], w[3][2], M[4];
-  const int32_t vid[3] = {a, b, c};
-  // [V][2] arrays: a vertex's pair is one 2-element load when both arrays
-  // are aligned to it (the caller's pointers need not be)
-  using T2 = typename std::conditional<sizeof(T) == 4, float2, double2>::type;
-  if (vec2) {
-#pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      const T2 xu = reinterpret_cast<const T2*>(x)[vid[k]];
-      const T2 xv = reinterpret_cast<const T2*>(v)[vid[k]];
-      u[k][0] = xu.x;
-      u[k][1] = xu.y;
-      w[k][0] = xv.x;
-      w[k][1] = xv.y;
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 3; ++k)
-#pragma unroll
-      for (int al = 0; al < 2; ++al) {
-        u[k][al] = x[(int64_t)vid[k] * 2 + al];
-        w[k][al] = v[(int64_t)vid[k] * 2 + al];
-      }
-  }
-  load4<T>(Minv + 4 * f, M);
-  T o[6];
-  with_face2_kind(kind, [&](auto kc) {
-    hv_symdir_face<T, FULL, decltype(kc)::value>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f],
-                                                 o);
-  });
-#pragma unroll
-  for (int q = 0; q < 6; ++q) out[6 * f + q] = o[q];
-}
-
-// Staging elements per warp: 32 mesh rows of s0 + 1 blocks, plus, when the
-// active pattern has inserted pair blocks, kWarpSpare blocks for them
-// (shared by the warp's rows; rows past the reserve are assembled in place),
-// rounded to 16 bytes, plus 16 bytes of alignment room.
-constexpr int kWarpSpare = 16;
-size_t wstage_elems(const RowsLaunch& L) {
-  const int vec = L.dtype == MAD_F64 ? 2 : 4;
-  const int blocks = 32 * (L.s0 + 1) + (L.rho > 0 ? kWarpSpare : 0);
-  const int elems = blocks * L.dof * L.dof;
-  return (size_t)(((elems + vec - 1) / vec) * vec + vec);
-}
-
-template <typename T>
-RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
-                    void* g, void* H, void* y, bool energy) {
-  RArgs<T> A;
-  A.fcslots = L.fcslots;
-  A.fcofl = L.fcofl;
-  A.fhv = (const T*)L.fhv;
-  A.fslots = L.fslots;
-  A.fofl_ptr = L.fofl_ptr;
-  A.fofl = L.fofl;
-  A.Minv = (const T*)t.face_Minv;
-  A.area = (const T*)t.face_area;
-  A.sf = L.sf;
-  A.slots = L.slots;
-  A.meta = L.meta;
-  A.ofl_ptr = L.ofl_ptr;
-  A.ofl = L.ofl;
-  A.rp = L.rp;
-  A.prow = L.prow;
-  A.pe_col = L.pe_col;
-  A.pe_pos = L.pe_pos;
-  A.pe_rest = (const T*)L.pe_rest;
-  A.x = (const T*)x;
-  A.v = (const T*)v;
-  A.g = (T*)g;
-  A.H = (T*)H;
-  A.y = (T*)y;
-  A.L0 = (const T*)t.spring_rest;
-  A.k = (T)t.spring_k;
-  A.xt = (const T*)t.inertia_xt;
-  A.w = (T)t.inertia_w;
-  A.kp = (T)t.pair_k;
-  A.ka = (T)t.area_k;
-  A.mask = t.mask;
-  A.epart = energy ? L.epart : nullptr;
-  A.V = L.V;
-  A.s0 = L.s0;
-  A.wstage = (int)wstage_elems(L);
-  return A;
-}
-
-__global__ void k_energy_sum_rows(const double* __restrict__ part, int n, double* out) {
-  __shared__ double red[32];
-  double s = 0.0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) s += part[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double t = 0.0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
-    *out = t;
-  }
-}
-
-// One instantiation of the assembly kernel, chosen by whether the active
-// pattern holds pair blocks; also sets (or, with set, only sets) its shared
-// memory limit.
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES>
-cudaError_t eval_k(const RArgs<T>& A, bool pairs, int nb, size_t smem, cudaStream_t s,
-                   bool set = false) {
-  const void* kp = (const void*)k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, true>;
-  const void* kn = (const void*)k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, false>;
-  if (set) {
-    cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  }
-  if (pairs)
-    k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, true><<<nb, kRowThreads, smem, s>>>(A);
-  else
-    k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, false><<<nb, kRowThreads, smem, s>>>(A);
-  return cudaGetLastError();
-}
-
-// Every (FULL, ENERGY) instantiation for one S0 and FACES.  FACES: 0 no face
-// terms; 1 the face term of the dof (symmetric Dirichlet for dof 2, area
-// preservation for dof 3); 2 (dof 2) ARAP alone or with symmetric Dirichlet,
-// an instantiation of its own so that the symmetric Dirichlet kernel keeps
-// its register budget.
-template <typename T, int DOF, int S0, int FACES>
-cudaError_t eval_k4(const RArgs<T>& A, bool full, bool energy, bool pairs, int nb, size_t smem,
-                    cudaStream_t s, bool set = false) {
-  if (set) {
-    cudaError_t e;
-    if ((e = eval_k<T, DOF, true, true, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
-    if ((e = eval_k<T, DOF, true, false, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
-    if ((e = eval_k<T, DOF, false, true, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
-    return eval_k<T, DOF, false, false, S0, FACES>(A, pairs, nb, smem, s, true);
-  }
-  if (full && energy) return eval_k<T, DOF, true, true, S0, FACES>(A, pairs, nb, smem, s);
-  if (full) return eval_k<T, DOF, true, false, S0, FACES>(A, pairs, nb, smem, s);
-  if (energy) return eval_k<T, DOF, false, true, S0, FACES>(A, pairs, nb, smem, s);
-  return eval_k<T, DOF, false, false, S0, FACES>(A, pairs, nb, smem, s);
-}
-
-template <typename T, int DOF>
-cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
-                          void* H, double* energy, cudaStream_t s) {
-  RArgs<T> A = make_rargs<T>(L, t, x, nullptr, g, H, nullptr, energy != nullptr);
-  const int nb = rows_blocks(L.V);
-  const size_t smem = rows_smem_bytes(L);
-  const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
-  const bool pairs = L.prow != nullptr;
-  const bool en = energy != nullptr;
-  cudaError_t e;
-  if ((DOF == 2 && (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP))) ||
-      (DOF == 3 && (t.mask & MAD_TERM_AREA))) {
-    // face terms: the face-row instantiations; without edge terms the kernel
-    // carries no edge-slot code (S0 = 0)
-    auto faces_k = [&](auto s0c) {
-      constexpr int S0F = decltype(s0c)::value;
-      if constexpr (DOF == 2) {
-        if (t.mask & MAD_TERM_ARAP) return eval_k4<T, DOF, S0F, 2>(A, full, en, pairs, nb, smem, s);
-      }
-      return eval_k4<T, DOF, S0F, 1>(A, full, en, pairs, nb, smem, s);
-    };
-    if (t.mask & MAD_TERM_SPRING)
-      e = faces_k(std::integral_constant<int, kS0Max>{});
-    else
-      e = faces_k(std::integral_constant<int, 0>{});
-  } else if (L.s0 <= 6) {
-    // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
-    // narrower instantiation: fewer registers
-    e = eval_k4<T, DOF, 6, 0>(A, full, en, pairs, nb, smem, s);
-  } else {
-    e = eval_k4<T, DOF, kS0Max, 0>(A, full, en, pairs, nb, smem, s);
-  }
-  if (e != cudaSuccess || !energy) return e;
-  k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
-  return cudaGetLastError();
-}
-
-template <typename T, int DOF>
-cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
-                         void* y, cudaStream_t s) {
-  RArgs<T> A = make_rargs<T>(L, t, x, v, nullptr, nullptr, y, false);
-  const int nb = rows_blocks(L.V);
-  const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
-  if constexpr (DOF == 2) {
-    if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
-      const int kind = face2_kind(t.mask);
-      if (L.nF > 0) {
-        const unsigned nbf = (unsigned)((L.nF + 255) / 256);
-        const bool vec2 = ((((uintptr_t)x) | ((uintptr_t)v)) % (2 * sizeof(T))) == 0;
-        if (full)
-          k_face_hv<T, true><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
-                                                 (const T*)t.face_Minv, (const T*)t.face_area,
-                                                 (T*)L.fhv, kind);
-        else
-          k_face_hv<T, false><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
-                                                  (const T*)t.face_Minv, (const T*)t.face_area,
-                                                  (T*)L.fhv, kind);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-      }
-      const bool sp = t.mask & MAD_TERM_SPRING;
-      if (sp && full)
-        k_rows_hvp<T, DOF, true, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (sp)
-        k_rows_hvp<T, DOF, false, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (full)
-        k_rows_hvp<T, DOF, true, 0, true><<<nb, kRowThreads, 0, s>>>(A);
-      else
-        k_rows_hvp<T, DOF, false, 0, true><<<nb, kRowThreads, 0, s>>>(A);
-      return cudaGetLastError();
-    }
-  }
-  if constexpr (DOF == 3) {
-    if (t.mask & MAD_TERM_AREA) {
-      if (L.nF > 0) {
-        const unsigned nbf = (unsigned)((L.nF + 255) / 256);
-        if (full)
-          k_face_hv_area<T, true><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
-                                                      (const T*)t.face_area, (T)t.area_k,
-                                                      (T*)L.fhv);
-        else
-          k_face_hv_area<T, false><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
-                                                       (const T*)t.face_area, (T)t.area_k,
-                                                       (T*)L.fhv);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-      }
-      const bool sp = t.mask & MAD_TERM_SPRING;
-      if (sp && full)
-        k_rows_hvp<T, DOF, true, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (sp)
-        k_rows_hvp<T, DOF, false, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (full)
-        k_rows_hvp<T, DOF, true, 0, true><<<nb, kRowThreads, 0, s>>>(A);
-      else
-        k_rows_hvp<T, DOF, false, 0, true><<<nb, kRowThreads, 0, s>>>(A);
-      return cudaGetLastError();
-    }
-  }
-  if (L.s0 <= 6) {
-    if (full)
-      k_rows_hvp<T, DOF, true, 6, false><<<nb, kRowThreads, 0, s>>>(A);
-    else
-      k_rows_hvp<T, DOF, false, 6, false><<<nb, kRowThreads, 0, s>>>(A);
-  } else {
-    if (full)
-      k_rows_hvp<T, DOF, true, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
-    else
-      k_rows_hvp<T, DOF, false, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
-  }
-  return cudaGetLastError();
-}
-
-template <typename T, int DOF>
-cudaError_t set_rows_limits(size_t bytes) {
-  RArgs<T> A{};
-  cudaError_t e;
-  if ((e = eval_k4<T, DOF, 6, 0>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
-    return e;
-  if ((e = eval_k4<T, DOF, kS0Max, 0>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
-    return e;
-  if ((e = eval_k4<T, DOF, kS0Max, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
-    return e;
-  if ((e = eval_k4<T, DOF, 0, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
-    return e;
-  if constexpr (DOF == 2) {
-    if ((e = eval_k4<T, DOF, kS0Max, 2>(A, false, false, false, 0, bytes, 0, true)) !=
-        cudaSuccess)
-      return e;
-    if ((e = eval_k4<T, DOF, 0, 2>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
-      return e;
-  }
-  return cudaSuccess;
-}
-
-}  // namespace
 
 int rows_blocks(int V) {
   const int tiles = (V + 31) / 32;
@@ -984,8 +17,8 @@ size_t rows_smem_bytes(const RowsLaunch& L) {
 
 cudaError_t rows_set_smem_limits(int dtype, int dof, size_t bytes) {
   if (dtype == MAD_F64)
-    return dof == 2 ? set_rows_limits<double, 2>(bytes) : set_rows_limits<double, 3>(bytes);
-  return dof == 2 ? set_rows_limits<float, 2>(bytes) : set_rows_limits<float, 3>(bytes);
+    return dof == 2 ? rows_limits_t<double, 2>(bytes) : rows_limits_t<double, 3>(bytes);
+  return dof == 2 ? rows_limits_t<float, 2>(bytes) : rows_limits_t<float, 3>(bytes);
 }
 
 cudaError_t launch_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
@@ -995,20 +28,20 @@ cudaError_t launch_rows_eval(const RowsLaunch& L, const mad_terms& t, const void
     return cudaSuccess;
   }
   if (L.dtype == MAD_F64)
-    return L.dof == 2 ? run_rows_eval<double, 2>(L, t, x, g, H, energy, s)
-                      : run_rows_eval<double, 3>(L, t, x, g, H, energy, s);
-  return L.dof == 2 ? run_rows_eval<float, 2>(L, t, x, g, H, energy, s)
-                    : run_rows_eval<float, 3>(L, t, x, g, H, energy, s);
+    return L.dof == 2 ? rows_eval_t<double, 2>(L, t, x, g, H, energy, s)
+                      : rows_eval_t<double, 3>(L, t, x, g, H, energy, s);
+  return L.dof == 2 ? rows_eval_t<float, 2>(L, t, x, g, H, energy, s)
+                    : rows_eval_t<float, 3>(L, t, x, g, H, energy, s);
 }
 
 cudaError_t launch_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
                             const void* v, void* y, cudaStream_t s) {
   if (L.V == 0) return cudaSuccess;
   if (L.dtype == MAD_F64)
-    return L.dof == 2 ? run_rows_hvp<double, 2>(L, t, x, v, y, s)
-                      : run_rows_hvp<double, 3>(L, t, x, v, y, s);
-  return L.dof == 2 ? run_rows_hvp<float, 2>(L, t, x, v, y, s)
-                    : run_rows_hvp<float, 3>(L, t, x, v, y, s);
+    return L.dof == 2 ? rows_hvp_t<double, 2>(L, t, x, v, y, s)
+                      : rows_hvp_t<double, 3>(L, t, x, v, y, s);
+  return L.dof == 2 ? rows_hvp_t<float, 2>(L, t, x, v, y, s)
+                    : rows_hvp_t<float, 3>(L, t, x, v, y, s);
 }
 
 }  // namespace mad
