@@ -40,6 +40,7 @@ ALGO_BYTES = 4 * (3 * V_FULL) + 8 * E_FULL + 4 * (3 * V_FULL) + 36 * NNZB_FULL
 PAGES_MS_1000 = 11.7  # the page's own 1000^2 mass-spring grad+Hessian time (RTX 4090)
 FALLBACK_HBM_GBS = 6650.0
 METRIC = "grad+Hessian assembly ms/step (1000^2 cloth); achieved HBM GB/s vs ~8 TB/s"
+KERNEL = "k_rows_eval_c<float,3> (row-streaming assembly, compact row tables)"
 WORKLOAD = ("mass-spring cloth 1000x1000 grid (10^6 vertices, 2,996,001 springs, "
             "6,992,002 3x3 blocks): springs + inertia, g + block-CSR H per step")
 
@@ -174,30 +175,24 @@ def run_ours(args, rank, world, dist):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    # per-launch events bracket every `event_every`-th step (all of them at 1):
-    # fewer event records between launches perturb the timed loop less
-    every = max(1, args.event_every)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(0, args.steps, every)]
+    # The timed loop has no events between its launches: a step is exactly
+    # one launch of the assembly kernel, so the loop's time per step is the
+    # kernel's time per launch (an event record between back-to-back
+    # launches adds about 2 us of device time).
     clocks = ClockSampler(dev.index)
     clocks.start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for k in range(args.steps):
-        if k % every == 0:
-            evs[k // every][0].record(stream)
-            step(args.warmup + k)
-            evs[k // every][1].record(stream)
-        else:
-            step(args.warmup + k)
+        step(args.warmup + k)
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     if dist:
         dist.barrier()
-    total_ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
-    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    own_ms = t0.elapsed_time(t1)
+    total_ms = max_over_ranks(own_ms, dist, dev)
     ms_per_step = total_ms / args.steps
     value = job_ms_per_unit(total_ms, args.steps, world)
 
@@ -225,13 +220,15 @@ def run_ours(args, rank, world, dist):
                "steps": n_e2e, "api": "mad_eval_host"}
 
     hbm, peak_kind = peaks()
-    avg_launch_ms = statistics.mean(launch_ms)
+    avg_launch_ms = own_ms / args.steps
     achieved = ALGO_BYTES / (avg_launch_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "traffic": kernel_traffic(),
-            "kernel": "k_rows_eval<float,3> (row-streaming assembly)",
+            "kernel": KERNEL,
             "algorithmic_bytes_per_launch": ALGO_BYTES,
-            "avg_launch_ms": round(avg_launch_ms, 5), "launches_timed": len(launch_ms),
+            "avg_launch_ms": round(avg_launch_ms, 5), "launches_timed": args.steps,
+            "launch_time": "this rank's timed loop / steps (one launch per step, no events "
+                           "between launches)",
             "peak_kind": peak_kind}
     out = {
         "metric": METRIC, "value": round(value, 5), "unit": "ms/step", "n_gpus": world,
@@ -247,12 +244,101 @@ def run_ours(args, rank, world, dist):
         "impl": "ours",
     }
     if rank == 0 and world == 1 and not args.no_cpu:
-        out["cpu_baseline"] = cpu_baseline(st)
-        if not args.no_extra:
-            out["cpu_baseline"]["rows"] = cpu_baseline_rows(st)
+        with pinned_core() as core:
+            out["cpu_baseline"] = cpu_baseline(st)
+            if not args.no_extra:
+                out["cpu_baseline"]["rows"] = cpu_baseline_rows(st)
+        out["cpu_baseline"].update(cpu_info(core))
     if not args.no_extra and rank == 0:
         out["workloads"] = extra_workloads(args)
+        out["rooflines"] = rooflines(out["workloads"], ms_per_step, hbm, peak_kind)
     ctx.close()
+    return out
+
+
+class pinned_core:
+    """Runs the block on one host core (the process's affinity is restored
+    afterwards); yields the core's index."""
+
+    def __enter__(self):
+        self.saved = os.sched_getaffinity(0)
+        core = max(self.saved)
+        os.sched_setaffinity(0, {core})
+        return core
+
+    def __exit__(self, *exc):
+        os.sched_setaffinity(0, self.saved)
+        return False
+
+
+def cpu_info(core):
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cpu_model": model, "pinned_core": core, "host_cores": os.cpu_count()}
+
+
+def cloth_bytes(n, esz):
+    """Algorithmic bytes of one cloth step (read x and the edge list, write g
+    and the Hessian blocks) on the n x n grid, floats of esz bytes."""
+    V = n * n
+    E = 2 * n * (n - 1) + (n - 1) ** 2
+    return esz * 3 * V + 8 * E + esz * 3 * V + esz * 9 * (V + 2 * E)
+
+
+def param_bytes(n):
+    """Algorithmic bytes of the 500^2 parameterization (fp32, dof 2): eval
+    reads UV and the face list and writes g and the 2x2 blocks; the product
+    reads UV, v and the face list and writes y."""
+    V = n * n
+    F = 2 * (n - 1) ** 2
+    E = 2 * n * (n - 1) + (n - 1) ** 2
+    return 8 * V + 12 * F + 8 * V + 16 * (V + 2 * E), 8 * V * 3 + 12 * F
+
+
+def rooflines(w, headline_ms, hbm, peak_kind):
+    """Fraction of the HBM peak per workload: algorithmic bytes / time."""
+    V, E, F, P = V_FULL, E_FULL, 2 * (N_GRID - 1) ** 2, 100_000
+    pe, ph = param_bytes(500)
+    rows = {
+        "cloth10": (cloth_bytes(10, 4), w.get("cloth10_graph_eval_ms")),
+        "cloth10_call": (cloth_bytes(10, 4), w.get("cloth10_eval_ms")),
+        "cloth100": (cloth_bytes(100, 4), w.get("cloth100_graph_eval_ms")),
+        "cloth100_call": (cloth_bytes(100, 4), w.get("cloth100_eval_ms")),
+        "cloth100_f64": (cloth_bytes(100, 8), w.get("cloth100_f64_eval_ms")),
+        "cloth1000": (ALGO_BYTES, headline_ms),
+        "symdir500_eval": (pe, w.get("symdir500_eval_ms")),
+        "symdir500_hvp": (ph, w.get("symdir500_hvp_ms")),
+        "arap500_eval": (pe, w.get("arap500_eval_ms")),
+        "arap500_hvp": (ph, w.get("arap500_hvp_ms")),
+        # pairs: x, edges, pair list, g and the blocks of the pattern with the pairs
+        "pairs1000_assembly": (12 * V + 8 * E + 8 * P + 12 * V + 36 * (V + 2 * E + 2 * P),
+                               w.get("pairs1000_assembly_ms")),
+        # insertion: read the mesh row_ptr and col_idx and the pairs, write the new ones
+        "pairs1000_insert": (4 * (V + 1) * 2 + 4 * (V + 2 * E) + 4 * (V + 2 * E + 2 * P) + 8 * P,
+                             w.get("pairs1000_insert_ms")),
+        "jac1000": (w.get("jac1000_bytes"), w.get("jac1000_ms")),
+        "area1000_eval": (ALGO_BYTES + 16 * F, w.get("area1000_eval_ms")),
+        "area1000_hvp": (12 * V * 3 + 12 * E + 16 * F, w.get("area1000_hvp_ms")),
+        "vf1000_eval": (w.get("vf1000_eval_bytes"), w.get("vf1000_eval_ms")),
+    }
+    out = {}
+    for k, (b, ms) in rows.items():
+        if not b or not ms:
+            continue
+        gbs = b / (ms * 1e-3) / 1e9
+        out[k] = {"bytes": int(b), "ms": round(ms, 5), "gbs": round(gbs, 1),
+                  "frac": round(gbs / hbm, 4)}
+    out["peak_gbs"] = hbm
+    out["peak_kind"] = peak_kind
+    out["note"] = ("algorithmic bytes (read x and topology, write g and the Hessian values "
+                   "or y) / median CUDA-event time; *_call rows are single launches, the "
+                   "others CUDA-graph replays where named so in workloads")
     return out
 
 
@@ -439,6 +525,12 @@ def vf1000(res, mad, torch, dev, stream, timeit):
     y = torch.empty((st["V"], 3), device=dev)
     H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
     res["vf1000_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+    # read x, the edge list, the terms (vertex, face, rest) and their faces'
+    # corners; write g and the blocks of the pattern holding the terms' pairs
+    _, _, nz = ctx.mad_pattern()
+    nnzb = int(nz.cpu()[0])
+    V, E = st["V"], len(st["edges"])
+    res["vf1000_eval_bytes"] = 12 * V + 8 * E + 24 * N_VF + 12 * V + 36 * nnzb
     res["vf1000_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
     res["vf1000_status"] = ctx.mad_status_sync()
     ctx.close()
@@ -567,38 +659,52 @@ def pairs1000(res, mad, torch, dev, stream):
 # ---------------------------------------------------------------- reference
 
 
+# Whole 1000^2 oracle steps take about 2 s each on one host core; runs of
+# more steps than this time a bounded sample per step instead.
+REF_FULL_STEPS_MAX = 40
+
+
 def run_reference(args):
-    """The oracle on the host cores: each step assembles a bounded sample (the
-    250x250 grid, same energy and noise law) and is scaled to a 1000^2 step by
-    the ratio of term counts."""
+    """The oracle on one pinned host core.  Each step is a whole 1000^2 cloth
+    step (fp64 closed forms, COO sort + merge) on a fresh perturbation, when
+    warm-up + timed steps <= REF_FULL_STEPS_MAX; otherwise each step is the
+    same workload on the 250x250 grid, scaled to a 1000^2 step by the ratio
+    of term counts (stated in `sample`)."""
     import oracle
     orc = oracle.load()
-    ns = args.ref_sample_n
+    full = args.steps + args.warmup <= REF_FULL_STEPS_MAX
+    ns = N_GRID if full else args.ref_sample_n
     st = mi.cloth_static(ns, np.float32)
     rp, ci = orc.pattern(st["V"], st["F"])
     terms_s = st["edges"].shape[0] + st["V"]
     scale = (E_FULL + V_FULL) / terms_s
-    x = mi.cloth_x(ns, SEED, 0, np.float32)
+    xs = [mi.cloth_x(ns, SEED, 30_000 + s, np.float32) for s in range(2)]
 
-    def step():
-        orc.eval(st["V"], 3, x, 3, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
+    def step(k):
+        orc.eval(st["V"], 3, xs[k % 2], 3, rp, ci, edges=st["edges"], L0=st["L0"], k=st["k"],
                  xt=st["xt"], w=st["w"])
 
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    ms = (time.perf_counter() - t0) * 1e3 / args.steps * scale
-    sample = (f"{ns}x{ns} grid per step ({terms_s} terms), scaled by {scale:.3f} to a "
-              "1000x1000 step")
+    with pinned_core() as core:
+        for k in range(args.warmup):
+            step(k)
+        t0 = time.perf_counter()
+        for k in range(args.steps):
+            step(k)
+        ms = (time.perf_counter() - t0) * 1e3 / args.steps * scale
+    if full:
+        sample = f"whole {N_GRID}x{N_GRID} steps ({terms_s} terms), two perturbations alternating"
+    else:
+        sample = (f"{ns}x{ns} grid per step ({terms_s} terms), scaled by {scale:.3f} to a "
+                  f"{N_GRID}x{N_GRID} step")
+    cpu = {"value": round(ms, 3), "unit": "ms/step", "cores": 1, "kind": "oracle",
+           "sample": sample}
+    cpu.update(cpu_info(core))
     return {"metric": METRIC, "value": round(ms, 3), "unit": "ms/step", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": round(ms / PAGES_MS_1000, 4),
             "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD, "n": N_GRID, "sample": sample},
-            "cpu_baseline": {"value": round(ms, 3), "unit": "ms/step", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": cpu,
             "e2e": {"value": round(ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -610,9 +716,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--pool", type=int, default=32)
-    ap.add_argument("--event-every", type=int, default=4,
-                    help="bracket every n-th timed launch with CUDA events (per-launch "
-                         "duration for the roofline)")
     ap.add_argument("--patch-faces", type=int, default=512)
     ap.add_argument("--flags", type=int, default=0, help="MAD_EVAL_* bits for the timed step")
     ap.add_argument("--no-e2e", action="store_true")

@@ -56,7 +56,8 @@ STATUS_NAMES = {0: "MAD_OK", 1: "MAD_ERR_INVALID_ARG", 2: "MAD_ERR_CUDA", 3: "MA
 EXPORTS = ("mad_default_opts", "mad_create", "mad_info", "mad_edges", "mad_pattern",
            "mad_eval", "mad_hvp", "mad_add_pairs", "mad_status_sync", "mad_eval_host",
            "mad_last_error", "mad_destroy", "mad_selftest_dual", "mad_energy_noalloc",
-           "mad_jacobian_shape", "mad_jacobian_pattern", "mad_jacobian")
+           "mad_jacobian_shape", "mad_jacobian_pattern", "mad_jacobian", "mad_shard_plan",
+           "mad_shard_halo", "mad_eval_shard")
 
 
 class mad_opts(ctypes.Structure):
@@ -81,7 +82,8 @@ class mad_info_t(ctypes.Structure):
                 ("nnzb_base", ctypes.c_int32), ("capacity_blocks", ctypes.c_int32),
                 ("max_pairs", ctypes.c_int32), ("n_patches", ctypes.c_int32),
                 ("max_patch_vertices", ctypes.c_int32), ("max_patch_owned", ctypes.c_int32),
-                ("smem_bytes", ctypes.c_int32), ("device_bytes", ctypes.c_int64)]
+                ("smem_bytes", ctypes.c_int32), ("device_bytes", ctypes.c_int64),
+                ("row_slot_bytes", ctypes.c_int32)]
 
 
 class MadError(RuntimeError):
@@ -130,6 +132,13 @@ def load_library(path: str = LIB_PATH):
     lib.mad_destroy.restype = None
     lib.mad_selftest_dual.argtypes = [i32, vp, vp]
     lib.mad_selftest_dual.restype = ctypes.c_int
+    lib.mad_shard_plan.argtypes = [i32, i32, i32p, i32, i32p, ctypes.POINTER(ctypes.c_int64)]
+    lib.mad_shard_plan.restype = ctypes.c_int
+    lib.mad_shard_halo.argtypes = [i32, i32, i32p, i32, i32, i32p, i32p, i32]
+    lib.mad_shard_halo.restype = ctypes.c_int
+    lib.mad_eval_shard.argtypes = [vp, i32, i32p, ctypes.POINTER(vp), i32,
+                                   ctypes.POINTER(mad_terms), vp, vp, vp, vp]
+    lib.mad_eval_shard.restype = ctypes.c_int
     i64p = ctypes.POINTER(ctypes.c_int64)
     lib.mad_jacobian_shape.argtypes = [vp, ctypes.c_uint32, i64p, i64p]
     lib.mad_jacobian_shape.restype = ctypes.c_int
@@ -300,6 +309,28 @@ class Context:
                                _stream_ptr(stream))
         self._check(st)
 
+    def mad_eval_shard(self, row_begin, x_parts, rank, terms: Terms, g_part, H_part,
+                       energy=None, stream=None):
+        """Rows of shard `rank` (see include/mad.h).  row_begin: int array
+        [nranks+1]; x_parts: per shard a CUDA tensor [rows][dof] or a raw
+        device address (int) readable from this device."""
+        torch = _torch()
+        rb = np.ascontiguousarray(np.asarray(row_begin, np.int32))
+        n = rb.shape[0] - 1
+        ptrs = (ctypes.c_void_p * max(n, 1))()
+        for r, xp in enumerate(x_parts):
+            if isinstance(xp, int):
+                ptrs[r] = xp
+            elif rb[r + 1] > rb[r]:
+                ptrs[r] = _dev_ptr(xp, self.torch_dtype, f"x_parts[{r}]")
+        t = terms.to_c(self.torch_dtype)
+        st = self.lib.mad_eval_shard(
+            self.h, n, rb.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), ptrs, int(rank),
+            ctypes.byref(t), _dev_ptr(g_part, self.torch_dtype, "g_part", allow_none=True),
+            _dev_ptr(H_part, self.torch_dtype, "H_part", allow_none=True),
+            _dev_ptr(energy, torch.float64, "energy", allow_none=True), _stream_ptr(stream))
+        self._check(st)
+
     def mad_hvp(self, x, terms: Terms, v, y, stream=None):
         t = terms.to_c(self.torch_dtype)
         st = self.lib.mad_hvp(self.h, _dev_ptr(x, self.torch_dtype, "x"), ctypes.byref(t),
@@ -363,6 +394,43 @@ load_library()  # fail loudly at import when the CUDA library is missing
 
 def mad_create(V, F, dof, dtype="float32", **kw) -> Context:
     return Context(V, F, dof, dtype, **kw)
+
+
+def _faces_arg(F):
+    F = np.ascontiguousarray(np.asarray(F, np.int32).reshape(-1, 3))
+    return F, F.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def mad_shard_plan(V: int, F, nranks: int):
+    """(row_begin int32 [nranks+1], block_begin int64 [nranks+1]): contiguous
+    row ranges balanced by block count (host only, see include/mad.h)."""
+    lib = load_library()
+    F, fp = _faces_arg(F)
+    rb = np.zeros(nranks + 1, np.int32)
+    bb = np.zeros(nranks + 1, np.int64)
+    st = lib.mad_shard_plan(int(V), F.shape[0], fp, int(nranks),
+                            rb.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                            bb.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+    if st != MAD_OK:
+        raise MadError(st, "mad_shard_plan")
+    return rb, bb
+
+
+def mad_shard_halo(V: int, F, row_lo: int, row_hi: int) -> np.ndarray:
+    """Sorted vertices outside [row_lo, row_hi) that its rows couple to."""
+    lib = load_library()
+    F, fp = _faces_arg(F)
+    n = ctypes.c_int32(0)
+    st = lib.mad_shard_halo(int(V), F.shape[0], fp, int(row_lo), int(row_hi), ctypes.byref(n),
+                            None, 0)
+    if st != MAD_OK:
+        raise MadError(st, "mad_shard_halo")
+    out = np.zeros(max(n.value, 1), np.int32)
+    st = lib.mad_shard_halo(int(V), F.shape[0], fp, int(row_lo), int(row_hi), ctypes.byref(n),
+                            out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), out.shape[0])
+    if st != MAD_OK:
+        raise MadError(st, "mad_shard_halo")
+    return out[:n.value]
 
 
 def mad_selftest_dual(ab: np.ndarray) -> np.ndarray:

@@ -53,6 +53,9 @@ struct mad_ctx {
   uint32_t* rows_meta = nullptr;
   int32_t* rows_ofl_ptr = nullptr;
   int2* rows_ofl = nullptr;
+  std::vector<int32_t> rp_host;    // the mesh pattern's row_ptr (host copy)
+  int4* rows_ctile = nullptr;      // compact slots (nullptr when they do not fit)
+  uint32_t* rows_cslots = nullptr;
   // face rows of the same kernel (rows_sf == 0: face terms use the patch kernel)
   int rows_sf = 0;
   int4* rows_fslots = nullptr;
@@ -180,6 +183,8 @@ RowsLaunch rows_launch(const mad_ctx* c) {
   L.meta = c->rows_meta;
   L.ofl_ptr = c->rows_ofl_ptr;
   L.ofl = c->rows_ofl;
+  L.ctile = c->rows_ctile;
+  L.cslots = c->rows_cslots;
   L.sf = c->rows_sf;
   L.fslots = c->rows_fslots;
   L.fofl_ptr = c->rows_fofl_ptr;
@@ -441,10 +446,15 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
       return MAD_ERR_UNIMPLEMENTED;
     }
     c->rows_s0 = rt.s0;
+    c->rp_host = rp;
     CREATE_CK(upload(c, &c->rows_slots, rt.slots));
     CREATE_CK(upload(c, &c->rows_meta, rt.meta));
     CREATE_CK(upload(c, &c->rows_ofl_ptr, rt.ofl_ptr));
     CREATE_CK(upload(c, &c->rows_ofl, rt.ofl));
+    if (!rt.cslots.empty()) {
+      CREATE_CK(upload(c, &c->rows_ctile, rt.ctile));
+      CREATE_CK(upload(c, &c->rows_cslots, rt.cslots));
+    }
     if (nF > 0) {
       HostFaceRows fr;
       if (build_face_rows(V, nF, F, rp.data(), ci.data(), fr).empty()) {
@@ -550,6 +560,7 @@ mad_status mad_info(const mad_ctx* c, mad_info_t* info) {
   info->max_patch_owned = c->no_max;
   info->smem_bytes = (int32_t)c->smem_eval;
   info->device_bytes = c->device_bytes;
+  info->row_slot_bytes = c->rows_cslots ? 4 : 8;
   return MAD_OK;
 }
 
@@ -610,6 +621,44 @@ mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t, const void* v,
     e = launch_vf_hvp(c->dtype, vf_launch(c, t, x), v, y, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(c, e, "mad_hvp vertex-face launch");
   }
+  return MAD_OK;
+}
+
+mad_status mad_eval_shard(mad_ctx* c, int32_t nranks, const int32_t* row_begin,
+                          const void* const* x_parts, int32_t rank, const mad_terms* t,
+                          void* g_part, void* H_part, double* energy, void* stream) {
+  if (!c) return MAD_ERR_INVALID_ARG;
+  mad_status st = check_terms(c, t);
+  if (st != MAD_OK) return st;
+  if (nranks < 1 || nranks > MAD_MAX_SHARDS || !row_begin || !x_parts || rank < 0 ||
+      rank >= nranks)
+    return fail(c, MAD_ERR_INVALID_ARG, "nranks, row_begin, x_parts or rank");
+  if (row_begin[0] != 0 || row_begin[nranks] != c->V)
+    return fail(c, MAD_ERR_INVALID_ARG, "row_begin must run from 0 to V");
+  for (int r = 0; r < nranks; ++r) {
+    if (row_begin[r + 1] < row_begin[r])
+      return fail(c, MAD_ERR_INVALID_ARG, "row_begin must not decrease");
+    if (row_begin[r] % 32 != 0 && row_begin[r] != c->V)
+      return fail(c, MAD_ERR_INVALID_ARG, "shard boundaries must be multiples of 32 rows");
+    if (row_begin[r + 1] > row_begin[r] && !x_parts[r])
+      return fail(c, MAD_ERR_INVALID_ARG, "x_parts of a non-empty shard is NULL");
+  }
+  if (t->mask & ~(uint32_t)(MAD_TERM_SPRING | MAD_TERM_INERTIA))
+    return fail(c, MAD_ERR_UNIMPLEMENTED, "sharded evaluation takes spring and inertia terms");
+  if (t->flags & (MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED))
+    return fail(c, MAD_ERR_UNIMPLEMENTED, "sharded evaluation uses the row kernel");
+  if (c->active >= 0)
+    return fail(c, MAD_ERR_UNIMPLEMENTED, "sharded evaluation needs the mesh pattern (no pairs)");
+  if (!c->rows_cslots)
+    return fail(c, MAD_ERR_UNIMPLEMENTED, "sharded evaluation needs compact row tables");
+  const int lo = row_begin[rank], hi = row_begin[rank + 1];
+  if (hi > lo && (!g_part || !H_part))
+    return fail(c, MAD_ERR_INVALID_ARG, "g_part and H_part must be device pointers");
+  const int64_t block_lo = c->rp_host[lo];
+  cudaError_t e = launch_rows_eval_shard(rows_launch(c), *t, nranks, row_begin, block_lo,
+                                         x_parts, rank, g_part, H_part, energy,
+                                         as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval_shard launch");
   return MAD_OK;
 }
 

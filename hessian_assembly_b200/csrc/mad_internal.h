@@ -106,6 +106,16 @@ struct HostRowTables {
   std::vector<uint32_t> meta;     // [V] off-diagonal count | diagonal position << 16
   std::vector<int32_t> ofl_ptr;   // [V+1] overflow slots per row (prefix sums)
   std::vector<int2> ofl;          // overflow slots
+  // Compact form of the same slots, built when every delta below fits 16
+  // bits (empty vectors otherwise).  Per tile t of 32 rows: ctile[t] =
+  // {row_ptr of row 32t, id of the first edge (a, b) with a >= 32t, mask of
+  // the tile's rows that continue in the overflow table, 0}.  Per slot: the
+  // column minus the row and the edge id minus the tile's first edge id, as
+  // two int16 halves (low, high) of one word; 0 marks an empty slot (a
+  // column never equals its row).  Row pointers follow from the tile's
+  // row_ptr and the rows' lengths, so neither row_ptr nor meta is read.
+  std::vector<int4> ctile;        // [ntiles]
+  std::vector<uint32_t> cslots;   // [ntiles][s0][32]
 };
 std::string build_row_tables(int V, const int32_t* rp, const int32_t* ci, int s0_cap,
                              HostRowTables& out);
@@ -254,6 +264,8 @@ struct RowsLaunch {
   const uint32_t* meta;
   const int32_t* ofl_ptr;
   const int2* ofl;
+  const int4* ctile;        // compact slots (see HostRowTables); nullptr if absent
+  const uint32_t* cslots;
   const int32_t* rp;  // active row_ptr
   const int32_t* prow;
   const int32_t* pe_col;
@@ -268,6 +280,11 @@ cudaError_t launch_rows_eval(const RowsLaunch& L, const mad_terms& t, const void
                              void* H, double* energy, cudaStream_t s);
 cudaError_t launch_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
                             const void* v, void* y, cudaStream_t s);
+// the rows of one shard (edge and vertex terms, compact row tables)
+cudaError_t launch_rows_eval_shard(const RowsLaunch& L, const mad_terms& t, int nranks,
+                                   const int32_t* row_begin, int64_t block_lo,
+                                   const void* const* x_parts, int rank, void* g, void* H,
+                                   double* energy, cudaStream_t s);
 
 // jacobian.cu
 void jac_shape(int V, int dof, unsigned mask, int nE, int nF, int64_t* rows, int64_t* nnz);

@@ -28,15 +28,21 @@ static __device__ __align__(256) double g_partials[kNaMaxBlocks];
 double* g_partials_addr[kNaMaxDevices] = {};
 std::mutex g_setup_mutex;
 
-// Device address of g_partials on the current device (looked up once per
-// device; host code must not use the symbol itself as an address).
-cudaError_t partials_address(double** out) {
+// Device address of g_partials on the current device (host code must not
+// use the symbol itself as an address).  A call on a stream that is not
+// being captured looks the address up again, so a context created anew on
+// the device (after cudaDeviceReset) is picked up; a call under capture
+// takes the address the last uncaptured call found.
+cudaError_t partials_address(cudaStream_t s, double** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kNaMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_partials_addr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone || !g_partials_addr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_partials);
     if (e != cudaSuccess) return e;
@@ -45,6 +51,10 @@ cudaError_t partials_address(double** out) {
   *out = g_partials_addr[dev];
   return cudaSuccess;
 }
+
+// A vertex index the term may read: in [0, V).  A term with any other index
+// is skipped and contributes a NaN, so the returned energy shows it.
+__device__ __forceinline__ bool vok(int v, int V) { return (unsigned)v < (unsigned)V; }
 
 template <typename T>
 struct NaArgs {
@@ -79,12 +89,17 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
                           : 0;
   const int64_t nPr = (A.mask & MAD_TERM_PAIR) ? A.nP : 0;
   double e = 0.0;
+  const double bad = __longlong_as_double(0x7FF8000000000000LL);  // quiet NaN
   if (t < nS) {
     const int a = A.edges[2 * t], b = A.edges[2 * t + 1];
-    T d[DOF];
+    if (vok(a, A.V) && vok(b, A.V)) {
+      T d[DOF];
 #pragma unroll
-    for (int c = 0; c < DOF; ++c) d[c] = A.x[(int64_t)a * DOF + c] - A.x[(int64_t)b * DOF + c];
-    e = (double)spring_energy(d, A.L0[t], A.k);
+      for (int c = 0; c < DOF; ++c) d[c] = A.x[(int64_t)a * DOF + c] - A.x[(int64_t)b * DOF + c];
+      e = (double)spring_energy(d, A.L0[t], A.k);
+    } else {
+      e = bad;
+    }
   } else if (t < nS + nI) {
     const int64_t i = t - nS;
     T s = T(0);
@@ -92,11 +107,14 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
     for (int c = 0; c < DOF; ++c) s += sq(A.x[i * DOF + c] - A.xt[i * DOF + c]);
     e = (double)(s * (T(0.5) * A.w));
   } else if (t < nS + nI + nFc) {
-    if constexpr (DOF == 2) {
-      const int64_t f = t - nS - nI;
-      const T* u0 = A.x + (int64_t)A.F[3 * f] * 2;
-      const T* u1 = A.x + (int64_t)A.F[3 * f + 1] * 2;
-      const T* u2 = A.x + (int64_t)A.F[3 * f + 2] * 2;
+    const int64_t f = t - nS - nI;
+    const int c0 = A.F[3 * f], c1 = A.F[3 * f + 1], c2 = A.F[3 * f + 2];
+    if (!(vok(c0, A.V) && vok(c1, A.V) && vok(c2, A.V))) {
+      e = bad;
+    } else if constexpr (DOF == 2) {
+      const T* u0 = A.x + (int64_t)c0 * 2;
+      const T* u1 = A.x + (int64_t)c1 * 2;
+      const T* u2 = A.x + (int64_t)c2 * 2;
       const T* M = A.Minv + 4 * f;
       T j[4];
 #pragma unroll
@@ -106,10 +124,9 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
           j[2 * al + ga] = (u1[al] - u0[al]) * M[ga] + (u2[al] - u0[al]) * M[2 + ga];
       e = (double)face2_energy(j, A.area[f], face2_kind(A.mask));
     } else {
-      const int64_t f = t - nS - nI;
-      const T* u0 = A.x + (int64_t)A.F[3 * f] * 3;
-      const T* u1 = A.x + (int64_t)A.F[3 * f + 1] * 3;
-      const T* u2 = A.x + (int64_t)A.F[3 * f + 2] * 3;
+      const T* u0 = A.x + (int64_t)c0 * 3;
+      const T* u1 = A.x + (int64_t)c1 * 3;
+      const T* u2 = A.x + (int64_t)c2 * 3;
       T e1[3], e2[3];
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
@@ -121,10 +138,14 @@ __global__ void __launch_bounds__(kNaThreads) k_energy_terms(const NaArgs<T> A) 
   } else if (t < nS + nI + nFc + nPr) {
     const int64_t p = t - nS - nI - nFc;
     const int a = A.pairs[2 * p], b = A.pairs[2 * p + 1];
-    T d[DOF];
+    if (vok(a, A.V) && vok(b, A.V)) {
+      T d[DOF];
 #pragma unroll
-    for (int c = 0; c < DOF; ++c) d[c] = A.x[(int64_t)a * DOF + c] - A.x[(int64_t)b * DOF + c];
-    e = (double)spring_energy(d, A.prest[p], A.kp);
+      for (int c = 0; c < DOF; ++c) d[c] = A.x[(int64_t)a * DOF + c] - A.x[(int64_t)b * DOF + c];
+      e = (double)spring_energy(d, A.prest[p], A.kp);
+    } else {
+      e = bad;
+    }
   }
   __shared__ double red[kNaThreads / 32];
 #pragma unroll
@@ -210,11 +231,11 @@ extern "C" mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, c
     return MAD_ERR_CAPACITY;
   }
   double* partials = nullptr;
-  cudaError_t e = mad::partials_address(&partials);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = mad::partials_address(s, &partials);
   if (e != cudaSuccess) {
     return MAD_ERR_CUDA;
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const unsigned mask = (sp ? MAD_TERM_SPRING : 0u) | (in ? MAD_TERM_INERTIA : 0u) |
                         (sd ? MAD_TERM_SYMDIR : 0u) | (rp ? MAD_TERM_ARAP : 0u) |
                         (ar ? MAD_TERM_AREA : 0u) |

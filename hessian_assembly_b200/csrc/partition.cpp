@@ -450,6 +450,33 @@ std::string build_row_tables(int V, const int32_t* rp, const int32_t* ci, int s0
       ++k;
     }
   }
+  // the compact slots, when every delta fits its 16 bits
+  out.ctile.resize(ntiles);
+  out.cslots.assign((size_t)ntiles * s0 * 32, 0u);
+  bool fits = true;
+  for (int t = 0; t < ntiles && fits; ++t) {
+    const int v0 = 32 * t;
+    uint32_t ofl_mask = 0;
+    for (int l = 0; l < 32 && v0 + l < V; ++l)
+      if (out.ofl_ptr[v0 + l + 1] > out.ofl_ptr[v0 + l]) ofl_mask |= 1u << l;
+    out.ctile[t] = make_int4(rp[v0], (int32_t)eptr[v0], (int32_t)ofl_mask, 0);
+    for (int k = 0; k < s0 && fits; ++k)
+      for (int l = 0; l < 32; ++l) {
+        const size_t q = ((size_t)t * s0 + k) * 32 + l;
+        const int2 e = out.slots[q];
+        if (e.x < 0) continue;
+        const int64_t dc = (int64_t)e.x - (v0 + l), de = (int64_t)e.y - eptr[v0];
+        if (dc < -32768 || dc > 32767 || de < -32768 || de > 32767) {
+          fits = false;
+          break;
+        }
+        out.cslots[q] = (uint32_t)(uint16_t)(int16_t)dc | ((uint32_t)(uint16_t)(int16_t)de << 16);
+      }
+  }
+  if (!fits) {
+    out.ctile.clear();
+    out.cslots.clear();
+  }
   return "";
 }
 

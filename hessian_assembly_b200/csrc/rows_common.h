@@ -33,5 +33,20 @@ cudaError_t rows_hvp_t(const RowsLaunch& L, const mad_terms& t, const void* x, c
                        void* y, cudaStream_t s);
 template <typename T, int DOF>
 cudaError_t rows_limits_t(size_t bytes);
+// The same assembly for edge and vertex terms on the mesh pattern, driven by
+// the compact slot tables (rows_compact.cu); needs L.cslots.
+template <typename T, int DOF>
+cudaError_t rows_eval_compact_t(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
+                                void* H, double* energy, cudaStream_t s);
+template <typename T, int DOF>
+cudaError_t rows_compact_limits_t(size_t bytes);
+// The rows [row_begin[rank], row_begin[rank+1]) of the same assembly, with
+// the positions of shard r at x_parts[r]; g and H hold the shard's rows and
+// blocks only (H's first block is block_lo of the mesh pattern).
+template <typename T, int DOF>
+cudaError_t rows_eval_shard_t(const RowsLaunch& L, const mad_terms& t, int nranks,
+                              const int32_t* row_begin, int64_t block_lo,
+                              const void* const* x_parts, int rank, void* g, void* H,
+                              double* energy, cudaStream_t s);
 
 }  // namespace mad

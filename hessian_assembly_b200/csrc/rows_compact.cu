@@ -1,0 +1,413 @@
+// rows_compact.cu -- the row-streaming assembly of edge and vertex terms
+// driven by the compact slot tables.
+//
+// Page "Locality-Aware Automatic Differentiation on the GPU for Mesh-Based
+// Computations", section 方法, key design 1: the only global traffic of the
+// step should be reading the mesh and writing the final sparse derivatives;
+// key design 3: the CSR block offsets come from a table built once per
+// topology, so assembly needs no search.
+//
+// Same work as k_rows_eval (rows_impl.cuh) for a term set of springs and
+// inertia on the mesh pattern: one thread per Hessian row, the row's edge
+// terms evaluated with forward-mode AD numbers in registers, each row staged
+// in its warp's slice of shared memory and written back with one 1-D bulk
+// copy per warp.  The row tables it reads are the compact ones
+// (HostRowTables::cslots): 4 bytes per slot instead of 8 and no per-row
+// row_ptr or meta word.  A row's block positions follow from its slots
+// (columns ascend, the diagonal sits after the columns below the row), and
+// the row's first block from the tile's row_ptr plus a warp prefix sum of
+// the row lengths.
+#include "rows_impl.cuh"
+
+namespace mad {
+namespace {
+
+template <typename T>
+struct CArgs {
+  const int4* ctile;
+  const uint32_t* cslots;
+  const int32_t* ofl_ptr;
+  const int2* ofl;
+  const T* x;
+  T* g;
+  T* H;
+  const T* L0;
+  T k;
+  const T* xt;
+  T w;
+  unsigned mask;
+  double* epart;
+  int V, s0, wstage;
+};
+
+// A launch over the rows of one shard (mad_eval_shard): tiles from tile0,
+// rows below row_hi; positions of shard s at xp[s] (rows rbeg[s] ..
+// rbeg[s+1]); g and H hold the shard's rows and blocks only (g's first row
+// is rbeg[own], H's first block hoff).
+template <typename T>
+struct ShardArgs {
+  int tile0, row_hi, own, nparts;
+  int64_t hoff;
+  int rbeg[MAD_MAX_SHARDS + 1];
+  const T* xp[MAD_MAX_SHARDS];
+};
+
+// Positions of vertex v: the own shard's part, else the owner's.
+template <typename T, int DOF>
+__device__ __forceinline__ const T* shard_x(const ShardArgs<T>& S, int v) {
+  const int rb = S.rbeg[S.own], re = S.rbeg[S.own + 1];
+  if ((unsigned)(v - rb) < (unsigned)(re - rb)) return S.xp[S.own] + (uint32_t)((v - rb) * DOF);
+  int o = 0;
+  while (o + 1 < S.nparts && v >= S.rbeg[o + 1]) ++o;
+  return S.xp[o] + (uint32_t)((v - S.rbeg[o]) * DOF);
+}
+
+// Tiles ahead of its own whose slot, position and target lines a warp asks
+// the L2 to fetch before it starts (0: none).  Tiles run in about index
+// order, so tile t + D starts roughly D / (resident warps) waves later.
+#ifndef MAD_ROWSC_PREFETCH_TILES
+#define MAD_ROWSC_PREFETCH_TILES 0
+#endif
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ int slot_dcol(uint32_t w) { return (int)(int16_t)(w & 0xFFFFu); }
+__device__ __forceinline__ int slot_deid(uint32_t w) { return (int)(int16_t)(w >> 16); }
+
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool SHARD>
+__device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T>* S) {
+  constexpr int B = DOF * DOF;
+  constexpr int TD = Tri<DOF>::size;
+  constexpr int VEC = 16 / (int)sizeof(T);
+  extern __shared__ __align__(16) char smem_raw[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int tile = (SHARD ? S->tile0 : 0) + blockIdx.x * kWarps + wib;
+  const int i = tile * 32 + lane;
+  const int row_hi = SHARD ? S->row_hi : A.V;
+  const int goff = SHARD ? S->rbeg[S->own] : 0;   // g's first row
+  const int64_t hoff = SHARD ? S->hoff : 0;        // H's first block
+  const bool tile_live = tile * 32 < row_hi;
+  const bool has = i < row_hi;
+  T* stage = (T*)smem_raw + wib * A.wstage;
+  double energy = 0.0;
+  const bool springs = A.mask & MAD_TERM_SPRING;
+  if constexpr (MAD_ROWSC_PREFETCH_TILES > 0 && !SHARD) {
+    // one 128-byte line per lane: the later tile's slot words, then its
+    // positions and targets (lines past the arrays' ends are skipped)
+    const int tp = tile + MAD_ROWSC_PREFETCH_TILES;
+    constexpr int XL = 32 * DOF * (int)sizeof(T) / 128;  // lines of a tile's rows
+    if (tp * 32 < A.V) {
+      const int64_t nx = (int64_t)A.V * DOF;
+      if (lane < A.s0) {
+        prefetch_l2(A.cslots + (size_t)(tp * A.s0 + lane) * 32);
+      } else if (lane >= 8 && lane < 8 + XL) {
+        const int64_t e = (int64_t)tp * 32 * DOF + (lane - 8) * (128 / (int)sizeof(T));
+        if (e < nx) prefetch_l2(A.x + e);
+      } else if (lane >= 16 && lane < 16 + XL && (A.mask & MAD_TERM_INERTIA)) {
+        const int64_t e = (int64_t)tp * 32 * DOF + (lane - 16) * (128 / (int)sizeof(T));
+        if (e < nx) prefetch_l2(A.xt + e);
+      }
+    }
+  }
+
+  int4 th = make_int4(0, 0, 0, 0);
+  if (tile_live) th = A.ctile[tile];
+  uint32_t sw[S0];
+#pragma unroll
+  for (int k = 0; k < S0; ++k) {
+    sw[k] = 0u;
+    if (has && k < A.s0) sw[k] = A.cslots[(uint32_t)((tile * A.s0 + k) * 32 + lane)];
+  }
+  T xi[DOF], xti[DOF];
+  if (has) {
+    const T* xs = SHARD ? shard_x<T, DOF>(*S, i) : A.x + (uint32_t)(i * DOF);
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xi[a] = xs[a];
+    if (A.mask & MAD_TERM_INERTIA) {
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) xti[a] = A.xt[(uint32_t)(i * DOF + a)];
+    }
+  }
+  // positions and rest lengths behind the slots
+  T xb[S0][DOF];
+  T l0[S0];
+#pragma unroll
+  for (int k = 0; k < S0; ++k) {
+    if (sw[k] == 0u || !springs) continue;
+    const int col = i + slot_dcol(sw[k]);
+    const T* xs = SHARD ? shard_x<T, DOF>(*S, col) : A.x + (uint32_t)(col * DOF);
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xb[k][a] = xs[a];
+    l0[k] = A.L0[th.y + slot_deid(sw[k])];
+  }
+  // row length (off-diagonal slots + overflow + the diagonal) and the row's
+  // first block: the tile's row_ptr plus the lengths of the rows before it
+  int noff = 0, dpos = 0, o0 = 0, no = 0;
+#pragma unroll
+  for (int k = 0; k < S0; ++k) {
+    noff += sw[k] != 0u;
+    dpos += sw[k] != 0u && slot_dcol(sw[k]) < 0;
+  }
+  if (has && ((uint32_t)th.z >> lane) & 1u) {
+    o0 = A.ofl_ptr[i];
+    no = A.ofl_ptr[i + 1] - o0;
+    for (int q = 0; q < no; ++q) dpos += A.ofl[o0 + q].x < i;
+  }
+  noff += no;
+  const int len = has ? noff + 1 : 0;
+  int incl = len;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int d0 = th.x + incl - len, d1 = d0 + len;
+
+  const int dfirst = __shfl_sync(0xffffffffu, d0, 0);
+  T* const h0 = A.H + (uint32_t)((dfirst - hoff) * B);  // the warp's first block in H
+  const int mis = (int)(((uintptr_t)h0 / sizeof(T)) % VEC);
+  const int off = mis + (d0 - dfirst) * B;
+  const bool staged = has && off + (d1 - d0) * B <= A.wstage;
+  if (has) {
+    T* row = staged ? stage + off : h0 + (uint32_t)((d0 - dfirst) * B);
+    T acc[TD], gr[DOF];
+    if (A.mask & MAD_TERM_INERTIA) {
+      T Ei, Hi[B];
+      eval_inertia<T, DOF>(xi, xti, A.w, Ei, gr, Hi);
+      if (ENERGY) energy += (double)Ei;
+#pragma unroll
+      for (int a = 0; a < DOF; ++a)
+#pragma unroll
+        for (int b = a; b < DOF; ++b) acc[Tri<DOF>::idx(a, b)] = Hi[a * DOF + b];
+    } else {
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) gr[a] = T(0);
+#pragma unroll
+      for (int q = 0; q < TD; ++q) acc[q] = T(0);
+    }
+    if (springs) {
+#pragma unroll
+      for (int k = 0; k < S0; ++k) {
+        if (sw[k] == 0u) continue;
+        EdgeRes<T, DOF, FULL> R;
+        eval_edge_res<T, DOF, FULL>(xi, xb[k], l0[k], A.k, R);
+        // block position: the slots before it plus the diagonal when the
+        // column lies above the row
+        const int p = k + (slot_dcol(sw[k]) > 0);
+        apply_edge_side<true>(R, 0, acc, row + p * B, gr);
+        if (ENERGY) energy += 0.5 * (double)edge_energy(R);
+      }
+      for (int q = 0; q < no; ++q) {  // rows longer than the slot table
+        const int2 e = A.ofl[o0 + q];
+        const T* xs = SHARD ? shard_x<T, DOF>(*S, e.x) : A.x + (uint32_t)(e.x * DOF);
+        T xo[DOF];
+#pragma unroll
+        for (int a = 0; a < DOF; ++a) xo[a] = xs[a];
+        EdgeRes<T, DOF, FULL> R;
+        eval_edge_res<T, DOF, FULL>(xi, xo, A.L0[e.y], A.k, R);
+        const int p = A.s0 + q + (e.x > i);
+        apply_edge_side<true>(R, 0, acc, row + p * B, gr);
+        if (ENERGY) energy += 0.5 * (double)edge_energy(R);
+      }
+    } else {
+      // without edge terms every off-diagonal block of the row is zero
+      for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
+    }
+    T* d = row + dpos * B;
+#pragma unroll
+    for (int a = 0; a < DOF; ++a)
+#pragma unroll
+      for (int b = 0; b < DOF; ++b)
+        d[a * DOF + b] = a <= b ? acc[Tri<DOF>::idx(a, b)] : acc[Tri<DOF>::idx(b, a)];
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) A.g[(uint32_t)((i - goff) * DOF + a)] = gr[a];
+  }
+  // ---- write-back of the warp's staged rows (a prefix of its 32 rows) ------
+  fence_async_smem();
+  __syncwarp();
+  if (tile_live) {
+    const unsigned st = __ballot_sync(0xffffffffu, staged);
+    if (st) {
+      const int last = 31 - __clz(st);
+      const int dend = __shfl_sync(0xffffffffu, d1, last);
+      const int n = (dend - dfirst) * B;
+      T* dst = h0;
+      const T* src = stage + mis;
+      const int head = min(n, (VEC - mis) % VEC);
+      const int body = ((n - head) / VEC) * VEC;
+      for (int e = lane; e < head; e += 32) dst[e] = src[e];
+      for (int e = head + body + lane; e < n; e += 32) dst[e] = src[e];
+      const bool aligned = ((((uintptr_t)(dst + head)) | ((uintptr_t)(src + head))) & 15u) == 0;
+      if (body > 0 && !aligned)
+        for (int e = head + lane; e < head + body; e += 32) dst[e] = src[e];
+      if (lane == 0 && body > 0 && aligned) {
+        bulk_store(dst + head, src + head, (uint32_t)(body * sizeof(T)));
+        bulk_commit_and_wait_read();
+      }
+    }
+  }
+  if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
+}
+
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, false>())
+    k_rows_eval_c(const CArgs<T> A) {
+  rows_c_body<T, DOF, FULL, ENERGY, S0, false>(A, nullptr);
+}
+
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, false>())
+    k_rows_eval_cs(const CArgs<T> A, const __grid_constant__ ShardArgs<T> S) {
+  rows_c_body<T, DOF, FULL, ENERGY, S0, true>(A, &S);
+}
+
+// Shared-memory carve-out asked for the kernel, in percent of the unified
+// L1 / shared memory (-1: the driver's choice); a smaller carve-out fits
+// fewer blocks per SM and leaves more L1 for the neighbour gathers.
+#ifndef MAD_ROWSC_CARVEOUT
+#define MAD_ROWSC_CARVEOUT -1
+#endif
+
+template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, int nb, size_t smem,
+                     cudaStream_t s, bool set) {
+  if (set) {
+    const void* ks[2] = {(const void*)k_rows_eval_c<T, DOF, FULL, ENERGY, S0>,
+                         (const void*)k_rows_eval_cs<T, DOF, FULL, ENERGY, S0>};
+    for (const void* k : ks) {
+      cudaError_t e;
+      if (MAD_ROWSC_CARVEOUT >= 0) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 MAD_ROWSC_CARVEOUT);
+        if (e != cudaSuccess) return e;
+      }
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  if (S)
+    k_rows_eval_cs<T, DOF, FULL, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A, *S);
+  else
+    k_rows_eval_c<T, DOF, FULL, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A);
+  return cudaGetLastError();
+}
+
+template <typename T, int DOF, int S0>
+cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, bool full, bool energy, int nb,
+                      size_t smem, cudaStream_t s, bool set) {
+  if (set) {
+    cudaError_t e;
+    if ((e = launch_c<T, DOF, true, true, S0>(A, S, nb, smem, s, true)) != cudaSuccess) return e;
+    if ((e = launch_c<T, DOF, true, false, S0>(A, S, nb, smem, s, true)) != cudaSuccess) return e;
+    if ((e = launch_c<T, DOF, false, true, S0>(A, S, nb, smem, s, true)) != cudaSuccess) return e;
+    return launch_c<T, DOF, false, false, S0>(A, S, nb, smem, s, true);
+  }
+  if (full && energy) return launch_c<T, DOF, true, true, S0>(A, S, nb, smem, s, false);
+  if (full) return launch_c<T, DOF, true, false, S0>(A, S, nb, smem, s, false);
+  if (energy) return launch_c<T, DOF, false, true, S0>(A, S, nb, smem, s, false);
+  return launch_c<T, DOF, false, false, S0>(A, S, nb, smem, s, false);
+}
+
+template <typename T>
+CArgs<T> make_cargs(const RowsLaunch& L, const mad_terms& t, const void* x, void* g, void* H,
+                    bool energy) {
+  CArgs<T> A;
+  A.ctile = L.ctile;
+  A.cslots = L.cslots;
+  A.ofl_ptr = L.ofl_ptr;
+  A.ofl = L.ofl;
+  A.x = (const T*)x;
+  A.g = (T*)g;
+  A.H = (T*)H;
+  A.L0 = (const T*)t.spring_rest;
+  A.k = (T)t.spring_k;
+  A.xt = (const T*)t.inertia_xt;
+  A.w = (T)t.inertia_w;
+  A.mask = t.mask;
+  A.epart = energy ? L.epart : nullptr;
+  A.V = L.V;
+  A.s0 = L.s0;
+  A.wstage = (int)wstage_elems(L);
+  return A;
+}
+
+template <typename T, int DOF>
+cudaError_t dispatch_c(const RowsLaunch& L, const CArgs<T>& A, const ShardArgs<T>* S, bool full,
+                       double* energy, int nb, cudaStream_t s) {
+  const size_t smem = rows_smem_bytes(L);
+  cudaError_t e = L.s0 <= 6
+                      ? launch_c4<T, DOF, 6>(A, S, full, energy != nullptr, nb, smem, s, false)
+                      : launch_c4<T, DOF, kS0Max>(A, S, full, energy != nullptr, nb, smem, s,
+                                                  false);
+  if (e != cudaSuccess || !energy) return e;
+  k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+template <typename T, int DOF>
+cudaError_t rows_eval_compact_t(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
+                                void* H, double* energy, cudaStream_t s) {
+  const CArgs<T> A = make_cargs<T>(L, t, x, g, H, energy != nullptr);
+  return dispatch_c<T, DOF>(L, A, nullptr, t.flags & MAD_EVAL_FULL_STENCIL_AD, energy,
+                            rows_blocks(L.V), s);
+}
+
+template <typename T, int DOF>
+cudaError_t rows_eval_shard_t(const RowsLaunch& L, const mad_terms& t, int nranks,
+                              const int32_t* row_begin, int64_t block_lo,
+                              const void* const* x_parts, int rank, void* g, void* H,
+                              double* energy, cudaStream_t s) {
+  const int lo = row_begin[rank], hi = row_begin[rank + 1];
+  if (hi <= lo) return energy ? cudaMemsetAsync(energy, 0, sizeof(double), s) : cudaSuccess;
+  const CArgs<T> A = make_cargs<T>(L, t, nullptr, g, H, energy != nullptr);
+  ShardArgs<T> S{};
+  S.tile0 = lo / 32;
+  S.row_hi = hi;
+  S.own = rank;
+  S.nparts = nranks;
+  S.hoff = block_lo;
+  for (int r = 0; r <= nranks; ++r) S.rbeg[r] = row_begin[r];
+  for (int r = 0; r < nranks; ++r) S.xp[r] = (const T*)x_parts[r];
+  const int tiles = (hi - lo + 31) / 32;
+  const int nb = (tiles + kWarps - 1) / kWarps;
+  return dispatch_c<T, DOF>(L, A, &S, t.flags & MAD_EVAL_FULL_STENCIL_AD, energy, nb, s);
+}
+
+template <typename T, int DOF>
+cudaError_t rows_compact_limits_t(size_t bytes) {
+  CArgs<T> A{};
+  cudaError_t e = launch_c4<T, DOF, 6>(A, nullptr, false, false, 0, bytes, 0, true);
+  if (e != cudaSuccess) return e;
+  return launch_c4<T, DOF, kS0Max>(A, nullptr, false, false, 0, bytes, 0, true);
+}
+
+template cudaError_t rows_eval_compact_t<float, 2>(const RowsLaunch&, const mad_terms&, const void*,
+                                                   void*, void*, double*, cudaStream_t);
+template cudaError_t rows_eval_compact_t<float, 3>(const RowsLaunch&, const mad_terms&, const void*,
+                                                   void*, void*, double*, cudaStream_t);
+template cudaError_t rows_eval_compact_t<double, 2>(const RowsLaunch&, const mad_terms&,
+                                                    const void*, void*, void*, double*,
+                                                    cudaStream_t);
+template cudaError_t rows_eval_compact_t<double, 3>(const RowsLaunch&, const mad_terms&,
+                                                    const void*, void*, void*, double*,
+                                                    cudaStream_t);
+#define MAD_SHARD_INST(T, D)                                                                    \
+  template cudaError_t rows_eval_shard_t<T, D>(const RowsLaunch&, const mad_terms&, int,          \
+                                               const int32_t*, int64_t, const void* const*, int, \
+                                               void*, void*, double*, cudaStream_t);
+MAD_SHARD_INST(float, 2)
+MAD_SHARD_INST(float, 3)
+MAD_SHARD_INST(double, 2)
+MAD_SHARD_INST(double, 3)
+#undef MAD_SHARD_INST
+template cudaError_t rows_compact_limits_t<float, 2>(size_t);
+template cudaError_t rows_compact_limits_t<float, 3>(size_t);
+template cudaError_t rows_compact_limits_t<double, 2>(size_t);
+template cudaError_t rows_compact_limits_t<double, 3>(size_t);
+
+}  // namespace mad

@@ -159,6 +159,12 @@ typedef struct {
   int32_t max_patch_owned;
   int32_t smem_bytes;       /* dynamic shared memory of the assembly kernel  */
   int64_t device_bytes;     /* device memory the context holds               */
+  int32_t row_slot_bytes;   /* bytes per slot of the row tables that edge and
+                               vertex terms on the mesh pattern read: 4 when
+                               every column and edge id of a 32-row tile
+                               lies within 16 bits of the row and of the
+                               tile's first edge (bandwidth-ordered meshes),
+                               else 8                                        */
 } mad_info_t;
 
 /* Fill *o with the defaults listed in mad_opts. */
@@ -320,27 +326,93 @@ void mad_destroy(mad_ctx* c);
  * HOST struct as for mad_eval, and `energy` is a DEVICE double (out).
  *   springs  nE edges [nE][2] with t->spring_rest [nE] (e.g. mad_edges order)
  *   inertia  the V vertices with t->inertia_xt [V][dof]
- *   faces    nF faces F [nF][3] with t->face_Minv, t->face_area (dof 2)
+ *   faces    nF faces F [nF][3]: with dof 2, MAD_TERM_SYMDIR and/or
+ *            MAD_TERM_ARAP read t->face_Minv and t->face_area; with dof 3,
+ *            MAD_TERM_AREA reads t->face_area (A0) and t->area_k
  *   pairs    nP pairs [nP][2] with pair_rest [nP] and t->pair_k
  * Only the bits of t->mask select terms; t->flags is ignored.  No paper
  * counterpart: it is the energy reduction of mad_eval without a context.
+ * Indices: every vertex index of edges, F and pairs should lie in [0, V).  A
+ * term with an index outside it is skipped (nothing is read through that
+ * index) and makes the energy NaN, so bad input is visible in the result.
  * Memory: the per-block partial sums live in a fixed device array of this
  * library (65,536 doubles, held by every device that loads the library until
  * the process exits); nothing is allocated or freed.  The array is shared by
  * every call on a device and keeps the last call's values; each call writes
  * every slot it reads, so nothing needs clearing, but calls that overlap on
- * the GPU (different streams at once) race.  The first call on a device looks
- * up the array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.
- * Errors: MAD_ERR_INVALID_ARG (sizes, dtype, missing arrays),
- * MAD_ERR_UNIMPLEMENTED (faces with dof 3), MAD_ERR_CAPACITY (more than
- * 16,777,216 terms in total: the fixed array holds 65,536 sums of 256 terms),
- * MAD_ERR_CUDA.                                                            */
+ * the GPU (different streams at once) race.  Each call on a stream that is
+ * not being captured looks up the array's device address
+ * (cudaGetSymbolAddress); a call under stream capture reuses the address
+ * found by the last such call, so make one call before any capture, and
+ * again after a cudaDeviceReset.
+ * Errors: MAD_ERR_INVALID_ARG (sizes, dtype, missing arrays, unknown mask
+ * bits), MAD_ERR_UNIMPLEMENTED (MAD_TERM_SYMDIR or MAD_TERM_ARAP with dof
+ * other than 2, MAD_TERM_AREA with dof other than 3, any MAD_TERM_VF bit),
+ * MAD_ERR_CAPACITY (more than 16,777,216 terms in total: the fixed array
+ * holds 65,536 sums of 256 terms), MAD_ERR_CUDA.                           */
 mad_status mad_energy_noalloc(int32_t V, int32_t dof, mad_dtype dt, const void* x,
                               const mad_terms* t, int32_t nE, const int32_t* edges,
                               int32_t nF, const int32_t* F, int32_t nP,
                               const int32_t* pairs, const void* pair_rest,
                               double* energy, void* stream);
+
+/* ---- owner-computes sharding over several GPUs ---------------------------
+ * One mesh split across GPUs by Hessian rows (section 方法, key design 2,
+ * carried from patches to GPUs): each GPU owns a contiguous range of rows,
+ * evaluates every term that touches an owned vertex, and writes only its
+ * rows of g and H, so no reduction is needed; the only exchange is the
+ * positions of the vertices across its range's border (its halo), which
+ * the evaluation reads directly from their owners' buffers (peer device
+ * pointers, e.g. over NVLink).  Each GPU's Hessian values are the contiguous
+ * range [block_begin[r], block_begin[r+1]) of the mesh pattern's blocks.  */
+#define MAD_MAX_SHARDS 64
+
+/* Split the rows of the mesh pattern of (V, nF, F) into nranks contiguous
+ * ranges [row_begin[r], row_begin[r+1]), balanced by block count, every
+ * boundary a multiple of 32 rows (or V).  HOST only, no GPU needed.
+ *   F            HOST [nF][3] (as for mad_create)
+ *   row_begin    HOST int32 [nranks+1] (out); row_begin[0] = 0, [nranks] = V
+ *   block_begin  HOST int64 [nranks+1] (out, may be NULL): the mesh
+ *                pattern's row_ptr at each boundary
+ * Ranges may be empty when V is small.  Errors: MAD_ERR_INVALID_ARG (sizes,
+ * 1 <= nranks <= MAD_MAX_SHARDS, a bad face).                              */
+mad_status mad_shard_plan(int32_t V, int32_t nF, const int32_t* F, int32_t nranks,
+                          int32_t* row_begin, int64_t* block_begin);
+
+/* The halo of rows [row_lo, row_hi): every vertex outside the range that
+ * one of its rows couples to (the columns of its mesh-pattern rows outside
+ * the range), sorted.  HOST only.  *n_halo receives the count; halo (HOST
+ * int32 [cap]) receives the list when cap >= *n_halo (cap = 0 only counts;
+ * else MAD_ERR_CAPACITY).  Errors: MAD_ERR_INVALID_ARG.                     */
+mad_status mad_shard_halo(int32_t V, int32_t nF, const int32_t* F, int32_t row_lo,
+                          int32_t row_hi, int32_t* n_halo, int32_t* halo, int32_t cap);
+
+/* mad_eval for the rows of one shard.  c is a context of the whole mesh
+ * (same V and F on every GPU); the mesh pattern must be active (no pair
+ * set) and t->mask may hold MAD_TERM_SPRING and MAD_TERM_INERTIA only.
+ *   nranks, row_begin  HOST: a plan from mad_shard_plan (or any ranges
+ *                      with boundaries at multiples of 32 rows)
+ *   x_parts            HOST array of nranks DEVICE pointers: shard s's
+ *                      positions [row_begin[s+1] - row_begin[s]][dof] (the
+ *                      caller's own part and its peers' parts, readable
+ *                      from this device, e.g. peer memory over NVLink)
+ *   rank               the shard to evaluate
+ *   t                  as for mad_eval, arrays over the whole mesh
+ *                      (spring_rest [E], inertia_xt [V][dof])
+ *   g_part             DEVICE [rows of the shard][dof] (out)
+ *   H_part             DEVICE [block_begin[rank+1] - block_begin[rank]]
+ *                      [dof][dof] (out): the shard's blocks of the mesh
+ *                      pattern, in order
+ *   energy             DEVICE double (out) or NULL: the shard's share of
+ *                      the energy (the shares of all shards sum to E)
+ * Reads x_parts[s] only at the vertices of shard s in this shard's halo.
+ * The caller orders the peers' writes of their parts before this call
+ * (e.g. a barrier between steps).  Stream-ordered, no allocation.
+ * Errors: MAD_ERR_INVALID_ARG, MAD_ERR_UNIMPLEMENTED (other terms, active
+ * pairs, a mesh without compact row tables: see mad_info_t), MAD_ERR_CUDA. */
+mad_status mad_eval_shard(mad_ctx* c, int32_t nranks, const int32_t* row_begin,
+                          const void* const* x_parts, int32_t rank, const mad_terms* t,
+                          void* g_part, void* H_part, double* energy, void* stream);
 
 /* Self-test of the forward-mode number types on the device, used by the test
  * suite.  For each of n inputs (a, b) (HOST double [n][2]) it evaluates, in

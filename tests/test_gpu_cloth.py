@@ -62,31 +62,41 @@ def test_cloth_1000x1000_patch_staged(orc):
     check_cloth(orc, 1000, "float32", seed=1003, step=5, flags=PATCH)
 
 
-def test_permuted_vertex_numbering(orc):
+@pytest.mark.parametrize("n,dtype,slot_bytes", [(40, "float64", 4), (190, "float32", 8)])
+def test_permuted_vertex_numbering(orc, n, dtype, slot_bytes):
+    # A random numbering: at 40^2 every column and edge id of a tile still
+    # lies within 16 bits (compact row tables, irregular deltas); at 190^2
+    # (36,100 vertices) they do not, and the wide tables are used.
     import hessian_assembly_b200 as mad
-    n = 40
     st = mi.cloth_static(n, np.float64)
     V = st["V"]
     perm = np.random.default_rng(3).permutation(V)   # new id of old vertex
     inv = np.argsort(perm)
     F = perm[st["F"]].astype(np.int32)
     X = st["X"][inv]
-    ctx = mad.Context(V, F, 3, "float64", part_xyz=X)
+    ctx = mad.Context(V, F, 3, dtype, part_xyz=X)
+    assert ctx.info.row_slot_bytes == slot_bytes
     e = np.sort(perm[mi.grid_edges(n)], axis=1)
     edges = e[np.lexsort((e[:, 1], e[:, 0]))].astype(np.int32)
-    L0 = np.linalg.norm(X[edges[:, 0]] - X[edges[:, 1]], axis=1)
-    x = mi.cloth_x(n, 9, 0, np.float64)[inv]
-    xt = X.copy()
+    L0 = np.linalg.norm(X[edges[:, 0]] - X[edges[:, 1]], axis=1).astype(dtype)
+    x = mi.cloth_x(n, 9, 0, np.float64)[inv].astype(dtype)
+    xt = X.astype(dtype)
     terms = mad.Terms(mask=3, spring_rest=to_dev(L0), spring_k=st["k"], inertia_xt=to_dev(xt),
                       inertia_w=st["w"])
-    g, H, E = run_eval(ctx, x, terms, "float64")
+    g, H, E = run_eval(ctx, x, terms, dtype)
     rp, ci, nnzb = gpu_pattern(ctx)
     orp, oci = orc.pattern(V, F)
     np.testing.assert_array_equal(rp, orp)
     np.testing.assert_array_equal(ci, oci)
     og, oH, oE = orc.eval(V, 3, x, 3, orp, oci, edges=edges, L0=L0, k=st["k"], xt=xt, w=st["w"])
-    assert_close("g", g, og, "float64")
-    assert_close("H", H[:nnzb], oH, "float64")
+    assert_close("g", g, og, dtype)
+    assert_close("H", H[:nnzb], oH, dtype)
+
+
+def test_grid_uses_compact_row_tables():
+    ctx, _ = cloth_context(1000)
+    assert ctx.info.row_slot_bytes == 4
+    ctx.close()
 
 
 def test_deterministic_run_to_run():
