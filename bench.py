@@ -312,6 +312,9 @@ def rooflines(w, headline_ms, hbm, peak_kind):
         "cloth100_call": (cloth_bytes(100, 4), w.get("cloth100_eval_ms")),
         "cloth100_f64": (cloth_bytes(100, 8), w.get("cloth100_f64_eval_ms")),
         "cloth1000": (ALGO_BYTES, headline_ms),
+        "cloth1000_generic": (ALGO_BYTES, w.get("cloth1000_generic_eval_ms")),
+        "symdir500_generic_eval": (pe, w.get("symdir500_generic_eval_ms")),
+        "area1000_generic_eval": (ALGO_BYTES + 16 * F, w.get("area1000_generic_eval_ms")),
         "symdir500_eval": (pe, w.get("symdir500_eval_ms")),
         "symdir500_hvp": (ph, w.get("symdir500_hvp_ms")),
         "arap500_eval": (pe, w.get("arap500_eval_ms")),
@@ -428,7 +431,8 @@ def cpu_baseline(st):
             "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
 
 
-EXTRA = ("cloth_small", "symdir500", "pairs1000", "jac1000", "area1000", "vf1000")
+EXTRA = ("cloth_small", "generic1000", "symdir500", "pairs1000", "jac1000", "area1000", "vf1000")
+GENERIC_AD = 8  # MAD_EVAL_GENERIC_AD
 
 
 def extra_workloads(args, only=None):
@@ -484,6 +488,8 @@ def extra_workloads(args, only=None):
             res[f"cloth{n}_graph_eval_ms"] = round(timeit(graph.replay) / reps, 5)
             del graph
         ctx.close()
+    if run("generic1000"):
+        generic1000(res, mad, torch, dev, stream, timeit)
     # parameterization 500^2: eval and HVP
     if run("symdir500"):
         symdir500(res, mad, torch, dev, stream, timeit)
@@ -536,6 +542,27 @@ def vf1000(res, mad, torch, dev, stream, timeit):
     ctx.close()
 
 
+def generic1000(res, mad, torch, dev, stream, timeit):
+    """The headline step with MAD_EVAL_GENERIC_AD: the spring energy as a plain
+    expression, differentiated by the AD number types alone."""
+    st = mi.cloth_static(N_GRID, np.float32)
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    terms = mad.Terms(mask=3, flags=GENERIC_AD, spring_rest=torch.from_numpy(st["L0"]).to(dev),
+                      spring_k=st["k"], inertia_xt=torch.from_numpy(st["xt"]).to(dev),
+                      inertia_w=st["w"])
+    xs = [torch.from_numpy(mi.cloth_x(N_GRID, SEED, 40_000 + s, np.float32)).to(dev)
+          for s in range(4)]
+    g = torch.empty((st["V"], 3), device=dev)
+    H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
+    k = [0]
+
+    def step():
+        ctx.mad_eval(xs[k[0] % 4], terms, g, H, None, stream)
+        k[0] += 1
+    res["cloth1000_generic_eval_ms"] = round(timeit(step), 5)
+    ctx.close()
+
+
 def cloth_rest_area(st):
     X, F = st["X"], st["F"]
     return 0.5 * np.linalg.norm(np.cross(X[F[:, 1]] - X[F[:, 0]], X[F[:, 2]] - X[F[:, 0]]), axis=1)
@@ -569,6 +596,9 @@ def area1000(res, mad, torch, dev, stream, timeit):
     ms = timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream))
     res["area1000_hvp_ms"] = round(ms, 5)
     res["area1000_hvp_gbs"] = round(hb / (ms * 1e-3) / 1e9, 1)
+    terms.flags = GENERIC_AD
+    res["area1000_generic_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+    res["area1000_generic_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
     ctx.close()
 
 
@@ -608,6 +638,9 @@ def symdir500(res, mad, torch, dev, stream, timeit):
     H = torch.empty((ctx.info.capacity_blocks, 2, 2), device=dev)
     res["symdir500_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
     res["symdir500_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
+    tg = mad.Terms(mask=4, flags=GENERIC_AD, face_Minv=terms.face_Minv, face_area=terms.face_area)
+    res["symdir500_generic_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, tg, g, H, None, stream)), 5)
+    res["symdir500_generic_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, tg, v, y, stream)), 5)
     # the same term set through the patch-staged kernel, for comparison
     tp = mad.Terms(mask=4, flags=mad.MAD_EVAL_PATCH_STAGED, face_Minv=terms.face_Minv,
                    face_area=terms.face_area)

@@ -227,6 +227,7 @@ VfLaunch vf_launch(const mad_ctx* c, const mad_terms* t, const void* x) {
   L.rp = c->active < 0 ? c->pat.rp : c->buf[c->active].rp;
   L.ci = c->active < 0 ? c->pat.ci : c->buf[c->active].ci;
   L.status = c->status;
+  L.generic = (t->flags & MAD_EVAL_GENERIC_AD) != 0;
   return L;
 }
 
@@ -252,9 +253,14 @@ mad_status check_terms(mad_ctx* c, const mad_terms* t) {
     if (t->vf_n > 0 && (!t->vf || !t->vf_rest))
       return fail(c, MAD_ERR_INVALID_ARG, "vertex-face terms need vf and vf_rest");
   }
-  if (t->flags &
-      ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED))
+  if (t->flags & ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER |
+                             MAD_EVAL_PATCH_STAGED | MAD_EVAL_GENERIC_AD))
     return fail(c, MAD_ERR_INVALID_ARG, "unknown evaluation flags");
+  if ((t->flags & MAD_EVAL_GENERIC_AD) && (t->flags & MAD_EVAL_FULL_STENCIL_AD))
+    return fail(c, MAD_ERR_INVALID_ARG, "MAD_EVAL_GENERIC_AD with MAD_EVAL_FULL_STENCIL_AD");
+  if ((t->flags & MAD_EVAL_GENERIC_AD) &&
+      (t->flags & (MAD_EVAL_EDGE_SCATTER | MAD_EVAL_PATCH_STAGED)))
+    return fail(c, MAD_ERR_UNIMPLEMENTED, "MAD_EVAL_GENERIC_AD runs on the row kernel only");
   if ((t->mask & MAD_TERM_SPRING) && c->E > 0 && !t->spring_rest)
     return fail(c, MAD_ERR_INVALID_ARG, "spring term active but spring_rest is NULL");
   if ((t->mask & MAD_TERM_INERTIA) && c->V > 0 && !t->inertia_xt)

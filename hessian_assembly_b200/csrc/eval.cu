@@ -568,10 +568,10 @@ __device__ __forceinline__ void mv_add(T* y, const T* Hblk, const T* vv) {
 }
 
 // y_a += H_aa v_a + H_ab v_b for one edge term seen from endpoint a
-template <typename T, int DOF, bool FULL>
-__device__ __forceinline__ void edge_hv(const EdgeRes<T, DOF, FULL>& R, const T* va, const T* vb,
+template <typename T, int DOF, int AD>
+__device__ __forceinline__ void edge_hv(const EdgeRes<T, DOF, AD>& R, const T* va, const T* vb,
                                         T* y) {
-  if constexpr (!FULL) {
+  if constexpr (AD != kAdFull) {
     T dv[DOF];
 #pragma unroll
     for (int a = 0; a < DOF; ++a) dv[a] = va[a] - vb[a];

@@ -167,6 +167,7 @@ struct VfLaunch {
   const int32_t* rp = nullptr;
   const int32_t* ci = nullptr;
   int32_t* status = nullptr;
+  bool generic = false;  // the energy as a plain expression (MAD_EVAL_GENERIC_AD)
 };
 cudaError_t launch_vf_eval(int dtype, const VfLaunch& L, void* g, void* H, double* energy,
                            cudaStream_t s);

@@ -66,7 +66,13 @@ __device__ __forceinline__ const T* shard_x(const ShardArgs<T>& S, int v) {
 // the L2 to fetch before it starts (0: none).  Tiles run in about index
 // order, so tile t + D starts roughly D / (resident warps) waves later.
 #ifndef MAD_ROWSC_PREFETCH_TILES
-#define MAD_ROWSC_PREFETCH_TILES 0
+#define MAD_ROWSC_PREFETCH_TILES 512
+#endif
+// Also ask for the later tile's rest lengths of the edges above its rows
+// (their ids start at that tile's first edge id, read at the start and used
+// once this tile's terms are done).
+#ifndef MAD_ROWSC_PREFETCH_L0
+#define MAD_ROWSC_PREFETCH_L0 0
 #endif
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
@@ -76,7 +82,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 __device__ __forceinline__ int slot_dcol(uint32_t w) { return (int)(int16_t)(w & 0xFFFFu); }
 __device__ __forceinline__ int slot_deid(uint32_t w) { return (int)(int16_t)(w >> 16); }
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, bool SHARD>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, bool SHARD>
 __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T>* S) {
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
@@ -114,6 +120,15 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
 
   int4 th = make_int4(0, 0, 0, 0);
   if (tile_live) th = A.ctile[tile];
+  constexpr bool kPfL0 = MAD_ROWSC_PREFETCH_TILES > 0 && MAD_ROWSC_PREFETCH_L0 && !SHARD;
+  int pf_e0 = -1, pf_e1 = -1;  // the later tile's first edge id and the next tile's
+  if constexpr (kPfL0) {
+    const int tp = tile + MAD_ROWSC_PREFETCH_TILES;
+    if (lane == 24 && (tp + 1) * 32 < A.V && springs) {
+      pf_e0 = A.ctile[tp].y;
+      pf_e1 = A.ctile[tp + 1].y;
+    }
+  }
   uint32_t sw[S0];
 #pragma unroll
   for (int k = 0; k < S0; ++k) {
@@ -191,8 +206,8 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
 #pragma unroll
       for (int k = 0; k < S0; ++k) {
         if (sw[k] == 0u) continue;
-        EdgeRes<T, DOF, FULL> R;
-        eval_edge_res<T, DOF, FULL>(xi, xb[k], l0[k], A.k, R);
+        EdgeRes<T, DOF, AD> R;
+        eval_edge_res<T, DOF, AD>(xi, xb[k], l0[k], A.k, R);
         // block position: the slots before it plus the diagonal when the
         // column lies above the row
         const int p = k + (slot_dcol(sw[k]) > 0);
@@ -205,8 +220,8 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
         T xo[DOF];
 #pragma unroll
         for (int a = 0; a < DOF; ++a) xo[a] = xs[a];
-        EdgeRes<T, DOF, FULL> R;
-        eval_edge_res<T, DOF, FULL>(xi, xo, A.L0[e.y], A.k, R);
+        EdgeRes<T, DOF, AD> R;
+        eval_edge_res<T, DOF, AD>(xi, xo, A.L0[e.y], A.k, R);
         const int p = A.s0 + q + (e.x > i);
         apply_edge_side<true>(R, 0, acc, row + p * B, gr);
         if (ENERGY) energy += 0.5 * (double)edge_energy(R);
@@ -223,6 +238,10 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
         d[a * DOF + b] = a <= b ? acc[Tri<DOF>::idx(a, b)] : acc[Tri<DOF>::idx(b, a)];
 #pragma unroll
     for (int a = 0; a < DOF; ++a) A.g[(uint32_t)((i - goff) * DOF + a)] = gr[a];
+  }
+  if constexpr (kPfL0) {
+    if (pf_e0 >= 0)
+      for (int e = pf_e0; e < pf_e1; e += 128 / (int)sizeof(T)) prefetch_l2(A.L0 + e);
   }
   // ---- write-back of the warp's staged rows (a prefix of its 32 rows) ------
   fence_async_smem();
@@ -251,16 +270,16 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
   if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
 }
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+template <typename T, int DOF, int AD, bool ENERGY, int S0>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, false>())
     k_rows_eval_c(const CArgs<T> A) {
-  rows_c_body<T, DOF, FULL, ENERGY, S0, false>(A, nullptr);
+  rows_c_body<T, DOF, AD, ENERGY, S0, false>(A, nullptr);
 }
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+template <typename T, int DOF, int AD, bool ENERGY, int S0>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, false>())
     k_rows_eval_cs(const CArgs<T> A, const __grid_constant__ ShardArgs<T> S) {
-  rows_c_body<T, DOF, FULL, ENERGY, S0, true>(A, &S);
+  rows_c_body<T, DOF, AD, ENERGY, S0, true>(A, &S);
 }
 
 // Shared-memory carve-out asked for the kernel, in percent of the unified
@@ -270,12 +289,12 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, false>())
 #define MAD_ROWSC_CARVEOUT -1
 #endif
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0>
+template <typename T, int DOF, int AD, bool ENERGY, int S0>
 cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, int nb, size_t smem,
                      cudaStream_t s, bool set) {
   if (set) {
-    const void* ks[2] = {(const void*)k_rows_eval_c<T, DOF, FULL, ENERGY, S0>,
-                         (const void*)k_rows_eval_cs<T, DOF, FULL, ENERGY, S0>};
+    const void* ks[2] = {(const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0>,
+                         (const void*)k_rows_eval_cs<T, DOF, AD, ENERGY, S0>};
     for (const void* k : ks) {
       cudaError_t e;
       if (MAD_ROWSC_CARVEOUT >= 0) {
@@ -289,26 +308,32 @@ cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, int nb, size_t sm
     return cudaSuccess;
   }
   if (S)
-    k_rows_eval_cs<T, DOF, FULL, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A, *S);
+    k_rows_eval_cs<T, DOF, AD, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A, *S);
   else
-    k_rows_eval_c<T, DOF, FULL, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A);
+    k_rows_eval_c<T, DOF, AD, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A);
   return cudaGetLastError();
 }
 
 template <typename T, int DOF, int S0>
-cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, bool full, bool energy, int nb,
+cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, int ad, bool energy, int nb,
                       size_t smem, cudaStream_t s, bool set) {
   if (set) {
-    cudaError_t e;
-    if ((e = launch_c<T, DOF, true, true, S0>(A, S, nb, smem, s, true)) != cudaSuccess) return e;
-    if ((e = launch_c<T, DOF, true, false, S0>(A, S, nb, smem, s, true)) != cudaSuccess) return e;
-    if ((e = launch_c<T, DOF, false, true, S0>(A, S, nb, smem, s, true)) != cudaSuccess) return e;
-    return launch_c<T, DOF, false, false, S0>(A, S, nb, smem, s, true);
+    for (int a : {kAdReduced, kAdFull, kAdGeneric}) {
+      const cudaError_t e = with_ad(a, [&](auto adc) {
+        constexpr int AD = decltype(adc)::value;
+        const cudaError_t e1 = launch_c<T, DOF, AD, true, S0>(A, S, nb, smem, s, true);
+        if (e1 != cudaSuccess) return e1;
+        return launch_c<T, DOF, AD, false, S0>(A, S, nb, smem, s, true);
+      });
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
   }
-  if (full && energy) return launch_c<T, DOF, true, true, S0>(A, S, nb, smem, s, false);
-  if (full) return launch_c<T, DOF, true, false, S0>(A, S, nb, smem, s, false);
-  if (energy) return launch_c<T, DOF, false, true, S0>(A, S, nb, smem, s, false);
-  return launch_c<T, DOF, false, false, S0>(A, S, nb, smem, s, false);
+  return with_ad(ad, [&](auto adc) {
+    constexpr int AD = decltype(adc)::value;
+    if (energy) return launch_c<T, DOF, AD, true, S0>(A, S, nb, smem, s, false);
+    return launch_c<T, DOF, AD, false, S0>(A, S, nb, smem, s, false);
+  });
 }
 
 template <typename T>
@@ -335,12 +360,12 @@ CArgs<T> make_cargs(const RowsLaunch& L, const mad_terms& t, const void* x, void
 }
 
 template <typename T, int DOF>
-cudaError_t dispatch_c(const RowsLaunch& L, const CArgs<T>& A, const ShardArgs<T>* S, bool full,
+cudaError_t dispatch_c(const RowsLaunch& L, const CArgs<T>& A, const ShardArgs<T>* S, int ad,
                        double* energy, int nb, cudaStream_t s) {
   const size_t smem = rows_smem_bytes(L);
   cudaError_t e = L.s0 <= 6
-                      ? launch_c4<T, DOF, 6>(A, S, full, energy != nullptr, nb, smem, s, false)
-                      : launch_c4<T, DOF, kS0Max>(A, S, full, energy != nullptr, nb, smem, s,
+                      ? launch_c4<T, DOF, 6>(A, S, ad, energy != nullptr, nb, smem, s, false)
+                      : launch_c4<T, DOF, kS0Max>(A, S, ad, energy != nullptr, nb, smem, s,
                                                   false);
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
@@ -353,7 +378,7 @@ template <typename T, int DOF>
 cudaError_t rows_eval_compact_t(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
                                 void* H, double* energy, cudaStream_t s) {
   const CArgs<T> A = make_cargs<T>(L, t, x, g, H, energy != nullptr);
-  return dispatch_c<T, DOF>(L, A, nullptr, t.flags & MAD_EVAL_FULL_STENCIL_AD, energy,
+  return dispatch_c<T, DOF>(L, A, nullptr, ad_form(t.flags), energy,
                             rows_blocks(L.V), s);
 }
 
@@ -375,15 +400,15 @@ cudaError_t rows_eval_shard_t(const RowsLaunch& L, const mad_terms& t, int nrank
   for (int r = 0; r < nranks; ++r) S.xp[r] = (const T*)x_parts[r];
   const int tiles = (hi - lo + 31) / 32;
   const int nb = (tiles + kWarps - 1) / kWarps;
-  return dispatch_c<T, DOF>(L, A, &S, t.flags & MAD_EVAL_FULL_STENCIL_AD, energy, nb, s);
+  return dispatch_c<T, DOF>(L, A, &S, ad_form(t.flags), energy, nb, s);
 }
 
 template <typename T, int DOF>
 cudaError_t rows_compact_limits_t(size_t bytes) {
   CArgs<T> A{};
-  cudaError_t e = launch_c4<T, DOF, 6>(A, nullptr, false, false, 0, bytes, 0, true);
+  cudaError_t e = launch_c4<T, DOF, 6>(A, nullptr, kAdReduced, false, 0, bytes, 0, true);
   if (e != cudaSuccess) return e;
-  return launch_c4<T, DOF, kS0Max>(A, nullptr, false, false, 0, bytes, 0, true);
+  return launch_c4<T, DOF, kS0Max>(A, nullptr, kAdReduced, false, 0, bytes, 0, true);
 }
 
 template cudaError_t rows_eval_compact_t<float, 2>(const RowsLaunch&, const mad_terms&, const void*,

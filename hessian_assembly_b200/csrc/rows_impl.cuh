@@ -158,7 +158,7 @@ __device__ __forceinline__ void block_energy(double e, double* out) {
 // Calls on_term(R, p, col) for every edge term (i, col) of row i, where p is
 // the block position of column col in the mesh-pattern row.
 // S0 (compile time) >= the slot table's row width A.s0.
-template <typename T, int DOF, bool FULL, int S0, typename OnTerm>
+template <typename T, int DOF, int AD, int S0, typename OnTerm>
 __device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, int lane,
                                           uint32_t m, const T* xi, OnTerm on_term) {
   const int noff = (int)(m & 0xFFFFu), dpos = (int)(m >> 16);
@@ -180,8 +180,8 @@ __device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, in
 #pragma unroll
   for (int k = 0; k < S0; ++k) {
     if (sl[k].x < 0) continue;
-    EdgeRes<T, DOF, FULL> R;
-    eval_edge_res<T, DOF, FULL>(xi, xb[k], l0[k], A.k, R);
+    EdgeRes<T, DOF, AD> R;
+    eval_edge_res<T, DOF, AD>(xi, xb[k], l0[k], A.k, R);
     on_term(R, k < dpos ? k : k + 1, sl[k].x);
   }
   if (noff > A.s0) {  // rows longer than the slot table: the overflow slots
@@ -191,8 +191,8 @@ __device__ __forceinline__ void row_edges(const RArgs<T>& A, int i, int tile, in
       T xo[DOF];
 #pragma unroll
       for (int a = 0; a < DOF; ++a) xo[a] = A.x[(uint32_t)(e.x * DOF + a)];
-      EdgeRes<T, DOF, FULL> R;
-      eval_edge_res<T, DOF, FULL>(xi, xo, A.L0[e.y], A.k, R);
+      EdgeRes<T, DOF, AD> R;
+      eval_edge_res<T, DOF, AD>(xi, xo, A.L0[e.y], A.k, R);
       on_term(R, k < dpos ? k : k + 1, e.x);
     }
   }
@@ -325,7 +325,7 @@ __device__ __forceinline__ void add4(T* b, const T* v) {
 
 // The work of one row, writing the row's blocks through `row` (a shared-memory
 // staging slot or, for rows that do not fit, the row's place in H).
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES, bool PAIRS>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, int FACES, bool PAIRS>
 __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile, int lane,
                                               uint32_t m, int d0, int d1, int pb, int pn,
                                               const T* xi, const T* xti, T* row, double& energy) {
@@ -387,8 +387,8 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   }
   if constexpr (S0 > 0) {  // S0 == 0: an instantiation without edge terms
     if (springs) {
-      row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
-                              [&](const EdgeRes<T, DOF, FULL>& R, int p, int) {
+      row_edges<T, DOF, AD, S0>(A, i, tile, lane, m, xi,
+                              [&](const EdgeRes<T, DOF, AD>& R, int p, int) {
                                 const int op =
                                     !PAIRS || nins == 0 ? p : row_pos_new(rn, A.pe_pos, pb, pn, nins, p);
                                 apply_edge_side<true>(R, 0, acc, row + op * B, gr);
@@ -402,7 +402,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
       row_faces3<T>(A, i, tile, lane,
                     [&](const T* xj, const T* xk, int, int pj, int pk, T A0) {
                       FaceRow3<T> o;
-                      eval_area_row<T, FULL>(xi, xj, xk, A0, A.ka, o);
+                      eval_area_row<T, AD>(xi, xj, xk, A0, A.ka, o);
 #pragma unroll
                       for (int a = 0; a < 3; ++a)
 #pragma unroll
@@ -426,7 +426,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                      [&](const T* xj, const T* xk, int, int, int c, int pj, int pk, const T* M,
                          T ar) {
                        FaceRow<T> o;
-                       eval_symdir_row<T, FULL, KIND>(xi, xj, xk, c, M, ar, o);
+                       eval_symdir_row<T, AD, KIND>(xi, xj, xk, c, M, ar, o);
                        acc[0] += o.H[0][0];
                        acc[1] += o.H[0][1];
                        acc[2] += o.H[0][3];
@@ -463,8 +463,8 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
 #pragma unroll
         for (int a = 0; a < DOF; ++a) xj[a] = A.x[(uint32_t)(j * DOF + a)];
       }
-      EdgeRes<T, DOF, FULL> Rp;
-      eval_edge_res<T, DOF, FULL>(xi, xj, rest, A.kp, Rp);
+      EdgeRes<T, DOF, AD> Rp;
+      eval_edge_res<T, DOF, AD>(xi, xj, rest, A.kp, Rp);
       apply_edge_side<false>(Rp, 0, acc, row + (pw & kPairPosMask) * B, gr);
       if (ENERGY) energy += 0.5 * (double)edge_energy(Rp);
     }
@@ -480,7 +480,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   for (int a = 0; a < DOF; ++a) A.g[(uint32_t)(i * DOF + a)] = gr[a];
 }
 
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES, bool PAIRS>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, int FACES, bool PAIRS>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, (FACES != 0)>()) k_rows_eval(const RArgs<T> A) {
   constexpr int B = DOF * DOF;
   constexpr int VEC = 16 / (int)sizeof(T);
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, (FACES != 0)>(
   const bool staged = has && off + (d1 - d0) * B <= A.wstage;
   // rows that do not fit their warp's slice are assembled in place in H
   if (has)
-    rows_eval_row<T, DOF, FULL, ENERGY, S0, FACES, PAIRS>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
+    rows_eval_row<T, DOF, AD, ENERGY, S0, FACES, PAIRS>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
                                         staged ? stage + off : A.H + (uint32_t)(d0 * B), energy);
   // ---- write-back of the warp's staged rows (a prefix of its 32 rows) -------
   fence_async_smem();
@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, (FACES != 0)>(
   if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
 }
 
-template <typename T, int DOF, bool FULL, int S0, bool FACES>
+template <typename T, int DOF, int AD, int S0, bool FACES>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_hvp(const RArgs<T> A) {
   constexpr int TD = Tri<DOF>::size;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -584,8 +584,8 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
 #pragma unroll
       for (int b = 0; b < DOF; ++b) yr[a] += Hi[a * DOF + b] * vi[b];
   }
-  auto hv = [&](const EdgeRes<T, DOF, FULL>& R, const T* vj) {
-    if constexpr (!FULL) {
+  auto hv = [&](const EdgeRes<T, DOF, AD>& R, const T* vj) {
+    if constexpr (AD != kAdFull) {
 #pragma unroll
       for (int a = 0; a < DOF; ++a) {
         T s = T(0);
@@ -604,8 +604,8 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   };
   if constexpr (S0 > 0) {
     if (A.mask & MAD_TERM_SPRING) {
-      row_edges<T, DOF, FULL, S0>(A, i, tile, lane, m, xi,
-                              [&](const EdgeRes<T, DOF, FULL>& R, int, int col) {
+      row_edges<T, DOF, AD, S0>(A, i, tile, lane, m, xi,
+                              [&](const EdgeRes<T, DOF, AD>& R, int, int col) {
                                 T vj[DOF];
 #pragma unroll
                                 for (int a = 0; a < DOF; ++a) vj[a] = A.v[(uint32_t)(col * DOF + a)];
@@ -648,8 +648,8 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
         xj[a] = A.x[(uint32_t)(j * DOF + a)];
         vj[a] = A.v[(uint32_t)(j * DOF + a)];
       }
-      EdgeRes<T, DOF, FULL> Rp;
-      eval_edge_res<T, DOF, FULL>(xi, xj, A.pe_rest[e], A.kp, Rp);
+      EdgeRes<T, DOF, AD> Rp;
+      eval_edge_res<T, DOF, AD>(xi, xj, A.pe_rest[e], A.kp, Rp);
       hv(Rp, vj);
     }
   }
@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
 
 // Per-face pass of the Hessian-vector product for area-preservation faces
 // (dof 3): one thread per face writes (H_f v_f) for its three corners.
-template <typename T, bool FULL>
+template <typename T, int AD>
 __global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __restrict__ F,
                                                       const T* __restrict__ x,
                                                       const T* __restrict__ v,
@@ -679,7 +679,7 @@ __global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __r
     }
   }
   T o[9];
-  hv_area_face<T, FULL>(u[0], u[1], u[2], w[0], w[1], w[2], area[f], ka, o);
+  hv_area_face<T, AD>(u[0], u[1], u[2], w[0], w[1], w[2], area[f], ka, o);
 #pragma unroll
   for (int q = 0; q < 9; ++q) out[9 * f + q] = o[q];
 }
@@ -688,7 +688,7 @@ __global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __r
 // (H_f v_f) for its three corners once; the row kernel then adds, for each
 // row, its corners' results.  Each face is differentiated once instead of
 // once per corner, and no atomics are needed.
-template <typename T, bool FULL>
+template <typename T, int AD>
 __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_t* __restrict__ F,
                                                  const T* __restrict__ x, const T* __restrict__ v,
                                                  const T* __restrict__ Minv,
@@ -724,7 +724,7 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
   load4<T>(Minv + 4 * f, M);
   T o[6];
   with_face2_kind(kind, [&](auto kc) {
-    hv_symdir_face<T, FULL, decltype(kc)::value>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f],
+    hv_symdir_face<T, AD, decltype(kc)::value>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f],
                                                  o);
   });
 #pragma unroll
@@ -791,42 +791,56 @@ __global__ void k_energy_sum_rows(const double* __restrict__ part, int n, double
 // One instantiation of the assembly kernel, chosen by whether the active
 // pattern holds pair blocks; also sets (or, with set, only sets) its shared
 // memory limit.
-template <typename T, int DOF, bool FULL, bool ENERGY, int S0, int FACES>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, int FACES>
 cudaError_t eval_k(const RArgs<T>& A, bool pairs, int nb, size_t smem, cudaStream_t s,
                    bool set = false) {
-  const void* kp = (const void*)k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, true>;
-  const void* kn = (const void*)k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, false>;
+  const void* kp = (const void*)k_rows_eval<T, DOF, AD, ENERGY, S0, FACES, true>;
+  const void* kn = (const void*)k_rows_eval<T, DOF, AD, ENERGY, S0, FACES, false>;
   if (set) {
     cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   }
   if (pairs)
-    k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, true><<<nb, kRowThreads, smem, s>>>(A);
+    k_rows_eval<T, DOF, AD, ENERGY, S0, FACES, true><<<nb, kRowThreads, smem, s>>>(A);
   else
-    k_rows_eval<T, DOF, FULL, ENERGY, S0, FACES, false><<<nb, kRowThreads, smem, s>>>(A);
+    k_rows_eval<T, DOF, AD, ENERGY, S0, FACES, false><<<nb, kRowThreads, smem, s>>>(A);
   return cudaGetLastError();
 }
 
-// Every (FULL, ENERGY) instantiation for one S0 and FACES.  FACES: 0 no face
+// calls f(std::integral_constant<int, AD>) for the run-time AD form
+template <typename F>
+cudaError_t with_ad(int ad, F&& f) {
+  if (ad == kAdFull) return f(std::integral_constant<int, kAdFull>{});
+  if (ad == kAdGeneric) return f(std::integral_constant<int, kAdGeneric>{});
+  return f(std::integral_constant<int, kAdReduced>{});
+}
+
+// Every (AD, ENERGY) instantiation for one S0 and FACES.  FACES: 0 no face
 // terms; 1 the face term of the dof (symmetric Dirichlet for dof 2, area
 // preservation for dof 3); 2 (dof 2) ARAP alone or with symmetric Dirichlet,
 // an instantiation of its own so that the symmetric Dirichlet kernel keeps
 // its register budget.
 template <typename T, int DOF, int S0, int FACES>
-cudaError_t eval_k4(const RArgs<T>& A, bool full, bool energy, bool pairs, int nb, size_t smem,
+cudaError_t eval_k4(const RArgs<T>& A, int ad, bool energy, bool pairs, int nb, size_t smem,
                     cudaStream_t s, bool set = false) {
   if (set) {
-    cudaError_t e;
-    if ((e = eval_k<T, DOF, true, true, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
-    if ((e = eval_k<T, DOF, true, false, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
-    if ((e = eval_k<T, DOF, false, true, S0, FACES>(A, pairs, nb, smem, s, true)) != cudaSuccess) return e;
-    return eval_k<T, DOF, false, false, S0, FACES>(A, pairs, nb, smem, s, true);
+    for (int a : {kAdReduced, kAdFull, kAdGeneric}) {
+      const cudaError_t e = with_ad(a, [&](auto adc) {
+        constexpr int AD = decltype(adc)::value;
+        const cudaError_t e1 = eval_k<T, DOF, AD, true, S0, FACES>(A, pairs, nb, smem, s, true);
+        if (e1 != cudaSuccess) return e1;
+        return eval_k<T, DOF, AD, false, S0, FACES>(A, pairs, nb, smem, s, true);
+      });
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
   }
-  if (full && energy) return eval_k<T, DOF, true, true, S0, FACES>(A, pairs, nb, smem, s);
-  if (full) return eval_k<T, DOF, true, false, S0, FACES>(A, pairs, nb, smem, s);
-  if (energy) return eval_k<T, DOF, false, true, S0, FACES>(A, pairs, nb, smem, s);
-  return eval_k<T, DOF, false, false, S0, FACES>(A, pairs, nb, smem, s);
+  return with_ad(ad, [&](auto adc) {
+    constexpr int AD = decltype(adc)::value;
+    if (energy) return eval_k<T, DOF, AD, true, S0, FACES>(A, pairs, nb, smem, s);
+    return eval_k<T, DOF, AD, false, S0, FACES>(A, pairs, nb, smem, s);
+  });
 }
 
 template <typename T, int DOF>
@@ -835,7 +849,7 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   RArgs<T> A = make_rargs<T>(L, t, x, nullptr, g, H, nullptr, energy != nullptr);
   const int nb = rows_blocks(L.V);
   const size_t smem = rows_smem_bytes(L);
-  const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
+  const int ad = ad_form(t.flags);
   const bool pairs = L.prow != nullptr;
   const bool en = energy != nullptr;
   cudaError_t e;
@@ -846,9 +860,9 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
     auto faces_k = [&](auto s0c) {
       constexpr int S0F = decltype(s0c)::value;
       if constexpr (DOF == 2) {
-        if (t.mask & MAD_TERM_ARAP) return eval_k4<T, DOF, S0F, 2>(A, full, en, pairs, nb, smem, s);
+        if (t.mask & MAD_TERM_ARAP) return eval_k4<T, DOF, S0F, 2>(A, ad, en, pairs, nb, smem, s);
       }
-      return eval_k4<T, DOF, S0F, 1>(A, full, en, pairs, nb, smem, s);
+      return eval_k4<T, DOF, S0F, 1>(A, ad, en, pairs, nb, smem, s);
     };
     if (t.mask & MAD_TERM_SPRING)
       e = faces_k(std::integral_constant<int, kS0Max>{});
@@ -860,9 +874,9 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   } else if (L.s0 <= 6) {
     // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
     // narrower instantiation: fewer registers
-    e = eval_k4<T, DOF, 6, 0>(A, full, en, pairs, nb, smem, s);
+    e = eval_k4<T, DOF, 6, 0>(A, ad, en, pairs, nb, smem, s);
   } else {
-    e = eval_k4<T, DOF, kS0Max, 0>(A, full, en, pairs, nb, smem, s);
+    e = eval_k4<T, DOF, kS0Max, 0>(A, ad, en, pairs, nb, smem, s);
   }
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
@@ -874,75 +888,47 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
                          void* y, cudaStream_t s) {
   RArgs<T> A = make_rargs<T>(L, t, x, v, nullptr, nullptr, y, false);
   const int nb = rows_blocks(L.V);
-  const bool full = t.flags & MAD_EVAL_FULL_STENCIL_AD;
-  if constexpr (DOF == 2) {
-    if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
-      const int kind = face2_kind(t.mask);
-      if (L.nF > 0) {
-        const unsigned nbf = (unsigned)((L.nF + 255) / 256);
-        const bool vec2 = ((((uintptr_t)x) | ((uintptr_t)v)) % (2 * sizeof(T))) == 0;
-        if (full)
-          k_face_hv<T, true><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
-                                                 (const T*)t.face_Minv, (const T*)t.face_area,
-                                                 (T*)L.fhv, kind);
-        else
-          k_face_hv<T, false><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
-                                                  (const T*)t.face_Minv, (const T*)t.face_area,
-                                                  (T*)L.fhv, kind);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-      }
-      const bool sp = t.mask & MAD_TERM_SPRING;
-      if (sp && full)
-        k_rows_hvp<T, DOF, true, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (sp)
-        k_rows_hvp<T, DOF, false, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (full)
-        k_rows_hvp<T, DOF, true, 0, true><<<nb, kRowThreads, 0, s>>>(A);
-      else
-        k_rows_hvp<T, DOF, false, 0, true><<<nb, kRowThreads, 0, s>>>(A);
+  return with_ad(ad_form(t.flags), [&](auto adc) -> cudaError_t {
+    constexpr int AD = decltype(adc)::value;
+    const bool sp = t.mask & MAD_TERM_SPRING;
+    // the row pass after a per-face pass (face terms), or alone
+    auto rows = [&](auto facesc) {
+      constexpr bool FC = decltype(facesc)::value;
+      if (sp) k_rows_hvp<T, DOF, AD, kS0Max, FC><<<nb, kRowThreads, 0, s>>>(A);
+      else k_rows_hvp<T, DOF, AD, 0, FC><<<nb, kRowThreads, 0, s>>>(A);
       return cudaGetLastError();
-    }
-  }
-  if constexpr (DOF == 3) {
-    if (t.mask & MAD_TERM_AREA) {
-      if (L.nF > 0) {
-        const unsigned nbf = (unsigned)((L.nF + 255) / 256);
-        if (full)
-          k_face_hv_area<T, true><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
-                                                      (const T*)t.face_area, (T)t.area_k,
-                                                      (T*)L.fhv);
-        else
-          k_face_hv_area<T, false><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
-                                                       (const T*)t.face_area, (T)t.area_k,
-                                                       (T*)L.fhv);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+    };
+    if constexpr (DOF == 2) {
+      if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
+        if (L.nF > 0) {
+          const unsigned nbf = (unsigned)((L.nF + 255) / 256);
+          const bool vec2 = ((((uintptr_t)x) | ((uintptr_t)v)) % (2 * sizeof(T))) == 0;
+          k_face_hv<T, AD><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
+                                               (const T*)t.face_Minv, (const T*)t.face_area,
+                                               (T*)L.fhv, face2_kind(t.mask));
+          const cudaError_t e = cudaGetLastError();
+          if (e != cudaSuccess) return e;
+        }
+        return rows(std::true_type{});
       }
-      const bool sp = t.mask & MAD_TERM_SPRING;
-      if (sp && full)
-        k_rows_hvp<T, DOF, true, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (sp)
-        k_rows_hvp<T, DOF, false, kS0Max, true><<<nb, kRowThreads, 0, s>>>(A);
-      else if (full)
-        k_rows_hvp<T, DOF, true, 0, true><<<nb, kRowThreads, 0, s>>>(A);
-      else
-        k_rows_hvp<T, DOF, false, 0, true><<<nb, kRowThreads, 0, s>>>(A);
-      return cudaGetLastError();
     }
-  }
-  if (L.s0 <= 6) {
-    if (full)
-      k_rows_hvp<T, DOF, true, 6, false><<<nb, kRowThreads, 0, s>>>(A);
-    else
-      k_rows_hvp<T, DOF, false, 6, false><<<nb, kRowThreads, 0, s>>>(A);
-  } else {
-    if (full)
-      k_rows_hvp<T, DOF, true, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
-    else
-      k_rows_hvp<T, DOF, false, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
-  }
-  return cudaGetLastError();
+    if constexpr (DOF == 3) {
+      if (t.mask & MAD_TERM_AREA) {
+        if (L.nF > 0) {
+          const unsigned nbf = (unsigned)((L.nF + 255) / 256);
+          k_face_hv_area<T, AD><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
+                                                    (const T*)t.face_area, (T)t.area_k,
+                                                    (T*)L.fhv);
+          const cudaError_t e = cudaGetLastError();
+          if (e != cudaSuccess) return e;
+        }
+        return rows(std::true_type{});
+      }
+    }
+    if (L.s0 <= 6) k_rows_hvp<T, DOF, AD, 6, false><<<nb, kRowThreads, 0, s>>>(A);
+    else k_rows_hvp<T, DOF, AD, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
+    return cudaGetLastError();
+  });
 }
 
 template <typename T, int DOF>

@@ -235,6 +235,71 @@ __device__ __forceinline__ SHD<T, N, G, (H | outer_mask<N>(G, G))> chain(
   return r;
 }
 
+// ---- elementary functions and scalar operations ----------------------------
+// sqrt and 1/x as chain-rule steps with their own first and second
+// derivatives, as for the dense numbers (dual.cuh); -a and a + c, a - c.
+template <typename T, int N, uint32_t G, uint64_t H>
+__device__ __forceinline__ auto sqrt(const SHD<T, N, G, H>& a) {
+  const T f0 = ::sqrt(a.v);
+  const T r0 = T(1) / f0;
+  return chain(a, f0, T(0.5) * r0, T(-0.25) * r0 * r0 * r0);
+}
+
+template <typename T, int N, uint32_t G, uint64_t H>
+__device__ __forceinline__ auto inv(const SHD<T, N, G, H>& a) {
+  const T f0 = T(1) / a.v;
+  const T f1 = -f0 * f0;
+  return chain(a, f0, f1, T(-2) * f1 * f0);
+}
+
+template <typename T, int N, uint32_t G, uint64_t H>
+__device__ __forceinline__ SHD<T, N, G, H> operator-(const SHD<T, N, G, H>& a) {
+  SHD<T, N, G, H> r;
+  r.v = -a.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (mbit(G, i)) r.g[i] = -a.g[i];
+#pragma unroll
+  for (int q = 0; q < Tri<N>::size; ++q)
+    if (mbit(H, q)) r.h[q] = -a.h[q];
+  return r;
+}
+
+template <typename T, int N, uint32_t G, uint64_t H>
+__device__ __forceinline__ SHD<T, N, G, H> operator+(const SHD<T, N, G, H>& a, T c) {
+  SHD<T, N, G, H> r = a;
+  r.v = a.v + c;
+  return r;
+}
+
+template <typename T, int N, uint32_t G, uint64_t H>
+__device__ __forceinline__ SHD<T, N, G, H> operator-(const SHD<T, N, G, H>& a, T c) {
+  SHD<T, N, G, H> r = a;
+  r.v = a.v - c;
+  return r;
+}
+
+template <typename T, int N, uint32_t G>
+__device__ __forceinline__ SLin<T, N, G> operator-(const SLin<T, N, G>& a) {
+  SLin<T, N, G> r;
+  r.v = -a.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (mbit(G, i)) r.g[i] = -a.g[i];
+  return r;
+}
+
+// an affine value as a number with a (structurally zero) Hessian
+template <typename T, int N, uint32_t G>
+__device__ __forceinline__ SHD<T, N, G, 0> to_shd(const SLin<T, N, G>& a) {
+  SHD<T, N, G, 0> r;
+  r.v = a.v;
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (mbit(G, i)) r.g[i] = a.g[i];
+  return r;
+}
+
 template <typename T, int N, uint32_t G, uint64_t H>
 __device__ __forceinline__ SHD<T, N, G, H> operator*(const SHD<T, N, G, H>& a, T c) {
   SHD<T, N, G, H> r;

@@ -14,8 +14,9 @@
 //   inertia         1/2 w |x - xt|^2
 //   sym. Dirichlet  A (|J|_F^2 + |J^-1|_F^2) = A a (1 + 1/det(J)^2), a = |J|_F^2
 //
-// Two seeding strategies give the same derivatives:
-//  * FULL: tangents on every stencil DOF (width 2*dof for an edge or pair
+// Two seeding strategies give the same derivatives (the AD forms of
+// kAdReduced, kAdFull and kAdGeneric below):
+//  * full: tangents on every stencil DOF (width 2*dof for an edge or pair
 //    term, 3*dof for a face term); the energy is evaluated through the
 //    stencil-to-variable map in HyperDual arithmetic;
 //  * reduced (default): tangents on the term's natural variables (the edge
@@ -32,6 +33,26 @@
 #include "sparse_ad.cuh"
 
 namespace mad {
+
+// ------------------------------------------------- forms of the local AD
+// Template argument AD of the evaluators and kernels:
+//  * kAdReduced: tangents on the term's natural variables; the spring,
+//    symmetric Dirichlet and area energies use one univariate chain-rule step
+//    with its derivatives written out (spring_of_s, symdir_scale, area_of_s);
+//  * kAdFull: tangents on every stencil DOF (MAD_EVAL_FULL_STENCIL_AD);
+//  * kAdGeneric: tangents as kAdReduced, and every energy written as a plain
+//    expression of its inputs, differentiated by the number types' own
+//    operations and elementary functions (sqrt, 1/x) alone
+//    (MAD_EVAL_GENERIC_AD).
+constexpr int kAdReduced = 0;
+constexpr int kAdFull = 1;
+constexpr int kAdGeneric = 2;
+__host__ __device__ constexpr int ad_form(uint32_t flags) {
+  return (flags & MAD_EVAL_FULL_STENCIL_AD) ? kAdFull
+         : (flags & MAD_EVAL_GENERIC_AD)    ? kAdGeneric
+                                            : kAdReduced;
+}
+
 
 // ---------------------------------------------------------------- energies
 // S is the number type of the inputs (plain T, Lin or HyperDual); products
@@ -162,11 +183,17 @@ __device__ __forceinline__ void with_face2_kind(int kind, F&& f) {
 // by KIND at J = Jv, seeded on vec J.  Symmetric Dirichlet runs on the masked
 // AD numbers (25.1 against 27.1 us per 500^2 eval); ARAP, alone or summed,
 // on the dense ones, which measured faster for it (27.1 against 37.2 us).
-template <int KIND, typename T>
+template <int KIND, int AD, typename T>
 __device__ __forceinline__ HyperDual<T, 4> face2_hd(const T (&Jv)[4], T A) {
   if constexpr (KIND == kFaceSymDir) {
-    const auto m = symdir_energy_m(slin_var<T, 4, 0>(Jv[0]), slin_var<T, 4, 1>(Jv[1]),
-                                   slin_var<T, 4, 2>(Jv[2]), slin_var<T, 4, 3>(Jv[3]), A);
+    const auto j0 = slin_var<T, 4, 0>(Jv[0]);
+    const auto j1 = slin_var<T, 4, 1>(Jv[1]);
+    const auto j2 = slin_var<T, 4, 2>(Jv[2]);
+    const auto j3 = slin_var<T, 4, 3>(Jv[3]);
+    const auto m = [&] {
+      if constexpr (AD == kAdGeneric) return symdir_energy_g(j0, j1, j2, j3, A);
+      else return symdir_energy_m(j0, j1, j2, j3, A);
+    }();
     HyperDual<T, 4> e;
     e.v = m.v;
 #pragma unroll
@@ -232,6 +259,45 @@ __device__ __forceinline__ auto area_energy_m(const A0_& a0, const A1_& a1, cons
   return area_of_s(sq(n0) + sq(n1) + sq(n2), A0, k);
 }
 
+// The energies as plain expressions (kAdGeneric), on masked AD numbers.
+// spring / pair: k/2 (|d| - L0)^2
+template <typename T, int D>
+__device__ __forceinline__ auto spring_energy_g(const T* d, T L0, T k) {
+  const auto l = sqrt(sqnorm_m<T, D>(d));
+  return sq(l - L0) * (T(0.5) * k);
+}
+// symmetric Dirichlet: A (|J|_F^2 + |J^-1|_F^2) with J^-1 = adj(J) / det(J)
+template <typename J0, typename J1, typename J2, typename J3, typename T>
+__device__ __forceinline__ auto symdir_energy_g(const J0& j0, const J1& j1, const J2& j2,
+                                                const J3& j3, T A) {
+  const auto a = sq(j0) + sq(j1) + sq(j2) + sq(j3);
+  const auto idet = inv(j0 * j3 - j1 * j2);
+  const auto b = sq(to_shd(j3) * idet) + sq(to_shd(-j1) * idet) + sq(to_shd(-j2) * idet) +
+                 sq(to_shd(j0) * idet);
+  return (a + b) * A;
+}
+// area preservation: k/2 (A - A0)^2 / A0 with A = |e1 x e2| / 2
+template <typename A0_, typename A1_, typename A2_, typename B0_, typename B1_, typename B2_,
+          typename T>
+__device__ __forceinline__ auto area_energy_g(const A0_& a0, const A1_& a1, const A2_& a2,
+                                              const B0_& b0, const B1_& b1, const B2_& b2, T A0,
+                                              T k) {
+  const auto n0 = a1 * b2 - a2 * b1;
+  const auto n1 = a2 * b0 - a0 * b2;
+  const auto n2 = a0 * b1 - a1 * b0;
+  const auto A = sqrt(sq(n0) + sq(n1) + sq(n2)) * T(0.5);
+  return sq(A - A0) * (T(0.5) * k / A0);
+}
+// the area energy of a reduced-seeded row in either form
+template <int AD, typename A0_, typename A1_, typename A2_, typename B0_, typename B1_,
+          typename B2_, typename T>
+__device__ __forceinline__ auto area_energy_ad(const A0_& a0, const A1_& a1, const A2_& a2,
+                                               const B0_& b0, const B1_& b1, const B2_& b2, T A0,
+                                               T k) {
+  if constexpr (AD == kAdGeneric) return area_energy_g(a0, a1, a2, b0, b1, b2, A0, k);
+  else return area_energy_m(a0, a1, a2, b0, b1, b2, A0, k);
+}
+
 // ---------------------------------------------------------------- results
 // Edge / pair term: blocks are D x D row-major; the (b, a) block is the
 // transpose of Hab.
@@ -242,14 +308,21 @@ struct EdgeDerivs {
   T Haa[D * D], Hab[D * D], Hbb[D * D];
 };
 
-template <typename T, int D, bool FULL>
+// the spring energy of the edge vector d in the reduced or generic form
+template <int AD, typename T, int D>
+__device__ __forceinline__ auto spring_energy_ad(const T* d, T L0, T k) {
+  if constexpr (AD == kAdGeneric) return spring_energy_g<T, D>(d, L0, k);
+  else return spring_of_s(sqnorm_m<T, D>(d), L0, k);
+}
+
+template <typename T, int D, int AD>
 __device__ __forceinline__ void eval_edge(const T* xa, const T* xb, T L0, T k,
                                           EdgeDerivs<T, D>& o) {
-  if constexpr (!FULL) {
+  if constexpr (AD != kAdFull) {
     T d[D];
 #pragma unroll
     for (int a = 0; a < D; ++a) d[a] = xa[a] - xb[a];
-    const auto e = spring_of_s(sqnorm_m<T, D>(d), L0, k);
+    const auto e = spring_energy_ad<AD, T, D>(d, L0, k);
     o.E = e.v;
 #pragma unroll
     for (int a = 0; a < D; ++a) {
@@ -288,25 +361,25 @@ __device__ __forceinline__ void eval_edge(const T* xa, const T* xb, T L0, T k,
 // a thread's edge terms and the colour phases that add them into the rows.
 // Reduced seeding: K = d2E/dd2 (packed symmetric), g = dE/dd; the blocks are
 // (a,a) = (b,b) = K, (a,b) = (b,a) = -K and g_a = g = -g_b.
-template <typename T, int D, bool FULL>
+template <typename T, int D, int AD>
 struct EdgeRes {
   T K[Tri<D>::size];
   T g[D];
   T E;
 };
 template <typename T, int D>
-struct EdgeRes<T, D, true> {
+struct EdgeRes<T, D, kAdFull> {
   EdgeDerivs<T, D> d;
 };
 
-template <typename T, int D, bool FULL>
+template <typename T, int D, int AD>
 __device__ __forceinline__ void eval_edge_res(const T* xa, const T* xb, T L0, T k,
-                                              EdgeRes<T, D, FULL>& R) {
-  if constexpr (!FULL) {
+                                              EdgeRes<T, D, AD>& R) {
+  if constexpr (AD != kAdFull) {
     T d[D];
 #pragma unroll
     for (int a = 0; a < D; ++a) d[a] = xa[a] - xb[a];
-    const auto e = spring_of_s(sqnorm_m<T, D>(d), L0, k);
+    const auto e = spring_energy_ad<AD, T, D>(d, L0, k);
     R.E = e.v;
 #pragma unroll
     for (int a = 0; a < D; ++a) R.g[a] = sgrad(e, a);
@@ -315,7 +388,7 @@ __device__ __forceinline__ void eval_edge_res(const T* xa, const T* xb, T L0, T 
 #pragma unroll
       for (int b = a; b < D; ++b) R.K[Tri<D>::idx(a, b)] = shess(e, a, b);
   } else {
-    eval_edge<T, D, true>(xa, xb, L0, k, R.d);
+    eval_edge<T, D, kAdFull>(xa, xb, L0, k, R.d);
   }
 }
 
@@ -328,10 +401,10 @@ __device__ __forceinline__ void put(T& dst, T v) {
   if constexpr (STORE) dst = v; else dst += v;
 }
 
-template <bool STORE_OFF, typename T, int D, bool FULL>
-__device__ __forceinline__ void apply_edge_side(const EdgeRes<T, D, FULL>& R, int side, T* dacc,
+template <bool STORE_OFF, typename T, int D, int AD>
+__device__ __forceinline__ void apply_edge_side(const EdgeRes<T, D, AD>& R, int side, T* dacc,
                                                 T* off, T* gr) {
-  if constexpr (!FULL) {
+  if constexpr (AD != kAdFull) {
     const T sg = side == 0 ? T(1) : T(-1);
 #pragma unroll
     for (int q = 0; q < Tri<D>::size; ++q) dacc[q] += R.K[q];
@@ -356,9 +429,9 @@ __device__ __forceinline__ void apply_edge_side(const EdgeRes<T, D, FULL>& R, in
   }
 }
 
-template <typename T, int D, bool FULL>
-__device__ __forceinline__ T edge_energy(const EdgeRes<T, D, FULL>& R) {
-  if constexpr (!FULL) return R.E; else return R.d.E;
+template <typename T, int D, int AD>
+__device__ __forceinline__ T edge_energy(const EdgeRes<T, D, AD>& R) {
+  if constexpr (AD != kAdFull) return R.E; else return R.d.E;
 }
 
 // Inertia: reduced seeding on r = x - xt (width D)
@@ -388,12 +461,14 @@ struct FaceDerivs {
   T H[3][3][4];
 };
 
-template <typename T, bool FULL, int KIND = kFaceSymDir>
+// (AD: kAdReduced or kAdFull; the dense number types)
+template <typename T, int AD, int KIND = kFaceSymDir>
 __device__ __forceinline__ void eval_symdir(const T* u0, const T* u1, const T* u2,
                                             const T* M, T A, FaceDerivs<T>& o) {
+  static_assert(AD != kAdGeneric, "the generic form runs on the row kernels");
   // corner weights w_k: dJ[al][ga]/du_k[be] = delta(al, be) w_k[ga]
   const T w[3][2] = {{-(M[0] + M[2]), -(M[1] + M[3])}, {M[0], M[1]}, {M[2], M[3]}};
-  if constexpr (!FULL) {
+  if constexpr (AD != kAdFull) {
     T Jv[4];
 #pragma unroll
     for (int al = 0; al < 2; ++al)
@@ -474,12 +549,12 @@ __device__ __forceinline__ T sel3(int c, T a, T b, T d) {
   return c == 0 ? a : (c == 1 ? b : d);
 }
 
-template <typename T, bool FULL, int KIND>
+template <typename T, int AD, int KIND>
 __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const T* xk, int c,
                                                 const T* M, T A, FaceRow<T>& o) {
   // corner weights of corners 0, 1, 2; then those of i, j, k
   const T w[3][2] = {{-(M[0] + M[2]), -(M[1] + M[3])}, {M[0], M[1]}, {M[2], M[3]}};
-  if constexpr (!FULL) {
+  if constexpr (AD != kAdFull) {
     T wr[3][2];
 #pragma unroll
     for (int ga = 0; ga < 2; ++ga) {
@@ -497,7 +572,7 @@ __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const 
 #pragma unroll
       for (int ga = 0; ga < 2; ++ga) Jv[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
     }
-    const HyperDual<T, 4> e = face2_hd<KIND>(Jv, A);
+    const HyperDual<T, 4> e = face2_hd<KIND, AD>(Jv, A);
     o.E = e.v;
 #pragma unroll
     for (int al = 0; al < 2; ++al) o.g[al] = e.g[2 * al] * wr[0][0] + e.g[2 * al + 1] * wr[0][1];
@@ -566,11 +641,11 @@ struct FaceRow3 {
   T H[3][9];  // (i,i), (i,j), (i,k)
 };
 
-template <typename T, bool FULL>
+template <typename T, int AD>
 __device__ __forceinline__ void eval_area_row(const T* xi, const T* xj, const T* xk, T A0, T k,
                                               FaceRow3<T>& o) {
-  if constexpr (!FULL) {
-    const auto e = area_energy_m(
+  if constexpr (AD != kAdFull) {
+    const auto e = area_energy_ad<AD>(
         slin_var<T, 6, 0>(xj[0] - xi[0]), slin_var<T, 6, 1>(xj[1] - xi[1]),
         slin_var<T, 6, 2>(xj[2] - xi[2]), slin_var<T, 6, 3>(xk[0] - xi[0]),
         slin_var<T, 6, 4>(xk[1] - xi[1]), slin_var<T, 6, 5>(xk[2] - xi[2]), A0, k);
@@ -611,12 +686,12 @@ __device__ __forceinline__ void eval_area_row(const T* xi, const T* xj, const T*
 // (H v) of one area-preservation face for its three corners (face order):
 // out[3a + al].  Reduced form: t = H_e dE with dE = (v1 - v0, v2 - v0), then
 // corner a takes p1[a] t_e1 + p2[a] t_e2 with p1 = (-1, 1, 0), p2 = (-1, 0, 1).
-template <typename T, bool FULL>
+template <typename T, int AD>
 __device__ __forceinline__ void hv_area_face(const T* u0, const T* u1, const T* u2,
                                              const T* v0, const T* v1, const T* v2, T A0, T k,
                                              T* out) {
-  if constexpr (!FULL) {
-    const auto e = area_energy_m(
+  if constexpr (AD != kAdFull) {
+    const auto e = area_energy_ad<AD>(
         slin_var<T, 6, 0>(u1[0] - u0[0]), slin_var<T, 6, 1>(u1[1] - u0[1]),
         slin_var<T, 6, 2>(u1[2] - u0[2]), slin_var<T, 6, 3>(u2[0] - u0[0]),
         slin_var<T, 6, 4>(u2[1] - u0[1]), slin_var<T, 6, 5>(u2[2] - u0[2]), A0, k);
@@ -663,11 +738,11 @@ __device__ __forceinline__ void hv_area_face(const T* u0, const T* u1, const T* 
 // = sum_l (H_kl v_l)[al], with u and v the corners' positions and direction
 // in face order.  The reduced form contracts in J space: dJ = sum_k v_k w_k^T,
 // t = H_J dJ, out_k = t projected on w_k.
-template <typename T, bool FULL, int KIND>
+template <typename T, int AD, int KIND>
 __device__ __forceinline__ void hv_symdir_face(const T* u0, const T* u1, const T* u2,
                                                const T* v0, const T* v1, const T* v2,
                                                const T* M, T A, T* out) {
-  if constexpr (!FULL) {
+  if constexpr (AD != kAdFull) {
     const T w[3][2] = {{-(M[0] + M[2]), -(M[1] + M[3])}, {M[0], M[1]}, {M[2], M[3]}};
     T Jv[4], dJ[4];
 #pragma unroll
@@ -677,7 +752,7 @@ __device__ __forceinline__ void hv_symdir_face(const T* u0, const T* u1, const T
         Jv[2 * al + ga] = (u1[al] - u0[al]) * M[ga] + (u2[al] - u0[al]) * M[2 + ga];
         dJ[2 * al + ga] = (v1[al] - v0[al]) * M[ga] + (v2[al] - v0[al]) * M[2 + ga];
       }
-    const HyperDual<T, 4> e = face2_hd<KIND>(Jv, A);
+    const HyperDual<T, 4> e = face2_hd<KIND, AD>(Jv, A);
     T t[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
@@ -692,7 +767,7 @@ __device__ __forceinline__ void hv_symdir_face(const T* u0, const T* u1, const T
       for (int al = 0; al < 2; ++al) out[2 * k + al] = t[2 * al] * w[k][0] + t[2 * al + 1] * w[k][1];
   } else {
     FaceDerivs<T> o;
-    eval_symdir<T, true, KIND>(u0, u1, u2, M, A, o);
+    eval_symdir<T, kAdFull, KIND>(u0, u1, u2, M, A, o);
     const T* vv[3] = {v0, v1, v2};
 #pragma unroll
     for (int k = 0; k < 3; ++k)

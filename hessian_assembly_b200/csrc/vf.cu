@@ -35,18 +35,12 @@ __host__ __device__ constexpr int vf_coef(int v, int s) {
   return v == 0 ? (s == 0 ? 1 : 0) : v == 1 ? -1 : (v - 1 == s ? 1 : 0);
 }
 
-template <typename T, int N, uint32_t G>
-__device__ __forceinline__ SHD<T, N, G, 0> to_shd(const SLin<T, N, G>& a) {
-  SHD<T, N, G, 0> r;
-  r.v = a.v;
-#pragma unroll
-  for (int i = 0; i < N; ++i)
-    if (mbit(G, i)) r.g[i] = a.g[i];
-  return r;
-}
-
-// E and its derivatives in z of one term: value, gradient [9], Hessian (packed)
-template <typename T>
+// E and its derivatives in z of one term: value, gradient [9], Hessian
+// (packed).  GEN: E written as a plain expression, d = (u . n) / sqrt(n . n)
+// and E = k/2 (d - r)^2, differentiated by the number types' operations and
+// elementary functions alone; otherwise 1/|n| and the final square are
+// single chain-rule steps with their derivatives written out.
+template <typename T, bool GEN>
 __device__ __forceinline__ auto vf_energy(const T* p, const T* a, const T* b, const T* c, T r,
                                           T k) {
   const auto u0 = to_shd(slin_var<T, 9, 0>(p[0] - a[0]));
@@ -63,13 +57,18 @@ __device__ __forceinline__ auto vf_energy(const T* p, const T* a, const T* b, co
   const auto n2 = e10 * e21 - e11 * e20;
   const auto un = u0 * n0 + u1 * n1 + u2 * n2;
   const auto nn = sq(n0) + sq(n1) + sq(n2);
-  // 1/|n| as one chain step: s^(-1/2), -1/2 s^(-3/2), 3/4 s^(-5/2)
-  const T is = T(1) / ::sqrt(nn.v);
-  const T is2 = is * is;
-  const auto inv_m = chain(nn, is, T(-0.5) * is * is2, T(0.75) * is * is2 * is2);
-  const auto d = un * inv_m;
-  const T dev = d.v - r;
-  return chain(d, T(0.5) * k * dev * dev, k * dev, k);
+  if constexpr (GEN) {
+    const auto d = un * inv(sqrt(nn));
+    return sq(d - r) * (T(0.5) * k);
+  } else {
+    // 1/|n| as one chain step: s^(-1/2), -1/2 s^(-3/2), 3/4 s^(-5/2)
+    const T is = T(1) / ::sqrt(nn.v);
+    const T is2 = is * is;
+    const auto inv_m = chain(nn, is, T(-0.5) * is * is2, T(0.75) * is * is2 * is2);
+    const auto d = un * inv_m;
+    const T dev = d.v - r;
+    return chain(d, T(0.5) * k * dev * dev, k * dev, k);
+  }
 }
 
 __device__ __forceinline__ int find_col(const int32_t* __restrict__ rp,
@@ -127,7 +126,7 @@ __device__ __forceinline__ bool load_term(int t, const int32_t* __restrict__ vf,
   return true;
 }
 
-template <typename T>
+template <typename T, bool GEN>
 __global__ void __launch_bounds__(kVfThreads) k_vf_eval(
     int n, const int32_t* __restrict__ vf, const T* __restrict__ rest, T k,
     const int32_t* __restrict__ F, int nF, int V, const T* __restrict__ x,
@@ -141,7 +140,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_eval(
     if (!load_term<T>(t, vf, F, nF, V, x, vid, X)) {
       atomicOr(status, kStatusIndex);
     } else {
-      const auto z = vf_energy<T>(X[0], X[1], X[2], X[3], rest[t], k);
+      const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
       e = (double)z.v;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -190,7 +189,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_eval(
   }
 }
 
-template <typename T>
+template <typename T, bool GEN>
 __global__ void __launch_bounds__(kVfThreads) k_vf_hvp(
     int n, const int32_t* __restrict__ vf, const T* __restrict__ rest, T k,
     const int32_t* __restrict__ F, int nF, int V, const T* __restrict__ x,
@@ -203,7 +202,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_hvp(
     atomicOr(status, kStatusIndex);
     return;
   }
-  const auto z = vf_energy<T>(X[0], X[1], X[2], X[3], rest[t], k);
+  const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
   // dz_s = sum_j c_j[s] v_j, t = H_z dz, y_i = sum_s c_i[s] t_s
   T dz[9];
 #pragma unroll
@@ -241,32 +240,43 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_hvp(
 
 }  // namespace
 
+template <typename T, bool GEN>
+void vf_eval_t(const VfLaunch& L, unsigned nb, void* g, void* H, double* energy, cudaStream_t s) {
+  k_vf_eval<T, GEN><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const T*)L.rest, (T)L.k, L.F, L.nF, L.V,
+                                              (const T*)L.x, L.rp, L.ci, (T*)g, (T*)H, energy,
+                                              L.status);
+}
+
+template <typename T, bool GEN>
+void vf_hvp_t(const VfLaunch& L, unsigned nb, const void* v, void* y, cudaStream_t s) {
+  k_vf_hvp<T, GEN><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const T*)L.rest, (T)L.k, L.F, L.nF, L.V,
+                                             (const T*)L.x, (const T*)v, (T*)y, L.status);
+}
+
 cudaError_t launch_vf_eval(int dtype, const VfLaunch& L, void* g, void* H, double* energy,
                            cudaStream_t s) {
   if (L.n <= 0) return cudaSuccess;
   const unsigned nb = (unsigned)((L.n + kVfThreads - 1) / kVfThreads);
-  if (dtype == MAD_F64)
-    k_vf_eval<double><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const double*)L.rest, L.k, L.F,
-                                               L.nF, L.V, (const double*)L.x, L.rp, L.ci,
-                                               (double*)g, (double*)H, energy, L.status);
-  else
-    k_vf_eval<float><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const float*)L.rest, (float)L.k, L.F,
-                                              L.nF, L.V, (const float*)L.x, L.rp, L.ci,
-                                              (float*)g, (float*)H, energy, L.status);
+  if (dtype == MAD_F64) {
+    if (L.generic) vf_eval_t<double, true>(L, nb, g, H, energy, s);
+    else vf_eval_t<double, false>(L, nb, g, H, energy, s);
+  } else {
+    if (L.generic) vf_eval_t<float, true>(L, nb, g, H, energy, s);
+    else vf_eval_t<float, false>(L, nb, g, H, energy, s);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_vf_hvp(int dtype, const VfLaunch& L, const void* v, void* y, cudaStream_t s) {
   if (L.n <= 0) return cudaSuccess;
   const unsigned nb = (unsigned)((L.n + kVfThreads - 1) / kVfThreads);
-  if (dtype == MAD_F64)
-    k_vf_hvp<double><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const double*)L.rest, L.k, L.F, L.nF,
-                                              L.V, (const double*)L.x, (const double*)v,
-                                              (double*)y, L.status);
-  else
-    k_vf_hvp<float><<<nb, kVfThreads, 0, s>>>(L.n, L.vf, (const float*)L.rest, (float)L.k, L.F,
-                                             L.nF, L.V, (const float*)L.x, (const float*)v,
-                                             (float*)y, L.status);
+  if (dtype == MAD_F64) {
+    if (L.generic) vf_hvp_t<double, true>(L, nb, v, y, s);
+    else vf_hvp_t<double, false>(L, nb, v, y, s);
+  } else {
+    if (L.generic) vf_hvp_t<float, true>(L, nb, v, y, s);
+    else vf_hvp_t<float, false>(L, nb, v, y, s);
+  }
   return cudaGetLastError();
 }
 

@@ -111,7 +111,17 @@ enum {
    * default row-streaming kernel (one warp per 32 consecutive rows, no
    * block-wide barriers).  Same results up to rounding.  The patch kernel
    * does not evaluate MAD_TERM_AREA or MAD_TERM_ARAP (MAD_ERR_UNIMPLEMENTED). */
-  MAD_EVAL_PATCH_STAGED = 4u
+  MAD_EVAL_PATCH_STAGED = 4u,
+  /* Differentiate every energy as written: the spring and pair, symmetric
+   * Dirichlet, area-preservation and vertex-face energies as plain
+   * expressions (square roots, products, 1/det), each differentiated by the
+   * AD number types' own operations and elementary functions, instead of
+   * the default, which evaluates each as a univariate function of one AD
+   * intermediate with that function's first and second derivatives written
+   * out (one chain-rule step).  Same derivatives up to rounding; the default
+   * is faster.  Not with MAD_EVAL_FULL_STENCIL_AD (MAD_ERR_INVALID_ARG), nor
+   * with the patch kernel (MAD_ERR_UNIMPLEMENTED).                          */
+  MAD_EVAL_GENERIC_AD = 8u
 };
 
 typedef struct {

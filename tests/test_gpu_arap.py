@@ -44,7 +44,7 @@ def run(orc, ctx, V, F, UV, Minv, area, mask, dtype, flags=0, seed=7, extra=None
     return terms, oE
 
 
-@pytest.mark.parametrize("flags", [0, FULL])
+@pytest.mark.parametrize("flags", [0, FULL, 8])
 @pytest.mark.parametrize("mask", [ARAP, ARAP | SYMDIR])
 @pytest.mark.parametrize("dtype", ["float32", "float64"])
 def test_arap_grid(orc, dtype, mask, flags):

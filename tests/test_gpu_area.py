@@ -10,6 +10,7 @@ from _parity import ETOL, assert_close, cloth_context, gpu_pattern, run_eval, to
 
 pytestmark = pytest.mark.gpu
 FULL = 1
+GEN = 8
 KA = 2.0e3
 
 
@@ -55,7 +56,7 @@ def check(orc, n, dtype, mask=1 | 2 | 16, flags=0, seed=5000, pairs=None):
     return ctx, st, x, terms, oE
 
 
-@pytest.mark.parametrize("flags", [0, FULL])
+@pytest.mark.parametrize("flags", [0, FULL, GEN])
 @pytest.mark.parametrize("mask", [16, 1 | 2 | 16])
 def test_area_cloth_fp64(orc, mask, flags):
     check(orc, 20, "float64", mask, flags)
@@ -63,6 +64,10 @@ def test_area_cloth_fp64(orc, mask, flags):
 
 def test_area_cloth_300x300_fp32(orc):
     check(orc, 300, "float32")
+
+
+def test_area_cloth_300x300_fp32_generic_ad(orc):
+    check(orc, 300, "float32", flags=GEN, seed=5003)
 
 
 def test_area_with_pairs(orc):

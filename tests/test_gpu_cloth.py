@@ -17,16 +17,17 @@ pytestmark = pytest.mark.gpu
 FULL = 1  # MAD_EVAL_FULL_STENCIL_AD
 SCAT = 2  # MAD_EVAL_EDGE_SCATTER
 PATCH = 4  # MAD_EVAL_PATCH_STAGED
+GEN = 8  # MAD_EVAL_GENERIC_AD
 
 
-@pytest.mark.parametrize("flags", [0, FULL, SCAT, FULL | SCAT, PATCH, PATCH | FULL])
+@pytest.mark.parametrize("flags", [0, FULL, SCAT, FULL | SCAT, PATCH, PATCH | FULL, GEN])
 @pytest.mark.parametrize("part", ["rcb", "bfs"])
 def test_cloth_10x10(orc, flags, part):
     check_cloth(orc, 10, "float32", flags=flags, part=part, seed=1001)
 
 
 @pytest.mark.parametrize("dtype", ["float32", "float64"])
-@pytest.mark.parametrize("flags", [0, FULL, SCAT, PATCH])
+@pytest.mark.parametrize("flags", [0, FULL, SCAT, PATCH, GEN])
 def test_cloth_100x100(orc, dtype, flags):
     check_cloth(orc, 100, dtype, flags=flags, seed=1002)
 
@@ -52,6 +53,25 @@ def test_cloth_1000x1000_full(orc):
 
 def test_cloth_1000x1000_second_step_and_full_ad(orc):
     check_cloth(orc, 1000, "float32", seed=1003, step=7, flags=FULL)
+
+
+def test_cloth_1000x1000_generic_ad(orc):
+    # the spring energy as a plain expression, differentiated by the AD types alone
+    check_cloth(orc, 1000, "float32", seed=1003, step=11, flags=GEN)
+
+
+def test_generic_ad_refusals():
+    import hessian_assembly_b200 as mad
+    import torch
+    ctx, st = cloth_context(6)
+    x = to_dev(mi.cloth_x(6, 1, 0, np.float32))
+    g = torch.zeros((st["V"], 3), device="cuda")
+    H = torch.zeros((ctx.info.capacity_blocks, 3, 3), device="cuda")
+    for flags, code in ((GEN | FULL, mad.MAD_ERR_INVALID_ARG), (GEN | PATCH, mad.MAD_ERR_UNIMPLEMENTED),
+                        (GEN | SCAT, mad.MAD_ERR_UNIMPLEMENTED)):
+        with pytest.raises(mad.MadError) as ei:
+            ctx.mad_eval(x, cloth_terms(st, "float32", 3, flags), g, H)
+        assert ei.value.status == code
 
 
 def test_cloth_1000x1000_scatter(orc):

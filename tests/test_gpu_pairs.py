@@ -27,7 +27,7 @@ def pair_case(orc, n, P, dtype="float32", seed=1005, step=0, flags=0, **kw):
                        prest=rest, ctx=ctx, st=st)
 
 
-@pytest.mark.parametrize("flags", [0, FULL, SCAT, PATCH])
+@pytest.mark.parametrize("flags", [0, FULL, SCAT, PATCH, 8])
 def test_pairs_small(orc, flags):
     pair_case(orc, 30, 60, flags=flags)
 

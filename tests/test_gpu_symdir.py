@@ -9,6 +9,7 @@ from _parity import ETOL, assert_close, gpu_pattern, to_dev
 pytestmark = pytest.mark.gpu
 FULL = 1
 PATCH = 4  # the patch-staged kernel instead of the row-streaming one
+GEN = 8  # the energy as a plain expression (MAD_EVAL_GENERIC_AD)
 
 
 def setup(n, dtype, seed=1004, **kw):
@@ -53,12 +54,12 @@ def check(orc, n, dtype, flags=0, seed=1004, **kw):
     return ctx
 
 
-@pytest.mark.parametrize("flags", [0, FULL, PATCH, PATCH | FULL])
+@pytest.mark.parametrize("flags", [0, FULL, PATCH, PATCH | FULL, GEN])
 def test_symdir_small(orc, flags):
     check(orc, 10, "float32", flags)
 
 
-@pytest.mark.parametrize("flags", [0, FULL, PATCH, PATCH | FULL])
+@pytest.mark.parametrize("flags", [0, FULL, PATCH, PATCH | FULL, GEN])
 def test_symdir_fp64(orc, flags):
     check(orc, 37, "float64", flags)
 
@@ -67,6 +68,10 @@ def test_symdir_fp64(orc, flags):
 def test_symdir_500x500_full(orc, flags):
     ctx = check(orc, 500, "float32", flags)
     assert ctx.info.n_patches > 100
+
+
+def test_symdir_500x500_generic_ad(orc):
+    check(orc, 500, "float32", GEN, seed=2005)
 
 
 def test_symdir_500x500_full_ad(orc):

@@ -29,7 +29,7 @@ def vf_terms_for(n, nvf, seed):
     return vf, rest, pairs
 
 
-def check(orc, n, dtype, nvf, seed, mask=1 | 2 | VF):
+def check(orc, n, dtype, nvf, seed, mask=1 | 2 | VF, flags=0):
     import hessian_assembly_b200 as mad
     import torch
     vf, rest, pairs = vf_terms_for(n, nvf, seed)
@@ -38,7 +38,7 @@ def check(orc, n, dtype, nvf, seed, mask=1 | 2 | VF):
     x = mi.cloth_x(n, seed, 0, np.dtype(dtype))
     x = (x + 0.02 * mi.grid_spacing(n) * np.random.default_rng(seed + 1).standard_normal(x.shape)
          ).astype(dtype)
-    terms = mad.Terms(mask=mask, spring_rest=to_dev(st["L0"], dtype), spring_k=st["k"],
+    terms = mad.Terms(mask=mask, flags=flags, spring_rest=to_dev(st["L0"], dtype), spring_k=st["k"],
                       inertia_xt=to_dev(st["xt"], dtype), inertia_w=st["w"],
                       vf=to_dev(vf), vf_rest=to_dev(rest, dtype), vf_k=KC)
     g, H, E = run_eval(ctx, x, terms, dtype)
@@ -64,6 +64,11 @@ def check(orc, n, dtype, nvf, seed, mask=1 | 2 | VF):
 @pytest.mark.parametrize("dtype", ["float32", "float64"])
 def test_vf_cloth(orc, dtype):
     check(orc, 30, dtype, 200, 6001)
+
+
+@pytest.mark.parametrize("dtype", ["float32", "float64"])
+def test_vf_cloth_generic_ad(orc, dtype):
+    check(orc, 30, dtype, 200, 6004, flags=8)
 
 
 def test_vf_only_terms(orc):
