@@ -1,0 +1,45 @@
+// pdl.cuh -- programmatic dependent launch between the kernels of one step.
+//
+// A kernel launched with programmatic stream serialization may start before
+// the previous kernel on its stream has finished: its blocks are scheduled
+// once every block of the previous kernel has signalled (or exited), load
+// what does not depend on that kernel, and wait before reading its results.
+// The launch latency and ramp of a chain of dependent kernels then overlap
+// the tails of their predecessors.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <utility>
+
+namespace mad {
+
+// Wait until the previous kernel on the stream has finished and its writes
+// are visible (returns at once for a kernel launched the ordinary way).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Let the next kernel on the stream start (it still waits for the results).
+__device__ __forceinline__ void grid_dependents_may_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launches k<<<grid, block, smem, s>>>(args...) with programmatic stream
+// serialization allowed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
+}  // namespace mad

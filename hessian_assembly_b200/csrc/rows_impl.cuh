@@ -26,6 +26,7 @@
 #include <type_traits>
 
 #include "mad_internal.h"
+#include "pdl.cuh"
 #include "rows_common.h"
 #include "terms.cuh"
 
@@ -547,6 +548,20 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, (FACES != 0)>(
   if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
 }
 
+// y += the per-face pass's result for incidence q = 3f + c (DOF values)
+template <typename T, int DOF>
+__device__ __forceinline__ void add_corner_hv(const T* __restrict__ fhv, uint32_t q, T* yr) {
+  if constexpr (DOF == 2) {
+    using T2 = typename std::conditional<sizeof(T) == 4, float2, double2>::type;
+    const T2 c = reinterpret_cast<const T2*>(fhv)[q];
+    yr[0] += c.x;
+    yr[1] += c.y;
+  } else {
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) yr[a] += fhv[DOF * q + a];
+  }
+}
+
 template <typename T, int DOF, int AD, int S0, bool FACES>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_hvp(const RArgs<T> A) {
   constexpr int TD = Tri<DOF>::size;
@@ -574,6 +589,14 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
     }
     m = A.meta[i];
   }
+  // face terms: the row's incidence entries (3f + c) of the per-face pass
+  constexpr int SF = kFaceRowSlots;
+  const bool face_terms =
+      FACES && (A.mask & (DOF == 2 ? (MAD_TERM_SYMDIR | MAD_TERM_ARAP) : MAD_TERM_AREA));
+  int32_t fe[SF];
+#pragma unroll
+  for (int k = 0; k < SF; ++k)
+    fe[k] = face_terms && k < A.sf ? A.fcslots[(uint32_t)((tile * A.sf + k) * 32 + lane)] : -1;
   if (A.mask & MAD_TERM_INERTIA) {
     T xti[DOF], Ei, gi[DOF], Hi[DOF * DOF];
 #pragma unroll
@@ -613,31 +636,6 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
                               });
     }
   }
-  if constexpr (FACES) {
-    if (A.mask & (DOF == 2 ? (MAD_TERM_SYMDIR | MAD_TERM_ARAP) : MAD_TERM_AREA)) {
-      // the row's corners' results of the per-face pass (k_face_hv)
-      constexpr int SF = kFaceRowSlots;
-      int32_t e[SF];
-#pragma unroll
-      for (int k = 0; k < SF; ++k)
-        e[k] = k < A.sf ? A.fcslots[(uint32_t)((tile * A.sf + k) * 32 + lane)] : -1;
-#pragma unroll
-      for (int k = 0; k < SF; ++k) {
-        if (e[k] == -1) continue;
-        const uint32_t q = (uint32_t)e[k] & 0x7FFFFFFFu;
-#pragma unroll
-        for (int a = 0; a < DOF; ++a) yr[a] += A.fhv[DOF * q + a];
-      }
-      if (e[SF - 1] != -1 && e[SF - 1] < 0) {  // the row continues in the overflow table
-        const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
-        for (int q = o0; q < o1; ++q) {
-          const uint32_t fc = (uint32_t)A.fcofl[q];
-#pragma unroll
-          for (int a = 0; a < DOF; ++a) yr[a] += A.fhv[DOF * fc + a];
-        }
-      }
-    }
-  }
   if (pairs) {
     const int pb = A.prow[i], pe = A.prow[i + 1];
     for (int e = pb; e < pe; ++e) {
@@ -653,6 +651,23 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
       hv(Rp, vj);
     }
   }
+  if constexpr (FACES) {
+    if (face_terms) {
+      // the row's corners' results of the per-face pass (k_face_hv): the
+      // table entries were loaded above; the results may be read once that
+      // pass has finished (a no-op when this grid was launched after it)
+      grid_dependency_wait();
+#pragma unroll
+      for (int k = 0; k < SF; ++k) {
+        if (fe[k] == -1) continue;
+        add_corner_hv<T, DOF>(A.fhv, (uint32_t)fe[k] & 0x7FFFFFFFu, yr);
+      }
+      if (fe[SF - 1] != -1 && fe[SF - 1] < 0) {  // the row continues in the overflow table
+        const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
+        for (int q = o0; q < o1; ++q) add_corner_hv<T, DOF>(A.fhv, (uint32_t)A.fcofl[q], yr);
+      }
+    }
+  }
   (void)TD;
 #pragma unroll
   for (int a = 0; a < DOF; ++a) A.y[(uint32_t)(i * DOF + a)] = yr[a];
@@ -666,6 +681,7 @@ __global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __r
                                                       const T* __restrict__ v,
                                                       const T* __restrict__ area, T ka,
                                                       T* __restrict__ out) {
+  grid_dependents_may_launch();  // the row pass may start; it waits for the results
   const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (f >= nF) return;
   T u[3][3], w[3][3];
@@ -694,6 +710,7 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
                                                  const T* __restrict__ Minv,
                                                  const T* __restrict__ area, T* __restrict__ out,
                                                  int kind) {
+  grid_dependents_may_launch();  // the row pass may start; it waits for the results
   const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (f >= nF) return;
   const int32_t a = F[3 * f], b = F[3 * f + 1], c = F[3 * f + 2];
@@ -727,8 +744,14 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
     hv_symdir_face<T, AD, decltype(kc)::value>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f],
                                                  o);
   });
+  T2* o2 = reinterpret_cast<T2*>(out) + 3 * f;  // one corner's pair per 8 (16) bytes
 #pragma unroll
-  for (int q = 0; q < 6; ++q) out[6 * f + q] = o[q];
+  for (int c2 = 0; c2 < 3; ++c2) {
+    T2 v2;
+    v2.x = o[2 * c2];
+    v2.y = o[2 * c2 + 1];
+    o2[c2] = v2;
+  }
 }
 
 
@@ -892,11 +915,14 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
     constexpr int AD = decltype(adc)::value;
     const bool sp = t.mask & MAD_TERM_SPRING;
     // the row pass after a per-face pass (face terms), or alone
+    // the row pass after the per-face pass, launched with programmatic
+    // stream serialization: its blocks start while the face pass finishes,
+    // load their own rows' inputs and wait for the face results
     auto rows = [&](auto facesc) {
       constexpr bool FC = decltype(facesc)::value;
-      if (sp) k_rows_hvp<T, DOF, AD, kS0Max, FC><<<nb, kRowThreads, 0, s>>>(A);
-      else k_rows_hvp<T, DOF, AD, 0, FC><<<nb, kRowThreads, 0, s>>>(A);
-      return cudaGetLastError();
+      if (sp)
+        return launch_pdl(k_rows_hvp<T, DOF, AD, kS0Max, FC>, dim3(nb), dim3(kRowThreads), 0, s, A);
+      return launch_pdl(k_rows_hvp<T, DOF, AD, 0, FC>, dim3(nb), dim3(kRowThreads), 0, s, A);
     };
     if constexpr (DOF == 2) {
       if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
