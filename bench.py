@@ -509,35 +509,42 @@ KC = 50.0
 
 
 def vf1000(res, mad, torch, dev, stream, timeit):
-    """Springs + inertia + 10^5 vertex-face terms on the 1000^2 cloth: the
-    insertion of their 3 x 10^5 (vertex, corner) pairs, then eval and the
-    product; the row kernel runs first, the vertex-face pass after it."""
+    """Springs + inertia + 10^5 vertex-face terms on the 1000^2 cloth.  The
+    set is installed once (mad_add_vf: its 3 x 10^5 (vertex, corner) pairs
+    inserted and the per-row term lists built), then evaluated per row after
+    the row kernel (eval and product).  The same terms passed per call
+    (t->vf), one thread per term adding with atomics, are timed beside it."""
     st = mi.cloth_static(N_GRID, np.float32)
     vf = mi.random_vf(N_GRID, N_VF, 1009, 0)
     pairs = mi.vf_pairs(vf, st["F"])
     ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"], max_pairs=len(pairs),
                       slack=0.2)
-    dp = torch.from_numpy(pairs).to(dev)
-    dr = torch.zeros(len(pairs), dtype=torch.float32, device=dev)
-    res["vf1000_insert_ms"] = round(timeit(lambda: ctx.mad_add_pairs(dp, dr, stream), n=16), 5)
+    dvf = torch.from_numpy(vf).to(dev)
+    res["vf1000_insert_ms"] = round(timeit(lambda: ctx.mad_add_vf(dvf, stream), n=16), 5)
     rest = (0.001 * np.random.default_rng(1010).standard_normal(N_VF)).astype(np.float32)
     terms = mad.Terms(mask=1 | 2 | 64, spring_rest=torch.from_numpy(st["L0"]).to(dev),
                       spring_k=st["k"], inertia_xt=torch.from_numpy(st["xt"]).to(dev),
-                      inertia_w=st["w"], vf=torch.from_numpy(vf).to(dev),
-                      vf_rest=torch.from_numpy(rest).to(dev), vf_k=KC)
+                      inertia_w=st["w"], vf=None, vf_rest=torch.from_numpy(rest).to(dev),
+                      vf_k=KC)
     x = torch.from_numpy(mi.cloth_x(N_GRID, 1011, 0, np.float32)).to(dev)
     v = torch.from_numpy(mi.probe_vector(st["V"], 3, 1012, np.float32)).to(dev)
     g = torch.empty((st["V"], 3), device=dev)
     y = torch.empty((st["V"], 3), device=dev)
     H = torch.empty((ctx.info.capacity_blocks, 3, 3), device=dev)
     res["vf1000_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
+    res["vf1000_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
     # read x, the edge list, the terms (vertex, face, rest) and their faces'
     # corners; write g and the blocks of the pattern holding the terms' pairs
     _, _, nz = ctx.mad_pattern()
     nnzb = int(nz.cpu()[0])
     V, E = st["V"], len(st["edges"])
     res["vf1000_eval_bytes"] = 12 * V + 8 * E + 24 * N_VF + 12 * V + 36 * nnzb
-    res["vf1000_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
+    # the same terms passed per call: atomics
+    ta = mad.Terms(mask=1 | 2 | 64, spring_rest=terms.spring_rest, spring_k=st["k"],
+                   inertia_xt=terms.inertia_xt, inertia_w=st["w"], vf=dvf,
+                   vf_rest=terms.vf_rest, vf_k=KC)
+    res["vf1000_atomic_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, ta, g, H, None, stream)), 5)
+    res["vf1000_atomic_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, ta, v, y, stream)), 5)
     res["vf1000_status"] = ctx.mad_status_sync()
     ctx.close()
 

@@ -57,7 +57,7 @@ EXPORTS = ("mad_default_opts", "mad_create", "mad_info", "mad_edges", "mad_patte
            "mad_eval", "mad_hvp", "mad_add_pairs", "mad_status_sync", "mad_eval_host",
            "mad_last_error", "mad_destroy", "mad_selftest_dual", "mad_energy_noalloc",
            "mad_jacobian_shape", "mad_jacobian_pattern", "mad_jacobian", "mad_shard_plan",
-           "mad_shard_halo", "mad_eval_shard")
+           "mad_shard_halo", "mad_eval_shard", "mad_add_vf")
 
 
 class mad_opts(ctypes.Structure):
@@ -132,6 +132,8 @@ def load_library(path: str = LIB_PATH):
     lib.mad_destroy.restype = None
     lib.mad_selftest_dual.argtypes = [i32, vp, vp]
     lib.mad_selftest_dual.restype = ctypes.c_int
+    lib.mad_add_vf.argtypes = [vp, i32, vp, vp]
+    lib.mad_add_vf.restype = ctypes.c_int
     lib.mad_shard_plan.argtypes = [i32, i32, i32p, i32, i32p, ctypes.POINTER(ctypes.c_int64)]
     lib.mad_shard_plan.restype = ctypes.c_int
     lib.mad_shard_halo.argtypes = [i32, i32, i32p, i32, i32, i32p, i32p, i32]
@@ -211,7 +213,9 @@ class Terms:
     def to_c(self, dtype) -> mad_terms:
         torch = _torch()
         p = lambda t, n: None if t is None else _dev_ptr(t, dtype, n)  # noqa: E731
-        nvf = 0 if self.vf is None else int(self.vf.shape[0])
+        # without vf, the installed set (mad_add_vf): its size from vf_rest
+        nvf = (int(self.vf.shape[0]) if self.vf is not None else
+               int(self.vf_rest.shape[0]) if self.vf_rest is not None else 0)
         return mad_terms(self.mask, self.flags, p(self.spring_rest, "spring_rest"),
                          float(self.spring_k), p(self.inertia_xt, "inertia_xt"),
                          float(self.inertia_w), p(self.face_Minv, "face_Minv"),
@@ -307,6 +311,14 @@ class Context:
                                _dev_ptr(H_vals, self.torch_dtype, "H_vals"),
                                _dev_ptr(energy, torch.float64, "energy", allow_none=True),
                                _stream_ptr(stream))
+        self._check(st)
+
+    def mad_add_vf(self, vf, stream=None):
+        """Install vertex-face terms: vf a CUDA int32 tensor [n][2] (p, f)."""
+        torch = _torch()
+        n = int(vf.shape[0]) if vf is not None else 0
+        st = self.lib.mad_add_vf(self.h, n, _dev_ptr(vf, torch.int32, "vf") if n else None,
+                                 _stream_ptr(stream))
         self._check(st)
 
     def mad_eval_shard(self, row_begin, x_parts, rank, terms: Terms, g_part, H_part,

@@ -69,6 +69,7 @@ struct mad_ctx {
   // dynamic pattern
   DynBuf buf[2];
   int active = -1;  // -1: mesh pattern, no pairs
+  VfSet vfs;        // the installed vertex-face term set (mad_add_vf)
   // insertion scratch
   int32_t *cnt = nullptr, *tsum = nullptr, *newcnt = nullptr, *pe_pid = nullptr,
           *status = nullptr;
@@ -250,8 +251,11 @@ mad_status check_terms(mad_ctx* c, const mad_terms* t) {
     if (t->mask & MAD_TERM_PAIR)
       return fail(c, MAD_ERR_UNIMPLEMENTED, "vertex-face terms with pair terms in one mask");
     if (t->vf_n < 0) return fail(c, MAD_ERR_INVALID_ARG, "vf_n < 0");
-    if (t->vf_n > 0 && (!t->vf || !t->vf_rest))
-      return fail(c, MAD_ERR_INVALID_ARG, "vertex-face terms need vf and vf_rest");
+    if (t->vf_n > 0 && !t->vf_rest)
+      return fail(c, MAD_ERR_INVALID_ARG, "vertex-face terms need vf_rest");
+    if (t->vf_n > 0 && !t->vf && t->vf_n != c->vfs.n)
+      return fail(c, MAD_ERR_INVALID_ARG,
+                  "vf is NULL but vf_n is not the size of the set installed by mad_add_vf");
   }
   if (t->flags & ~(uint32_t)(MAD_EVAL_FULL_STENCIL_AD | MAD_EVAL_EDGE_SCATTER |
                              MAD_EVAL_PATCH_STAGED | MAD_EVAL_GENERIC_AD))
@@ -542,6 +546,20 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     CREATE_CK(dev_alloc(c, &c->pe_pid, sizeof(int32_t) * pe));
     CREATE_CK(dev_alloc(c, &c->status, sizeof(int32_t)));
     CREATE_CK(cudaMemsetAsync(c->status, 0, sizeof(int32_t), s));
+    // vertex-face term sets: each term takes three pairs of the pair capacity
+    VfSet& vs = c->vfs;
+    vs.max_terms = c->max_pairs / 3;
+    const size_t mt = (size_t)vs.max_terms;
+    CREATE_CK(dev_alloc(c, &vs.terms, sizeof(int32_t) * 2 * std::max<size_t>(mt, 1)));
+    CREATE_CK(dev_alloc(c, &vs.pairs, sizeof(int32_t) * 6 * std::max<size_t>(mt, 1)));
+    char* zr = nullptr;
+    CREATE_CK(dev_alloc(c, &zr, (size_t)c->esz * 3 * std::max<size_t>(mt, 1)));
+    CREATE_CK(cudaMemsetAsync(zr, 0, (size_t)c->esz * 3 * std::max<size_t>(mt, 1), s));
+    vs.zero_rest = zr;
+    CREATE_CK(dev_alloc(c, &vs.vrow, sizeof(int32_t) * (V + 1)));
+    CREATE_CK(dev_alloc(c, &vs.ent, sizeof(int32_t) * 32 * std::max<size_t>(mt, 1)));
+    CREATE_CK(dev_alloc(c, &vs.scan_tmp, sizeof(int32_t) * scan_tmp_elems(V)));
+    CREATE_CK(dev_alloc(c, &vs.epart, sizeof(double) * (size_t)std::max(1, (V + 255) / 256)));
   }
   c->device_bytes += (int64_t)sizeof(int32_t) *
                      ((V + 1) + 2 * (int64_t)c->nnzb_base + V + 2 * (int64_t)c->E);
@@ -607,7 +625,11 @@ mad_status mad_eval(mad_ctx* c, const void* x, const mad_terms* t, void* g, void
   }
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval launch");
   if ((t->mask & MAD_TERM_VF) && t->vf_n > 0) {
-    e = launch_vf_eval(c->dtype, vf_launch(c, t, x), g, H_vals, energy, as_stream(stream));
+    // t->vf given: one thread per term, atomics; else the installed set,
+    // gathered per row
+    e = t->vf ? launch_vf_eval(c->dtype, vf_launch(c, t, x), g, H_vals, energy, as_stream(stream))
+              : launch_vf_rows_eval(c->dtype, c->vfs, vf_launch(c, t, x), g, H_vals, energy,
+                                    as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval vertex-face launch");
   }
   return MAD_OK;
@@ -624,7 +646,8 @@ mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t, const void* v,
                               : launch_hvp(eval_launch(c), *t, x, v, y, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_hvp launch");
   if ((t->mask & MAD_TERM_VF) && t->vf_n > 0) {
-    e = launch_vf_hvp(c->dtype, vf_launch(c, t, x), v, y, as_stream(stream));
+    e = t->vf ? launch_vf_hvp(c->dtype, vf_launch(c, t, x), v, y, as_stream(stream))
+              : launch_vf_rows_hvp(c->dtype, c->vfs, vf_launch(c, t, x), v, y, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(c, e, "mad_hvp vertex-face launch");
   }
   return MAD_OK;
@@ -673,6 +696,7 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij, const void* r
   if (!c) return MAD_ERR_INVALID_ARG;
   if (n < 0) return fail(c, MAD_ERR_INVALID_ARG, "n < 0");
   if (n > c->max_pairs) return fail(c, MAD_ERR_CAPACITY, "n exceeds max_pairs");
+  c->vfs.n = -1;  // a new pair set drops the installed vertex-face terms
   if (n == 0) {
     c->active = -1;  // the mesh pattern, no pairs
     return MAD_OK;
@@ -697,6 +721,27 @@ mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij, const void* r
   cudaError_t e = launch_add_pairs(L, n, ij, rest, c->buf[next], prev, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_add_pairs launch");
   c->active = next;
+  return MAD_OK;
+}
+
+mad_status mad_add_vf(mad_ctx* c, int32_t n, const int32_t* vf, void* stream) {
+  if (!c) return MAD_ERR_INVALID_ARG;
+  if (n < 0) return fail(c, MAD_ERR_INVALID_ARG, "n < 0");
+  if (n > c->vfs.max_terms)
+    return fail(c, MAD_ERR_CAPACITY, "n exceeds max_pairs / 3 vertex-face terms");
+  if (n > 0 && !vf) return fail(c, MAD_ERR_INVALID_ARG, "vf must be a device pointer");
+  if (c->dof != 3) return fail(c, MAD_ERR_UNIMPLEMENTED, "vertex-face terms need dof 3");
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = launch_vf_install_expand(c->vfs, n, vf, c->V, c->F_dev, c->nF, s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "mad_add_vf launch");
+  // the terms' (vertex, corner) pairs become the pair set
+  mad_status st = mad_add_pairs(c, 3 * n, c->vfs.pairs, c->vfs.zero_rest, stream);
+  if (st != MAD_OK) return st;
+  const int32_t* rp = c->active < 0 ? c->pat.rp : c->buf[c->active].rp;
+  const int32_t* ci = c->active < 0 ? c->pat.ci : c->buf[c->active].ci;
+  e = launch_vf_install_tables(c->vfs, n, c->V, c->F_dev, c->nF, rp, ci, c->cnt, c->status, s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "mad_add_vf tables");
+  c->vfs.n = n;
   return MAD_OK;
 }
 

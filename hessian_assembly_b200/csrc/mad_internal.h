@@ -171,6 +171,28 @@ struct VfLaunch {
 };
 cudaError_t launch_vf_eval(int dtype, const VfLaunch& L, void* g, void* H, double* energy,
                            cudaStream_t s);
+// An installed vertex-face term set (mad_add_vf): the terms, their pairs for
+// the insertion and the per-row incidence tables of the gather form (vf.cu).
+struct VfSet {
+  int max_terms = 0;        // largest set (max_pairs / 3)
+  int n = -1;               // installed terms; -1: none installed
+  int32_t* terms = nullptr; // [max_terms][2] (vertex p, face f)
+  int32_t* pairs = nullptr; // [3 max_terms][2] (p, corner) for the insertion
+  void* zero_rest = nullptr;// [3 max_terms] zeros in the dtype (rest of those pairs)
+  int32_t* vrow = nullptr;  // [V+1] incidences per row (exclusive scan)
+  int32_t* ent = nullptr;   // [4 max_terms][8] entries (see vf.cu)
+  int32_t* scan_tmp = nullptr;
+  double* epart = nullptr;  // [ceil(V / 256)] per-block energy
+};
+cudaError_t launch_vf_install_expand(const VfSet& S, int n, const int32_t* vf, int V,
+                                     const int32_t* F, int nF, cudaStream_t s);
+cudaError_t launch_vf_install_tables(const VfSet& S, int n, int V, const int32_t* F, int nF,
+                                     const int32_t* rp, const int32_t* ci, int32_t* cnt,
+                                     int32_t* status, cudaStream_t s);
+cudaError_t launch_vf_rows_eval(int dtype, const VfSet& S, const VfLaunch& L, void* g, void* H,
+                                double* energy, cudaStream_t s);
+cudaError_t launch_vf_rows_hvp(int dtype, const VfSet& S, const VfLaunch& L, const void* v,
+                               void* y, cudaStream_t s);
 cudaError_t launch_vf_hvp(int dtype, const VfLaunch& L, const void* v, void* y, cudaStream_t s);
 
 // ---- launchers (defined in the .cu files) ------------------------------

@@ -238,7 +238,349 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_hvp(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Installed term sets (mad_add_vf): the gather form.  Every term is listed in
+// the rows of its four vertices; one thread per row evaluates the row's
+// terms and adds only the row's share (its gradient and its four blocks) to
+// g and H, which the row kernel has just written.  No two threads touch the
+// same row, so no atomics are needed and the sums are reproducible.
+//
+// Entry of row i (32 bytes): term t and role r (which stencil vertex i is:
+// p, a, b or c) packed as t | r << 30, then the block positions of the
+// stencil's four vertices p, a, b, c in row i of the active pattern (-1:
+// missing, the entry is skipped).
+
+__device__ __forceinline__ bool vf_term(int t, const int32_t* __restrict__ terms,
+                                        const int32_t* __restrict__ F, int nF, int V,
+                                        int vid[4]) {
+  const int p = terms[2 * t], f = terms[2 * t + 1];
+  if (p < 0 || p >= V || f < 0 || f >= nF) return false;
+  vid[0] = p;
+  vid[1] = F[3 * f];
+  vid[2] = F[3 * f + 1];
+  vid[3] = F[3 * f + 2];
+  return p != vid[1] && p != vid[2] && p != vid[3];
+}
+
+// the terms' (vertex, corner) pairs for the insertion, and a copy of the terms
+__global__ void __launch_bounds__(kVfThreads) k_vf_expand(int n, const int32_t* __restrict__ vf,
+                                                          const int32_t* __restrict__ F, int nF,
+                                                          int V, int32_t* pairs,
+                                                          int32_t* terms) {
+  const int t = blockIdx.x * kVfThreads + threadIdx.x;
+  if (t >= n) return;
+  const int p = vf[2 * t], f = vf[2 * t + 1];
+  terms[2 * t] = p;
+  terms[2 * t + 1] = f;
+  int vid[4];
+  const bool ok = vf_term(t, terms, F, nF, V, vid);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {  // a bad term gives pairs the insertion rejects
+    pairs[2 * (3 * t + c)] = ok ? p : -1;
+    pairs[2 * (3 * t + c) + 1] = ok ? vid[1 + c] : -1;
+  }
+}
+
+__global__ void __launch_bounds__(kVfThreads) k_vf_count(int n, const int32_t* __restrict__ terms,
+                                                         const int32_t* __restrict__ F, int nF,
+                                                         int V, int32_t* cnt) {
+  const int t = blockIdx.x * kVfThreads + threadIdx.x;
+  int vid[4];
+  if (t >= n || !vf_term(t, terms, F, nF, V, vid)) return;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) atomicAdd(&cnt[vid[r]], 1);
+}
+
+// each incidence takes a slot of its row, counting the row counter back to 0
+__global__ void __launch_bounds__(kVfThreads) k_vf_fill(int n, const int32_t* __restrict__ terms,
+                                                        const int32_t* __restrict__ F, int nF,
+                                                        int V, const int32_t* __restrict__ vrow,
+                                                        int32_t* cnt, int32_t* ent) {
+  const int t = blockIdx.x * kVfThreads + threadIdx.x;
+  int vid[4];
+  if (t >= n || !vf_term(t, terms, F, nF, V, vid)) return;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int slot = vrow[vid[r]] + atomicSub(&cnt[vid[r]], 1) - 1;
+    ent[8 * slot] = t | (r << 30);
+  }
+}
+
+// per row: entries in (term, role) order, then the block positions
+__global__ void __launch_bounds__(kVfThreads) k_vf_finalize(
+    int V, const int32_t* __restrict__ vrow, int32_t* ent, const int32_t* __restrict__ terms,
+    const int32_t* __restrict__ F, int nF, const int32_t* __restrict__ rp,
+    const int32_t* __restrict__ ci, int32_t* status) {
+  const int i = blockIdx.x * kVfThreads + threadIdx.x;
+  if (i >= V) return;
+  const int b = vrow[i], e = vrow[i + 1];
+  for (int q = b + 1; q < e; ++q) {  // insertion sort: rows hold few entries
+    const int32_t key = ent[8 * q];
+    int j = q - 1;
+    while (j >= b && ent[8 * j] > key) {
+      ent[8 * (j + 1)] = ent[8 * j];
+      --j;
+    }
+    ent[8 * (j + 1)] = key;
+  }
+  const int r0 = rp[i];
+  for (int q = b; q < e; ++q) {
+    const int t = ent[8 * q] & 0x3FFFFFFF;
+    int vid[4];
+    vf_term(t, terms, F, nF, V, vid);
+    int4 w = make_int4(0, 0, 0, 0);
+    bool all = true;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int pos = find_col(rp, ci, i, vid[k]);
+      all &= pos >= 0;
+      const int rel = pos < 0 ? -1 : pos - r0;
+      if (k < 3) (k == 0 ? w.x : k == 1 ? w.y : w.z) = rel;
+      else w.w = rel;
+    }
+    if (!all) atomicOr(status, kStatusIndex);
+    reinterpret_cast<int4*>(ent)[2 * q] = make_int4(ent[8 * q], w.x, w.y, w.z);
+    reinterpret_cast<int4*>(ent)[2 * q + 1] = make_int4(w.w, all ? 1 : 0, 0, 0);
+  }
+}
+
+// one row's share of one term: gradient gi, blocks (role, j) for j = 0..3
+template <typename T, typename Z>
+__device__ __forceinline__ void vf_row_share(const Z& z, int role, T gi[3], T blk[4][9]) {
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
+    if (rr != role) continue;
+#pragma unroll
+    for (int al = 0; al < 3; ++al) {
+      T s = T(-0.0);
+#pragma unroll
+      for (int sv = 0; sv < 3; ++sv)
+        if (vf_coef(rr, sv) != 0) s += T(vf_coef(rr, sv)) * sgrad(z, 3 * sv + al);
+      gi[al] = s;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int al = 0; al < 3; ++al)
+#pragma unroll
+        for (int be = 0; be < 3; ++be) {
+          T s = T(-0.0);
+#pragma unroll
+          for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+            for (int tv = 0; tv < 3; ++tv)
+              if (vf_coef(rr, sv) * vf_coef(j, tv) != 0)
+                s += T(vf_coef(rr, sv) * vf_coef(j, tv)) * shess(z, 3 * sv + al, 3 * tv + be);
+          blk[j][3 * al + be] = s;
+        }
+  }
+}
+
+template <typename T, bool GEN>
+__global__ void __launch_bounds__(kVfThreads) k_vf_rows(
+    int V, const int32_t* __restrict__ vrow, const int32_t* __restrict__ ent,
+    const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF,
+    const T* __restrict__ rest, T k, const T* __restrict__ x, const int32_t* __restrict__ rp,
+    T* __restrict__ g, T* __restrict__ H, double* epart) {
+  const int i = blockIdx.x * kVfThreads + threadIdx.x;
+  double e = 0.0;
+  if (i < V) {
+    const int b = vrow[i], en = vrow[i + 1];
+    if (en > b) {
+      const int64_t r0 = rp[i];
+      T gacc[3] = {T(0), T(0), T(0)};
+      for (int q = b; q < en; ++q) {
+        const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
+        const int4 w1 = reinterpret_cast<const int4*>(ent)[2 * q + 1];
+        if (!w1.y) continue;
+        const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
+        int vid[4];
+        vf_term(t, terms, F, nF, V, vid);
+        T X[4][3];
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+#pragma unroll
+          for (int al = 0; al < 3; ++al) X[v4][al] = x[(int64_t)vid[v4] * 3 + al];
+        const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
+        e += 0.25 * (double)z.v;
+        T gi[3], blk[4][9];
+        vf_row_share<T>(z, role, gi, blk);
+#pragma unroll
+        for (int al = 0; al < 3; ++al) gacc[al] += gi[al];
+        const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          T* hb = H + (r0 + pos[j]) * 9;
+#pragma unroll
+          for (int q9 = 0; q9 < 9; ++q9) hb[q9] += blk[j][q9];
+        }
+      }
+#pragma unroll
+      for (int al = 0; al < 3; ++al) g[(int64_t)i * 3 + al] += gacc[al];
+    }
+  }
+  if (epart) {
+    __shared__ double red[kVfThreads / 32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e += __shfl_down_sync(0xFFFFFFFFu, e, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = e;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double s2 = 0.0;
+      for (int w = 0; w < kVfThreads / 32; ++w) s2 += red[w];
+      epart[blockIdx.x] = s2;
+    }
+  }
+}
+
+template <typename T, bool GEN>
+__global__ void __launch_bounds__(kVfThreads) k_vf_rows_hvp(
+    int V, const int32_t* __restrict__ vrow, const int32_t* __restrict__ ent,
+    const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF,
+    const T* __restrict__ rest, T k, const T* __restrict__ x, const T* __restrict__ v,
+    T* __restrict__ y) {
+  const int i = blockIdx.x * kVfThreads + threadIdx.x;
+  if (i >= V) return;
+  const int b = vrow[i], en = vrow[i + 1];
+  if (en <= b) return;
+  T yacc[3] = {T(0), T(0), T(0)};
+  for (int q = b; q < en; ++q) {
+    const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
+    const int4 w1 = reinterpret_cast<const int4*>(ent)[2 * q + 1];
+    if (!w1.y) continue;
+    const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
+    int vid[4];
+    vf_term(t, terms, F, nF, V, vid);
+    T X[4][3], W[4][3];
+#pragma unroll
+    for (int v4 = 0; v4 < 4; ++v4)
+#pragma unroll
+      for (int al = 0; al < 3; ++al) {
+        X[v4][al] = x[(int64_t)vid[v4] * 3 + al];
+        W[v4][al] = v[(int64_t)vid[v4] * 3 + al];
+      }
+    const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
+    T dz[9];
+#pragma unroll
+    for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+      for (int al = 0; al < 3; ++al) {
+        T s = T(-0.0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (vf_coef(j, sv) != 0) s += T(vf_coef(j, sv)) * W[j][al];
+        dz[3 * sv + al] = s;
+      }
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      if (rr != role) continue;
+#pragma unroll
+      for (int al = 0; al < 3; ++al) {
+        T s = T(-0.0);
+#pragma unroll
+        for (int sv = 0; sv < 3; ++sv) {
+          if (vf_coef(rr, sv) == 0) continue;
+          T tq = T(-0.0);
+#pragma unroll
+          for (int w = 0; w < 9; ++w) tq += shess(z, 3 * sv + al, w) * dz[w];
+          s += T(vf_coef(rr, sv)) * tq;
+        }
+        yacc[al] += s;
+      }
+    }
+  }
+#pragma unroll
+  for (int al = 0; al < 3; ++al) y[(int64_t)i * 3 + al] += yacc[al];
+}
+
+__global__ void k_energy_add(const double* __restrict__ part, int n, double* out) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += part[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    *out += t;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_vf_install_expand(const VfSet& S, int n, const int32_t* vf, int V,
+                                     const int32_t* F, int nF, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const unsigned nb = (unsigned)((n + kVfThreads - 1) / kVfThreads);
+  k_vf_expand<<<nb, kVfThreads, 0, s>>>(n, vf, F, nF, V, S.pairs, S.terms);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vf_install_tables(const VfSet& S, int n, int V, const int32_t* F, int nF,
+                                     const int32_t* rp, const int32_t* ci, int32_t* cnt,
+                                     int32_t* status, cudaStream_t s) {
+  cudaError_t e;
+  const unsigned nb = (unsigned)((n + kVfThreads - 1) / kVfThreads);
+  const unsigned nr = (unsigned)((V + kVfThreads - 1) / kVfThreads);
+  if (n > 0) {
+    k_vf_count<<<nb, kVfThreads, 0, s>>>(n, S.terms, F, nF, V, cnt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = scan_exclusive(cnt, S.vrow, V, S.scan_tmp, s)) != cudaSuccess) return e;
+  if (n > 0) {
+    k_vf_fill<<<nb, kVfThreads, 0, s>>>(n, S.terms, F, nF, V, S.vrow, cnt, S.ent);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_vf_finalize<<<nr, kVfThreads, 0, s>>>(V, S.vrow, S.ent, S.terms, F, nF, rp, ci, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+template <typename T, bool GEN>
+void vf_rows_t(const VfSet& S, const VfLaunch& L, void* g, void* H, double* energy,
+               cudaStream_t s) {
+  const unsigned nr = (unsigned)((L.V + kVfThreads - 1) / kVfThreads);
+  k_vf_rows<T, GEN><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, S.terms, L.F, L.nF,
+                                              (const T*)L.rest, (T)L.k, (const T*)L.x, L.rp,
+                                              (T*)g, (T*)H, energy ? S.epart : nullptr);
+  if (energy) k_energy_add<<<1, 1024, 0, s>>>(S.epart, (int)nr, energy);
+}
+
+template <typename T, bool GEN>
+void vf_rows_hvp_t(const VfSet& S, const VfLaunch& L, const void* v, void* y, cudaStream_t s) {
+  const unsigned nr = (unsigned)((L.V + kVfThreads - 1) / kVfThreads);
+  k_vf_rows_hvp<T, GEN><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, S.terms, L.F, L.nF,
+                                                  (const T*)L.rest, (T)L.k, (const T*)L.x,
+                                                  (const T*)v, (T*)y);
+}
+
+cudaError_t launch_vf_rows_eval(int dtype, const VfSet& S, const VfLaunch& L, void* g, void* H,
+                                double* energy, cudaStream_t s) {
+  if (L.V <= 0) return cudaSuccess;
+  if (dtype == MAD_F64) {
+    if (L.generic) vf_rows_t<double, true>(S, L, g, H, energy, s);
+    else vf_rows_t<double, false>(S, L, g, H, energy, s);
+  } else {
+    if (L.generic) vf_rows_t<float, true>(S, L, g, H, energy, s);
+    else vf_rows_t<float, false>(S, L, g, H, energy, s);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vf_rows_hvp(int dtype, const VfSet& S, const VfLaunch& L, const void* v,
+                               void* y, cudaStream_t s) {
+  if (L.V <= 0) return cudaSuccess;
+  if (dtype == MAD_F64) {
+    if (L.generic) vf_rows_hvp_t<double, true>(S, L, v, y, s);
+    else vf_rows_hvp_t<double, false>(S, L, v, y, s);
+  } else {
+    if (L.generic) vf_rows_hvp_t<float, true>(S, L, v, y, s);
+    else vf_rows_hvp_t<float, false>(S, L, v, y, s);
+  }
+  return cudaGetLastError();
+}
 
 template <typename T, bool GEN>
 void vf_eval_t(const VfLaunch& L, unsigned nb, void* g, void* H, double* energy, cudaStream_t s) {

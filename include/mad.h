@@ -83,13 +83,15 @@ enum {
                             closest rotation is unique there).              */
   MAD_TERM_VF = 64u      /* per vertex-face term (dof 3): 1/2 k_c (d - r)^2,
                             d the signed distance of vertex p to the plane of
-                            face f (n = (x1-x0) x (x2-x0)).  The blocks
-                            between p and the face's corners must be in the
-                            pattern: insert the pairs (p, corner) of every
-                            term with mad_add_pairs.  Not with MAD_TERM_PAIR
-                            (its pair list would hold those pairs too).
-                            Terms are added with atomics, so their blocks
-                            are not bit-reproducible across runs.           */
+                            face f (n = (x1-x0) x (x2-x0)).  Either install
+                            the terms with mad_add_vf and pass t->vf = NULL
+                            (gathered per row: reproducible), or insert the
+                            pairs (p, corner) of every term with
+                            mad_add_pairs and pass the terms in t->vf (one
+                            thread per term adds with atomics, so the
+                            blocks are not bit-reproducible across runs).
+                            Not with MAD_TERM_PAIR (its pair list would hold
+                            those pairs too).                               */
 };
 
 /* Evaluation flags. */
@@ -152,7 +154,8 @@ typedef struct {
   double pair_k;            /* k_p for the current pair set                  */
   double area_k;            /* k_a of MAD_TERM_AREA                          */
   int32_t vf_n;             /* number of vertex-face terms (MAD_TERM_VF)     */
-  const int32_t* vf;        /* [vf_n][2] (vertex p, face f) per term         */
+  const int32_t* vf;        /* [vf_n][2] (vertex p, face f) per term, or NULL
+                               for the set installed by mad_add_vf          */
   const void* vf_rest;      /* [vf_n] rest offset r per term                 */
   double vf_k;              /* k_c of MAD_TERM_VF                            */
 } mad_terms;
@@ -253,6 +256,25 @@ mad_status mad_hvp(mad_ctx* c, const void* x, const mad_terms* t,
  * (n > max_pairs).                                                         */
 mad_status mad_add_pairs(mad_ctx* c, int32_t n, const int32_t* ij,
                          const void* rest, void* stream);
+
+/* Install a set of vertex-face terms (MAD_TERM_VF) on the GPU (section 方法,
+ * key design 4: runtime terms are discovered apart from their evaluation,
+ * and their new blocks are inserted in parallel on the GPU).
+ *   n   number of terms, 0 <= n <= max_pairs / 3
+ *   vf  DEVICE [n][2] (vertex p, face f) per term
+ * Replaces the pair set with the terms' 3n (p, corner) pairs (as
+ * mad_add_pairs would) and builds, on the GPU, the list of the terms that
+ * touch each row with their blocks' positions.  mad_eval and mad_hvp with
+ * MAD_TERM_VF and t->vf == NULL then evaluate the installed terms: t->vf_n
+ * must equal n, t->vf_rest [n] and t->vf_k are read per call.  Each row's
+ * thread adds its own share of its terms (gradient and blocks), so the
+ * results need no atomics and are reproducible run to run.  A later
+ * mad_add_pairs drops the installed set.  A term with an index out of range
+ * or a vertex that is a corner of its face is skipped and sets
+ * MAD_ERR_INDEX in the device status.  Stream-ordered, no allocation.
+ * Errors: MAD_ERR_INVALID_ARG, MAD_ERR_CAPACITY (n > max_pairs / 3),
+ * MAD_ERR_UNIMPLEMENTED (dof 2), MAD_ERR_CUDA.                              */
+mad_status mad_add_vf(mad_ctx* c, int32_t n, const int32_t* vf, void* stream);
 
 /* ---- vector-valued objective: residuals and sparse Jacobian -------------
  * Section 方法: a vector-valued objective assembles the sparse Jacobian

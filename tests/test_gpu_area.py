@@ -66,6 +66,11 @@ def test_area_cloth_300x300_fp32(orc):
     check(orc, 300, "float32")
 
 
+def test_area_cloth_1000x1000_fp32(orc):
+    # the timed configuration (springs + inertia + area on the 1000^2 cloth)
+    check(orc, 1000, "float32", seed=1007)
+
+
 def test_area_cloth_300x300_fp32_generic_ad(orc):
     check(orc, 300, "float32", flags=GEN, seed=5003)
 

@@ -99,3 +99,111 @@ def test_vf_refusals():
     t = mad.Terms(mask=VF, vf=to_dev(vf), vf_rest=to_dev(rest, "float32"), vf_k=1.0)
     ctx.mad_eval(x, t, g, H)
     assert ctx.mad_status_sync() == mad.MAD_ERR_INDEX
+
+
+# ---- installed sets (mad_add_vf): gathered per row, no atomics -------------
+
+def check_installed(orc, n, dtype, nvf, seed, mask=1 | 2 | VF, flags=0, vf=None, rest=None):
+    import hessian_assembly_b200 as mad
+    import torch
+    if vf is None:
+        vf, rest, _ = vf_terms_for(n, nvf, seed)
+    st = mi.cloth_static(n, np.float64)
+    pairs = mi.vf_pairs(vf, st["F"])
+    ctx, st = cloth_context(n, dtype, max_pairs=3 * len(vf) + 8, slack=0.6)
+    ctx.mad_add_vf(to_dev(vf))
+    assert ctx.mad_status_sync() == mad.MAD_OK
+    x = mi.cloth_x(n, seed, 0, np.dtype(dtype))
+    x = (x + 0.02 * mi.grid_spacing(n) * np.random.default_rng(seed + 1).standard_normal(x.shape)
+         ).astype(dtype)
+    terms = mad.Terms(mask=mask, flags=flags, spring_rest=to_dev(st["L0"], dtype),
+                      spring_k=st["k"], inertia_xt=to_dev(st["xt"], dtype), inertia_w=st["w"],
+                      vf=None, vf_rest=to_dev(rest, dtype), vf_k=KC)
+    g, H, E = run_eval(ctx, x, terms, dtype)
+    assert ctx.mad_status_sync() == mad.MAD_OK
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(st["V"], st["F"], pairs)
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    og, oH, oE = orc.eval(st["V"], 3, x, mask, orp, oci, edges=st["edges"], L0=st["L0"],
+                          k=st["k"], xt=st["xt"], w=st["w"], F=st["F"], vf=vf,
+                          vf_rest=rest.astype(dtype), kc=KC)
+    assert_close("g", g, og, dtype)
+    assert_close("H", H[:nnzb], oH, dtype)
+    assert abs(E - oE) <= ETOL[dtype] * abs(oE)
+    v = mi.probe_vector(st["V"], 3, seed + 2, np.dtype(dtype))
+    y = torch.full((st["V"], 3), float("nan"), dtype=getattr(torch, dtype), device="cuda")
+    ctx.mad_hvp(to_dev(x, dtype), terms, to_dev(v, dtype), y)
+    torch.cuda.synchronize()
+    assert_close("y", y.cpu().numpy(), orc.bsr_mv(st["V"], 3, orp, oci, oH, v), dtype)
+    return ctx, x, terms, g, H
+
+
+@pytest.mark.parametrize("dtype", ["float32", "float64"])
+@pytest.mark.parametrize("flags", [0, 8])
+def test_vf_installed_cloth(orc, dtype, flags):
+    check_installed(orc, 30, dtype, 200, 6101, flags=flags)
+
+
+def test_vf_installed_only_terms(orc):
+    check_installed(orc, 20, "float64", 120, 6102, mask=VF)
+
+
+def test_vf_installed_1000x1000_benched_size(orc):
+    # the timed configuration: 10^5 terms on the 1000^2 cloth
+    n = 1000
+    vf = mi.random_vf(n, 100_000, 1009, 0)
+    rest = 0.001 * np.random.default_rng(1010).standard_normal(len(vf))
+    check_installed(orc, n, "float32", 0, 6103, vf=vf, rest=rest)
+
+
+def test_vf_installed_is_reproducible():
+    n = 60
+    vf, rest, _ = vf_terms_for(n, 900, 6104)
+    import hessian_assembly_b200 as mad
+    ctx, st = cloth_context(n, "float32", max_pairs=3 * len(vf) + 8, slack=0.6)
+    ctx.mad_add_vf(to_dev(vf))
+    x = mi.cloth_x(n, 6104, 0, np.float32)
+    terms = mad.Terms(mask=1 | 2 | VF, spring_rest=to_dev(st["L0"], "float32"), spring_k=st["k"],
+                      inertia_xt=to_dev(st["xt"], "float32"), inertia_w=st["w"],
+                      vf_rest=to_dev(rest, "float32"), vf_k=KC)
+    g1, H1, E1 = run_eval(ctx, x, terms, "float32")
+    g2, H2, E2 = run_eval(ctx, x, terms, "float32")
+    _, _, nnzb = gpu_pattern(ctx)
+    assert np.array_equal(g1, g2) and np.array_equal(H1[:nnzb], H2[:nnzb]) and E1 == E2
+
+
+def test_vf_installed_bad_terms_and_replacement(orc):
+    import hessian_assembly_b200 as mad
+    n = 16
+    vf, rest, _ = vf_terms_for(n, 40, 6105)
+    st = mi.cloth_static(n, np.float64)
+    bad = vf.copy()
+    bad[3, 0] = st["F"][bad[3, 1]][0]   # the vertex is a corner of its face
+    bad[7, 1] = len(st["F"])            # face index out of range
+    good = np.ones(len(vf), bool)
+    good[[3, 7]] = False
+    ctx, st = cloth_context(n, "float64", max_pairs=3 * len(vf) + 8, slack=0.6)
+    ctx.mad_add_vf(to_dev(bad))
+    assert ctx.mad_status_sync() == mad.MAD_ERR_INDEX
+    x = mi.cloth_x(n, 6105, 0, np.float64)
+    terms = mad.Terms(mask=VF, vf_rest=to_dev(rest), vf_k=KC)
+    g, H, E = run_eval(ctx, x, terms, "float64")
+    # the skipped terms' pairs are not in the pattern; the others evaluate as a set of their own
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(st["V"], st["F"], mi.vf_pairs(vf[good], st["F"]))
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    og, oH, oE = orc.eval(st["V"], 3, x, VF, orp, oci, F=st["F"], vf=vf[good],
+                          vf_rest=rest[good], kc=KC)
+    assert_close("g", g, og, "float64")
+    assert_close("H", H[:nnzb], oH, "float64")
+    # a new pair set drops the installed terms: vf = NULL is refused
+    ctx.mad_add_pairs(to_dev(np.array([[0, 5]], np.int32)), to_dev(np.ones(1)))
+    with pytest.raises(mad.MadError) as ei:
+        run_eval(ctx, x, terms, "float64")
+    assert ei.value.status == mad.MAD_ERR_INVALID_ARG
+    # more terms than max_pairs / 3
+    with pytest.raises(mad.MadError) as ei:
+        ctx.mad_add_vf(to_dev(np.zeros((len(vf) + 10, 2), np.int32)))
+    assert ei.value.status == mad.MAD_ERR_CAPACITY
