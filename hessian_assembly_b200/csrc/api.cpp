@@ -64,6 +64,7 @@ struct mad_ctx {
   int32_t* rows_fcslots = nullptr;
   int32_t* rows_fcofl = nullptr;
   void* face_hv = nullptr;  // [nF][3][2] scratch of the face Hessian-vector product
+  void* face_rec = nullptr; // [nF][16] J-space records of the dof-2 face pass
   double* epart = nullptr;
   size_t smem_eval = 0, smem_hvp = 0;
   // dynamic pattern
@@ -195,6 +196,7 @@ RowsLaunch rows_launch(const mad_ctx* c) {
   L.nF = c->nF;
   L.F = c->F_dev;
   L.fhv = c->face_hv;
+  L.frec = c->face_rec;
   L.epart = c->epart;
   if (c->active < 0) {
     L.rp = c->pat.rp;
@@ -477,6 +479,11 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
         char* hv = nullptr;
         CREATE_CK(dev_alloc(c, &hv, (size_t)c->esz * 3 * dof * (size_t)nF));
         c->face_hv = hv;
+        if (dof == 2) {  // the face pass's J-space records (16 values per face)
+          char* rec = nullptr;
+          CREATE_CK(dev_alloc(c, &rec, (size_t)c->esz * 16 * (size_t)nF));
+          c->face_rec = rec;
+        }
       }
     }
   }
@@ -559,7 +566,11 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     CREATE_CK(dev_alloc(c, &vs.vrow, sizeof(int32_t) * (V + 1)));
     CREATE_CK(dev_alloc(c, &vs.ent, sizeof(int32_t) * 32 * std::max<size_t>(mt, 1)));
     CREATE_CK(dev_alloc(c, &vs.scan_tmp, sizeof(int32_t) * scan_tmp_elems(V)));
-    CREATE_CK(dev_alloc(c, &vs.epart, sizeof(double) * (size_t)std::max(1, (V + 255) / 256)));
+    CREATE_CK(dev_alloc(c, &vs.epart,
+                        sizeof(double) * std::max<size_t>(1, (mt + 255) / 256)));
+    char* rec = nullptr;
+    CREATE_CK(dev_alloc(c, &rec, (size_t)c->esz * 56 * std::max<size_t>(mt, 1)));
+    vs.rec = rec;
   }
   c->device_bytes += (int64_t)sizeof(int32_t) *
                      ((V + 1) + 2 * (int64_t)c->nnzb_base + V + 2 * (int64_t)c->E);

@@ -182,7 +182,8 @@ struct VfSet {
   int32_t* vrow = nullptr;  // [V+1] incidences per row (exclusive scan)
   int32_t* ent = nullptr;   // [4 max_terms][8] entries (see vf.cu)
   int32_t* scan_tmp = nullptr;
-  double* epart = nullptr;  // [ceil(V / 256)] per-block energy
+  void* rec = nullptr;      // [max_terms][56] per-term records of the term pass
+  double* epart = nullptr;  // [ceil(max_terms / 256)] per-block energy of the term pass
 };
 cudaError_t launch_vf_install_expand(const VfSet& S, int n, const int32_t* vf, int V,
                                      const int32_t* F, int nF, cudaStream_t s);
@@ -283,6 +284,7 @@ struct RowsLaunch {
   int nF;
   const int32_t* F;        // [nF][3]
   void* fhv;               // [nF][3][2] per-face corner results of H v (scratch)
+  void* frec;              // [nF][16] per-face J-space records (dof 2; scratch)
   const int2* slots;
   const uint32_t* meta;
   const int32_t* ofl_ptr;

@@ -28,7 +28,6 @@
 //           every block instead copies its share of the previous pattern and
 //           pair set into the new buffer.
 #include "mad_internal.h"
-#include "pdl.cuh"
 
 namespace mad {
 namespace {
@@ -143,7 +142,6 @@ __device__ __forceinline__ int block_excl_scan(int v, int* total) {
 
 __global__ void __launch_bounds__(kB) k_pair_count(const int32_t* __restrict__ ij, int n, int V,
                                                    int32_t* cnt, int32_t* status) {
-  grid_dependents_may_launch();
   GRID_STRIDE(p, n) {
     const int32_t i = ij[2 * p], j = ij[2 * p + 1];
     if (!pair_ok(i, j, V)) {
@@ -159,8 +157,6 @@ __global__ void __launch_bounds__(kB) k_pair_count(const int32_t* __restrict__ i
 // kU*b .. kU*b + kU-1, thread t row t of each.
 __global__ void __launch_bounds__(kB) k_block_sums(const int32_t* __restrict__ cnt, int V,
                                                    int nunits, int32_t* blk, int32_t* sup) {
-  grid_dependents_may_launch();
-  grid_dependency_wait();  // the row counts
   const int64_t base = (int64_t)blockIdx.x * kU * kB + threadIdx.x;
   int4 x = make_int4(0, 0, 0, 0);
 #pragma unroll
@@ -188,8 +184,6 @@ __global__ void __launch_bounds__(kB) k_scan_rows(const int32_t* __restrict__ cn
                                                   const int32_t* __restrict__ sup,
                                                   const int32_t* __restrict__ blk,
                                                   int32_t* __restrict__ prow) {
-  grid_dependents_may_launch();
-  grid_dependency_wait();  // the block and super-tile counts
   const int U0 = blockIdx.x * kU, S = U0 / kSuper;
   const int64_t r0 = (int64_t)blockIdx.x * kU * kB + (int64_t)threadIdx.x * kU;
   int4 c = make_int4(0, 0, 0, 0);
@@ -229,8 +223,6 @@ __global__ void __launch_bounds__(kB) k_pair_fill(const int32_t* __restrict__ ij
                                                   int32_t* cnt, int32_t* pe_col,
                                                   int32_t* pe_pid, T* pe_rest,
                                                   const T* __restrict__ rest) {
-  grid_dependents_may_launch();
-  grid_dependency_wait();  // the row offsets
   GRID_STRIDE(p, n) {
     const int32_t i = ij[2 * p], j = ij[2 * p + 1];
     if (!pair_ok(i, j, V)) continue;
@@ -382,25 +374,18 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V, int nunits,
                                                   const T* __restrict__ rest, int32_t* newcnt,
                                                   int32_t* nblk, int32_t* nsupc) {
   __shared__ int s_unit[kU];
-  grid_dependents_may_launch();
   const int lane = threadIdx.x & 31;
   const int64_t base = (int64_t)blockIdx.x * kU * kB + threadIdx.x;
   int32_t b[kU], e[kU], r0[kU], r1[kU];
   unsigned has[kU];
-#pragma unroll
-  for (int u = 0; u < kU; ++u) {  // the mesh rows first: they do not wait
-    const int64_t v = base + (int64_t)u * kB;
-    const bool ok = v < V;
-    r0[u] = ok ? base_rp[v] : 0;
-    r1[u] = ok ? base_rp[v + 1] : 0;
-  }
-  grid_dependency_wait();  // the filled pair entries
 #pragma unroll
   for (int u = 0; u < kU; ++u) {
     const int64_t v = base + (int64_t)u * kB;
     const bool ok = v < V;
     b[u] = ok ? prow[v] : 0;
     e[u] = ok ? prow[v + 1] : 0;
+    r0[u] = ok ? base_rp[v] : 0;
+    r1[u] = ok ? base_rp[v + 1] : 0;
   }
   if (threadIdx.x < kU) s_unit[threadIdx.x] = 0;
   int total = 0;
@@ -489,10 +474,8 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
   const bool warp_live = g * 32 < nrows;
   const int gend = g * 32 + 32 < nrows ? g * 32 + 32 : nrows;
   // ---- round 1: row pointers, counts, pair offsets, the warp's column range
-  grid_dependents_may_launch();
   const int32_t b0 = valid ? base_rp[v] : 0x7FFFFFFF;
   const int32_t b1r = valid ? base_rp[v + 1] : 0x7FFFFFFF;
-  grid_dependency_wait();  // the merged rows and their new-block counts
   const int32_t nc0 = valid ? newcnt[v] : 0;
   const int32_t pr0 = valid ? prow[v] : 0;
   const int32_t pr1 = valid ? prow[v + 1] : 0;
@@ -701,31 +684,30 @@ cudaError_t add_pairs_t(const PairLaunch& L, int n, const int32_t* ij, const voi
   k_pair_count<<<grid_for(n), kB, 0, s>>>(ij, n, V, L.cnt, L.status);
   CK(cudaGetLastError());
   const int ngroups = (nblocks + kU - 1) / kU;
-  // the rest of the chain: each kernel starts during its predecessor's tail
-  // and waits for its results (pdl.cuh)
-  CK(launch_pdl(k_block_sums, dim3(ngroups), dim3(kB), 0, s, (const int32_t*)L.cnt, V, nblocks,
-                blk_c, sup_c));
-  CK(launch_pdl(k_scan_rows, dim3(ngroups), dim3(kB), 0, s, (const int32_t*)L.cnt, V,
-                (const int32_t*)sup_c, (const int32_t*)blk_c, nb.prow));
-  CK(launch_pdl(k_pair_fill<T>, dim3(grid_for(n)), dim3(kB), 0, s, ij, n, V,
-                (const int32_t*)nb.prow, L.cnt, nb.pe_col, L.pe_pid, (T*)nb.pe_rest,
-                (const T*)rest));
-  CK(launch_pdl(k_pair_rows<T>, dim3(ngroups), dim3(kB), 0, s, V, nblocks,
-                (const int32_t*)nb.prow, L.base_rp, L.base_ci, nb.pe_col, L.pe_pid, nb.pe_pos,
-                (T*)nb.pe_rest, (const T*)rest, L.newcnt, blk_n, sup_n));
-  const bool hp = prev != nullptr;
-  return launch_pdl(k_write_pattern<T>, dim3(nblocks), dim3(kB), 0, s, V, L.nnzb_base,
-                    L.capacity, L.base_rp, L.base_ci, (const int32_t*)L.newcnt, nsup,
-                    (const int32_t*)sup_n, (const int32_t*)blk_n, (const int32_t*)nb.prow,
-                    (const int32_t*)nb.pe_col, (const int32_t*)nb.pe_pos, nb.rp, nb.ci, nb.nnzb,
-                    L.status, hp ? (const int32_t*)prev->rp : L.base_rp,
-                    hp ? (const int32_t*)prev->ci : L.base_ci,
-                    hp ? (const int32_t*)prev->nnzb : L.base_nnzb_dev,
-                    hp ? (const int32_t*)prev->prow : nullptr,
-                    hp ? (const int32_t*)prev->pe_col : nullptr,
-                    hp ? (const int32_t*)prev->pe_pos : nullptr,
-                    hp ? (const T*)prev->pe_rest : nullptr, nb.prow, nb.pe_col, nb.pe_pos,
-                    (T*)nb.pe_rest);
+  k_block_sums<<<ngroups, kB, 0, s>>>(L.cnt, V, nblocks, blk_c, sup_c);
+  CK(cudaGetLastError());
+  k_scan_rows<<<ngroups, kB, 0, s>>>(L.cnt, V, sup_c, blk_c, nb.prow);
+  CK(cudaGetLastError());
+  k_pair_fill<T><<<grid_for(n), kB, 0, s>>>(ij, n, V, nb.prow, L.cnt, nb.pe_col, L.pe_pid,
+                                            (T*)nb.pe_rest, (const T*)rest);
+  CK(cudaGetLastError());
+  k_pair_rows<T><<<ngroups, kB, 0, s>>>(V, nblocks, nb.prow, L.base_rp, L.base_ci, nb.pe_col,
+                                        L.pe_pid, nb.pe_pos, (T*)nb.pe_rest, (const T*)rest,
+                                        L.newcnt, blk_n, sup_n);
+  CK(cudaGetLastError());
+  if (prev)
+    k_write_pattern<T><<<nblocks, kB, 0, s>>>(
+        V, L.nnzb_base, L.capacity, L.base_rp, L.base_ci, L.newcnt, nsup, sup_n, blk_n,
+        nb.prow, nb.pe_col, nb.pe_pos, nb.rp, nb.ci, nb.nnzb, L.status, prev->rp, prev->ci,
+        prev->nnzb, prev->prow, prev->pe_col, prev->pe_pos, (const T*)prev->pe_rest, nb.prow,
+        nb.pe_col, nb.pe_pos, (T*)nb.pe_rest);
+  else
+    k_write_pattern<T><<<nblocks, kB, 0, s>>>(
+        V, L.nnzb_base, L.capacity, L.base_rp, L.base_ci, L.newcnt, nsup, sup_n, blk_n,
+        nb.prow, nb.pe_col, nb.pe_pos, nb.rp, nb.ci, nb.nnzb, L.status, L.base_rp, L.base_ci,
+        L.base_nnzb_dev, nullptr, nullptr, nullptr, nullptr, nb.prow, nb.pe_col, nb.pe_pos,
+        (T*)nb.pe_rest);
+  return cudaGetLastError();
 }
 
 }  // namespace

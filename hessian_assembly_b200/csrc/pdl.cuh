@@ -4,8 +4,16 @@
 // the previous kernel on its stream has finished: its blocks are scheduled
 // once every block of the previous kernel has signalled (or exited), load
 // what does not depend on that kernel, and wait before reading its results.
-// The launch latency and ramp of a chain of dependent kernels then overlap
-// the tails of their predecessors.
+// The launch latency and ramp of a dependent kernel then overlap the tail of
+// its predecessor.
+//
+// Use it only for a kernel that reads (a) what its immediate predecessor
+// wrote, after grid_dependency_wait(), and (b) data written by work that had
+// finished before that predecessor started, i.e. a predecessor launched the
+// ordinary way.  After the wait, writes of a grid two steps back in a chain
+// of such launches were not visible: in a chain of five the third kernel
+// read stale row offsets from the first.  So every use here is one ordinary
+// launch followed by one programmatic launch.
 #pragma once
 
 #include <cuda_runtime.h>

@@ -549,6 +549,48 @@ __device__ __forceinline__ T sel3(int c, T a, T b, T d) {
   return c == 0 ? a : (c == 1 ? b : d);
 }
 
+// The share of corner i of a dof-2 face term given its value, gradient and
+// Hessian in J space (e, J in the face's own corner order): the corner
+// weights wr of i, j, k (rotated from those of corners 0, 1, 2) map
+// g_i[al] = sum_ga dE/dJ[al][ga] w_i[ga] and block (i, l)[al][be] =
+// sum_{ga,de} H_J[(al,ga),(be,de)] w_i[ga] w_l[de].
+template <typename T>
+__device__ __forceinline__ void project_face_row(const HyperDual<T, 4>& e, const T (&wr)[3][2],
+                                                 FaceRow<T>& o) {
+  o.E = e.v;
+#pragma unroll
+  for (int al = 0; al < 2; ++al) o.g[al] = e.g[2 * al] * wr[0][0] + e.g[2 * al + 1] * wr[0][1];
+  // q[al][be][de] = sum_ga H_J[(al,ga),(be,de)] w_i[ga]
+  T q[2][2][2];
+#pragma unroll
+  for (int al = 0; al < 2; ++al)
+#pragma unroll
+    for (int be = 0; be < 2; ++be)
+#pragma unroll
+      for (int de = 0; de < 2; ++de)
+        q[al][be][de] = hess(e, 2 * al + 0, 2 * be + de) * wr[0][0] +
+                        hess(e, 2 * al + 1, 2 * be + de) * wr[0][1];
+#pragma unroll
+  for (int l = 0; l < 3; ++l)
+#pragma unroll
+    for (int al = 0; al < 2; ++al)
+#pragma unroll
+      for (int be = 0; be < 2; ++be)
+        o.H[l][2 * al + be] = q[al][be][0] * wr[l][0] + q[al][be][1] * wr[l][1];
+}
+
+// the corner weights of i, j, k for the row of corner c of a face with Dm^-1 M
+template <typename T>
+__device__ __forceinline__ void rotated_weights(const T* M, int c, T (&wr)[3][2]) {
+  const T w[3][2] = {{-(M[0] + M[2]), -(M[1] + M[3])}, {M[0], M[1]}, {M[2], M[3]}};
+#pragma unroll
+  for (int ga = 0; ga < 2; ++ga) {
+    wr[0][ga] = sel3(c, w[0][ga], w[1][ga], w[2][ga]);
+    wr[1][ga] = sel3(c, w[1][ga], w[2][ga], w[0][ga]);
+    wr[2][ga] = sel3(c, w[2][ga], w[0][ga], w[1][ga]);
+  }
+}
+
 template <typename T, int AD, int KIND>
 __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const T* xk, int c,
                                                 const T* M, T A, FaceRow<T>& o) {
@@ -573,26 +615,7 @@ __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const 
       for (int ga = 0; ga < 2; ++ga) Jv[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
     }
     const HyperDual<T, 4> e = face2_hd<KIND, AD>(Jv, A);
-    o.E = e.v;
-#pragma unroll
-    for (int al = 0; al < 2; ++al) o.g[al] = e.g[2 * al] * wr[0][0] + e.g[2 * al + 1] * wr[0][1];
-    // q[al][be][de] = sum_ga H_J[(al,ga),(be,de)] w_i[ga]
-    T q[2][2][2];
-#pragma unroll
-    for (int al = 0; al < 2; ++al)
-#pragma unroll
-      for (int be = 0; be < 2; ++be)
-#pragma unroll
-        for (int de = 0; de < 2; ++de)
-          q[al][be][de] = hess(e, 2 * al + 0, 2 * be + de) * wr[0][0] +
-                          hess(e, 2 * al + 1, 2 * be + de) * wr[0][1];
-#pragma unroll
-    for (int l = 0; l < 3; ++l)
-#pragma unroll
-      for (int al = 0; al < 2; ++al)
-#pragma unroll
-        for (int be = 0; be < 2; ++be)
-          o.H[l][2 * al + be] = q[al][be][0] * wr[l][0] + q[al][be][1] * wr[l][1];
+    project_face_row<T>(e, wr, o);
   } else {
     // width-6 AD over (x_i, x_j, x_k)
     Lin<T, 6> ui[2], uj[2], uk[2];

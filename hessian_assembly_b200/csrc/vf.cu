@@ -23,6 +23,7 @@
 #include <stdint.h>
 
 #include "mad_internal.h"
+#include "pdl.cuh"
 #include "sparse_ad.cuh"
 
 namespace mad {
@@ -262,6 +263,39 @@ __device__ __forceinline__ bool vf_term(int t, const int32_t* __restrict__ terms
   return p != vid[1] && p != vid[2] && p != vid[3];
 }
 
+// N values at p (N a multiple of 4; p 16-byte aligned) in 16-byte accesses
+template <typename T, int N>
+__device__ __forceinline__ void store_rec(T* p, const T* r) {
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int q = 0; q < N; q += 4)
+      reinterpret_cast<float4*>(p)[q / 4] = make_float4(r[q], r[q + 1], r[q + 2], r[q + 3]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < N; q += 2) reinterpret_cast<double2*>(p)[q / 2] = make_double2(r[q], r[q + 1]);
+  }
+}
+template <typename T, int N>
+__device__ __forceinline__ void load_rec(const T* p, T* r) {
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int q = 0; q < N; q += 4) {
+      const float4 v4 = reinterpret_cast<const float4*>(p)[q / 4];
+      r[q] = v4.x;
+      r[q + 1] = v4.y;
+      r[q + 2] = v4.z;
+      r[q + 3] = v4.w;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < N; q += 2) {
+      const double2 v2 = reinterpret_cast<const double2*>(p)[q / 2];
+      r[q] = v2.x;
+      r[q + 1] = v2.y;
+    }
+  }
+}
+
 // the terms' (vertex, corner) pairs for the insertion, and a copy of the terms
 __global__ void __launch_bounds__(kVfThreads) k_vf_expand(int n, const int32_t* __restrict__ vf,
                                                           const int32_t* __restrict__ F, int nF,
@@ -344,80 +378,40 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_finalize(
   }
 }
 
-// one row's share of one term: gradient gi, blocks (role, j) for j = 0..3
-template <typename T, typename Z>
-__device__ __forceinline__ void vf_row_share(const Z& z, int role, T gi[3], T blk[4][9]) {
-#pragma unroll
-  for (int rr = 0; rr < 4; ++rr) {
-    if (rr != role) continue;
-#pragma unroll
-    for (int al = 0; al < 3; ++al) {
-      T s = T(-0.0);
-#pragma unroll
-      for (int sv = 0; sv < 3; ++sv)
-        if (vf_coef(rr, sv) != 0) s += T(vf_coef(rr, sv)) * sgrad(z, 3 * sv + al);
-      gi[al] = s;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int al = 0; al < 3; ++al)
-#pragma unroll
-        for (int be = 0; be < 3; ++be) {
-          T s = T(-0.0);
-#pragma unroll
-          for (int sv = 0; sv < 3; ++sv)
-#pragma unroll
-            for (int tv = 0; tv < 3; ++tv)
-              if (vf_coef(rr, sv) * vf_coef(j, tv) != 0)
-                s += T(vf_coef(rr, sv) * vf_coef(j, tv)) * shess(z, 3 * sv + al, 3 * tv + be);
-          blk[j][3 * al + be] = s;
-        }
-  }
-}
+// Term pass of an installed set: one thread per term differentiates it once
+// and writes its record: E, the gradient in z (9) and the packed Hessian in
+// z (45), padded to kVfRec values; the energies are summed per block.
+constexpr int kVfRec = 56;
+constexpr int kVfHz = 45;  // Tri<9>::size
 
 template <typename T, bool GEN>
-__global__ void __launch_bounds__(kVfThreads) k_vf_rows(
-    int V, const int32_t* __restrict__ vrow, const int32_t* __restrict__ ent,
-    const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF,
-    const T* __restrict__ rest, T k, const T* __restrict__ x, const int32_t* __restrict__ rp,
-    T* __restrict__ g, T* __restrict__ H, double* epart) {
-  const int i = blockIdx.x * kVfThreads + threadIdx.x;
+__global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
+    int n, const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF, int V,
+    const T* __restrict__ rest, T k, const T* __restrict__ x, T* __restrict__ rec,
+    double* epart) {
+  grid_dependents_may_launch();  // the row pass may start; it waits for the records
+  const int t = blockIdx.x * kVfThreads + threadIdx.x;
   double e = 0.0;
-  if (i < V) {
-    const int b = vrow[i], en = vrow[i + 1];
-    if (en > b) {
-      const int64_t r0 = rp[i];
-      T gacc[3] = {T(0), T(0), T(0)};
-      for (int q = b; q < en; ++q) {
-        const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
-        const int4 w1 = reinterpret_cast<const int4*>(ent)[2 * q + 1];
-        if (!w1.y) continue;
-        const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
-        int vid[4];
-        vf_term(t, terms, F, nF, V, vid);
-        T X[4][3];
+  int vid[4];
+  if (t < n && vf_term(t, terms, F, nF, V, vid)) {
+    T X[4][3];
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
+    for (int v4 = 0; v4 < 4; ++v4)
 #pragma unroll
-          for (int al = 0; al < 3; ++al) X[v4][al] = x[(int64_t)vid[v4] * 3 + al];
-        const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
-        e += 0.25 * (double)z.v;
-        T gi[3], blk[4][9];
-        vf_row_share<T>(z, role, gi, blk);
+      for (int al = 0; al < 3; ++al) X[v4][al] = x[(int64_t)vid[v4] * 3 + al];
+    const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
+    e = (double)z.v;
+    T r[kVfRec];
+    r[0] = z.v;
 #pragma unroll
-        for (int al = 0; al < 3; ++al) gacc[al] += gi[al];
-        const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
+    for (int q = 0; q < 9; ++q) r[1 + q] = sgrad(z, q);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          T* hb = H + (r0 + pos[j]) * 9;
+    for (int a = 0; a < 9; ++a)
 #pragma unroll
-          for (int q9 = 0; q9 < 9; ++q9) hb[q9] += blk[j][q9];
-        }
-      }
+      for (int b = a; b < 9; ++b) r[10 + Tri<9>::idx(a, b)] = shess(z, a, b);
 #pragma unroll
-      for (int al = 0; al < 3; ++al) g[(int64_t)i * 3 + al] += gacc[al];
-    }
+    for (int q = 10 + kVfHz; q < kVfRec; ++q) r[q] = T(0);
+    store_rec<T, kVfRec>(rec + (int64_t)t * kVfRec, r);
   }
   if (epart) {
     __shared__ double red[kVfThreads / 32];
@@ -433,61 +427,142 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(
   }
 }
 
-template <typename T, bool GEN>
-__global__ void __launch_bounds__(kVfThreads) k_vf_rows_hvp(
-    int V, const int32_t* __restrict__ vrow, const int32_t* __restrict__ ent,
-    const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF,
-    const T* __restrict__ rest, T k, const T* __restrict__ x, const T* __restrict__ v,
-    T* __restrict__ y) {
+// Row pass: one thread per row adds its share of each of its terms (from the
+// records) to its gradient and its four blocks per term.
+template <typename T>
+__global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __restrict__ vrow,
+                                                        const int32_t* __restrict__ ent,
+                                                        const T* __restrict__ rec,
+                                                        const int32_t* __restrict__ rp,
+                                                        T* __restrict__ g, T* __restrict__ H) {
   const int i = blockIdx.x * kVfThreads + threadIdx.x;
   if (i >= V) return;
   const int b = vrow[i], en = vrow[i + 1];
   if (en <= b) return;
+  const int64_t r0 = rp[i];
+  grid_dependency_wait();  // the term pass's records
+  T gacc[3] = {T(0), T(0), T(0)};
+  for (int q = b; q < en; ++q) {
+    const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
+    const int4 w1 = reinterpret_cast<const int4*>(ent)[2 * q + 1];
+    if (!w1.y) continue;
+    const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
+    T r[kVfRec];
+    load_rec<T, kVfRec>(rec + (int64_t)t * kVfRec, r);
+    const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {  // the role as a compile-time index
+      if (rr != role) continue;
+#pragma unroll
+      for (int al = 0; al < 3; ++al) {
+        T s2 = T(-0.0);
+#pragma unroll
+        for (int sv = 0; sv < 3; ++sv)
+          if (vf_coef(rr, sv) != 0) s2 += T(vf_coef(rr, sv)) * r[1 + 3 * sv + al];
+        gacc[al] += s2;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        T* hb = H + (r0 + pos[j]) * 9;
+#pragma unroll
+        for (int al = 0; al < 3; ++al)
+#pragma unroll
+          for (int be = 0; be < 3; ++be) {
+            T s2 = T(-0.0);
+#pragma unroll
+            for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+              for (int tv = 0; tv < 3; ++tv) {
+                const int a = 3 * sv + al, c = 3 * tv + be;
+                if (vf_coef(rr, sv) * vf_coef(j, tv) != 0)
+                  s2 += T(vf_coef(rr, sv) * vf_coef(j, tv)) *
+                        r[10 + (a <= c ? Tri<9>::idx(a, c) : Tri<9>::idx(c, a))];
+              }
+            hb[3 * al + be] += s2;
+          }
+      }
+    }
+  }
+#pragma unroll
+  for (int al = 0; al < 3; ++al) g[(int64_t)i * 3 + al] += gacc[al];
+}
+
+// Product, term pass: each term's (H v) restricted to each of its four
+// vertices, written per role (12 values, padded to 16).
+constexpr int kVfHvRec = 16;
+template <typename T, bool GEN>
+__global__ void __launch_bounds__(kVfThreads) k_vf_term_hv(
+    int n, const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF, int V,
+    const T* __restrict__ rest, T k, const T* __restrict__ x, const T* __restrict__ v,
+    T* __restrict__ rec) {
+  grid_dependents_may_launch();
+  const int t = blockIdx.x * kVfThreads + threadIdx.x;
+  int vid[4];
+  if (t >= n || !vf_term(t, terms, F, nF, V, vid)) return;
+  T X[4][3], W[4][3];
+#pragma unroll
+  for (int v4 = 0; v4 < 4; ++v4)
+#pragma unroll
+    for (int al = 0; al < 3; ++al) {
+      X[v4][al] = x[(int64_t)vid[v4] * 3 + al];
+      W[v4][al] = v[(int64_t)vid[v4] * 3 + al];
+    }
+  const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
+  T dz[9];
+#pragma unroll
+  for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+    for (int al = 0; al < 3; ++al) {
+      T s2 = T(-0.0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (vf_coef(j, sv) != 0) s2 += T(vf_coef(j, sv)) * W[j][al];
+      dz[3 * sv + al] = s2;
+    }
+  T tz[9];
+#pragma unroll
+  for (int q = 0; q < 9; ++q) {
+    T s2 = shess(z, q, 0) * dz[0];
+#pragma unroll
+    for (int w = 1; w < 9; ++w) s2 += shess(z, q, w) * dz[w];
+    tz[q] = s2;
+  }
+  T r[kVfHvRec];
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+    for (int al = 0; al < 3; ++al) {
+      T s2 = T(-0.0);
+#pragma unroll
+      for (int sv = 0; sv < 3; ++sv)
+        if (vf_coef(rr, sv) != 0) s2 += T(vf_coef(rr, sv)) * tz[3 * sv + al];
+      r[3 * rr + al] = s2;
+    }
+#pragma unroll
+  for (int q = 12; q < kVfHvRec; ++q) r[q] = T(0);
+  store_rec<T, kVfHvRec>(rec + (int64_t)t * kVfHvRec, r);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kVfThreads) k_vf_rows_hvp(int V,
+                                                            const int32_t* __restrict__ vrow,
+                                                            const int32_t* __restrict__ ent,
+                                                            const T* __restrict__ rec,
+                                                            T* __restrict__ y) {
+  const int i = blockIdx.x * kVfThreads + threadIdx.x;
+  if (i >= V) return;
+  const int b = vrow[i], en = vrow[i + 1];
+  if (en <= b) return;
+  grid_dependency_wait();  // the term pass's results
   T yacc[3] = {T(0), T(0), T(0)};
   for (int q = b; q < en; ++q) {
     const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
     const int4 w1 = reinterpret_cast<const int4*>(ent)[2 * q + 1];
     if (!w1.y) continue;
     const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
-    int vid[4];
-    vf_term(t, terms, F, nF, V, vid);
-    T X[4][3], W[4][3];
+    const T* rr = rec + (int64_t)t * kVfHvRec + 3 * role;
 #pragma unroll
-    for (int v4 = 0; v4 < 4; ++v4)
-#pragma unroll
-      for (int al = 0; al < 3; ++al) {
-        X[v4][al] = x[(int64_t)vid[v4] * 3 + al];
-        W[v4][al] = v[(int64_t)vid[v4] * 3 + al];
-      }
-    const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
-    T dz[9];
-#pragma unroll
-    for (int sv = 0; sv < 3; ++sv)
-#pragma unroll
-      for (int al = 0; al < 3; ++al) {
-        T s = T(-0.0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (vf_coef(j, sv) != 0) s += T(vf_coef(j, sv)) * W[j][al];
-        dz[3 * sv + al] = s;
-      }
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-      if (rr != role) continue;
-#pragma unroll
-      for (int al = 0; al < 3; ++al) {
-        T s = T(-0.0);
-#pragma unroll
-        for (int sv = 0; sv < 3; ++sv) {
-          if (vf_coef(rr, sv) == 0) continue;
-          T tq = T(-0.0);
-#pragma unroll
-          for (int w = 0; w < 9; ++w) tq += shess(z, 3 * sv + al, w) * dz[w];
-          s += T(vf_coef(rr, sv)) * tq;
-        }
-        yacc[al] += s;
-      }
-    }
+    for (int al = 0; al < 3; ++al) yacc[al] += rr[al];
   }
 #pragma unroll
   for (int al = 0; al < 3; ++al) y[(int64_t)i * 3 + al] += yacc[al];
@@ -539,47 +614,64 @@ cudaError_t launch_vf_install_tables(const VfSet& S, int n, int V, const int32_t
 }
 
 template <typename T, bool GEN>
-void vf_rows_t(const VfSet& S, const VfLaunch& L, void* g, void* H, double* energy,
-               cudaStream_t s) {
+cudaError_t vf_rows_t(const VfSet& S, const VfLaunch& L, void* g, void* H, double* energy,
+                      cudaStream_t s) {
+  const unsigned nt = (unsigned)((S.n + kVfThreads - 1) / kVfThreads);
   const unsigned nr = (unsigned)((L.V + kVfThreads - 1) / kVfThreads);
-  k_vf_rows<T, GEN><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, S.terms, L.F, L.nF,
-                                              (const T*)L.rest, (T)L.k, (const T*)L.x, L.rp,
-                                              (T*)g, (T*)H, energy ? S.epart : nullptr);
-  if (energy) k_energy_add<<<1, 1024, 0, s>>>(S.epart, (int)nr, energy);
+  if (S.n > 0) {
+    k_vf_term_rec<T, GEN><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+                                                    (const T*)L.rest, (T)L.k, (const T*)L.x,
+                                                    (T*)S.rec, energy ? S.epart : nullptr);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (energy) {  // E of the terms, summed once per term
+      k_energy_add<<<1, 1024, 0, s>>>(S.epart, (int)nt, energy);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      k_vf_rows<T><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, (const T*)S.rec, L.rp, (T*)g,
+                                             (T*)H);
+      return cudaGetLastError();
+    }
+  }
+  // directly after the term pass: starts during its tail (pdl.cuh)
+  return launch_pdl(k_vf_rows<T>, dim3(nr), dim3(kVfThreads), 0, s, L.V,
+                    (const int32_t*)S.vrow, (const int32_t*)S.ent, (const T*)S.rec, L.rp, (T*)g,
+                    (T*)H);
 }
 
 template <typename T, bool GEN>
-void vf_rows_hvp_t(const VfSet& S, const VfLaunch& L, const void* v, void* y, cudaStream_t s) {
+cudaError_t vf_rows_hvp_t(const VfSet& S, const VfLaunch& L, const void* v, void* y,
+                          cudaStream_t s) {
+  const unsigned nt = (unsigned)((S.n + kVfThreads - 1) / kVfThreads);
   const unsigned nr = (unsigned)((L.V + kVfThreads - 1) / kVfThreads);
-  k_vf_rows_hvp<T, GEN><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, S.terms, L.F, L.nF,
-                                                  (const T*)L.rest, (T)L.k, (const T*)L.x,
-                                                  (const T*)v, (T*)y);
+  if (S.n > 0) {
+    k_vf_term_hv<T, GEN><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+                                                   (const T*)L.rest, (T)L.k, (const T*)L.x,
+                                                   (const T*)v, (T*)S.rec);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(k_vf_rows_hvp<T>, dim3(nr), dim3(kVfThreads), 0, s, L.V,
+                    (const int32_t*)S.vrow, (const int32_t*)S.ent, (const T*)S.rec, (T*)y);
 }
 
 cudaError_t launch_vf_rows_eval(int dtype, const VfSet& S, const VfLaunch& L, void* g, void* H,
                                 double* energy, cudaStream_t s) {
   if (L.V <= 0) return cudaSuccess;
-  if (dtype == MAD_F64) {
-    if (L.generic) vf_rows_t<double, true>(S, L, g, H, energy, s);
-    else vf_rows_t<double, false>(S, L, g, H, energy, s);
-  } else {
-    if (L.generic) vf_rows_t<float, true>(S, L, g, H, energy, s);
-    else vf_rows_t<float, false>(S, L, g, H, energy, s);
-  }
-  return cudaGetLastError();
+  if (dtype == MAD_F64)
+    return L.generic ? vf_rows_t<double, true>(S, L, g, H, energy, s)
+                     : vf_rows_t<double, false>(S, L, g, H, energy, s);
+  return L.generic ? vf_rows_t<float, true>(S, L, g, H, energy, s)
+                   : vf_rows_t<float, false>(S, L, g, H, energy, s);
 }
 
 cudaError_t launch_vf_rows_hvp(int dtype, const VfSet& S, const VfLaunch& L, const void* v,
                                void* y, cudaStream_t s) {
   if (L.V <= 0) return cudaSuccess;
-  if (dtype == MAD_F64) {
-    if (L.generic) vf_rows_hvp_t<double, true>(S, L, v, y, s);
-    else vf_rows_hvp_t<double, false>(S, L, v, y, s);
-  } else {
-    if (L.generic) vf_rows_hvp_t<float, true>(S, L, v, y, s);
-    else vf_rows_hvp_t<float, false>(S, L, v, y, s);
-  }
-  return cudaGetLastError();
+  if (dtype == MAD_F64)
+    return L.generic ? vf_rows_hvp_t<double, true>(S, L, v, y, s)
+                     : vf_rows_hvp_t<double, false>(S, L, v, y, s);
+  return L.generic ? vf_rows_hvp_t<float, true>(S, L, v, y, s)
+                   : vf_rows_hvp_t<float, false>(S, L, v, y, s);
 }
 
 template <typename T, bool GEN>
