@@ -26,7 +26,6 @@
 #include <type_traits>
 
 #include "mad_internal.h"
-#include "pdl.cuh"
 #include "rows_common.h"
 #include "terms.cuh"
 
@@ -444,7 +443,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                               });
     }
   }
-  if constexpr (FACES && DOF == 3) {
+  if constexpr (FACES == 1 && DOF == 3) {
     // area preservation after the edge terms, which store their blocks
     if (A.mask & MAD_TERM_AREA) {
       row_faces3<T>(A, i, tile, lane,
@@ -465,7 +464,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                     });
     }
   }
-  if constexpr (FACES && DOF == 2) {
+  if constexpr ((FACES == 1 || FACES == 2) && DOF == 2) {
     // after the edge terms, which store their blocks: faces add to them
     if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
       auto faces = [&](auto kc) {
@@ -497,9 +496,8 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   }
   if constexpr (FACES == 3 && DOF == 2) {
     // dof-2 face terms from the face pass's records: each row projects its
-    // corner's share (the pass wrote them before this grid reads them)
+    // corner's share (the pass ran before this kernel on the stream)
     if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
-      grid_dependency_wait();
       row_face_ids<T>(A, i, tile, lane, [&](int f, int c, int pj, int pk) {
         T M[4];
         load4<T>(A.Minv + (uint32_t)f * 4u, M);
@@ -726,10 +724,8 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   }
   if constexpr (FACES) {
     if (face_terms) {
-      // the row's corners' results of the per-face pass (k_face_hv): the
-      // table entries were loaded above; the results may be read once that
-      // pass has finished (a no-op when this grid was launched after it)
-      grid_dependency_wait();
+      // the row's corners' results of the per-face pass (k_face_hv), whose
+      // table entries were loaded above
 #pragma unroll
       for (int k = 0; k < SF; ++k) {
         if (fe[k] == -1) continue;
@@ -754,7 +750,6 @@ __global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __r
                                                       const T* __restrict__ v,
                                                       const T* __restrict__ area, T ka,
                                                       T* __restrict__ out) {
-  grid_dependents_may_launch();  // the row pass may start; it waits for the results
   const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (f >= nF) return;
   T u[3][3], w[3][3];
@@ -783,7 +778,6 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
                                                  const T* __restrict__ Minv,
                                                  const T* __restrict__ area, T* __restrict__ out,
                                                  int kind) {
-  grid_dependents_may_launch();  // the row pass may start; it waits for the results
   const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (f >= nF) return;
   const int32_t a = F[3 * f], b = F[3 * f + 1], c = F[3 * f + 2];
@@ -837,7 +831,6 @@ __global__ void __launch_bounds__(256) k_face_rec(int nF, bool vec2, const int32
                                                   const T* __restrict__ x,
                                                   const T* __restrict__ Minv,
                                                   const T* __restrict__ area, T* __restrict__ rec) {
-  grid_dependents_may_launch();  // the row pass may start; it waits for the records
   const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (f >= nF) return;
   using T2 = typename std::conditional<sizeof(T) == 4, float2, double2>::type;
@@ -958,13 +951,6 @@ cudaError_t eval_k(const RArgs<T>& A, bool pairs, int nb, size_t smem, cudaStrea
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   }
-  if constexpr (FACES == 3) {  // after the face pass: starts during its tail
-    if (pairs)
-      return launch_pdl(k_rows_eval<T, DOF, AD, ENERGY, S0, FACES, true>, dim3(nb),
-                        dim3(kRowThreads), smem, s, A);
-    return launch_pdl(k_rows_eval<T, DOF, AD, ENERGY, S0, FACES, false>, dim3(nb),
-                      dim3(kRowThreads), smem, s, A);
-  }
   if (pairs)
     k_rows_eval<T, DOF, AD, ENERGY, S0, FACES, true><<<nb, kRowThreads, smem, s>>>(A);
   else
@@ -1079,14 +1065,12 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
     constexpr int AD = decltype(adc)::value;
     const bool sp = t.mask & MAD_TERM_SPRING;
     // the row pass after a per-face pass (face terms), or alone
-    // the row pass after the per-face pass, launched with programmatic
-    // stream serialization: its blocks start while the face pass finishes,
-    // load their own rows' inputs and wait for the face results
+    // the row pass after the per-face pass, or alone
     auto rows = [&](auto facesc) {
       constexpr bool FC = decltype(facesc)::value;
-      if (sp)
-        return launch_pdl(k_rows_hvp<T, DOF, AD, kS0Max, FC>, dim3(nb), dim3(kRowThreads), 0, s, A);
-      return launch_pdl(k_rows_hvp<T, DOF, AD, 0, FC>, dim3(nb), dim3(kRowThreads), 0, s, A);
+      if (sp) k_rows_hvp<T, DOF, AD, kS0Max, FC><<<nb, kRowThreads, 0, s>>>(A);
+      else k_rows_hvp<T, DOF, AD, 0, FC><<<nb, kRowThreads, 0, s>>>(A);
+      return cudaGetLastError();
     };
     if constexpr (DOF == 2) {
       if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {

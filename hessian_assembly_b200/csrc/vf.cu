@@ -23,7 +23,6 @@
 #include <stdint.h>
 
 #include "mad_internal.h"
-#include "pdl.cuh"
 #include "sparse_ad.cuh"
 
 namespace mad {
@@ -389,7 +388,6 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
     int n, const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF, int V,
     const T* __restrict__ rest, T k, const T* __restrict__ x, T* __restrict__ rec,
     double* epart) {
-  grid_dependents_may_launch();  // the row pass may start; it waits for the records
   const int t = blockIdx.x * kVfThreads + threadIdx.x;
   double e = 0.0;
   int vid[4];
@@ -440,7 +438,6 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __
   const int b = vrow[i], en = vrow[i + 1];
   if (en <= b) return;
   const int64_t r0 = rp[i];
-  grid_dependency_wait();  // the term pass's records
   T gacc[3] = {T(0), T(0), T(0)};
   for (int q = b; q < en; ++q) {
     const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
@@ -495,7 +492,6 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_term_hv(
     int n, const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF, int V,
     const T* __restrict__ rest, T k, const T* __restrict__ x, const T* __restrict__ v,
     T* __restrict__ rec) {
-  grid_dependents_may_launch();
   const int t = blockIdx.x * kVfThreads + threadIdx.x;
   int vid[4];
   if (t >= n || !vf_term(t, terms, F, nF, V, vid)) return;
@@ -553,7 +549,6 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows_hvp(int V,
   if (i >= V) return;
   const int b = vrow[i], en = vrow[i + 1];
   if (en <= b) return;
-  grid_dependency_wait();  // the term pass's results
   T yacc[3] = {T(0), T(0), T(0)};
   for (int q = b; q < en; ++q) {
     const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
@@ -627,15 +622,11 @@ cudaError_t vf_rows_t(const VfSet& S, const VfLaunch& L, void* g, void* H, doubl
     if (energy) {  // E of the terms, summed once per term
       k_energy_add<<<1, 1024, 0, s>>>(S.epart, (int)nt, energy);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      k_vf_rows<T><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, (const T*)S.rec, L.rp, (T*)g,
-                                             (T*)H);
-      return cudaGetLastError();
     }
   }
-  // directly after the term pass: starts during its tail (pdl.cuh)
-  return launch_pdl(k_vf_rows<T>, dim3(nr), dim3(kVfThreads), 0, s, L.V,
-                    (const int32_t*)S.vrow, (const int32_t*)S.ent, (const T*)S.rec, L.rp, (T*)g,
-                    (T*)H);
+  k_vf_rows<T><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, (const T*)S.rec, L.rp, (T*)g,
+                                         (T*)H);
+  return cudaGetLastError();
 }
 
 template <typename T, bool GEN>
@@ -650,8 +641,8 @@ cudaError_t vf_rows_hvp_t(const VfSet& S, const VfLaunch& L, const void* v, void
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(k_vf_rows_hvp<T>, dim3(nr), dim3(kVfThreads), 0, s, L.V,
-                    (const int32_t*)S.vrow, (const int32_t*)S.ent, (const T*)S.rec, (T*)y);
+  k_vf_rows_hvp<T><<<nr, kVfThreads, 0, s>>>(L.V, S.vrow, S.ent, (const T*)S.rec, (T*)y);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_vf_rows_eval(int dtype, const VfSet& S, const VfLaunch& L, void* g, void* H,
