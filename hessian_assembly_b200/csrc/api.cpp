@@ -64,7 +64,6 @@ struct mad_ctx {
   int32_t* rows_fcslots = nullptr;
   int32_t* rows_fcofl = nullptr;
   void* face_hv = nullptr;  // [nF][3][2] scratch of the face Hessian-vector product
-  void* face_rec = nullptr; // [nF][16] J-space records of the dof-2 face pass
   double* epart = nullptr;
   size_t smem_eval = 0, smem_hvp = 0;
   // dynamic pattern
@@ -196,7 +195,6 @@ RowsLaunch rows_launch(const mad_ctx* c) {
   L.nF = c->nF;
   L.F = c->F_dev;
   L.fhv = c->face_hv;
-  L.frec = c->face_rec;
   L.epart = c->epart;
   if (c->active < 0) {
     L.rp = c->pat.rp;
@@ -479,11 +477,6 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
         char* hv = nullptr;
         CREATE_CK(dev_alloc(c, &hv, (size_t)c->esz * 3 * dof * (size_t)nF));
         c->face_hv = hv;
-        if (dof == 2) {  // the face pass's J-space records (16 values per face)
-          char* rec = nullptr;
-          CREATE_CK(dev_alloc(c, &rec, (size_t)c->esz * 16 * (size_t)nF));
-          c->face_rec = rec;
-        }
       }
     }
   }

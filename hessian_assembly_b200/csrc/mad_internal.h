@@ -284,7 +284,6 @@ struct RowsLaunch {
   int nF;
   const int32_t* F;        // [nF][3]
   void* fhv;               // [nF][3][2] per-face corner results of H v (scratch)
-  void* frec;              // [nF][16] per-face J-space records (dof 2; scratch)
   const int2* slots;
   const uint32_t* meta;
   const int32_t* ofl_ptr;

@@ -43,7 +43,6 @@ constexpr int rows_min_blocks() {
 
 template <typename T>
 struct RArgs {
-  const T* frec;  // per-face J-space records of the face pass (FACES == 3)
   const int32_t* fcslots;
   const int32_t* fcofl;
   const T* fhv;
@@ -294,52 +293,6 @@ __device__ __forceinline__ void row_faces3(const RArgs<T>& A, int i, int tile, i
   }
 }
 
-// Calls on_face(f, c, pj, pk) for every face of row i (the face table of
-// row_faces, without loading the corners' positions).
-template <typename T, typename OnFace>
-__device__ __forceinline__ void row_face_ids(const RArgs<T>& A, int i, int tile, int lane,
-                                            OnFace on_face) {
-  constexpr uint32_t kPm = (1u << kFacePosBits) - 1u;
-  auto one = [&](const int4& e) {
-    const uint32_t w = (uint32_t)e.w;
-    on_face(e.x, (int)(w & 3u), (int)((w >> 2) & kPm), (int)(w >> (2 + kFacePosBits)));
-  };
-  const int4* p = A.fslots + (uint32_t)(tile * A.sf * 32 + lane);
-  int4 e = p[0];
-  bool more = false;
-#pragma unroll 1
-  for (int k = 0; k < A.sf; ++k) {
-    if (e.x < 0) break;
-    const int4 en = k + 1 < A.sf ? p[(uint32_t)((k + 1) * 32)] : make_int4(-1, 0, 0, 0);
-    if (k == kFaceRowSlots - 1) more = e.z < 0;
-    one(e);
-    e = en;
-  }
-  if (more) {
-    const int o0 = A.fofl_ptr[i], o1 = A.fofl_ptr[i + 1];
-#pragma unroll 1
-    for (int q = o0; q < o1; ++q) one(A.fofl[q]);
-  }
-}
-
-// The J-space record of face f: value, gradient, packed Hessian (16 values,
-// the last unused), read as 16-byte loads.
-constexpr int kFaceRec = 16;
-template <typename T>
-__device__ __forceinline__ HyperDual<T, 4> load_face_rec(const T* __restrict__ rec, int f) {
-  T r[kFaceRec];
-  const T* p = rec + (uint32_t)f * kFaceRec;
-#pragma unroll
-  for (int q = 0; q < kFaceRec; q += 4) load4<T>(p + q, r + q);
-  HyperDual<T, 4> e;
-  e.v = r[0];
-#pragma unroll
-  for (int a = 0; a < 4; ++a) e.g[a] = r[1 + a];
-#pragma unroll
-  for (int q = 0; q < 10; ++q) e.h[q] = r[5 + q];
-  return e;
-}
-
 // b[0..8] += v[0..8]
 template <typename T>
 __device__ __forceinline__ void add9(T* b, const T* v) {
@@ -443,7 +396,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                               });
     }
   }
-  if constexpr (FACES == 1 && DOF == 3) {
+  if constexpr (FACES && DOF == 3) {
     // area preservation after the edge terms, which store their blocks
     if (A.mask & MAD_TERM_AREA) {
       row_faces3<T>(A, i, tile, lane,
@@ -464,7 +417,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                     });
     }
   }
-  if constexpr ((FACES == 1 || FACES == 2) && DOF == 2) {
+  if constexpr (FACES && DOF == 2) {
     // after the edge terms, which store their blocks: faces add to them
     if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
       auto faces = [&](auto kc) {
@@ -492,31 +445,6 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
         if (!(A.mask & MAD_TERM_SYMDIR)) faces(std::integral_constant<int, kFaceArap>{});
         else faces(std::integral_constant<int, kFaceSymDir | kFaceArap>{});
       }
-    }
-  }
-  if constexpr (FACES == 3 && DOF == 2) {
-    // dof-2 face terms from the face pass's records: each row projects its
-    // corner's share (the pass ran before this kernel on the stream)
-    if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
-      row_face_ids<T>(A, i, tile, lane, [&](int f, int c, int pj, int pk) {
-        T M[4];
-        load4<T>(A.Minv + (uint32_t)f * 4u, M);
-        const HyperDual<T, 4> e = load_face_rec<T>(A.frec, f);
-        T wr[3][2];
-        rotated_weights<T>(M, c, wr);
-        FaceRow<T> o;
-        project_face_row<T>(e, wr, o);
-        acc[0] += o.H[0][0];
-        acc[1] += o.H[0][1];
-        acc[2] += o.H[0][3];
-        gr[0] += o.g[0];
-        gr[1] += o.g[1];
-        const int oj = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pj) : pj;
-        const int ok = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, pk) : pk;
-        add4<T>(row + oj * B, o.H[1]);
-        add4<T>(row + ok * B, o.H[2]);
-        if (ENERGY) energy += (double)o.E * (1.0 / 3.0);
-      });
     }
   }
   if (pairs) {
@@ -822,70 +750,10 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
 }
 
 
-// Per-face pass of the evaluation of dof-2 face terms: one thread per face
-// differentiates its energy once in J space (J in the face's own corner
-// order) and writes the record (value, gradient, packed Hessian); the row
-// kernel then projects each corner's share (FACES == 3).
-template <typename T, int AD, int KIND>
-__global__ void __launch_bounds__(256) k_face_rec(int nF, bool vec2, const int32_t* __restrict__ F,
-                                                  const T* __restrict__ x,
-                                                  const T* __restrict__ Minv,
-                                                  const T* __restrict__ area, T* __restrict__ rec) {
-  const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (f >= nF) return;
-  using T2 = typename std::conditional<sizeof(T) == 4, float2, double2>::type;
-  const int32_t vid[3] = {F[3 * f], F[3 * f + 1], F[3 * f + 2]};
-  T u[3][2], M[4];
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    if (vec2) {
-      const T2 xu = reinterpret_cast<const T2*>(x)[vid[k]];
-      u[k][0] = xu.x;
-      u[k][1] = xu.y;
-    } else {
-      u[k][0] = x[(int64_t)vid[k] * 2];
-      u[k][1] = x[(int64_t)vid[k] * 2 + 1];
-    }
-  }
-  load4<T>(Minv + 4 * f, M);
-  T Jv[4];
-#pragma unroll
-  for (int al = 0; al < 2; ++al)
-#pragma unroll
-    for (int ga = 0; ga < 2; ++ga)
-      Jv[2 * al + ga] = (u[1][al] - u[0][al]) * M[ga] + (u[2][al] - u[0][al]) * M[2 + ga];
-  const HyperDual<T, 4> e = face2_hd<KIND, AD>(Jv, area[f]);
-  T r[kFaceRec];
-  r[0] = e.v;
-#pragma unroll
-  for (int a = 0; a < 4; ++a) r[1 + a] = e.g[a];
-#pragma unroll
-  for (int q = 0; q < 10; ++q) r[5 + q] = e.h[q];
-  r[15] = T(0);
-  using T4 = typename std::conditional<sizeof(T) == 4, float4, double2>::type;
-  T4* o = reinterpret_cast<T4*>(rec + f * kFaceRec);
-  constexpr int W = (int)(sizeof(T4) / sizeof(T));
-#pragma unroll
-  for (int q = 0; q < kFaceRec / W; ++q) {
-    T4 v4;
-    if constexpr (W == 4) {
-      v4.x = r[4 * q];
-      v4.y = r[4 * q + 1];
-      v4.z = r[4 * q + 2];
-      v4.w = r[4 * q + 3];
-    } else {
-      v4.x = r[2 * q];
-      v4.y = r[2 * q + 1];
-    }
-    o[q] = v4;
-  }
-}
-
 template <typename T>
 RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
                     void* g, void* H, void* y, bool energy) {
   RArgs<T> A;
-  A.frec = (const T*)L.frec;
   A.fcslots = L.fcslots;
   A.fcofl = L.fcofl;
   A.fhv = (const T*)L.fhv;
@@ -1010,29 +878,6 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
     auto faces_k = [&](auto s0c) {
       constexpr int S0F = decltype(s0c)::value;
       if constexpr (DOF == 2) {
-        if (L.frec && ad != kAdFull) {
-          // each face differentiated once by the face pass, then projected
-          // per corner row
-          if (L.nF > 0) {
-            const unsigned nbf = (unsigned)((L.nF + 255) / 256);
-            const bool vec2 = (((uintptr_t)x) % (2 * sizeof(T))) == 0;
-            const int kind = face2_kind(t.mask);
-            const cudaError_t ef = with_ad(ad, [&](auto adc) {
-              constexpr int AD = decltype(adc)::value;
-              auto launch = [&](auto kc) {
-                k_face_rec<T, AD, decltype(kc)::value><<<nbf, 256, 0, s>>>(
-                    L.nF, vec2, L.F, (const T*)x, (const T*)t.face_Minv, (const T*)t.face_area,
-                    (T*)L.frec);
-              };
-              if (kind == kFaceSymDir) launch(std::integral_constant<int, kFaceSymDir>{});
-              else if (kind == kFaceArap) launch(std::integral_constant<int, kFaceArap>{});
-              else launch(std::integral_constant<int, kFaceSymDir | kFaceArap>{});
-              return cudaGetLastError();
-            });
-            if (ef != cudaSuccess) return ef;
-          }
-          return eval_k4<T, DOF, S0F, 3>(A, ad, en, pairs, nb, smem, s);
-        }
         if (t.mask & MAD_TERM_ARAP) return eval_k4<T, DOF, S0F, 2>(A, ad, en, pairs, nb, smem, s);
       }
       return eval_k4<T, DOF, S0F, 1>(A, ad, en, pairs, nb, smem, s);
@@ -1122,11 +967,6 @@ cudaError_t set_rows_limits(size_t bytes) {
         cudaSuccess)
       return e;
     if ((e = eval_k4<T, DOF, 0, 2>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
-      return e;
-    if ((e = eval_k4<T, DOF, kS0Max, 3>(A, false, false, false, 0, bytes, 0, true)) !=
-        cudaSuccess)
-      return e;
-    if ((e = eval_k4<T, DOF, 0, 3>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
       return e;
   }
   return cudaSuccess;

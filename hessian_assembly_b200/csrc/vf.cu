@@ -447,6 +447,14 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __
     T r[kVfRec];
     load_rec<T, kVfRec>(rec + (int64_t)t * kVfRec, r);
     const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
+    // the four blocks read first, in one round of independent loads: the
+    // updates go through the same pointer, so loads mixed with stores would
+    // each wait for the store before them
+    T cur[4][9];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q9 = 0; q9 < 9; ++q9) cur[j][q9] = H[(r0 + pos[j]) * 9 + q9];
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr) {  // the role as a compile-time index
       if (rr != role) continue;
@@ -459,8 +467,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __
         gacc[al] += s2;
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        T* hb = H + (r0 + pos[j]) * 9;
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int al = 0; al < 3; ++al)
 #pragma unroll
@@ -475,10 +482,13 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __
                   s2 += T(vf_coef(rr, sv) * vf_coef(j, tv)) *
                         r[10 + (a <= c ? Tri<9>::idx(a, c) : Tri<9>::idx(c, a))];
               }
-            hb[3 * al + be] += s2;
+            cur[j][3 * al + be] += s2;
           }
-      }
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q9 = 0; q9 < 9; ++q9) H[(r0 + pos[j]) * 9 + q9] = cur[j][q9];
   }
 #pragma unroll
   for (int al = 0; al < 3; ++al) g[(int64_t)i * 3 + al] += gacc[al];
