@@ -622,13 +622,25 @@ mad_status mad_eval(mad_ctx* c, const void* x, const mad_terms* t, void* g, void
   if (c->V > 0 && (!x || !g || !H_vals))
     return fail(c, MAD_ERR_INVALID_ARG, "x, g and H_vals must be device pointers");
   cudaError_t e;
+  // installed vertex-face terms without area terms: the term pass first,
+  // then the row kernel gathers each row's share into its staged row
+  const bool vf_in_rows = (t->mask & MAD_TERM_VF) && t->vf_n > 0 && !t->vf &&
+                          !(t->mask & MAD_TERM_AREA) && use_rows(c, t) && c->active >= 0;
   if (use_rows(c, t)) {
-    e = launch_rows_eval(rows_launch(c), *t, x, g, H_vals, energy, as_stream(stream));
+    RowsLaunch R = rows_launch(c);
+    if (vf_in_rows) {
+      e = launch_vf_term_pass(c->dtype, c->vfs, vf_launch(c, t, x), as_stream(stream));
+      if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval vertex-face term pass");
+      R.vrow = c->vfs.vrow;
+      R.vent = c->vfs.ent;
+      R.vrec = c->vfs.rec;
+    }
+    e = launch_rows_eval(R, *t, x, g, H_vals, energy, as_stream(stream));
   } else {
     e = launch_eval(eval_launch(c), *t, x, g, H_vals, energy, as_stream(stream));
   }
   if (e != cudaSuccess) return cuda_fail(c, e, "mad_eval launch");
-  if ((t->mask & MAD_TERM_VF) && t->vf_n > 0) {
+  if ((t->mask & MAD_TERM_VF) && t->vf_n > 0 && !vf_in_rows) {
     // t->vf given: one thread per term, atomics; else the installed set,
     // gathered per row
     e = t->vf ? launch_vf_eval(c->dtype, vf_launch(c, t, x), g, H_vals, energy, as_stream(stream))

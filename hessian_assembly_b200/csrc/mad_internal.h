@@ -192,6 +192,9 @@ cudaError_t launch_vf_install_tables(const VfSet& S, int n, int V, const int32_t
                                      int32_t* status, cudaStream_t s);
 cudaError_t launch_vf_rows_eval(int dtype, const VfSet& S, const VfLaunch& L, void* g, void* H,
                                 double* energy, cudaStream_t s);
+// the term pass alone: one record per installed term (S.rec), for the row
+// kernel to gather
+cudaError_t launch_vf_term_pass(int dtype, const VfSet& S, const VfLaunch& L, cudaStream_t s);
 cudaError_t launch_vf_rows_hvp(int dtype, const VfSet& S, const VfLaunch& L, const void* v,
                                void* y, cudaStream_t s);
 cudaError_t launch_vf_hvp(int dtype, const VfLaunch& L, const void* v, void* y, cudaStream_t s);
@@ -296,6 +299,10 @@ struct RowsLaunch {
   const int32_t* pe_pos;
   const void* pe_rest;
   double* epart;  // [rows_blocks(V)]
+  // installed vertex-face terms gathered into the rows (nullptr: none)
+  const int32_t* vrow = nullptr;
+  const int32_t* vent = nullptr;
+  const void* vrec = nullptr;
 };
 int rows_blocks(int V);
 size_t rows_smem_bytes(const RowsLaunch& L);

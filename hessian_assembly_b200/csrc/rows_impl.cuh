@@ -43,6 +43,11 @@ constexpr int rows_min_blocks() {
 
 template <typename T>
 struct RArgs {
+  // installed vertex-face terms (FACES == 4): per-row entries and the term
+  // pass's records (see vf.cu)
+  const int32_t* vrow;
+  const int32_t* vent;
+  const T* vrec;
   const int32_t* fcslots;
   const int32_t* fcofl;
   const T* fhv;
@@ -293,6 +298,15 @@ __device__ __forceinline__ void row_faces3(const RArgs<T>& A, int i, int tile, i
   }
 }
 
+// Vertex-face records of the term pass (vf.cu): E, the gradient in
+// z = (p - a, b - a, c - a) (9), the packed Hessian in z (45), padded to 56;
+// the coefficient of stencil vertex v (p, a, b, c) on z block s is
+// vf_coef_s(v, s).
+constexpr int kVfRecVals = 56;
+__host__ __device__ constexpr int vf_coef_s(int v, int s) {
+  return v == 0 ? (s == 0 ? 1 : 0) : v == 1 ? -1 : (v - 1 == s ? 1 : 0);
+}
+
 // b[0..8] += v[0..8]
 template <typename T>
 __device__ __forceinline__ void add9(T* b, const T* v) {
@@ -396,7 +410,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                               });
     }
   }
-  if constexpr (FACES && DOF == 3) {
+  if constexpr (FACES == 1 && DOF == 3) {
     // area preservation after the edge terms, which store their blocks
     if (A.mask & MAD_TERM_AREA) {
       row_faces3<T>(A, i, tile, lane,
@@ -417,7 +431,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
                     });
     }
   }
-  if constexpr (FACES && DOF == 2) {
+  if constexpr ((FACES == 1 || FACES == 2) && DOF == 2) {
     // after the edge terms, which store their blocks: faces add to them
     if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
       auto faces = [&](auto kc) {
@@ -467,6 +481,63 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
       eval_edge_res<T, DOF, AD>(xi, xj, rest, A.kp, Rp);
       apply_edge_side<false>(Rp, 0, acc, row + (pw & kPairPosMask) * B, gr);
       if (ENERGY) energy += 0.5 * (double)edge_energy(Rp);
+    }
+  }
+  if constexpr (FACES == 4 && DOF == 3 && PAIRS) {
+    // installed vertex-face terms: this row's share of each of its terms,
+    // from the records the term pass wrote before this kernel; the blocks go
+    // to the staged row, the diagonal block to the register accumulator
+    if (A.mask & MAD_TERM_VF) {
+      const int vb = A.vrow[i], ve = A.vrow[i + 1];
+      for (int q = vb; q < ve; ++q) {
+        const int4 w0 = reinterpret_cast<const int4*>(A.vent)[2 * q];
+        const int4 w1 = reinterpret_cast<const int4*>(A.vent)[2 * q + 1];
+        if (!w1.y) continue;
+        const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
+        const T* r = A.vrec + (uint32_t)t * kVfRecVals;
+        if (ENERGY) energy += 0.25 * (double)r[0];
+        const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {  // the role as a compile-time index
+          if (rr != role) continue;
+#pragma unroll
+          for (int al = 0; al < 3; ++al) {
+            T s2 = T(-0.0);
+#pragma unroll
+            for (int sv = 0; sv < 3; ++sv)
+              if (vf_coef_s(rr, sv) != 0) s2 += T(vf_coef_s(rr, sv)) * r[1 + 3 * sv + al];
+            gr[al] += s2;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            T blk[9];
+#pragma unroll
+            for (int al = 0; al < 3; ++al)
+#pragma unroll
+              for (int be = 0; be < 3; ++be) {
+                T s2 = T(-0.0);
+#pragma unroll
+                for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+                  for (int tv = 0; tv < 3; ++tv) {
+                    const int a = 3 * sv + al, c2 = 3 * tv + be;
+                    if (vf_coef_s(rr, sv) * vf_coef_s(j, tv) != 0)
+                      s2 += T(vf_coef_s(rr, sv) * vf_coef_s(j, tv)) *
+                            r[10 + (a <= c2 ? Tri<9>::idx(a, c2) : Tri<9>::idx(c2, a))];
+                  }
+                blk[3 * al + be] = s2;
+              }
+            if (j == rr) {
+#pragma unroll
+              for (int a = 0; a < 3; ++a)
+#pragma unroll
+                for (int b2 = a; b2 < 3; ++b2) acc[Tri<3>::idx(a, b2)] += blk[3 * a + b2];
+            } else {
+              add9<T>(row + pos[j] * B, blk);
+            }
+          }
+        }
+      }
     }
   }
   const int dp = PAIRS ? row_pos_new(rn, A.pe_pos, pb, pn, nins, (int)(m >> 16)) : (int)(m >> 16);
@@ -754,6 +825,9 @@ template <typename T>
 RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
                     void* g, void* H, void* y, bool energy) {
   RArgs<T> A;
+  A.vrow = L.vrow;
+  A.vent = L.vent;
+  A.vrec = (const T*)L.vrec;
   A.fcslots = L.fcslots;
   A.fcofl = L.fcofl;
   A.fhv = (const T*)L.fhv;
@@ -838,7 +912,8 @@ cudaError_t with_ad(int ad, F&& f) {
 // terms; 1 the face term of the dof (symmetric Dirichlet for dof 2, area
 // preservation for dof 3); 2 (dof 2) ARAP alone or with symmetric Dirichlet,
 // an instantiation of its own so that the symmetric Dirichlet kernel keeps
-// its register budget.
+// its register budget; 4 (dof 3) the installed vertex-face terms gathered
+// from the term pass's records.
 template <typename T, int DOF, int S0, int FACES>
 cudaError_t eval_k4(const RArgs<T>& A, int ad, bool energy, bool pairs, int nb, size_t smem,
                     cudaStream_t s, bool set = false) {
@@ -871,7 +946,13 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   const bool pairs = L.prow != nullptr;
   const bool en = energy != nullptr;
   cudaError_t e;
-  if ((DOF == 2 && (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP))) ||
+  if (DOF == 3 && L.vrow && pairs && (t.mask & MAD_TERM_VF) && !(t.mask & MAD_TERM_AREA)) {
+    // installed vertex-face terms gathered into the rows (FACES == 4)
+    if (t.mask & MAD_TERM_SPRING)
+      e = eval_k4<T, DOF, kS0Max, 4>(A, ad, en, pairs, nb, smem, s);
+    else
+      e = eval_k4<T, DOF, 0, 4>(A, ad, en, pairs, nb, smem, s);
+  } else if ((DOF == 2 && (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP))) ||
       (DOF == 3 && (t.mask & MAD_TERM_AREA))) {
     // face terms: the face-row instantiations; without edge terms the kernel
     // carries no edge-slot code (S0 = 0)
@@ -962,6 +1043,13 @@ cudaError_t set_rows_limits(size_t bytes) {
     return e;
   if ((e = eval_k4<T, DOF, 0, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
     return e;
+  if constexpr (DOF == 3) {
+    if ((e = eval_k4<T, DOF, kS0Max, 4>(A, false, false, false, 0, bytes, 0, true)) !=
+        cudaSuccess)
+      return e;
+    if ((e = eval_k4<T, DOF, 0, 4>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+      return e;
+  }
   if constexpr (DOF == 2) {
     if ((e = eval_k4<T, DOF, kS0Max, 2>(A, false, false, false, 0, bytes, 0, true)) !=
         cudaSuccess)

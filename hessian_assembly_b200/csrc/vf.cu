@@ -655,6 +655,35 @@ cudaError_t vf_rows_hvp_t(const VfSet& S, const VfLaunch& L, const void* v, void
   return cudaGetLastError();
 }
 
+cudaError_t launch_vf_term_pass(int dtype, const VfSet& S, const VfLaunch& L, cudaStream_t s) {
+  if (S.n <= 0) return cudaSuccess;
+  const unsigned nt = (unsigned)((S.n + kVfThreads - 1) / kVfThreads);
+  if (dtype == MAD_F64) {
+    if (L.generic)
+      k_vf_term_rec<double, true><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+                                                             (const double*)L.rest, L.k,
+                                                             (const double*)L.x, (double*)S.rec,
+                                                             nullptr);
+    else
+      k_vf_term_rec<double, false><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+                                                              (const double*)L.rest, L.k,
+                                                              (const double*)L.x,
+                                                              (double*)S.rec, nullptr);
+  } else {
+    if (L.generic)
+      k_vf_term_rec<float, true><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+                                                            (const float*)L.rest, (float)L.k,
+                                                            (const float*)L.x, (float*)S.rec,
+                                                            nullptr);
+    else
+      k_vf_term_rec<float, false><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+                                                             (const float*)L.rest, (float)L.k,
+                                                             (const float*)L.x, (float*)S.rec,
+                                                             nullptr);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_vf_rows_eval(int dtype, const VfSet& S, const VfLaunch& L, void* g, void* H,
                                 double* energy, cudaStream_t s) {
   if (L.V <= 0) return cudaSuccess;
