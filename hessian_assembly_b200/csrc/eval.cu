@@ -37,6 +37,24 @@
 namespace mad {
 namespace {
 
+// Asynchronous copies of single elements from global to shared memory
+// (cp.async, 4 or 8 bytes): the staging of a patch's positions is issued in
+// one go, without a register round trip per element, and is in flight while
+// the thread loads its row's tables; cp_async_wait_all() then waits for the
+// thread's own copies (a block barrier after it publishes them to all).
+template <typename T>
+__device__ __forceinline__ void cp_async_elem(T* sdst, const T* gsrc) {
+  static_assert(sizeof(T) == 4 || sizeof(T) == 8, "4- or 8-byte elements");
+  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(sdst);
+  if constexpr (sizeof(T) == 4)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(gsrc) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 constexpr int kThreads = 256;
 constexpr int kUnr = 8;  // row slots loaded and evaluated together
 #ifndef MAD_EVAL_MIN_BLOCKS
@@ -322,14 +340,15 @@ __global__ void __launch_bounds__(kThreads, MAD_EVAL_MIN_BLOCKS) k_eval(const KA
   double energy = 0.0;
 
   // ---- 1. prologue: all global loads of the patch --------------------------
-  RowIn<T> in;
-  const bool has_row = tid < hd.no;
-  if (has_row) load_row<T, DOF>(A, hd, tid, gather, pairs_layout, in);
+  // the positions of the owned and ribbon vertices, staged by cp.async
   for (int lv = tid; lv < hd.nv; lv += kThreads) {
     const int64_t gv = (int64_t)A.vgid[hd.vbeg + lv] * DOF;
 #pragma unroll
-    for (int c = 0; c < DOF; ++c) S.x[lv * DOF + c] = A.x[gv + c];
+    for (int c = 0; c < DOF; ++c) cp_async_elem<T>(&S.x[lv * DOF + c], &A.x[gv + c]);
   }
+  RowIn<T> in;
+  const bool has_row = tid < hd.no;
+  if (has_row) load_row<T, DOF>(A, hd, tid, gather, pairs_layout, in);
   T xt[DOF];
   if (has_row && inertia) {
 #pragma unroll
@@ -343,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, MAD_EVAL_MIN_BLOCKS) k_eval(const KA
     S.len[tid] = in.d1 - in.d0;
     S.gid[tid] = in.gid;
   }
+  cp_async_wait_all();
   __syncthreads();
 
   // ---- 2. per row: inertia, then the row's edge terms (gather mode) --------
@@ -602,6 +622,15 @@ __global__ void __launch_bounds__(kThreads) k_hvp(const KArgs<T> A) {
   const bool faces = DOF == 2 && (A.mask & MAD_TERM_SYMDIR) && hd.nf > 0;
   const bool inertia = A.mask & MAD_TERM_INERTIA;
 
+  // positions and direction of the owned and ribbon vertices, by cp.async
+  for (int lv = tid; lv < hd.nv; lv += kThreads) {
+    const int64_t gv = (int64_t)A.vgid[hd.vbeg + lv] * DOF;
+#pragma unroll
+    for (int c = 0; c < DOF; ++c) {
+      cp_async_elem<T>(&S.x[lv * DOF + c], &A.x[gv + c]);
+      cp_async_elem<T>(&S.v[lv * DOF + c], &A.v[gv + c]);
+    }
+  }
   RowIn<T> in;
   const bool has_row = tid < hd.no;
   if (has_row) load_row<T, DOF>(A, hd, tid, springs, pairs, in);
@@ -610,15 +639,8 @@ __global__ void __launch_bounds__(kThreads) k_hvp(const KArgs<T> A) {
 #pragma unroll
     for (int a = 0; a < DOF; ++a) xt[a] = A.xt[(int64_t)in.gid * DOF + a];
   }
-  for (int lv = tid; lv < hd.nv; lv += kThreads) {
-    const int64_t gv = (int64_t)A.vgid[hd.vbeg + lv] * DOF;
-#pragma unroll
-    for (int c = 0; c < DOF; ++c) {
-      S.x[lv * DOF + c] = A.x[gv + c];
-      S.v[lv * DOF + c] = A.v[gv + c];
-    }
-  }
   if (has_row) S.gid[tid] = in.gid;
+  cp_async_wait_all();
   __syncthreads();
   T yr[DOF];
 #pragma unroll

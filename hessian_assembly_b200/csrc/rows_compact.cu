@@ -271,13 +271,13 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
 }
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, false>())
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
     k_rows_eval_c(const CArgs<T> A) {
   rows_c_body<T, DOF, AD, ENERGY, S0, false>(A, nullptr);
 }
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, false>())
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
     k_rows_eval_cs(const CArgs<T> A, const __grid_constant__ ShardArgs<T> S) {
   rows_c_body<T, DOF, AD, ENERGY, S0, true>(A, &S);
 }

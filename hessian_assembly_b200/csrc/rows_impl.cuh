@@ -36,9 +36,14 @@ constexpr int kS0Max = 8;         // most slots per row in the slot table
 #ifndef MAD_ROWS_MIN_BLOCKS
 #define MAD_ROWS_MIN_BLOCKS 6  // resident blocks per SM (fp32) the register budget targets
 #endif
-template <typename T, bool FACES>
+// FACES: 0 none; 1, 2 face terms (their evaluators need more registers);
+// 4 installed vertex-face terms, whose branch runs on few rows and is held
+// to the budget of the plain kernel (it may spill rather than lower the
+// occupancy of every row)
+template <typename T, int FACES>
 constexpr int rows_min_blocks() {
-  return FACES ? (sizeof(T) == 4 ? 4 : 2) : (sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3);
+  return (FACES == 1 || FACES == 2) ? (sizeof(T) == 4 ? 4 : 2)
+                                    : (sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3);
 }
 
 template <typename T>
@@ -298,14 +303,10 @@ __device__ __forceinline__ void row_faces3(const RArgs<T>& A, int i, int tile, i
   }
 }
 
-// Vertex-face records of the term pass (vf.cu): E, the gradient in
-// z = (p - a, b - a, c - a) (9), the packed Hessian in z (45), padded to 56;
-// the coefficient of stencil vertex v (p, a, b, c) on z block s is
-// vf_coef_s(v, s).
-constexpr int kVfRecVals = 56;
-__host__ __device__ constexpr int vf_coef_s(int v, int s) {
-  return v == 0 ? (s == 0 ? 1 : 0) : v == 1 ? -1 : (v - 1 == s ? 1 : 0);
-}
+// Vertex-face records of the term pass (vf.cu): per term and role (the
+// term's vertex p, a, b or c) kVfRoleVals values: that vertex's gradient
+// (3), its blocks with p, a, b, c (4 x 9, row-major), and E.
+constexpr int kVfRoleVals = 40;
 
 // b[0..8] += v[0..8]
 template <typename T>
@@ -485,8 +486,9 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   }
   if constexpr (FACES == 4 && DOF == 3 && PAIRS) {
     // installed vertex-face terms: this row's share of each of its terms,
-    // from the records the term pass wrote before this kernel; the blocks go
-    // to the staged row, the diagonal block to the register accumulator
+    // written by the term pass before this kernel (its role's slice: the
+    // gradient, its four blocks, E); the blocks go to the staged row, the
+    // diagonal block to the register accumulator
     if (A.mask & MAD_TERM_VF) {
       const int vb = A.vrow[i], ve = A.vrow[i + 1];
       for (int q = vb; q < ve; ++q) {
@@ -494,47 +496,23 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
         const int4 w1 = reinterpret_cast<const int4*>(A.vent)[2 * q + 1];
         if (!w1.y) continue;
         const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
-        const T* r = A.vrec + (uint32_t)t * kVfRecVals;
-        if (ENERGY) energy += 0.25 * (double)r[0];
+        const T* r = A.vrec + (size_t)t * (4 * kVfRoleVals) + role * kVfRoleVals;
+        T v[kVfRoleVals];
+#pragma unroll
+        for (int q4 = 0; q4 < kVfRoleVals; q4 += 4) load4<T>(r + q4, v + q4);
+        if (ENERGY) energy += 0.25 * (double)v[kVfRoleVals - 1];
+#pragma unroll
+        for (int a = 0; a < 3; ++a) gr[a] += v[a];
         const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {  // the role as a compile-time index
-          if (rr != role) continue;
+        for (int j = 0; j < 4; ++j) {
+          if (j == role) {
 #pragma unroll
-          for (int al = 0; al < 3; ++al) {
-            T s2 = T(-0.0);
+            for (int a = 0; a < 3; ++a)
 #pragma unroll
-            for (int sv = 0; sv < 3; ++sv)
-              if (vf_coef_s(rr, sv) != 0) s2 += T(vf_coef_s(rr, sv)) * r[1 + 3 * sv + al];
-            gr[al] += s2;
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            T blk[9];
-#pragma unroll
-            for (int al = 0; al < 3; ++al)
-#pragma unroll
-              for (int be = 0; be < 3; ++be) {
-                T s2 = T(-0.0);
-#pragma unroll
-                for (int sv = 0; sv < 3; ++sv)
-#pragma unroll
-                  for (int tv = 0; tv < 3; ++tv) {
-                    const int a = 3 * sv + al, c2 = 3 * tv + be;
-                    if (vf_coef_s(rr, sv) * vf_coef_s(j, tv) != 0)
-                      s2 += T(vf_coef_s(rr, sv) * vf_coef_s(j, tv)) *
-                            r[10 + (a <= c2 ? Tri<9>::idx(a, c2) : Tri<9>::idx(c2, a))];
-                  }
-                blk[3 * al + be] = s2;
-              }
-            if (j == rr) {
-#pragma unroll
-              for (int a = 0; a < 3; ++a)
-#pragma unroll
-                for (int b2 = a; b2 < 3; ++b2) acc[Tri<3>::idx(a, b2)] += blk[3 * a + b2];
-            } else {
-              add9<T>(row + pos[j] * B, blk);
-            }
+              for (int b2 = a; b2 < 3; ++b2) acc[Tri<3>::idx(a, b2)] += v[3 + 9 * j + 3 * a + b2];
+          } else {
+            add9<T>(row + pos[j] * B, v + 3 + 9 * j);
           }
         }
       }
@@ -552,7 +530,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
 }
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0, int FACES, bool PAIRS>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, (FACES != 0)>()) k_rows_eval(const RArgs<T> A) {
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_eval(const RArgs<T> A) {
   constexpr int B = DOF * DOF;
   constexpr int VEC = 16 / (int)sizeof(T);
   extern __shared__ __align__(16) char smem_raw[];
@@ -633,7 +611,7 @@ __device__ __forceinline__ void add_corner_hv(const T* __restrict__ fhv, uint32_
 }
 
 template <typename T, int DOF, int AD, int S0, bool FACES>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_hvp(const RArgs<T> A) {
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES ? 1 : 0>()) k_rows_hvp(const RArgs<T> A) {
   constexpr int TD = Tri<DOF>::size;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int tile = blockIdx.x * kWarps + wib;

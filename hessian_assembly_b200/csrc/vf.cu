@@ -378,10 +378,12 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_finalize(
 }
 
 // Term pass of an installed set: one thread per term differentiates it once
-// and writes its record: E, the gradient in z (9) and the packed Hessian in
-// z (45), padded to kVfRec values; the energies are summed per block.
-constexpr int kVfRec = 56;
-constexpr int kVfHz = 45;  // Tri<9>::size
+// and writes, for each of its four vertices (role p, a, b, c), that
+// vertex's share: its gradient (3) and its blocks with the four stencil
+// vertices (4 x 9), then E in the last of kVfRoleVals values.  A row then
+// only adds its role's slice.
+constexpr int kVfRoleVals = 40;             // 3 + 36 + E
+constexpr int kVfRec = 4 * kVfRoleVals;     // per term
 
 template <typename T, bool GEN>
 __global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
@@ -399,17 +401,35 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
       for (int al = 0; al < 3; ++al) X[v4][al] = x[(int64_t)vid[v4] * 3 + al];
     const auto z = vf_energy<T, GEN>(X[0], X[1], X[2], X[3], rest[t], k);
     e = (double)z.v;
-    T r[kVfRec];
-    r[0] = z.v;
 #pragma unroll
-    for (int q = 0; q < 9; ++q) r[1 + q] = sgrad(z, q);
+    for (int rr = 0; rr < 4; ++rr) {
+      T r[kVfRoleVals];
 #pragma unroll
-    for (int a = 0; a < 9; ++a)
+      for (int al = 0; al < 3; ++al) {
+        T s2 = T(-0.0);
 #pragma unroll
-      for (int b = a; b < 9; ++b) r[10 + Tri<9>::idx(a, b)] = shess(z, a, b);
+        for (int sv = 0; sv < 3; ++sv)
+          if (vf_coef(rr, sv) != 0) s2 += T(vf_coef(rr, sv)) * sgrad(z, 3 * sv + al);
+        r[al] = s2;
+      }
 #pragma unroll
-    for (int q = 10 + kVfHz; q < kVfRec; ++q) r[q] = T(0);
-    store_rec<T, kVfRec>(rec + (int64_t)t * kVfRec, r);
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int al = 0; al < 3; ++al)
+#pragma unroll
+          for (int be = 0; be < 3; ++be) {
+            T s2 = T(-0.0);
+#pragma unroll
+            for (int sv = 0; sv < 3; ++sv)
+#pragma unroll
+              for (int tv = 0; tv < 3; ++tv)
+                if (vf_coef(rr, sv) * vf_coef(j, tv) != 0)
+                  s2 += T(vf_coef(rr, sv) * vf_coef(j, tv)) * shess(z, 3 * sv + al, 3 * tv + be);
+            r[3 + 9 * j + 3 * al + be] = s2;
+          }
+      r[kVfRoleVals - 1] = z.v;
+      store_rec<T, kVfRoleVals>(rec + (int64_t)t * kVfRec + rr * kVfRoleVals, r);
+    }
   }
   if (epart) {
     __shared__ double red[kVfThreads / 32];
@@ -425,8 +445,9 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
   }
 }
 
-// Row pass: one thread per row adds its share of each of its terms (from the
-// records) to its gradient and its four blocks per term.
+// Row pass (used when the row kernel does not gather the terms itself): one
+// thread per row adds its role's slice of each of its terms to its gradient
+// and blocks; each term's four blocks are read before any is written.
 template <typename T>
 __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __restrict__ vrow,
                                                         const int32_t* __restrict__ ent,
@@ -444,47 +465,20 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __
     const int4 w1 = reinterpret_cast<const int4*>(ent)[2 * q + 1];
     if (!w1.y) continue;
     const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
-    T r[kVfRec];
-    load_rec<T, kVfRec>(rec + (int64_t)t * kVfRec, r);
+    T r[kVfRoleVals];
+    load_rec<T, kVfRoleVals>(rec + (int64_t)t * kVfRec + role * kVfRoleVals, r);
     const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
-    // the four blocks read first, in one round of independent loads: the
-    // updates go through the same pointer, so loads mixed with stores would
-    // each wait for the store before them
     T cur[4][9];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int q9 = 0; q9 < 9; ++q9) cur[j][q9] = H[(r0 + pos[j]) * 9 + q9];
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {  // the role as a compile-time index
-      if (rr != role) continue;
+    for (int al = 0; al < 3; ++al) gacc[al] += r[al];
 #pragma unroll
-      for (int al = 0; al < 3; ++al) {
-        T s2 = T(-0.0);
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int sv = 0; sv < 3; ++sv)
-          if (vf_coef(rr, sv) != 0) s2 += T(vf_coef(rr, sv)) * r[1 + 3 * sv + al];
-        gacc[al] += s2;
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int al = 0; al < 3; ++al)
-#pragma unroll
-          for (int be = 0; be < 3; ++be) {
-            T s2 = T(-0.0);
-#pragma unroll
-            for (int sv = 0; sv < 3; ++sv)
-#pragma unroll
-              for (int tv = 0; tv < 3; ++tv) {
-                const int a = 3 * sv + al, c = 3 * tv + be;
-                if (vf_coef(rr, sv) * vf_coef(j, tv) != 0)
-                  s2 += T(vf_coef(rr, sv) * vf_coef(j, tv)) *
-                        r[10 + (a <= c ? Tri<9>::idx(a, c) : Tri<9>::idx(c, a))];
-              }
-            cur[j][3 * al + be] += s2;
-          }
-    }
+      for (int q9 = 0; q9 < 9; ++q9) cur[j][q9] += r[3 + 9 * j + q9];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
