@@ -561,6 +561,7 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
     CREATE_CK(dev_alloc(c, &vs.scan_tmp, sizeof(int32_t) * scan_tmp_elems(V)));
     CREATE_CK(dev_alloc(c, &vs.epart,
                         sizeof(double) * std::max<size_t>(1, (mt + 255) / 256)));
+    CREATE_CK(dev_alloc(c, &vs.vslot, sizeof(int32_t) * 4 * std::max<size_t>(mt, 1)));
     char* rec = nullptr;
     CREATE_CK(dev_alloc(c, &rec, (size_t)c->esz * 160 * std::max<size_t>(mt, 1)));
     vs.rec = rec;

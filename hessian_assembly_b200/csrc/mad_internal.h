@@ -182,7 +182,8 @@ struct VfSet {
   int32_t* vrow = nullptr;  // [V+1] incidences per row (exclusive scan)
   int32_t* ent = nullptr;   // [4 max_terms][8] entries (see vf.cu)
   int32_t* scan_tmp = nullptr;
-  void* rec = nullptr;      // [max_terms][4][40] per-term, per-role records of the term pass
+  int32_t* vslot = nullptr; // [max_terms][4] entry index of each (term, role)
+  void* rec = nullptr;      // [4 max_terms][40] per-entry shares written by the term pass
   double* epart = nullptr;  // [ceil(max_terms / 256)] per-block energy of the term pass
 };
 cudaError_t launch_vf_install_expand(const VfSet& S, int n, const int32_t* vf, int V,

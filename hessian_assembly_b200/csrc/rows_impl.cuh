@@ -343,7 +343,8 @@ __device__ __forceinline__ void add4(T* b, const T* v) {
 template <typename T, int DOF, int AD, bool ENERGY, int S0, int FACES, bool PAIRS>
 __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile, int lane,
                                               uint32_t m, int d0, int d1, int pb, int pn,
-                                              const T* xi, const T* xti, T* row, double& energy) {
+                                              int vb, int ve, const T* xi, const T* xti, T* row,
+                                              double& energy) {
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
   const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
@@ -352,6 +353,17 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
   T acc[TD], gr[DOF];
   RowNew rn;
   if constexpr (PAIRS) load_row_new(A.pe_pos, pb, pn, nins, rn);
+  if constexpr (FACES == 4) {
+    // the row's first vertex-face share and entry, asked of L1 now, read
+    // after the edge terms
+    if (ve > vb && (A.mask & MAD_TERM_VF)) {
+      const char* p = reinterpret_cast<const char*>(A.vrec + (size_t)vb * kVfRoleVals);
+#pragma unroll
+      for (int l = 0; l < (int)(kVfRoleVals * sizeof(T)); l += 128)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(p + l));
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(A.vent + 8 * (size_t)vb));
+    }
+  }
   // The row's first pair entry is loaded before the edge terms are evaluated,
   // so that its partner's position (a random vertex) arrives meanwhile.
   int pc0 = 0, pw0 = 0;
@@ -490,13 +502,12 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
     // gradient, its four blocks, E); the blocks go to the staged row, the
     // diagonal block to the register accumulator
     if (A.mask & MAD_TERM_VF) {
-      const int vb = A.vrow[i], ve = A.vrow[i + 1];
       for (int q = vb; q < ve; ++q) {
         const int4 w0 = reinterpret_cast<const int4*>(A.vent)[2 * q];
         const int4 w1 = reinterpret_cast<const int4*>(A.vent)[2 * q + 1];
         if (!w1.y) continue;
-        const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
-        const T* r = A.vrec + (size_t)t * (4 * kVfRoleVals) + role * kVfRoleVals;
+        const int role = (int)((uint32_t)w0.x >> 30);
+        const T* r = A.vrec + (size_t)q * kVfRoleVals;
         T v[kVfRoleVals];
 #pragma unroll
         for (int q4 = 0; q4 < kVfRoleVals; q4 += 4) load4<T>(r + q4, v + q4);
@@ -542,7 +553,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   T* stage = (T*)smem_raw + wib * A.wstage;
   double energy = 0.0;
 
-  int d0 = 0, d1 = 0, pb = 0, pn = 0;
+  int d0 = 0, d1 = 0, pb = 0, pn = 0, vb = 0, ve = 0;
   uint32_t m = 0;
   T xi[DOF], xti[DOF];
   if (has) {
@@ -559,6 +570,12 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
       pb = A.prow[i];
       pn = A.prow[i + 1] - pb;
     }
+    if constexpr (FACES == 4) {
+      if (A.vrow) {
+        vb = A.vrow[i];
+        ve = A.vrow[i + 1];
+      }
+    }
   }
   // the warp's rows are consecutive in H: stage them from the first one
   const int dfirst = __shfl_sync(0xffffffffu, d0, 0);
@@ -567,7 +584,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_ro
   const bool staged = has && off + (d1 - d0) * B <= A.wstage;
   // rows that do not fit their warp's slice are assembled in place in H
   if (has)
-    rows_eval_row<T, DOF, AD, ENERGY, S0, FACES, PAIRS>(A, i, tile, lane, m, d0, d1, pb, pn, xi, xti,
+    rows_eval_row<T, DOF, AD, ENERGY, S0, FACES, PAIRS>(A, i, tile, lane, m, d0, d1, pb, pn, vb, ve, xi, xti,
                                         staged ? stage + off : A.H + (uint32_t)(d0 * B), energy);
   // ---- write-back of the warp's staged rows (a prefix of its 32 rows) -------
   fence_async_smem();

@@ -339,11 +339,13 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_fill(int n, const int32_t* __
   }
 }
 
-// per row: entries in (term, role) order, then the block positions
+// per row: entries in (term, role) order, then the block positions, and
+// for every (term, role) its entry's index (where the term pass writes that
+// vertex's share)
 __global__ void __launch_bounds__(kVfThreads) k_vf_finalize(
     int V, const int32_t* __restrict__ vrow, int32_t* ent, const int32_t* __restrict__ terms,
     const int32_t* __restrict__ F, int nF, const int32_t* __restrict__ rp,
-    const int32_t* __restrict__ ci, int32_t* status) {
+    const int32_t* __restrict__ ci, int32_t* vslot, int32_t* status) {
   const int i = blockIdx.x * kVfThreads + threadIdx.x;
   if (i >= V) return;
   const int b = vrow[i], e = vrow[i + 1];
@@ -372,6 +374,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_finalize(
       else w.w = rel;
     }
     if (!all) atomicOr(status, kStatusIndex);
+    vslot[4 * t + (int)((uint32_t)ent[8 * q] >> 30)] = q;
     reinterpret_cast<int4*>(ent)[2 * q] = make_int4(ent[8 * q], w.x, w.y, w.z);
     reinterpret_cast<int4*>(ent)[2 * q + 1] = make_int4(w.w, all ? 1 : 0, 0, 0);
   }
@@ -388,8 +391,8 @@ constexpr int kVfRec = 4 * kVfRoleVals;     // per term
 template <typename T, bool GEN>
 __global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
     int n, const int32_t* __restrict__ terms, const int32_t* __restrict__ F, int nF, int V,
-    const T* __restrict__ rest, T k, const T* __restrict__ x, T* __restrict__ rec,
-    double* epart) {
+    const int32_t* __restrict__ vslot, const T* __restrict__ rest, T k,
+    const T* __restrict__ x, T* __restrict__ rec, double* epart) {
   const int t = blockIdx.x * kVfThreads + threadIdx.x;
   double e = 0.0;
   int vid[4];
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
             r[3 + 9 * j + 3 * al + be] = s2;
           }
       r[kVfRoleVals - 1] = z.v;
-      store_rec<T, kVfRoleVals>(rec + (int64_t)t * kVfRec + rr * kVfRoleVals, r);
+      store_rec<T, kVfRoleVals>(rec + (int64_t)vslot[4 * t + rr] * kVfRoleVals, r);
     }
   }
   if (epart) {
@@ -466,7 +469,7 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __
     if (!w1.y) continue;
     const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
     T r[kVfRoleVals];
-    load_rec<T, kVfRoleVals>(rec + (int64_t)t * kVfRec + role * kVfRoleVals, r);
+    load_rec<T, kVfRoleVals>(rec + (int64_t)q * kVfRoleVals, r);
     const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
     T cur[4][9];
 #pragma unroll
@@ -606,7 +609,8 @@ cudaError_t launch_vf_install_tables(const VfSet& S, int n, int V, const int32_t
   if (n > 0) {
     k_vf_fill<<<nb, kVfThreads, 0, s>>>(n, S.terms, F, nF, V, S.vrow, cnt, S.ent);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_vf_finalize<<<nr, kVfThreads, 0, s>>>(V, S.vrow, S.ent, S.terms, F, nF, rp, ci, status);
+    k_vf_finalize<<<nr, kVfThreads, 0, s>>>(V, S.vrow, S.ent, S.terms, F, nF, rp, ci, S.vslot,
+                                            status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -618,7 +622,7 @@ cudaError_t vf_rows_t(const VfSet& S, const VfLaunch& L, void* g, void* H, doubl
   const unsigned nt = (unsigned)((S.n + kVfThreads - 1) / kVfThreads);
   const unsigned nr = (unsigned)((L.V + kVfThreads - 1) / kVfThreads);
   if (S.n > 0) {
-    k_vf_term_rec<T, GEN><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+    k_vf_term_rec<T, GEN><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V, S.vslot,
                                                     (const T*)L.rest, (T)L.k, (const T*)L.x,
                                                     (T*)S.rec, energy ? S.epart : nullptr);
     cudaError_t e = cudaGetLastError();
@@ -654,23 +658,23 @@ cudaError_t launch_vf_term_pass(int dtype, const VfSet& S, const VfLaunch& L, cu
   const unsigned nt = (unsigned)((S.n + kVfThreads - 1) / kVfThreads);
   if (dtype == MAD_F64) {
     if (L.generic)
-      k_vf_term_rec<double, true><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+      k_vf_term_rec<double, true><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V, S.vslot,
                                                              (const double*)L.rest, L.k,
                                                              (const double*)L.x, (double*)S.rec,
                                                              nullptr);
     else
-      k_vf_term_rec<double, false><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+      k_vf_term_rec<double, false><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V, S.vslot,
                                                               (const double*)L.rest, L.k,
                                                               (const double*)L.x,
                                                               (double*)S.rec, nullptr);
   } else {
     if (L.generic)
-      k_vf_term_rec<float, true><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+      k_vf_term_rec<float, true><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V, S.vslot,
                                                             (const float*)L.rest, (float)L.k,
                                                             (const float*)L.x, (float*)S.rec,
                                                             nullptr);
     else
-      k_vf_term_rec<float, false><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V,
+      k_vf_term_rec<float, false><<<nt, kVfThreads, 0, s>>>(S.n, S.terms, L.F, L.nF, L.V, S.vslot,
                                                              (const float*)L.rest, (float)L.k,
                                                              (const float*)L.x, (float*)S.rec,
                                                              nullptr);
