@@ -507,23 +507,25 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
         const int4 w1 = reinterpret_cast<const int4*>(A.vent)[2 * q + 1];
         if (!w1.y) continue;
         const int role = (int)((uint32_t)w0.x >> 30);
+        // the slice is read a block at a time (few registers: this branch
+        // runs on few rows and must not lower every row's occupancy)
         const T* r = A.vrec + (size_t)q * kVfRoleVals;
-        T v[kVfRoleVals];
+        if (ENERGY) energy += 0.25 * (double)r[kVfRoleVals - 1];
 #pragma unroll
-        for (int q4 = 0; q4 < kVfRoleVals; q4 += 4) load4<T>(r + q4, v + q4);
-        if (ENERGY) energy += 0.25 * (double)v[kVfRoleVals - 1];
-#pragma unroll
-        for (int a = 0; a < 3; ++a) gr[a] += v[a];
+        for (int a = 0; a < 3; ++a) gr[a] += r[a];
         const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+          T b9[9];
+#pragma unroll
+          for (int q9 = 0; q9 < 9; ++q9) b9[q9] = r[3 + 9 * j + q9];
           if (j == role) {
 #pragma unroll
             for (int a = 0; a < 3; ++a)
 #pragma unroll
-              for (int b2 = a; b2 < 3; ++b2) acc[Tri<3>::idx(a, b2)] += v[3 + 9 * j + 3 * a + b2];
+              for (int b2 = a; b2 < 3; ++b2) acc[Tri<3>::idx(a, b2)] += b9[3 * a + b2];
           } else {
-            add9<T>(row + pos[j] * B, v + 3 + 9 * j);
+            add9<T>(row + pos[j] * B, b9);
           }
         }
       }
@@ -762,6 +764,8 @@ __global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __r
   for (int q = 0; q < 9; ++q) out[9 * f + q] = o[q];
 }
 
+constexpr int kFacesPerThread = 2;
+
 // Per-face pass of the Hessian-vector product: one thread per face computes
 // (H_f v_f) for its three corners once; the row kernel then adds, for each
 // row, its corners' results.  Each face is differentiated once instead of
@@ -772,49 +776,59 @@ __global__ void __launch_bounds__(256) k_face_hv(int nF, bool vec2, const int32_
                                                  const T* __restrict__ Minv,
                                                  const T* __restrict__ area, T* __restrict__ out,
                                                  int kind) {
-  const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (f >= nF) return;
-  const int32_t a = F[3 * f], b = F[3 * f + 1], c = F[3 * f + 2];
-  T u[3][2], w[3][2], M[4];
-  const int32_t vid[3] = {a, b, c};
-  // [V][2] arrays: a vertex's pair is one 2-element load when both arrays
-  // are aligned to it (the caller's pointers need not be)
+  // kFacesPerThread faces per thread, their loads issued together: the
+  // grid is about one wave, and each thread overlaps its faces' latencies
   using T2 = typename std::conditional<sizeof(T) == 4, float2, double2>::type;
-  if (vec2) {
+  T u[kFacesPerThread][3][2], w[kFacesPerThread][3][2], M[kFacesPerThread][4],
+      ar[kFacesPerThread];
+  int64_t fs[kFacesPerThread];
+#pragma unroll
+  for (int h = 0; h < kFacesPerThread; ++h) {
+    const int64_t f = ((int64_t)blockIdx.x * kFacesPerThread + h) * 256 + threadIdx.x;
+    fs[h] = f;
+    if (f >= nF) continue;
+    const int32_t vid[3] = {F[3 * f], F[3 * f + 1], F[3 * f + 2]};
+    // [V][2] arrays: a vertex's pair is one 2-element load when both arrays
+    // are aligned to it (the caller's pointers need not be)
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      const T2 xu = reinterpret_cast<const T2*>(x)[vid[k]];
-      const T2 xv = reinterpret_cast<const T2*>(v)[vid[k]];
-      u[k][0] = xu.x;
-      u[k][1] = xu.y;
-      w[k][0] = xv.x;
-      w[k][1] = xv.y;
-    }
-  } else {
+      if (vec2) {
+        const T2 xu = reinterpret_cast<const T2*>(x)[vid[k]];
+        const T2 xv = reinterpret_cast<const T2*>(v)[vid[k]];
+        u[h][k][0] = xu.x;
+        u[h][k][1] = xu.y;
+        w[h][k][0] = xv.x;
+        w[h][k][1] = xv.y;
+      } else {
 #pragma unroll
-    for (int k = 0; k < 3; ++k)
-#pragma unroll
-      for (int al = 0; al < 2; ++al) {
-        u[k][al] = x[(int64_t)vid[k] * 2 + al];
-        w[k][al] = v[(int64_t)vid[k] * 2 + al];
+        for (int al = 0; al < 2; ++al) {
+          u[h][k][al] = x[(int64_t)vid[k] * 2 + al];
+          w[h][k][al] = v[(int64_t)vid[k] * 2 + al];
+        }
       }
+    }
+    load4<T>(Minv + 4 * f, M[h]);
+    ar[h] = area[f];
   }
-  load4<T>(Minv + 4 * f, M);
-  T o[6];
-  with_face2_kind(kind, [&](auto kc) {
-    hv_symdir_face<T, AD, decltype(kc)::value>(u[0], u[1], u[2], w[0], w[1], w[2], M, area[f],
-                                                 o);
-  });
-  T2* o2 = reinterpret_cast<T2*>(out) + 3 * f;  // one corner's pair per 8 (16) bytes
 #pragma unroll
-  for (int c2 = 0; c2 < 3; ++c2) {
-    T2 v2;
-    v2.x = o[2 * c2];
-    v2.y = o[2 * c2 + 1];
-    o2[c2] = v2;
+  for (int h = 0; h < kFacesPerThread; ++h) {
+    const int64_t f = fs[h];
+    if (f >= nF) continue;
+    T o[6];
+    with_face2_kind(kind, [&](auto kc) {
+      hv_symdir_face<T, AD, decltype(kc)::value>(u[h][0], u[h][1], u[h][2], w[h][0], w[h][1],
+                                                 w[h][2], M[h], ar[h], o);
+    });
+    T2* o2 = reinterpret_cast<T2*>(out) + 3 * f;  // one corner's pair per 8 (16) bytes
+#pragma unroll
+    for (int c2 = 0; c2 < 3; ++c2) {
+      T2 v2;
+      v2.x = o[2 * c2];
+      v2.y = o[2 * c2 + 1];
+      o2[c2] = v2;
+    }
   }
 }
-
 
 template <typename T>
 RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, const void* v,
@@ -996,7 +1010,7 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
     if constexpr (DOF == 2) {
       if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
         if (L.nF > 0) {
-          const unsigned nbf = (unsigned)((L.nF + 255) / 256);
+          const unsigned nbf = (unsigned)((L.nF + 256 * kFacesPerThread - 1) / (256 * kFacesPerThread));
           const bool vec2 = ((((uintptr_t)x) | ((uintptr_t)v)) % (2 * sizeof(T))) == 0;
           k_face_hv<T, AD><<<nbf, 256, 0, s>>>(L.nF, vec2, L.F, (const T*)x, (const T*)v,
                                                (const T*)t.face_Minv, (const T*)t.face_area,
