@@ -629,12 +629,8 @@ __device__ __forceinline__ void add_corner_hv(const T* __restrict__ fhv, uint32_
   }
 }
 
-// FMODE: 0 no face terms; 1 face terms from the per-face pass (k_face_hv,
-// k_face_hv_area); 2, 3, 4 (dof 2) each row evaluates its corner's share of
-// its faces' products itself, for symmetric Dirichlet, ARAP or both.
-template <typename T, int DOF, int AD, int S0, int FMODE>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FMODE ? 1 : 0>()) k_rows_hvp(const RArgs<T> A) {
-  constexpr bool FACES = FMODE == 1;
+template <typename T, int DOF, int AD, int S0, bool FACES>
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES ? 1 : 0>()) k_rows_hvp(const RArgs<T> A) {
   constexpr int TD = Tri<DOF>::size;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int tile = blockIdx.x * kWarps + wib;
@@ -643,7 +639,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FMODE ? 1 : 0>
   const bool pairs = (A.mask & MAD_TERM_PAIR) && A.prow != nullptr;
   // the row's own position, direction and slot meta are needed only by the
   // vertex, edge and pair terms (face terms come from the per-face pass)
-  const bool own = (A.mask & (MAD_TERM_INERTIA | MAD_TERM_SPRING | MAD_TERM_PAIR)) || FMODE >= 2;
+  const bool own = A.mask & (MAD_TERM_INERTIA | MAD_TERM_SPRING | MAD_TERM_PAIR);
   T xi[DOF], vi[DOF], yr[DOF];
   uint32_t m = 0;
 #pragma unroll
@@ -720,22 +716,6 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FMODE ? 1 : 0>
       EdgeRes<T, DOF, AD> Rp;
       eval_edge_res<T, DOF, AD>(xi, xj, A.pe_rest[e], A.kp, Rp);
       hv(Rp, vj);
-    }
-  }
-  if constexpr (FMODE >= 2 && DOF == 2) {
-    // the row's corner share of each of its faces' products, evaluated here
-    constexpr int KIND = FMODE == 2 ? kFaceSymDir : FMODE == 3 ? kFaceArap : (kFaceSymDir | kFaceArap);
-    if (A.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
-      row_faces<T>(A, i, tile, lane,
-                   [&](const T* xj, const T* xk, int j, int k, int c, int, int, const T* M,
-                       T ar) {
-                     const T vj[2] = {A.v[(uint32_t)(j * 2)], A.v[(uint32_t)(j * 2 + 1)]};
-                     const T vk[2] = {A.v[(uint32_t)(k * 2)], A.v[(uint32_t)(k * 2 + 1)]};
-                     T o[2];
-                     hv_symdir_row<T, AD, KIND>(xi, xj, xk, vi, vj, vk, c, M, ar, o);
-                     yr[0] += o[0];
-                     yr[1] += o[1];
-                   });
     }
   }
   if constexpr (FACES) {
@@ -1021,21 +1001,12 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
     const bool sp = t.mask & MAD_TERM_SPRING;
     // the row pass after a per-face pass (face terms), or alone
     // the row pass after the per-face pass, or alone
-    auto rows = [&](auto fmc) {
-      constexpr int FM = decltype(fmc)::value;
-      if (sp) k_rows_hvp<T, DOF, AD, kS0Max, FM><<<nb, kRowThreads, 0, s>>>(A);
-      else k_rows_hvp<T, DOF, AD, 0, FM><<<nb, kRowThreads, 0, s>>>(A);
+    auto rows = [&](auto facesc) {
+      constexpr bool FC = decltype(facesc)::value;
+      if (sp) k_rows_hvp<T, DOF, AD, kS0Max, FC><<<nb, kRowThreads, 0, s>>>(A);
+      else k_rows_hvp<T, DOF, AD, 0, FC><<<nb, kRowThreads, 0, s>>>(A);
       return cudaGetLastError();
     };
-    if constexpr (DOF == 2 && AD != kAdFull) {
-      // dof-2 faces: one pass, each row evaluating its corners' shares
-      if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
-        const int kind = face2_kind(t.mask);
-        if (kind == kFaceSymDir) return rows(std::integral_constant<int, 2>{});
-        if (kind == kFaceArap) return rows(std::integral_constant<int, 3>{});
-        return rows(std::integral_constant<int, 4>{});
-      }
-    }
     if constexpr (DOF == 2) {
       if (t.mask & (MAD_TERM_SYMDIR | MAD_TERM_ARAP)) {
         if (L.nF > 0) {
@@ -1047,7 +1018,7 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
           const cudaError_t e = cudaGetLastError();
           if (e != cudaSuccess) return e;
         }
-        return rows(std::integral_constant<int, 1>{});
+        return rows(std::true_type{});
       }
     }
     if constexpr (DOF == 3) {
@@ -1060,11 +1031,11 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
           const cudaError_t e = cudaGetLastError();
           if (e != cudaSuccess) return e;
         }
-        return rows(std::integral_constant<int, 1>{});
+        return rows(std::true_type{});
       }
     }
-    if (L.s0 <= 6) k_rows_hvp<T, DOF, AD, 6, 0><<<nb, kRowThreads, 0, s>>>(A);
-    else k_rows_hvp<T, DOF, AD, kS0Max, 0><<<nb, kRowThreads, 0, s>>>(A);
+    if (L.s0 <= 6) k_rows_hvp<T, DOF, AD, 6, false><<<nb, kRowThreads, 0, s>>>(A);
+    else k_rows_hvp<T, DOF, AD, kS0Max, false><<<nb, kRowThreads, 0, s>>>(A);
     return cudaGetLastError();
   });
 }

@@ -591,46 +591,6 @@ __device__ __forceinline__ void rotated_weights(const T* M, int c, T (&wr)[3][2]
   }
 }
 
-// One corner's share of (H_f v_f) for a dof-2 face term, for the row of
-// corner i: J and dJ = sum_l v_l w_l^T in the face's own corner order, the
-// J-space product t = H_J dJ, and t projected on the row's corner weights.
-// (AD: reduced or generic seeding on J.)
-template <typename T, int AD, int KIND>
-__device__ __forceinline__ void hv_symdir_row(const T* xi, const T* xj, const T* xk,
-                                              const T* vi, const T* vj, const T* vk, int c,
-                                              const T* M, T A, T* out) {
-  static_assert(AD != kAdFull, "the full-stencil seeding uses the per-face pass");
-  T wr[3][2];
-  rotated_weights<T>(M, c, wr);
-  T Jv[4], dJ[4];
-#pragma unroll
-  for (int al = 0; al < 2; ++al) {
-    // corners 0, 1, 2 of the face: c = 0 -> (i, j, k), 1 -> (k, i, j), 2 -> (j, k, i)
-    const T u0 = sel3(c, xi[al], xk[al], xj[al]);
-    const T u1 = sel3(c, xj[al], xi[al], xk[al]);
-    const T u2 = sel3(c, xk[al], xj[al], xi[al]);
-    const T d0 = sel3(c, vi[al], vk[al], vj[al]);
-    const T d1 = sel3(c, vj[al], vi[al], vk[al]);
-    const T d2 = sel3(c, vk[al], vj[al], vi[al]);
-#pragma unroll
-    for (int ga = 0; ga < 2; ++ga) {
-      Jv[2 * al + ga] = (u1 - u0) * M[ga] + (u2 - u0) * M[2 + ga];
-      dJ[2 * al + ga] = (d1 - d0) * M[ga] + (d2 - d0) * M[2 + ga];
-    }
-  }
-  const HyperDual<T, 4> e = face2_hd<KIND, AD>(Jv, A);
-  T t[4];
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    T s = T(0);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) s += hess(e, p, q) * dJ[q];
-    t[p] = s;
-  }
-#pragma unroll
-  for (int al = 0; al < 2; ++al) out[al] = t[2 * al] * wr[0][0] + t[2 * al + 1] * wr[0][1];
-}
-
 template <typename T, int AD, int KIND>
 __device__ __forceinline__ void eval_symdir_row(const T* xi, const T* xj, const T* xk, int c,
                                                 const T* M, T A, FaceRow<T>& o) {
