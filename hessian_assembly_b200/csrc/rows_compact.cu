@@ -7,8 +7,8 @@
 // key design 3: the CSR block offsets come from a table built once per
 // topology, so assembly needs no search.
 //
-// Same work as k_rows_eval (rows_impl.cuh) for a term set of springs and
-// inertia on the mesh pattern: one thread per Hessian row, the row's edge
+// Same work as k_rows_eval (rows_impl.cuh) for a term set of springs,
+// inertia and runtime pairs: one thread per Hessian row, the row's edge
 // terms evaluated with forward-mode AD numbers in registers, each row staged
 // in its warp's slice of shared memory and written back with one 1-D bulk
 // copy per warp.  The row tables it reads are the compact ones
@@ -16,7 +16,10 @@
 // row_ptr or meta word.  A row's block positions follow from its slots
 // (columns ascend, the diagonal sits after the columns below the row), and
 // the row's first block from the tile's row_ptr plus a warp prefix sum of
-// the row lengths.
+// the row lengths.  With runtime pairs active (method section, key design 4:
+// blocks inserted into the pattern between steps) the rows come from the
+// active row_ptr instead, and a mesh block's position is moved past the
+// pair blocks inserted before it in its row.
 #include "rows_impl.cuh"
 
 namespace mad {
@@ -35,6 +38,13 @@ struct CArgs {
   T k;
   const T* xt;
   T w;
+  // runtime pairs (the active pattern's row_ptr and per-row pair entries)
+  const int32_t* rp;
+  const int32_t* prow;
+  const int32_t* pe_col;
+  const int32_t* pe_pos;
+  const T* pe_rest;
+  T kp;
   unsigned mask;
   double* epart;
   int V, s0, wstage;
@@ -82,8 +92,9 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 __device__ __forceinline__ int slot_dcol(uint32_t w) { return (int)(int16_t)(w & 0xFFFFu); }
 __device__ __forceinline__ int slot_deid(uint32_t w) { return (int)(int16_t)(w >> 16); }
 
-template <typename T, int DOF, int AD, bool ENERGY, int S0, bool SHARD>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, bool SHARD, bool PAIRS>
 __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T>* S) {
+  static_assert(!(SHARD && PAIRS), "a shard launch carries no pairs");
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
   constexpr int VEC = 16 / (int)sizeof(T);
@@ -114,6 +125,10 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
       } else if (lane >= 16 && lane < 16 + XL && (A.mask & MAD_TERM_INERTIA)) {
         const int64_t e = (int64_t)tp * 32 * DOF + (lane - 16) * (128 / (int)sizeof(T));
         if (e < nx) prefetch_l2(A.xt + e);
+      } else if (PAIRS && lane == 28) {
+        prefetch_l2(A.rp + (size_t)tp * 32);
+      } else if (PAIRS && lane == 29) {
+        prefetch_l2(A.prow + (size_t)tp * 32);
       }
     }
   }
@@ -134,6 +149,14 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
   for (int k = 0; k < S0; ++k) {
     sw[k] = 0u;
     if (has && k < A.s0) sw[k] = A.cslots[(uint32_t)((tile * A.s0 + k) * 32 + lane)];
+  }
+  // the row's place in the active pattern and its pair entries
+  int pd0 = 0, pd1 = 0, pb = 0, pn = 0;
+  if (PAIRS && has) {
+    pd0 = A.rp[i];
+    pd1 = A.rp[i + 1];
+    pb = A.prow[i];
+    pn = A.prow[i + 1] - pb;
   }
   T xi[DOF], xti[DOF];
   if (has) {
@@ -157,6 +180,18 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     for (int a = 0; a < DOF; ++a) xb[k][a] = xs[a];
     l0[k] = A.L0[th.y + slot_deid(sw[k])];
   }
+  // the row's first pair entry and its partner's position (a random vertex),
+  // asked for before the edge terms are evaluated
+  const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
+  int pw0 = 0;
+  T pr0 = T(0), xp0[DOF];
+  if (pairs && pn > 0) {
+    const int pc0 = A.pe_col[pb];
+    pw0 = A.pe_pos[pb];
+    pr0 = A.pe_rest[pb];
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xp0[a] = A.x[(uint32_t)(pc0 * DOF + a)];
+  }
   // row length (off-diagonal slots + overflow + the diagonal) and the row's
   // first block: the tile's row_ptr plus the lengths of the rows before it
   int noff = 0, dpos = 0, o0 = 0, no = 0;
@@ -171,14 +206,31 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     for (int q = 0; q < no; ++q) dpos += A.ofl[o0 + q].x < i;
   }
   noff += no;
-  const int len = has ? noff + 1 : 0;
-  int incl = len;
+  int d0, d1;
+  if constexpr (PAIRS) {
+    d0 = pd0;
+    d1 = pd1;
+  } else {
+    const int len = has ? noff + 1 : 0;
+    int incl = len;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    d0 = th.x + incl - len;
+    d1 = d0 + len;
   }
-  const int d0 = th.x + incl - len, d1 = d0 + len;
+  // blocks the pairs inserted into the row, and (the first kRowNew of them)
+  // their positions
+  const int nins = PAIRS ? (d1 - d0) - (noff + 1) : 0;
+  RowNew rn;
+  if constexpr (PAIRS) load_row_new(A.pe_pos, pb, pn, nins, rn);
+  // a mesh block's position in the active row
+  auto at = [&](int p) {
+    if constexpr (PAIRS) return nins == 0 ? p : row_pos_new(rn, A.pe_pos, pb, pn, nins, p);
+    return p;
+  };
 
   const int dfirst = __shfl_sync(0xffffffffu, d0, 0);
   T* const h0 = A.H + (uint32_t)((dfirst - hoff) * B);  // the warp's first block in H
@@ -187,6 +239,26 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
   const bool staged = has && off + (d1 - d0) * B <= A.wstage;
   if (has) {
     T* row = staged ? stage + off : h0 + (uint32_t)((d0 - dfirst) * B);
+    if (PAIRS && springs && nins > 0) {
+      // inserted blocks no edge term stores start at 0
+#pragma unroll
+      for (int k = 0; k < kRowNew; ++k)
+        if (k < nins) {
+          T* b = row + rn.np[k] * B;
+#pragma unroll
+          for (int q = 0; q < B; ++q) b[q] = T(0);
+        }
+      if (nins > kRowNew) {
+        for (int e = pb; e < pb + pn; ++e) {
+          const int32_t wv = A.pe_pos[e];
+          if (wv & kPairNewBlock) {
+            T* b = row + (wv & kPairPosMask) * B;
+#pragma unroll
+            for (int q = 0; q < B; ++q) b[q] = T(0);
+          }
+        }
+      }
+    }
     T acc[TD], gr[DOF];
     if (A.mask & MAD_TERM_INERTIA) {
       T Ei, Hi[B];
@@ -210,7 +282,7 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
         eval_edge_res<T, DOF, AD>(xi, xb[k], l0[k], A.k, R);
         // block position: the slots before it plus the diagonal when the
         // column lies above the row
-        const int p = k + (slot_dcol(sw[k]) > 0);
+        const int p = at(k + (slot_dcol(sw[k]) > 0));
         apply_edge_side<true>(R, 0, acc, row + p * B, gr);
         if (ENERGY) energy += 0.5 * (double)edge_energy(R);
       }
@@ -222,7 +294,7 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
         for (int a = 0; a < DOF; ++a) xo[a] = xs[a];
         EdgeRes<T, DOF, AD> R;
         eval_edge_res<T, DOF, AD>(xi, xo, A.L0[e.y], A.k, R);
-        const int p = A.s0 + q + (e.x > i);
+        const int p = at(A.s0 + q + (e.x > i));
         apply_edge_side<true>(R, 0, acc, row + p * B, gr);
         if (ENERGY) energy += 0.5 * (double)edge_energy(R);
       }
@@ -230,7 +302,29 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
       // without edge terms every off-diagonal block of the row is zero
       for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
     }
-    T* d = row + dpos * B;
+    if (pairs) {
+      for (int e = pb; e < pb + pn; ++e) {
+        int pw;
+        T xj[DOF], rest;
+        if (e == pb) {
+          pw = pw0;
+          rest = pr0;
+#pragma unroll
+          for (int a = 0; a < DOF; ++a) xj[a] = xp0[a];
+        } else {
+          const int j = A.pe_col[e];
+          pw = A.pe_pos[e];
+          rest = A.pe_rest[e];
+#pragma unroll
+          for (int a = 0; a < DOF; ++a) xj[a] = A.x[(uint32_t)(j * DOF + a)];
+        }
+        EdgeRes<T, DOF, AD> Rp;
+        eval_edge_res<T, DOF, AD>(xi, xj, rest, A.kp, Rp);
+        apply_edge_side<false>(Rp, 0, acc, row + (pw & kPairPosMask) * B, gr);
+        if (ENERGY) energy += 0.5 * (double)edge_energy(Rp);
+      }
+    }
+    T* d = row + at(dpos) * B;
 #pragma unroll
     for (int a = 0; a < DOF; ++a)
 #pragma unroll
@@ -270,16 +364,16 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
   if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
 }
 
-template <typename T, int DOF, int AD, bool ENERGY, int S0>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, bool PAIRS>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
     k_rows_eval_c(const CArgs<T> A) {
-  rows_c_body<T, DOF, AD, ENERGY, S0, false>(A, nullptr);
+  rows_c_body<T, DOF, AD, ENERGY, S0, false, PAIRS>(A, nullptr);
 }
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
     k_rows_eval_cs(const CArgs<T> A, const __grid_constant__ ShardArgs<T> S) {
-  rows_c_body<T, DOF, AD, ENERGY, S0, true>(A, &S);
+  rows_c_body<T, DOF, AD, ENERGY, S0, true, false>(A, &S);
 }
 
 // Shared-memory carve-out asked for the kernel, in percent of the unified
@@ -290,10 +384,11 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
 #endif
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0>
-cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, int nb, size_t smem,
+cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, int nb, size_t smem,
                      cudaStream_t s, bool set) {
   if (set) {
-    const void* ks[2] = {(const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0>,
+    const void* ks[3] = {(const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0, false>,
+                         (const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0, true>,
                          (const void*)k_rows_eval_cs<T, DOF, AD, ENERGY, S0>};
     for (const void* k : ks) {
       cudaError_t e;
@@ -309,21 +404,23 @@ cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, int nb, size_t sm
   }
   if (S)
     k_rows_eval_cs<T, DOF, AD, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A, *S);
+  else if (pairs)
+    k_rows_eval_c<T, DOF, AD, ENERGY, S0, true><<<nb, kRowThreads, smem, s>>>(A);
   else
-    k_rows_eval_c<T, DOF, AD, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A);
+    k_rows_eval_c<T, DOF, AD, ENERGY, S0, false><<<nb, kRowThreads, smem, s>>>(A);
   return cudaGetLastError();
 }
 
 template <typename T, int DOF, int S0>
-cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, int ad, bool energy, int nb,
-                      size_t smem, cudaStream_t s, bool set) {
+cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, int ad, bool energy,
+                      int nb, size_t smem, cudaStream_t s, bool set) {
   if (set) {
     for (int a : {kAdReduced, kAdFull, kAdGeneric}) {
       const cudaError_t e = with_ad(a, [&](auto adc) {
         constexpr int AD = decltype(adc)::value;
-        const cudaError_t e1 = launch_c<T, DOF, AD, true, S0>(A, S, nb, smem, s, true);
+        const cudaError_t e1 = launch_c<T, DOF, AD, true, S0>(A, S, false, nb, smem, s, true);
         if (e1 != cudaSuccess) return e1;
-        return launch_c<T, DOF, AD, false, S0>(A, S, nb, smem, s, true);
+        return launch_c<T, DOF, AD, false, S0>(A, S, false, nb, smem, s, true);
       });
       if (e != cudaSuccess) return e;
     }
@@ -331,8 +428,8 @@ cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, int ad, bool ene
   }
   return with_ad(ad, [&](auto adc) {
     constexpr int AD = decltype(adc)::value;
-    if (energy) return launch_c<T, DOF, AD, true, S0>(A, S, nb, smem, s, false);
-    return launch_c<T, DOF, AD, false, S0>(A, S, nb, smem, s, false);
+    if (energy) return launch_c<T, DOF, AD, true, S0>(A, S, pairs, nb, smem, s, false);
+    return launch_c<T, DOF, AD, false, S0>(A, S, pairs, nb, smem, s, false);
   });
 }
 
@@ -351,6 +448,12 @@ CArgs<T> make_cargs(const RowsLaunch& L, const mad_terms& t, const void* x, void
   A.k = (T)t.spring_k;
   A.xt = (const T*)t.inertia_xt;
   A.w = (T)t.inertia_w;
+  A.rp = L.rp;
+  A.prow = L.prow;
+  A.pe_col = L.pe_col;
+  A.pe_pos = L.pe_pos;
+  A.pe_rest = (const T*)L.pe_rest;
+  A.kp = (T)t.pair_k;
   A.mask = t.mask;
   A.epart = energy ? L.epart : nullptr;
   A.V = L.V;
@@ -363,10 +466,11 @@ template <typename T, int DOF>
 cudaError_t dispatch_c(const RowsLaunch& L, const CArgs<T>& A, const ShardArgs<T>* S, int ad,
                        double* energy, int nb, cudaStream_t s) {
   const size_t smem = rows_smem_bytes(L);
-  cudaError_t e = L.s0 <= 6
-                      ? launch_c4<T, DOF, 6>(A, S, ad, energy != nullptr, nb, smem, s, false)
-                      : launch_c4<T, DOF, kS0Max>(A, S, ad, energy != nullptr, nb, smem, s,
-                                                  false);
+  const bool pairs = !S && L.prow != nullptr;
+  cudaError_t e =
+      L.s0 <= 6
+          ? launch_c4<T, DOF, 6>(A, S, pairs, ad, energy != nullptr, nb, smem, s, false)
+          : launch_c4<T, DOF, kS0Max>(A, S, pairs, ad, energy != nullptr, nb, smem, s, false);
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
   return cudaGetLastError();
@@ -406,9 +510,9 @@ cudaError_t rows_eval_shard_t(const RowsLaunch& L, const mad_terms& t, int nrank
 template <typename T, int DOF>
 cudaError_t rows_compact_limits_t(size_t bytes) {
   CArgs<T> A{};
-  cudaError_t e = launch_c4<T, DOF, 6>(A, nullptr, kAdReduced, false, 0, bytes, 0, true);
+  cudaError_t e = launch_c4<T, DOF, 6>(A, nullptr, false, kAdReduced, false, 0, bytes, 0, true);
   if (e != cudaSuccess) return e;
-  return launch_c4<T, DOF, kS0Max>(A, nullptr, kAdReduced, false, 0, bytes, 0, true);
+  return launch_c4<T, DOF, kS0Max>(A, nullptr, false, kAdReduced, false, 0, bytes, 0, true);
 }
 
 template cudaError_t rows_eval_compact_t<float, 2>(const RowsLaunch&, const mad_terms&, const void*,

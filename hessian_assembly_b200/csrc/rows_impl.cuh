@@ -976,8 +976,8 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
       e = faces_k(std::integral_constant<int, kS0Max>{});
     else
       e = faces_k(std::integral_constant<int, 0>{});
-  } else if (L.cslots != nullptr && !pairs) {
-    // the mesh pattern with compact slot tables
+  } else if (L.cslots != nullptr) {
+    // edge, vertex and pair terms with compact slot tables
     return rows_eval_compact_t<T, DOF>(L, t, x, g, H, energy, s);
   } else if (L.s0 <= 6) {
     // slot-table rows of width <= 6 (triangle meshes of valence <= 6) use the
