@@ -64,6 +64,7 @@ struct mad_ctx {
   int32_t* rows_fcslots = nullptr;
   int32_t* rows_fcofl = nullptr;
   void* face_hv = nullptr;  // [nF][3][2] scratch of the face Hessian-vector product
+  void* pe_xr = nullptr;    // [2*max_pairs][4] partner position + rest per pair entry
   double* epart = nullptr;
   size_t smem_eval = 0, smem_hvp = 0;
   // dynamic pattern
@@ -209,6 +210,7 @@ RowsLaunch rows_launch(const mad_ctx* c) {
     L.pe_col = b.pe_col;
     L.pe_pos = b.pe_pos;
     L.pe_rest = b.pe_rest;
+    L.pe_xr = c->pe_xr;
   }
   return L;
 }
@@ -538,6 +540,7 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
       CREATE_CK(dev_alloc(c, &rest_buf, (size_t)c->esz * pe));
       b.pe_rest = rest_buf;
     }
+    CREATE_CK(dev_alloc(c, &c->pe_xr, (size_t)c->esz * 4 * pe));
     CREATE_CK(dev_alloc(c, &c->cnt, sizeof(int32_t) * (V + 1)));
     CREATE_CK(cudaMemsetAsync(c->cnt, 0, sizeof(int32_t) * (V + 1), s));
     CREATE_CK(dev_alloc(c, &c->tsum, sizeof(int32_t) * pair_scratch_elems(V)));

@@ -299,6 +299,10 @@ struct RowsLaunch {
   const int32_t* pe_col;
   const int32_t* pe_pos;
   const void* pe_rest;
+  // [2*max_pairs][4] per pair entry: the partner's position (DOF values,
+  // zero padded) and the rest length in the last value; scratch the compact
+  // row kernel fills before each assembly with pairs
+  void* pe_xr = nullptr;
   double* epart;  // [rows_blocks(V)]
   // installed vertex-face terms gathered into the rows (nullptr: none)
   const int32_t* vrow = nullptr;

@@ -43,7 +43,7 @@ struct CArgs {
   const int32_t* prow;
   const int32_t* pe_col;
   const int32_t* pe_pos;
-  const T* pe_rest;
+  const T* pe_xr;  // per entry: partner position (zero padded to 4) + rest length
   T kp;
   unsigned mask;
   double* epart;
@@ -87,6 +87,65 @@ __device__ __forceinline__ const T* shard_x(const ShardArgs<T>& S, int v) {
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Entry e's partner position (DOF values) and rest length, gathered by
+// k_pair_gather: four values, one 16-byte load for fp32, two for fp64.
+template <typename T, int DOF>
+__device__ __forceinline__ void load_xr(const T* __restrict__ xr, int e, T* xj, T& rest) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 q = reinterpret_cast<const float4*>(xr)[e];
+    xj[0] = q.x;
+    xj[1] = q.y;
+    if constexpr (DOF == 3) xj[2] = q.z;
+    rest = q.w;
+  } else {
+    const double2 q0 = reinterpret_cast<const double2*>(xr)[2 * e];
+    const double2 q1 = reinterpret_cast<const double2*>(xr)[2 * e + 1];
+    xj[0] = q0.x;
+    xj[1] = q0.y;
+    if constexpr (DOF == 3) xj[2] = q1.x;
+    rest = q1.y;
+  }
+}
+
+// Before an assembly with pairs: for every live pair entry e (prow[V] of
+// them) the partner's position and the entry's rest length, side by side.
+// The row kernel then finds them next to the entry's position word instead
+// of behind a dependent load at a random vertex.
+constexpr int kGatherBlocks = 4 * 148;
+template <typename T, int DOF>
+__global__ void __launch_bounds__(256) k_pair_gather(const int32_t* __restrict__ nent,
+                                                     const int32_t* __restrict__ pe_col,
+                                                     const T* __restrict__ pe_rest,
+                                                     const T* __restrict__ x, T* __restrict__ xr) {
+  const int n = *nent;
+  const int stride = gridDim.x * blockDim.x;
+#pragma unroll 1
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += 2 * stride) {
+    const int e2 = e + stride;
+    const int j0 = pe_col[e];
+    const int j1 = e2 < n ? pe_col[e2] : j0;
+    T q0[4] = {T(0), T(0), T(0), T(0)}, q1[4] = {T(0), T(0), T(0), T(0)};
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) {
+      q0[a] = x[(uint32_t)(j0 * DOF + a)];
+      q1[a] = x[(uint32_t)(j1 * DOF + a)];
+    }
+    q0[3] = pe_rest[e];
+    q1[3] = e2 < n ? pe_rest[e2] : T(0);
+    if constexpr (sizeof(T) == 4) {
+      reinterpret_cast<float4*>(xr)[e] = make_float4(q0[0], q0[1], q0[2], q0[3]);
+      if (e2 < n) reinterpret_cast<float4*>(xr)[e2] = make_float4(q1[0], q1[1], q1[2], q1[3]);
+    } else {
+      reinterpret_cast<double2*>(xr)[2 * e] = make_double2(q0[0], q0[1]);
+      reinterpret_cast<double2*>(xr)[2 * e + 1] = make_double2(q0[2], q0[3]);
+      if (e2 < n) {
+        reinterpret_cast<double2*>(xr)[2 * e2] = make_double2(q1[0], q1[1]);
+        reinterpret_cast<double2*>(xr)[2 * e2 + 1] = make_double2(q1[2], q1[3]);
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ int slot_dcol(uint32_t w) { return (int)(int16_t)(w & 0xFFFFu); }
@@ -180,17 +239,14 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     for (int a = 0; a < DOF; ++a) xb[k][a] = xs[a];
     l0[k] = A.L0[th.y + slot_deid(sw[k])];
   }
-  // the row's first pair entry and its partner's position (a random vertex),
-  // asked for before the edge terms are evaluated
+  // the row's first pair entry, asked for before the edge terms are
+  // evaluated
   const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
   int pw0 = 0;
   T pr0 = T(0), xp0[DOF];
   if (pairs && pn > 0) {
-    const int pc0 = A.pe_col[pb];
     pw0 = A.pe_pos[pb];
-    pr0 = A.pe_rest[pb];
-#pragma unroll
-    for (int a = 0; a < DOF; ++a) xp0[a] = A.x[(uint32_t)(pc0 * DOF + a)];
+    load_xr<T, DOF>(A.pe_xr, pb, xp0, pr0);
   }
   // row length (off-diagonal slots + overflow + the diagonal) and the row's
   // first block: the tile's row_ptr plus the lengths of the rows before it
@@ -312,11 +368,8 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
 #pragma unroll
           for (int a = 0; a < DOF; ++a) xj[a] = xp0[a];
         } else {
-          const int j = A.pe_col[e];
           pw = A.pe_pos[e];
-          rest = A.pe_rest[e];
-#pragma unroll
-          for (int a = 0; a < DOF; ++a) xj[a] = A.x[(uint32_t)(j * DOF + a)];
+          load_xr<T, DOF>(A.pe_xr, e, xj, rest);
         }
         EdgeRes<T, DOF, AD> Rp;
         eval_edge_res<T, DOF, AD>(xi, xj, rest, A.kp, Rp);
@@ -452,7 +505,7 @@ CArgs<T> make_cargs(const RowsLaunch& L, const mad_terms& t, const void* x, void
   A.prow = L.prow;
   A.pe_col = L.pe_col;
   A.pe_pos = L.pe_pos;
-  A.pe_rest = (const T*)L.pe_rest;
+  A.pe_xr = (const T*)L.pe_xr;
   A.kp = (T)t.pair_k;
   A.mask = t.mask;
   A.epart = energy ? L.epart : nullptr;
@@ -482,6 +535,13 @@ template <typename T, int DOF>
 cudaError_t rows_eval_compact_t(const RowsLaunch& L, const mad_terms& t, const void* x, void* g,
                                 void* H, double* energy, cudaStream_t s) {
   const CArgs<T> A = make_cargs<T>(L, t, x, g, H, energy != nullptr);
+  if (L.prow && (t.mask & MAD_TERM_PAIR)) {
+    // four blocks per SM (148 on a B200) stride over the live entries
+    k_pair_gather<T, DOF><<<kGatherBlocks, 256, 0, s>>>(L.prow + L.V, L.pe_col, (const T*)L.pe_rest,
+                                                  (const T*)x, (T*)L.pe_xr);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   return dispatch_c<T, DOF>(L, A, nullptr, ad_form(t.flags), energy,
                             rows_blocks(L.V), s);
 }

@@ -386,7 +386,6 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_finalize(
 // vertices (4 x 9), then E in the last of kVfRoleVals values.  A row then
 // only adds its role's slice.
 constexpr int kVfRoleVals = 40;             // 3 + 36 + E
-constexpr int kVfRec = 4 * kVfRoleVals;     // per term
 
 template <typename T, bool GEN>
 __global__ void __launch_bounds__(kVfThreads) k_vf_term_rec(
@@ -467,7 +466,6 @@ __global__ void __launch_bounds__(kVfThreads) k_vf_rows(int V, const int32_t* __
     const int4 w0 = reinterpret_cast<const int4*>(ent)[2 * q];
     const int4 w1 = reinterpret_cast<const int4*>(ent)[2 * q + 1];
     if (!w1.y) continue;
-    const int t = w0.x & 0x3FFFFFFF, role = (int)((uint32_t)w0.x >> 30);
     T r[kVfRoleVals];
     load_rec<T, kVfRoleVals>(rec + (int64_t)q * kVfRoleVals, r);
     const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
