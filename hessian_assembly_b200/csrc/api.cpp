@@ -203,6 +203,7 @@ RowsLaunch rows_launch(const mad_ctx* c) {
     L.pe_col = nullptr;
     L.pe_pos = nullptr;
     L.pe_rest = nullptr;
+    L.pmask = nullptr;
   } else {
     const DynBuf& b = c->buf[c->active];
     L.rp = b.rp;
@@ -210,6 +211,7 @@ RowsLaunch rows_launch(const mad_ctx* c) {
     L.pe_col = b.pe_col;
     L.pe_pos = b.pe_pos;
     L.pe_rest = b.pe_rest;
+    L.pmask = b.pmask;
     L.pe_xr = c->pe_xr;
   }
   return L;
@@ -534,6 +536,7 @@ mad_status mad_create(int32_t V, int32_t nF, const int32_t* F, int32_t dof, mad_
       CREATE_CK(dev_alloc(c, &b.ci, sizeof(int32_t) * (size_t)c->capacity));
       CREATE_CK(dev_alloc(c, &b.nnzb, sizeof(int32_t)));
       CREATE_CK(dev_alloc(c, &b.prow, sizeof(int32_t) * (V + 1)));
+      CREATE_CK(dev_alloc(c, &b.pmask, sizeof(uint32_t) * std::max(1, V)));
       CREATE_CK(dev_alloc(c, &b.pe_col, sizeof(int32_t) * pe));
       CREATE_CK(dev_alloc(c, &b.pe_pos, sizeof(int32_t) * pe));
       char* rest_buf = nullptr;

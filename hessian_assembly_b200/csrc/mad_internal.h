@@ -54,6 +54,7 @@ constexpr uint16_t kNoSlot = 0xFFFF;
 // block (first entry of its column and the column is not in the mesh row).
 constexpr int32_t kPairNewBlock = 1 << 30;
 constexpr int32_t kPairPosMask = (1 << 30) - 1;
+constexpr uint32_t kPmaskOverflow = 1u << 31;
 
 // Per-owned-vertex meta: x = mesh-pattern row length | diagonal position << 16,
 // y = first row of the vertex's run | run index << 16.  A run is a maximal
@@ -154,6 +155,9 @@ struct DynBuf {
   int32_t* pe_col = nullptr;  // [2*max_pairs] partner vertex, sorted per row
   int32_t* pe_pos = nullptr;  // [2*max_pairs] position word (see above)
   void* pe_rest = nullptr;    // [2*max_pairs] rest length (dtype)
+  // [V] per row: bit p set when merged position p (< 31) holds an inserted
+  // block; kPmaskOverflow | count when an inserted position is 31 or more
+  uint32_t* pmask = nullptr;
 };
 
 // vertex-face terms (vf.cu): the active pattern, the terms and positions
@@ -299,6 +303,7 @@ struct RowsLaunch {
   const int32_t* pe_col;
   const int32_t* pe_pos;
   const void* pe_rest;
+  const uint32_t* pmask;  // inserted positions per row (DynBuf::pmask)
   // [2*max_pairs][4] per pair entry: the partner's position (DOF values,
   // zero padded) and the rest length in the last value; scratch the compact
   // row kernel fills before each assembly with pairs

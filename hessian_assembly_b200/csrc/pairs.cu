@@ -20,7 +20,8 @@
 //   rows    per row, in registers: sort the entries by (partner, pair id),
 //           merge them with the mesh row, give every entry the position of
 //           its block in the merged row, mark the entries that create a
-//           block; new blocks per row, block and super tile
+//           block; new blocks per row, block and super tile; the row's
+//           inserted positions as a bit mask (DynBuf::pmask)
 //   write   per block: total and prefix of the new-block counts, capacity
 //           check, new row_ptr, merged
 //           col_idx (mesh columns copied with coalesced loads, each to its
@@ -240,10 +241,23 @@ __global__ void __launch_bounds__(kB) k_pair_fill(const int32_t* __restrict__ ij
 
 // Merge of one row with more entries, or a longer mesh row, than the
 // register path holds: in place in global memory.
+// The bit of merged position `pos` in a row's inserted-block mask, or the
+// overflow bit when the position does not fit.
+__device__ __forceinline__ uint32_t pmask_bit(int pos) {
+  return pos < 31 ? (1u << pos) : kPmaskOverflow;
+}
+
+// A row's mask word: the inserted positions, or (when one of them is 31 or
+// more) the overflow bit and the count of inserted blocks.
+__device__ __forceinline__ uint32_t pmask_word(uint32_t bits, int kn) {
+  return (bits & kPmaskOverflow) ? (kPmaskOverflow | (uint32_t)kn) : bits;
+}
+
 template <typename T>
 __device__ int row_merge_global(int32_t b, int32_t e, const int32_t* __restrict__ base_ci,
                                 int32_t r0, int32_t blen, int32_t* pe_col, int32_t* pe_pid,
-                                int32_t* pe_pos, T* pe_rest, const T* __restrict__ rest) {
+                                int32_t* pe_pos, T* pe_rest, const T* __restrict__ rest,
+                                uint32_t& mask) {
   for (int32_t i = b + 1; i < e; ++i) {  // insertion sort by (col, pid)
     const int32_t kc = pe_col[i], kp = pe_pid[i];
     int32_t j = i - 1;
@@ -265,10 +279,12 @@ __device__ int row_merge_global(int32_t b, int32_t e, const int32_t* __restrict_
     const bool in_mesh = kb < blen && base_ci[r0 + kb] == c;
     if (first) prev_new = !in_mesh;
     pe_pos[i] = (kb + kn) | ((first && !in_mesh) ? kPairNewBlock : 0);
+    if (first && !in_mesh) mask |= pmask_bit(kb + kn);
     pe_rest[i] = rest[pe_pid[i]];
     prev_col = c;
   }
   if (prev_new) ++kn;
+  mask = pmask_word(mask, kn);
   return kn;
 }
 
@@ -296,11 +312,13 @@ template <typename T>
 __device__ __forceinline__ int merge_row(int32_t b, int32_t e, int32_t r0, int32_t r1,
                                          const int32_t* __restrict__ base_ci, int32_t* pe_col,
                                          int32_t* pe_pid, int32_t* pe_pos, T* pe_rest,
-                                         const T* __restrict__ rest) {
+                                         const T* __restrict__ rest, uint32_t& mask) {
   const int32_t blen = r1 - r0;
   const int n = e - b;
+  mask = 0u;
   if (n > kRegEntries || blen > kRegMesh)
-    return row_merge_global<T>(b, e, base_ci, r0, blen, pe_col, pe_pid, pe_pos, pe_rest, rest);
+    return row_merge_global<T>(b, e, base_ci, r0, blen, pe_col, pe_pid, pe_pos, pe_rest, rest,
+                               mask);
   int kn = 0;
   int32_t col[kRegEntries], pid[kRegEntries], bc[kRegMesh];
   T rs[kRegEntries];
@@ -352,10 +370,14 @@ __device__ __forceinline__ int merge_row(int32_t b, int32_t e, int32_t r0, int32
       pe_col[b + q] = c;
       pe_pos[b + q] = (kb + kn_group) | (fresh ? kPairNewBlock : 0);
       pe_rest[b + q] = rs[q];
-      if (fresh) ++kn;
+      if (fresh) {
+        mask |= pmask_bit(kb + kn_group);
+        ++kn;
+      }
       prev_col = c;
     }
   }
+  mask = pmask_word(mask, kn);
   return kn;
 }
 
@@ -372,7 +394,8 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V, int nunits,
                                                   int32_t* pe_col, int32_t* pe_pid,
                                                   int32_t* pe_pos, T* pe_rest,
                                                   const T* __restrict__ rest, int32_t* newcnt,
-                                                  int32_t* nblk, int32_t* nsupc) {
+                                                  uint32_t* pmask, int32_t* nblk,
+                                                  int32_t* nsupc) {
   __shared__ int s_unit[kU];
   const int lane = threadIdx.x & 31;
   const int64_t base = (int64_t)blockIdx.x * kU * kB + threadIdx.x;
@@ -394,7 +417,10 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V, int nunits,
     const int64_t v = base + (int64_t)u * kB;
     has[u] = __ballot_sync(0xffffffffu, e[u] > b[u]);
     total += __popc(has[u]);
-    if (v < V && e[u] <= b[u]) newcnt[v] = 0;
+    if (v < V && e[u] <= b[u]) {
+      newcnt[v] = 0;
+      pmask[v] = 0u;
+    }
   }
   __syncthreads();
   for (int round = 0; round * 32 < total; ++round) {
@@ -427,9 +453,11 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V, int nunits,
     if (uu >= 0) {
       const int64_t v = (int64_t)blockIdx.x * kU * kB + (int64_t)uu * kB +
                         (threadIdx.x - lane) + src;
+      uint32_t mask;
       const int kn = merge_row<T>(rb, re, rr0, rr1, base_ci, pe_col, pe_pid, pe_pos, pe_rest,
-                                  rest);
+                                  rest, mask);
       newcnt[v] = kn;
+      pmask[v] = mask;
       if (kn) atomicAdd(&s_unit[uu], kn);
     }
   }
@@ -460,8 +488,9 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
     const int32_t* __restrict__ prev_rp, const int32_t* __restrict__ prev_ci,
     const int32_t* __restrict__ prev_nnzb, const int32_t* __restrict__ prev_prow,
     const int32_t* __restrict__ prev_pe_col, const int32_t* __restrict__ prev_pe_pos,
-    const T* __restrict__ prev_pe_rest, int32_t* out_prow, int32_t* out_pe_col,
-    int32_t* out_pe_pos, T* out_pe_rest) {
+    const T* __restrict__ prev_pe_rest, const uint32_t* __restrict__ prev_pmask,
+    int32_t* out_prow, int32_t* out_pe_col, int32_t* out_pe_pos, T* out_pe_rest,
+    uint32_t* out_pmask) {
   constexpr int kBatch = kMapPerWarp / 32;  // mesh columns per lane held in registers
   __shared__ int32_t s_shift[kB + 1];
   __shared__ int32_t s_dst[kB / 32][kMapPerWarp];
@@ -520,6 +549,7 @@ __global__ void __launch_bounds__(kB, 4) k_write_pattern(
     for (int64_t i = tid; i <= V; i += step) {
       rp[i] = prev_rp[i];
       out_prow[i] = prev_prow ? prev_prow[i] : 0;
+      if (i < V) out_pmask[i] = prev_pmask ? prev_pmask[i] : 0u;
     }
     for (int64_t i = tid; i < nb; i += step) ci[i] = prev_ci[i];
     if (prev_prow) {
@@ -693,20 +723,20 @@ cudaError_t add_pairs_t(const PairLaunch& L, int n, const int32_t* ij, const voi
   CK(cudaGetLastError());
   k_pair_rows<T><<<ngroups, kB, 0, s>>>(V, nblocks, nb.prow, L.base_rp, L.base_ci, nb.pe_col,
                                         L.pe_pid, nb.pe_pos, (T*)nb.pe_rest, (const T*)rest,
-                                        L.newcnt, blk_n, sup_n);
+                                        L.newcnt, nb.pmask, blk_n, sup_n);
   CK(cudaGetLastError());
   if (prev)
     k_write_pattern<T><<<nblocks, kB, 0, s>>>(
         V, L.nnzb_base, L.capacity, L.base_rp, L.base_ci, L.newcnt, nsup, sup_n, blk_n,
         nb.prow, nb.pe_col, nb.pe_pos, nb.rp, nb.ci, nb.nnzb, L.status, prev->rp, prev->ci,
-        prev->nnzb, prev->prow, prev->pe_col, prev->pe_pos, (const T*)prev->pe_rest, nb.prow,
-        nb.pe_col, nb.pe_pos, (T*)nb.pe_rest);
+        prev->nnzb, prev->prow, prev->pe_col, prev->pe_pos, (const T*)prev->pe_rest,
+        prev->pmask, nb.prow, nb.pe_col, nb.pe_pos, (T*)nb.pe_rest, nb.pmask);
   else
     k_write_pattern<T><<<nblocks, kB, 0, s>>>(
         V, L.nnzb_base, L.capacity, L.base_rp, L.base_ci, L.newcnt, nsup, sup_n, blk_n,
         nb.prow, nb.pe_col, nb.pe_pos, nb.rp, nb.ci, nb.nnzb, L.status, L.base_rp, L.base_ci,
-        L.base_nnzb_dev, nullptr, nullptr, nullptr, nullptr, nb.prow, nb.pe_col, nb.pe_pos,
-        (T*)nb.pe_rest);
+        L.base_nnzb_dev, nullptr, nullptr, nullptr, nullptr, nullptr, nb.prow, nb.pe_col,
+        nb.pe_pos, (T*)nb.pe_rest, nb.pmask);
   return cudaGetLastError();
 }
 

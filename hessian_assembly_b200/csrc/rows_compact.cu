@@ -38,8 +38,10 @@ struct CArgs {
   T k;
   const T* xt;
   T w;
-  // runtime pairs (the active pattern's row_ptr and per-row pair entries)
+  // runtime pairs (the active pattern's row_ptr, per-row inserted-block
+  // masks and pair entries)
   const int32_t* rp;
+  const uint32_t* pmask;
   const int32_t* prow;
   const int32_t* pe_col;
   const int32_t* pe_pos;
@@ -83,6 +85,11 @@ __device__ __forceinline__ const T* shard_x(const ShardArgs<T>& S, int v) {
 // once this tile's terms are done).
 #ifndef MAD_ROWSC_PREFETCH_L0
 #define MAD_ROWSC_PREFETCH_L0 0
+#endif
+// With pairs: each row's first block read from the active row_ptr (1), or
+// the tile's first block plus a warp prefix sum of the row lengths (0).
+#ifndef MAD_ROWSC_PAIRS_RP
+#define MAD_ROWSC_PAIRS_RP 1
 #endif
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
@@ -185,7 +192,7 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
         const int64_t e = (int64_t)tp * 32 * DOF + (lane - 16) * (128 / (int)sizeof(T));
         if (e < nx) prefetch_l2(A.xt + e);
       } else if (PAIRS && lane == 28) {
-        prefetch_l2(A.rp + (size_t)tp * 32);
+        prefetch_l2(A.pmask + (size_t)tp * 32);
       } else if (PAIRS && lane == 29) {
         prefetch_l2(A.prow + (size_t)tp * 32);
       }
@@ -209,13 +216,21 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     sw[k] = 0u;
     if (has && k < A.s0) sw[k] = A.cslots[(uint32_t)((tile * A.s0 + k) * 32 + lane)];
   }
-  // the row's place in the active pattern and its pair entries
-  int pd0 = 0, pd1 = 0, pb = 0, pn = 0;
-  if (PAIRS && has) {
-    pd0 = A.rp[i];
-    pd1 = A.rp[i + 1];
-    pb = A.prow[i];
-    pn = A.prow[i + 1] - pb;
+  // the row's inserted blocks and pair entries, the tile's first block in
+  // the active pattern
+  int pb = 0, pn = 0, prp = 0, pd0 = 0, pd1 = 0;
+  uint32_t pm = 0u;
+  if (PAIRS) {
+    if (has) {
+      pm = A.pmask[i];
+      pb = A.prow[i];
+      pn = A.prow[i + 1] - pb;
+      if (MAD_ROWSC_PAIRS_RP) {
+        pd0 = A.rp[i];
+        pd1 = A.rp[i + 1];
+      }
+    }
+    if (!MAD_ROWSC_PAIRS_RP && lane == 0 && tile_live) prp = A.rp[tile * 32];
   }
   T xi[DOF], xti[DOF];
   if (has) {
@@ -262,32 +277,52 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     for (int q = 0; q < no; ++q) dpos += A.ofl[o0 + q].x < i;
   }
   noff += no;
+  // blocks the pairs inserted into the row (their positions are the set bits
+  // of pm, or, past the mask's reach, the flagged pair entries)
+  const bool pofl = PAIRS && (pm & kPmaskOverflow);
+  const int nins = !PAIRS ? 0 : (pofl ? (int)(pm & ~kPmaskOverflow) : __popc(pm));
   int d0, d1;
-  if constexpr (PAIRS) {
+  if (PAIRS && MAD_ROWSC_PAIRS_RP) {
     d0 = pd0;
     d1 = pd1;
   } else {
-    const int len = has ? noff + 1 : 0;
+    const int len = has ? noff + 1 + nins : 0;
     int incl = len;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
-    d0 = th.x + incl - len;
+    d0 = (PAIRS ? __shfl_sync(0xffffffffu, prp, 0) : th.x) + incl - len;
     d1 = d0 + len;
   }
-  // blocks the pairs inserted into the row, and (the first kRowNew of them)
-  // their positions
-  const int nins = PAIRS ? (d1 - d0) - (noff + 1) : 0;
+  // the first kRowNew inserted positions, ascending (0x7FFFFFFF past them)
   RowNew rn;
-  if constexpr (PAIRS) load_row_new(A.pe_pos, pb, pn, nins, rn);
-  // a mesh block's position in the active row
+  if constexpr (PAIRS) {
+    uint32_t m = pofl ? 0u : pm;
+#pragma unroll
+    for (int k = 0; k < kRowNew; ++k) {
+      rn.np[k] = m ? __ffs(m) - 1 : 0x7FFFFFFF;
+      m &= m - 1u;
+    }
+  }
+  // a mesh block's position in the active row: past the inserted blocks at
+  // or before it
   auto at = [&](int p) {
-    if constexpr (PAIRS) return nins == 0 ? p : row_pos_new(rn, A.pe_pos, pb, pn, nins, p);
+    if constexpr (PAIRS) {
+      if (nins > kRowNew) {
+        if (pofl) return row_pos(A.pe_pos, pb, pn, nins, p);
+        for (uint32_t m = pm; m; m &= m - 1u) {
+          if (__ffs(m) - 1 > p) break;
+          ++p;
+        }
+        return p;
+      }
+#pragma unroll
+      for (int k = 0; k < kRowNew; ++k) p += rn.np[k] <= p;
+    }
     return p;
   };
-
   const int dfirst = __shfl_sync(0xffffffffu, d0, 0);
   T* const h0 = A.H + (uint32_t)((dfirst - hoff) * B);  // the warp's first block in H
   const int mis = (int)(((uintptr_t)h0 / sizeof(T)) % VEC);
@@ -297,14 +332,24 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     T* row = staged ? stage + off : h0 + (uint32_t)((d0 - dfirst) * B);
     if (PAIRS && springs && nins > 0) {
       // inserted blocks no edge term stores start at 0
+      if (!pofl) {
 #pragma unroll
-      for (int k = 0; k < kRowNew; ++k)
-        if (k < nins) {
-          T* b = row + rn.np[k] * B;
+        for (int k = 0; k < kRowNew; ++k)
+          if (k < nins) {
+            T* b = row + rn.np[k] * B;
 #pragma unroll
-          for (int q = 0; q < B; ++q) b[q] = T(0);
+            for (int q = 0; q < B; ++q) b[q] = T(0);
+          }
+        if (nins > kRowNew) {
+          uint32_t m = pm;
+          for (int k = 0; k < kRowNew; ++k) m &= m - 1u;
+          for (; m; m &= m - 1u) {
+            T* b = row + (__ffs(m) - 1) * B;
+#pragma unroll
+            for (int q = 0; q < B; ++q) b[q] = T(0);
+          }
         }
-      if (nins > kRowNew) {
+      } else {
         for (int e = pb; e < pb + pn; ++e) {
           const int32_t wv = A.pe_pos[e];
           if (wv & kPairNewBlock) {
@@ -502,6 +547,7 @@ CArgs<T> make_cargs(const RowsLaunch& L, const mad_terms& t, const void* x, void
   A.xt = (const T*)t.inertia_xt;
   A.w = (T)t.inertia_w;
   A.rp = L.rp;
+  A.pmask = L.pmask;
   A.prow = L.prow;
   A.pe_col = L.pe_col;
   A.pe_pos = L.pe_pos;

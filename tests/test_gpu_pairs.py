@@ -212,3 +212,42 @@ def test_pairs_on_a_long_mesh_row(orc):
     assert_close("g", g, og, "float64")
     assert_close("H", H[:nnzb], oH, "float64")
     assert ctx.mad_status_sync() == 0
+
+
+def test_inserted_blocks_before_a_long_mesh_row(orc):
+    """A fan hub (mesh row of 41 blocks) that gains blocks with lower
+    columns: every mesh block of the hub row, those past position 31 too,
+    moves behind the inserted ones."""
+    import hessian_assembly_b200 as mad
+    m = 40
+    ang = 2 * np.pi * np.arange(m) / m
+    tri = np.array([[3.0, 0.0, 0.0], [3.5, 0.0, 0.0], [3.0, 0.5, 0.0]])
+    hub = np.array([[0.0, 0.0, 0.0]])
+    rim = np.stack([np.cos(ang), np.sin(ang), 0 * ang], 1)
+    X = np.concatenate([tri, hub, rim])
+    F = np.array([[0, 1, 2]] + [[3, 4 + i, 4 + (i + 1) % m] for i in range(m)], np.int32)
+    V = 4 + m
+    ctx = mad.Context(V, F, 3, "float64", part_xyz=X)
+    edges = ctx.mad_edges().cpu().numpy()
+    L0 = np.linalg.norm(X[edges[:, 0]] - X[edges[:, 1]], axis=1)
+    rng = np.random.default_rng(14)
+    x = X + 0.01 * rng.standard_normal(X.shape)
+    xt = X.copy()
+    # the hub (3) gains columns 0 and 1 ahead of its mesh row; rim vertex 20
+    # gains column 2; row 2 gains column 20 after its mesh columns
+    pairs = np.array([[3, 1], [0, 3], [2, 20], [1, 3]], np.int32)
+    prest = 0.9 * np.linalg.norm(x[pairs[:, 0]] - x[pairs[:, 1]], axis=1)
+    ctx.mad_add_pairs(to_dev(pairs), to_dev(prest))
+    terms = mad.Terms(mask=11, spring_rest=to_dev(L0), spring_k=10.0, inertia_xt=to_dev(xt),
+                      inertia_w=3.0, pair_k=5.0)
+    g, H, E = run_eval(ctx, x, terms, "float64")
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(V, F, pairs)
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    assert orp[4] - orp[3] == 43  # the hub row: 2 inserted + 41 mesh blocks
+    og, oH, oE = orc.eval(V, 3, x, 11, orp, oci, edges=edges, L0=L0, k=10.0, xt=xt, w=3.0,
+                          pairs=pairs, prest=prest, kp=5.0)
+    assert_close("g", g, og, "float64")
+    assert_close("H", H[:nnzb], oH, "float64")
+    assert ctx.mad_status_sync() == 0
