@@ -254,15 +254,7 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     for (int a = 0; a < DOF; ++a) xb[k][a] = xs[a];
     l0[k] = A.L0[th.y + slot_deid(sw[k])];
   }
-  // the row's first pair entry, asked for before the edge terms are
-  // evaluated
   const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
-  int pw0 = 0;
-  T pr0 = T(0), xp0[DOF];
-  if (pairs && pn > 0) {
-    pw0 = A.pe_pos[pb];
-    load_xr<T, DOF>(A.pe_xr, pb, xp0, pr0);
-  }
   // row length (off-diagonal slots + overflow + the diagonal) and the row's
   // first block: the tile's row_ptr plus the lengths of the rows before it
   int noff = 0, dpos = 0, o0 = 0, no = 0;
@@ -404,18 +396,13 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
       for (int e = 0; e < (d1 - d0) * B; ++e) row[e] = T(0);
     }
     if (pairs) {
+      // the gathered entries (L2 hits: the gather kernel has just written
+      // them) are read after the edge terms, not ahead of them: asked for
+      // early they held registers through the edge terms for little gain
       for (int e = pb; e < pb + pn; ++e) {
-        int pw;
+        const int pw = A.pe_pos[e];
         T xj[DOF], rest;
-        if (e == pb) {
-          pw = pw0;
-          rest = pr0;
-#pragma unroll
-          for (int a = 0; a < DOF; ++a) xj[a] = xp0[a];
-        } else {
-          pw = A.pe_pos[e];
-          load_xr<T, DOF>(A.pe_xr, e, xj, rest);
-        }
+        load_xr<T, DOF>(A.pe_xr, e, xj, rest);
         EdgeRes<T, DOF, AD> Rp;
         eval_edge_res<T, DOF, AD>(xi, xj, rest, A.kp, Rp);
         apply_edge_side<false>(Rp, 0, acc, row + (pw & kPairPosMask) * B, gr);
