@@ -47,6 +47,11 @@ struct CArgs {
   const int32_t* pe_pos;
   const T* pe_xr;  // per entry: partner position (zero padded to 4) + rest length
   T kp;
+  // installed vertex-face terms: per-row entries and the term pass's
+  // per-role shares (see vf.cu)
+  const int32_t* vrow;
+  const int32_t* vent;
+  const T* vrec;
   unsigned mask;
   double* epart;
   int V, s0, wstage;
@@ -158,9 +163,10 @@ __global__ void __launch_bounds__(256) k_pair_gather(const int32_t* __restrict__
 __device__ __forceinline__ int slot_dcol(uint32_t w) { return (int)(int16_t)(w & 0xFFFFu); }
 __device__ __forceinline__ int slot_deid(uint32_t w) { return (int)(int16_t)(w >> 16); }
 
-template <typename T, int DOF, int AD, bool ENERGY, int S0, bool SHARD, bool PAIRS>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, bool SHARD, bool PAIRS, bool VF>
 __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T>* S) {
   static_assert(!(SHARD && PAIRS), "a shard launch carries no pairs");
+  static_assert(!VF || (PAIRS && DOF == 3), "vertex-face terms come with their pair blocks");
   constexpr int B = DOF * DOF;
   constexpr int TD = Tri<DOF>::size;
   constexpr int VEC = 16 / (int)sizeof(T);
@@ -218,8 +224,12 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
   }
   // the row's inserted blocks and pair entries, the tile's first block in
   // the active pattern
-  int pb = 0, pn = 0, prp = 0, pd0 = 0, pd1 = 0;
+  int pb = 0, pn = 0, prp = 0, pd0 = 0, pd1 = 0, vb = 0, ve = 0;
   uint32_t pm = 0u;
+  if (VF && has) {
+    vb = A.vrow[i];
+    ve = A.vrow[i + 1];
+  }
   if (PAIRS) {
     if (has) {
       pm = A.pmask[i];
@@ -255,6 +265,17 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
     l0[k] = A.L0[th.y + slot_deid(sw[k])];
   }
   const bool pairs = PAIRS && (A.mask & MAD_TERM_PAIR);
+  if constexpr (VF) {
+    // the row's first vertex-face share and entry, asked of L1 now, read
+    // after the edge terms
+    if (ve > vb && (A.mask & MAD_TERM_VF)) {
+      const char* p = reinterpret_cast<const char*>(A.vrec + (size_t)vb * kVfRoleVals);
+#pragma unroll
+      for (int l = 0; l < (int)(kVfRoleVals * sizeof(T)); l += 128)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(p + l));
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(A.vent + 8 * (size_t)vb));
+    }
+  }
   // row length (off-diagonal slots + overflow + the diagonal) and the row's
   // first block: the tile's row_ptr plus the lengths of the rows before it
   int noff = 0, dpos = 0, o0 = 0, no = 0;
@@ -409,6 +430,39 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
         if (ENERGY) energy += 0.5 * (double)edge_energy(Rp);
       }
     }
+    if constexpr (VF) {
+      // installed vertex-face terms: this row's share of each of its terms
+      // (its role's slice: the gradient, its four blocks, E); the blocks go
+      // to the staged row, the diagonal block to the register accumulator
+      if (A.mask & MAD_TERM_VF) {
+        for (int q = vb; q < ve; ++q) {
+          const int4 w0 = reinterpret_cast<const int4*>(A.vent)[2 * q];
+          const int4 w1 = reinterpret_cast<const int4*>(A.vent)[2 * q + 1];
+          if (!w1.y) continue;
+          const int role = (int)((uint32_t)w0.x >> 30);
+          // the slice is read a block at a time (few live registers)
+          const T* r = A.vrec + (size_t)q * kVfRoleVals;
+          if (ENERGY) energy += 0.25 * (double)r[kVfRoleVals - 1];
+#pragma unroll
+          for (int a = 0; a < 3; ++a) gr[a] += r[a];
+          const int pos[4] = {w0.y, w0.z, w0.w, w1.x};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            T b9[9];
+#pragma unroll
+            for (int q9 = 0; q9 < 9; ++q9) b9[q9] = r[3 + 9 * j + q9];
+            if (j == role) {
+#pragma unroll
+              for (int a = 0; a < 3; ++a)
+#pragma unroll
+                for (int b2 = a; b2 < 3; ++b2) acc[Tri<3>::idx(a, b2)] += b9[3 * a + b2];
+            } else {
+              add9<T>(row + pos[j] * B, b9);
+            }
+          }
+        }
+      }
+    }
     T* d = row + at(dpos) * B;
 #pragma unroll
     for (int a = 0; a < DOF; ++a)
@@ -449,16 +503,16 @@ __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T
   if (ENERGY) block_energy(energy, A.epart + blockIdx.x);
 }
 
-template <typename T, int DOF, int AD, bool ENERGY, int S0, bool PAIRS>
+template <typename T, int DOF, int AD, bool ENERGY, int S0, bool PAIRS, bool VF>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
     k_rows_eval_c(const CArgs<T> A) {
-  rows_c_body<T, DOF, AD, ENERGY, S0, false, PAIRS>(A, nullptr);
+  rows_c_body<T, DOF, AD, ENERGY, S0, false, PAIRS, VF>(A, nullptr);
 }
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0>
 __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
     k_rows_eval_cs(const CArgs<T> A, const __grid_constant__ ShardArgs<T> S) {
-  rows_c_body<T, DOF, AD, ENERGY, S0, true, false>(A, &S);
+  rows_c_body<T, DOF, AD, ENERGY, S0, true, false, false>(A, &S);
 }
 
 // Shared-memory carve-out asked for the kernel, in percent of the unified
@@ -469,11 +523,13 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, 0>())
 #endif
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0>
-cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, int nb, size_t smem,
-                     cudaStream_t s, bool set) {
+cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, bool vf, int nb,
+                     size_t smem, cudaStream_t s, bool set) {
+  constexpr bool kVf = DOF == 3;  // vertex-face terms have dof 3
   if (set) {
-    const void* ks[3] = {(const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0, false>,
-                         (const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0, true>,
+    const void* ks[4] = {(const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0, false, false>,
+                         (const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0, true, false>,
+                         (const void*)k_rows_eval_c<T, DOF, AD, ENERGY, S0, true, kVf>,
                          (const void*)k_rows_eval_cs<T, DOF, AD, ENERGY, S0>};
     for (const void* k : ks) {
       cudaError_t e;
@@ -489,23 +545,26 @@ cudaError_t launch_c(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, int n
   }
   if (S)
     k_rows_eval_cs<T, DOF, AD, ENERGY, S0><<<nb, kRowThreads, smem, s>>>(A, *S);
+  else if (pairs && vf && kVf)
+    k_rows_eval_c<T, DOF, AD, ENERGY, S0, true, kVf><<<nb, kRowThreads, smem, s>>>(A);
   else if (pairs)
-    k_rows_eval_c<T, DOF, AD, ENERGY, S0, true><<<nb, kRowThreads, smem, s>>>(A);
+    k_rows_eval_c<T, DOF, AD, ENERGY, S0, true, false><<<nb, kRowThreads, smem, s>>>(A);
   else
-    k_rows_eval_c<T, DOF, AD, ENERGY, S0, false><<<nb, kRowThreads, smem, s>>>(A);
+    k_rows_eval_c<T, DOF, AD, ENERGY, S0, false, false><<<nb, kRowThreads, smem, s>>>(A);
   return cudaGetLastError();
 }
 
 template <typename T, int DOF, int S0>
-cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, int ad, bool energy,
-                      int nb, size_t smem, cudaStream_t s, bool set) {
+cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, bool vf, int ad,
+                      bool energy, int nb, size_t smem, cudaStream_t s, bool set) {
   if (set) {
     for (int a : {kAdReduced, kAdFull, kAdGeneric}) {
       const cudaError_t e = with_ad(a, [&](auto adc) {
         constexpr int AD = decltype(adc)::value;
-        const cudaError_t e1 = launch_c<T, DOF, AD, true, S0>(A, S, false, nb, smem, s, true);
+        const cudaError_t e1 =
+            launch_c<T, DOF, AD, true, S0>(A, S, false, false, nb, smem, s, true);
         if (e1 != cudaSuccess) return e1;
-        return launch_c<T, DOF, AD, false, S0>(A, S, false, nb, smem, s, true);
+        return launch_c<T, DOF, AD, false, S0>(A, S, false, false, nb, smem, s, true);
       });
       if (e != cudaSuccess) return e;
     }
@@ -513,8 +572,8 @@ cudaError_t launch_c4(const CArgs<T>& A, const ShardArgs<T>* S, bool pairs, int 
   }
   return with_ad(ad, [&](auto adc) {
     constexpr int AD = decltype(adc)::value;
-    if (energy) return launch_c<T, DOF, AD, true, S0>(A, S, pairs, nb, smem, s, false);
-    return launch_c<T, DOF, AD, false, S0>(A, S, pairs, nb, smem, s, false);
+    if (energy) return launch_c<T, DOF, AD, true, S0>(A, S, pairs, vf, nb, smem, s, false);
+    return launch_c<T, DOF, AD, false, S0>(A, S, pairs, vf, nb, smem, s, false);
   });
 }
 
@@ -540,6 +599,9 @@ CArgs<T> make_cargs(const RowsLaunch& L, const mad_terms& t, const void* x, void
   A.pe_pos = L.pe_pos;
   A.pe_xr = (const T*)L.pe_xr;
   A.kp = (T)t.pair_k;
+  A.vrow = L.vrow;
+  A.vent = L.vent;
+  A.vrec = (const T*)L.vrec;
   A.mask = t.mask;
   A.epart = energy ? L.epart : nullptr;
   A.V = L.V;
@@ -553,10 +615,14 @@ cudaError_t dispatch_c(const RowsLaunch& L, const CArgs<T>& A, const ShardArgs<T
                        double* energy, int nb, cudaStream_t s) {
   const size_t smem = rows_smem_bytes(L);
   const bool pairs = !S && L.prow != nullptr;
+  // installed vertex-face shares gathered into the rows (their blocks are
+  // pair blocks of the active pattern)
+  const bool vf = pairs && DOF == 3 && L.vrow != nullptr && (A.mask & MAD_TERM_VF);
   cudaError_t e =
       L.s0 <= 6
-          ? launch_c4<T, DOF, 6>(A, S, pairs, ad, energy != nullptr, nb, smem, s, false)
-          : launch_c4<T, DOF, kS0Max>(A, S, pairs, ad, energy != nullptr, nb, smem, s, false);
+          ? launch_c4<T, DOF, 6>(A, S, pairs, vf, ad, energy != nullptr, nb, smem, s, false)
+          : launch_c4<T, DOF, kS0Max>(A, S, pairs, vf, ad, energy != nullptr, nb, smem, s,
+                                      false);
   if (e != cudaSuccess || !energy) return e;
   k_energy_sum_rows<<<1, 1024, 0, s>>>(L.epart, nb, energy);
   return cudaGetLastError();
@@ -603,9 +669,10 @@ cudaError_t rows_eval_shard_t(const RowsLaunch& L, const mad_terms& t, int nrank
 template <typename T, int DOF>
 cudaError_t rows_compact_limits_t(size_t bytes) {
   CArgs<T> A{};
-  cudaError_t e = launch_c4<T, DOF, 6>(A, nullptr, false, kAdReduced, false, 0, bytes, 0, true);
+  cudaError_t e =
+      launch_c4<T, DOF, 6>(A, nullptr, false, false, kAdReduced, false, 0, bytes, 0, true);
   if (e != cudaSuccess) return e;
-  return launch_c4<T, DOF, kS0Max>(A, nullptr, false, kAdReduced, false, 0, bytes, 0, true);
+  return launch_c4<T, DOF, kS0Max>(A, nullptr, false, false, kAdReduced, false, 0, bytes, 0, true);
 }
 
 template cudaError_t rows_eval_compact_t<float, 2>(const RowsLaunch&, const mad_terms&, const void*,

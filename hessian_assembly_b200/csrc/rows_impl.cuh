@@ -955,8 +955,10 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
   const bool pairs = L.prow != nullptr;
   const bool en = energy != nullptr;
   cudaError_t e;
-  if (DOF == 3 && L.vrow && pairs && (t.mask & MAD_TERM_VF) && !(t.mask & MAD_TERM_AREA)) {
-    // installed vertex-face terms gathered into the rows (FACES == 4)
+  if (DOF == 3 && L.vrow && pairs && (t.mask & MAD_TERM_VF) && !(t.mask & MAD_TERM_AREA) &&
+      L.cslots == nullptr) {
+    // installed vertex-face terms gathered into the rows (FACES == 4); with
+    // compact slot tables the compact kernel does the same (below)
     if (t.mask & MAD_TERM_SPRING)
       e = eval_k4<T, DOF, kS0Max, 4>(A, ad, en, pairs, nb, smem, s);
     else
