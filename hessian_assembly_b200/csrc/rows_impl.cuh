@@ -624,8 +624,18 @@ __device__ __forceinline__ void add_corner_hv(const T* __restrict__ fhv, uint32_
     yr[0] += c.x;
     yr[1] += c.y;
   } else {
+    // dof 3 (area faces): the pass stores corners 1 and 2 only; corner 0's
+    // result is minus their sum (the term is translation invariant, and the
+    // pass computes corner 0 that way)
+    const uint32_t f = q / 3u, c = q - 3u * f;
+    const T* h = fhv + 6 * (size_t)f;
+    if (c == 0) {
 #pragma unroll
-    for (int a = 0; a < DOF; ++a) yr[a] += fhv[DOF * q + a];
+      for (int a = 0; a < 3; ++a) yr[a] -= h[a] + h[3 + a];
+    } else {
+#pragma unroll
+      for (int a = 0; a < 3; ++a) yr[a] += h[3 * (c - 1) + a];
+    }
   }
 }
 
@@ -739,29 +749,47 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES ? 1 : 0>
 }
 
 // Per-face pass of the Hessian-vector product for area-preservation faces
-// (dof 3): one thread per face writes (H_f v_f) for its three corners.
+// (dof 3): each thread takes kAreaHvFaces faces (their loads issued
+// together) and writes (H_f v_f) of corners 1 and 2 of each.
+#ifndef MAD_AREA_HV_FACES
+#define MAD_AREA_HV_FACES 1
+#endif
+constexpr int kAreaHvFaces = MAD_AREA_HV_FACES;
+
 template <typename T, int AD>
 __global__ void __launch_bounds__(256) k_face_hv_area(int nF, const int32_t* __restrict__ F,
                                                       const T* __restrict__ x,
                                                       const T* __restrict__ v,
                                                       const T* __restrict__ area, T ka,
                                                       T* __restrict__ out) {
-  const int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (f >= nF) return;
-  T u[3][3], w[3][3];
+  T u[kAreaHvFaces][3][3], w[kAreaHvFaces][3][3], ar[kAreaHvFaces];
+  int64_t fs[kAreaHvFaces];
 #pragma unroll
-  for (int c = 0; c < 3; ++c) {
-    const int32_t vid = F[3 * f + c];
+  for (int h = 0; h < kAreaHvFaces; ++h) {
+    const int64_t f = ((int64_t)blockIdx.x * kAreaHvFaces + h) * 256 + threadIdx.x;
+    fs[h] = f;
+    if (f >= nF) continue;
 #pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      u[c][a] = x[(int64_t)vid * 3 + a];
-      w[c][a] = v[(int64_t)vid * 3 + a];
+    for (int c = 0; c < 3; ++c) {
+      const int32_t vid = F[3 * f + c];
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        u[h][c][a] = x[(int64_t)vid * 3 + a];
+        w[h][c][a] = v[(int64_t)vid * 3 + a];
+      }
     }
+    ar[h] = area[f];
   }
-  T o[9];
-  hv_area_face<T, AD>(u[0], u[1], u[2], w[0], w[1], w[2], area[f], ka, o);
 #pragma unroll
-  for (int q = 0; q < 9; ++q) out[9 * f + q] = o[q];
+  for (int h = 0; h < kAreaHvFaces; ++h) {
+    const int64_t f = fs[h];
+    if (f >= nF) continue;
+    T o[9];
+    hv_area_face<T, AD>(u[h][0], u[h][1], u[h][2], w[h][0], w[h][1], w[h][2], ar[h], ka, o);
+    // corners 1 and 2; the row pass takes corner 0 as minus their sum
+#pragma unroll
+    for (int q = 3; q < 9; ++q) out[6 * f + q - 3] = o[q];
+  }
 }
 
 constexpr int kFacesPerThread = 2;
@@ -1026,7 +1054,7 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
     if constexpr (DOF == 3) {
       if (t.mask & MAD_TERM_AREA) {
         if (L.nF > 0) {
-          const unsigned nbf = (unsigned)((L.nF + 255) / 256);
+          const unsigned nbf = (unsigned)((L.nF + 256 * kAreaHvFaces - 1) / (256 * kAreaHvFaces));
           k_face_hv_area<T, AD><<<nbf, 256, 0, s>>>(L.nF, L.F, (const T*)x, (const T*)v,
                                                     (const T*)t.face_area, (T)t.area_k,
                                                     (T*)L.fhv);

@@ -748,12 +748,15 @@ __device__ __forceinline__ void hv_area_face(const T* u0, const T* u1, const T* 
                                  A0, k);
     const T* vv[3] = {v0, v1, v2};
 #pragma unroll
-    for (int p = 0; p < 9; ++p) {
+    for (int p = 3; p < 9; ++p) {
       T s = shess(e, p, 0) * vv[0][0];
 #pragma unroll
       for (int q = 1; q < 9; ++q) s += shess(e, p, q) * vv[q / 3][q % 3];
       out[p] = s;
     }
+    // the term is translation invariant: corner 0 is minus corners 1 and 2
+#pragma unroll
+    for (int al = 0; al < 3; ++al) out[al] = -(out[3 + al] + out[6 + al]);
   }
 }
 
