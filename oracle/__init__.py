@@ -18,6 +18,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+import shutil
 import tempfile
 
 import numpy as np
@@ -311,6 +312,10 @@ def load() -> Oracle:
 
 
 def load_mutant(mutant: int) -> Oracle:
-    """A build of oracle.c with planted mistake number ``mutant`` (tests only)."""
+    """A build of oracle.c with planted mistake number ``mutant`` (tests only).
+    The library stays mapped once loaded, so its build folder is removed."""
     d = tempfile.mkdtemp(prefix="oracle_mutant_")
-    return Oracle(build(os.path.join(d, f"liboracle_m{mutant}.so"), mutant))
+    try:
+        return Oracle(build(os.path.join(d, f"liboracle_m{mutant}.so"), mutant))
+    finally:
+        shutil.rmtree(d, ignore_errors=True)
