@@ -251,3 +251,48 @@ def test_inserted_blocks_before_a_long_mesh_row(orc):
     assert_close("g", g, og, "float64")
     assert_close("H", H[:nnzb], oH, "float64")
     assert ctx.mad_status_sync() == 0
+
+
+@pytest.mark.parametrize("n,dtype,slot_bytes", [(40, "float64", 4), (190, "float32", 8)])
+def test_pairs_on_permuted_numbering(orc, n, dtype, slot_bytes):
+    """Pairs on a randomly renumbered cloth: at 40^2 the compact row tables
+    (irregular deltas), at 190^2 the wide ones (deltas past 16 bits), so both
+    row kernels' pair paths run; eval and the product against the oracle."""
+    import hessian_assembly_b200 as mad
+    import torch
+    st = mi.cloth_static(n, np.float64)
+    V = st["V"]
+    perm = np.random.default_rng(5).permutation(V)   # new id of old vertex
+    inv = np.argsort(perm)
+    F = perm[st["F"]].astype(np.int32)
+    X = st["X"][inv]
+    ctx = mad.Context(V, F, 3, dtype, part_xyz=X)
+    assert ctx.info.row_slot_bytes == slot_bytes
+    e = np.sort(perm[mi.grid_edges(n)], axis=1)
+    edges = e[np.lexsort((e[:, 1], e[:, 0]))].astype(np.int32)
+    L0 = np.linalg.norm(X[edges[:, 0]] - X[edges[:, 1]], axis=1).astype(dtype)
+    x = mi.cloth_x(n, 15, 0, np.float64)[inv].astype(dtype)
+    xt = X.astype(dtype)
+    pairs = perm[mi.random_pairs(n, 4 * n, 15, 0)].astype(np.int32)
+    prest = mi.pair_rest(x, pairs, np.dtype(dtype))
+    add_pairs(ctx, pairs, prest, dtype)
+    assert ctx.mad_status_sync() == 0
+    terms = mad.Terms(mask=11, spring_rest=to_dev(L0), spring_k=st["k"], inertia_xt=to_dev(xt),
+                      inertia_w=st["w"], pair_k=mi.PAIR_K)
+    g, H, E = run_eval(ctx, x, terms, dtype)
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(V, F, pairs)
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    og, oH, oE = orc.eval(V, 3, x, 11, orp, oci, edges=edges, L0=L0, k=st["k"], xt=xt, w=st["w"],
+                          pairs=pairs, prest=prest, kp=mi.PAIR_K)
+    assert_close("g", g, og, dtype)
+    assert_close("H", H[:nnzb], oH, dtype)
+    # the product: y = H v with the oracle's assembled H
+    v = np.random.default_rng(16).standard_normal((V, 3)).astype(dtype)
+    tdt = getattr(torch, dtype)
+    y = torch.zeros((V, 3), dtype=tdt, device="cuda")
+    ctx.mad_hvp(to_dev(x, dtype), terms, to_dev(v, dtype), y)
+    torch.cuda.synchronize()
+    oy = orc.bsr_mv(V, 3, orp, oci, oH, v.astype(np.float64))
+    assert_close("y", y.cpu().numpy(), oy, dtype)

@@ -207,3 +207,53 @@ def test_vf_installed_bad_terms_and_replacement(orc):
     with pytest.raises(mad.MadError) as ei:
         ctx.mad_add_vf(to_dev(np.zeros((len(vf) + 10, 2), np.int32)))
     assert ei.value.status == mad.MAD_ERR_CAPACITY
+
+
+def test_vf_installed_on_permuted_numbering(orc):
+    """Installed vertex-face terms on a randomly renumbered 190^2 cloth, whose
+    column deltas pass 16 bits: the wide-table row kernel gathers the shares
+    (the compact one does on grid numberings); eval and product vs the oracle."""
+    import hessian_assembly_b200 as mad
+    import torch
+    n, dtype = 190, "float32"
+    st = mi.cloth_static(n, np.float64)
+    V = st["V"]
+    perm = np.random.default_rng(7).permutation(V)   # new id of old vertex
+    inv = np.argsort(perm)
+    F = perm[st["F"]].astype(np.int32)
+    X = st["X"][inv]
+    vf0 = mi.random_vf(n, 1500, 6107, 0)
+    vf = np.stack([perm[vf0[:, 0]], vf0[:, 1]], axis=1).astype(np.int32)  # faces keep their ids
+    rest = 0.001 * np.random.default_rng(6108).standard_normal(len(vf))
+    ctx = mad.Context(V, F, 3, dtype, part_xyz=X, max_pairs=3 * len(vf) + 8, slack=0.6)
+    assert ctx.info.row_slot_bytes == 8
+    ctx.mad_add_vf(to_dev(vf))
+    assert ctx.mad_status_sync() == mad.MAD_OK
+    e = np.sort(perm[mi.grid_edges(n)], axis=1)
+    edges = e[np.lexsort((e[:, 1], e[:, 0]))].astype(np.int32)
+    L0 = np.linalg.norm(X[edges[:, 0]] - X[edges[:, 1]], axis=1)
+    x = mi.cloth_x(n, 6107, 0, np.float64)[inv]
+    x = (x + 0.02 * mi.grid_spacing(n) * np.random.default_rng(6109).standard_normal(x.shape)
+         ).astype(dtype)
+    xt = X
+    mask = 1 | 2 | VF
+    terms = mad.Terms(mask=mask, spring_rest=to_dev(L0, dtype), spring_k=st["k"],
+                      inertia_xt=to_dev(xt, dtype), inertia_w=st["w"], vf=None,
+                      vf_rest=to_dev(rest, dtype), vf_k=KC)
+    g, H, E = run_eval(ctx, x, terms, dtype)
+    assert ctx.mad_status_sync() == mad.MAD_OK
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(V, F, mi.vf_pairs(vf, F))
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    og, oH, oE = orc.eval(V, 3, x, mask, orp, oci, edges=edges, L0=L0.astype(dtype), k=st["k"],
+                          xt=xt.astype(dtype), w=st["w"], F=F, vf=vf,
+                          vf_rest=rest.astype(dtype), kc=KC)
+    assert_close("g", g, og, dtype)
+    assert_close("H", H[:nnzb], oH, dtype)
+    assert abs(E - oE) <= ETOL[dtype] * abs(oE)
+    v = mi.probe_vector(V, 3, 6110, np.dtype(dtype))
+    y = torch.full((V, 3), float("nan"), dtype=torch.float32, device="cuda")
+    ctx.mad_hvp(to_dev(x, dtype), terms, to_dev(v, dtype), y)
+    torch.cuda.synchronize()
+    assert_close("y", y.cpu().numpy(), orc.bsr_mv(V, 3, orp, oci, oH, v), dtype)
