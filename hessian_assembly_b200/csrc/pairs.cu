@@ -40,6 +40,13 @@ constexpr int kRegEntries = 4; // pair entries of a row merged in registers
 constexpr int kRegMesh = 8;    // mesh columns of a row held in registers
 constexpr int kRegNew = 4;     // new columns of a row the write kernel keeps in registers
 constexpr int kMapPerWarp = 256;  // mesh columns of 32 rows the write kernel maps in smem
+// resident blocks per SM the merge and write kernels are compiled for
+#ifndef MAD_PAIR_ROWS_MINB
+#define MAD_PAIR_ROWS_MINB 4
+#endif
+#ifndef MAD_WRITE_MINB
+#define MAD_WRITE_MINB 4
+#endif
 
 inline unsigned grid_for(int64_t n) {
   int64_t b = (n + kB - 1) / kB;
@@ -387,7 +394,7 @@ __device__ __forceinline__ int merge_row(int32_t b, int32_t e, int32_t r0, int32
 // so each warp deals its rows that have them out to its lanes, one per lane,
 // and runs the merge once per 32 such rows.
 template <typename T>
-__global__ void __launch_bounds__(kB) k_pair_rows(int V, int nunits,
+__global__ void __launch_bounds__(kB, MAD_PAIR_ROWS_MINB) k_pair_rows(int V, int nunits,
                                                   const int32_t* __restrict__ prow,
                                                   const int32_t* __restrict__ base_rp,
                                                   const int32_t* __restrict__ base_ci,
@@ -477,7 +484,7 @@ __global__ void __launch_bounds__(kB) k_pair_rows(int V, int nunits,
 // Every load that does not depend on the new-block prefix is issued first,
 // so that a block waits for memory about twice.
 template <typename T>
-__global__ void __launch_bounds__(kB, 4) k_write_pattern(
+__global__ void __launch_bounds__(kB, MAD_WRITE_MINB) k_write_pattern(
     int V, int nnzb_base, int capacity, const int32_t* __restrict__ base_rp,
     const int32_t* __restrict__ base_ci, const int32_t* __restrict__ newcnt,
     int nsup, const int32_t* __restrict__ nsupc, const int32_t* __restrict__ nblk,
