@@ -160,8 +160,6 @@ __global__ void __launch_bounds__(256) k_pair_gather(const int32_t* __restrict__
   }
 }
 
-__device__ __forceinline__ int slot_dcol(uint32_t w) { return (int)(int16_t)(w & 0xFFFFu); }
-__device__ __forceinline__ int slot_deid(uint32_t w) { return (int)(int16_t)(w >> 16); }
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0, bool SHARD, bool PAIRS, bool VF>
 __device__ __forceinline__ void rows_c_body(const CArgs<T>& A, const ShardArgs<T>* S) {

@@ -65,6 +65,10 @@ struct RArgs {
   const uint32_t* meta;
   const int32_t* ofl_ptr;
   const int2* ofl;
+  // compact slot tables (rows_compact.cu; nullptr when absent): the product
+  // reads its edge terms from them
+  const int4* ctile;
+  const uint32_t* cslots;
   const int32_t* rp;
   const int32_t* prow;
   const int32_t* pe_col;
@@ -162,6 +166,58 @@ __device__ __forceinline__ void block_energy(double e, double* out) {
     double s = 0.0;
     for (int i = 0; i < kWarps; ++i) s += red[i];
     *out = s;
+  }
+}
+
+// 1: the product reads its edge terms from the compact slot tables when the
+// context has them (0: always the wide ones)
+#ifndef MAD_HVP_COMPACT
+#define MAD_HVP_COMPACT 1
+#endif
+
+// Compact slot word: column minus row (low 16 bits), edge id minus the
+// tile's first edge id (high 16 bits), both signed; 0 marks an empty slot.
+__device__ __forceinline__ int slot_dcol(uint32_t w) { return (int)(int16_t)(w & 0xFFFFu); }
+__device__ __forceinline__ int slot_deid(uint32_t w) { return (int)(int16_t)(w >> 16); }
+
+// Calls on_term(R, col) for every edge term (i, col) of row i, read from the
+// compact slot tables (positions are not needed: the product).
+template <typename T, int DOF, int AD, int S0, typename OnTerm>
+__device__ __forceinline__ void row_edges_c(const RArgs<T>& A, int i, int tile, int lane,
+                                            const T* xi, OnTerm on_term) {
+  const int4 th = A.ctile[tile];
+  uint32_t sw[S0];
+#pragma unroll
+  for (int k = 0; k < S0; ++k)
+    sw[k] = k < A.s0 ? A.cslots[(uint32_t)((tile * A.s0 + k) * 32 + lane)] : 0u;
+  T xb[S0][DOF];
+  T l0[S0];
+#pragma unroll
+  for (int k = 0; k < S0; ++k) {
+    if (sw[k] == 0u) continue;
+    const int col = i + slot_dcol(sw[k]);
+#pragma unroll
+    for (int a = 0; a < DOF; ++a) xb[k][a] = A.x[(uint32_t)(col * DOF + a)];
+    l0[k] = A.L0[th.y + slot_deid(sw[k])];
+  }
+#pragma unroll
+  for (int k = 0; k < S0; ++k) {
+    if (sw[k] == 0u) continue;
+    EdgeRes<T, DOF, AD> R;
+    eval_edge_res<T, DOF, AD>(xi, xb[k], l0[k], A.k, R);
+    on_term(R, i + slot_dcol(sw[k]));
+  }
+  if (((uint32_t)th.z >> lane) & 1u) {  // rows longer than the slot table
+    const int o0 = A.ofl_ptr[i], o1 = A.ofl_ptr[i + 1];
+    for (int q = o0; q < o1; ++q) {
+      const int2 e = A.ofl[q];
+      T xo[DOF];
+#pragma unroll
+      for (int a = 0; a < DOF; ++a) xo[a] = A.x[(uint32_t)(e.x * DOF + a)];
+      EdgeRes<T, DOF, AD> R;
+      eval_edge_res<T, DOF, AD>(xi, xo, A.L0[e.y], A.k, R);
+      on_term(R, e.x);
+    }
   }
 }
 
@@ -664,7 +720,7 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES ? 1 : 0>
       xi[a] = A.x[(uint32_t)(i * DOF + a)];
       vi[a] = A.v[(uint32_t)(i * DOF + a)];
     }
-    m = A.meta[i];
+    if (!(MAD_HVP_COMPACT && A.cslots)) m = A.meta[i];
   }
   // face terms: the row's incidence entries (3f + c) of the per-face pass
   constexpr int SF = kFaceRowSlots;
@@ -704,13 +760,17 @@ __global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES ? 1 : 0>
   };
   if constexpr (S0 > 0) {
     if (A.mask & MAD_TERM_SPRING) {
-      row_edges<T, DOF, AD, S0>(A, i, tile, lane, m, xi,
-                              [&](const EdgeRes<T, DOF, AD>& R, int, int col) {
-                                T vj[DOF];
+      auto edge = [&](const EdgeRes<T, DOF, AD>& R, int col) {
+        T vj[DOF];
 #pragma unroll
-                                for (int a = 0; a < DOF; ++a) vj[a] = A.v[(uint32_t)(col * DOF + a)];
-                                hv(R, vj);
-                              });
+        for (int a = 0; a < DOF; ++a) vj[a] = A.v[(uint32_t)(col * DOF + a)];
+        hv(R, vj);
+      };
+      if (MAD_HVP_COMPACT && A.cslots)
+        row_edges_c<T, DOF, AD, S0>(A, i, tile, lane, xi, edge);
+      else
+        row_edges<T, DOF, AD, S0>(A, i, tile, lane, m, xi,
+                                  [&](const EdgeRes<T, DOF, AD>& R, int, int col) { edge(R, col); });
     }
   }
   if (pairs) {
@@ -875,6 +935,8 @@ RArgs<T> make_rargs(const RowsLaunch& L, const mad_terms& t, const void* x, cons
   A.area = (const T*)t.face_area;
   A.sf = L.sf;
   A.slots = L.slots;
+  A.ctile = L.ctile;
+  A.cslots = L.cslots;
   A.meta = L.meta;
   A.ofl_ptr = L.ofl_ptr;
   A.ofl = L.ofl;
