@@ -235,11 +235,14 @@ __global__ void __launch_bounds__(kB) k_pair_fill(const int32_t* __restrict__ ij
     const int32_t i = ij[2 * p], j = ij[2 * p + 1];
     if (!pair_ok(i, j, V)) continue;
     const T r = rest[p];
-    int32_t s = prow[i] + atomicSub(&cnt[i], 1) - 1;
+    // both slots are claimed before either entry is written, so that the two
+    // atomics' round trips overlap
+    const int32_t ci = atomicSub(&cnt[i], 1), cj = atomicSub(&cnt[j], 1);
+    int32_t s = prow[i] + ci - 1;
     pe_col[s] = j;
     pe_pid[s] = (int32_t)p;
     pe_rest[s] = r;
-    s = prow[j] + atomicSub(&cnt[j], 1) - 1;
+    s = prow[j] + cj - 1;
     pe_col[s] = i;
     pe_pid[s] = (int32_t)p;
     pe_rest[s] = r;
