@@ -32,6 +32,11 @@ namespace mad {
 namespace {
 
 constexpr int kJT = 256;
+// spring rows per thread of the residual/Jacobian kernel
+#ifndef MAD_JAC_EDGES_PER_THREAD
+#define MAD_JAC_EDGES_PER_THREAD 2
+#endif
+constexpr int kJE = MAD_JAC_EDGES_PER_THREAD;
 
 inline unsigned jgrid(int64_t n) {
   int64_t b = (n + kJT - 1) / kJT;
@@ -120,9 +125,9 @@ __device__ __forceinline__ void jbulk_store(void* gdst, const void* ssrc, uint32
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
-// Springs and inertia in one launch: blocks [0, nbs) take kJT edges each,
-// the rest kJT inertia rows each.  A block's spring rows (kJT * 2*DOF values,
-// contiguous in J) are staged in shared memory and leave with one 1-D bulk
+// Springs and inertia in one launch: blocks [0, nbs) take kJT * kJE edges
+// each, the rest kJT inertia rows each.  A block's spring rows (2*DOF values
+// per edge, contiguous in J) are staged in shared memory and leave with one 1-D bulk
 // copy when its first value and its size are 16-byte aligned; otherwise
 // every thread stores its own row.
 template <typename T, int DOF>
@@ -130,27 +135,49 @@ __global__ void __launch_bounds__(kJT) k_jac_edges_vertices(
     Segs S, int nE, int nbs, int64_t nin, const int32_t* __restrict__ edges,
     const T* __restrict__ x, const T* __restrict__ L0, T sk, const T* __restrict__ xt, T sw,
     T* __restrict__ r, T* __restrict__ J) {
-  __shared__ __align__(16) T stage[kJT * 2 * DOF];
+  __shared__ __align__(16) T stage[kJT * kJE * 2 * DOF];
   if ((int)blockIdx.x < nbs) {
-    const int64_t e0 = (int64_t)blockIdx.x * kJT;
-    const int64_t e = e0 + threadIdx.x;
-    const int cnt = (int)((nE - e0) < kJT ? (nE - e0) : kJT);
-    if (e < nE) {
-      const int2 ab = reinterpret_cast<const int2*>(edges)[e];
+    // kJE edges per thread (edges e0 + h*kJT + thread), every load of them
+    // issued before the first is used
+    const int64_t e0 = (int64_t)blockIdx.x * kJT * kJE;
+    const int cnt = (int)((nE - e0) < kJT * kJE ? (nE - e0) : kJT * kJE);
+    int2 ab[kJE];
+    T l0[kJE], xa[kJE][DOF], xb[kJE][DOF];
+#pragma unroll
+    for (int h = 0; h < kJE; ++h) {
+      const int64_t e = e0 + h * kJT + threadIdx.x;
+      if (e < nE) {
+        ab[h] = reinterpret_cast<const int2*>(edges)[e];
+        l0[h] = L0[e];
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kJE; ++h) {
+      if (e0 + h * kJT + threadIdx.x >= nE) continue;
+#pragma unroll
+      for (int c = 0; c < DOF; ++c) {
+        xa[h][c] = x[(int64_t)ab[h].x * DOF + c];
+        xb[h][c] = x[(int64_t)ab[h].y * DOF + c];
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kJE; ++h) {
+      const int64_t e = e0 + h * kJT + threadIdx.x;
+      if (e >= nE) continue;
       Dual<T, DOF> s = d_const<T, DOF>(T(0));
 #pragma unroll
       for (int c = 0; c < DOF; ++c) {
-        const Dual<T, DOF> d =
-            d_var<T, DOF>(x[(int64_t)ab.x * DOF + c] - x[(int64_t)ab.y * DOF + c], c);
+        const Dual<T, DOF> d = d_var<T, DOF>(xa[h][c] - xb[h][c], c);
         s = s + d * d;
       }
-      const Dual<T, DOF> res = (sqrt(s) - L0[e]) * sk;
+      const Dual<T, DOF> res = (sqrt(s) - l0[h]) * sk;
       r[S.r_sp + e] = res.v;
       // dr/dx_a = dr/dd, dr/dx_b = -dr/dd
+      T* st = stage + (h * kJT + threadIdx.x) * 2 * DOF;
 #pragma unroll
       for (int c = 0; c < DOF; ++c) {
-        stage[threadIdx.x * 2 * DOF + c] = res.g[c];
-        stage[threadIdx.x * 2 * DOF + DOF + c] = -res.g[c];
+        st[c] = res.g[c];
+        st[DOF + c] = -res.g[c];
       }
     }
     __syncthreads();
@@ -247,7 +274,7 @@ static cudaError_t jac_values(int V, int dof, unsigned mask, int nE, const int32
   const int64_t ne = (mask & MAD_TERM_SPRING) ? nE : 0;
   const int64_t nin = (mask & MAD_TERM_INERTIA) ? (int64_t)V * dof : 0;
   if (ne + nin > 0) {
-    const int nbs = (int)((ne + kJT - 1) / kJT);
+    const int nbs = (int)((ne + kJT * kJE - 1) / (kJT * kJE));
     const int nbi = (int)((nin + kJT - 1) / kJT);
     const T sk = (T)std::sqrt(t.spring_k), sw = (T)std::sqrt(t.inertia_w);
     if (dof == 3)
