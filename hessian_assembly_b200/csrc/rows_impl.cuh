@@ -695,8 +695,18 @@ __device__ __forceinline__ void add_corner_hv(const T* __restrict__ fhv, uint32_
   }
 }
 
+// Resident blocks per SM the product's row pass with face terms is compiled
+// for (fp32); the pass is latency-bound, so occupancy pays.
+#ifndef MAD_HVP_FACES_MIN_BLOCKS
+#define MAD_HVP_FACES_MIN_BLOCKS 4
+#endif
+template <typename T, bool FACES>
+constexpr int hvp_min_blocks() {
+  return FACES ? (sizeof(T) == 4 ? MAD_HVP_FACES_MIN_BLOCKS : 2) : rows_min_blocks<T, 0>();
+}
+
 template <typename T, int DOF, int AD, int S0, bool FACES>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES ? 1 : 0>()) k_rows_hvp(const RArgs<T> A) {
+__global__ void __launch_bounds__(kRowThreads, hvp_min_blocks<T, FACES>()) k_rows_hvp(const RArgs<T> A) {
   constexpr int TD = Tri<DOF>::size;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int tile = blockIdx.x * kWarps + wib;
@@ -1095,7 +1105,10 @@ cudaError_t run_rows_hvp(const RowsLaunch& L, const mad_terms& t, const void* x,
     // the row pass after the per-face pass, or alone
     auto rows = [&](auto facesc) {
       constexpr bool FC = decltype(facesc)::value;
-      if (sp) k_rows_hvp<T, DOF, AD, kS0Max, FC><<<nb, kRowThreads, 0, s>>>(A);
+      // slot tables of width <= 6 (triangle meshes of valence <= 6) take the
+      // narrower instantiation: fewer registers
+      if (sp && L.s0 <= 6) k_rows_hvp<T, DOF, AD, 6, FC><<<nb, kRowThreads, 0, s>>>(A);
+      else if (sp) k_rows_hvp<T, DOF, AD, kS0Max, FC><<<nb, kRowThreads, 0, s>>>(A);
       else k_rows_hvp<T, DOF, AD, 0, FC><<<nb, kRowThreads, 0, s>>>(A);
       return cudaGetLastError();
     };
