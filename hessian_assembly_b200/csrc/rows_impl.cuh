@@ -40,10 +40,16 @@ constexpr int kS0Max = 8;         // most slots per row in the slot table
 // 4 installed vertex-face terms, whose branch runs on few rows and is held
 // to the budget of the plain kernel (it may spill rather than lower the
 // occupancy of every row)
-template <typename T, int FACES>
+// The area face rows (dof 3) are held to 6 blocks per SM (80 registers, no
+// spill): 131.5 us against 139.9 us at 4 per 1000x1000 eval.
+#ifndef MAD_ROWS_FACES3_MIN_BLOCKS
+#define MAD_ROWS_FACES3_MIN_BLOCKS 6
+#endif
+template <typename T, int FACES, int DOF = 2>
 constexpr int rows_min_blocks() {
-  return (FACES == 1 || FACES == 2) ? (sizeof(T) == 4 ? 4 : 2)
-                                    : (sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3);
+  return (FACES == 1 || FACES == 2)
+             ? (sizeof(T) == 4 ? (DOF == 3 ? MAD_ROWS_FACES3_MIN_BLOCKS : 4) : 2)
+             : (sizeof(T) == 4 ? MAD_ROWS_MIN_BLOCKS : 3);
 }
 
 template <typename T>
@@ -599,7 +605,7 @@ __device__ __forceinline__ void rows_eval_row(const RArgs<T>& A, int i, int tile
 }
 
 template <typename T, int DOF, int AD, bool ENERGY, int S0, int FACES, bool PAIRS>
-__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES>()) k_rows_eval(const RArgs<T> A) {
+__global__ void __launch_bounds__(kRowThreads, rows_min_blocks<T, FACES, DOF>()) k_rows_eval(const RArgs<T> A) {
   constexpr int B = DOF * DOF;
   constexpr int VEC = 16 / (int)sizeof(T);
   extern __shared__ __align__(16) char smem_raw[];
@@ -1074,7 +1080,9 @@ cudaError_t run_rows_eval(const RowsLaunch& L, const mad_terms& t, const void* x
       }
       return eval_k4<T, DOF, S0F, 1>(A, ad, en, pairs, nb, smem, s);
     };
-    if (t.mask & MAD_TERM_SPRING)
+    if ((t.mask & MAD_TERM_SPRING) && L.s0 <= 6)
+      e = faces_k(std::integral_constant<int, 6>{});  // valence <= 6: fewer registers
+    else if (t.mask & MAD_TERM_SPRING)
       e = faces_k(std::integral_constant<int, kS0Max>{});
     else
       e = faces_k(std::integral_constant<int, 0>{});
@@ -1153,6 +1161,8 @@ cudaError_t set_rows_limits(size_t bytes) {
     return e;
   if ((e = eval_k4<T, DOF, kS0Max, 0>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
     return e;
+  if ((e = eval_k4<T, DOF, 6, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+    return e;
   if ((e = eval_k4<T, DOF, kS0Max, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
     return e;
   if ((e = eval_k4<T, DOF, 0, 1>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
@@ -1165,6 +1175,8 @@ cudaError_t set_rows_limits(size_t bytes) {
       return e;
   }
   if constexpr (DOF == 2) {
+    if ((e = eval_k4<T, DOF, 6, 2>(A, false, false, false, 0, bytes, 0, true)) != cudaSuccess)
+      return e;
     if ((e = eval_k4<T, DOF, kS0Max, 2>(A, false, false, false, 0, bytes, 0, true)) !=
         cudaSuccess)
       return e;
