@@ -296,3 +296,50 @@ def test_pairs_on_permuted_numbering(orc, n, dtype, slot_bytes):
     torch.cuda.synchronize()
     oy = orc.bsr_mv(V, 3, orp, oci, oH, v.astype(np.float64))
     assert_close("y", y.cpu().numpy(), oy, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["float32", "float64"])
+def test_pairs_dof2_compact_rows(orc, dtype):
+    """Springs, inertia and pairs on a 2-D grid (no face terms): the compact
+    row kernel's pair path at dof 2, with the gathered partner entries in
+    their 2-D layout; eval and the product against the oracle."""
+    import hessian_assembly_b200 as mad
+    import torch
+    n = 40
+    ps = mi.param_static(n, 41, np.float64)
+    V, F, X, UV = ps["V"], ps["F"], ps["X"], ps["UV"]
+    ctx = mad.Context(V, F, 2, dtype, part_xyz=X, max_pairs=400)
+    assert ctx.info.row_slot_bytes == 4
+    edges = ctx.mad_edges().cpu().numpy()
+    L0 = np.linalg.norm(X[edges[:, 0]] - X[edges[:, 1]], axis=1)
+    xt = X + 0.01 * mi.probe_vector(V, 2, 42, np.float64)
+    rng = np.random.default_rng(43)
+    pairs = []
+    while len(pairs) < 300:
+        a, b = rng.integers(0, V, 2)
+        if a != b and not mi.grid_adjacent(n, a, b):
+            pairs.append((a, b))
+    pairs = np.array(pairs, np.int32)
+    prest = 0.9 * np.linalg.norm(UV[pairs[:, 0]] - UV[pairs[:, 1]], axis=1)
+    add_pairs(ctx, pairs, prest, dtype)
+    assert ctx.mad_status_sync() == 0
+    mask = 1 | 2 | 8
+    terms = mad.Terms(mask=mask, spring_rest=to_dev(L0, dtype), spring_k=3.0,
+                      inertia_xt=to_dev(xt, dtype), inertia_w=50.0, pair_k=7.0)
+    x = UV.astype(dtype)
+    g, H, E = run_eval(ctx, x, terms, dtype)
+    rp, ci, nnzb = gpu_pattern(ctx)
+    orp, oci = orc.pattern(V, F, pairs)
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    og, oH, oE = orc.eval(V, 2, x, mask, orp, oci, edges=edges, L0=L0.astype(dtype), k=3.0,
+                          xt=xt.astype(dtype), w=50.0, pairs=pairs, prest=prest.astype(dtype),
+                          kp=7.0)
+    assert_close("g", g, og, dtype)
+    assert_close("H", H[:nnzb], oH, dtype)
+    v = mi.probe_vector(V, 2, 44, np.dtype(dtype))
+    tdt = getattr(torch, dtype)
+    y = torch.full((V, 2), float("nan"), dtype=tdt, device="cuda")
+    ctx.mad_hvp(to_dev(x, dtype), terms, to_dev(v, dtype), y)
+    torch.cuda.synchronize()
+    assert_close("y", y.cpu().numpy(), orc.bsr_mv(V, 2, orp, oci, oH, v), dtype)
