@@ -431,7 +431,8 @@ def cpu_baseline(st):
             "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
 
 
-EXTRA = ("cloth_small", "generic1000", "symdir500", "pairs1000", "jac1000", "area1000", "vf1000")
+EXTRA = ("cloth_small", "generic1000", "symdir500", "pairs1000", "jac1000", "area1000", "vf1000",
+         "shard1000")
 GENERIC_AD = 8  # MAD_EVAL_GENERIC_AD
 
 
@@ -501,6 +502,8 @@ def extra_workloads(args, only=None):
         area1000(res, mad, torch, dev, stream, timeit)
     if run("vf1000"):
         vf1000(res, mad, torch, dev, stream, timeit)
+    if run("shard1000"):
+        shard1000(res, mad, torch, dev, stream, timeit)
     return res
 
 
@@ -606,6 +609,33 @@ def area1000(res, mad, torch, dev, stream, timeit):
     terms.flags = GENERIC_AD
     res["area1000_generic_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
     res["area1000_generic_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
+    ctx.close()
+
+
+def shard1000(res, mad, torch, dev, stream, timeit):
+    """The 1000^2 cloth step split into 2 and 4 owner-computes shards
+    (mad_eval_shard), each shard's positions in a buffer of its own, timed
+    one shard at a time on this GPU: what each rank's kernel would take on
+    its own GPU (the halo read from the other buffers stays on this GPU's
+    memory here, not over NVLink)."""
+    st = mi.cloth_static(N_GRID, np.float32)
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    terms = mad.Terms(mask=3, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
+                      inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"])
+    x = torch.from_numpy(mi.cloth_x(N_GRID, SEED, 0, np.float32)).to(dev)
+    for nranks in (2, 4):
+        rb, bb = mad.mad_shard_plan(st["V"], st["F"], nranks)
+        parts = [x[rb[r]:rb[r + 1]].clone() for r in range(nranks)]
+        ms = []
+        for r in range(nranks):
+            nr, nb = int(rb[r + 1] - rb[r]), int(bb[r + 1] - bb[r])
+            g = torch.empty((max(nr, 1), 3), device=dev)
+            H = torch.empty((max(nb, 1), 3, 3), device=dev)
+            ms.append(timeit(lambda: ctx.mad_eval_shard(rb, parts, r, terms, g, H, None,
+                                                          stream)))
+            del g, H
+        res[f"shard1000_{nranks}_rank_ms"] = [round(m, 5) for m in ms]
+        res[f"shard1000_{nranks}_max_rank_ms"] = round(max(ms), 5)
     ctx.close()
 
 
