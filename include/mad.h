@@ -35,7 +35,11 @@
  *     launched.  Errors found on the device (a pair index out of range, CSR
  *     capacity exceeded) are recorded in a sticky device status word and are
  *     reported by mad_status_sync(); no kernel traps or asserts.
- *   - A context is used by one host thread at a time.
+ *   - A context is used by one host thread at a time, and its calls are
+ *     issued on one stream (or streams ordered by events): the context keeps
+ *     per-call device scratch (per-face product results, the gathered pair
+ *     partner positions, the vertex-face shares, energy partials) that two
+ *     calls running at once on unordered streams would share.
  */
 #ifndef MAD_H_
 #define MAD_H_
