@@ -326,6 +326,8 @@ def rooflines(w, headline_ms, hbm, peak_kind):
         "pairs1000_insert": (4 * (V + 1) * 2 + 4 * (V + 2 * E) + 4 * (V + 2 * E + 2 * P) + 8 * P,
                              w.get("pairs1000_insert_ms")),
         "jac1000": (w.get("jac1000_bytes"), w.get("jac1000_ms")),
+        # the product: read x, v and the edge list, write y
+        "cloth1000_hvp": (12 * V * 3 + 8 * E, w.get("cloth1000_hvp_ms")),
         "area1000_eval": (ALGO_BYTES + 16 * F, w.get("area1000_eval_ms")),
         "area1000_hvp": (12 * V * 3 + 12 * E + 16 * F, w.get("area1000_hvp_ms")),
         "vf1000_eval": (w.get("vf1000_eval_bytes"), w.get("vf1000_eval_ms")),
@@ -431,8 +433,8 @@ def cpu_baseline(st):
             "sample": "2 full 1000x1000 steps (fp64 closed forms, COO sort + merge), median"}
 
 
-EXTRA = ("cloth_small", "generic1000", "symdir500", "pairs1000", "jac1000", "area1000", "vf1000",
-         "shard1000")
+EXTRA = ("cloth_small", "generic1000", "hvp1000", "symdir500", "pairs1000", "jac1000", "area1000",
+         "vf1000", "shard1000")
 GENERIC_AD = 8  # MAD_EVAL_GENERIC_AD
 
 
@@ -491,6 +493,8 @@ def extra_workloads(args, only=None):
         ctx.close()
     if run("generic1000"):
         generic1000(res, mad, torch, dev, stream, timeit)
+    if run("hvp1000"):
+        hvp1000(res, mad, torch, dev, stream, timeit)
     # parameterization 500^2: eval and HVP
     if run("symdir500"):
         symdir500(res, mad, torch, dev, stream, timeit)
@@ -609,6 +613,20 @@ def area1000(res, mad, torch, dev, stream, timeit):
     terms.flags = GENERIC_AD
     res["area1000_generic_eval_ms"] = round(timeit(lambda: ctx.mad_eval(x, terms, g, H, None, stream)), 5)
     res["area1000_generic_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
+    ctx.close()
+
+
+def hvp1000(res, mad, torch, dev, stream, timeit):
+    """The matrix-free product y = H v of the 1000^2 cloth (springs +
+    inertia), with a seeded N(0,1) direction."""
+    st = mi.cloth_static(N_GRID, np.float32)
+    ctx = mad.Context(st["V"], st["F"], 3, "float32", part_xyz=st["X"])
+    terms = mad.Terms(mask=3, spring_rest=torch.from_numpy(st["L0"]).to(dev), spring_k=st["k"],
+                      inertia_xt=torch.from_numpy(st["xt"]).to(dev), inertia_w=st["w"])
+    x = torch.from_numpy(mi.cloth_x(N_GRID, SEED, 0, np.float32)).to(dev)
+    v = torch.from_numpy(mi.probe_vector(st["V"], 3, 1009, np.float32)).to(dev)
+    y = torch.empty((st["V"], 3), device=dev)
+    res["cloth1000_hvp_ms"] = round(timeit(lambda: ctx.mad_hvp(x, terms, v, y, stream)), 5)
     ctx.close()
 
 

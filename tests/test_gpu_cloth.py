@@ -161,3 +161,21 @@ def test_eval_host_matches_device(orc):
     assert np.array_equal(hg.numpy(), g)
     assert np.array_equal(hH.numpy(), H[:nnzb])
     assert he.item() == E
+
+
+@pytest.mark.parametrize("n,dtype", [(100, "float64"), (1000, "float32")])
+def test_cloth_hvp(orc, n, dtype):
+    """The matrix-free product of springs + inertia (at 1000^2 the benched
+    size) against the oracle's assembled H applied to the same direction."""
+    import torch
+    ctx, st = cloth_context(n, dtype)
+    x = mi.cloth_x(n, 1010, 0, np.dtype(dtype))
+    v = mi.probe_vector(st["V"], 3, 1011, np.dtype(dtype))
+    terms = cloth_terms(st, dtype, 3)
+    y = torch.full((st["V"], 3), float("nan"), dtype=getattr(torch, dtype), device="cuda")
+    ctx.mad_hvp(to_dev(x, dtype), terms, to_dev(v, dtype), y)
+    torch.cuda.synchronize()
+    orp, oci = orc.pattern(st["V"], st["F"])
+    _, oH, _ = orc.eval(st["V"], 3, x, 3, orp, oci, edges=st["edges"], L0=st["L0"], k=st["k"],
+                        xt=st["xt"], w=st["w"])
+    assert_close("y", y.cpu().numpy(), orc.bsr_mv(st["V"], 3, orp, oci, oH, v), dtype)
